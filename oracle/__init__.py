@@ -1,0 +1,171 @@
+"""Wall attention CPU oracle (double precision) -- TEST INFRASTRUCTURE ONLY.
+
+Python wrapper over ``wall_oracle.c``.  Only ``tests/``, ``__graft_entry__.smoke``
+and the benchmark's CPU-baseline leg may import this package; the product path
+(``decayed_softmax_attention_b200``) never does.  The oracle shares no code with
+the CUDA path: inputs are numpy float32 arrays holding already-rounded values,
+outputs are float64.
+
+Functions (each follows the Wall Attention README; see the C file's header for
+the exact formulas and the readings taken where the page is silent):
+  wall_fwd           -- prefill forward by the pairwise definition
+  kv_cache           -- P, r_cache and k_tilde of the "Decode" section
+  decode_from_cache  -- one decode step over (k_tilde, r_cache)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import sys
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "wall_oracle.c")
+_LIB_DIR = os.path.join(_HERE, "_build")
+_LIB = os.path.join(_LIB_DIR, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2, IEEE double, OpenMP). Returns the .so path."""
+    if (not force and os.path.exists(_LIB)
+            and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
+        return _LIB
+    os.makedirs(_LIB_DIR, exist_ok=True)
+    tmp = _LIB + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-fno-fast-math",
+           "-std=c11", "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(build())
+    P = ctypes.c_void_p
+    i, d, i64 = ctypes.c_int, ctypes.c_double, ctypes.c_int64
+    lib.wall_oracle_fwd.argtypes = [P, P, P, P, P, P, i, P, i, i, i, i, i, i, i, d, P, i64, P, P, i]
+    lib.wall_oracle_kv_cache.argtypes = [P, P, i, i, i, i, i, i, P, P, P, P, i]
+    lib.wall_oracle_decode_cache.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, i, i, d, P, P, i]
+    for f in (lib.wall_oracle_fwd, lib.wall_oracle_kv_cache, lib.wall_oracle_decode_cache):
+        f.restype = ctypes.c_int
+    lib.wall_oracle_max_threads.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def max_threads() -> int:
+    return int(_load().wall_oracle_max_threads())
+
+
+def _f32(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor
+        x = x.detach().float().cpu().numpy()
+    return np.ascontiguousarray(x, dtype=np.float32)
+
+
+def _f64(x):
+    if x is None:
+        return None
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise RuntimeError(f"oracle {what} failed with status {rc}")
+
+
+def wall_fwd(q, k, v, g, g_scalar=None, sink_bias=None, window=0, cu_seqlens=None,
+             scale=None, rows=None, threads=0):
+    """Prefill forward by the definition.
+
+    q [B,T,HQ,K], k [B,T,H,K], v [B,T,H,V], g [B,T,HQ,K]; g_scalar [B,T,HQ] or None;
+    sink_bias [HQ] or None; cu_seqlens int [N+1] or None (B == 1).
+    rows: None (all rows) or an int array of flattened b*T + t indices.
+    Returns (o, lse): o [B,T,HQ,V] / [nrows,HQ,V], lse [B,T,HQ] / [nrows,HQ], float64.
+    """
+    q, k, v, g = _f32(q), _f32(k), _f32(v), _f32(g)
+    gs, sink = _f32(g_scalar), _f32(sink_bias)
+    B, T, HQ, K = q.shape
+    H, V = k.shape[2], v.shape[3]
+    cu = None
+    nseq = 0
+    if cu_seqlens is not None:
+        if hasattr(cu_seqlens, "detach"):
+            cu_seqlens = cu_seqlens.detach().cpu().numpy()
+        cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+        nseq = cu.shape[0] - 1
+    if scale is None or scale <= 0:
+        scale = K ** -0.5
+    if rows is None:
+        nrows, rows_arr = B * T, None
+    else:
+        rows_arr = np.ascontiguousarray(rows, dtype=np.int64)
+        nrows = rows_arr.shape[0]
+    o = np.empty((nrows, HQ, V), dtype=np.float64)
+    lse = np.empty((nrows, HQ), dtype=np.float64)
+    rc = _load().wall_oracle_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gs), _ptr(sink),
+                                 int(window or 0), _ptr(cu), nseq, B, T, HQ, H, K, V, float(scale),
+                                 _ptr(rows_arr), nrows, _ptr(o), _ptr(lse), int(threads))
+    _check(rc, "wall_fwd")
+    if rows is None:
+        return o.reshape(B, T, HQ, V), lse.reshape(B, T, HQ)
+    return o, lse
+
+
+def kv_cache(k, g, HQ=None, chunk=64, anchors=None, threads=0):
+    """P, r_cache and k_tilde of the decode cache (double).
+
+    k [B,T,H,K], g [B,T,HQ,K]. anchors: optional [B,ceil(T/C),HQ,K] replacing R_c.
+    Returns (k_tilde [B,T,HQ,K], r_cache [B,ceil(T/C),HQ,K], P [B,T,HQ,K]).
+    """
+    k, g = _f32(k), _f32(g)
+    B, T, H, K = k.shape
+    HQ = g.shape[2]
+    nc = (T + chunk - 1) // chunk
+    kt = np.empty((B, T, HQ, K), dtype=np.float64)
+    rc_ = np.empty((B, nc, HQ, K), dtype=np.float64)
+    P = np.empty((B, T, HQ, K), dtype=np.float64)
+    anc = _f64(anchors)
+    rc = _load().wall_oracle_kv_cache(_ptr(k), _ptr(g), B, T, HQ, H, K, int(chunk), _ptr(anc),
+                                      _ptr(kt), _ptr(rc_), _ptr(P), int(threads))
+    _check(rc, "kv_cache")
+    return kt, rc_, P
+
+
+def decode_from_cache(q, p_curr, v, k_tilde, r_cache, T_kv, sink_bias=None, chunk=64,
+                      scale=None, threads=0):
+    """One decode step over the pre-rescaled cache (double).
+
+    q [B,HQ,K] (or [B,1,HQ,K]); p_curr [B,HQ,K]; v [B,cap,H,V]; k_tilde [B,cap,HQ,K];
+    r_cache [B,ceil(cap/C),HQ,K]; the first T_kv cache rows are attended.
+    Returns (o [B,HQ,V], lse [B,HQ]).
+    """
+    q = _f32(q)
+    q = q.reshape(q.shape[0], q.shape[-2], q.shape[-1])
+    p = _f64(np.asarray(p_curr).reshape(q.shape))
+    v, kt, r = _f32(v), _f64(k_tilde), _f64(r_cache)
+    sink = _f32(sink_bias)
+    B, HQ, K = q.shape
+    cap, H, V = v.shape[1], v.shape[2], v.shape[3]
+    if scale is None or scale <= 0:
+        scale = K ** -0.5
+    o = np.empty((B, HQ, V), dtype=np.float64)
+    lse = np.empty((B, HQ), dtype=np.float64)
+    rc = _load().wall_oracle_decode_cache(_ptr(q), _ptr(p), _ptr(v), _ptr(kt), _ptr(r), _ptr(sink),
+                                          B, int(T_kv), cap, HQ, H, K, V, int(chunk), float(scale),
+                                          _ptr(o), _ptr(lse), int(threads))
+    _check(rc, "decode_from_cache")
+    return o, lse
+

@@ -1,0 +1,274 @@
+/*
+ * Wall attention CPU oracle -- TEST INFRASTRUCTURE ONLY.
+ *
+ * Plain, slow, double-precision evaluation of what the Wall attention hot path
+ * computes.  Only the tests, the smoke check and the benchmark's CPU-baseline
+ * leg may load this file's library.  It shares no code, header or constant
+ * with the CUDA path (decayed_softmax_attention_b200/csrc).
+ *
+ * Sources (the Wall Attention GitHub README, as mirrored on news.ainew.jp):
+ *   - intro: a pair (i, j) is scored by sum_n q[i,n] k[j,n] weighted, per
+ *     channel n, by the learned decay accumulated between the two positions;
+ *     g = 0 gives vanilla softmax attention.  The accumulated decay between
+ *     j <= i is exp(G[i,n] - G[j,n]) with G the inclusive cumulative sum of
+ *     the per-channel log-decay g over time.
+ *   - "Usage / Training-Prefill": shapes q [B,T,HQ,K], k [B,T,H,K],
+ *     v [B,T,H,V], g [B,T,HQ,K]; optional g_scalar [B,T,HQ] (a FoX-style
+ *     additive gate), sink_bias [HQ] (attention sink), window_size (sliding
+ *     window), cu_seqlens (variable-length packing, B == 1).
+ *   - "Decode (cache build)": P = cumsum(g) * (1/ln 2) (exp2 domain),
+ *     k_tilde[j] = k[j] * exp2(R_c - P[j]) with one anchor vector R_c per
+ *     chunk of C tokens; the decode reads k_tilde and r_cache.
+ * Readings of points the page leaves open (each is also listed in the design doc):
+ *   - scale multiplies only the decayed q.k sum (not g_scalar, not the sink);
+ *   - g_scalar adds Gs[i] - Gs[j] to the logit, Gs its inclusive cumsum;
+ *   - sink_bias is one extra logit per head with a zero value vector;
+ *   - window W keeps keys with 0 <= i - j < W (W counts the query itself),
+ *     following the sliding-window mask_mod statement on the FlexAttention
+ *     review page ("technical mechanism" section); W <= 0 means no window;
+ *   - cumulative sums restart at every cu_seqlens document start;
+ *   - query head hq reads KV head hq / (HQ / H);
+ *   - lse is the natural-log normaliser, sink included;
+ *   - the cache anchor is R_c = P[c*C], the chunk's first token.
+ *
+ * Inputs are float32 arrays holding already-rounded values (bf16 or fp32);
+ * every value is widened to double on use.  No blocking, fusion or reordering
+ * beyond the definitions above.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_OK 0
+#define ORACLE_BAD_ARG 1
+#define ORACLE_NO_MEM 2
+
+/* Document [s, e) that contains token t (whole row [0, T) without packing). */
+static void doc_of(const int32_t* cu, int nseq, int T, int t, int* s, int* e) {
+  if (!cu) {
+    *s = 0;
+    *e = T;
+    return;
+  }
+  for (int d = 0; d < nseq; ++d) {
+    if (t >= cu[d] && t < cu[d + 1]) {
+      *s = cu[d];
+      *e = cu[d + 1];
+      return;
+    }
+  }
+  *s = t;
+  *e = t + 1;
+}
+
+static void set_threads(int nthreads) {
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+  (void)nthreads;
+#endif
+}
+
+/*
+ * Prefill forward, by the definition.
+ *
+ * For every requested row r = b*T + t and every query head hq:
+ *   kv = hq / (HQ/H);  [s, e) = document of t;
+ *   G[u,n]  = sum_{w=s..u} g[b,w,hq,n]        (inclusive, restarts at s)
+ *   Gs[u]   = sum_{w=s..u} g_scalar[b,w,hq]   (0 without g_scalar)
+ *   keys j in [s, t] with (window <= 0 or t - j < window);
+ *   x_j = scale * sum_n q[t,n] k[j,n] exp(G[t,n] - G[j,n]) + Gs[t] - Gs[j];
+ *   M = max(x_j, sink);  Z = sum_j exp(x_j - M) + exp(sink - M);
+ *   o = sum_j exp(x_j - M) v[j] / Z;  lse = M + log Z.
+ * rows == NULL means every row (nrows must be B*T).  o: [nrows, HQ, V],
+ * lse: [nrows, HQ], both double.
+ */
+int wall_oracle_fwd(const float* q, const float* k, const float* v, const float* g,
+                    const float* g_scalar, const float* sink, int window,
+                    const int32_t* cu_seqlens, int num_seqs, int B, int T, int HQ, int H,
+                    int K, int V, double scale, const int64_t* rows, int64_t nrows,
+                    double* o, double* lse, int nthreads) {
+  if (B <= 0 || T <= 0 || HQ <= 0 || H <= 0 || K <= 0 || V <= 0 || HQ % H) return ORACLE_BAD_ARG;
+  if (cu_seqlens && (B != 1 || num_seqs <= 0 || cu_seqlens[0] != 0 || cu_seqlens[num_seqs] != T))
+    return ORACLE_BAD_ARG;
+  if (!rows && nrows != (int64_t)B * T) return ORACLE_BAD_ARG;
+  const int group = HQ / H;
+  set_threads(nthreads);
+  int status = ORACLE_OK;
+
+#pragma omp parallel
+  {
+    double* G = (double*)malloc(sizeof(double) * (size_t)T * K);
+    double* Gs = (double*)malloc(sizeof(double) * (size_t)T);
+    double* x = (double*)malloc(sizeof(double) * (size_t)T);
+    if (!G || !Gs || !x) {
+#pragma omp atomic write
+      status = ORACLE_NO_MEM;
+    } else {
+#pragma omp for schedule(dynamic, 1)
+      for (int64_t bh = 0; bh < (int64_t)B * HQ; ++bh) {
+        const int b = (int)(bh / HQ), hq = (int)(bh % HQ), kv = hq / group;
+        /* inclusive prefix sums, restarting at each document start */
+        for (int u = 0; u < T; ++u) {
+          int s, e;
+          doc_of(cu_seqlens, num_seqs, T, u, &s, &e);
+          const float* gu = g + (((size_t)b * T + u) * HQ + hq) * K;
+          for (int n = 0; n < K; ++n)
+            G[(size_t)u * K + n] = (u == s ? 0.0 : G[(size_t)(u - 1) * K + n]) + (double)gu[n];
+          const double gsu = g_scalar ? (double)g_scalar[((size_t)b * T + u) * HQ + hq] : 0.0;
+          Gs[u] = (u == s ? 0.0 : Gs[u - 1]) + gsu;
+        }
+        for (int64_t r = 0; r < nrows; ++r) {
+          const int64_t row = rows ? rows[r] : r;
+          if (row / T != b) continue;
+          const int t = (int)(row % T);
+          int s, e;
+          doc_of(cu_seqlens, num_seqs, T, t, &s, &e);
+          int j0 = s;
+          if (window > 0 && t - window + 1 > j0) j0 = t - window + 1;
+          const float* qt = q + (((size_t)b * T + t) * HQ + hq) * K;
+          const double* Gt = G + (size_t)t * K;
+          double M = -INFINITY;
+          for (int j = j0; j <= t; ++j) {
+            const float* kj = k + (((size_t)b * T + j) * H + kv) * K;
+            const double* Gj = G + (size_t)j * K;
+            double dot = 0.0;
+            for (int n = 0; n < K; ++n) dot += (double)qt[n] * (double)kj[n] * exp(Gt[n] - Gj[n]);
+            x[j] = scale * dot + (Gs[t] - Gs[j]);
+            if (x[j] > M) M = x[j];
+          }
+          const double sb = sink ? (double)sink[hq] : -INFINITY;
+          if (sb > M) M = sb;
+          double Z = sink ? exp(sb - M) : 0.0;
+          double* orow = o + ((size_t)r * HQ + hq) * V;
+          for (int c = 0; c < V; ++c) orow[c] = 0.0;
+          for (int j = j0; j <= t; ++j) {
+            const double w = exp(x[j] - M);
+            Z += w;
+            const float* vj = v + (((size_t)b * T + j) * H + kv) * V;
+            for (int c = 0; c < V; ++c) orow[c] += w * (double)vj[c];
+          }
+          for (int c = 0; c < V; ++c) orow[c] /= Z;
+          lse[(size_t)r * HQ + hq] = M + log(Z);
+        }
+      }
+    }
+    free(G);
+    free(Gs);
+    free(x);
+  }
+  return status;
+}
+
+/*
+ * Decode cache build, following the README's "Decode" section.
+ *   P[t,n]  = (1/ln 2) * sum_{u=0..t} g[b,u,hq,n]        (exp2-domain prefix)
+ *   R[c,n]  = P[c*C, n]           (chunk-start anchor; or anchors[] if given)
+ *   k_tilde[t,hq,n] = k[t, kv(hq), n] * 2^(R[t/C, n] - P[t, n])
+ * Outputs (double): k_tilde [B,T,HQ,K], r_cache [B,ceil(T/C),HQ,K], P [B,T,HQ,K].
+ * `anchors` (nullable, [B,ceil(T/C),HQ,K]) replaces R to test that the choice of
+ * anchor leaves every decode score unchanged.
+ */
+int wall_oracle_kv_cache(const float* k, const float* g, int B, int T, int HQ, int H, int K,
+                         int C, const double* anchors, double* k_tilde, double* r_cache,
+                         double* P, int nthreads) {
+  if (B <= 0 || T <= 0 || HQ <= 0 || H <= 0 || K <= 0 || C <= 0 || HQ % H) return ORACLE_BAD_ARG;
+  const int group = HQ / H;
+  const int nc = (T + C - 1) / C;
+  const double rcp_ln2 = 1.0 / log(2.0);
+  set_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t bh = 0; bh < (int64_t)B * HQ; ++bh) {
+    const int b = (int)(bh / HQ), hq = (int)(bh % HQ), kv = hq / group;
+    for (int n = 0; n < K; ++n) {
+      double acc = 0.0;
+      for (int t = 0; t < T; ++t) {
+        acc += (double)g[(((size_t)b * T + t) * HQ + hq) * K + n];
+        P[(((size_t)b * T + t) * HQ + hq) * K + n] = acc * rcp_ln2;
+      }
+      for (int c = 0; c < nc; ++c) {
+        const size_t ridx = (((size_t)b * nc + c) * HQ + hq) * K + n;
+        r_cache[ridx] = anchors ? anchors[ridx] : P[(((size_t)b * T + (size_t)c * C) * HQ + hq) * K + n];
+      }
+      for (int t = 0; t < T; ++t) {
+        const size_t pidx = (((size_t)b * T + t) * HQ + hq) * K + n;
+        const double R = r_cache[(((size_t)b * nc + t / C) * HQ + hq) * K + n];
+        k_tilde[pidx] = (double)k[(((size_t)b * T + t) * H + kv) * K + n] * exp2(R - P[pidx]);
+      }
+    }
+  }
+  return ORACLE_OK;
+}
+
+/*
+ * Single-step decode over the pre-rescaled cache, following the README's
+ * "Decode" section: for the current query q (its prefix P = p_curr) and cached
+ * keys j in [0, T_kv):
+ *   x_j = scale * sum_n q[n] * k_tilde[j,n] * 2^(p_curr[n] - R[j/C, n])
+ *   softmax over j (plus the optional sink logit), o = sum_j w_j v[j].
+ * q [B,HQ,K] float; p_curr [B,HQ,K], k_tilde [B,cap,HQ,K], r_cache
+ * [B,ceil(cap/C),HQ,K] double; v [B,cap,H,V] float.  o [B,HQ,V], lse [B,HQ].
+ */
+int wall_oracle_decode_cache(const float* q, const double* p_curr, const float* v,
+                             const double* k_tilde, const double* r_cache, const float* sink,
+                             int B, int T_kv, int cap, int HQ, int H, int K, int V, int C,
+                             double scale, double* o, double* lse, int nthreads) {
+  if (B <= 0 || T_kv <= 0 || cap < T_kv || HQ <= 0 || H <= 0 || K <= 0 || V <= 0 || C <= 0 ||
+      HQ % H)
+    return ORACLE_BAD_ARG;
+  const int group = HQ / H;
+  const int nc = (cap + C - 1) / C;
+  set_threads(nthreads);
+  int status = ORACLE_OK;
+#pragma omp parallel
+  {
+    double* x = (double*)malloc(sizeof(double) * (size_t)T_kv);
+    if (!x) {
+#pragma omp atomic write
+      status = ORACLE_NO_MEM;
+    } else {
+#pragma omp for schedule(dynamic, 1)
+      for (int64_t bh = 0; bh < (int64_t)B * HQ; ++bh) {
+        const int b = (int)(bh / HQ), hq = (int)(bh % HQ), kv = hq / group;
+        const float* qv = q + ((size_t)b * HQ + hq) * K;
+        const double* pc = p_curr + ((size_t)b * HQ + hq) * K;
+        double M = -INFINITY;
+        for (int j = 0; j < T_kv; ++j) {
+          const double* kt = k_tilde + (((size_t)b * cap + j) * HQ + hq) * K;
+          const double* R = r_cache + (((size_t)b * nc + j / C) * HQ + hq) * K;
+          double dot = 0.0;
+          for (int n = 0; n < K; ++n) dot += (double)qv[n] * kt[n] * exp2(pc[n] - R[n]);
+          x[j] = scale * dot;
+          if (x[j] > M) M = x[j];
+        }
+        const double sb = sink ? (double)sink[hq] : -INFINITY;
+        if (sb > M) M = sb;
+        double Z = sink ? exp(sb - M) : 0.0;
+        double* orow = o + ((size_t)b * HQ + hq) * V;
+        for (int c = 0; c < V; ++c) orow[c] = 0.0;
+        for (int j = 0; j < T_kv; ++j) {
+          const double w = exp(x[j] - M);
+          Z += w;
+          const float* vj = v + (((size_t)b * cap + j) * H + kv) * V;
+          for (int c = 0; c < V; ++c) orow[c] += w * (double)vj[c];
+        }
+        for (int c = 0; c < V; ++c) orow[c] /= Z;
+        lse[(size_t)b * HQ + hq] = M + log(Z);
+      }
+    }
+    free(x);
+  }
+  return status;
+}
+
+int wall_oracle_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
