@@ -1,0 +1,259 @@
+"""Wall attention (decayed softmax attention) for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI in ``include/wall_attn.h``: argument
+marshalling only (dtype/shape checks, device pointers, the current CUDA
+stream, caller-side workspace allocation through torch).  Every step of the
+computation runs in the library's CUDA kernels; there is no CPU fallback, and
+importing this module on a machine without the built library raises.
+
+Public calls (same names as the C ABI):
+  wall_attn_fwd(q, k, v, g, g_scalar=None, sink_bias=None, window=0,
+                cu_seqlens=None, scale=None, return_lse=False)
+  wall_build_kv_cache(k_new, g_new, k_tilde, r_cache, p_last, t_start=0,
+                      p_prev=None, chunk=64)
+  wall_attn_decode(q, p_curr, v, k_tilde, r_cache, T_kv, sink_bias=None,
+                   scale=None, chunk=64, out=None, lse=None, workspace=None)
+plus KVCache, a small helper that owns the cache tensors of a streaming loop.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "WallError", "lib_path", "load_library", "wall_attn_fwd", "wall_attn_fwd_workspace_size",
+    "wall_build_kv_cache", "wall_attn_decode", "wall_attn_decode_workspace_size",
+    "wall_device_error", "wall_debug_set_fault", "KVCache", "EXPORTED_SYMBOLS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "_lib", "libwall_attn.so")
+
+WALL_OK = 0
+WALL_DTYPE_F32 = 0
+WALL_DTYPE_BF16 = 1
+_STATUS = {
+    0: "WALL_OK", 1: "WALL_ERR_INVALID_ARG", 2: "WALL_ERR_UNSUPPORTED", 3: "WALL_ERR_CUDA",
+    4: "WALL_ERR_DEVICE_TIMEOUT", 5: "WALL_ERR_WORKSPACE",
+}
+
+EXPORTED_SYMBOLS = (
+    "wall_status_string", "wall_attn_fwd_workspace_size", "wall_attn_fwd",
+    "wall_build_kv_cache", "wall_attn_decode_workspace_size", "wall_attn_decode",
+    "wall_device_error", "wall_debug_set_fault",
+)
+
+
+class WallError(RuntimeError):
+    """A C-ABI call returned a status other than WALL_OK."""
+
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_STATUS.get(status, status)} ({_lib_status_string(status)})")
+
+
+_lib = None
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load the in-tree CUDA library (build it with ``python -m decayed_softmax_attention_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            f"Wall attention CUDA library not built: {_LIB_PATH} is missing "
+            "(run `python -m decayed_softmax_attention_b200.build`)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.wall_status_string.argtypes = [I]
+    lib.wall_status_string.restype = ctypes.c_char_p
+    lib.wall_attn_fwd_workspace_size.argtypes = [I, I, I, I, I, I, I]
+    lib.wall_attn_fwd_workspace_size.restype = S
+    lib.wall_attn_fwd.argtypes = [P, P, P, P, P, P, I, P, I, I, I, I, I, I, I, I, F, P, P, P, S, P]
+    lib.wall_attn_fwd.restype = I
+    lib.wall_build_kv_cache.argtypes = [P, P, P, I, I, I, I, I, I, I, I, I, P, P, P, P]
+    lib.wall_build_kv_cache.restype = I
+    lib.wall_attn_decode_workspace_size.argtypes = [I, I, I, I, I, I]
+    lib.wall_attn_decode_workspace_size.restype = S
+    lib.wall_attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, P, P, P, S, P]
+    lib.wall_attn_decode.restype = I
+    lib.wall_device_error.argtypes = [P]
+    lib.wall_device_error.restype = I
+    lib.wall_debug_set_fault.argtypes = [I, I]
+    lib.wall_debug_set_fault.restype = None
+    _lib = lib
+    return lib
+
+
+def _lib_status_string(status: int) -> str:
+    try:
+        return load_library().wall_status_string(int(status)).decode()
+    except Exception:  # pragma: no cover
+        return "?"
+
+
+def _check(status: int, what: str):
+    if status != WALL_OK:
+        raise WallError(status, what)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return WALL_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return WALL_DTYPE_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _dev(t, name, dtype=None, shape=None):
+    """Device pointer of a contiguous CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must live in CUDA device memory")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+# ----------------------------------------------------------------- prefill
+def wall_attn_fwd_workspace_size(B, T, HQ, H, K, V, dtype) -> int:
+    code = WALL_DTYPE_BF16 if dtype == torch.bfloat16 else WALL_DTYPE_F32
+    return int(load_library().wall_attn_fwd_workspace_size(B, T, HQ, H, K, V, code))
+
+
+def wall_attn_fwd(q, k, v, g, g_scalar=None, sink_bias=None, window=0, cu_seqlens=None,
+                  scale=None, return_lse=False, out=None, lse=None, workspace=None):
+    """Prefill forward (README "Usage"): o [B,T,HQ,V] (and lse [B,T,HQ] fp32, natural log)."""
+    lib = load_library()
+    B, T, HQ, K = q.shape
+    H, V = k.shape[2], v.shape[3]
+    dt = q.dtype
+    code = _dtype_code(q)
+    if out is None:
+        out = torch.empty((B, T, HQ, V), dtype=dt, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((B, T, HQ), dtype=torch.float32, device=q.device)
+    need = wall_attn_fwd_workspace_size(B, T, HQ, H, K, V, dt)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    nseq = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    st = lib.wall_attn_fwd(
+        _dev(q, "q", dt), _dev(k, "k", dt, (B, T, H, K)), _dev(v, "v", dt, (B, T, H, V)),
+        _dev(g, "g", dt, (B, T, HQ, K)), _dev(g_scalar, "g_scalar", dt, (B, T, HQ)),
+        _dev(sink_bias, "sink_bias", torch.float32, (HQ,)), int(window or 0),
+        _dev(cu_seqlens, "cu_seqlens", torch.int32), nseq, B, T, HQ, H, K, V, code,
+        float(scale) if scale else 0.0, _dev(out, "out", dt, (B, T, HQ, V)),
+        _dev(lse, "lse", torch.float32, (B, T, HQ)), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(q.device))
+    _check(st, "wall_attn_fwd")
+    return (out, lse) if return_lse else out
+
+
+# ----------------------------------------------------------------- decode
+def wall_build_kv_cache(k_new, g_new, k_tilde, r_cache, p_last, t_start=0, p_prev=None,
+                        chunk=64):
+    """Build (t_start=0) or append to the pre-rescaled key cache (README "Decode")."""
+    lib = load_library()
+    B, T_new, H, K = k_new.shape
+    HQ = g_new.shape[2]
+    cap = k_tilde.shape[1]
+    dt = k_new.dtype
+    st = lib.wall_build_kv_cache(
+        _dev(k_new, "k_new", dt), _dev(g_new, "g_new", dt, (B, T_new, HQ, K)),
+        _dev(p_prev, "p_prev", torch.float32), B, int(t_start), T_new, cap, HQ, H, K, int(chunk),
+        _dtype_code(k_new), _dev(k_tilde, "k_tilde", dt, (B, cap, HQ, K)),
+        _dev(r_cache, "r_cache", torch.float32, (B, (cap + chunk - 1) // chunk, HQ, K)),
+        _dev(p_last, "p_last", torch.float32), _stream(k_new.device))
+    _check(st, "wall_build_kv_cache")
+    return p_last
+
+
+def wall_attn_decode_workspace_size(B, T_kv, HQ, H, V, chunk=64) -> int:
+    return int(load_library().wall_attn_decode_workspace_size(B, T_kv, HQ, H, V, chunk))
+
+
+def wall_attn_decode(q, p_curr, v, k_tilde, r_cache, T_kv, sink_bias=None, scale=None, chunk=64,
+                     out=None, lse=None, workspace=None):
+    """One decode step over cache rows [0, T_kv): o [B,1,HQ,V] (lse [B,1,HQ] if given)."""
+    lib = load_library()
+    B, cap, HQ, K = k_tilde.shape
+    H, V = v.shape[2], v.shape[3]
+    dt = k_tilde.dtype
+    if out is None:
+        out = torch.empty((B, 1, HQ, V), dtype=dt, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(wall_attn_decode_workspace_size(B, T_kv, HQ, H, V, chunk), 1),
+                                dtype=torch.uint8, device=q.device)
+    st = lib.wall_attn_decode(
+        _dev(q, "q", dt), _dev(p_curr, "p_curr", torch.float32), _dev(v, "v", dt, (B, cap, H, V)),
+        _dev(k_tilde, "k_tilde", dt), _dev(r_cache, "r_cache", torch.float32),
+        _dev(sink_bias, "sink_bias", torch.float32, (HQ,)), B, int(T_kv), cap, HQ, H, K, V,
+        int(chunk), _dtype_code(k_tilde), float(scale) if scale else 0.0,
+        _dev(out, "out", dt), _dev(lse, "lse", torch.float32), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(q.device))
+    _check(st, "wall_attn_decode")
+    return out
+
+
+def wall_device_error(device=None) -> int:
+    """Synchronise the current stream and return (and clear) the device error status."""
+    return int(load_library().wall_device_error(_stream(device)))
+
+
+def wall_debug_set_fault(mode: int, wait_ms: int = 0):
+    """Testing hook: mode 1 starves the prefill consumers so their bounded waits expire."""
+    load_library().wall_debug_set_fault(int(mode), int(wait_ms))
+
+
+class KVCache:
+    """Device tensors of a streaming decode: k_tilde, r_cache, v cache and the running prefix P.
+
+    The caller writes value rows into ``v``; ``append`` folds the decay of new
+    keys into ``k_tilde`` (README "Decode": build once, then append token by
+    token) and returns P at the last appended row, which is the ``p_curr`` of
+    the next decode step.
+    """
+
+    def __init__(self, B, cap, HQ, H, K, V, dtype=torch.bfloat16, chunk=64, device="cuda"):
+        self.B, self.cap, self.HQ, self.H, self.K, self.V, self.chunk = B, cap, HQ, H, K, V, chunk
+        nc = (cap + chunk - 1) // chunk
+        self.k_tilde = torch.empty((B, cap, HQ, K), dtype=dtype, device=device)
+        self.r_cache = torch.empty((B, nc, HQ, K), dtype=torch.float32, device=device)
+        self.v = torch.empty((B, cap, H, V), dtype=dtype, device=device)
+        self.p = torch.zeros((B, HQ, K), dtype=torch.float32, device=device)
+        self.length = 0
+        self.workspace = torch.empty(max(wall_attn_decode_workspace_size(B, cap, HQ, H, V, chunk), 1),
+                                     dtype=torch.uint8, device=device)
+
+    def append(self, k_new, g_new, v_new=None):
+        T_new = k_new.shape[1]
+        if v_new is not None:
+            self.v[:, self.length:self.length + T_new].copy_(v_new)
+        wall_build_kv_cache(k_new, g_new, self.k_tilde, self.r_cache, self.p,
+                            t_start=self.length, p_prev=self.p if self.length > 0 else None,
+                            chunk=self.chunk)
+        self.length += T_new
+        return self.p
+
+    def decode(self, q, sink_bias=None, scale=None, out=None, lse=None):
+        return wall_attn_decode(q, self.p, self.v, self.k_tilde, self.r_cache, self.length,
+                                sink_bias=sink_bias, scale=scale, chunk=self.chunk, out=out,
+                                lse=lse, workspace=self.workspace)

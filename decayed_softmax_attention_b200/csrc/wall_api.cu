@@ -1,0 +1,253 @@
+// C ABI of the Wall attention library: argument validation, workspace
+// layout, TMA descriptor encoding and kernel launches.  Every public entry
+// point validates everything it can on the host before queuing any work and
+// reports problems as wall_status_t; nothing here aborts or synchronises
+// (unless WALL_DEBUG_SYNC=1).
+#include <atomic>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "wall_attn.h"
+#include "wall_common.cuh"
+#include "wall_internal.h"
+
+namespace {
+
+__device__ int g_wall_err;  // per-device error word (bit 0: a bounded wait gave up)
+
+std::atomic<int> g_fault_mode{0};
+std::atomic<int> g_wait_ms{2000};
+
+bool debug_sync() {
+  static const bool on = [] {
+    const char* s = std::getenv("WALL_DEBUG_SYNC");
+    return s != nullptr && s[0] == '1';
+  }();
+  return on;
+}
+
+constexpr int kMaxDevices = 64;
+std::mutex g_err_mu;
+int* g_err_addr[kMaxDevices] = {};
+
+int* device_err_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_err_mu);
+  if (g_err_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_wall_err) != cudaSuccess) return nullptr;
+    g_err_addr[dev] = static_cast<int*>(p);
+  }
+  return g_err_addr[dev];
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+wall_status_t finish(cudaError_t e, cudaStream_t st) {
+  if (e != cudaSuccess) return WALL_ERR_CUDA;
+  if (debug_sync()) return wall_device_error(reinterpret_cast<wall_stream_t>(st));
+  return WALL_OK;
+}
+
+bool supported_dim(int x) { return x == 64 || x == 128; }
+
+}  // namespace
+
+extern "C" {
+
+const char* wall_status_string(wall_status_t s) {
+  switch (s) {
+    case WALL_OK: return "WALL_OK";
+    case WALL_ERR_INVALID_ARG: return "WALL_ERR_INVALID_ARG: bad pointer, shape, size or alignment";
+    case WALL_ERR_UNSUPPORTED: return "WALL_ERR_UNSUPPORTED: head dimension, group size or chunk not supported";
+    case WALL_ERR_CUDA: return "WALL_ERR_CUDA: a CUDA call failed";
+    case WALL_ERR_DEVICE_TIMEOUT: return "WALL_ERR_DEVICE_TIMEOUT: a bounded device wait gave up";
+    case WALL_ERR_WORKSPACE: return "WALL_ERR_WORKSPACE: workspace too small";
+  }
+  return "WALL_ERR_UNKNOWN";
+}
+
+size_t wall_attn_fwd_workspace_size(int B, int T, int HQ, int H, int K, int V, wall_dtype_t dt) {
+  (void)H;
+  (void)V;
+  if (B <= 0 || T <= 0 || HQ <= 0 || K <= 0) return 0;
+  return wall::fwd_workspace_layout(B, T, HQ, K, dt == WALL_DTYPE_BF16, nullptr, nullptr);
+}
+
+wall_status_t wall_attn_fwd(const void* q, const void* k, const void* v, const void* g,
+                            const void* g_scalar, const float* sink_bias, int window,
+                            const int32_t* cu_seqlens, int num_seqs, int B, int T, int HQ, int H,
+                            int K, int V, wall_dtype_t dt, float scale, void* o, float* lse,
+                            void* workspace, size_t workspace_bytes, wall_stream_t stream) {
+  if (B < 0 || T < 0 || HQ <= 0 || H <= 0 || HQ % H != 0) return WALL_ERR_INVALID_ARG;
+  if (dt != WALL_DTYPE_F32 && dt != WALL_DTYPE_BF16) return WALL_ERR_INVALID_ARG;
+  if (!supported_dim(K) || !supported_dim(V)) return WALL_ERR_UNSUPPORTED;
+  if (cu_seqlens != nullptr && (B != 1 || num_seqs < 1)) return WALL_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) return WALL_OK;
+  const size_t esz = dt == WALL_DTYPE_BF16 ? 2 : 4;
+  if (!q || !k || !v || !g || !o || !workspace) return WALL_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(g, 16) ||
+      !aligned(o, 16) || !aligned(workspace, 256))
+    return WALL_ERR_INVALID_ARG;
+  if ((g_scalar && !aligned(g_scalar, esz)) || (sink_bias && !aligned(sink_bias, 4)) ||
+      (lse && !aligned(lse, 4)) || (cu_seqlens && !aligned(cu_seqlens, 4)))
+    return WALL_ERR_INVALID_ARG;
+  const long long NB = (static_cast<long long>(T) + wall::kBlockRows - 1) / wall::kBlockRows;
+  if (NB * B * HQ > 0x7fffffffLL) return WALL_ERR_UNSUPPORTED;
+  const bool bf16 = dt == WALL_DTYPE_BF16;
+  const size_t need = wall::fwd_workspace_layout(B, T, HQ, K, bf16, nullptr, nullptr);
+  if (workspace_bytes < need) return WALL_ERR_WORKSPACE;
+  if (!(scale > 0.f) || !std::isfinite(scale)) scale = 1.f / std::sqrt(static_cast<float>(K));
+
+  int* err = device_err_word();
+  if (err == nullptr) return WALL_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+  wall::FwdArgs a;
+  a.q = q; a.k = k; a.v = v; a.g = g; a.g_scalar = g_scalar; a.sink = sink_bias;
+  a.cu_seqlens = cu_seqlens; a.num_seqs = num_seqs; a.window = window > 0 ? window : 0;
+  a.B = B; a.T = T; a.HQ = HQ; a.H = H; a.K = K; a.V = V; a.NB = static_cast<int>(NB);
+  a.scale = scale; a.o = o; a.lse = lse; a.err = err;
+  a.wait_ns = static_cast<uint64_t>(g_wait_ms.load()) * 1000000ull;
+  a.fault = g_fault_mode.load();
+  wall::FwdWork w;
+  wall::fwd_workspace_layout(B, T, HQ, K, bf16, &w, static_cast<char*>(workspace));
+
+  cudaError_t e = wall::launch_prep(a, w, bf16, st);
+  if (e != cudaSuccess) return WALL_ERR_CUDA;
+  if (!bf16) return finish(wall::launch_fwd_simt(a, w, st), st);
+
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return WALL_ERR_CUDA;
+  CUtensorMap tmQ, tmK, tmV;
+  {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(T),
+                                static_cast<cuuint64_t>(B) * HQ};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * 2,
+                                   static_cast<cuuint64_t>(T) * K * 2};
+    const cuuint32_t box[3] = {64, 128, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    if (enc(&tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, w.qh, dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return WALL_ERR_CUDA;
+    if (enc(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, w.kh, dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return WALL_ERR_CUDA;
+  }
+  {
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(V), static_cast<cuuint64_t>(H),
+                                static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(V) * 2,
+                                   static_cast<cuuint64_t>(H) * V * 2,
+                                   static_cast<cuuint64_t>(T) * H * V * 2};
+    const cuuint32_t box[4] = {64, 1, 128, 1};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    if (enc(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(v), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return WALL_ERR_CUDA;
+  }
+  return finish(wall::launch_fwd_tc(a, w, tmQ, tmK, tmV, st), st);
+}
+
+wall_status_t wall_build_kv_cache(const void* k_new, const void* g_new, const float* p_prev,
+                                  int B, int t_start, int T_new, int cap, int HQ, int H, int K,
+                                  int chunk, wall_dtype_t dt, void* k_tilde, float* r_cache,
+                                  float* p_last, wall_stream_t stream) {
+  if (B < 0 || t_start < 0 || T_new < 0 || cap < 0 || HQ <= 0 || H <= 0 || HQ % H != 0)
+    return WALL_ERR_INVALID_ARG;
+  if (dt != WALL_DTYPE_F32 && dt != WALL_DTYPE_BF16) return WALL_ERR_INVALID_ARG;
+  if (static_cast<long long>(t_start) + T_new > cap) return WALL_ERR_INVALID_ARG;
+  if (!supported_dim(K)) return WALL_ERR_UNSUPPORTED;
+  if (chunk != 32 && chunk != 64 && chunk != 128) return WALL_ERR_UNSUPPORTED;
+  if (B == 0 || T_new == 0) return WALL_OK;
+  if ((t_start > 0) != (p_prev != nullptr)) return WALL_ERR_INVALID_ARG;
+  if (!k_new || !g_new || !k_tilde || !r_cache || !p_last) return WALL_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(g_new, 16) || !aligned(k_tilde, 16) ||
+      !aligned(r_cache, 16) || !aligned(p_last, 16) || (p_prev && !aligned(p_prev, 16)))
+    return WALL_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * HQ > 0x7fffffffLL) return WALL_ERR_UNSUPPORTED;
+  wall::CacheArgs a;
+  a.k_new = k_new; a.g_new = g_new; a.p_prev = p_prev;
+  a.B = B; a.t_start = t_start; a.T_new = T_new; a.cap = cap; a.HQ = HQ; a.H = H; a.K = K;
+  a.chunk = chunk; a.k_tilde = k_tilde; a.r_cache = r_cache; a.p_last = p_last;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(wall::launch_cache_build(a, dt == WALL_DTYPE_BF16, st), st);
+}
+
+size_t wall_attn_decode_workspace_size(int B, int T_kv, int HQ, int H, int V, int chunk) {
+  if (B <= 0 || T_kv <= 0 || HQ <= 0 || H <= 0 || V <= 0 || chunk <= 0) return 0;
+  const int ns = wall::decode_max_splits(B, T_kv, HQ, H, chunk);
+  return wall::decode_workspace_bytes(B, HQ, V, ns);
+}
+
+wall_status_t wall_attn_decode(const void* q, const float* p_curr, const void* v,
+                               const void* k_tilde, const float* r_cache, const float* sink_bias,
+                               int B, int T_kv, int cap, int HQ, int H, int K, int V, int chunk,
+                               wall_dtype_t dt, float scale, void* o, float* lse, void* workspace,
+                               size_t workspace_bytes, wall_stream_t stream) {
+  if (B < 0 || T_kv < 1 || cap < T_kv || HQ <= 0 || H <= 0 || HQ % H != 0)
+    return WALL_ERR_INVALID_ARG;
+  if (dt != WALL_DTYPE_F32 && dt != WALL_DTYPE_BF16) return WALL_ERR_INVALID_ARG;
+  if (!wall::decode_supported(K, V, HQ / H)) return WALL_ERR_UNSUPPORTED;
+  if (chunk != 32 && chunk != 64 && chunk != 128) return WALL_ERR_UNSUPPORTED;
+  if (B == 0) return WALL_OK;
+  if (!q || !p_curr || !v || !k_tilde || !r_cache || !o || !workspace) return WALL_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(p_curr, 16) || !aligned(v, 16) || !aligned(k_tilde, 16) ||
+      !aligned(r_cache, 16) || !aligned(o, 16) || !aligned(workspace, 16) ||
+      (sink_bias && !aligned(sink_bias, 4)) || (lse && !aligned(lse, 4)))
+    return WALL_ERR_INVALID_ARG;
+  const int ns = wall::decode_num_splits(B, T_kv, HQ, H, chunk);
+  if (workspace_bytes < wall::decode_workspace_bytes(B, HQ, V, ns)) return WALL_ERR_WORKSPACE;
+  if (!(scale > 0.f) || !std::isfinite(scale)) scale = 1.f / std::sqrt(static_cast<float>(K));
+  wall::DecodeArgs a;
+  a.q = q; a.p_curr = p_curr; a.v = v; a.k_tilde = k_tilde; a.r_cache = r_cache;
+  a.sink = sink_bias; a.B = B; a.T_kv = T_kv; a.cap = cap; a.HQ = HQ; a.H = H; a.K = K;
+  a.V = V; a.chunk = chunk; a.scale = scale; a.o = o; a.lse = lse;
+  a.part = static_cast<float*>(workspace); a.nsplit = ns;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(wall::launch_decode(a, dt == WALL_DTYPE_BF16, st), st);
+}
+
+wall_status_t wall_device_error(wall_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return WALL_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpyFromSymbol(&h, g_wall_err, sizeof(int)) != cudaSuccess) return WALL_ERR_CUDA;
+  if (h != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_wall_err, &zero, sizeof(int)) != cudaSuccess) return WALL_ERR_CUDA;
+    return WALL_ERR_DEVICE_TIMEOUT;
+  }
+  return WALL_OK;
+}
+
+void wall_debug_set_fault(int mode, int wait_ms) {
+  g_fault_mode.store(mode);
+  g_wait_ms.store(wait_ms > 0 ? wait_ms : 2000);
+}
+
+}  // extern "C"

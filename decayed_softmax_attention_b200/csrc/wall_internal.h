@@ -1,0 +1,92 @@
+// Host-side launchers shared by the translation units of the Wall attention
+// library.  Not part of the public C ABI (include/wall_attn.h is).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace wall {
+
+constexpr int kBlockRows = 128;  // anchor block / tile height shared by the prefill kernels
+
+// Workspace of the prefill forward.  NB = ceil(T / 128) anchor blocks.
+//   qh, kh  [B*HQ][T][K]   anchored q and k (input dtype):
+//           qh[t] = q[t] * exp(G[t] - AQ[blk(t)]),  kh[t] = k[t] * exp(AK[blk(t)] - G[t])
+//   bsum    [B*HQ][NB][K]  per-block sum of g (natural log)
+//   AQ, AK  [B*HQ][NB][K]  G just before the block's first row / at its last row
+//   ssl     [B*HQ][NB*128] block-local inclusive prefix of g_scalar * log2(e)
+//   ssb     [B*HQ][NB]     block sum of g_scalar * log2(e)
+//   ssa     [B*HQ][NB][4]  prefix of g_scalar * log2(e) before the block ([0] used)
+//   rowlo   [T]            first admitted key per row (packed documents only)
+struct FwdWork {
+  void* qh;
+  void* kh;
+  float* bsum;
+  float* AQ;
+  float* AK;
+  float* ssl;
+  float* ssb;
+  float* ssa;
+  int* rowlo;
+};
+
+struct FwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* g;
+  const void* g_scalar;
+  const float* sink;
+  const int32_t* cu_seqlens;
+  int num_seqs;
+  int window;
+  int B, T, HQ, H, K, V, NB;
+  float scale;
+  void* o;
+  float* lse;
+  int* err;
+  uint64_t wait_ns;
+  int fault;
+};
+
+size_t fwd_workspace_layout(int B, int T, int HQ, int K, bool bf16, FwdWork* w, char* base);
+
+cudaError_t launch_prep(const FwdArgs& a, const FwdWork& w, bool bf16, cudaStream_t st);
+cudaError_t launch_fwd_tc(const FwdArgs& a, const FwdWork& w, const CUtensorMap& tmQ,
+                          const CUtensorMap& tmK, const CUtensorMap& tmV, cudaStream_t st);
+cudaError_t launch_fwd_simt(const FwdArgs& a, const FwdWork& w, cudaStream_t st);
+
+struct CacheArgs {
+  const void* k_new;
+  const void* g_new;
+  const float* p_prev;
+  int B, t_start, T_new, cap, HQ, H, K, chunk;
+  void* k_tilde;
+  float* r_cache;
+  float* p_last;
+};
+cudaError_t launch_cache_build(const CacheArgs& a, bool bf16, cudaStream_t st);
+
+struct DecodeArgs {
+  const void* q;
+  const float* p_curr;
+  const void* v;
+  const void* k_tilde;
+  const float* r_cache;
+  const float* sink;
+  int B, T_kv, cap, HQ, H, K, V, chunk;
+  float scale;
+  void* o;
+  float* lse;
+  float* part;  // workspace
+  int nsplit;
+};
+int decode_max_splits(int B, int T_kv, int HQ, int H, int chunk);
+int decode_num_splits(int B, int T_kv, int HQ, int H, int chunk);
+size_t decode_workspace_bytes(int B, int HQ, int V, int nsplit);
+bool decode_supported(int K, int V, int group);
+cudaError_t launch_decode(const DecodeArgs& a, bool bf16, cudaStream_t st);
+
+}  // namespace wall

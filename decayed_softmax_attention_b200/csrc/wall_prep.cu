@@ -1,0 +1,210 @@
+// Prefill prepass of Wall attention (Wall Attention README, "Usage" shapes;
+// the decay of the intro formula folded into anchored operands).
+//
+// The score's per-channel factor exp(G[i,n] - G[j,n]) splits exactly as
+//   exp(G[i] - AQ) * exp(AQ - AK) * exp(AK - G[j])
+// for any anchors AQ, AK.  With AQ = G just before the query's 128-row block
+// and AK = G at the last row of the key's block, the first and last factors
+// are folded once into qh and kh here, and the middle one (one vector per
+// (query block, key block) pair) is applied to each key tile inside the main
+// kernel.  Every factor then spans at most one 128-row block, so the
+// exponents stay bounded at any sequence length.  Prefix sums run over the
+// whole row; with packed documents only differences inside a document are
+// ever used, so they equal the per-document sums of the definition.
+#include "wall_common.cuh"
+#include "wall_internal.h"
+
+namespace wall {
+namespace {
+
+// One CTA per (128-row block, batch*query head).  Thread layout: CG channel
+// groups of 8 channels x RG row groups of RPG consecutive rows.
+template <typename Tin, int KD>
+__global__ void __launch_bounds__(128) prep_local_kernel(
+    const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ g,
+    const Tin* __restrict__ gs, const int32_t* __restrict__ cu, int nseq, int window, int T,
+    int HQ, int H, int NB, Tin* __restrict__ qh, Tin* __restrict__ kh, float* __restrict__ bsum,
+    float* __restrict__ ssl, float* __restrict__ ssb, int* __restrict__ rowlo) {
+  constexpr int CG = KD / 8;
+  constexpr int RG = 128 / CG;
+  constexpr int RPG = 128 / RG;
+  __shared__ float tot[RG][KD];
+  __shared__ float wsum[4];
+
+  const int blk = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / HQ, hq = bh % HQ, kvh = hq / (HQ / H);
+  const int tid = threadIdx.x, cg = tid % CG, rg = tid / CG;
+  const int t0 = blk * kBlockRows + rg * RPG;
+  const size_t qrow = static_cast<size_t>(HQ) * KD;  // elements between time steps (q, g)
+  const size_t krow = static_cast<size_t>(H) * KD;   // (k)
+  const Tin* gb = g + (static_cast<size_t>(b) * T) * qrow + static_cast<size_t>(hq) * KD + cg * 8;
+
+  float acc[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+  for (int m = 0; m < RPG; ++m) {
+    const int t = t0 + m;
+    if (t >= T) break;
+    float f[8];
+    load8(gb + static_cast<size_t>(t) * qrow, f);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] += f[c];
+  }
+#pragma unroll
+  for (int c = 0; c < 8; ++c) tot[rg][cg * 8 + c] = acc[c];
+  __syncthreads();
+
+  float run[8], total[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float pre = 0.f, all = 0.f;
+    for (int r = 0; r < RG; ++r) {
+      const float x = tot[r][cg * 8 + c];
+      all += x;
+      if (r < rg) pre += x;
+    }
+    run[c] = pre;
+    total[c] = all;
+  }
+  if (rg == 0) {
+    float* dst = bsum + (static_cast<size_t>(bh) * NB + blk) * KD + cg * 8;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) dst[c] = total[c];
+  }
+
+  const Tin* qb = q + (static_cast<size_t>(b) * T) * qrow + static_cast<size_t>(hq) * KD + cg * 8;
+  const Tin* kb = k + (static_cast<size_t>(b) * T) * krow + static_cast<size_t>(kvh) * KD + cg * 8;
+  Tin* qo = qh + static_cast<size_t>(bh) * T * KD + cg * 8;
+  Tin* ko = kh + static_cast<size_t>(bh) * T * KD + cg * 8;
+  for (int m = 0; m < RPG; ++m) {
+    const int t = t0 + m;
+    if (t >= T) break;
+    float f[8], x[8], y[8];
+    load8(gb + static_cast<size_t>(t) * qrow, f);
+    load8(qb + static_cast<size_t>(t) * qrow, x);
+    load8(kb + static_cast<size_t>(t) * krow, y);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      run[c] += f[c];
+      x[c] *= expf(run[c]);
+      y[c] *= expf(total[c] - run[c]);
+    }
+    store8(qo + static_cast<size_t>(t) * KD, x);
+    store8(ko + static_cast<size_t>(t) * KD, y);
+  }
+
+  // Scalar gate: block-local inclusive prefix (log2 units), one row per thread.
+  if (gs != nullptr) {
+    const int t = blk * kBlockRows + tid;
+    float x = (t < T) ? load1(gs + (static_cast<size_t>(b) * T + t) * HQ + hq) * kLog2e : 0.f;
+    const int lane = tid & 31, wid = tid >> 5;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += y;
+    }
+    if (lane == 31) wsum[wid] = x;
+    __syncthreads();
+    for (int w = 0; w < wid; ++w) x += wsum[w];
+    ssl[static_cast<size_t>(bh) * NB * kBlockRows + blk * kBlockRows + tid] = x;
+    if (tid == kBlockRows - 1) ssb[static_cast<size_t>(bh) * NB + blk] = x;
+  }
+
+  // First admitted key of each row for packed documents (shared by all heads).
+  if (cu != nullptr && bh == 0) {
+    const int t = blk * kBlockRows + tid;
+    if (t < T) {
+      int lo = 0, hi = nseq;  // largest d with cu[d] <= t
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (cu[mid] <= t) lo = mid; else hi = mid;
+      }
+      int s = cu[lo];
+      s = s < 0 ? 0 : (s > t ? t : s);
+      if (window > 0 && t - window + 1 > s) s = t - window + 1;
+      rowlo[t] = s;
+    }
+  }
+}
+
+// Exclusive scan of the block sums over the blocks of one (batch, head).
+template <int KD>
+__global__ void __launch_bounds__(KD + 32) prep_scan_kernel(const float* __restrict__ bsum,
+                                                            const float* __restrict__ ssb, int NB,
+                                                            float* __restrict__ AQ,
+                                                            float* __restrict__ AK,
+                                                            float* __restrict__ ssa) {
+  const int bh = blockIdx.x, tid = threadIdx.x;
+  if (tid < KD) {
+    float acc = 0.f;
+    const size_t base = static_cast<size_t>(bh) * NB * KD + tid;
+    for (int blk = 0; blk < NB; ++blk) {
+      const size_t i = base + static_cast<size_t>(blk) * KD;
+      AQ[i] = acc;
+      acc += bsum[i];
+      AK[i] = acc;
+    }
+  } else if (tid == KD && ssb != nullptr) {
+    float acc = 0.f;
+    for (int blk = 0; blk < NB; ++blk) {
+      const size_t i = static_cast<size_t>(bh) * NB + blk;
+      ssa[i * 4] = acc;
+      ssa[i * 4 + 1] = 0.f;
+      ssa[i * 4 + 2] = 0.f;
+      ssa[i * 4 + 3] = 0.f;
+      acc += ssb[i];
+    }
+  }
+}
+
+template <typename Tin, int KD>
+cudaError_t prep_impl(const FwdArgs& a, const FwdWork& w, cudaStream_t st) {
+  const int BHQ = a.B * a.HQ;
+  dim3 grid(a.NB, BHQ);
+  prep_local_kernel<Tin, KD><<<grid, 128, 0, st>>>(
+      static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.g),
+      static_cast<const Tin*>(a.g_scalar), a.cu_seqlens, a.num_seqs, a.window, a.T, a.HQ, a.H,
+      a.NB, static_cast<Tin*>(w.qh), static_cast<Tin*>(w.kh), w.bsum, w.ssl, w.ssb, w.rowlo);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  prep_scan_kernel<KD><<<BHQ, KD + 32, 0, st>>>(w.bsum, a.g_scalar ? w.ssb : nullptr, a.NB, w.AQ,
+                                                 w.AK, w.ssa);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prep(const FwdArgs& a, const FwdWork& w, bool bf16, cudaStream_t st) {
+  if (bf16) {
+    return a.K == 64 ? prep_impl<__nv_bfloat16, 64>(a, w, st) : prep_impl<__nv_bfloat16, 128>(a, w, st);
+  }
+  return a.K == 64 ? prep_impl<float, 64>(a, w, st) : prep_impl<float, 128>(a, w, st);
+}
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t fwd_workspace_layout(int B, int T, int HQ, int K, bool bf16, FwdWork* w, char* base) {
+  const size_t BHQ = static_cast<size_t>(B) * HQ;
+  const size_t NB = (static_cast<size_t>(T) + kBlockRows - 1) / kBlockRows;
+  const size_t esz = bf16 ? 2 : 4;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return base ? static_cast<void*>(base + o) : nullptr;
+  };
+  FwdWork tmp;
+  FwdWork* p = w ? w : &tmp;
+  p->qh = take(BHQ * T * K * esz);
+  p->kh = take(BHQ * T * K * esz);
+  p->bsum = static_cast<float*>(take(BHQ * NB * K * 4));
+  p->AQ = static_cast<float*>(take(BHQ * NB * K * 4));
+  p->AK = static_cast<float*>(take(BHQ * NB * K * 4));
+  p->ssl = static_cast<float*>(take(BHQ * NB * kBlockRows * 4));
+  p->ssb = static_cast<float*>(take(BHQ * NB * 4));
+  p->ssa = static_cast<float*>(take(BHQ * NB * 16));
+  p->rowlo = static_cast<int*>(take(static_cast<size_t>(T) * 4 + 16));
+  return off;
+}
+
+}  // namespace wall

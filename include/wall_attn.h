@@ -1,0 +1,174 @@
+/*
+ * wall_attn.h -- C ABI of the B200 (sm_100a) Wall attention library.
+ *
+ * Wall attention ("decayed softmax attention") scores a query/key pair (i, j)
+ * by the q.k dot product in which every channel n carries the learned decay
+ * accumulated between the two positions (Wall Attention README, intro):
+ *
+ *   x(i,j) = scale * sum_n q[i,n] k[j,n] exp(G[i,n] - G[j,n]) + Gs[i] - Gs[j]
+ *
+ * with G the inclusive cumulative sum of the per-channel log-decay g over
+ * time and Gs that of the optional scalar gate g_scalar.  Softmax runs over
+ * the admitted keys j <= i (plus an optional sink logit); g = 0 gives vanilla
+ * causal softmax attention.
+ *
+ * Conventions shared by every call
+ *   - All tensors are dense, row-major, last dimension contiguous, in DEVICE
+ *     memory, and owned by the caller.  The library never allocates, frees or
+ *     synchronises (except when the environment variable WALL_DEBUG_SYNC=1 is
+ *     set, which makes every call synchronise and report device errors).
+ *   - Every call is asynchronous on `stream` (NULL = the legacy default stream)
+ *     and is reentrant; the only global mutable state is the per-device
+ *     error word read by wall_device_error().
+ *   - Element types: `wall_dtype_t` selects bf16 or fp32 for q, k, v, g,
+ *     g_scalar, o and k_tilde; sink_bias, lse, p_prev/p_last/p_curr and
+ *     r_cache are always fp32.
+ *   - Supported head dims: K, V in {64, 128}; HQ % H == 0 (GQA: query head hq
+ *     reads KV head hq / (HQ / H)).  Anything else: WALL_ERR_UNSUPPORTED.
+ *   - Pointers must be 16-byte aligned; a misaligned or NULL required pointer,
+ *     a negative size or an inconsistent shape returns WALL_ERR_INVALID_ARG
+ *     before any work is queued.  Errors never abort the process; there is no
+ *     CPU fallback.
+ */
+#ifndef WALL_ATTN_H_
+#define WALL_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t (a pointer to the driver's opaque stream struct). */
+struct CUstream_st;
+typedef struct CUstream_st* wall_stream_t;
+
+typedef enum {
+  WALL_OK = 0,
+  WALL_ERR_INVALID_ARG = 1,    /* bad pointer, shape, size or alignment */
+  WALL_ERR_UNSUPPORTED = 2,    /* valid but not implemented (e.g. K = 96) */
+  WALL_ERR_CUDA = 3,           /* a CUDA runtime/driver call failed */
+  WALL_ERR_DEVICE_TIMEOUT = 4, /* a bounded device-side wait gave up */
+  WALL_ERR_WORKSPACE = 5       /* workspace too small */
+} wall_status_t;
+
+typedef enum { WALL_DTYPE_F32 = 0, WALL_DTYPE_BF16 = 1 } wall_dtype_t;
+
+/* Human-readable name of a status code (static string). */
+const char* wall_status_string(wall_status_t status);
+
+/*
+ * Prefill forward (Wall Attention README, "Usage / Training-Prefill"):
+ *   o = wall_attn(q, k, v, g, scale, g_scalar, sink_bias, window_size, cu_seqlens)
+ *
+ *   q         [B, T, HQ, K]  dtype dt
+ *   k         [B, T, H,  K]  dtype dt
+ *   v         [B, T, H,  V]  dtype dt
+ *   g         [B, T, HQ, K]  dtype dt  per-channel log-decay (natural log)
+ *   g_scalar  [B, T, HQ]     dtype dt  nullable; additive FoX-style gate: the
+ *                                      logit gains Gs[i] - Gs[j]
+ *   sink_bias [HQ]           fp32      nullable; one extra logit per head with
+ *                                      a zero value (adds to the normaliser)
+ *   window    keep keys with 0 <= i - j < window; window <= 0: no window
+ *   cu_seqlens int32 [num_seqs + 1] device, nullable; variable-length packing
+ *             (requires B == 1): cu[0] = 0, cu[num_seqs] = T, strictly
+ *             increasing; attention never crosses a document boundary and the
+ *             cumulative sums restart at each document.  The values are read
+ *             on the device only; out-of-range values are clamped, never
+ *             dereferenced out of bounds, but give unspecified results.
+ *   scale     softmax scale on the decayed q.k sum; <= 0 means K^-0.5
+ *   o         [B, T, HQ, V]  dtype dt  output
+ *   lse       [B, T, HQ]     fp32      nullable; natural-log normaliser,
+ *                                      sink included
+ *   workspace caller-owned device scratch of at least
+ *             wall_attn_fwd_workspace_size(...) bytes, 256-byte aligned; its
+ *             contents need no initialisation and are clobbered.
+ * T == 0 (or B == 0) is a no-op returning WALL_OK.
+ */
+size_t wall_attn_fwd_workspace_size(int B, int T, int HQ, int H, int K, int V,
+                                    wall_dtype_t dt);
+
+wall_status_t wall_attn_fwd(const void* q, const void* k, const void* v, const void* g,
+                            const void* g_scalar, const float* sink_bias, int window,
+                            const int32_t* cu_seqlens, int num_seqs, int B, int T, int HQ,
+                            int H, int K, int V, wall_dtype_t dt, float scale, void* o,
+                            float* lse, void* workspace, size_t workspace_bytes,
+                            wall_stream_t stream);
+
+/*
+ * Decode cache build / append (Wall Attention README, "Decode"):
+ *   P = cumsum(g) * (1/ln 2);  k_tilde[j] = k[j] * exp2(R_c - P[j])
+ * with one anchor vector R_c = P[c * chunk] per chunk of `chunk` tokens (the
+ * chunk's first token, so appending never rewrites earlier rows).
+ * Writes cache rows t_start .. t_start + T_new - 1.
+ *
+ *   k_new   [B, T_new, H,  K]  dtype dt   keys of the new tokens
+ *   g_new   [B, T_new, HQ, K]  dtype dt   log-decay of the new tokens
+ *   p_prev  [B, HQ, K] fp32    P at row t_start - 1; NULL iff t_start == 0
+ *   k_tilde [B, cap, HQ, K]    dtype dt   cache (rows below t_start untouched)
+ *   r_cache [B, ceil(cap/chunk), HQ, K] fp32  anchors; a chunk whose first row
+ *           is below t_start must already hold its anchor (it is read)
+ *   p_last  [B, HQ, K] fp32    out: P at row t_start + T_new - 1 (pass it as
+ *           p_curr to wall_attn_decode and as p_prev to the next append)
+ * Requires 0 <= t_start, t_start + T_new <= cap, chunk in {32, 64, 128}
+ * (WALL_ERR_UNSUPPORTED otherwise).  p_last may alias p_prev.  T_new == 0 is
+ * a no-op.
+ */
+wall_status_t wall_build_kv_cache(const void* k_new, const void* g_new, const float* p_prev,
+                                  int B, int t_start, int T_new, int cap, int HQ, int H, int K,
+                                  int chunk, wall_dtype_t dt, void* k_tilde, float* r_cache,
+                                  float* p_last, wall_stream_t stream);
+
+/*
+ * Single-step decode over the pre-rescaled cache (Wall Attention README,
+ * "Decode"): the current query attends cache rows 0 .. T_kv - 1 (the current
+ * token included: append first, then attend):
+ *   x_j = scale * sum_n q[n] k_tilde[j,n] exp2(p_curr[n] - R_{j/chunk}[n])
+ *
+ *   q        [B, 1, HQ, K]  dtype dt
+ *   p_curr   [B, 1, HQ, K]  fp32  P at the current token (p_last of the append)
+ *   v        [B, cap, H, V] dtype dt  value cache (rows < T_kv valid)
+ *   k_tilde  [B, cap, HQ, K] dtype dt, r_cache [B, ceil(cap/chunk), HQ, K] fp32
+ *   sink_bias [HQ] fp32, nullable
+ *   o        [B, 1, HQ, V]  dtype dt;  lse [B, 1, HQ] fp32, nullable
+ *   workspace >= wall_attn_decode_workspace_size(B, T_kv, HQ, H, V, chunk)
+ *            bytes, 16-byte aligned, no initialisation needed.
+ * Split-KV: partial (o, max, sum) per split, merged by a combine pass.  The
+ * split count grows with T_kv, so a workspace sized for T_kv = cap serves
+ * every step of a streaming loop.
+ * Requires 1 <= T_kv <= cap, chunk in {32, 64, 128}, HQ / H in
+ * {1, 2, 4, 8, 16}.  Decode has no g_scalar term (the README's decode call
+ * takes none).
+ */
+size_t wall_attn_decode_workspace_size(int B, int T_kv, int HQ, int H, int V, int chunk);
+
+wall_status_t wall_attn_decode(const void* q, const float* p_curr, const void* v,
+                               const void* k_tilde, const float* r_cache, const float* sink_bias,
+                               int B, int T_kv, int cap, int HQ, int H, int K, int V, int chunk,
+                               wall_dtype_t dt, float scale, void* o, float* lse, void* workspace,
+                               size_t workspace_bytes, wall_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears this device's error word.
+ * Returns WALL_ERR_DEVICE_TIMEOUT if any kernel since the last read gave up a
+ * bounded wait (its outputs are then unspecified), WALL_ERR_CUDA if the
+ * synchronisation failed, WALL_OK otherwise.
+ */
+wall_status_t wall_device_error(wall_stream_t stream);
+
+/*
+ * Testing hook (not for production use): mode 1 makes the next prefill
+ * launches skip the producer's first K/V tile load, so the consumers' bounded
+ * waits run out and report WALL_ERR_DEVICE_TIMEOUT through the error word
+ * (no GPU fault, no hang: every wait gives up after about wait_ms
+ * milliseconds).  mode 0 restores normal operation.  wait_ms <= 0 keeps the
+ * default limit (2000 ms).
+ */
+void wall_debug_set_fault(int mode, int wait_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WALL_ATTN_H_ */

@@ -1,0 +1,157 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function the
+public header declares, and rejects bad arguments on the host before any
+CUDA call (status codes, no crash)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import decayed_softmax_attention_b200 as wall
+from decayed_softmax_attention_b200 import build as wall_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wall_attn.h")
+
+INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 5
+BF16, F32 = 1, 0
+
+
+@pytest.fixture(scope="module")
+def lib():
+    wall_build.build()
+    return wall.load_library()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(wall_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_three_calls():
+    names = _declared_functions()
+    for n in ("wall_attn_fwd", "wall_build_kv_cache", "wall_attn_decode"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert set(names) == set(wall.EXPORTED_SYMBOLS)
+    for n in names:
+        assert hasattr(lib, n), f"{n} missing from {wall.lib_path()}"
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        s = lib.wall_status_string(code).decode()
+        assert s.startswith("WALL_")
+
+
+def _fake(addr=0x1000):
+    return ctypes.c_void_p(addr)
+
+
+def _fwd(lib, **kw):
+    a = dict(q=_fake(), k=_fake(), v=_fake(), g=_fake(), gs=None, sink=None, window=0, cu=None,
+             nseq=0, B=1, T=64, HQ=4, H=2, K=64, V=64, dt=BF16, scale=0.0, o=_fake(), lse=None,
+             ws=_fake(0x100000), wsb=1 << 40, stream=None)
+    a.update(kw)
+    return lib.wall_attn_fwd(a["q"], a["k"], a["v"], a["g"], a["gs"], a["sink"], a["window"],
+                             a["cu"], a["nseq"], a["B"], a["T"], a["HQ"], a["H"], a["K"], a["V"],
+                             a["dt"], a["scale"], a["o"], a["lse"], a["ws"], a["wsb"], a["stream"])
+
+
+def test_fwd_host_validation(lib):
+    assert _fwd(lib, HQ=6, H=4) == INVALID            # HQ % H != 0
+    assert _fwd(lib, K=96) == UNSUPPORTED
+    assert _fwd(lib, V=32) == UNSUPPORTED
+    assert _fwd(lib, dt=7) == INVALID
+    assert _fwd(lib, B=-1) == INVALID
+    assert _fwd(lib, q=None) == INVALID
+    assert _fwd(lib, o=None) == INVALID
+    assert _fwd(lib, q=_fake(0x1008)) == INVALID      # not 16-byte aligned
+    assert _fwd(lib, ws=_fake(0x100010)) == INVALID   # workspace not 256-byte aligned
+    assert _fwd(lib, cu=_fake(), nseq=2, B=2) == INVALID  # packing needs B == 1
+    assert _fwd(lib, cu=_fake(), nseq=0) == INVALID
+    assert _fwd(lib, wsb=16) == WORKSPACE
+    assert _fwd(lib, T=0) == 0                        # empty input: no-op
+    assert _fwd(lib, B=0) == 0
+
+
+def test_fwd_workspace_size(lib):
+    small = lib.wall_attn_fwd_workspace_size(1, 128, 2, 2, 64, 64, BF16)
+    big = lib.wall_attn_fwd_workspace_size(1, 8192, 32, 8, 128, 128, BF16)
+    f32 = lib.wall_attn_fwd_workspace_size(1, 128, 2, 2, 64, 64, F32)
+    assert 0 < small < f32
+    # anchored q and k dominate: 2 * B*HQ*T*K elements
+    assert big >= 2 * 32 * 8192 * 128 * 2
+    assert lib.wall_attn_fwd_workspace_size(0, 128, 2, 2, 64, 64, BF16) == 0
+
+
+def _cache(lib, **kw):
+    a = dict(k=_fake(), g=_fake(), p_prev=None, B=2, t0=0, Tn=64, cap=128, HQ=4, H=2, K=128,
+             C=64, dt=BF16, kt=_fake(), r=_fake(), pl=_fake(), stream=None)
+    a.update(kw)
+    return lib.wall_build_kv_cache(a["k"], a["g"], a["p_prev"], a["B"], a["t0"], a["Tn"], a["cap"],
+                                   a["HQ"], a["H"], a["K"], a["C"], a["dt"], a["kt"], a["r"],
+                                   a["pl"], a["stream"])
+
+
+def test_cache_host_validation(lib):
+    assert _cache(lib, t0=100, Tn=64) == INVALID          # beyond capacity
+    assert _cache(lib, t0=10, p_prev=None) == INVALID      # append needs the previous prefix
+    assert _cache(lib, t0=0, p_prev=_fake()) == INVALID    # fresh build takes none
+    assert _cache(lib, C=48) == UNSUPPORTED
+    assert _cache(lib, K=80) == UNSUPPORTED
+    assert _cache(lib, HQ=3) == INVALID
+    assert _cache(lib, kt=None) == INVALID
+    assert _cache(lib, r=_fake(0x1004)) == INVALID
+    assert _cache(lib, Tn=0) == 0
+
+
+def _dec(lib, **kw):
+    a = dict(q=_fake(), pc=_fake(), v=_fake(), kt=_fake(), r=_fake(), sink=None, B=2, Tkv=100,
+             cap=128, HQ=8, H=2, K=128, V=128, C=64, dt=BF16, scale=0.0, o=_fake(), lse=None,
+             ws=_fake(), wsb=1 << 40, stream=None)
+    a.update(kw)
+    return lib.wall_attn_decode(a["q"], a["pc"], a["v"], a["kt"], a["r"], a["sink"], a["B"],
+                                a["Tkv"], a["cap"], a["HQ"], a["H"], a["K"], a["V"], a["C"],
+                                a["dt"], a["scale"], a["o"], a["lse"], a["ws"], a["wsb"],
+                                a["stream"])
+
+
+def test_decode_host_validation(lib):
+    assert _dec(lib, Tkv=0) == INVALID
+    assert _dec(lib, Tkv=200) == INVALID                  # more rows than the cache holds
+    assert _dec(lib, HQ=96, H=3) == UNSUPPORTED           # group of 32 query heads
+    assert _dec(lib, K=32) == UNSUPPORTED
+    assert _dec(lib, C=50) == UNSUPPORTED
+    assert _dec(lib, kt=None) == INVALID
+    assert _dec(lib, o=_fake(0x1002)) == INVALID
+    assert _dec(lib, wsb=8) == WORKSPACE
+
+
+def test_decode_workspace_monotone_in_length(lib):
+    prev = 0
+    for T in (1, 63, 64, 65, 640, 6400, 32768, 32832):
+        ws = lib.wall_attn_decode_workspace_size(32, T, 32, 8, 128, 64)
+        assert ws >= prev
+        prev = ws
+
+
+def test_binding_fails_loudly_without_cuda_tensors():
+    import torch
+    q = torch.zeros(1, 4, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises((ValueError, ImportError)):
+        wall.wall_attn_fwd(q, torch.zeros(1, 4, 2, 64, dtype=torch.bfloat16),
+                           torch.zeros(1, 4, 2, 64, dtype=torch.bfloat16), q)
+
+
+def test_product_path_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "decayed_softmax_attention_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in text.lower().replace("oracle/", ""), f
