@@ -1,0 +1,528 @@
+#!/usr/bin/env python
+"""Wall attention benchmark on B200.
+
+One step is one pass of the whole hot path over synthetic inputs:
+  * prefill forward on the long workload (B=1, T=8192, HQ=32, H=8, K=V=128,
+    bf16, g = -softplus(N(0,1)-4) per channel, g_scalar likewise): prepass +
+    tcgen05 attention kernel;
+  * a 64-token streaming decode on the decode workload (B=32, prefix
+    T_kv=32768 built once in set-up, HQ=32, H=8, K=V=128, C=64): per token,
+    append to the pre-rescaled cache, then split-KV decode + combine.
+
+Printed (rank 0, one JSON line): prefill TFLOP/s (the headline `value`),
+decode KV GB/s (`decode`), each with its roofline fraction against the
+measured B200 peaks; an end-to-end prefill number through host buffers
+(`e2e`); the CPU oracle's throughput on a bounded sample (`cpu_baseline`).
+
+Multi-GPU (torchrun): every rank runs its own independent shard (its own
+prefill sequence and its own decode batch, seeded by rank) -- the method has
+no exchange step -- and `value` is all ranks' work over the slowest rank's
+device time (weak scaling).
+
+`--impl reference` times the CPU oracle on bounded samples of the same
+prefill workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from dataclasses import replace
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic of the prefill attention kernel per launch on the long workload
+# (dram__bytes_read.sum + dram__bytes_write.sum from one ncu capture) and the
+# hash of the kernel source it was taken on; reported as null once the kernel
+# source changes.  Filled from profiles/ after each capture.
+TRAFFIC = {
+    # profiles/wall_fwd_tc_long_prefill.md: 428.170496 MB read + 58.283776 MB written
+    "prefill_main": {"bytes": 486454272, "source_sha": "3d917672a9a73f4d"},
+    # profiles/decode_split_b4_tkv32k.md, batch 4 scaled by 8 to batch 32 (traffic is
+    # proportional to the batch): (1.375986 GB + 5.748480 MB) * 8
+    "decode_split": {"bytes": 11053875840, "source_sha": "609266ee7d00583d"},
+}
+KERNEL_SOURCES = {
+    "prefill_main": "decayed_softmax_attention_b200/csrc/wall_fwd_tc.cu",
+    "decode_split": "decayed_softmax_attention_b200/csrc/wall_decode.cu",
+}
+
+
+# ----------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def source_sha(rel):
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def traffic_for(name):
+    t = TRAFFIC[name]
+    if t["bytes"] is None or t["source_sha"] != source_sha(KERNEL_SOURCES[name]):
+        return None
+    return t["bytes"]
+
+
+def prefill_pairs(spec):
+    """Admitted (query, key) pairs per (batch row, query head): causal, window, documents."""
+    W_ = spec.window
+    docs = spec.docs if spec.docs is not None else (spec.T,)
+    total = 0
+    for L in docs:
+        if W_ <= 0 or L <= W_:
+            total += L * (L + 1) // 2
+        else:
+            total += W_ * (W_ + 1) // 2 + (L - W_) * W_
+    return total
+
+
+def prefill_flops(spec):
+    """2*(K+V) FLOPs per admitted pair (QK^T and PV), all batch rows and query heads."""
+    return float(spec.B * spec.HQ * prefill_pairs(spec) * 2 * (spec.K + spec.V))
+
+
+def decode_bytes(spec, T_kv):
+    """Algorithmic HBM bytes of one decode step attending T_kv cache rows."""
+    esz = 2 if spec.dtype == "bf16" else 4
+    B, HQ, H, K, V, C = spec.B, spec.HQ, spec.H, spec.K, spec.V, spec.C
+    ktilde = B * T_kv * HQ * K * esz
+    vals = B * T_kv * H * V * esz
+    anchors = B * ((T_kv + C - 1) // C) * HQ * K * 4
+    small = B * HQ * (K * esz + K * 4 + V * esz + 4)  # q, p_curr, o, lse
+    return ktilde + vals + anchors + small
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            sel = []
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="wall_clocks_", suffix=".csv")
+            self.fh = os.fdopen(fd, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, power, reasons = [], None, [], set()
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    smax = float(parts[1])
+                    power.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names[1:], parts[4:8]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        loaded = [s for s in sm if smax and s > 0.3 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": smax,
+                "power_w_max": max(power) if power else None, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_max(x, world, device):
+    """Max over ranks of a host float (timing only; no data-path collective)."""
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def shard_specs(rank):
+    """This rank's independent shard: the long prefill and the decode batch, seeded by rank."""
+    p = W.PREFILL["long"]
+    d = W.DECODE["decode"]
+    return replace(p, seed=p.seed + 100 * rank), replace(d, seed=d.seed + 100 * rank)
+
+
+# ----------------------------------------------------------------- CPU oracle timing
+def oracle_sample_rows(spec, n_rows):
+    """n_rows query rows spread evenly over the sequence (all heads), batch row 0."""
+    import numpy as np
+    return np.unique(np.linspace(0, spec.T - 1, n_rows).round().astype(np.int64))
+
+
+def time_oracle(spec, host, n_rows, threads):
+    import oracle
+    rows = oracle_sample_rows(spec, n_rows)
+    t0 = time.perf_counter()
+    oracle.wall_fwd(host["q"], host["k"], host["v"], host["g"], host["g_scalar"],
+                    host["sink_bias"], window=spec.window, scale=spec.softmax_scale, rows=rows,
+                    threads=threads)
+    dt = time.perf_counter() - t0
+    flops = float(sum(spec.HQ * (int(t) + 1) * 2 * (spec.K + spec.V) for t in rows))
+    return dt, flops, rows
+
+
+def cpu_baseline(spec, host, budget_s=15.0):
+    import oracle
+    threads = oracle.max_threads()
+    n = 8
+    dt, flops, rows = time_oracle(spec, host, n, threads)
+    if dt < budget_s / 4:
+        n = int(min(spec.T, max(n, n * budget_s / max(dt, 1e-3) * 0.8)))
+        dt, flops, rows = time_oracle(spec, host, n, threads)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{len(rows)} query rows evenly spaced over T={spec.T}, all {spec.HQ} heads "
+                      f"of the long prefill workload (batch row 0), double precision; "
+                      f"{dt:.1f} s"}
+
+
+def host_inputs(d):
+    return {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+
+
+# ----------------------------------------------------------------- reference arm
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    import oracle
+    spec, _ = shard_specs(0)
+    host = host_inputs(W.gen_prefill(spec, device="cpu"))
+    threads = oracle.max_threads()
+    # size the per-step sample to about 2 s of oracle work
+    dt, _, _ = time_oracle(spec, host, 4, threads)
+    n_rows = int(max(4, min(spec.T, 4 * 2.0 / max(dt, 1e-3))))
+    for _ in range(args.warmup):
+        time_oracle(spec, host, n_rows, threads)
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        dt, fl, rows = time_oracle(spec, host, n_rows, threads)
+        times.append(dt)
+        flops += fl
+    total = sum(times)
+    value = flops / total / 1e12
+    sample = (f"{n_rows} query rows evenly spaced over T={spec.T}, all {spec.HQ} heads of the "
+              f"long prefill workload per step, double precision")
+    line = {
+        "impl": "reference", "metric": "wall_attn_fwd TFLOP/s @ T=8K (long prefill)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(spec, None, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_block(pspec, dspec, n):
+    c = {
+        "workload": (f"prefill: long B={pspec.B} T={pspec.T} HQ={pspec.HQ} H={pspec.H} "
+                     f"K={pspec.K} V={pspec.V} {pspec.dtype} causal, g=-softplus(N(0,1)-4), "
+                     f"g_scalar=-softplus(N(0,1)-4)"),
+        "global_batch": pspec.B * n,
+        "seq_len": pspec.T,
+        "parallelism": f"dp{n} (independent shards, no collective)",
+        "l2": "inputs larger than L2: each step streams the 11 GB decode cache 64 times "
+              "between prefill passes (126 MB L2)",
+    }
+    if dspec is not None:
+        c["workload"] += (f"; decode: B={dspec.B} T_kv={dspec.T0}->{dspec.cap} HQ={dspec.HQ} "
+                          f"H={dspec.H} K={dspec.K} V={dspec.V} C={dspec.C} {dspec.dtype}, "
+                          f"{dspec.steps} streaming steps (append + decode)")
+    return c
+
+
+# ----------------------------------------------------------------- our arm
+def run_ours(args, world, rank, local):
+    import decayed_softmax_attention_b200 as wall
+    from decayed_softmax_attention_b200 import build as wall_build
+    if not os.path.exists(wall.lib_path()):
+        wall_build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks, peak_src = load_peaks()
+    pspec, dspec = shard_specs(rank)
+    dspec = replace(dspec, steps=args.decode_steps)
+    if args.decode_batch:
+        dspec = replace(dspec, B=args.decode_batch)
+    do_prefill = args.only in (None, "prefill")
+    do_decode = args.only in (None, "decode")
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    # ---- prefill set-up
+    if do_prefill:
+        pd = W.gen_prefill(pspec, device=dev)
+        B, T, HQ, H, K, V = pspec.B, pspec.T, pspec.HQ, pspec.H, pspec.K, pspec.V
+        o = torch.empty((B, T, HQ, V), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((B, T, HQ), dtype=torch.float32, device=dev)
+        ws = torch.empty(wall.wall_attn_fwd_workspace_size(B, T, HQ, H, K, V, torch.bfloat16),
+                         dtype=torch.uint8, device=dev)
+
+    def prefill():
+        wall.wall_attn_fwd(pd["q"], pd["k"], pd["v"], pd["g"], pd["g_scalar"], pd["sink_bias"],
+                           window=pd["window"], scale=pd["scale"], out=o, lse=lse, workspace=ws,
+                           return_lse=True)
+
+    # ---- decode set-up: build the prefix cache once (timed as a side number)
+    T0, S = dspec.T0, (dspec.steps if do_decode else 0)
+    build_ms = build_bytes = None
+    if do_decode:
+        dd = W.gen_decode(dspec, device=dev)
+        cache = wall.KVCache(dspec.B, dspec.cap, dspec.HQ, dspec.H, dspec.K, dspec.V,
+                             dtype=torch.bfloat16, chunk=dspec.C, device=dev)
+        cache.v.copy_(dd["v"])                   # value cache is the caller's; preload all rows
+        k_pre = dd["k"][:, :T0].contiguous()
+        g_pre = dd["g"][:, :T0].contiguous()
+        k_steps = [dd["k"][:, T0 + s:T0 + s + 1].contiguous() for s in range(S)]
+        g_steps = [dd["g"][:, T0 + s:T0 + s + 1].contiguous() for s in range(S)]
+        q_steps = [dd["q"][:, s:s + 1].contiguous() for s in range(S)]
+        del dd
+        dout = torch.empty((dspec.B, 1, dspec.HQ, dspec.V), dtype=torch.bfloat16, device=dev)
+        dlse = torch.empty((dspec.B, 1, dspec.HQ), dtype=torch.float32, device=dev)
+        p_prefix = torch.empty_like(cache.p)
+        e0, e1 = ev(), ev()
+        torch.cuda.synchronize()
+        e0.record()
+        cache.length = 0
+        cache.append(k_pre, g_pre)
+        e1.record()
+        torch.cuda.synchronize()
+        build_ms = e0.elapsed_time(e1)
+        esz = 2
+        build_bytes = (dspec.B * T0 * (dspec.H * dspec.K + dspec.HQ * dspec.K) * esz  # read k, g
+                       + dspec.B * T0 * dspec.HQ * dspec.K * esz                       # k_tilde
+                       + dspec.B * (T0 // dspec.C) * dspec.HQ * dspec.K * 4)            # anchors
+        p_prefix.copy_(cache.p)
+        del k_pre, g_pre
+
+    pre_ev = [[ev() for _ in range(3)] for _ in range(args.steps)] if do_prefill else []
+    dec_ev = [[[ev() for _ in range(3)] for _ in range(S)] for _ in range(args.steps)]
+    # torch creates the underlying cudaEvent_t on first record: record every
+    # event once here so the library receives valid handles to re-record.
+    for trio in pre_ev + [t for row in dec_ev for t in row]:
+        for e in trio:
+            e.record()
+    torch.cuda.synchronize()
+
+    def step(i=None):
+        if do_prefill:
+            if i is not None:
+                wall.wall_debug_set_stage_events(*pre_ev[i])
+            prefill()
+            if i is not None:
+                wall.wall_debug_set_stage_events()
+        if do_decode:
+            cache.length = T0
+            cache.p.copy_(p_prefix)
+            for s in range(S):
+                cache.append(k_steps[s], g_steps[s])
+                if i is not None:
+                    wall.wall_debug_set_stage_events(*dec_ev[i][s])
+                cache.decode(q_steps[s], scale=dspec.K ** -0.5, out=dout, lse=dlse)
+                if i is not None:
+                    wall.wall_debug_set_stage_events()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert wall.wall_device_error(dev) == 0
+
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    t_start, t_end = ev(), ev()
+    t_start.record()
+    for i in range(args.steps):
+        step(i)
+    t_end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    status = wall.wall_device_error(dev)
+    if status != 0:
+        raise RuntimeError(f"device error status {status} during the timed region")
+    total_ms = reduce_max(t_start.elapsed_time(t_end), world, dev)
+
+    line = {
+        "metric": "wall_attn_fwd TFLOP/s @ T=8K (long prefill)",
+        "value": None, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_block(pspec, dspec if do_decode else None, world),
+    }
+    side = {}
+    bf16_peak = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
+    hbm_peak = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+    if do_prefill:
+        pre_ms = [e[0].elapsed_time(e[2]) for e in pre_ev]
+        pre_prep_ms = [e[0].elapsed_time(e[1]) for e in pre_ev]
+        pre_main_ms = [e[1].elapsed_time(e[2]) for e in pre_ev]
+        flops = prefill_flops(pspec)
+        pre_total_ms = reduce_max(sum(pre_ms), world, dev)
+        value = world * flops * args.steps / (pre_total_ms * 1e-3) / 1e12
+        main_avg = statistics.mean(pre_main_ms)
+        achieved = flops / (main_avg * 1e-3) / 1e12
+        line["value"] = value
+        line["roofline"] = {
+            "kernel": "wall_fwd_tc_kernel (prefill attention)", "bound": "tensor",
+            "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s", "frac": achieved / bf16_peak,
+            "traffic": traffic_for("prefill_main"),
+            "peak_source": f"{peak_src} bf16_tflops (burst)",
+            "algorithmic_flops_per_launch": flops}
+        side.update({"prefill_ms": statistics.mean(pre_ms),
+                     "prefill_prepass_ms": statistics.mean(pre_prep_ms),
+                     "prefill_main_ms": main_avg,
+                     "frac_of_measured_peak_whole_prefill": value / world / bf16_peak})
+    if do_decode:
+        dec_ms = [[e[0].elapsed_time(e[2]) for e in row] for row in dec_ev]
+        dec_split_ms = [[e[0].elapsed_time(e[1]) for e in row] for row in dec_ev]
+        step_bytes = [decode_bytes(dspec, T0 + s + 1) for s in range(S)]
+        dec_total_ms = reduce_max(sum(sum(r) for r in dec_ms), world, dev)
+        dec_value = world * args.steps * sum(step_bytes) / (dec_total_ms * 1e-3) / 1e9
+        split_avg = statistics.mean(x for r in dec_split_ms for x in r)
+        dec_achieved = statistics.mean(step_bytes) / (split_avg * 1e-3) / 1e9
+        line["decode"] = {
+            "metric": f"wall_attn_decode KV GB/s (B={dspec.B}, T_kv {T0 + 1}..{T0 + S})",
+            "value": dec_value, "unit": "GB/s",
+            "ms_per_token": statistics.mean(x for r in dec_ms for x in r),
+            "roofline": {"kernel": "decode_split_kernel", "bound": "hbm", "achieved": dec_achieved,
+                         "peak": hbm_peak, "unit": "GB/s", "frac": dec_achieved / hbm_peak,
+                         "traffic": traffic_for("decode_split"),
+                         "peak_source": f"{peak_src} hbm_gbs",
+                         "algorithmic_bytes_per_launch": statistics.mean(step_bytes)},
+            "frac_of_hbm_incl_combine": dec_value / world / hbm_peak,
+        }
+        side.update({"cache_build_prefix_ms": build_ms,
+                     "cache_build_prefix_GBps": build_bytes / (build_ms * 1e-3) / 1e9})
+        if not do_prefill:
+            line["metric"] = line["decode"]["metric"]
+            line["value"], line["unit"] = dec_value, "GB/s"
+            line["roofline"] = line["decode"]["roofline"]
+    line["side"] = side
+
+    # ---- end to end through host buffers (pinned), prefill headline metric
+    if do_prefill and not args.no_e2e:
+        names = ["q", "k", "v", "g", "g_scalar"]
+        host = {n: pd[n].cpu().pin_memory() for n in names}
+        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+        d2h = o_host.numel() * o_host.element_size()
+
+        def e2e_step():
+            for n in names:
+                pd[n].copy_(host[n], non_blocking=True)
+            prefill()
+            o_host.copy_(o, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        a, b_ = ev(), ev()
+        a.record()
+        for _ in range(args.steps):
+            e2e_step()
+        b_.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = reduce_max(a.elapsed_time(b_), world, dev)
+        line["e2e"] = {"value": world * prefill_flops(pspec) * args.steps / (e2e_ms * 1e-3) / 1e12,
+                       "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    line["gpu_launches"] = args.steps * ((3 if do_prefill else 0) + 3 * S)
+    line["clocks"] = clk
+    if rank != 0:
+        return 0
+    if world == 1 and do_prefill and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(pspec, host_inputs(pd))
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--decode-steps", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+                    help="profiling runs: time one half of the step only")
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="profiling runs: smaller decode batch (default: the workload's B=32)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    try:
+        return run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

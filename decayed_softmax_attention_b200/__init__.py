@@ -3,8 +3,9 @@
 Thin Python binding over the C ABI in ``include/wall_attn.h``: argument
 marshalling only (dtype/shape checks, device pointers, the current CUDA
 stream, caller-side workspace allocation through torch).  Every step of the
-computation runs in the library's CUDA kernels; there is no CPU fallback, and
-importing this module on a machine without the built library raises.
+computation runs in the library's CUDA kernels; there is no CPU fallback: any
+entry point raises ImportError when the built library is missing, and
+ValueError when a tensor does not live in CUDA device memory.
 
 Public calls (same names as the C ABI):
   wall_attn_fwd(q, k, v, g, g_scalar=None, sink_bias=None, window=0,
@@ -25,7 +26,8 @@ import torch
 __all__ = [
     "WallError", "lib_path", "load_library", "wall_attn_fwd", "wall_attn_fwd_workspace_size",
     "wall_build_kv_cache", "wall_attn_decode", "wall_attn_decode_workspace_size",
-    "wall_device_error", "wall_debug_set_fault", "KVCache", "EXPORTED_SYMBOLS",
+    "wall_device_error", "wall_debug_set_fault", "wall_debug_set_stage_events", "KVCache",
+    "EXPORTED_SYMBOLS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -42,7 +44,7 @@ _STATUS = {
 EXPORTED_SYMBOLS = (
     "wall_status_string", "wall_attn_fwd_workspace_size", "wall_attn_fwd",
     "wall_build_kv_cache", "wall_attn_decode_workspace_size", "wall_attn_decode",
-    "wall_device_error", "wall_debug_set_fault",
+    "wall_device_error", "wall_debug_set_fault", "wall_debug_set_stage_events",
 )
 
 
@@ -88,6 +90,8 @@ def load_library():
     lib.wall_device_error.restype = I
     lib.wall_debug_set_fault.argtypes = [I, I]
     lib.wall_debug_set_fault.restype = None
+    lib.wall_debug_set_stage_events.argtypes = [P, P, P]
+    lib.wall_debug_set_stage_events.restype = None
     _lib = lib
     return lib
 
@@ -216,6 +220,12 @@ def wall_attn_decode(q, p_curr, v, k_tilde, r_cache, T_kv, sink_bias=None, scale
 def wall_device_error(device=None) -> int:
     """Synchronise the current stream and return (and clear) the device error status."""
     return int(load_library().wall_device_error(_stream(device)))
+
+
+def wall_debug_set_stage_events(before=None, between=None, after=None):
+    """Profiling hook: torch.cuda.Event objects recorded at kernel boundaries (None clears)."""
+    h = [ctypes.c_void_p(e.cuda_event) if e is not None else None for e in (before, between, after)]
+    load_library().wall_debug_set_stage_events(*h)
 
 
 def wall_debug_set_fault(mode: int, wait_ms: int = 0):

@@ -19,6 +19,13 @@ __device__ int g_wall_err;  // per-device error word (bit 0: a bounded wait gave
 
 std::atomic<int> g_fault_mode{0};
 std::atomic<int> g_wait_ms{2000};
+std::atomic<void*> g_stage_ev[3] = {};
+
+// Records the caller's profiling event `i` (if any) on `st`.
+void stage_event(int i, cudaStream_t st) {
+  void* e = g_stage_ev[i].load();
+  if (e != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(e), st);
+}
 
 bool debug_sync() {
   static const bool on = [] {
@@ -134,9 +141,15 @@ wall_status_t wall_attn_fwd(const void* q, const void* k, const void* v, const v
   wall::FwdWork w;
   wall::fwd_workspace_layout(B, T, HQ, K, bf16, &w, static_cast<char*>(workspace));
 
+  stage_event(0, st);
   cudaError_t e = wall::launch_prep(a, w, bf16, st);
   if (e != cudaSuccess) return WALL_ERR_CUDA;
-  if (!bf16) return finish(wall::launch_fwd_simt(a, w, st), st);
+  stage_event(1, st);
+  if (!bf16) {
+    e = wall::launch_fwd_simt(a, w, st);
+    stage_event(2, st);
+    return finish(e, st);
+  }
 
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return WALL_ERR_CUDA;
@@ -170,7 +183,9 @@ wall_status_t wall_attn_fwd(const void* q, const void* k, const void* v, const v
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return WALL_ERR_CUDA;
   }
-  return finish(wall::launch_fwd_tc(a, w, tmQ, tmK, tmV, st), st);
+  e = wall::launch_fwd_tc(a, w, tmQ, tmK, tmV, st);
+  stage_event(2, st);
+  return finish(e, st);
 }
 
 wall_status_t wall_build_kv_cache(const void* k_new, const void* g_new, const float* p_prev,
@@ -228,8 +243,12 @@ wall_status_t wall_attn_decode(const void* q, const float* p_curr, const void* v
   a.sink = sink_bias; a.B = B; a.T_kv = T_kv; a.cap = cap; a.HQ = HQ; a.H = H; a.K = K;
   a.V = V; a.chunk = chunk; a.scale = scale; a.o = o; a.lse = lse;
   a.part = static_cast<float*>(workspace); a.nsplit = ns;
+  a.mid_event = g_stage_ev[1].load();
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return finish(wall::launch_decode(a, dt == WALL_DTYPE_BF16, st), st);
+  stage_event(0, st);
+  const cudaError_t e = wall::launch_decode(a, dt == WALL_DTYPE_BF16, st);
+  stage_event(2, st);
+  return finish(e, st);
 }
 
 wall_status_t wall_device_error(wall_stream_t stream) {
@@ -243,6 +262,12 @@ wall_status_t wall_device_error(wall_stream_t stream) {
     return WALL_ERR_DEVICE_TIMEOUT;
   }
   return WALL_OK;
+}
+
+void wall_debug_set_stage_events(void* before, void* between, void* after) {
+  g_stage_ev[0].store(before);
+  g_stage_ev[1].store(between);
+  g_stage_ev[2].store(after);
 }
 
 void wall_debug_set_fault(int mode, int wait_ms) {

@@ -361,6 +361,7 @@ cudaError_t decode_impl(const DecodeArgs& a, cudaStream_t st) {
       a.nsplit, a.scale * kLog2e, a.part);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (a.mid_event != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(a.mid_event), st);
   const int nbh = a.B * a.HQ;
   decode_combine_kernel<T, VD><<<(nbh + 3) / 4, 128, 0, st>>>(a.part, a.nsplit, nbh, a.HQ, a.sink,
                                                              static_cast<T*>(a.o), a.lse);

@@ -82,6 +82,7 @@ struct DecodeArgs {
   float* lse;
   float* part;  // workspace
   int nsplit;
+  void* mid_event;  // optional cudaEvent_t recorded between the split and combine kernels
 };
 int decode_max_splits(int B, int T_kv, int HQ, int H, int chunk);
 int decode_num_splits(int B, int T_kv, int HQ, int H, int chunk);

@@ -167,6 +167,17 @@ wall_status_t wall_device_error(wall_stream_t stream);
  */
 void wall_debug_set_fault(int mode, int wait_ms);
 
+/*
+ * Profiling hook (not for production use): while set, every wall_attn_fwd
+ * records the caller's CUDA events (cudaEvent_t, NULL = skip) on its stream
+ * before the prepass (`before`), between the prepass and the main attention
+ * kernel (`between`) and after the main kernel (`after`); every
+ * wall_attn_decode records them before the split kernel, between the split and
+ * the combine kernel, and after the combine.  Lets a caller time each kernel
+ * with events on the launching stream.  Process-global; not thread-safe.
+ */
+void wall_debug_set_stage_events(void* before, void* between, void* after);
+
 #ifdef __cplusplus
 }
 #endif
