@@ -177,12 +177,19 @@ def dist_setup():
 
 
 def reduce_max(x, world, device):
-    """Max over ranks of a host float (timing only; no data-path collective)."""
+    """Max over ranks of a host float (timing only; no data-path collective).
+
+    `device` is the rank's CUDA device under NCCL, or "cpu" under gloo."""
     if world == 1:
         return x
     t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_rate(units_per_rank, steps, world, max_ms):
+    """Whole-job rate: the units every rank processed over the slowest rank's time (per s)."""
+    return world * units_per_rank * steps / (max_ms * 1e-3)
 
 
 def barrier(world):
@@ -415,7 +422,7 @@ def run_ours(args, world, rank, local):
         pre_main_ms = [e[1].elapsed_time(e[2]) for e in pre_ev]
         flops = prefill_flops(pspec)
         pre_total_ms = reduce_max(sum(pre_ms), world, dev)
-        value = world * flops * args.steps / (pre_total_ms * 1e-3) / 1e12
+        value = weak_scaling_rate(flops, args.steps, world, pre_total_ms) / 1e12
         main_avg = statistics.mean(pre_main_ms)
         achieved = flops / (main_avg * 1e-3) / 1e12
         line["value"] = value
@@ -434,7 +441,7 @@ def run_ours(args, world, rank, local):
         dec_split_ms = [[e[0].elapsed_time(e[1]) for e in row] for row in dec_ev]
         step_bytes = [decode_bytes(dspec, T0 + s + 1) for s in range(S)]
         dec_total_ms = reduce_max(sum(sum(r) for r in dec_ms), world, dev)
-        dec_value = world * args.steps * sum(step_bytes) / (dec_total_ms * 1e-3) / 1e9
+        dec_value = weak_scaling_rate(sum(step_bytes), args.steps, world, dec_total_ms) / 1e9
         split_avg = statistics.mean(x for r in dec_split_ms for x in r)
         dec_achieved = statistics.mean(step_bytes) / (split_avg * 1e-3) / 1e9
         line["decode"] = {
@@ -482,7 +489,7 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
         barrier(world)
         e2e_ms = reduce_max(a.elapsed_time(b_), world, dev)
-        line["e2e"] = {"value": world * prefill_flops(pspec) * args.steps / (e2e_ms * 1e-3) / 1e12,
+        line["e2e"] = {"value": weak_scaling_rate(prefill_flops(pspec), args.steps, world, e2e_ms) / 1e12,
                        "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     line["gpu_launches"] = args.steps * ((3 if do_prefill else 0) + 3 * S)
     line["clocks"] = clk
