@@ -26,6 +26,7 @@ import torch
 __all__ = [
     "WallError", "lib_path", "load_library", "wall_attn_fwd", "wall_attn_fwd_workspace_size",
     "wall_build_kv_cache", "wall_attn_decode", "wall_attn_decode_workspace_size",
+    "wall_attn_decode_noalloc",
     "wall_device_error", "wall_debug_set_fault", "wall_debug_set_stage_events", "KVCache",
     "EXPORTED_SYMBOLS",
 ]
@@ -45,6 +46,7 @@ EXPORTED_SYMBOLS = (
     "wall_status_string", "wall_attn_fwd_workspace_size", "wall_attn_fwd",
     "wall_build_kv_cache", "wall_attn_decode_workspace_size", "wall_attn_decode",
     "wall_device_error", "wall_debug_set_fault", "wall_debug_set_stage_events",
+    "wall_attn_decode_noalloc",
 )
 
 
@@ -86,6 +88,8 @@ def load_library():
     lib.wall_attn_decode_workspace_size.restype = S
     lib.wall_attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, P, P, P, S, P]
     lib.wall_attn_decode.restype = I
+    lib.wall_attn_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, P, P, P]
+    lib.wall_attn_decode_noalloc.restype = I
     lib.wall_device_error.argtypes = [P]
     lib.wall_device_error.restype = I
     lib.wall_debug_set_fault.argtypes = [I, I]
@@ -214,6 +218,25 @@ def wall_attn_decode(q, p_curr, v, k_tilde, r_cache, T_kv, sink_bias=None, scale
         _dev(out, "out", dt), _dev(lse, "lse", torch.float32), _dev(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(q.device))
     _check(st, "wall_attn_decode")
+    return out
+
+
+def wall_attn_decode_noalloc(q, p_curr, v, k_tilde, r_cache, T_kv, out, lse=None,
+                             sink_bias=None, scale=None, chunk=64):
+    """wall_attn_decode without a workspace: the split partials live in a fixed
+    4 MiB device array inside the library (for callers that cannot allocate at
+    decode time).  `out` (and `lse`) must be allocated by the caller."""
+    lib = load_library()
+    B, cap, HQ, K = k_tilde.shape
+    H, V = v.shape[2], v.shape[3]
+    dt = k_tilde.dtype
+    st = lib.wall_attn_decode_noalloc(
+        _dev(q, "q", dt), _dev(p_curr, "p_curr", torch.float32), _dev(v, "v", dt, (B, cap, H, V)),
+        _dev(k_tilde, "k_tilde", dt), _dev(r_cache, "r_cache", torch.float32),
+        _dev(sink_bias, "sink_bias", torch.float32, (HQ,)), B, int(T_kv), cap, HQ, H, K, V,
+        int(chunk), _dtype_code(k_tilde), float(scale) if scale else 0.0,
+        _dev(out, "out", dt, (B, 1, HQ, V)), _dev(lse, "lse", torch.float32), _stream(q.device))
+    _check(st, "wall_attn_decode_noalloc")
     return out
 
 

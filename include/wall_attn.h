@@ -150,6 +150,40 @@ wall_status_t wall_attn_decode(const void* q, const float* p_curr, const void* v
                                size_t workspace_bytes, wall_stream_t stream);
 
 /*
+ * Decode without scratch allocation (no counterpart in the paper: this entry
+ * point exists for callers of this library, not for the method).
+ *
+ * Same arguments and result as wall_attn_decode, minus the workspace.  Some
+ * callers cannot allocate device memory at decode time: an inference server or
+ * host application that owns every byte of device memory through its own
+ * planner or pool and forbids outside allocations, a token loop that must not
+ * stall on an allocator (cudaMalloc can synchronise the device), or plain C
+ * code that is handed tensor pointers and no allocator at all.  This call
+ * keeps the split partials in a fixed 4 MiB array in the library's own device
+ * memory (one per GPU that loads the library, held until the process exits)
+ * and calls no cudaMalloc, cudaFree or allocating library routine.
+ *
+ *   - Limit: one (V + 2)-float partial per (batch row, query head, split) must
+ *     fit in 4 MiB.  The split count is lowered as needed (results stay within
+ *     the usual tolerance); if even one split per (batch row, query head) does
+ *     not fit (B * HQ * (V + 2) * 4 bytes > 4 MiB, e.g. B * HQ > 8065 at
+ *     V = 128) the call returns WALL_ERR_WORKSPACE before queuing any work.
+ *   - The array is shared by every call on the device and keeps the last
+ *     call's contents; nothing in it needs to start at zero (the split pass
+ *     writes every partial the combine pass reads).  Calls whose kernels
+ *     overlap on the GPU (different streams without ordering between them)
+ *     race on the array and give wrong results: order them on one stream.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture begins.
+ */
+wall_status_t wall_attn_decode_noalloc(const void* q, const float* p_curr, const void* v,
+                                       const void* k_tilde, const float* r_cache,
+                                       const float* sink_bias, int B, int T_kv, int cap, int HQ,
+                                       int H, int K, int V, int chunk, wall_dtype_t dt,
+                                       float scale, void* o, float* lse, wall_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears this device's error word.
  * Returns WALL_ERR_DEVICE_TIMEOUT if any kernel since the last read gave up a
  * bounded wait (its outputs are then unspecified), WALL_ERR_CUDA if the

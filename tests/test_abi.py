@@ -132,6 +132,24 @@ def test_decode_host_validation(lib):
     assert _dec(lib, wsb=8) == WORKSPACE
 
 
+def test_noalloc_decode_host_validation(lib):
+    def call(**kw):
+        a = dict(q=_fake(), pc=_fake(), v=_fake(), kt=_fake(), r=_fake(), sink=None, B=2, Tkv=100,
+                 cap=128, HQ=8, H=2, K=128, V=128, C=64, dt=BF16, scale=0.0, o=_fake(), lse=None,
+                 stream=None)
+        a.update(kw)
+        return lib.wall_attn_decode_noalloc(a["q"], a["pc"], a["v"], a["kt"], a["r"], a["sink"],
+                                            a["B"], a["Tkv"], a["cap"], a["HQ"], a["H"], a["K"],
+                                            a["V"], a["C"], a["dt"], a["scale"], a["o"], a["lse"],
+                                            a["stream"])
+    assert call(Tkv=0) == INVALID
+    assert call(o=None) == INVALID
+    assert call(K=96) == UNSUPPORTED
+    # one split per (batch row, query head) no longer fits the fixed 4 MiB scratch
+    assert call(B=512, HQ=16, H=4, Tkv=64, cap=64) == WORKSPACE
+    assert call(B=0) == 0
+
+
 def test_decode_workspace_monotone_in_length(lib):
     prev = 0
     for T in (1, 63, 64, 65, 640, 6400, 32768, 32832):
