@@ -41,7 +41,8 @@ __global__ void __launch_bounds__(256) wall_fwd_simt_kernel(
   const int b = bh / HQ, hq = bh % HQ, kvh = hq / (HQ / H);
   const int q0 = qb * SB;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  const int ablk = q0 / kBlockRows;  // anchor block of the queries
+  const int ablk = 2 * (q0 / (2 * kBlockRows));  // query anchor (256-row blocks)
+  const int rblk = q0 / kBlockRows;                // 128-row block of these rows
 
   if (tid == 0) s_lo = 0x7fffffff;
   // anchored q block, transposed
@@ -65,7 +66,7 @@ __global__ void __launch_bounds__(256) wall_fwd_simt_kernel(
     }
     hi[a] = ok ? i : -1;
     rowA[a] = 0.f;
-    if (HAS_GS) rowA[a] = ssa[(static_cast<size_t>(bh) * NB + ablk) * 4] +
+    if (HAS_GS) rowA[a] = ssa[(static_cast<size_t>(bh) * NB + rblk) * 4] -
                           ssl[static_cast<size_t>(bh) * NB * kBlockRows + min(i, NB * kBlockRows - 1)];
   }
   __syncthreads();
@@ -88,7 +89,7 @@ __global__ void __launch_bounds__(256) wall_fwd_simt_kernel(
       sCv[tid] = exp2f((AQ[(static_cast<size_t>(bh) * NB + ablk) * KD + tid] -
                         AK[(static_cast<size_t>(bh) * NB + kblk) * KD + tid]) * kLog2e);
     if (HAS_GS && tid < SB)
-      sCol[tid] = ssa[(static_cast<size_t>(bh) * NB + kblk) * 4] +
+      sCol[tid] = ssa[(static_cast<size_t>(bh) * NB + kblk) * 4] -
                   ssl[static_cast<size_t>(bh) * NB * kBlockRows + j0 + tid];
     __syncthreads();
     for (int e = tid; e < SB * KD; e += 256) {

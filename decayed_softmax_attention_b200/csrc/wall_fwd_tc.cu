@@ -1,25 +1,33 @@
 // Wall attention prefill forward, bf16, on the 5th-generation tensor cores
 // (tcgen05 + TMEM) of sm_100a.
 //
-// One CTA computes a 128-row query block of one (batch, query head).  The
-// score of the Wall Attention README intro,
+// One CTA computes a 256-row query block (two 128-row tiles, A and B) of one
+// (batch, query head).  The score of the Wall Attention README intro,
 //   x(i,j) = scale * sum_n q[i,n] k[j,n] exp(G[i,n] - G[j,n]) + Gs[i] - Gs[j],
 // becomes a dense contraction per (query block, key tile) pair:
 //   S = Qh * diag(c) * Kh^T,  c[n] = exp(AQ[n] - AK[n])
-// where Qh/Kh are the anchored operands written by the prepass.  The rescale
-// warpgroup multiplies each key tile by c in shared memory (in place), the MMA
-// warp issues S = Qh * Kt^T into TMEM, the softmax warpgroup (one query row
-// per thread, read straight from its TMEM lane) runs the online softmax in the
-// exp2 domain and writes P (bf16) back into TMEM over S, and the MMA warp
-// accumulates O += P * V with P taken from TMEM.  This is the streaming
-// (FlashAttention-style) softmax the README names; the decay factor never
-// leaves the tile.
+// where Qh/Kh are the anchored operands of the prepass (query anchor per
+// 256-row block, key anchor per 128-row block), so one rescaled key tile
+// serves both query tiles.  The rescale warpgroup multiplies each key tile by
+// c in shared memory (in place), the MMA warp issues S_X = Qh_X * Kt^T into
+// TMEM, each softmax warpgroup (one query row per thread, read straight from
+// its TMEM lane) runs the online softmax in the exp2 domain and writes P
+// (bf16) back into TMEM over S_X, and the MMA warp accumulates O_X += P_X * V
+// with P taken from TMEM.  This is the streaming (FlashAttention-style)
+// softmax the README names; the decay factor never leaves the tile.
 //
-// Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2
-// TMEM allocator, warps 4-7 softmax + epilogue, warps 8-11 key rescale.
-// Key tiles are visited from the diagonal backwards so the running maximum is
-// found early; O is rescaled only when a row maximum grows by more than 2^8
-// (exact: the final normalisation uses the same stale maximum).
+// Warp roles (512 threads): warpgroup 0 = warp 0 TMA producer, warp 1 MMA
+// issuer, warp 2 TMEM allocator; warpgroups 1 and 2 = softmax + epilogue of
+// query tiles A and B; warpgroup 3 = key-tile rescale.  Registers are
+// re-balanced at start (setmaxnreg): the softmax warpgroups get 184.
+//
+// MMA issue order per key tile j: PV_A(j-1), QK_A(j), PV_B(j-1), QK_B(j), so
+// one softmax warpgroup works while the tensor core serves the other, and
+// "S_X(j) complete" implies "PV_X(j-1) complete" (tcgen05 ops of one thread
+// run in issue order): a softmax warpgroup may rescale O_X as soon as it has
+// read S_X(j).  Key tiles are visited from the diagonal backwards so the row
+// maximum is found early; O is rescaled only when a row maximum grows by more
+// than 2^8 (exact: the final normalisation uses the same stale maximum).
 #include "wall_common.cuh"
 #include "wall_internal.h"
 
@@ -45,14 +53,14 @@ struct TcParams {
 
 template <int KD, int VD>
 struct TcCfg {
-  static constexpr int BM = 128, BN = 128;
-  static constexpr int KS = 3, VS = 2;
+  static constexpr int BM = 128, BN = 128, NQ = 2;
+  static constexpr int KS = 2, VS = 2;
   static constexpr int QBOX = KD / 64, VBOX = VD / 64;
   static constexpr int Q_BYTES = BM * KD * 2;
   static constexpr int K_BYTES = BN * KD * 2;
   static constexpr int V_BYTES = BN * VD * 2;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_K = OFF_Q + NQ * Q_BYTES;
   static constexpr int OFF_V = OFF_K + KS * K_BYTES;
   static constexpr int OFF_AQ = OFF_V + VS * V_BYTES;
   static constexpr int OFF_AK = OFF_AQ + KD * 4;
@@ -61,16 +69,15 @@ struct TcCfg {
   static constexpr int OFF_C = OFF_COLA + VS * 16;
   static constexpr int OFF_BAR = OFF_C + 2 * KD * 4;
   // qfull, kfull[KS], kready[KS], kempty[KS], vfull[VS], vempty[VS], sfull[2], pfull[2],
-  // odone, ofinal, mdrain
-  static constexpr int NBAR = 1 + 3 * KS + 2 * VS + 2 + 2 + 3;
+  // ofinal, mdrain
+  static constexpr int NBAR = 1 + 3 * KS + 2 * VS + 2 + 2 + 2;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_USED = OFF_MISC + 64;
   // At least 116 KB so that a second CTA never shares the SM (each CTA takes
   // all 512 TMEM columns).
-  static constexpr int SMEM_ALLOC =
-      (SMEM_USED + 1024) > 118784 ? (SMEM_USED + 1024) : 118784;
+  static constexpr int SMEM_ALLOC = (SMEM_USED + 1024) > 118784 ? (SMEM_USED + 1024) : 118784;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_S0 = 0, COL_O = 256;
+  static constexpr uint32_t COL_S = 0, COL_O = 256;  // + 128 * tile
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, VD, 0, 1);
 };
@@ -78,10 +85,14 @@ struct TcCfg {
 // Pack the 8 bf16 of one 16-byte chunk, scaled by c[0..7].
 __device__ __forceinline__ uint4 scale_chunk(uint4 u, const float* c) {
   uint4 r;
-  r.x = pack_bf16(bf16_lo(u.x) * c[0], bf16_hi(u.x) * c[1]);
-  r.y = pack_bf16(bf16_lo(u.y) * c[2], bf16_hi(u.y) * c[3]);
-  r.z = pack_bf16(bf16_lo(u.z) * c[4], bf16_hi(u.z) * c[5]);
-  r.w = pack_bf16(bf16_lo(u.w) * c[6], bf16_hi(u.w) * c[7]);
+  const float2 a = fmul2(make_float2(bf16_lo(u.x), bf16_hi(u.x)), make_float2(c[0], c[1]));
+  const float2 b = fmul2(make_float2(bf16_lo(u.y), bf16_hi(u.y)), make_float2(c[2], c[3]));
+  const float2 d = fmul2(make_float2(bf16_lo(u.z), bf16_hi(u.z)), make_float2(c[4], c[5]));
+  const float2 e = fmul2(make_float2(bf16_lo(u.w), bf16_hi(u.w)), make_float2(c[6], c[7]));
+  r.x = pack_bf16(a.x, a.y);
+  r.y = pack_bf16(b.x, b.y);
+  r.z = pack_bf16(d.x, d.y);
+  r.w = pack_bf16(e.x, e.y);
   return r;
 }
 
@@ -99,7 +110,7 @@ __device__ __forceinline__ bool bar_or(int id, int nthreads, bool pred) {
 }
 
 // Keeps the compiler from touching registers filled by tcgen05.ld before the
-// matching tcgen05.wait::ld (and from recycling tcgen05.st sources early).
+// matching tcgen05.wait::ld.
 __device__ __forceinline__ void reg_fence32(float* r) {
   asm volatile(""
                : "+f"(r[0]), "+f"(r[1]), "+f"(r[2]), "+f"(r[3]), "+f"(r[4]), "+f"(r[5]),
@@ -109,18 +120,8 @@ __device__ __forceinline__ void reg_fence32(float* r) {
                  "+f"(r[24]), "+f"(r[25]), "+f"(r[26]), "+f"(r[27]), "+f"(r[28]), "+f"(r[29]),
                  "+f"(r[30]), "+f"(r[31]));
 }
-__device__ __forceinline__ void reg_fence32u(uint32_t* r) {
-  asm volatile(""
-               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
-                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
-                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
-                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
-                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
-                 "+r"(r[30]), "+r"(r[31]));
-}
-
 template <int KD, int VD, bool HAS_GS>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     wall_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const TcParams p) {
@@ -145,19 +146,21 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* vempty = vfull + C::VS;
   uint64_t* sfull = vempty + C::VS;
   uint64_t* pfull = sfull + 2;
-  uint64_t* odone = pfull + 2;
-  uint64_t* ofinal = odone + 1;
+  uint64_t* ofinal = pfull + 2;
   uint64_t* mdrain = ofinal + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
-  int* sched_lo = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
+  int* sched_lo = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);  // [2]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wg = warp >> 2;
   const int BHQ = p.B * p.HQ;
-  const int qb = p.NB - 1 - static_cast<int>(blockIdx.x / BHQ);
+  const int NQB = (p.NB + 1) / 2;
+  const int qblk = NQB - 1 - static_cast<int>(blockIdx.x / BHQ);
   const int bh = static_cast<int>(blockIdx.x % BHQ);
   const int b = bh / p.HQ, hq = bh % p.HQ, kvh = hq / (p.HQ / p.H);
-  const int q0 = qb * C::BM;
+  const int q0 = qblk * 2 * C::BM;
+  const bool has_b = q0 + C::BM < p.T;
 
   if (tid == 0) {
     mbar_init(qfull, 1);
@@ -170,15 +173,15 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&vfull[s], 1);
       mbar_init(&vempty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&sfull[s], 1);
-      mbar_init(&pfull[s], 128);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&sfull[x], 1);
+      mbar_init(&pfull[x], 128);
     }
-    mbar_init(odone, 1);
     mbar_init(ofinal, 1);
     mbar_init(mdrain, 1);
     *abort_flag = 0;
-    *sched_lo = 0x7fffffff;
+    sched_lo[0] = 0x7fffffff;
+    sched_lo[1] = 0x7fffffff;
     fence_mbar_init();
   }
   if (warp == 2) {
@@ -189,54 +192,63 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
 
   // Admitted key range per query row: [lo_i, i] (causal, window, document).
-  int my_lo = 0;
-  const bool is_softmax = (warp >= 4 && warp < 8);
-  const int row = tid - 128;
-  const int gi = q0 + row;
+  const bool is_softmax = (wg == 1 || wg == 2);
+  const int X = wg - 1;  // query tile of a softmax warpgroup
+  const int row = tid - 128 * wg;
+  const int gi = q0 + C::BM * X + row;
   const bool row_ok = is_softmax && gi < p.T;
+  int my_lo = 0;
   if (row_ok) {
     if (p.rowlo != nullptr) {
       my_lo = p.rowlo[gi];
     } else if (p.window > 0) {
       my_lo = gi - p.window + 1 > 0 ? gi - p.window + 1 : 0;
     }
-    atomicMin(sched_lo, my_lo);
+    atomicMin(&sched_lo[X], my_lo);
   }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int lo_all = *sched_lo;
-  const int kt_hi = qb;
-  const int kt_lo = lo_all == 0x7fffffff ? kt_hi : (lo_all / C::BN);
-  const int nt = kt_hi - kt_lo + 1;
+  // key-tile ranges (tile index kt = key row / 128) of query tiles A and B
+  const int ktA_hi = 2 * qblk, ktB_hi = 2 * qblk + 1;
+  const int ktA_lo = sched_lo[0] / C::BN;
+  const int ktB_lo = has_b ? sched_lo[1] / C::BN : ktB_hi + 1;
+  const int kt_hi = has_b ? ktB_hi : ktA_hi;
+  const int kt_lo = has_b ? min(ktA_lo, ktB_lo) : ktA_lo;
+  const int nt = kt_hi - kt_lo + 1;  // visit order j = 0..nt-1 is kt = kt_hi - j
+  // visit indices of the first/last key tile of each query tile (B may have none)
+  const int jfA = kt_hi - ktA_hi, jlA = kt_hi - ktA_lo;
+  const int jfB = has_b ? kt_hi - ktB_hi : 0, jlB = has_b ? kt_hi - ktB_lo : -1;
   const WaitCtl wc{abort_flag, p.err, p.wait_ns};
 
-  if (warp == 0) {
-    // ------------------------------------------------------------- TMA producer
-    if (lane == 0) {
+  if (wg == 0) {
+    reg_dealloc<56>();
+    if (warp == 0 && lane == 0) {
+      // ----------------------------------------------------------- TMA producer
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      int last_k[C::KS], last_v[C::VS];
-      for (int s = 0; s < C::KS; ++s) last_k[s] = -1;
-      for (int s = 0; s < C::VS; ++s) last_v[s] = -1;
-      mbar_arrive_expect_tx(qfull, C::Q_BYTES + KD * 4);
-      for (int bx = 0; bx < C::QBOX; ++bx) tma_load_3d(sQ + bx * 16384, &tmQ, qfull, bx * 64, q0, bh);
-      bulk_load(sAQ, p.AQ + (static_cast<size_t>(bh) * p.NB + qb) * KD, KD * 4, qfull);
-      for (int n = 0; n < nt; ++n) {
-        const int kt = kt_hi - n;
-        const int ks = n % C::KS;
-        if (n >= C::KS && !mbar_wait(&kempty[ks], ((n / C::KS) - 1) & 1, wc)) break;
-        if (!(p.fault == 1 && n == 0)) {
+      int nk = 0, nv = 0;  // key / value tiles whose copies were issued
+      mbar_arrive_expect_tx(qfull, (has_b ? 2 : 1) * C::Q_BYTES + KD * 4);
+      for (int bx = 0; bx < C::QBOX; ++bx) {
+        tma_load_3d(sQ + bx * 16384, &tmQ, qfull, bx * 64, q0, bh);
+        if (has_b) tma_load_3d(sQ + C::Q_BYTES + bx * 16384, &tmQ, qfull, bx * 64, q0 + C::BM, bh);
+      }
+      bulk_load(sAQ, p.AQ + (static_cast<size_t>(bh) * p.NB + 2 * qblk) * KD, KD * 4, qfull);
+      for (int j = 0; j < nt; ++j) {
+        const int kt = kt_hi - j;
+        const int ks = j % C::KS;
+        if (j >= C::KS && !mbar_wait(&kempty[ks], ((j / C::KS) - 1) & 1, wc)) break;
+        if (!(p.fault == 1 && j == 0)) {
           mbar_arrive_expect_tx(&kfull[ks], C::K_BYTES + KD * 4);
           for (int bx = 0; bx < C::QBOX; ++bx)
             tma_load_3d(sK + ks * C::K_BYTES + bx * 16384, &tmK, &kfull[ks], bx * 64, kt * C::BN, bh);
           bulk_load(sAK + ks * KD, p.AK + (static_cast<size_t>(bh) * p.NB + kt) * KD, KD * 4,
                     &kfull[ks]);
-          last_k[ks] = n;
         }
-        const int vs = n % C::VS;
-        if (n >= C::VS && !mbar_wait(&vempty[vs], ((n / C::VS) - 1) & 1, wc)) break;
+        nk = j + 1;
+        const int vs = j % C::VS;
+        if (j >= C::VS && !mbar_wait(&vempty[vs], ((j / C::VS) - 1) & 1, wc)) break;
         mbar_arrive_expect_tx(&vfull[vs], C::V_BYTES + (HAS_GS ? C::BN * 4 + 16 : 0));
         for (int bx = 0; bx < C::VBOX; ++bx)
           tma_load_4d(sV + vs * C::V_BYTES + bx * 16384, &tmV, &vfull[vs], bx * 64, kvh,
@@ -248,76 +260,102 @@ __global__ void __launch_bounds__(384, 1)
           bulk_load(sColA + vs * 4, p.ssa + (static_cast<size_t>(bh) * p.NB + kt) * 4, 16,
                     &vfull[vs]);
         }
-        last_v[vs] = n;
+        nv = j + 1;
       }
-      // Every copy issued must land before the CTA may exit.
+      // Every copy issued must land before the CTA may exit: the last KS (VS)
+      // tiles issued are the only ones a consumer may not have waited for.
       mbar_drain(qfull, 0, p.wait_ns);
-      for (int s = 0; s < C::KS; ++s)
-        if (last_k[s] >= 0) mbar_drain(&kfull[s], (last_k[s] / C::KS) & 1, p.wait_ns);
-      for (int s = 0; s < C::VS; ++s)
-        if (last_v[s] >= 0) mbar_drain(&vfull[s], (last_v[s] / C::VS) & 1, p.wait_ns);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+      for (int j = nk > C::KS ? nk - C::KS : 0; j < nk; ++j)
+        if (!(p.fault == 1 && j == 0)) mbar_drain(&kfull[j % C::KS], (j / C::KS) & 1, p.wait_ns);
+      for (int j = nv > C::VS ? nv - C::VS : 0; j < nv; ++j)
+        mbar_drain(&vfull[j % C::VS], (j / C::VS) & 1, p.wait_ns);
+    } else if (warp == 1 && lane == 0) {
+      // ----------------------------------------------------------- MMA issuer
       bool ok = mbar_wait(qfull, 0, wc);
       tc_fence_after();
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-      auto issue_pv = [&](int m) -> bool {
-        const int pb = m & 1, vs = m % C::VS;
-        if (!mbar_wait(&pfull[pb], (m >> 1) & 1, wc)) return false;
-        if (!mbar_wait(&vfull[vs], (m / C::VS) & 1, wc)) return false;
+      // Only the previous key tile's P*V products can be pending at tile j.
+      bool pendA = false, pendB = false;
+      int vrem_prev = 0;  // P*V reads still to issue for the previous tile's V stage
+      auto issue_pv = [&](int x, int jj) -> bool {
+        const int cnt = jj - (x == 0 ? jfA : jfB), vs = jj % C::VS;
+        if (!mbar_wait(&pfull[x], cnt & 1, wc)) return false;
+        if (!mbar_wait(&vfull[vs], (jj / C::VS) & 1, wc)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
           const uint64_t bdesc = sw128_desc(sVa + vs * C::V_BYTES + kk * 2048, 16384, 1024);
-          umma_ts(tmem_base + C::COL_O, tmem_base + C::COL_S0 + pb * 128 + kk * 8, bdesc,
-                  C::IDESC_PV, (m > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tmem_base + C::COL_O + 128 * x, tmem_base + C::COL_S + 128 * x + kk * 8, bdesc,
+                  C::IDESC_PV, (cnt > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&vempty[vs]);
-        umma_commit(odone);
+        if (--vrem_prev == 0) umma_commit(&vempty[vs]);
         return true;
       };
-      for (int n = 0; ok && n < nt; ++n) {
-        const int ks = n % C::KS;
-        if (!mbar_wait(&kready[ks], (n / C::KS) & 1, wc)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t dS = tmem_base + C::COL_S0 + (n & 1) * 128;
+      auto issue_qk = [&](int x, int j, int ks) {
+        const uint32_t dS = tmem_base + C::COL_S + 128 * x;
 #pragma unroll
         for (int kk = 0; kk < KD / 16; ++kk) {
           const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint64_t adesc = sw128_desc(sQa + koff, 16, 1024);
+          const uint64_t adesc = sw128_desc(sQa + x * C::Q_BYTES + koff, 16, 1024);
           const uint64_t bdesc = sw128_desc(sKa + ks * C::K_BYTES + koff, 16, 1024);
           umma_ss(dS, adesc, bdesc, C::IDESC_QK, kk > 0 ? 1u : 0u);
         }
+        umma_commit(&sfull[x]);
+      };
+      for (int j = 0; ok && j < nt; ++j) {
+        const int ks = j % C::KS;
+        int vrem_cur = 0;
+        if (pendA) {
+          if (!issue_pv(0, j - 1)) { ok = false; break; }
+          pendA = false;
+        }
+        if (!mbar_wait(&kready[ks], (j / C::KS) & 1, wc)) { ok = false; break; }
+        tc_fence_after();
+        if (j >= jfA && j <= jlA) {
+          issue_qk(0, j, ks);
+          pendA = true;
+          ++vrem_cur;
+        }
+        if (pendB) {
+          if (!issue_pv(1, j - 1)) { ok = false; break; }
+          pendB = false;
+        }
+        if (j >= jfB && j <= jlB) {
+          issue_qk(1, j, ks);
+          pendB = true;
+          ++vrem_cur;
+        }
         umma_commit(&kempty[ks]);
-        umma_commit(&sfull[n & 1]);
-        if (n > 0 && !issue_pv(n - 1)) ok = false;
+        if (vrem_cur == 0) umma_commit(&vempty[j % C::VS]);  // no P*V reads this tile
+        vrem_prev = vrem_cur;
       }
-      if (ok && nt > 0) ok = issue_pv(nt - 1);
+      if (ok && pendA) ok = issue_pv(0, nt - 1);
+      if (ok && pendB) ok = issue_pv(1, nt - 1);
       if (ok) umma_commit(ofinal);
       umma_commit(mdrain);
       mbar_drain(mdrain, 0, p.wait_ns);
     }
   } else if (is_softmax) {
     // ------------------------------------------------------------- softmax + epilogue
+    reg_alloc<184>();
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t colS = C::COL_S + 128 * X, colO = C::COL_O + 128 * X;
     const int lo = row_ok ? my_lo : 0;
     const int hi = row_ok ? gi : 0x7fffffff;
     float rowA = 0.f;
-    if (HAS_GS) {
-      rowA = p.ssa[(static_cast<size_t>(bh) * p.NB + qb) * 4] +
+    if (HAS_GS && row_ok) {
+      rowA = p.ssa[(static_cast<size_t>(bh) * p.NB + gi / C::BM) * 4] -
              p.ssl[static_cast<size_t>(bh) * p.NB * C::BM + gi];
     }
+    const float2 sc2 = make_float2(p.sc, p.sc);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int n = 0; n < nt; ++n) {
-      const int kt = kt_hi - n, sb = n & 1, vs = n % C::VS;
-      bool got = mbar_wait(&sfull[sb], (n >> 1) & 1, wc);
-      if (HAS_GS && got) got = mbar_wait(&vfull[vs], (n / C::VS) & 1, wc);
+    const int jf = X == 0 ? jfA : jfB, jl = X == 0 ? jlA : jlB;
+    for (int j = jf; j <= jl; ++j) {
+      const int cnt = j - jf;
+      const int kt = kt_hi - j, vs = j % C::VS;
+      bool got = mbar_wait(&sfull[X], cnt & 1, wc);
+      if (HAS_GS && got) got = mbar_wait(&vfull[vs], (j / C::VS) & 1, wc);
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
@@ -325,7 +363,7 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       float s[C::BN];
 #pragma unroll
-      for (int c = 0; c < C::BN; c += 32) tmem_ld32(lane_base + C::COL_S0 + sb * 128 + c, s + c);
+      for (int c = 0; c < C::BN; c += 32) tmem_ld32(lane_base + colS + c, s + c);
       tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < C::BN; c += 32) reg_fence32(s + c);
@@ -333,28 +371,32 @@ __global__ void __launch_bounds__(384, 1)
       const int j0 = kt * C::BN;
       float w = 0.f;
       if (HAS_GS) {
+        // t = S * scale*log2e - (key-side gate prefix); the row side joins below
         const float* col = sCol + vs * C::BN;
         w = rowA - sColA[vs * 4];
 #pragma unroll
-        for (int j = 0; j < C::BN; j += 4) {
-          const float4 cv = *reinterpret_cast<const float4*>(col + j);
-          s[j] = fmaf(s[j], p.sc, -cv.x);
-          s[j + 1] = fmaf(s[j + 1], p.sc, -cv.y);
-          s[j + 2] = fmaf(s[j + 2], p.sc, -cv.z);
-          s[j + 3] = fmaf(s[j + 3], p.sc, -cv.w);
+        for (int jj = 0; jj < C::BN; jj += 4) {
+          const float4 cv = *reinterpret_cast<const float4*>(col + jj);
+          const float2 t0 = ffma2(make_float2(s[jj], s[jj + 1]), sc2, make_float2(cv.x, cv.y));
+          const float2 t1 = ffma2(make_float2(s[jj + 2], s[jj + 3]), sc2, make_float2(cv.z, cv.w));
+          s[jj] = t0.x; s[jj + 1] = t0.y; s[jj + 2] = t1.x; s[jj + 3] = t1.y;
         }
       }
       const bool partial = !__all_sync(0xffffffffu, lo <= j0 && hi >= j0 + C::BN - 1);
       if (partial) {
 #pragma unroll
-        for (int j = 0; j < C::BN; ++j) {
-          const int jg = j0 + j;
-          if (jg < lo || jg > hi) s[j] = -INFINITY;
+        for (int jj = 0; jj < C::BN; ++jj) {
+          const int jg = j0 + jj;
+          if (jg < lo || jg > hi) s[jj] = -INFINITY;
         }
       }
-      float mt = -INFINITY;
+      float mx0 = s[0], mx1 = s[1];
 #pragma unroll
-      for (int j = 0; j < C::BN; ++j) mt = fmaxf(mt, s[j]);
+      for (int jj = 2; jj < C::BN; jj += 4) {
+        mx0 = fmax3(mx0, s[jj], s[jj + 1]);
+        mx1 = fmax3(mx1, s[jj + 2], s[jj + 3]);
+      }
+      float mt = fmaxf(mx0, mx1);
       mt = HAS_GS ? mt + w : mt * p.sc;
       const bool need = mt > m_used + 8.f;
       float alpha = 1.f;
@@ -363,61 +405,53 @@ __global__ void __launch_bounds__(384, 1)
         l *= alpha;
         m_used = mt;
       }
-      if (n > 0 && __any_sync(0xffffffffu, need)) {
-        const bool g2 = mbar_wait(odone, (n - 1) & 1, wc);
-        if (!__all_sync(0xffffffffu, g2)) {
-          ok = false;
-          break;
+      const float base = (m_used == -INFINITY) ? 0.f : m_used;
+      const float2 off = HAS_GS ? make_float2(w - base, w - base) : make_float2(-base, -base);
+      float2 rs = make_float2(0.f, 0.f);
+      // P in 32-column chunks: each chunk's scores die once its 16 packed
+      // bf16x2 columns are stored over S (the chunk's own, already-read columns).
+#pragma unroll
+      for (int c = 0; c < C::BN; c += 32) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int jj = 0; jj < 32; jj += 2) {
+          const float2 sv = make_float2(s[c + jj], s[c + jj + 1]);
+          const float2 t = HAS_GS ? fadd2(sv, off) : ffma2(sv, sc2, off);
+          const float2 pv = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+          rs = fadd2(rs, pv);
+          pk[jj >> 1] = pack_bf16(pv.x, pv.y);
         }
-        tc_fence_after();
+        tmem_st16(lane_base + colS + (c >> 1), pk);
+      }
+      l += rs.x + rs.y;
+      if (cnt > 0 && __any_sync(0xffffffffu, need)) {
+        // PV_X(j-1) was issued before QK_X(j), so it is complete: rescale O_X now.
+        const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll 1
         for (int c = 0; c < VD; c += 32) {
           float ov[32];
-          tmem_ld32(lane_base + C::COL_O + c, ov);
+          tmem_ld32(lane_base + colO + c, ov);
           tmem_wait_ld();
           reg_fence32(ov);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-          tmem_st32(lane_base + C::COL_O + c, reinterpret_cast<uint32_t*>(ov));
-          tmem_wait_st();
-          reg_fence32(ov);
+          for (int e = 0; e < 32; e += 2) {
+            const float2 t = fmul2(make_float2(ov[e], ov[e + 1]), a2);
+            ov[e] = t.x;
+            ov[e + 1] = t.y;
+          }
+          tmem_st32(lane_base + colO + c, reinterpret_cast<uint32_t*>(ov));
         }
+        tmem_wait_st();
       }
-      const float base = (m_used == -INFINITY) ? 0.f : m_used;
-      uint32_t pk[C::BN / 2];
-      float rs = 0.f;
-      if (HAS_GS) {
-        const float off = w - base;
-#pragma unroll
-        for (int j = 0; j < C::BN; j += 2) {
-          const float p0 = ex2_approx(s[j] + off), p1 = ex2_approx(s[j + 1] + off);
-          rs += p0 + p1;
-          pk[j >> 1] = pack_bf16(p0, p1);
-        }
-      } else {
-        const float off = -base;
-#pragma unroll
-        for (int j = 0; j < C::BN; j += 2) {
-          const float p0 = ex2_approx(fmaf(s[j], p.sc, off));
-          const float p1 = ex2_approx(fmaf(s[j + 1], p.sc, off));
-          rs += p0 + p1;
-          pk[j >> 1] = pack_bf16(p0, p1);
-        }
-      }
-      l += rs;
-      tmem_st32(lane_base + C::COL_S0 + sb * 128, pk);
-      tmem_st32(lane_base + C::COL_S0 + sb * 128 + 32, pk + 32);
       tmem_wait_st();
-      reg_fence32u(pk);
-      reg_fence32u(pk + 32);
       tc_fence_before();
-      mbar_arrive(&pfull[sb]);
+      mbar_arrive(&pfull[X]);
     }
-    if (ok) {
+    if (ok && jl >= jf) {
       const bool got = mbar_wait(ofinal, 0, wc);
       ok = __all_sync(0xffffffffu, got);
     }
-    if (ok) {
+    if (ok && jl >= jf) {
       tc_fence_after();
       float Z = l;
       if (p.sink != nullptr && m_used != -INFINITY) Z += ex2_approx(p.sink[hq] * kLog2e - m_used);
@@ -427,7 +461,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll 1
       for (int c = 0; c < VD; c += 32) {
         float ov[32];
-        tmem_ld32(lane_base + C::COL_O + c, ov);
+        tmem_ld32(lane_base + colO + c, ov);
         tmem_wait_ld();
         reg_fence32(ov);
         if (row_ok) {
@@ -445,9 +479,10 @@ __global__ void __launch_bounds__(384, 1)
       if (row_ok && p.lse != nullptr)
         p.lse[(static_cast<size_t>(b) * p.T + gi) * p.HQ + hq] = (m_used + log2f(Z)) * kLn2;
     }
-  } else if (warp >= 8) {
+  } else {
     // ------------------------------------------------------------- key-tile rescale
-    const int r = tid - 256;
+    reg_dealloc<80>();
+    const int r = tid - 384;
     bool ok = mbar_wait(qfull, 0, wc);
     ok = !bar_or(1, 128, !ok);
     constexpr int CPR = KD / 8;        // 16-byte chunks per key row
@@ -455,10 +490,10 @@ __global__ void __launch_bounds__(384, 1)
     const int L = r % CPR, box = L >> 3, c16 = L & 7;
     const int row0 = r / CPR;
     const uint32_t phys = static_cast<uint32_t>((c16 ^ (row0 & 7)) << 4);
-    for (int n = 0; ok && n < nt; ++n) {
-      const int ks = n % C::KS;
-      const bool got = mbar_wait(&kfull[ks], (n / C::KS) & 1, wc);
-      float* cb = sC + (n & 1) * KD;
+    for (int j = 0; ok && j < nt; ++j) {
+      const int ks = j % C::KS;
+      const bool got = mbar_wait(&kfull[ks], (j / C::KS) & 1, wc);
+      float* cb = sC + (j & 1) * KD;
       if (got && r < KD) cb[r] = ex2_approx((sAQ[r] - sAK[ks * KD + r]) * kLog2e);
       if (bar_or(1, 128, !got || *abort_flag != 0)) break;
       float cv[8];
@@ -511,8 +546,8 @@ cudaError_t tc_impl(const FwdArgs& a, const FwdWork& w, const CUtensorMap& tmQ,
   p.err = a.err;
   p.wait_ns = a.wait_ns;
   p.fault = a.fault;
-  const unsigned grid = static_cast<unsigned>(a.NB) * a.B * a.HQ;
-  kern<<<grid, 384, C::SMEM_ALLOC, st>>>(tmQ, tmK, tmV, p);
+  const unsigned grid = static_cast<unsigned>((a.NB + 1) / 2) * a.B * a.HQ;
+  kern<<<grid, 512, C::SMEM_ALLOC, st>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
 }
 

@@ -13,10 +13,11 @@ constexpr int kBlockRows = 128;  // anchor block / tile height shared by the pre
 
 // Workspace of the prefill forward.  NB = ceil(T / 128) anchor blocks.
 //   qh, kh  [B*HQ][T][K]   anchored q and k (input dtype):
-//           qh[t] = q[t] * exp(G[t] - AQ[blk(t)]),  kh[t] = k[t] * exp(AK[blk(t)] - G[t])
-//   bsum    [B*HQ][NB][K]  per-block sum of g (natural log)
+//           qh[t] = q[t] * exp(G[t] - AQ[2 * (t / 256)]),  kh[t] = k[t] * exp(AK[t / 128] - G[t])
+//           (query anchors per 256-row block, key anchors per 128-row block)
+//   bsum    [B*HQ][NB][K]  per-128-row-block sum of g (natural log)
 //   AQ, AK  [B*HQ][NB][K]  G just before the block's first row / at its last row
-//   ssl     [B*HQ][NB*128] block-local inclusive prefix of g_scalar * log2(e)
+//   ssl     [B*HQ][NB*128] minus the block-local inclusive prefix of g_scalar * log2(e)
 //   ssb     [B*HQ][NB]     block sum of g_scalar * log2(e)
 //   ssa     [B*HQ][NB][4]  prefix of g_scalar * log2(e) before the block ([0] used)
 //   rowlo   [T]            first admitted key per row (packed documents only)

@@ -3,24 +3,28 @@
 //
 // The score's per-channel factor exp(G[i,n] - G[j,n]) splits exactly as
 //   exp(G[i] - AQ) * exp(AQ - AK) * exp(AK - G[j])
-// for any anchors AQ, AK.  With AQ = G just before the query's 128-row block
-// and AK = G at the last row of the key's block, the first and last factors
-// are folded once into qh and kh here, and the middle one (one vector per
-// (query block, key block) pair) is applied to each key tile inside the main
-// kernel.  Every factor then spans at most one 128-row block, so the
-// exponents stay bounded at any sequence length.  Prefix sums run over the
-// whole row; with packed documents only differences inside a document are
-// ever used, so they equal the per-document sums of the definition.
+// for any anchors AQ, AK.  With AQ = G just before the query's 256-row block
+// and AK = G at the last row of the key's 128-row block, the first and last
+// factors are folded once into qh and kh here, and the middle one (one vector
+// per (query block, key block) pair) is applied to each key tile inside the
+// main kernel.  Every factor then spans at most 256 rows, so the exponents
+// stay bounded at any sequence length.  Prefix sums run over the whole row;
+// with packed documents only differences inside a document are ever used, so
+// they equal the per-document sums of the definition.
 #include "wall_common.cuh"
 #include "wall_internal.h"
 
 namespace wall {
 namespace {
 
-// One CTA per (128-row block, batch*query head).  Thread layout: CG channel
-// groups of 8 channels x RG row groups of RPG consecutive rows.
+// One CTA per (256-row query block, batch*query head); each half of the CTA
+// (128 threads) owns one 128-row key block.  Thread layout per half: CG
+// channel groups of 8 channels x RG row groups of RPG consecutive rows.
+// Key operands are anchored per 128-row block (AK = G at the block's last
+// row); query operands per 256-row block (AQ = G just before the block), so
+// the two 128-row query tiles of one prefill CTA share one anchor.
 template <typename Tin, int KD>
-__global__ void __launch_bounds__(128) prep_local_kernel(
+__global__ void __launch_bounds__(256) prep_local_kernel(
     const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ g,
     const Tin* __restrict__ gs, const int32_t* __restrict__ cu, int nseq, int window, int T,
     int HQ, int H, int NB, Tin* __restrict__ qh, Tin* __restrict__ kh, float* __restrict__ bsum,
@@ -28,12 +32,14 @@ __global__ void __launch_bounds__(128) prep_local_kernel(
   constexpr int CG = KD / 8;
   constexpr int RG = 128 / CG;
   constexpr int RPG = 128 / RG;
-  __shared__ float tot[RG][KD];
-  __shared__ float wsum[4];
+  __shared__ float tot[2][RG][KD];
+  __shared__ float wsum[2][4];
 
-  const int blk = blockIdx.x, bh = blockIdx.y;
+  const int half = threadIdx.x >> 7, tid = threadIdx.x & 127;
+  const int blk = blockIdx.x * 2 + half;  // 128-row block of this half
+  const int bh = blockIdx.y;
   const int b = bh / HQ, hq = bh % HQ, kvh = hq / (HQ / H);
-  const int tid = threadIdx.x, cg = tid % CG, rg = tid / CG;
+  const int cg = tid % CG, rg = tid / CG;
   const int t0 = blk * kBlockRows + rg * RPG;
   const size_t qrow = static_cast<size_t>(HQ) * KD;  // elements between time steps (q, g)
   const size_t krow = static_cast<size_t>(H) * KD;   // (k)
@@ -51,22 +57,24 @@ __global__ void __launch_bounds__(128) prep_local_kernel(
     for (int c = 0; c < 8; ++c) acc[c] += f[c];
   }
 #pragma unroll
-  for (int c = 0; c < 8; ++c) tot[rg][cg * 8 + c] = acc[c];
+  for (int c = 0; c < 8; ++c) tot[half][rg][cg * 8 + c] = acc[c];
   __syncthreads();
 
-  float run[8], total[8];
+  float run[8], total[8], qoff[8];
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
-    float pre = 0.f, all = 0.f;
+    float pre = 0.f, all = 0.f, first = 0.f;
     for (int r = 0; r < RG; ++r) {
-      const float x = tot[r][cg * 8 + c];
+      const float x = tot[half][r][cg * 8 + c];
       all += x;
       if (r < rg) pre += x;
+      if (half == 1) first += tot[0][r][cg * 8 + c];
     }
     run[c] = pre;
     total[c] = all;
+    qoff[c] = first;  // g summed over the first half of the query block
   }
-  if (rg == 0) {
+  if (rg == 0 && blk < NB) {
     float* dst = bsum + (static_cast<size_t>(bh) * NB + blk) * KD + cg * 8;
 #pragma unroll
     for (int c = 0; c < 8; ++c) dst[c] = total[c];
@@ -86,14 +94,14 @@ __global__ void __launch_bounds__(128) prep_local_kernel(
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       run[c] += f[c];
-      x[c] *= expf(run[c]);
+      x[c] *= expf(qoff[c] + run[c]);
       y[c] *= expf(total[c] - run[c]);
     }
     store8(qo + static_cast<size_t>(t) * KD, x);
     store8(ko + static_cast<size_t>(t) * KD, y);
   }
 
-  // Scalar gate: block-local inclusive prefix (log2 units), one row per thread.
+  // Scalar gate: negated 128-block-local inclusive prefix (log2 units), one row per thread.
   if (gs != nullptr) {
     const int t = blk * kBlockRows + tid;
     float x = (t < T) ? load1(gs + (static_cast<size_t>(b) * T + t) * HQ + hq) * kLog2e : 0.f;
@@ -103,11 +111,13 @@ __global__ void __launch_bounds__(128) prep_local_kernel(
       const float y = __shfl_up_sync(0xffffffffu, x, off);
       if (lane >= off) x += y;
     }
-    if (lane == 31) wsum[wid] = x;
+    if (lane == 31) wsum[half][wid] = x;
     __syncthreads();
-    for (int w = 0; w < wid; ++w) x += wsum[w];
-    ssl[static_cast<size_t>(bh) * NB * kBlockRows + blk * kBlockRows + tid] = x;
-    if (tid == kBlockRows - 1) ssb[static_cast<size_t>(bh) * NB + blk] = x;
+    for (int w = 0; w < wid; ++w) x += wsum[half][w];
+    if (blk < NB) {
+      ssl[static_cast<size_t>(bh) * NB * kBlockRows + blk * kBlockRows + tid] = -x;  // negated
+      if (tid == kBlockRows - 1) ssb[static_cast<size_t>(bh) * NB + blk] = x;
+    }
   }
 
   // First admitted key of each row for packed documents (shared by all heads).
@@ -160,8 +170,8 @@ __global__ void __launch_bounds__(KD + 32) prep_scan_kernel(const float* __restr
 template <typename Tin, int KD>
 cudaError_t prep_impl(const FwdArgs& a, const FwdWork& w, cudaStream_t st) {
   const int BHQ = a.B * a.HQ;
-  dim3 grid(a.NB, BHQ);
-  prep_local_kernel<Tin, KD><<<grid, 128, 0, st>>>(
+  dim3 grid((a.NB + 1) / 2, BHQ);
+  prep_local_kernel<Tin, KD><<<grid, 256, 0, st>>>(
       static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.g),
       static_cast<const Tin*>(a.g_scalar), a.cu_seqlens, a.num_seqs, a.window, a.T, a.HQ, a.H,
       a.NB, static_cast<Tin*>(w.qh), static_cast<Tin*>(w.kh), w.bsum, w.ssl, w.ssb, w.rowlo);
