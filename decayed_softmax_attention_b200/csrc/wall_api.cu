@@ -39,18 +39,6 @@ constexpr int kMaxDevices = 64;
 std::mutex g_err_mu;
 int* g_err_addr[kMaxDevices] = {};
 
-int* device_err_word() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_err_mu);
-  if (g_err_addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_wall_err) != cudaSuccess) return nullptr;
-    g_err_addr[dev] = static_cast<int*>(p);
-  }
-  return g_err_addr[dev];
-}
-
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -80,6 +68,35 @@ wall_status_t finish(cudaError_t e, cudaStream_t st) {
 bool supported_dim(int x) { return x == 64 || x == 128; }
 
 }  // namespace
+
+namespace wall {
+
+int* device_error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_err_mu);
+  if (g_err_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_wall_err) != cudaSuccess) return nullptr;
+    g_err_addr[dev] = static_cast<int*>(p);
+  }
+  return g_err_addr[dev];
+}
+
+uint64_t wait_limit_ns() { return static_cast<uint64_t>(g_wait_ms.load()) * 1000000ull; }
+
+bool encode_tiled(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
+                  const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
+                  CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return enc(map, dt, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace wall
 
 extern "C" {
 
@@ -127,7 +144,7 @@ wall_status_t wall_attn_fwd(const void* q, const void* k, const void* v, const v
   if (workspace_bytes < need) return WALL_ERR_WORKSPACE;
   if (!(scale > 0.f) || !std::isfinite(scale)) scale = 1.f / std::sqrt(static_cast<float>(K));
 
-  int* err = device_err_word();
+  int* err = wall::device_error_word();
   if (err == nullptr) return WALL_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
@@ -136,7 +153,7 @@ wall_status_t wall_attn_fwd(const void* q, const void* k, const void* v, const v
   a.cu_seqlens = cu_seqlens; a.num_seqs = num_seqs; a.window = window > 0 ? window : 0;
   a.B = B; a.T = T; a.HQ = HQ; a.H = H; a.K = K; a.V = V; a.NB = static_cast<int>(NB);
   a.scale = scale; a.o = o; a.lse = lse; a.err = err;
-  a.wait_ns = static_cast<uint64_t>(g_wait_ms.load()) * 1000000ull;
+  a.wait_ns = wall::wait_limit_ns();
   a.fault = g_fault_mode.load();
   wall::FwdWork w;
   wall::fwd_workspace_layout(B, T, HQ, K, bf16, &w, static_cast<char*>(workspace));
@@ -151,36 +168,28 @@ wall_status_t wall_attn_fwd(const void* q, const void* k, const void* v, const v
     return finish(e, st);
   }
 
-  EncodeTiledFn enc = encode_fn();
-  if (enc == nullptr) return WALL_ERR_CUDA;
   CUtensorMap tmQ, tmK, tmV;
-  {
+  {  // anchored q / k: [B*HQ][T][K], 64-channel x 128-row boxes, 128-byte swizzle
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(T),
                                 static_cast<cuuint64_t>(B) * HQ};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * 2,
                                    static_cast<cuuint64_t>(T) * K * 2};
     const cuuint32_t box[3] = {64, 128, 1};
-    const cuuint32_t es[3] = {1, 1, 1};
-    if (enc(&tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, w.qh, dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return WALL_ERR_CUDA;
-    if (enc(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, w.kh, dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    if (!wall::encode_tiled(&tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, w.qh, dims, strides, box,
+                            CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !wall::encode_tiled(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, w.kh, dims, strides, box,
+                            CU_TENSOR_MAP_SWIZZLE_128B))
       return WALL_ERR_CUDA;
   }
-  {
+  {  // v: [B, T, H, V], 64-channel x 128-row boxes, 128-byte swizzle
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(V), static_cast<cuuint64_t>(H),
                                 static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B)};
     const cuuint64_t strides[3] = {static_cast<cuuint64_t>(V) * 2,
                                    static_cast<cuuint64_t>(H) * V * 2,
                                    static_cast<cuuint64_t>(T) * H * V * 2};
     const cuuint32_t box[4] = {64, 1, 128, 1};
-    const cuuint32_t es[4] = {1, 1, 1, 1};
-    if (enc(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(v), dims, strides, box,
-            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    if (!wall::encode_tiled(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, v, dims, strides, box,
+                            CU_TENSOR_MAP_SWIZZLE_128B))
       return WALL_ERR_CUDA;
   }
   e = wall::launch_fwd_tc(a, w, tmQ, tmK, tmV, st);
@@ -244,6 +253,9 @@ wall_status_t wall_attn_decode(const void* q, const float* p_curr, const void* v
   a.V = V; a.chunk = chunk; a.scale = scale; a.o = o; a.lse = lse;
   a.part = static_cast<float*>(workspace); a.nsplit = ns;
   a.mid_event = g_stage_ev[1].load();
+  a.err = wall::device_error_word();
+  if (a.err == nullptr) return WALL_ERR_CUDA;
+  a.wait_ns = wall::wait_limit_ns();
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   stage_event(0, st);
   const cudaError_t e = wall::launch_decode(a, dt == WALL_DTYPE_BF16, st);

@@ -156,85 +156,157 @@ __global__ void __launch_bounds__(256) cache_build_kernel(
 }
 
 // ----------------------------------------------------------------- split-KV decode
-constexpr int kDecWarps = 4;
-constexpr int kRowBatch = 8;
+// Rows of one (batch, KV head) are streamed through a ring of shared-memory
+// stages by TMA: per stage SR rows of the group's k_tilde ([SR][G][K]), of v
+// ([SR][V]) and the anchor vectors of their chunk ([G][K] fp32).  The tensor
+// maps end at T_kv, so rows past the cache length arrive as zeros (and are
+// masked).  One producer thread issues the copies; NW consumer warps split
+// each stage's rows.  Bytes in flight = stages x stage size, independent of
+// registers.
+template <typename T, int KD, int VD, int G>
+struct DecCfg {
+  static constexpr int GK = G * KD;
+  static constexpr int ESZ = static_cast<int>(sizeof(T));
+  static constexpr int SR0 = 32768 / (GK * ESZ);
+  static constexpr int SR = SR0 > 32 ? 32 : (SR0 < 8 ? 8 : SR0);  // rows per stage
+  static constexpr int NW = 4;                                     // consumer warps
+  static constexpr int RPW = SR / NW;                              // rows per warp per stage
+  static constexpr int K_BYTES = SR * GK * ESZ;
+  static constexpr int V_BYTES = SR * VD * ESZ;
+  static constexpr int R_BYTES = GK * 4;
+  static constexpr int STAGE = K_BYTES + V_BYTES + R_BYTES;
+  static constexpr int MERGE = NW * G * (VD + 2) * 4;
+  static constexpr int NS0 = (196608 - MERGE) / STAGE;
+  static constexpr int NS = NS0 > 4 ? 4 : NS0;                     // stages in the ring
+  static constexpr int OFF_BAR = NS * STAGE;
+  static constexpr int OFF_MERGE = OFF_BAR + 2 * NS * 8 + 16;
+  static constexpr int SMEM = OFF_MERGE + MERGE + 128;
+  static_assert(NS >= 2, "decode stage does not fit");
+  static_assert(SR % NW == 0, "rows per stage must split over the consumer warps");
+};
 
 template <typename T, int KD, int VD, int G>
-__global__ void __launch_bounds__(kDecWarps * 32) decode_split_kernel(
-    const T* __restrict__ q, const float* __restrict__ p_curr, const T* __restrict__ v,
-    const T* __restrict__ k_tilde, const float* __restrict__ r_cache, int T_kv, int cap, int HQ,
-    int H, int C, int cps, int nsplit, float sc, float* __restrict__ part) {
+__global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_split_kernel(
+    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+    const T* __restrict__ q, const float* __restrict__ p_curr, const float* __restrict__ r_cache,
+    int T_kv, int cap, int HQ, int C, int cps, int nsplit, float sc, float* __restrict__ part,
+    int* err, uint64_t wait_ns) {
+  using D = DecCfg<T, KD, VD, G>;
   constexpr int LPH = 32 / G;    // lanes per query head
   constexpr int CPL = KD / LPH;  // k_tilde channels per lane
   constexpr int VPL = VD / 32;   // v channels per lane
-  __shared__ float sm_m[kDecWarps][G], sm_l[kDecWarps][G];
-  __shared__ __align__(16) float sm_o[kDecWarps][G][VD];
+  extern __shared__ __align__(128) uint8_t dsm[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(dsm + D::OFF_BAR);
+  uint64_t* empty = full + D::NS;
+  int* abort_flag = reinterpret_cast<int*>(dsm + D::OFF_BAR + 2 * D::NS * 8);
+  float* sm_ml = reinterpret_cast<float*>(dsm + D::OFF_MERGE);       // [NW][G][2]
+  float* sm_o = sm_ml + D::NW * G * 2;                               // [NW][G][VD]
 
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int hl = lane / LPH;
-  const int hq = h * G + hl;
-  const int cofs = (lane % LPH) * CPL;
   const int nchunks = (T_kv + C - 1) / C;
   const int ncap = (cap + C - 1) / C;
+  const int ck0 = s * cps;
+  const int ck1 = min(ck0 + cps, nchunks);
+  const int row_begin = ck0 * C;
+  const int row_end = min(ck1 * C, T_kv);
+  const int nst = row_end > row_begin ? (row_end - row_begin + D::SR - 1) / D::SR : 0;
 
-  float qv[CPL], pc[CPL];
-  load_n<T, CPL>(q + (static_cast<size_t>(b) * HQ + hq) * KD + cofs, qv);
-  load_n<float, CPL>(p_curr + (static_cast<size_t>(b) * HQ + hq) * KD + cofs, pc);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < D::NS; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], D::NW);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const WaitCtl wc{abort_flag, err, wait_ns};
 
-  float m = -INFINITY, l = 0.f;
-  float o[G][VPL];
-#pragma unroll
-  for (int hh = 0; hh < G; ++hh)
-#pragma unroll
-    for (int c = 0; c < VPL; ++c) o[hh][c] = 0.f;
-
-  const size_t krow = static_cast<size_t>(HQ) * KD;
-  const size_t vrow = static_cast<size_t>(H) * VD;
-  const T* kbase = k_tilde + static_cast<size_t>(b) * cap * krow + static_cast<size_t>(h) * G * KD +
-                   static_cast<size_t>(lane) * CPL;
-  const T* vbase = v + static_cast<size_t>(b) * cap * vrow + static_cast<size_t>(h) * VD + lane * VPL;
-
-  const int ck_end = min((s + 1) * cps, nchunks);
-  for (int ck = s * cps + warp; ck < ck_end; ck += kDecWarps) {
-    float qt[CPL], R[CPL];
-    load_n<float, CPL>(r_cache + ((static_cast<size_t>(b) * ncap + ck) * HQ + hq) * KD + cofs, R);
-#pragma unroll
-    for (int e = 0; e < CPL; ++e) qt[e] = qv[e] * sc * exp2f(pc[e] - R[e]);
-    const int r0 = ck * C, r1 = min(r0 + C, T_kv);
-    for (int j = r0; j < r1; j += kRowBatch) {
-      float sres[kRowBatch], vv[kRowBatch][VPL];
-#pragma unroll
-      for (int rr = 0; rr < kRowBatch; ++rr) {
-        const int jj = j + rr;
-        float part_dot = 0.f;
-        if (jj < r1) {
-          float kf[CPL];
-          load_n<T, CPL>(kbase + static_cast<size_t>(jj) * krow, kf);
-          load_n<T, VPL>(vbase + static_cast<size_t>(jj) * vrow, vv[rr]);
-#pragma unroll
-          for (int e = 0; e < CPL; ++e) part_dot = fmaf(qt[e], kf[e], part_dot);
-        } else {
-#pragma unroll
-          for (int c = 0; c < VPL; ++c) vv[rr][c] = 0.f;
-        }
-        sres[rr] = part_dot;
+  if (warp == D::NW) {
+    // ------------------------------------------------------------- producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      int issued = 0;
+      for (int i = 0; i < nst; ++i) {
+        const int slot = i % D::NS;
+        if (i >= D::NS && !mbar_wait(&empty[slot], ((i / D::NS) - 1) & 1, wc)) break;
+        const int row0 = row_begin + i * D::SR;
+        uint8_t* st = dsm + slot * D::STAGE;
+        mbar_arrive_expect_tx(&full[slot], D::STAGE);
+        tma_load_4d(st, &tmK, &full[slot], 0, h * G, row0, b);
+        tma_load_4d(st + D::K_BYTES, &tmV, &full[slot], 0, h, row0, b);
+        bulk_load(st + D::K_BYTES + D::V_BYTES,
+                  r_cache + ((static_cast<size_t>(b) * ncap + row0 / C) * HQ + h * G) * KD,
+                  D::R_BYTES, &full[slot]);
+        issued = i + 1;
       }
+      for (int i = issued > D::NS ? issued - D::NS : 0; i < issued; ++i)
+        mbar_drain(&full[i % D::NS], (i / D::NS) & 1, wait_ns);
+    }
+  } else {
+    // ------------------------------------------------------------- consumers
+    const int hl = lane / LPH;
+    const int hq = h * G + hl;
+    const int cofs = (lane % LPH) * CPL;
+    float qv[CPL], pc[CPL], qt[CPL];
+    load_n<T, CPL>(q + (static_cast<size_t>(b) * HQ + hq) * KD + cofs, qv);
+    load_n<float, CPL>(p_curr + (static_cast<size_t>(b) * HQ + hq) * KD + cofs, pc);
 #pragma unroll
-      for (int rr = 0; rr < kRowBatch; ++rr) {
+    for (int e = 0; e < CPL; ++e) qv[e] *= sc;
+    float m = -INFINITY, l = 0.f;
+    float o[G][VPL];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+      for (int c = 0; c < VPL; ++c) o[hh][c] = 0.f;
+    int cur_chunk = -1;
+    for (int i = 0; i < nst; ++i) {
+      const int slot = i % D::NS;
+      const bool got = mbar_wait(&full[slot], (i / D::NS) & 1, wc);
+      if (!__all_sync(0xffffffffu, got)) break;
+      const uint8_t* st = dsm + slot * D::STAGE;
+      const int row0 = row_begin + i * D::SR;
+      if (row0 / C != cur_chunk) {
+        cur_chunk = row0 / C;
+        float R[CPL];
+        load_n<float, CPL>(reinterpret_cast<const float*>(st + D::K_BYTES + D::V_BYTES) +
+                               lane * CPL, R);
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) qt[e] = qv[e] * exp2f(pc[e] - R[e]);
+      }
+      const int r0 = warp * D::RPW;
+      float sres[D::RPW], vv[D::RPW][VPL];
+#pragma unroll
+      for (int rr = 0; rr < D::RPW; ++rr) {
+        float kf[CPL];
+        load_n<T, CPL>(reinterpret_cast<const T*>(st) + (r0 + rr) * D::GK + lane * CPL, kf);
+        load_n<T, VPL>(reinterpret_cast<const T*>(st + D::K_BYTES) + (r0 + rr) * VD + lane * VPL,
+                       vv[rr]);
+        float d = 0.f;
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) d = fmaf(qt[e], kf[e], d);
+        sres[rr] = d;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+#pragma unroll
+      for (int rr = 0; rr < D::RPW; ++rr) {
 #pragma unroll
         for (int off = LPH / 2; off > 0; off >>= 1)
           sres[rr] += __shfl_xor_sync(0xffffffffu, sres[rr], off);
-        if (j + rr >= r1) sres[rr] = -INFINITY;
+        if (row0 + r0 + rr >= row_end) sres[rr] = -INFINITY;
       }
       float mloc = sres[0];
 #pragma unroll
-      for (int rr = 1; rr < kRowBatch; ++rr) mloc = fmaxf(mloc, sres[rr]);
-      const float mn = fmaxf(m, mloc);  // finite: row j is always admitted
+      for (int rr = 1; rr < D::RPW; ++rr) mloc = fmaxf(mloc, sres[rr]);
+      const float mn = fmaxf(m, mloc);
+      if (mn == -INFINITY) continue;  // every row of this warp's slice is past the end
       const float alpha = exp2f(m - mn);
-      float pr[kRowBatch], rs = 0.f;
+      float pr[D::RPW], rs = 0.f;
 #pragma unroll
-      for (int rr = 0; rr < kRowBatch; ++rr) {
+      for (int rr = 0; rr < D::RPW; ++rr) {
         pr[rr] = exp2f(sres[rr] - mn);
         rs += pr[rr];
       }
@@ -246,30 +318,29 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_split_kernel(
 #pragma unroll
         for (int c = 0; c < VPL; ++c) o[hh][c] *= ah;
 #pragma unroll
-        for (int rr = 0; rr < kRowBatch; ++rr) {
+        for (int rr = 0; rr < D::RPW; ++rr) {
           const float ph = __shfl_sync(0xffffffffu, pr[rr], hh * LPH);
 #pragma unroll
           for (int c = 0; c < VPL; ++c) o[hh][c] = fmaf(ph, vv[rr][c], o[hh][c]);
         }
       }
     }
-  }
-
-  // merge the warps of this CTA
-  if (lane % LPH == 0) {
-    sm_m[warp][hl] = m;
-    sm_l[warp][hl] = l;
-  }
+    if (lane % LPH == 0) {
+      sm_ml[(warp * G + hl) * 2] = m;
+      sm_ml[(warp * G + hl) * 2 + 1] = l;
+    }
 #pragma unroll
-  for (int hh = 0; hh < G; ++hh)
+    for (int hh = 0; hh < G; ++hh)
 #pragma unroll
-    for (int c = 0; c < VPL; ++c) sm_o[warp][hh][lane * VPL + c] = o[hh][c];
+      for (int c = 0; c < VPL; ++c) sm_o[(warp * G + hh) * VD + lane * VPL + c] = o[hh][c];
+  }
   __syncthreads();
-  for (int e = threadIdx.x; e < G * (VD + 2); e += kDecWarps * 32) {
+  // merge the consumer warps of this CTA into one partial per query head
+  for (int e = threadIdx.x; e < G * (VD + 2); e += (D::NW + 1) * 32) {
     const int hh = e / (VD + 2), c = e % (VD + 2);
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, sm_m[w][hh]);
+    for (int w = 0; w < D::NW; ++w) M = fmaxf(M, sm_ml[(w * G + hh) * 2]);
     float val;
     if (M == -INFINITY) {
       val = (c == VD) ? -INFINITY : 0.f;
@@ -278,9 +349,11 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_split_kernel(
     } else {
       val = 0.f;
 #pragma unroll
-      for (int w = 0; w < kDecWarps; ++w) {
-        const float wt = exp2f(sm_m[w][hh] - M);
-        val += wt * (c == VD + 1 ? sm_l[w][hh] : sm_o[w][hh][c]);
+      for (int w = 0; w < D::NW; ++w) {
+        const float mw = sm_ml[(w * G + hh) * 2];
+        if (mw == -INFINITY) continue;
+        const float wt = exp2f(mw - M);
+        val += wt * (c == VD + 1 ? sm_ml[(w * G + hh) * 2 + 1] : sm_o[(w * G + hh) * VD + c]);
       }
     }
     part[((static_cast<size_t>(b) * HQ + h * G + hh) * nsplit + s) * (VD + 2) + c] = val;
@@ -352,14 +425,41 @@ cudaError_t cache_dispatch(const CacheArgs& a, cudaStream_t st) {
 
 template <typename T, int KD, int VD, int G>
 cudaError_t decode_impl(const DecodeArgs& a, cudaStream_t st) {
+  using D = DecCfg<T, KD, VD, G>;
+  const CUtensorMapDataType tdt =
+      sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  CUtensorMap tmK, tmV;
+  {  // k_tilde [B, cap, HQ, K], rows limited to T_kv
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(KD), static_cast<cuuint64_t>(a.HQ),
+                                static_cast<cuuint64_t>(a.T_kv), static_cast<cuuint64_t>(a.B)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(KD) * sizeof(T),
+                                   static_cast<cuuint64_t>(a.HQ) * KD * sizeof(T),
+                                   static_cast<cuuint64_t>(a.cap) * a.HQ * KD * sizeof(T)};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(KD), static_cast<cuuint32_t>(G),
+                               static_cast<cuuint32_t>(D::SR), 1};
+    if (!encode_tiled(&tmK, tdt, 4, a.k_tilde, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+  }
+  {  // v [B, cap, H, V]
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(VD), static_cast<cuuint64_t>(a.H),
+                                static_cast<cuuint64_t>(a.T_kv), static_cast<cuuint64_t>(a.B)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(VD) * sizeof(T),
+                                   static_cast<cuuint64_t>(a.H) * VD * sizeof(T),
+                                   static_cast<cuuint64_t>(a.cap) * a.H * VD * sizeof(T)};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(VD), 1, static_cast<cuuint32_t>(D::SR), 1};
+    if (!encode_tiled(&tmV, tdt, 4, a.v, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+  }
+  auto kern = decode_split_kernel<T, KD, VD, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, D::SMEM);
+  if (e != cudaSuccess) return e;
   const int nchunks = (a.T_kv + a.chunk - 1) / a.chunk;
   const int cps = (nchunks + a.nsplit - 1) / a.nsplit;
   dim3 grid(a.nsplit, a.H, a.B);
-  decode_split_kernel<T, KD, VD, G><<<grid, kDecWarps * 32, 0, st>>>(
-      static_cast<const T*>(a.q), a.p_curr, static_cast<const T*>(a.v),
-      static_cast<const T*>(a.k_tilde), a.r_cache, a.T_kv, a.cap, a.HQ, a.H, a.chunk, cps,
-      a.nsplit, a.scale * kLog2e, a.part);
-  cudaError_t e = cudaGetLastError();
+  kern<<<grid, (D::NW + 1) * 32, D::SMEM, st>>>(
+      tmK, tmV, static_cast<const T*>(a.q), a.p_curr, a.r_cache, a.T_kv, a.cap, a.HQ, a.chunk,
+      cps, a.nsplit, a.scale * kLog2e, a.part, a.err, a.wait_ns);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (a.mid_event != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(a.mid_event), st);
   const int nbh = a.B * a.HQ;
@@ -402,12 +502,12 @@ bool decode_supported(int K, int V, int group) {
   return kv && g;
 }
 
-// Upper bound on the split count: enough CTAs to fill every SM several times
-// over, never more splits than chunks.  Non-decreasing in T_kv.
+// Upper bound on the split count (sizes the workspace): enough CTAs for several
+// full waves over the SMs, never more splits than chunks.  Non-decreasing in T_kv.
 int decode_max_splits(int B, int T_kv, int HQ, int H, int chunk) {
   (void)HQ;
   const long nchunks = (static_cast<long>(T_kv) + chunk - 1) / chunk;
-  const long target = 148L * 8;
+  const long target = 148L * 16;
   const long groups = static_cast<long>(B) * H;
   long ns = (target + groups - 1) / groups;
   if (ns < 1) ns = 1;
@@ -415,13 +515,29 @@ int decode_max_splits(int B, int T_kv, int HQ, int H, int chunk) {
   return static_cast<int>(ns);
 }
 
-// Splits actually launched: chunks are dealt out evenly, so trailing splits
-// are never empty.  Never above decode_max_splits().
+// Splits actually launched (one CTA per SM is resident): the count up to the
+// bound whose CTAs fill the last wave best, preferring fewer splits; chunks are
+// dealt out evenly so no split is empty.
 int decode_num_splits(int B, int T_kv, int HQ, int H, int chunk) {
-  const int ns = decode_max_splits(B, T_kv, HQ, H, chunk);
+  const int ns_max = decode_max_splits(B, T_kv, HQ, H, chunk);
   const int nchunks = (T_kv + chunk - 1) / chunk;
-  const int cps = (nchunks + ns - 1) / ns;
-  return (nchunks + cps - 1) / cps;
+  const long groups = static_cast<long>(B) * H;
+  const long sms = 148;
+  int best = 1;
+  double best_eff = -1.0;
+  for (int ns = 1; ns <= ns_max; ++ns) {
+    const int cps = (nchunks + ns - 1) / ns;
+    const int used = (nchunks + cps - 1) / cps;
+    const long ctas = groups * used;
+    const long waves = (ctas + sms - 1) / sms;
+    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * sms);
+    const double score = eff * (ctas >= sms ? 1.0 : static_cast<double>(ctas) / sms);
+    if (score > best_eff + 0.02) {
+      best_eff = score;
+      best = used;
+    }
+  }
+  return best;
 }
 
 size_t decode_workspace_bytes(int B, int HQ, int V, int nsplit) {

@@ -84,6 +84,9 @@ extern "C" wall_status_t wall_attn_decode_noalloc(
   a.sink = sink_bias; a.B = B; a.T_kv = T_kv; a.cap = cap; a.HQ = HQ; a.H = H; a.K = K;
   a.V = V; a.chunk = chunk; a.scale = scale; a.o = o; a.lse = lse;
   a.part = scratch; a.nsplit = ns; a.mid_event = nullptr;
+  a.err = wall::device_error_word();
+  if (a.err == nullptr) return WALL_ERR_CUDA;
+  a.wait_ns = wall::wait_limit_ns();
   const cudaError_t e = wall::launch_decode(a, dt == WALL_DTYPE_BF16,
                                             reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;

@@ -9,7 +9,17 @@
 
 namespace wall {
 
-constexpr int kBlockRows = 128;  // anchor block / tile height shared by the prefill kernels
+constexpr int kBlockRows = 128;
+
+// Device address of this device's error word (bit 0: a bounded wait gave up).
+int* device_error_word();
+// Current limit of every bounded device-side wait, in nanoseconds.
+uint64_t wait_limit_ns();
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda
+// link): unit element strides, zero fill out of bounds.  strides in bytes.
+bool encode_tiled(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
+                  const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
+                  CUtensorMapSwizzle swizzle);  // anchor block / tile height shared by the prefill kernels
 
 // Workspace of the prefill forward.  NB = ceil(T / 128) anchor blocks.
 //   qh, kh  [B*HQ][T][K]   anchored q and k (input dtype):
@@ -84,6 +94,8 @@ struct DecodeArgs {
   float* part;  // workspace
   int nsplit;
   void* mid_event;  // optional cudaEvent_t recorded between the split and combine kernels
+  int* err;         // device error word
+  uint64_t wait_ns; // bounded-wait limit
 };
 int decode_max_splits(int B, int T_kv, int HQ, int H, int chunk);
 int decode_num_splits(int B, int T_kv, int HQ, int H, int chunk);
