@@ -192,7 +192,16 @@ wall_status_t wall_attn_fwd(const void* q, const void* k, const void* v, const v
                             CU_TENSOR_MAP_SWIZZLE_128B))
       return WALL_ERR_CUDA;
   }
-  e = wall::launch_fwd_tc(a, w, tmQ, tmK, tmV, st);
+  CUtensorMap tmKX = tmK;
+  if (g_scalar != nullptr) {  // key-side gate channels: [B*HQ][T][16] bf16, 32-byte swizzle
+    const cuuint64_t dims[3] = {16, static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B) * HQ};
+    const cuuint64_t strides[2] = {32, static_cast<cuuint64_t>(T) * 32};
+    const cuuint32_t box[3] = {16, 128, 1};
+    if (!wall::encode_tiled(&tmKX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, w.kx, dims, strides, box,
+                            CU_TENSOR_MAP_SWIZZLE_32B))
+      return WALL_ERR_CUDA;
+  }
+  e = wall::launch_fwd_tc(a, w, tmQ, tmK, tmV, tmKX, st);
   stage_event(2, st);
   return finish(e, st);
 }

@@ -19,7 +19,8 @@
 // Warp roles (512 threads): warpgroup 0 = warp 0 TMA producer, warp 1 MMA
 // issuer, warp 2 TMEM allocator; warpgroups 1 and 2 = softmax + epilogue of
 // query tiles A and B; warpgroup 3 = key-tile rescale.  Registers are
-// re-balanced at start (setmaxnreg): the softmax warpgroups get 184.
+// re-balanced at start (setmaxnreg): softmax warpgroups 192, warpgroup 0 80,
+// rescale 48 (sum 512 per thread slot = the 65536 registers of the launch).
 //
 // MMA issue order per key tile j: PV_A(j-1), QK_A(j), PV_B(j-1), QK_B(j), so
 // one softmax warpgroup works while the tensor core serves the other, and
@@ -64,10 +65,13 @@ struct TcCfg {
   static constexpr int OFF_V = OFF_K + KS * K_BYTES;
   static constexpr int OFF_AQ = OFF_V + VS * V_BYTES;
   static constexpr int OFF_AK = OFF_AQ + KD * 4;
-  static constexpr int OFF_COL = OFF_AK + KS * KD * 4;
-  static constexpr int OFF_COLA = OFF_COL + VS * BN * 4;
-  static constexpr int OFF_C = OFF_COLA + VS * 16;
-  static constexpr int OFF_BAR = OFF_C + 2 * KD * 4;
+  static constexpr int OFF_C = OFF_AK + KS * KD * 4;
+  // gate channels of the QK contraction (one 16-channel K slice, 32-byte
+  // swizzle): query side constant (1, 1, 0, ...), key side per stage
+  static constexpr int GX_BYTES = BM * 32;
+  static constexpr int OFF_QX = (OFF_C + 2 * KD * 4 + 1023) / 1024 * 1024;
+  static constexpr int OFF_KX = OFF_QX + GX_BYTES;
+  static constexpr int OFF_BAR = OFF_KX + KS * GX_BYTES;
   // qfull, kfull[KS], kready[KS], kempty[KS], vfull[VS], vempty[VS], sfull[2], pfull[2],
   // ofinal, mdrain
   static constexpr int NBAR = 1 + 3 * KS + 2 * VS + 2 + 2 + 2;
@@ -82,17 +86,16 @@ struct TcCfg {
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, VD, 0, 1);
 };
 
-// Pack the 8 bf16 of one 16-byte chunk, scaled by c[0..7].
-__device__ __forceinline__ uint4 scale_chunk(uint4 u, const float* c) {
+// Scale the 8 bf16 of one 16-byte chunk by c[0..7], with c split into a bf16
+// head and a bf16 tail (chi + clo == c to ~16 bits): x*clo is formed first and
+// x*chi + x*clo is rounded once, so the result carries a single bf16 rounding.
+__device__ __forceinline__ uint4 scale_chunk(uint4 u, const __nv_bfloat162* chi,
+                                             const __nv_bfloat162* clo) {
   uint4 r;
-  const float2 a = fmul2(make_float2(bf16_lo(u.x), bf16_hi(u.x)), make_float2(c[0], c[1]));
-  const float2 b = fmul2(make_float2(bf16_lo(u.y), bf16_hi(u.y)), make_float2(c[2], c[3]));
-  const float2 d = fmul2(make_float2(bf16_lo(u.z), bf16_hi(u.z)), make_float2(c[4], c[5]));
-  const float2 e = fmul2(make_float2(bf16_lo(u.w), bf16_hi(u.w)), make_float2(c[6], c[7]));
-  r.x = pack_bf16(a.x, a.y);
-  r.y = pack_bf16(b.x, b.y);
-  r.z = pack_bf16(d.x, d.y);
-  r.w = pack_bf16(e.x, e.y);
+  const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&u);
+  __nv_bfloat162* y = reinterpret_cast<__nv_bfloat162*>(&r);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) y[i] = __hfma2(x[i], chi[i], __hmul2(x[i], clo[i]));
   return r;
 }
 
@@ -124,7 +127,8 @@ template <int KD, int VD, bool HAS_GS>
 __global__ void __launch_bounds__(512, 1)
     wall_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmV, const TcParams p) {
+                       const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ CUtensorMap tmKX, const TcParams p) {
   using C = TcCfg<KD, VD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -134,9 +138,9 @@ __global__ void __launch_bounds__(512, 1)
   uint8_t* sV = smem + C::OFF_V;
   float* sAQ = reinterpret_cast<float*>(smem + C::OFF_AQ);
   float* sAK = reinterpret_cast<float*>(smem + C::OFF_AK);
-  float* sCol = reinterpret_cast<float*>(smem + C::OFF_COL);
-  float* sColA = reinterpret_cast<float*>(smem + C::OFF_COLA);
   float* sC = reinterpret_cast<float*>(smem + C::OFF_C);
+  uint8_t* sQX = smem + C::OFF_QX;
+  uint8_t* sKX = smem + C::OFF_KX;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* qfull = bars;
   uint64_t* kfull = bars + 1;
@@ -189,6 +193,14 @@ __global__ void __launch_bounds__(512, 1)
     tmem_relinquish();
     tc_fence_before();
   }
+  if (HAS_GS && tid >= 128 && tid < 256) {
+    // query-side gate channels (1, 1, 0, ..., 0) per row, 32-byte swizzled
+    const int r = tid - 128;
+    const int half = (r >> 2) & 1;  // where the logical first 16 bytes land
+    *reinterpret_cast<uint4*>(sQX + r * 32 + half * 16) = make_uint4(0x3F803F80u, 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(sQX + r * 32 + (half ^ 1) * 16) = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+  }
   __syncthreads();
 
   // Admitted key range per query row: [lo_i, i] (causal, window, document).
@@ -222,7 +234,7 @@ __global__ void __launch_bounds__(512, 1)
   const WaitCtl wc{abort_flag, p.err, p.wait_ns};
 
   if (wg == 0) {
-    reg_dealloc<56>();
+    reg_dealloc<80>();
     if (warp == 0 && lane == 0) {
       // ----------------------------------------------------------- TMA producer
       tma_prefetch_desc(&tmQ);
@@ -240,26 +252,20 @@ __global__ void __launch_bounds__(512, 1)
         const int ks = j % C::KS;
         if (j >= C::KS && !mbar_wait(&kempty[ks], ((j / C::KS) - 1) & 1, wc)) break;
         if (!(p.fault == 1 && j == 0)) {
-          mbar_arrive_expect_tx(&kfull[ks], C::K_BYTES + KD * 4);
+          mbar_arrive_expect_tx(&kfull[ks], C::K_BYTES + KD * 4 + (HAS_GS ? C::GX_BYTES : 0));
           for (int bx = 0; bx < C::QBOX; ++bx)
             tma_load_3d(sK + ks * C::K_BYTES + bx * 16384, &tmK, &kfull[ks], bx * 64, kt * C::BN, bh);
+          if (HAS_GS) tma_load_3d(sKX + ks * C::GX_BYTES, &tmKX, &kfull[ks], 0, kt * C::BN, bh);
           bulk_load(sAK + ks * KD, p.AK + (static_cast<size_t>(bh) * p.NB + kt) * KD, KD * 4,
                     &kfull[ks]);
         }
         nk = j + 1;
         const int vs = j % C::VS;
         if (j >= C::VS && !mbar_wait(&vempty[vs], ((j / C::VS) - 1) & 1, wc)) break;
-        mbar_arrive_expect_tx(&vfull[vs], C::V_BYTES + (HAS_GS ? C::BN * 4 + 16 : 0));
+        mbar_arrive_expect_tx(&vfull[vs], C::V_BYTES);
         for (int bx = 0; bx < C::VBOX; ++bx)
           tma_load_4d(sV + vs * C::V_BYTES + bx * 16384, &tmV, &vfull[vs], bx * 64, kvh,
                       kt * C::BN, b);
-        if (HAS_GS) {
-          bulk_load(sCol + vs * C::BN,
-                    p.ssl + static_cast<size_t>(bh) * p.NB * C::BN + static_cast<size_t>(kt) * C::BN,
-                    C::BN * 4, &vfull[vs]);
-          bulk_load(sColA + vs * 4, p.ssa + (static_cast<size_t>(bh) * p.NB + kt) * 4, 16,
-                    &vfull[vs]);
-        }
         nv = j + 1;
       }
       // Every copy issued must land before the CTA may exit: the last KS (VS)
@@ -300,6 +306,11 @@ __global__ void __launch_bounds__(512, 1)
           const uint64_t bdesc = sw128_desc(sKa + ks * C::K_BYTES + koff, 16, 1024);
           umma_ss(dS, adesc, bdesc, C::IDESC_QK, kk > 0 ? 1u : 0u);
         }
+        if (HAS_GS) {
+          // + key-side gate term: (1, 1, 0..) x (hi, lo, 0..) over one more K slice
+          const uint32_t qx = smem_u32(sQX), kx = smem_u32(sKX + ks * C::GX_BYTES);
+          umma_ss(dS, sw32_desc(qx, 256), sw32_desc(kx, 256), C::IDESC_QK, 1u);
+        }
         umma_commit(&sfull[x]);
       };
       for (int j = 0; ok && j < nt; ++j) {
@@ -337,7 +348,7 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (is_softmax) {
     // ------------------------------------------------------------- softmax + epilogue
-    reg_alloc<184>();
+    reg_alloc<192>();
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const uint32_t colS = C::COL_S + 128 * X, colO = C::COL_O + 128 * X;
     const int lo = row_ok ? my_lo : 0;
@@ -351,11 +362,15 @@ __global__ void __launch_bounds__(512, 1)
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     const int jf = X == 0 ? jfA : jfB, jl = X == 0 ? jlA : jlB;
+    // gate prefix before the key tile (log2 units), fetched one tile ahead
+    float colA_next = 0.f;
+    if (HAS_GS && jl >= jf) colA_next = p.ssa[(static_cast<size_t>(bh) * p.NB + (kt_hi - jf)) * 4];
     for (int j = jf; j <= jl; ++j) {
       const int cnt = j - jf;
-      const int kt = kt_hi - j, vs = j % C::VS;
-      bool got = mbar_wait(&sfull[X], cnt & 1, wc);
-      if (HAS_GS && got) got = mbar_wait(&vfull[vs], (j / C::VS) & 1, wc);
+      const int kt = kt_hi - j;
+      const float colA = colA_next;
+      if (HAS_GS && j < jl) colA_next = p.ssa[(static_cast<size_t>(bh) * p.NB + (kt - 1)) * 4];
+      const bool got = mbar_wait(&sfull[X], cnt & 1, wc);
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
@@ -368,20 +383,10 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
       for (int c = 0; c < C::BN; c += 32) reg_fence32(s + c);
 
+      // S already holds scale^-1 * (key-side gate term) for gated inputs; the
+      // row side joins through w.
       const int j0 = kt * C::BN;
-      float w = 0.f;
-      if (HAS_GS) {
-        // t = S * scale*log2e - (key-side gate prefix); the row side joins below
-        const float* col = sCol + vs * C::BN;
-        w = rowA - sColA[vs * 4];
-#pragma unroll
-        for (int jj = 0; jj < C::BN; jj += 4) {
-          const float4 cv = *reinterpret_cast<const float4*>(col + jj);
-          const float2 t0 = ffma2(make_float2(s[jj], s[jj + 1]), sc2, make_float2(cv.x, cv.y));
-          const float2 t1 = ffma2(make_float2(s[jj + 2], s[jj + 3]), sc2, make_float2(cv.z, cv.w));
-          s[jj] = t0.x; s[jj + 1] = t0.y; s[jj + 2] = t1.x; s[jj + 3] = t1.y;
-        }
-      }
+      const float w = HAS_GS ? rowA - colA : 0.f;
       const bool partial = !__all_sync(0xffffffffu, lo <= j0 && hi >= j0 + C::BN - 1);
       if (partial) {
 #pragma unroll
@@ -396,8 +401,7 @@ __global__ void __launch_bounds__(512, 1)
         mx0 = fmax3(mx0, s[jj], s[jj + 1]);
         mx1 = fmax3(mx1, s[jj + 2], s[jj + 3]);
       }
-      float mt = fmaxf(mx0, mx1);
-      mt = HAS_GS ? mt + w : mt * p.sc;
+      const float mt = fmaxf(mx0, mx1) * p.sc + w;
       const bool need = mt > m_used + 8.f;
       float alpha = 1.f;
       if (need) {
@@ -406,7 +410,7 @@ __global__ void __launch_bounds__(512, 1)
         m_used = mt;
       }
       const float base = (m_used == -INFINITY) ? 0.f : m_used;
-      const float2 off = HAS_GS ? make_float2(w - base, w - base) : make_float2(-base, -base);
+      const float2 off = make_float2(w - base, w - base);
       float2 rs = make_float2(0.f, 0.f);
       // P in 32-column chunks: each chunk's scores die once its 16 packed
       // bf16x2 columns are stored over S (the chunk's own, already-read columns).
@@ -415,8 +419,7 @@ __global__ void __launch_bounds__(512, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int jj = 0; jj < 32; jj += 2) {
-          const float2 sv = make_float2(s[c + jj], s[c + jj + 1]);
-          const float2 t = HAS_GS ? fadd2(sv, off) : ffma2(sv, sc2, off);
+          const float2 t = ffma2(make_float2(s[c + jj], s[c + jj + 1]), sc2, off);
           const float2 pv = make_float2(ex2_approx(t.x), ex2_approx(t.y));
           rs = fadd2(rs, pv);
           pk[jj >> 1] = pack_bf16(pv.x, pv.y);
@@ -481,7 +484,7 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else {
     // ------------------------------------------------------------- key-tile rescale
-    reg_dealloc<80>();
+    reg_dealloc<48>();
     const int r = tid - 384;
     bool ok = mbar_wait(qfull, 0, wc);
     ok = !bar_or(1, 128, !ok);
@@ -496,16 +499,23 @@ __global__ void __launch_bounds__(512, 1)
       float* cb = sC + (j & 1) * KD;
       if (got && r < KD) cb[r] = ex2_approx((sAQ[r] - sAK[ks * KD + r]) * kLog2e);
       if (bar_or(1, 128, !got || *abort_flag != 0)) break;
-      float cv[8];
-      const float4 c0 = *reinterpret_cast<const float4*>(cb + box * 64 + c16 * 8);
-      const float4 c1 = *reinterpret_cast<const float4*>(cb + box * 64 + c16 * 8 + 4);
-      cv[0] = c0.x; cv[1] = c0.y; cv[2] = c0.z; cv[3] = c0.w;
-      cv[4] = c1.x; cv[5] = c1.y; cv[6] = c1.z; cv[7] = c1.w;
+      __nv_bfloat162 chi[4], clo[4];
+      {
+        const float4 c0 = *reinterpret_cast<const float4*>(cb + box * 64 + c16 * 8);
+        const float4 c1 = *reinterpret_cast<const float4*>(cb + box * 64 + c16 * 8 + 4);
+        const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          chi[i] = __floats2bfloat162_rn(cv[2 * i], cv[2 * i + 1]);
+          const float2 h = __bfloat1622float2(chi[i]);
+          clo[i] = __floats2bfloat162_rn(cv[2 * i] - h.x, cv[2 * i + 1] - h.y);
+        }
+      }
       uint8_t* tile = sK + ks * C::K_BYTES + box * 16384;
 #pragma unroll 4
       for (int m = 0; m < CPR; ++m) {
         uint4* ptr = reinterpret_cast<uint4*>(tile + (row0 + m * RSTEP) * 128 + phys);
-        *ptr = scale_chunk(*ptr, cv);
+        *ptr = scale_chunk(*ptr, chi, clo);
       }
       fence_proxy_async_smem();
       mbar_arrive(&kready[ks]);
@@ -521,7 +531,8 @@ __global__ void __launch_bounds__(512, 1)
 
 template <int KD, int VD, bool HAS_GS>
 cudaError_t tc_impl(const FwdArgs& a, const FwdWork& w, const CUtensorMap& tmQ,
-                    const CUtensorMap& tmK, const CUtensorMap& tmV, cudaStream_t st) {
+                    const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmKX,
+                    cudaStream_t st) {
   using C = TcCfg<KD, VD>;
   auto kern = wall_fwd_tc_kernel<KD, VD, HAS_GS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -547,19 +558,20 @@ cudaError_t tc_impl(const FwdArgs& a, const FwdWork& w, const CUtensorMap& tmQ,
   p.wait_ns = a.wait_ns;
   p.fault = a.fault;
   const unsigned grid = static_cast<unsigned>((a.NB + 1) / 2) * a.B * a.HQ;
-  kern<<<grid, 512, C::SMEM_ALLOC, st>>>(tmQ, tmK, tmV, p);
+  kern<<<grid, 512, C::SMEM_ALLOC, st>>>(tmQ, tmK, tmV, tmKX, p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_fwd_tc(const FwdArgs& a, const FwdWork& w, const CUtensorMap& tmQ,
-                          const CUtensorMap& tmK, const CUtensorMap& tmV, cudaStream_t st) {
+                          const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmKX,
+                          cudaStream_t st) {
   const bool gs = a.g_scalar != nullptr;
 #define WALL_TC(KD_, VD_)                                                      \
   if (a.K == KD_ && a.V == VD_)                                                \
-    return gs ? tc_impl<KD_, VD_, true>(a, w, tmQ, tmK, tmV, st)               \
-              : tc_impl<KD_, VD_, false>(a, w, tmQ, tmK, tmV, st);
+    return gs ? tc_impl<KD_, VD_, true>(a, w, tmQ, tmK, tmV, tmKX, st)         \
+              : tc_impl<KD_, VD_, false>(a, w, tmQ, tmK, tmV, tmKX, st);
   WALL_TC(64, 64)
   WALL_TC(64, 128)
   WALL_TC(128, 64)

@@ -30,6 +30,8 @@ bool encode_tiled(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void
 //   ssl     [B*HQ][NB*128] minus the block-local inclusive prefix of g_scalar * log2(e)
 //   ssb     [B*HQ][NB]     block sum of g_scalar * log2(e)
 //   ssa     [B*HQ][NB][4]  prefix of g_scalar * log2(e) before the block ([0] used)
+//   kx      [B*HQ][T][16]  bf16 key-side gate channels for the QK contraction:
+//           (hi, lo, 0, ..., 0) with hi + lo = ssl[t] / (scale * log2(e)), bf16 head/tail
 //   rowlo   [T]            first admitted key per row (packed documents only)
 struct FwdWork {
   void* qh;
@@ -40,6 +42,7 @@ struct FwdWork {
   float* ssl;
   float* ssb;
   float* ssa;
+  void* kx;
   int* rowlo;
 };
 
@@ -66,7 +69,8 @@ size_t fwd_workspace_layout(int B, int T, int HQ, int K, bool bf16, FwdWork* w, 
 
 cudaError_t launch_prep(const FwdArgs& a, const FwdWork& w, bool bf16, cudaStream_t st);
 cudaError_t launch_fwd_tc(const FwdArgs& a, const FwdWork& w, const CUtensorMap& tmQ,
-                          const CUtensorMap& tmK, const CUtensorMap& tmV, cudaStream_t st);
+                          const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmKX,
+                          cudaStream_t st);
 cudaError_t launch_fwd_simt(const FwdArgs& a, const FwdWork& w, cudaStream_t st);
 
 struct CacheArgs {

@@ -28,7 +28,8 @@ __global__ void __launch_bounds__(256) prep_local_kernel(
     const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ g,
     const Tin* __restrict__ gs, const int32_t* __restrict__ cu, int nseq, int window, int T,
     int HQ, int H, int NB, Tin* __restrict__ qh, Tin* __restrict__ kh, float* __restrict__ bsum,
-    float* __restrict__ ssl, float* __restrict__ ssb, int* __restrict__ rowlo) {
+    float* __restrict__ ssl, float* __restrict__ ssb, __nv_bfloat16* __restrict__ kx,
+    float inv_scale, int* __restrict__ rowlo) {
   constexpr int CG = KD / 8;
   constexpr int RG = 128 / CG;
   constexpr int RPG = 128 / RG;
@@ -118,6 +119,22 @@ __global__ void __launch_bounds__(256) prep_local_kernel(
       ssl[static_cast<size_t>(bh) * NB * kBlockRows + blk * kBlockRows + tid] = -x;  // negated
       if (tid == kBlockRows - 1) ssb[static_cast<size_t>(bh) * NB + blk] = x;
     }
+    // Key-side gate term as two extra bf16 channels of the key operand (the
+    // query operand carries ones there), so the QK contraction adds it: the
+    // attention kernel scales S by scale * log2(e), so hi + lo = -x / (scale *
+    // log2(e)) to ~16 significant bits.
+    if (kx != nullptr && t < T) {
+      const float val = -x * inv_scale;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(val);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(val - __bfloat162float(hi));
+      uint4 u;
+      u.x = static_cast<uint32_t>(__bfloat16_as_ushort(hi)) |
+            (static_cast<uint32_t>(__bfloat16_as_ushort(lo)) << 16);
+      u.y = u.z = u.w = 0u;
+      uint4* dst = reinterpret_cast<uint4*>(kx + (static_cast<size_t>(bh) * T + t) * 16);
+      dst[0] = u;
+      dst[1] = make_uint4(0u, 0u, 0u, 0u);
+    }
   }
 
   // First admitted key of each row for packed documents (shared by all heads).
@@ -174,7 +191,9 @@ cudaError_t prep_impl(const FwdArgs& a, const FwdWork& w, cudaStream_t st) {
   prep_local_kernel<Tin, KD><<<grid, 256, 0, st>>>(
       static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.g),
       static_cast<const Tin*>(a.g_scalar), a.cu_seqlens, a.num_seqs, a.window, a.T, a.HQ, a.H,
-      a.NB, static_cast<Tin*>(w.qh), static_cast<Tin*>(w.kh), w.bsum, w.ssl, w.ssb, w.rowlo);
+      a.NB, static_cast<Tin*>(w.qh), static_cast<Tin*>(w.kh), w.bsum, w.ssl, w.ssb,
+      sizeof(Tin) == 2 ? static_cast<__nv_bfloat16*>(w.kx) : nullptr, 1.f / (a.scale * kLog2e),
+      w.rowlo);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   prep_scan_kernel<KD><<<BHQ, KD + 32, 0, st>>>(w.bsum, a.g_scalar ? w.ssb : nullptr, a.NB, w.AQ,
@@ -213,6 +232,7 @@ size_t fwd_workspace_layout(int B, int T, int HQ, int K, bool bf16, FwdWork* w, 
   p->ssl = static_cast<float*>(take(BHQ * NB * kBlockRows * 4));
   p->ssb = static_cast<float*>(take(BHQ * NB * 4));
   p->ssa = static_cast<float*>(take(BHQ * NB * 16));
+  p->kx = take(BHQ * static_cast<size_t>(T) * 16 * 2);
   p->rowlo = static_cast<int*>(take(static_cast<size_t>(T) * 4 + 16));
   return off;
 }
