@@ -49,11 +49,11 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # hash of the kernel source it was taken on; reported as null once the kernel
 # source changes.  Filled from profiles/ after each capture.
 TRAFFIC = {
-    # profiles/wall_fwd_tc_long_prefill.md: 428.170496 MB read + 58.283776 MB written
-    "prefill_main": {"bytes": 486454272, "source_sha": "3d917672a9a73f4d"},
+    # profiles/wall_fwd_tc_long_prefill.md: 315.239680 MB read + 43.282432 MB written
+    "prefill_main": {"bytes": 358522112, "source_sha": "71f6c2251b5462ea"},
     # profiles/decode_split_b4_tkv32k.md, batch 4 scaled by 8 to batch 32 (traffic is
-    # proportional to the batch): (1.375986 GB + 5.748480 MB) * 8
-    "decode_split": {"bytes": 11053875840, "source_sha": "609266ee7d00583d"},
+    # proportional to the batch): (1.376493 GB + 5.271552 MB) * 8
+    "decode_split": {"bytes": 11054116416, "source_sha": "1660d8d5e042ca50"},
 }
 KERNEL_SOURCES = {
     "prefill_main": "decayed_softmax_attention_b200/csrc/wall_fwd_tc.cu",
@@ -344,10 +344,12 @@ def run_ours(args, world, rank, local):
         dlse = torch.empty((dspec.B, 1, dspec.HQ), dtype=torch.float32, device=dev)
         p_prefix = torch.empty_like(cache.p)
         e0, e1 = ev(), ev()
+        cache.length = 0
+        cache.append(k_pre, g_pre)     # first launch loads the kernel module: untimed
         torch.cuda.synchronize()
         e0.record()
         cache.length = 0
-        cache.append(k_pre, g_pre)
+        cache.append(k_pre, g_pre)     # timed rebuild (writes the same values)
         e1.record()
         torch.cuda.synchronize()
         build_ms = e0.elapsed_time(e1)
