@@ -59,100 +59,132 @@ __device__ __forceinline__ void store1(__nv_bfloat16* p, float x) { *p = __float
 __device__ __forceinline__ void store1(float* p, float x) { *p = x; }
 
 // ----------------------------------------------------------------- cache build / append
-// One CTA per (batch, query head) walks the new rows chunk by chunk, carrying
-// the running prefix P.  Thread layout per chunk: CG channel groups of 8 x RG
-// row groups of RPG rows.
-template <typename T, int KD, int RPG>
-__global__ void __launch_bounds__(256) cache_build_kernel(
+// The prefix P runs along time, so each (batch, query head) sequence is walked
+// in order by TPS = K/4 threads, each owning four channels for the whole walk:
+// the prefix is a running sum in registers, with no exchange between threads.
+// A warp covers one sequence (K = 128) or two (K = 64); a CTA holds SPC
+// sequences.  Rows are fetched D at a time into two register buffers, so the
+// loads of the next D rows are in flight while the current ones are scanned.
+//
+// Precision: the running sum is kept as carry (P at the end of the previous
+// chunk) + loc (sum inside the current chunk), so exp2(R_c - P[j]) is taken
+// from chunk-local values only; anchors are stored as carry + loc.
+template <typename T>
+struct Vec4;  // four consecutive channels
+template <>
+struct Vec4<__nv_bfloat16> {
+  uint2 u;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = *reinterpret_cast<const uint2*>(p); }
+  __device__ __forceinline__ void get(float* f) const {
+    f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x); f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
+  }
+  __device__ __forceinline__ static void store(__nv_bfloat16* p, const float* f) {
+    *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]));
+  }
+};
+template <>
+struct Vec4<float> {
+  float4 u;
+  __device__ __forceinline__ void load(const float* p) { u = *reinterpret_cast<const float4*>(p); }
+  __device__ __forceinline__ void get(float* f) const { f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w; }
+  __device__ __forceinline__ static void store(float* p, const float* f) {
+    *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
+  }
+};
+
+template <typename T, int KD>
+struct CacheCfg {
+  static constexpr int TPS = KD / 4;                   // threads per sequence
+  static constexpr int SPC = 128 / TPS;                // sequences per CTA
+  static constexpr int D = sizeof(T) == 2 ? 16 : 8;    // rows per register buffer
+};
+
+template <typename T, int KD>
+__global__ void __launch_bounds__(128) cache_build_kernel(
     const T* __restrict__ k_new, const T* __restrict__ g_new, const float* __restrict__ p_prev,
-    int t_start, int T_new, int cap, int HQ, int H, T* __restrict__ k_tilde,
+    int BHQ, int t_start, int T_new, int cap, int HQ, int H, int C, T* __restrict__ k_tilde,
     float* __restrict__ r_cache, float* __restrict__ p_last) {
-  constexpr int CG = KD / 8;
-  constexpr int RG = 256 / CG;
-  constexpr int C = RG * RPG;
-  __shared__ float tot[2][RG][KD];
-  __shared__ float rloc[2][KD];
-
-  const int bh = blockIdx.x;
+  using CC = CacheCfg<T, KD>;
+  constexpr int D = CC::D;
+  const int bh = static_cast<int>(blockIdx.x) * CC::SPC + static_cast<int>(threadIdx.x) / CC::TPS;
+  if (bh >= BHQ) return;
+  const int ch = (static_cast<int>(threadIdx.x) % CC::TPS) * 4;
   const int b = bh / HQ, hq = bh % HQ, kvh = hq / (HQ / H);
-  const int tid = threadIdx.x, cg = tid % CG, rg = tid / CG;
-  const int ch = cg * 8;
   const int ncap = (cap + C - 1) / C;
-  const int t_end = t_start + T_new;
+  const size_t gstep = static_cast<size_t>(HQ) * KD, kstep = static_cast<size_t>(H) * KD;
+  const T* gp = g_new + (static_cast<size_t>(b) * T_new * HQ + hq) * KD + ch;
+  const T* kp = k_new + (static_cast<size_t>(b) * T_new * H + kvh) * KD + ch;
+  T* op = k_tilde + ((static_cast<size_t>(b) * cap + t_start) * HQ + hq) * KD + ch;
+  float* rp = r_cache + (static_cast<size_t>(b) * ncap * HQ + hq) * KD + ch;  // + chunk * gstep
+  const size_t rstep = gstep;
 
-  float carry[8];
+  float carry[4], loc[4], r0[4];
 #pragma unroll
-  for (int c = 0; c < 8; ++c)
+  for (int c = 0; c < 4; ++c) {
     carry[c] = p_prev ? p_prev[static_cast<size_t>(bh) * KD + ch + c] : 0.f;
+    loc[c] = 0.f;
+    r0[c] = 0.f;
+  }
+  if (t_start % C != 0) {
+    // the chunk holding t_start was anchored by an earlier call
+    const float* rr = rp + static_cast<size_t>(t_start / C) * rstep;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) r0[c] = rr[c] - carry[c];
+  }
 
-  int buf = 0;
-  for (int c0 = (t_start / C) * C; c0 < t_end; c0 += C, buf ^= 1) {
-    const int chunk = c0 / C;
-    const bool fresh = c0 >= t_start;  // this call writes the chunk's anchor
-    float acc[8], loc[RPG][8];
+  Vec4<T> gA[D], kA[D], gB[D], kB[D];
+  auto fetch = [&](Vec4<T>* gb, Vec4<T>* kb, int t0) {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-#pragma unroll
-    for (int m = 0; m < RPG; ++m) {
-      const int t = c0 + rg * RPG + m;
-      if (t >= t_start && t < t_end) {
-        float f[8];
-        load8(g_new + ((static_cast<size_t>(b) * T_new + (t - t_start)) * HQ + hq) * KD + ch, f);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[c] += f[c] * kLog2e;
-      }
-#pragma unroll
-      for (int c = 0; c < 8; ++c) loc[m][c] = acc[c];
-    }
-#pragma unroll
-    for (int c = 0; c < 8; ++c) tot[buf][rg][ch + c] = acc[c];
-    if (fresh && rg == 0) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) rloc[buf][ch + c] = loc[0][c];
-    }
-    __syncthreads();
-    float pre[8], total[8], R[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      float a = 0.f, all = 0.f;
-      for (int r = 0; r < RG; ++r) {
-        const float x = tot[buf][r][ch + c];
-        all += x;
-        if (r < rg) a += x;
-      }
-      pre[c] = a;
-      total[c] = all;
-    }
-    float* rrow = r_cache + ((static_cast<size_t>(b) * ncap + chunk) * HQ + hq) * KD + ch;
-    if (fresh) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) R[c] = rloc[buf][ch + c];  // local to this chunk's start
-      if (rg == 0) {
-#pragma unroll
-        for (int c = 0; c < 8; ++c) rrow[c] = carry[c] + R[c];
-      }
-    } else {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) R[c] = rrow[c] - carry[c];  // anchor written by an earlier call
-    }
-#pragma unroll
-    for (int m = 0; m < RPG; ++m) {
-      const int t = c0 + rg * RPG + m;
-      if (t >= t_start && t < t_end) {
-        float kf[8];
-        load8(k_new + ((static_cast<size_t>(b) * T_new + (t - t_start)) * H + kvh) * KD + ch, kf);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) kf[c] *= exp2f(R[c] - (pre[c] + loc[m][c]));
-        store8(k_tilde + ((static_cast<size_t>(b) * cap + t) * HQ + hq) * KD + ch, kf);
+    for (int i = 0; i < D; ++i) {
+      if (t0 + i < T_new) {
+        gb[i].load(gp + static_cast<size_t>(t0 + i) * gstep);
+        kb[i].load(kp + static_cast<size_t>(t0 + i) * kstep);
       }
     }
+  };
+  auto scan = [&](const Vec4<T>* gb, const Vec4<T>* kb, int t0) {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) carry[c] += total[c];
+    for (int i = 0; i < D; ++i) {
+      const int t = t0 + i;
+      if (t < T_new) {
+        const int ta = t_start + t;
+        const bool head = (ta % C) == 0;  // first row of a chunk: this call anchors it
+        float g[4], k[4];
+        gb[i].get(g);
+        kb[i].get(k);
+        if (head) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            carry[c] += loc[c];
+            loc[c] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) loc[c] = fmaf(g[c], kLog2e, loc[c]);
+        if (head) {
+          float* rr = rp + static_cast<size_t>(ta / C) * rstep;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) r0[c] = loc[c];
+          *reinterpret_cast<float4*>(rr) =
+              make_float4(carry[0] + loc[0], carry[1] + loc[1], carry[2] + loc[2], carry[3] + loc[3]);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) k[c] *= ex2_approx(r0[c] - loc[c]);
+        Vec4<T>::store(op + static_cast<size_t>(t) * gstep, k);
+      }
+    }
+  };
+
+  fetch(gA, kA, 0);
+  for (int t0 = 0; t0 < T_new; t0 += 2 * D) {
+    if (t0 + D < T_new) fetch(gB, kB, t0 + D);
+    scan(gA, kA, t0);
+    if (t0 + D >= T_new) break;
+    if (t0 + 2 * D < T_new) fetch(gA, kA, t0 + 2 * D);
+    scan(gB, kB, t0 + D);
   }
-  if (rg == 0) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) p_last[static_cast<size_t>(bh) * KD + ch + c] = carry[c];
-  }
+  *reinterpret_cast<float4*>(p_last + static_cast<size_t>(bh) * KD + ch) =
+      make_float4(carry[0] + loc[0], carry[1] + loc[1], carry[2] + loc[2], carry[3] + loc[3]);
 }
 
 // ----------------------------------------------------------------- split-KV decode
@@ -402,25 +434,15 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
   if (lse != nullptr && lane == 0) lse[bhq] = (M + log2f(Z)) * kLn2;
 }
 
-template <typename T, int KD, int RPG>
-cudaError_t cache_impl(const CacheArgs& a, cudaStream_t st) {
-  cache_build_kernel<T, KD, RPG><<<a.B * a.HQ, 256, 0, st>>>(
-      static_cast<const T*>(a.k_new), static_cast<const T*>(a.g_new), a.p_prev, a.t_start,
-      a.T_new, a.cap, a.HQ, a.H, static_cast<T*>(a.k_tilde), a.r_cache, a.p_last);
-  return cudaGetLastError();
-}
-
 template <typename T, int KD>
-cudaError_t cache_dispatch(const CacheArgs& a, cudaStream_t st) {
-  constexpr int RG = 256 / (KD / 8);
-  const int rpg = a.chunk / RG;
-  switch (rpg) {
-    case 1: return cache_impl<T, KD, 1>(a, st);
-    case 2: return cache_impl<T, KD, 2>(a, st);
-    case 4: return cache_impl<T, KD, 4>(a, st);
-    case 8: return cache_impl<T, KD, 8>(a, st);
-    default: return cudaErrorInvalidValue;
-  }
+cudaError_t cache_impl(const CacheArgs& a, cudaStream_t st) {
+  using CC = CacheCfg<T, KD>;
+  const int BHQ = a.B * a.HQ;
+  const unsigned grid = static_cast<unsigned>((BHQ + CC::SPC - 1) / CC::SPC);
+  cache_build_kernel<T, KD><<<grid, 128, 0, st>>>(
+      static_cast<const T*>(a.k_new), static_cast<const T*>(a.g_new), a.p_prev, BHQ, a.t_start,
+      a.T_new, a.cap, a.HQ, a.H, a.chunk, static_cast<T*>(a.k_tilde), a.r_cache, a.p_last);
+  return cudaGetLastError();
 }
 
 template <typename T, int KD, int VD, int G>
@@ -492,8 +514,8 @@ cudaError_t decode_by_dims(const DecodeArgs& a, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_cache_build(const CacheArgs& a, bool bf16, cudaStream_t st) {
-  if (bf16) return a.K == 64 ? cache_dispatch<__nv_bfloat16, 64>(a, st) : cache_dispatch<__nv_bfloat16, 128>(a, st);
-  return a.K == 64 ? cache_dispatch<float, 64>(a, st) : cache_dispatch<float, 128>(a, st);
+  if (bf16) return a.K == 64 ? cache_impl<__nv_bfloat16, 64>(a, st) : cache_impl<__nv_bfloat16, 128>(a, st);
+  return a.K == 64 ? cache_impl<float, 64>(a, st) : cache_impl<float, 128>(a, st);
 }
 
 bool decode_supported(int K, int V, int group) {
