@@ -227,6 +227,9 @@ wall_status_t wall_build_kv_cache(const void* k_new, const void* g_new, const fl
   a.k_new = k_new; a.g_new = g_new; a.p_prev = p_prev;
   a.B = B; a.t_start = t_start; a.T_new = T_new; a.cap = cap; a.HQ = HQ; a.H = H; a.K = K;
   a.chunk = chunk; a.k_tilde = k_tilde; a.r_cache = r_cache; a.p_last = p_last;
+  a.err = wall::device_error_word();
+  if (a.err == nullptr) return WALL_ERR_CUDA;
+  a.wait_ns = wall::wait_limit_ns();
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   return finish(wall::launch_cache_build(a, dt == WALL_DTYPE_BF16, st), st);
 }

@@ -81,6 +81,8 @@ struct CacheArgs {
   void* k_tilde;
   float* r_cache;
   float* p_last;
+  int* err;          // device error word (bounded waits)
+  uint64_t wait_ns;  // limit of each bounded wait
 };
 cudaError_t launch_cache_build(const CacheArgs& a, bool bf16, cudaStream_t st);
 
