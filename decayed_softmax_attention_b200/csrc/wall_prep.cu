@@ -24,7 +24,7 @@ namespace {
 // row); query operands per 256-row block (AQ = G just before the block), so
 // the two 128-row query tiles of one prefill CTA share one anchor.
 template <typename Tin, int KD>
-__global__ void __launch_bounds__(256) prep_local_kernel(
+__global__ void __launch_bounds__(256, 3) prep_local_kernel(
     const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ g,
     const Tin* __restrict__ gs, const int32_t* __restrict__ cu, int nseq, int window, int T,
     int HQ, int H, int NB, Tin* __restrict__ qh, Tin* __restrict__ kh, float* __restrict__ bsum,
@@ -49,13 +49,25 @@ __global__ void __launch_bounds__(256) prep_local_kernel(
   float acc[8];
 #pragma unroll
   for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-  for (int m = 0; m < RPG; ++m) {
-    const int t = t0 + m;
-    if (t >= T) break;
-    float f[8];
-    load8(gb + static_cast<size_t>(t) * qrow, f);
+  // Loads of U1 (U2) rows are issued before any is used, so each thread keeps
+  // several rows in flight.
+  constexpr int U1 = sizeof(Tin) == 2 ? 8 : 2;
+  constexpr int U2 = sizeof(Tin) == 2 ? 2 : 1;
+  static_assert(RPG % U1 == 0 && RPG % U2 == 0, "row batch must divide the rows per thread");
+  for (int m0 = 0; m0 < RPG; m0 += U1) {
+    Raw8<Tin> rg[U1];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) acc[c] += f[c];
+    for (int u = 0; u < U1; ++u)
+      if (t0 + m0 + u < T) rg[u].load(gb + static_cast<size_t>(t0 + m0 + u) * qrow);
+#pragma unroll
+    for (int u = 0; u < U1; ++u) {
+      if (t0 + m0 + u < T) {
+        float f[8];
+        rg[u].get(f);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] += f[c];
+      }
+    }
   }
 #pragma unroll
   for (int c = 0; c < 8; ++c) tot[half][rg][cg * 8 + c] = acc[c];
@@ -85,21 +97,35 @@ __global__ void __launch_bounds__(256) prep_local_kernel(
   const Tin* kb = k + (static_cast<size_t>(b) * T) * krow + static_cast<size_t>(kvh) * KD + cg * 8;
   Tin* qo = qh + static_cast<size_t>(bh) * T * KD + cg * 8;
   Tin* ko = kh + static_cast<size_t>(bh) * T * KD + cg * 8;
-  for (int m = 0; m < RPG; ++m) {
-    const int t = t0 + m;
-    if (t >= T) break;
-    float f[8], x[8], y[8];
-    load8(gb + static_cast<size_t>(t) * qrow, f);
-    load8(qb + static_cast<size_t>(t) * qrow, x);
-    load8(kb + static_cast<size_t>(t) * krow, y);
+  for (int m0 = 0; m0 < RPG; m0 += U2) {
+    Raw8<Tin> rg[U2], rq[U2], rk[U2];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      run[c] += f[c];
-      x[c] *= expf(qoff[c] + run[c]);
-      y[c] *= expf(total[c] - run[c]);
+    for (int u = 0; u < U2; ++u) {
+      const int t = t0 + m0 + u;
+      if (t < T) {
+        rg[u].load(gb + static_cast<size_t>(t) * qrow);
+        rq[u].load(qb + static_cast<size_t>(t) * qrow);
+        rk[u].load(kb + static_cast<size_t>(t) * krow);
+      }
     }
-    store8(qo + static_cast<size_t>(t) * KD, x);
-    store8(ko + static_cast<size_t>(t) * KD, y);
+#pragma unroll
+    for (int u = 0; u < U2; ++u) {
+      const int t = t0 + m0 + u;
+      if (t < T) {
+        float f[8], x[8], y[8];
+        rg[u].get(f);
+        rq[u].get(x);
+        rk[u].get(y);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          run[c] += f[c];
+          x[c] *= expf(qoff[c] + run[c]);
+          y[c] *= expf(total[c] - run[c]);
+        }
+        store8(qo + static_cast<size_t>(t) * KD, x);
+        store8(ko + static_cast<size_t>(t) * KD, y);
+      }
+    }
   }
 
   // Scalar gate: negated 128-block-local inclusive prefix (log2 units), one row per thread.
