@@ -49,15 +49,19 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # hash of the kernel source it was taken on; reported as null once the kernel
 # source changes.  Filled from profiles/ after each capture.
 TRAFFIC = {
-    # profiles/wall_fwd_tc_long_prefill.md: 315.239680 MB read + 43.282432 MB written
-    "prefill_main": {"bytes": 358522112, "source_sha": "71f6c2251b5462ea"},
+    # profiles/wall_fwd_tc_long_prefill.md: 316.535808 MB read + 43.428608 MB written
+    "prefill_main": {"bytes": 359964416, "source_sha": "820590f83f572f63"},
     # profiles/decode_split_b4_tkv32k.md, batch 4 scaled by 8 to batch 32 (traffic is
     # proportional to the batch): (1.376493 GB + 5.271552 MB) * 8
     "decode_split": {"bytes": 11054116416, "source_sha": "1660d8d5e042ca50"},
+    # profiles/cache_build_b4_t32k.md, batch 4 scaled by 8 to batch 32:
+    # (1.342212 GB + 1.070139 GB) * 8
+    "cache_build": {"bytes": 19298808000, "source_sha": "c4f6efa03b7cc36b"},
 }
 KERNEL_SOURCES = {
     "prefill_main": "decayed_softmax_attention_b200/csrc/wall_fwd_tc.cu",
     "decode_split": "decayed_softmax_attention_b200/csrc/wall_decode.cu",
+    "cache_build": "decayed_softmax_attention_b200/csrc/wall_cache.cu",
 }
 
 
@@ -478,8 +482,15 @@ def run_ours(args, world, rank, local):
                          "share_of_step": sum(sum(r) for r in dec_split_ms) / total_ms},
             "frac_of_hbm_incl_combine": dec_value / world / hbm_peak,
         }
+        build_gbps = build_bytes / (build_ms * 1e-3) / 1e9
         side.update({"cache_build_prefix_ms": build_ms,
-                     "cache_build_prefix_GBps": build_bytes / (build_ms * 1e-3) / 1e9})
+                     "cache_build_prefix_GBps": build_gbps,
+                     "cache_build_roofline": {
+                         "kernel": "cache_build_kernel", "bound": "hbm", "achieved": build_gbps,
+                         "peak": hbm_peak, "unit": "GB/s", "frac": build_gbps / hbm_peak,
+                         "algorithmic_bytes_per_launch": build_bytes,
+                         "traffic": (traffic_for("cache_build")
+                                     if dspec.B == 32 and T0 == 32768 else None)}})
         if not do_prefill:
             line["metric"] = line["decode"]["metric"]
             line["value"], line["unit"] = dec_value, "GB/s"

@@ -23,7 +23,9 @@
 // rescale 48 (sum 512 per thread slot = the 65536 registers of the launch).
 //
 // MMA issue order per key tile j: PV_A(j-1), QK_A(j), PV_B(j-1), QK_B(j), so
-// one softmax warpgroup works while the tensor core serves the other, and
+// one softmax warpgroup works while the tensor core serves the other (the
+// rescaled key tile is waited for before PV_A(j-1), so PV_A and QK_A issue back
+// to back: the MMA issue queue is only a few instructions deep), and
 // "S_X(j) complete" implies "PV_X(j-1) complete" (tcgen05 ops of one thread
 // run in issue order): a softmax warpgroup may rescale O_X as soon as it has
 // read S_X(j).  Key tiles are visited from the diagonal backwards so the row
@@ -279,48 +281,56 @@ __global__ void __launch_bounds__(512, 1)
       // ----------------------------------------------------------- MMA issuer
       bool ok = mbar_wait(qfull, 0, wc);
       tc_fence_after();
-      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+      // Descriptors of every operand stage, built once: a K step only adds a
+      // constant to the start-address field, so each MMA costs one add per operand.
+      const uint64_t dQ0 = sw128_desc(smem_u32(sQ), 16, 1024);
+      const uint64_t dK0 = sw128_desc(smem_u32(sK), 16, 1024);
+      const uint64_t dV0 = sw128_desc(smem_u32(sV), 16384, 1024);
+      const uint64_t dQX = HAS_GS ? sw32_desc(smem_u32(sQX), 256) : 0;
+      const uint64_t dKX0 = HAS_GS ? sw32_desc(smem_u32(sKX), 256) : 0;
       // Only the previous key tile's P*V products can be pending at tile j.
       bool pendA = false, pendB = false;
+      bool vseen = false;  // V stage of the previous tile already waited for
       int vrem_prev = 0;  // P*V reads still to issue for the previous tile's V stage
       auto issue_pv = [&](int x, int jj) -> bool {
         const int cnt = jj - (x == 0 ? jfA : jfB), vs = jj % C::VS;
         if (!mbar_wait(&pfull[x], cnt & 1, wc)) return false;
-        if (!mbar_wait(&vfull[vs], (jj / C::VS) & 1, wc)) return false;
+        if ((x == 0 || !vseen) && !mbar_wait(&vfull[vs], (jj / C::VS) & 1, wc)) return false;
+        vseen = true;
         tc_fence_after();
+        const uint64_t dV = dV0 + static_cast<uint64_t>(vs * (C::V_BYTES >> 4));
+        const uint32_t dO = tmem_base + C::COL_O + 128 * x, aP = tmem_base + C::COL_S + 128 * x;
+        umma_ts(dO, aP, dV, C::IDESC_PV, cnt > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk) {
-          const uint64_t bdesc = sw128_desc(sVa + vs * C::V_BYTES + kk * 2048, 16384, 1024);
-          umma_ts(tmem_base + C::COL_O + 128 * x, tmem_base + C::COL_S + 128 * x + kk * 8, bdesc,
-                  C::IDESC_PV, (cnt > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 1; kk < C::BN / 16; ++kk)
+          umma_ts(dO, aP + kk * 8, dV + static_cast<uint64_t>((kk * 2048) >> 4), C::IDESC_PV, 1u);
         if (--vrem_prev == 0) umma_commit(&vempty[vs]);
         return true;
       };
       auto issue_qk = [&](int x, int j, int ks) {
         const uint32_t dS = tmem_base + C::COL_S + 128 * x;
+        const uint64_t dA = dQ0 + static_cast<uint64_t>(x * (C::Q_BYTES >> 4));
+        const uint64_t dB = dK0 + static_cast<uint64_t>(ks * (C::K_BYTES >> 4));
 #pragma unroll
         for (int kk = 0; kk < KD / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint64_t adesc = sw128_desc(sQa + x * C::Q_BYTES + koff, 16, 1024);
-          const uint64_t bdesc = sw128_desc(sKa + ks * C::K_BYTES + koff, 16, 1024);
-          umma_ss(dS, adesc, bdesc, C::IDESC_QK, kk > 0 ? 1u : 0u);
+          const uint64_t koff = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+          umma_ss(dS, dA + koff, dB + koff, C::IDESC_QK, kk > 0 ? 1u : 0u);
         }
         if (HAS_GS) {
           // + key-side gate term: (1, 1, 0..) x (hi, lo, 0..) over one more K slice
-          const uint32_t qx = smem_u32(sQX), kx = smem_u32(sKX + ks * C::GX_BYTES);
-          umma_ss(dS, sw32_desc(qx, 256), sw32_desc(kx, 256), C::IDESC_QK, 1u);
+          umma_ss(dS, dQX, dKX0 + static_cast<uint64_t>(ks * (C::GX_BYTES >> 4)), C::IDESC_QK, 1u);
         }
         umma_commit(&sfull[x]);
       };
       for (int j = 0; ok && j < nt; ++j) {
         const int ks = j % C::KS;
         int vrem_cur = 0;
+        vseen = false;
+        if (!mbar_wait(&kready[ks], (j / C::KS) & 1, wc)) { ok = false; break; }
         if (pendA) {
           if (!issue_pv(0, j - 1)) { ok = false; break; }
           pendA = false;
         }
-        if (!mbar_wait(&kready[ks], (j / C::KS) & 1, wc)) { ok = false; break; }
         tc_fence_after();
         if (j >= jfA && j <= jlA) {
           issue_qk(0, j, ks);
