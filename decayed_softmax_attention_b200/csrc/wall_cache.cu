@@ -59,8 +59,8 @@ template <typename T, int KD>
 __global__ void __launch_bounds__(160) cache_build_kernel(
     const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmK,
     const float* __restrict__ p_prev, int t_start, int T_new, int cap, int HQ, int G, int HPC,
-    int NKV, int C, T* __restrict__ k_tilde, float* __restrict__ r_cache,
-    float* __restrict__ p_last, int* err, uint64_t wait_ns) {
+    int NKV, int C, int seg_first, int seg_rows, T* __restrict__ k_tilde,
+    float* __restrict__ r_cache, float* __restrict__ p_last, int* err, uint64_t wait_ns) {
   using CC = CacheCfg<T, KD>;
   constexpr int D = CC::D;
   extern __shared__ __align__(128) uint8_t csm[];
@@ -73,7 +73,13 @@ __global__ void __launch_bounds__(160) cache_build_kernel(
   const int nwc = (ncons + 31) / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hq0 = blockIdx.x * HPC, b = blockIdx.y;
-  const int nst = (T_new + D - 1) / D;
+  // Rows [rb, re) of this call (relative to t_start): all of them, or one
+  // chunk-aligned segment (blockIdx.z) whose starting prefix an earlier pass
+  // left in the anchor slot of its first chunk.
+  const bool segmented = seg_rows > 0;
+  const int rb = segmented ? seg_first + static_cast<int>(blockIdx.z) * seg_rows : 0;
+  const int re = segmented ? min(rb + seg_rows, T_new) : T_new;
+  const int nst = (re - rb + D - 1) / D;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < CC::NS; ++i) {
@@ -97,8 +103,8 @@ __global__ void __launch_bounds__(160) cache_build_kernel(
         if (i >= CC::NS && !mbar_wait(&empty[slot], ((i / CC::NS) - 1) & 1, wc)) break;
         uint8_t* st = csm + slot * stage;
         mbar_arrive_expect_tx(&full[slot], stage);
-        tma_load_4d(st, &tmG, &full[slot], 0, hq0, i * D, b);
-        tma_load_4d(st + gbytes, &tmK, &full[slot], 0, hq0 / G, i * D, b);
+        tma_load_4d(st, &tmG, &full[slot], 0, hq0, rb + i * D, b);
+        tma_load_4d(st + gbytes, &tmK, &full[slot], 0, hq0 / G, rb + i * D, b);
         issued = i + 1;
       }
       for (int i = issued > CC::NS ? issued - CC::NS : 0; i < issued; ++i)
@@ -122,11 +128,20 @@ __global__ void __launch_bounds__(160) cache_build_kernel(
   float carry[4], loc[4], r0[4];
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
-    carry[c] = (active && p_prev) ? p_prev[bh * KD + ch + c] : 0.f;
+    carry[c] = (active && p_prev && !segmented) ? p_prev[bh * KD + ch + c] : 0.f;
     loc[c] = 0.f;
     r0[c] = 0.f;
   }
-  if (active && t_start % C != 0) {
+  if (active && segmented) {
+    // P just before the segment (read before this thread overwrites the slot
+    // with the chunk's anchor at the segment's first row)
+    const float4 c4 = *reinterpret_cast<const float4*>(
+        rp + static_cast<size_t>((t_start + rb) / C) * hstep);
+    carry[0] = c4.x;
+    carry[1] = c4.y;
+    carry[2] = c4.z;
+    carry[3] = c4.w;
+  } else if (active && t_start % C != 0) {
     // the chunk holding t_start was anchored by an earlier call
     const float* rr = rp + static_cast<size_t>(t_start / C) * hstep;
 #pragma unroll
@@ -176,11 +191,11 @@ __global__ void __launch_bounds__(160) cache_build_kernel(
     const T* sg = reinterpret_cast<const T*>(st) + hl * KD + ch;
     const T* sk = reinterpret_cast<const T*>(st + gbytes) + kl * KD + ch;
     if (active) {
-      const int t0 = i * D;
+      const int t0 = rb + i * D;
       const int ta0 = t_start + t0;
       const int hr = (C - (ta0 & cmask)) & cmask;  // stage row that opens a chunk (>= D: none)
       T* ob = op + static_cast<size_t>(t0) * hstep;
-      if (t0 + D <= T_new) {
+      if (t0 + D <= re) {
 #pragma unroll
         for (int r = 0; r < D; ++r) {
           row(sg, sk, ob, r == hr, ta0 + r);
@@ -189,7 +204,7 @@ __global__ void __launch_bounds__(160) cache_build_kernel(
           ob += hstep;
         }
       } else {
-        for (int r = 0; r < T_new - t0; ++r) {
+        for (int r = 0; r < re - t0; ++r) {
           row(sg, sk, ob, r == hr, ta0 + r);
           sg += gstr;
           sk += kstr;
@@ -200,9 +215,98 @@ __global__ void __launch_bounds__(160) cache_build_kernel(
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);
   }
-  if (ok && active)
+  if (ok && active && !segmented)
     *reinterpret_cast<float4*>(p_last + bh * KD + ch) =
         make_float4(carry[0] + loc[0], carry[1] + loc[1], carry[2] + loc[2], carry[3] + loc[3]);
+}
+
+__device__ __forceinline__ void store_one(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
+__device__ __forceinline__ void store_one(float* p, float x) { *p = x; }
+
+// Segmented build, pass 1 (when B * HQ / HPC CTAs cannot fill the GPU): for
+// every (batch, query head, chunk-aligned segment) the channel sums of g over
+// the segment (log2 units, summed chunk by chunk like the walk's carry), kept
+// in the anchor slot of the segment's first chunk until pass 3 overwrites it.
+template <typename T, int KD>
+__global__ void __launch_bounds__(128) cache_segsum_kernel(
+    const T* __restrict__ g_new, int t_start, int T_new, int cap, int HQ, int HPC, int C,
+    int seg_first, int seg_rows, float* __restrict__ r_cache) {
+  using CC = CacheCfg<T, KD>;
+  constexpr int U = 8;  // rows whose loads are issued together
+  const int ct = threadIdx.x;
+  if (ct >= HPC * CC::TPS) return;
+  const int hl = ct / CC::TPS, ch = (ct % CC::TPS) * 4;
+  const int hq = static_cast<int>(blockIdx.x) * HPC + hl, b = blockIdx.y;
+  const int rb = seg_first + static_cast<int>(blockIdx.z) * seg_rows;
+  const int re = min(rb + seg_rows, T_new);
+  const size_t gstep = static_cast<size_t>(HQ) * KD;
+  const T* gp = g_new + (static_cast<size_t>(b) * T_new * HQ + hq) * KD + ch;
+  float tot[4] = {0.f, 0.f, 0.f, 0.f}, loc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int t0 = rb; t0 < re; t0 += U) {
+    Vec4<T> v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (t0 + u < re) v[u].load(gp + static_cast<size_t>(t0 + u) * gstep);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (t0 + u < re) {
+        if (((t_start + t0 + u) & (C - 1)) == 0) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            tot[c] += loc[c];
+            loc[c] = 0.f;
+          }
+        }
+        float g[4];
+        v[u].get(g);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) loc[c] = fmaf(g[c], kLog2e, loc[c]);
+      }
+    }
+  }
+  const int ncap = (cap + C - 1) / C;
+  float* rr = r_cache + ((static_cast<size_t>(b) * ncap + (t_start + rb) / C) * HQ + hq) * KD + ch;
+  *reinterpret_cast<float4*>(rr) =
+      make_float4(tot[0] + loc[0], tot[1] + loc[1], tot[2] + loc[2], tot[3] + loc[3]);
+}
+
+// Segmented build, pass 2: one thread per (batch, query head, channel).  The
+// rows of a partial first chunk (t_start inside a chunk anchored by an earlier
+// call) are rescaled here; then the segment sums become the prefix P just
+// before each segment (in place, in order), and the final P goes to p_last.
+template <typename T, int KD>
+__global__ void __launch_bounds__(128) cache_segscan_kernel(
+    const T* __restrict__ k_new, const T* __restrict__ g_new, const float* __restrict__ p_prev,
+    int B, int t_start, int T_new, int cap, int HQ, int H, int C, int seg_first, int seg_rows,
+    int nseg, T* __restrict__ k_tilde, float* __restrict__ r_cache, float* __restrict__ p_last) {
+  const long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<long>(B) * HQ * KD) return;
+  const int n = static_cast<int>(idx % KD);
+  const long bh = idx / KD;
+  const int b = static_cast<int>(bh / HQ), hq = static_cast<int>(bh % HQ), kvh = hq / (HQ / H);
+  const int ncap = (cap + C - 1) / C;
+  const size_t hstep = static_cast<size_t>(HQ) * KD;
+  float* rp = r_cache + (static_cast<size_t>(b) * ncap * HQ + hq) * KD + n;  // + chunk * hstep
+  float carry = p_prev ? p_prev[static_cast<size_t>(bh) * KD + n] : 0.f;
+  if (seg_first > 0) {
+    const float r0 = rp[static_cast<size_t>(t_start / C) * hstep] - carry;
+    float loc = 0.f;
+    for (int t = 0; t < seg_first; ++t) {
+      const size_t row = static_cast<size_t>(b) * T_new + t;
+      loc = fmaf(load1(g_new + (row * HQ + hq) * KD + n), kLog2e, loc);
+      const float kv = load1(k_new + (row * H + kvh) * KD + n);
+      store_one(k_tilde + ((static_cast<size_t>(b) * cap + t_start + t) * HQ + hq) * KD + n,
+                kv * ex2_approx(r0 - loc));
+    }
+    carry += loc;
+  }
+  for (int s = 0; s < nseg; ++s) {
+    float* rr = rp + static_cast<size_t>((t_start + seg_first + s * seg_rows) / C) * hstep;
+    const float tot = *rr;
+    *rr = carry;
+    carry += tot;
+  }
+  p_last[static_cast<size_t>(bh) * KD + n] = carry;
 }
 
 template <typename T, int KD>
@@ -242,16 +346,48 @@ cudaError_t cache_impl(const CacheArgs& a, cudaStream_t st) {
     if (!encode_tiled(&tmK, tdt, 4, a.k_new, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   }
+  // Split each sequence into chunk-aligned segments when the (batch, head
+  // group) CTAs alone would leave most SMs idle and there are enough rows.
+  const int ctas = a.B * (a.HQ / hpc);
+  int seg_first = 0, seg_rows = 0, nseg = 0;
+  {
+    const int c0 = (a.t_start + a.chunk - 1) / a.chunk * a.chunk;
+    const int head = min(c0 - a.t_start, a.T_new);  // rows of a partial first chunk
+    const int rest = a.T_new - head;
+    if (ctas < 148 && rest >= 4 * a.chunk) {
+      const int want = (296 + ctas - 1) / ctas;  // segments per sequence group: ~2 CTAs per SM
+      int L = (rest + want - 1) / want;
+      L = max(4 * a.chunk, (L + a.chunk - 1) / a.chunk * a.chunk);
+      seg_first = head;
+      seg_rows = L;
+      nseg = (rest + L - 1) / L;
+    }
+  }
   const int stage = CC::D * (hpc + nkv) * CC::ROWB;
   const int smem = CC::NS * stage + 2 * CC::NS * 8 + 16;
   auto kern = cache_build_kernel<T, KD>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
+  if (nseg > 0) {
+    cache_segsum_kernel<T, KD><<<dim3(a.HQ / hpc, a.B, nseg), 128, 0, st>>>(
+        static_cast<const T*>(a.g_new), a.t_start, a.T_new, a.cap, a.HQ, hpc, a.chunk, seg_first,
+        seg_rows, a.r_cache);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const long nthr = static_cast<long>(a.B) * a.HQ * KD;
+    cache_segscan_kernel<T, KD><<<static_cast<unsigned>((nthr + 127) / 128), 128, 0, st>>>(
+        static_cast<const T*>(a.k_new), static_cast<const T*>(a.g_new), a.p_prev, a.B, a.t_start,
+        a.T_new, a.cap, a.HQ, a.H, a.chunk, seg_first, seg_rows, nseg,
+        static_cast<T*>(a.k_tilde), a.r_cache, a.p_last);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   const int nwc = (hpc * CC::TPS + 31) / 32;
-  dim3 grid(a.HQ / hpc, a.B);
+  dim3 grid(a.HQ / hpc, a.B, nseg > 0 ? nseg : 1);
   kern<<<grid, (nwc + 1) * 32, smem, st>>>(tmG, tmK, a.p_prev, a.t_start, a.T_new, a.cap, a.HQ, G,
-                                           hpc, nkv, a.chunk, static_cast<T*>(a.k_tilde),
-                                           a.r_cache, a.p_last, a.err, a.wait_ns);
+                                           hpc, nkv, a.chunk, seg_first, seg_rows,
+                                           static_cast<T*>(a.k_tilde), a.r_cache, a.p_last,
+                                           a.err, a.wait_ns);
   return cudaGetLastError();
 }
 

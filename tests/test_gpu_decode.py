@@ -63,6 +63,30 @@ def test_ragged_appends_equal_one_build(wall, pieces):
         np.testing.assert_allclose(c.r_cache.double().cpu().numpy(), r, rtol=1e-5, atol=1e-4)
 
 
+@pytest.mark.parametrize("dtype,B,HQ,H,K,pieces", [
+    ("bf16", 1, 8, 2, 128, (37, 4000)),     # second append: partial chunk + 16 segments
+    ("f32", 1, 4, 4, 64, (100, 3000, 5)),   # K = 64, fp32, a short tail append
+    ("bf16", 3, 4, 1, 128, (0, 2500)),      # several batch rows, chunk-aligned start
+])
+def test_segmented_build_matches_oracle(wall, dtype, B, HQ, H, K, pieces):
+    """Small batches split every sequence into chunk-aligned segments (segment sums,
+    their prefix, then a parallel walk); the cache must equal the oracle's."""
+    T = sum(pieces)
+    spec, d = _inputs(B, T, HQ, H, K, K, dtype, seed=35)
+    cache = wall.KVCache(B, T + 3, HQ, H, K, K, dtype=spec.torch_dtype, chunk=64)
+    t = 0
+    for n in pieces:
+        if n:
+            cache.append(d["k"][:, t:t + n].contiguous(), d["g"][:, t:t + n].contiguous())
+        t += n
+    torch.cuda.synchronize()
+    kt, r, P = oracle.kv_cache(d["k"], d["g"], chunk=64, threads=ORACLE_THREADS)
+    assert_close(cache.k_tilde[:, :T], kt, spec.torch_dtype, "k_tilde")
+    nc = (T + 63) // 64
+    np.testing.assert_allclose(cache.r_cache[:, :nc].double().cpu().numpy(), r, rtol=1e-5, atol=1e-4)
+    np.testing.assert_allclose(cache.p.double().cpu().numpy(), P[:, -1], rtol=1e-5, atol=1e-4)
+
+
 STREAM = [
     dict(B=2, T0=200, steps=24, HQ=8, H=2, K=128, V=128, dtype="bf16", sink=True),
     dict(B=3, T0=130, steps=10, HQ=4, H=4, K=64, V=64, dtype="bf16", sink=False),
