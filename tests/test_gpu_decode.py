@@ -92,6 +92,7 @@ STREAM = [
     dict(B=3, T0=130, steps=10, HQ=4, H=4, K=64, V=64, dtype="bf16", sink=False),
     dict(B=1, T0=64, steps=12, HQ=16, H=2, K=128, V=64, dtype="bf16", sink=True),
     dict(B=2, T0=100, steps=8, HQ=2, H=1, K=64, V=128, dtype="f32", sink=True),
+    dict(B=2, T0=150, steps=6, HQ=16, H=1, K=64, V=128, dtype="bf16", sink=True),
     dict(B=1, T0=1, steps=5, HQ=4, H=1, K=128, V=128, dtype="bf16", sink=False),
 ]
 

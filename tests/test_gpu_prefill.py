@@ -90,6 +90,7 @@ EDGE = [
     dict(T=256, g_scalar=True, sink=True), dict(T=333, g_kind="negsoftplus", g_scalar=True),
     dict(T=257, K=64, V=128), dict(T=257, K=128, V=64), dict(T=200, HQ=4, H=1),
     dict(T=200, HQ=6, H=3, sink=True, window=50),
+    dict(T=300, HQ=16, H=1), dict(T=200, HQ=8, H=1, window=100, g_scalar=True),
 ]
 
 
