@@ -84,6 +84,7 @@ int* device_error_word() {
 }
 
 uint64_t wait_limit_ns() { return static_cast<uint64_t>(g_wait_ms.load()) * 1000000ull; }
+int fault_mode() { return g_fault_mode.load(); }
 
 bool encode_tiled(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
                   const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
@@ -230,6 +231,7 @@ wall_status_t wall_build_kv_cache(const void* k_new, const void* g_new, const fl
   a.err = wall::device_error_word();
   if (a.err == nullptr) return WALL_ERR_CUDA;
   a.wait_ns = wall::wait_limit_ns();
+  a.fault = wall::fault_mode();
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   return finish(wall::launch_cache_build(a, dt == WALL_DTYPE_BF16, st), st);
 }
@@ -268,6 +270,7 @@ wall_status_t wall_attn_decode(const void* q, const float* p_curr, const void* v
   a.err = wall::device_error_word();
   if (a.err == nullptr) return WALL_ERR_CUDA;
   a.wait_ns = wall::wait_limit_ns();
+  a.fault = wall::fault_mode();
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   stage_event(0, st);
   const cudaError_t e = wall::launch_decode(a, dt == WALL_DTYPE_BF16, st);

@@ -60,7 +60,8 @@ __global__ void __launch_bounds__(160) cache_build_kernel(
     const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmK,
     const float* __restrict__ p_prev, int t_start, int T_new, int cap, int HQ, int G, int HPC,
     int NKV, int C, int seg_first, int seg_rows, T* __restrict__ k_tilde,
-    float* __restrict__ r_cache, float* __restrict__ p_last, int* err, uint64_t wait_ns) {
+    float* __restrict__ r_cache, float* __restrict__ p_last, int* err, uint64_t wait_ns,
+    int fault) {
   using CC = CacheCfg<T, KD>;
   constexpr int D = CC::D;
   extern __shared__ __align__(128) uint8_t csm[];
@@ -102,13 +103,15 @@ __global__ void __launch_bounds__(160) cache_build_kernel(
         const int slot = i % CC::NS;
         if (i >= CC::NS && !mbar_wait(&empty[slot], ((i / CC::NS) - 1) & 1, wc)) break;
         uint8_t* st = csm + slot * stage;
-        mbar_arrive_expect_tx(&full[slot], stage);
-        tma_load_4d(st, &tmG, &full[slot], 0, hq0, rb + i * D, b);
-        tma_load_4d(st + gbytes, &tmK, &full[slot], 0, hq0 / G, rb + i * D, b);
+        if (!(fault == 3 && i == 0)) {  // testing hook: starve the consumers
+          mbar_arrive_expect_tx(&full[slot], stage);
+          tma_load_4d(st, &tmG, &full[slot], 0, hq0, rb + i * D, b);
+          tma_load_4d(st + gbytes, &tmK, &full[slot], 0, hq0 / G, rb + i * D, b);
+        }
         issued = i + 1;
       }
       for (int i = issued > CC::NS ? issued - CC::NS : 0; i < issued; ++i)
-        mbar_drain(&full[i % CC::NS], (i / CC::NS) & 1, wait_ns);
+        if (!(fault == 3 && i == 0)) mbar_drain(&full[i % CC::NS], (i / CC::NS) & 1, wait_ns);
     }
     return;
   }
@@ -387,7 +390,7 @@ cudaError_t cache_impl(const CacheArgs& a, cudaStream_t st) {
   kern<<<grid, (nwc + 1) * 32, smem, st>>>(tmG, tmK, a.p_prev, a.t_start, a.T_new, a.cap, a.HQ, G,
                                            hpc, nkv, a.chunk, seg_first, seg_rows,
                                            static_cast<T*>(a.k_tilde), a.r_cache, a.p_last,
-                                           a.err, a.wait_ns);
+                                           a.err, a.wait_ns, a.fault);
   return cudaGetLastError();
 }
 

@@ -91,7 +91,7 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
     const T* __restrict__ q, const float* __restrict__ p_curr, const float* __restrict__ r_cache,
     int T_kv, int cap, int HQ, int C, int cps, int nsplit, float sc, float* __restrict__ part,
-    int* err, uint64_t wait_ns) {
+    int* err, uint64_t wait_ns, int fault) {
   using D = DecCfg<T, KD, VD, G>;
   constexpr int LPH = 32 / G;    // lanes per query head
   constexpr int CPL = KD / LPH;  // k_tilde channels per lane
@@ -135,16 +135,18 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
         if (i >= D::NS && !mbar_wait(&empty[slot], ((i / D::NS) - 1) & 1, wc)) break;
         const int row0 = row_begin + i * D::SR;
         uint8_t* st = dsm + slot * D::STAGE;
-        mbar_arrive_expect_tx(&full[slot], D::STAGE);
-        tma_load_4d(st, &tmK, &full[slot], 0, h * G, row0, b);
-        tma_load_4d(st + D::K_BYTES, &tmV, &full[slot], 0, h, row0, b);
-        bulk_load(st + D::K_BYTES + D::V_BYTES,
-                  r_cache + ((static_cast<size_t>(b) * ncap + row0 / C) * HQ + h * G) * KD,
-                  D::R_BYTES, &full[slot]);
+        if (!(fault == 2 && i == 0)) {  // testing hook: starve the consumers
+          mbar_arrive_expect_tx(&full[slot], D::STAGE);
+          tma_load_4d(st, &tmK, &full[slot], 0, h * G, row0, b);
+          tma_load_4d(st + D::K_BYTES, &tmV, &full[slot], 0, h, row0, b);
+          bulk_load(st + D::K_BYTES + D::V_BYTES,
+                    r_cache + ((static_cast<size_t>(b) * ncap + row0 / C) * HQ + h * G) * KD,
+                    D::R_BYTES, &full[slot]);
+        }
         issued = i + 1;
       }
       for (int i = issued > D::NS ? issued - D::NS : 0; i < issued; ++i)
-        mbar_drain(&full[i % D::NS], (i / D::NS) & 1, wait_ns);
+        if (!(fault == 2 && i == 0)) mbar_drain(&full[i % D::NS], (i / D::NS) & 1, wait_ns);
     }
   } else {
     // ------------------------------------------------------------- consumers
@@ -338,7 +340,7 @@ cudaError_t decode_impl(const DecodeArgs& a, cudaStream_t st) {
   dim3 grid(a.nsplit, a.H, a.B);
   kern<<<grid, (D::NW + 1) * 32, D::SMEM, st>>>(
       tmK, tmV, static_cast<const T*>(a.q), a.p_curr, a.r_cache, a.T_kv, a.cap, a.HQ, a.chunk,
-      cps, a.nsplit, a.scale * kLog2e, a.part, a.err, a.wait_ns);
+      cps, a.nsplit, a.scale * kLog2e, a.part, a.err, a.wait_ns, a.fault);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (a.mid_event != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(a.mid_event), st);

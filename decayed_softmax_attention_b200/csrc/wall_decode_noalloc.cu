@@ -87,6 +87,7 @@ extern "C" wall_status_t wall_attn_decode_noalloc(
   a.err = wall::device_error_word();
   if (a.err == nullptr) return WALL_ERR_CUDA;
   a.wait_ns = wall::wait_limit_ns();
+  a.fault = wall::fault_mode();
   const cudaError_t e = wall::launch_decode(a, dt == WALL_DTYPE_BF16,
                                             reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? WALL_OK : WALL_ERR_CUDA;

@@ -15,6 +15,8 @@ constexpr int kBlockRows = 128;
 int* device_error_word();
 // Current limit of every bounded device-side wait, in nanoseconds.
 uint64_t wait_limit_ns();
+// Current testing fault mode (wall_debug_set_fault); 0 in normal operation.
+int fault_mode();
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda
 // link): unit element strides, zero fill out of bounds.  strides in bytes.
 bool encode_tiled(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
@@ -83,6 +85,7 @@ struct CacheArgs {
   float* p_last;
   int* err;          // device error word (bounded waits)
   uint64_t wait_ns;  // limit of each bounded wait
+  int fault;         // testing hook: 3 = producer skips its first stage
 };
 cudaError_t launch_cache_build(const CacheArgs& a, bool bf16, cudaStream_t st);
 
@@ -102,6 +105,7 @@ struct DecodeArgs {
   void* mid_event;  // optional cudaEvent_t recorded between the split and combine kernels
   int* err;         // device error word
   uint64_t wait_ns; // bounded-wait limit
+  int fault;        // testing hook: 2 = producer skips its first stage
 };
 int decode_max_splits(int B, int T_kv, int HQ, int H, int chunk);
 int decode_num_splits(int B, int T_kv, int HQ, int H, int chunk);

@@ -192,12 +192,14 @@ wall_status_t wall_attn_decode_noalloc(const void* q, const float* p_curr, const
 wall_status_t wall_device_error(wall_stream_t stream);
 
 /*
- * Testing hook (not for production use): mode 1 makes the next prefill
- * launches skip the producer's first K/V tile load, so the consumers' bounded
- * waits run out and report WALL_ERR_DEVICE_TIMEOUT through the error word
- * (no GPU fault, no hang: every wait gives up after about wait_ms
- * milliseconds).  mode 0 restores normal operation.  wait_ms <= 0 keeps the
- * default limit (2000 ms).
+ * Testing hook (not for production use): while mode is set, the producer of
+ * one kernel skips its first load, so that kernel's consumers' bounded waits
+ * run out and report WALL_ERR_DEVICE_TIMEOUT through the error word (no GPU
+ * fault, no hang: every wait gives up after about wait_ms milliseconds):
+ *   mode 1: prefill attention (first K/V tile), mode 2: decode split (first
+ *   k_tilde/v stage), mode 3: cache build (first g/k stage).
+ * Outputs of the starved call are unspecified.  mode 0 restores normal
+ * operation.  wait_ms <= 0 keeps the default limit (2000 ms).
  */
 void wall_debug_set_fault(int mode, int wait_ms);
 

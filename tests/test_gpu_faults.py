@@ -1,7 +1,8 @@
-"""Failure detection without a GPU fault: the prefill kernel's bounded waits.
+"""Failure detection without a GPU fault: the kernels' bounded waits.
 
-`wall_debug_set_fault(1, ms)` makes the producer skip the first key tile, so
-the consumers' waits run out after `ms` milliseconds.  The kernel must then
+`wall_debug_set_fault(mode, ms)` makes one kernel's producer skip its first
+load (1: prefill attention, 2: decode split, 3: cache build), so the
+consumers' waits run out after `ms` milliseconds.  The kernel must then
 wind down on its own (drain its copies, free tensor memory), report
 WALL_ERR_DEVICE_TIMEOUT through the device error word, and leave the context
 usable: the next normal call must succeed and match the oracle.  Nothing here
@@ -37,3 +38,53 @@ def test_starved_consumers_time_out_and_recover():
     assert wall.wall_device_error() == 0
     ro, _ = oracle.wall_fwd(d["q"], d["k"], d["v"], d["g"], d["g_scalar"], scale=d["scale"])
     assert_close(o, ro, torch.bfloat16, "after recovery")
+
+
+def _decode_inputs(wall, B=2, T=300, HQ=8, H=2, K=128, seed=5):
+    spec = W.PrefillSpec("fault_dec", B=B, T=T, HQ=HQ, H=H, K=K, V=K, dtype="bf16",
+                         g_kind="negsoftplus", seed=seed)
+    d = W.gen_prefill(spec, device="cuda")
+    return spec, d
+
+
+def test_decode_starved_consumers_time_out_and_recover():
+    """Mode 2: the decode split kernel's producer skips its first stage."""
+    import decayed_softmax_attention_b200 as wall
+    spec, d = _decode_inputs(wall)
+    cache = wall.KVCache(spec.B, spec.T, spec.HQ, spec.H, spec.K, spec.V, dtype=torch.bfloat16)
+    cache.append(d["k"], d["g"], d["v"])
+    q = d["q"][:, -1:].contiguous()
+    assert wall.wall_device_error() == 0
+    wall.wall_debug_set_fault(2, 100)
+    try:
+        cache.decode(q, scale=d["scale"])
+        status = wall.wall_device_error()
+    finally:
+        wall.wall_debug_set_fault(0, 0)
+    assert status == WALL_ERR_DEVICE_TIMEOUT
+    o = cache.decode(q, scale=d["scale"])
+    assert wall.wall_device_error() == 0
+    # the decode of the last token equals the last prefill row of each sequence
+    rows = [b * spec.T + spec.T - 1 for b in range(spec.B)]
+    ro, _ = oracle.wall_fwd(d["q"], d["k"], d["v"], d["g"], scale=d["scale"], rows=rows)
+    assert_close(o[:, 0], ro, torch.bfloat16, "decode after recovery")
+
+
+def test_cache_build_starved_consumers_time_out_and_recover():
+    """Mode 3: the cache build kernel's producer skips its first stage."""
+    import decayed_softmax_attention_b200 as wall
+    spec, d = _decode_inputs(wall, B=2, T=300, HQ=8, H=2, K=128, seed=6)
+    assert wall.wall_device_error() == 0
+    bad = wall.KVCache(spec.B, spec.T, spec.HQ, spec.H, spec.K, spec.V, dtype=torch.bfloat16)
+    wall.wall_debug_set_fault(3, 100)
+    try:
+        bad.append(d["k"], d["g"])
+        status = wall.wall_device_error()
+    finally:
+        wall.wall_debug_set_fault(0, 0)
+    assert status == WALL_ERR_DEVICE_TIMEOUT
+    good = wall.KVCache(spec.B, spec.T, spec.HQ, spec.H, spec.K, spec.V, dtype=torch.bfloat16)
+    good.append(d["k"], d["g"])
+    assert wall.wall_device_error() == 0
+    kt, _, _ = oracle.kv_cache(d["k"], d["g"], chunk=64)
+    assert_close(good.k_tilde, kt, torch.bfloat16, "cache after recovery")
