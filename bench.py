@@ -475,6 +475,46 @@ def run_ours(args, world, rank, local):
                      "prefill_alone_main_TFLOPs": flops / (alone_main * 1e-3) / 1e12,
                      "prefill_alone_main_frac_of_burst_peak":
                          flops / (alone_main * 1e-3) / 1e12 / bf16_peak})
+        # prefill that also emits its decode cache, against prefill + a separate build
+        pc = wall.KVCache(B, T, HQ, H, K, V, dtype=torch.bfloat16, chunk=64, device=dev)
+
+        def prefill_cache():
+            wall.wall_attn_fwd(pd["q"], pd["k"], pd["v"], pd["g"], pd["g_scalar"],
+                               pd["sink_bias"], window=pd["window"], scale=pd["scale"], out=o,
+                               lse=lse, workspace=ws, return_lse=True, cache=pc)
+
+        def build_only():
+            pc.length = 0
+            pc.append(pd["k"], pd["g"])
+
+        def time_fn(fn, n):
+            fn()
+            a, z = ev(), ev()
+            torch.cuda.synchronize()
+            a.record()
+            for _ in range(n):
+                fn()
+            z.record()
+            torch.cuda.synchronize()
+            return a.elapsed_time(z) / n
+
+        n_rep = max(args.steps, 5)
+        cev = [[ev() for _ in range(3)] for _ in range(n_rep)]
+        for trio in cev:
+            for e in trio:
+                e.record()
+        for i in range(n_rep):
+            wall.wall_debug_set_stage_events(*cev[i])
+            prefill_cache()
+            wall.wall_debug_set_stage_events()
+        torch.cuda.synchronize()
+        side.update({
+            "prefill_with_cache_prepass_ms": statistics.mean(e[0].elapsed_time(e[1]) for e in cev),
+            "prefill_with_cache_main_ms": statistics.mean(e[1].elapsed_time(e[2]) for e in cev)})
+        side.update({"prefill_with_cache_ms": time_fn(prefill_cache, n_rep),
+                     "prefill_plain_ms": time_fn(prefill, n_rep),
+                     "cache_build_of_prefill_ms": time_fn(build_only, n_rep)})
+        del pc
         side.update({"prefill_ms": statistics.mean(pre_ms),
                      "prefill_prepass_ms": statistics.mean(pre_prep_ms),
                      "prefill_main_ms": main_avg,

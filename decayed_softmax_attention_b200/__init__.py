@@ -46,7 +46,7 @@ EXPORTED_SYMBOLS = (
     "wall_status_string", "wall_attn_fwd_workspace_size", "wall_attn_fwd",
     "wall_build_kv_cache", "wall_attn_decode_workspace_size", "wall_attn_decode",
     "wall_device_error", "wall_debug_set_fault", "wall_debug_set_stage_events",
-    "wall_attn_decode_noalloc",
+    "wall_attn_decode_noalloc", "wall_attn_fwd_with_cache",
 )
 
 
@@ -82,6 +82,9 @@ def load_library():
     lib.wall_attn_fwd_workspace_size.restype = S
     lib.wall_attn_fwd.argtypes = [P, P, P, P, P, P, I, P, I, I, I, I, I, I, I, I, F, P, P, P, S, P]
     lib.wall_attn_fwd.restype = I
+    lib.wall_attn_fwd_with_cache.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P, P,
+                                             P, S, I, I, P, P, P, P]
+    lib.wall_attn_fwd_with_cache.restype = I
     lib.wall_build_kv_cache.argtypes = [P, P, P, I, I, I, I, I, I, I, I, I, P, P, P, P]
     lib.wall_build_kv_cache.restype = I
     lib.wall_attn_decode_workspace_size.argtypes = [I, I, I, I, I, I]
@@ -148,8 +151,13 @@ def wall_attn_fwd_workspace_size(B, T, HQ, H, K, V, dtype) -> int:
 
 
 def wall_attn_fwd(q, k, v, g, g_scalar=None, sink_bias=None, window=0, cu_seqlens=None,
-                  scale=None, return_lse=False, out=None, lse=None, workspace=None):
-    """Prefill forward (README "Usage"): o [B,T,HQ,V] (and lse [B,T,HQ] fp32, natural log)."""
+                  scale=None, return_lse=False, out=None, lse=None, workspace=None, cache=None):
+    """Prefill forward (README "Usage"): o [B,T,HQ,V] (and lse [B,T,HQ] fp32, natural log).
+
+    cache: optional KVCache (capacity >= T); the prefill then also writes its decode
+    cache rows 0 .. T-1 (k_tilde, anchors, P at row T-1) and sets cache.length = T.
+    Value rows are the caller's (copy v into cache.v).
+    """
     lib = load_library()
     B, T, HQ, K = q.shape
     H, V = k.shape[2], v.shape[3]
@@ -163,6 +171,23 @@ def wall_attn_fwd(q, k, v, g, g_scalar=None, sink_bias=None, window=0, cu_seqlen
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     nseq = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if cache is not None:
+        # the prefill also fills the decode cache (rows 0 .. T-1); no packed documents
+        if cu_seqlens is not None:
+            raise ValueError("cache output needs one sequence per batch row (no cu_seqlens)")
+        st = lib.wall_attn_fwd_with_cache(
+            _dev(q, "q", dt), _dev(k, "k", dt, (B, T, H, K)), _dev(v, "v", dt, (B, T, H, V)),
+            _dev(g, "g", dt, (B, T, HQ, K)), _dev(g_scalar, "g_scalar", dt, (B, T, HQ)),
+            _dev(sink_bias, "sink_bias", torch.float32, (HQ,)), int(window or 0),
+            B, T, HQ, H, K, V, code, float(scale) if scale else 0.0,
+            _dev(out, "out", dt, (B, T, HQ, V)), _dev(lse, "lse", torch.float32, (B, T, HQ)),
+            _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+            cache.cap, cache.chunk, _dev(cache.k_tilde, "k_tilde", dt, (B, cache.cap, HQ, K)),
+            _dev(cache.r_cache, "r_cache", torch.float32), _dev(cache.p, "p_last", torch.float32),
+            _stream(q.device))
+        _check(st, "wall_attn_fwd_with_cache")
+        cache.length = T
+        return (out, lse) if return_lse else out
     st = lib.wall_attn_fwd(
         _dev(q, "q", dt), _dev(k, "k", dt, (B, T, H, K)), _dev(v, "v", dt, (B, T, H, V)),
         _dev(g, "g", dt, (B, T, HQ, K)), _dev(g_scalar, "g_scalar", dt, (B, T, HQ)),

@@ -120,11 +120,24 @@ size_t wall_attn_fwd_workspace_size(int B, int T, int HQ, int H, int K, int V, w
   return wall::fwd_workspace_layout(B, T, HQ, K, dt == WALL_DTYPE_BF16, nullptr, nullptr);
 }
 
-wall_status_t wall_attn_fwd(const void* q, const void* k, const void* v, const void* g,
-                            const void* g_scalar, const float* sink_bias, int window,
-                            const int32_t* cu_seqlens, int num_seqs, int B, int T, int HQ, int H,
-                            int K, int V, wall_dtype_t dt, float scale, void* o, float* lse,
-                            void* workspace, size_t workspace_bytes, wall_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Decode cache outputs of wall_attn_fwd_with_cache (validated by the caller).
+struct CacheOut {
+  void* k_tilde;
+  float* r_cache;
+  float* p_last;
+  int cap, chunk;
+};
+
+wall_status_t fwd_impl(const void* q, const void* k, const void* v, const void* g,
+                       const void* g_scalar, const float* sink_bias, int window,
+                       const int32_t* cu_seqlens, int num_seqs, int B, int T, int HQ, int H,
+                       int K, int V, wall_dtype_t dt, float scale, void* o, float* lse,
+                       void* workspace, size_t workspace_bytes, wall_stream_t stream,
+                       const CacheOut* co) {
   if (B < 0 || T < 0 || HQ <= 0 || H <= 0 || HQ % H != 0) return WALL_ERR_INVALID_ARG;
   if (dt != WALL_DTYPE_F32 && dt != WALL_DTYPE_BF16) return WALL_ERR_INVALID_ARG;
   if (!supported_dim(K) || !supported_dim(V)) return WALL_ERR_UNSUPPORTED;
@@ -156,6 +169,13 @@ wall_status_t wall_attn_fwd(const void* q, const void* k, const void* v, const v
   a.scale = scale; a.o = o; a.lse = lse; a.err = err;
   a.wait_ns = wall::wait_limit_ns();
   a.fault = g_fault_mode.load();
+  if (co != nullptr) {
+    a.kt_out = co->k_tilde;
+    a.r_out = co->r_cache;
+    a.plast_out = co->p_last;
+    a.cache_cap = co->cap;
+    a.cache_chunk = co->chunk;
+  }
   wall::FwdWork w;
   wall::fwd_workspace_layout(B, T, HQ, K, bf16, &w, static_cast<char*>(workspace));
 
@@ -205,6 +225,37 @@ wall_status_t wall_attn_fwd(const void* q, const void* k, const void* v, const v
   e = wall::launch_fwd_tc(a, w, tmQ, tmK, tmV, tmKX, st);
   stage_event(2, st);
   return finish(e, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+wall_status_t wall_attn_fwd(const void* q, const void* k, const void* v, const void* g,
+                            const void* g_scalar, const float* sink_bias, int window,
+                            const int32_t* cu_seqlens, int num_seqs, int B, int T, int HQ, int H,
+                            int K, int V, wall_dtype_t dt, float scale, void* o, float* lse,
+                            void* workspace, size_t workspace_bytes, wall_stream_t stream) {
+  return fwd_impl(q, k, v, g, g_scalar, sink_bias, window, cu_seqlens, num_seqs, B, T, HQ, H, K,
+                  V, dt, scale, o, lse, workspace, workspace_bytes, stream, nullptr);
+}
+
+wall_status_t wall_attn_fwd_with_cache(const void* q, const void* k, const void* v, const void* g,
+                                       const void* g_scalar, const float* sink_bias, int window,
+                                       int B, int T, int HQ, int H, int K, int V, wall_dtype_t dt,
+                                       float scale, void* o, float* lse, void* workspace,
+                                       size_t workspace_bytes, int cap, int chunk, void* k_tilde,
+                                       float* r_cache, float* p_last, wall_stream_t stream) {
+  if (chunk != 32 && chunk != 64 && chunk != 128) return WALL_ERR_UNSUPPORTED;
+  if (cap < T || cap < 0) return WALL_ERR_INVALID_ARG;
+  if (B > 0 && T > 0) {
+    if (!k_tilde || !r_cache || !p_last) return WALL_ERR_INVALID_ARG;
+    if (!aligned(k_tilde, 16) || !aligned(r_cache, 16) || !aligned(p_last, 16))
+      return WALL_ERR_INVALID_ARG;
+  }
+  const CacheOut co{k_tilde, r_cache, p_last, cap, chunk};
+  return fwd_impl(q, k, v, g, g_scalar, sink_bias, window, nullptr, 0, B, T, HQ, H, K, V, dt,
+                  scale, o, lse, workspace, workspace_bytes, stream, &co);
 }
 
 wall_status_t wall_build_kv_cache(const void* k_new, const void* g_new, const float* p_prev,

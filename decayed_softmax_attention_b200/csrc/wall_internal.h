@@ -65,6 +65,11 @@ struct FwdArgs {
   int* err;
   uint64_t wait_ns;
   int fault;
+  // Decode cache emitted by the prepass (null k_tilde: none).
+  void* kt_out = nullptr;     // [B, cap, HQ, K] input dtype
+  float* r_out = nullptr;     // [B, ceil(cap/chunk), HQ, K] fp32
+  float* plast_out = nullptr; // [B, HQ, K] fp32
+  int cache_cap = 0, cache_chunk = 64;
 };
 
 size_t fwd_workspace_layout(int B, int T, int HQ, int K, bool bf16, FwdWork* w, char* base);

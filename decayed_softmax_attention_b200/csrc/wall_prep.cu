@@ -29,11 +29,13 @@ __global__ void __launch_bounds__(256, 3) prep_local_kernel(
     const Tin* __restrict__ gs, const int32_t* __restrict__ cu, int nseq, int window, int T,
     int HQ, int H, int NB, Tin* __restrict__ qh, Tin* __restrict__ kh, float* __restrict__ bsum,
     float* __restrict__ ssl, float* __restrict__ ssb, __nv_bfloat16* __restrict__ kx,
-    float inv_scale, int* __restrict__ rowlo) {
+    float inv_scale, int* __restrict__ rowlo, Tin* __restrict__ kt, float* __restrict__ rc,
+    int cap, int C) {
   constexpr int CG = KD / 8;
   constexpr int RG = 128 / CG;
   constexpr int RPG = 128 / RG;
   __shared__ float tot[2][RG][KD];
+  __shared__ float gfirst[2][RG][KD];  // g at the first row of each row group (cache output)
   __shared__ float wsum[2][4];
 
   const int half = threadIdx.x >> 7, tid = threadIdx.x & 127;
@@ -55,15 +57,19 @@ __global__ void __launch_bounds__(256, 3) prep_local_kernel(
   constexpr int U2 = sizeof(Tin) == 2 ? 2 : 1;
   static_assert(RPG % U1 == 0 && RPG % U2 == 0, "row batch must divide the rows per thread");
   for (int m0 = 0; m0 < RPG; m0 += U1) {
-    Raw8<Tin> rg[U1];
+    Raw8<Tin> gv[U1];
 #pragma unroll
     for (int u = 0; u < U1; ++u)
-      if (t0 + m0 + u < T) rg[u].load(gb + static_cast<size_t>(t0 + m0 + u) * qrow);
+      if (t0 + m0 + u < T) gv[u].load(gb + static_cast<size_t>(t0 + m0 + u) * qrow);
 #pragma unroll
     for (int u = 0; u < U1; ++u) {
       if (t0 + m0 + u < T) {
         float f[8];
-        rg[u].get(f);
+        gv[u].get(f);
+        if (m0 + u == 0 && kt != nullptr) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) gfirst[half][rg][cg * 8 + c] = f[c];
+        }
 #pragma unroll
         for (int c = 0; c < 8; ++c) acc[c] += f[c];
       }
@@ -73,19 +79,31 @@ __global__ void __launch_bounds__(256, 3) prep_local_kernel(
   for (int c = 0; c < 8; ++c) tot[half][rg][cg * 8 + c] = acc[c];
   __syncthreads();
 
-  float run[8], total[8], qoff[8];
+  // Decode cache: this thread's rows lie in one chunk (C is a multiple of RPG
+  // and divides 128); its anchor R = G at the chunk's first row, block-local.
+  const int rgc = ((rg * RPG) / C) * C / RPG;  // row group that opens the chunk
+  float run[8], total[8], qoff[8], cst[8];
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
-    float pre = 0.f, all = 0.f, first = 0.f;
+    float pre = 0.f, all = 0.f, first = 0.f, cpre = 0.f;
     for (int r = 0; r < RG; ++r) {
       const float x = tot[half][r][cg * 8 + c];
       all += x;
       if (r < rg) pre += x;
+      if (r < rgc) cpre += x;
       if (half == 1) first += tot[0][r][cg * 8 + c];
     }
     run[c] = pre;
     total[c] = all;
     qoff[c] = first;  // g summed over the first half of the query block
+    cst[c] = kt != nullptr ? cpre + gfirst[half][rgc][cg * 8 + c] : 0.f;
+  }
+  if (kt != nullptr && rg == rgc && t0 < T) {
+    // block-local anchor of the chunk; the scan adds the block's offset
+    const int ncap = (cap + C - 1) / C;
+    float* dst = rc + ((static_cast<size_t>(b) * ncap + t0 / C) * HQ + hq) * KD + cg * 8;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) dst[c] = cst[c];
   }
   if (rg == 0 && blk < NB) {
     float* dst = bsum + (static_cast<size_t>(bh) * NB + blk) * KD + cg * 8;
@@ -98,12 +116,12 @@ __global__ void __launch_bounds__(256, 3) prep_local_kernel(
   Tin* qo = qh + static_cast<size_t>(bh) * T * KD + cg * 8;
   Tin* ko = kh + static_cast<size_t>(bh) * T * KD + cg * 8;
   for (int m0 = 0; m0 < RPG; m0 += U2) {
-    Raw8<Tin> rg[U2], rq[U2], rk[U2];
+    Raw8<Tin> gv[U2], rq[U2], rk[U2];
 #pragma unroll
     for (int u = 0; u < U2; ++u) {
       const int t = t0 + m0 + u;
       if (t < T) {
-        rg[u].load(gb + static_cast<size_t>(t) * qrow);
+        gv[u].load(gb + static_cast<size_t>(t) * qrow);
         rq[u].load(qb + static_cast<size_t>(t) * qrow);
         rk[u].load(kb + static_cast<size_t>(t) * krow);
       }
@@ -113,17 +131,22 @@ __global__ void __launch_bounds__(256, 3) prep_local_kernel(
       const int t = t0 + m0 + u;
       if (t < T) {
         float f[8], x[8], y[8];
-        rg[u].get(f);
+        gv[u].get(f);
         rq[u].get(x);
         rk[u].get(y);
+        float z[8];
+        // exp(a) as 2^(a log2 e): one MUFU op each (relative error ~2^-22)
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           run[c] += f[c];
-          x[c] *= expf(qoff[c] + run[c]);
-          y[c] *= expf(total[c] - run[c]);
+          z[c] = y[c] * ex2_approx((cst[c] - run[c]) * kLog2e);  // decode cache row (if kt)
+          x[c] *= ex2_approx((qoff[c] + run[c]) * kLog2e);
+          y[c] *= ex2_approx((total[c] - run[c]) * kLog2e);
         }
         store8(qo + static_cast<size_t>(t) * KD, x);
         store8(ko + static_cast<size_t>(t) * KD, y);
+        if (kt != nullptr)
+          store8(kt + ((static_cast<size_t>(b) * cap + t) * HQ + hq) * KD + cg * 8, z);
       }
     }
   }
@@ -182,11 +205,9 @@ __global__ void __launch_bounds__(256, 3) prep_local_kernel(
 
 // Exclusive scan of the block sums over the blocks of one (batch, head).
 template <int KD>
-__global__ void __launch_bounds__(KD + 32) prep_scan_kernel(const float* __restrict__ bsum,
-                                                            const float* __restrict__ ssb, int NB,
-                                                            float* __restrict__ AQ,
-                                                            float* __restrict__ AK,
-                                                            float* __restrict__ ssa) {
+__global__ void __launch_bounds__(KD + 32) prep_scan_kernel(
+    const float* __restrict__ bsum, const float* __restrict__ ssb, int NB, float* __restrict__ AQ,
+    float* __restrict__ AK, float* __restrict__ ssa, float* __restrict__ plast) {
   const int bh = blockIdx.x, tid = threadIdx.x;
   if (tid < KD) {
     float acc = 0.f;
@@ -197,6 +218,7 @@ __global__ void __launch_bounds__(KD + 32) prep_scan_kernel(const float* __restr
       acc += bsum[i];
       AK[i] = acc;
     }
+    if (plast != nullptr) plast[static_cast<size_t>(bh) * KD + tid] = acc * kLog2e;
   } else if (tid == KD && ssb != nullptr) {
     float acc = 0.f;
     for (int blk = 0; blk < NB; ++blk) {
@@ -210,6 +232,21 @@ __global__ void __launch_bounds__(KD + 32) prep_scan_kernel(const float* __restr
   }
 }
 
+// Decode cache anchors (when the prefill emits the cache): the prepass left
+// each chunk's block-local G in its slot; add the block's prefix, in log2 units.
+// One CTA per (batch * query head, chunk), one thread per channel.
+template <int KD>
+__global__ void __launch_bounds__(KD) cache_anchor_kernel(const float* __restrict__ AQ, int NB,
+                                                          int HQ, int cap, int C, int nchunk,
+                                                          float* __restrict__ rc) {
+  const int bh = static_cast<int>(blockIdx.x) / nchunk, c = static_cast<int>(blockIdx.x) % nchunk;
+  const int b = bh / HQ, hq = bh % HQ, n = threadIdx.x;
+  const int ncap = (cap + C - 1) / C;
+  const int blk = c * C / kBlockRows;
+  float* slot = rc + ((static_cast<size_t>(b) * ncap + c) * HQ + hq) * KD + n;
+  *slot = (*slot + AQ[(static_cast<size_t>(bh) * NB + blk) * KD + n]) * kLog2e;
+}
+
 template <typename Tin, int KD>
 cudaError_t prep_impl(const FwdArgs& a, const FwdWork& w, cudaStream_t st) {
   const int BHQ = a.B * a.HQ;
@@ -219,11 +256,16 @@ cudaError_t prep_impl(const FwdArgs& a, const FwdWork& w, cudaStream_t st) {
       static_cast<const Tin*>(a.g_scalar), a.cu_seqlens, a.num_seqs, a.window, a.T, a.HQ, a.H,
       a.NB, static_cast<Tin*>(w.qh), static_cast<Tin*>(w.kh), w.bsum, w.ssl, w.ssb,
       sizeof(Tin) == 2 ? static_cast<__nv_bfloat16*>(w.kx) : nullptr, 1.f / (a.scale * kLog2e),
-      w.rowlo);
+      w.rowlo, static_cast<Tin*>(a.kt_out), a.r_out, a.cache_cap, a.cache_chunk);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   prep_scan_kernel<KD><<<BHQ, KD + 32, 0, st>>>(w.bsum, a.g_scalar ? w.ssb : nullptr, a.NB, w.AQ,
-                                                 w.AK, w.ssa);
+                                                 w.AK, w.ssa, a.kt_out ? a.plast_out : nullptr);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || a.kt_out == nullptr) return e;
+  const int nchunk = (a.T + a.cache_chunk - 1) / a.cache_chunk;  // chunks that start below T
+  cache_anchor_kernel<KD><<<static_cast<unsigned>(BHQ) * nchunk, KD, 0, st>>>(
+      w.AQ, a.NB, a.HQ, a.cache_cap, a.cache_chunk, nchunk, a.r_out);
   return cudaGetLastError();
 }
 

@@ -97,6 +97,27 @@ wall_status_t wall_attn_fwd(const void* q, const void* k, const void* v, const v
                             wall_stream_t stream);
 
 /*
+ * Prefill forward that also emits the decode cache of its rows (Wall Attention
+ * README, "Decode": the cache the decode path attends over, built here as a
+ * side output of the prefill prepass instead of a separate
+ * wall_build_kv_cache pass).  Same arguments and results as wall_attn_fwd,
+ * without packed documents (one sequence per batch row), plus:
+ *   cap      rows of the cache (>= T); chunk in {32, 64, 128}
+ *   k_tilde  [B, cap, HQ, K] dtype dt   out: rows 0 .. T-1 (others untouched)
+ *   r_cache  [B, ceil(cap/chunk), HQ, K] fp32  out: anchors of chunks starting below T
+ *   p_last   [B, HQ, K] fp32            out: P at row T-1
+ * The result equals wall_build_kv_cache(k, g, NULL, B, 0, T, cap, ...) up to
+ * fp32 rounding; further tokens are appended with wall_build_kv_cache
+ * (t_start = T, p_prev = p_last).  All three pointers 16-byte aligned.
+ */
+wall_status_t wall_attn_fwd_with_cache(const void* q, const void* k, const void* v, const void* g,
+                                       const void* g_scalar, const float* sink_bias, int window,
+                                       int B, int T, int HQ, int H, int K, int V, wall_dtype_t dt,
+                                       float scale, void* o, float* lse, void* workspace,
+                                       size_t workspace_bytes, int cap, int chunk, void* k_tilde,
+                                       float* r_cache, float* p_last, wall_stream_t stream);
+
+/*
  * Decode cache build / append (Wall Attention README, "Decode"):
  *   P = cumsum(g) * (1/ln 2);  k_tilde[j] = k[j] * exp2(R_c - P[j])
  * with one anchor vector R_c = P[c * chunk] per chunk of `chunk` tokens (the

@@ -79,6 +79,30 @@ def test_fwd_host_validation(lib):
     assert _fwd(lib, B=0) == 0
 
 
+def _fwd_cache(lib, **kw):
+    a = dict(q=_fake(), k=_fake(), v=_fake(), g=_fake(), gs=None, sink=None, window=0,
+             B=1, T=64, HQ=4, H=2, K=64, V=64, dt=BF16, scale=0.0, o=_fake(), lse=None,
+             ws=_fake(0x100000), wsb=1 << 40, cap=64, C=64, kt=_fake(0x2000), r=_fake(0x3000),
+             p=_fake(0x4000), stream=None)
+    a.update(kw)
+    return lib.wall_attn_fwd_with_cache(
+        a["q"], a["k"], a["v"], a["g"], a["gs"], a["sink"], a["window"], a["B"], a["T"],
+        a["HQ"], a["H"], a["K"], a["V"], a["dt"], a["scale"], a["o"], a["lse"], a["ws"],
+        a["wsb"], a["cap"], a["C"], a["kt"], a["r"], a["p"], a["stream"])
+
+
+def test_fwd_with_cache_host_validation(lib):
+    assert _fwd_cache(lib, C=48) == UNSUPPORTED
+    assert _fwd_cache(lib, cap=32) == INVALID             # cache smaller than the prefill
+    assert _fwd_cache(lib, kt=None) == INVALID
+    assert _fwd_cache(lib, r=_fake(0x3004)) == INVALID    # anchors not 16-byte aligned
+    assert _fwd_cache(lib, p=None) == INVALID
+    assert _fwd_cache(lib, HQ=6, H=4) == INVALID          # the forward's own checks still apply
+    assert _fwd_cache(lib, K=96) == UNSUPPORTED
+    assert _fwd_cache(lib, wsb=16) == WORKSPACE
+    assert _fwd_cache(lib, T=0, cap=0) == 0               # empty input: no-op
+
+
 def test_fwd_workspace_size(lib):
     small = lib.wall_attn_fwd_workspace_size(1, 128, 2, 2, 64, 64, BF16)
     big = lib.wall_attn_fwd_workspace_size(1, 8192, 32, 8, 128, 128, BF16)

@@ -87,6 +87,42 @@ def test_segmented_build_matches_oracle(wall, dtype, B, HQ, H, K, pieces):
     np.testing.assert_allclose(cache.p.double().cpu().numpy(), P[:, -1], rtol=1e-5, atol=1e-4)
 
 
+@pytest.mark.parametrize("dtype,B,T,HQ,H,K,V,chunk,gs", [
+    ("bf16", 2, 1000, 8, 2, 128, 128, 64, True),
+    ("f32", 1, 300, 4, 4, 64, 64, 32, False),
+    ("bf16", 1, 517, 16, 4, 64, 128, 128, False),
+])
+def test_prefill_emits_decode_cache(wall, dtype, B, T, HQ, H, K, V, chunk, gs):
+    """wall_attn_fwd(cache=...) writes the decode cache of its T rows: equal to the oracle's
+    cache, the prefill output unchanged, and a decode step appended after it equal to the
+    prefill row of the next token."""
+    spec = W.PrefillSpec("emit", B=B, T=T + 1, HQ=HQ, H=H, K=K, V=V, dtype=dtype,
+                         g_kind="negsoftplus", g_scalar=gs, seed=41)
+    d = W.gen_prefill(spec, device="cuda")
+    pre = {n: d[n][:, :T].contiguous() for n in ("q", "k", "v", "g")}
+    gsc = d["g_scalar"][:, :T].contiguous() if gs else None
+    cache = wall.KVCache(B, T + 8, HQ, H, K, V, dtype=spec.torch_dtype, chunk=chunk)
+    o = wall.wall_attn_fwd(pre["q"], pre["k"], pre["v"], pre["g"], gsc, scale=d["scale"],
+                           cache=cache)
+    o_plain = wall.wall_attn_fwd(pre["q"], pre["k"], pre["v"], pre["g"], gsc, scale=d["scale"])
+    torch.cuda.synchronize()
+    assert cache.length == T
+    assert torch.equal(o, o_plain)
+    kt, r, P = oracle.kv_cache(pre["k"], pre["g"], chunk=chunk, threads=ORACLE_THREADS)
+    assert_close(cache.k_tilde[:, :T], kt, spec.torch_dtype, "emitted k_tilde")
+    nc = (T + chunk - 1) // chunk
+    np.testing.assert_allclose(cache.r_cache[:, :nc].double().cpu().numpy(), r, rtol=1e-5, atol=1e-4)
+    np.testing.assert_allclose(cache.p.double().cpu().numpy(), P[:, -1], rtol=1e-5, atol=1e-4)
+    if not gs:  # decode has no gate term (README decode call takes none)
+        cache.v[:, :T + 1].copy_(d["v"])
+        cache.append(d["k"][:, T:T + 1].contiguous(), d["g"][:, T:T + 1].contiguous())
+        od = cache.decode(d["q"][:, T:T + 1].contiguous(), scale=d["scale"])
+        rows = [b * (T + 1) + T for b in range(B)]
+        ro, _ = oracle.wall_fwd(d["q"], d["k"], d["v"], d["g"], scale=d["scale"], rows=rows,
+                                threads=ORACLE_THREADS)
+        assert_close(od[:, 0], ro, spec.torch_dtype, "decode after emitted cache")
+
+
 STREAM = [
     dict(B=2, T0=200, steps=24, HQ=8, H=2, K=128, V=128, dtype="bf16", sink=True),
     dict(B=3, T0=130, steps=10, HQ=4, H=4, K=64, V=64, dtype="bf16", sink=False),
