@@ -540,6 +540,33 @@ def run_ours(args, world, rank, local):
             "frac_of_hbm_incl_combine": dec_value / world / hbm_peak,
         }
         build_gbps = build_bytes / (build_ms * 1e-3) / 1e9
+        # per-sequence lengths: row b attends rows [0, len_b), len_b ~ U[T0/2, T0] (seeded)
+        gl = torch.Generator().manual_seed(4242)
+        lens = torch.randint(T0 // 2, T0 + 1, (dspec.B,), generator=gl, dtype=torch.int32)
+        seqlens = lens.to(dev)
+        cache.length = T0
+        cache.p.copy_(p_prefix)
+        qv = q_steps[0] if S else torch.zeros((dspec.B, 1, dspec.HQ, dspec.K),
+                                               dtype=torch.bfloat16, device=dev)
+
+        def dec_varlen():
+            wall.wall_attn_decode(qv, cache.p[:, None], cache.v, cache.k_tilde, cache.r_cache, T0,
+                                  scale=dspec.K ** -0.5, chunk=dspec.C, out=dout, seqlens=seqlens)
+
+        dec_varlen()
+        va, vz = ev(), ev()
+        torch.cuda.synchronize()
+        va.record()
+        for _ in range(10):
+            dec_varlen()
+        vz.record()
+        torch.cuda.synchronize()
+        var_ms = va.elapsed_time(vz) / 10
+        var_bytes = sum(int(L) * (dspec.HQ * dspec.K + dspec.H * dspec.V) * 2
+                        + ((int(L) + dspec.C - 1) // dspec.C) * dspec.HQ * dspec.K * 4 for L in lens)
+        side.update({"decode_varlen_ms": var_ms,
+                     "decode_varlen_GBps": var_bytes / (var_ms * 1e-3) / 1e9,
+                     "decode_varlen_frac_of_hbm": var_bytes / (var_ms * 1e-3) / 1e9 / hbm_peak})
         side.update({"cache_build_prefix_ms": build_ms,
                      "cache_build_prefix_GBps": build_gbps,
                      "cache_build_roofline": {

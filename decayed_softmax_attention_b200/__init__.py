@@ -26,7 +26,7 @@ import torch
 __all__ = [
     "WallError", "lib_path", "load_library", "wall_attn_fwd", "wall_attn_fwd_workspace_size",
     "wall_build_kv_cache", "wall_attn_decode", "wall_attn_decode_workspace_size",
-    "wall_attn_decode_noalloc",
+    "wall_attn_decode_noalloc", "wall_append_kv_cache_varlen",
     "wall_device_error", "wall_debug_set_fault", "wall_debug_set_stage_events", "KVCache",
     "EXPORTED_SYMBOLS",
 ]
@@ -46,7 +46,8 @@ EXPORTED_SYMBOLS = (
     "wall_status_string", "wall_attn_fwd_workspace_size", "wall_attn_fwd",
     "wall_build_kv_cache", "wall_attn_decode_workspace_size", "wall_attn_decode",
     "wall_device_error", "wall_debug_set_fault", "wall_debug_set_stage_events",
-    "wall_attn_decode_noalloc", "wall_attn_fwd_with_cache",
+    "wall_attn_decode_noalloc", "wall_attn_fwd_with_cache", "wall_attn_decode_varlen",
+    "wall_append_kv_cache_varlen",
 )
 
 
@@ -87,10 +88,15 @@ def load_library():
     lib.wall_attn_fwd_with_cache.restype = I
     lib.wall_build_kv_cache.argtypes = [P, P, P, I, I, I, I, I, I, I, I, I, P, P, P, P]
     lib.wall_build_kv_cache.restype = I
+    lib.wall_append_kv_cache_varlen.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P, P, P, P]
+    lib.wall_append_kv_cache_varlen.restype = I
     lib.wall_attn_decode_workspace_size.argtypes = [I, I, I, I, I, I]
     lib.wall_attn_decode_workspace_size.restype = S
     lib.wall_attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, P, P, P, S, P]
     lib.wall_attn_decode.restype = I
+    lib.wall_attn_decode_varlen.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, P,
+                                            P, P, S, P]
+    lib.wall_attn_decode_varlen.restype = I
     lib.wall_attn_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, P, P, P]
     lib.wall_attn_decode_noalloc.restype = I
     lib.wall_device_error.argtypes = [P]
@@ -219,13 +225,42 @@ def wall_build_kv_cache(k_new, g_new, k_tilde, r_cache, p_last, t_start=0, p_pre
     return p_last
 
 
+def wall_append_kv_cache_varlen(k_new, g_new, k_tilde, r_cache, p_last, t_pos, p_prev=None,
+                                chunk=64):
+    """Append one token per batch row at row b's own position t_pos[b] (device int32 [B]).
+
+    k_new [B,1,H,K], g_new [B,1,HQ,K]; p_prev [B,HQ,K] fp32 (defaults to p_last, updated in
+    place) holds P at row t_pos[b] - 1.
+    """
+    lib = load_library()
+    B, _, H, K = k_new.shape
+    HQ = g_new.shape[2]
+    cap = k_tilde.shape[1]
+    dt = k_new.dtype
+    if p_prev is None:
+        p_prev = p_last
+    st = lib.wall_append_kv_cache_varlen(
+        _dev(k_new, "k_new", dt, (B, 1, H, K)), _dev(g_new, "g_new", dt, (B, 1, HQ, K)),
+        _dev(p_prev, "p_prev", torch.float32, (B, HQ, K)), _dev(t_pos, "t_pos", torch.int32, (B,)),
+        B, cap, HQ, H, K, int(chunk), _dtype_code(k_new),
+        _dev(k_tilde, "k_tilde", dt, (B, cap, HQ, K)),
+        _dev(r_cache, "r_cache", torch.float32, (B, (cap + chunk - 1) // chunk, HQ, K)),
+        _dev(p_last, "p_last", torch.float32, (B, HQ, K)), _stream(k_new.device))
+    _check(st, "wall_append_kv_cache_varlen")
+    return p_last
+
+
 def wall_attn_decode_workspace_size(B, T_kv, HQ, H, V, chunk=64) -> int:
     return int(load_library().wall_attn_decode_workspace_size(B, T_kv, HQ, H, V, chunk))
 
 
 def wall_attn_decode(q, p_curr, v, k_tilde, r_cache, T_kv, sink_bias=None, scale=None, chunk=64,
-                     out=None, lse=None, workspace=None):
-    """One decode step over cache rows [0, T_kv): o [B,1,HQ,V] (lse [B,1,HQ] if given)."""
+                     out=None, lse=None, workspace=None, seqlens=None):
+    """One decode step over cache rows [0, T_kv): o [B,1,HQ,V] (lse [B,1,HQ] if given).
+
+    seqlens: optional device int32 [B]; batch row b then attends rows
+    [0, seqlens[b]) (each in [1, T_kv]; T_kv is then the largest length).
+    """
     lib = load_library()
     B, cap, HQ, K = k_tilde.shape
     H, V = v.shape[2], v.shape[3]
@@ -235,6 +270,18 @@ def wall_attn_decode(q, p_curr, v, k_tilde, r_cache, T_kv, sink_bias=None, scale
     if workspace is None:
         workspace = torch.empty(max(wall_attn_decode_workspace_size(B, T_kv, HQ, H, V, chunk), 1),
                                 dtype=torch.uint8, device=q.device)
+    if seqlens is not None:
+        st = lib.wall_attn_decode_varlen(
+            _dev(q, "q", dt), _dev(p_curr, "p_curr", torch.float32),
+            _dev(v, "v", dt, (B, cap, H, V)), _dev(k_tilde, "k_tilde", dt),
+            _dev(r_cache, "r_cache", torch.float32),
+            _dev(sink_bias, "sink_bias", torch.float32, (HQ,)),
+            _dev(seqlens, "seqlens", torch.int32, (B,)), B, int(T_kv), cap, HQ, H, K, V,
+            int(chunk), _dtype_code(k_tilde), float(scale) if scale else 0.0,
+            _dev(out, "out", dt), _dev(lse, "lse", torch.float32), _dev(workspace, "workspace"),
+            workspace.numel() * workspace.element_size(), _stream(q.device))
+        _check(st, "wall_attn_decode_varlen")
+        return out
     st = lib.wall_attn_decode(
         _dev(q, "q", dt), _dev(p_curr, "p_curr", torch.float32), _dev(v, "v", dt, (B, cap, H, V)),
         _dev(k_tilde, "k_tilde", dt), _dev(r_cache, "r_cache", torch.float32),

@@ -287,17 +287,43 @@ wall_status_t wall_build_kv_cache(const void* k_new, const void* g_new, const fl
   return finish(wall::launch_cache_build(a, dt == WALL_DTYPE_BF16, st), st);
 }
 
+wall_status_t wall_append_kv_cache_varlen(const void* k_new, const void* g_new,
+                                          const float* p_prev, const int32_t* t_pos, int B,
+                                          int cap, int HQ, int H, int K, int chunk,
+                                          wall_dtype_t dt, void* k_tilde, float* r_cache,
+                                          float* p_last, wall_stream_t stream) {
+  if (B < 0 || cap < 1 || HQ <= 0 || H <= 0 || HQ % H != 0) return WALL_ERR_INVALID_ARG;
+  if (dt != WALL_DTYPE_F32 && dt != WALL_DTYPE_BF16) return WALL_ERR_INVALID_ARG;
+  if (!supported_dim(K)) return WALL_ERR_UNSUPPORTED;
+  if (chunk != 32 && chunk != 64 && chunk != 128) return WALL_ERR_UNSUPPORTED;
+  if (B == 0) return WALL_OK;
+  if (!k_new || !g_new || !p_prev || !t_pos || !k_tilde || !r_cache || !p_last)
+    return WALL_ERR_INVALID_ARG;
+  const size_t esz = dt == WALL_DTYPE_BF16 ? 2 : 4;
+  if (!aligned(k_new, 4 * esz) || !aligned(g_new, 4 * esz) || !aligned(k_tilde, 4 * esz) ||
+      !aligned(r_cache, 16) || !aligned(p_last, 16) || !aligned(p_prev, 16) || !aligned(t_pos, 4))
+    return WALL_ERR_INVALID_ARG;
+  wall::CacheArgs a;
+  a.k_new = k_new; a.g_new = g_new; a.p_prev = p_prev;
+  a.B = B; a.t_start = 0; a.T_new = 1; a.cap = cap; a.HQ = HQ; a.H = H; a.K = K;
+  a.chunk = chunk; a.k_tilde = k_tilde; a.r_cache = r_cache; a.p_last = p_last;
+  a.err = nullptr; a.wait_ns = 0; a.fault = 0;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(wall::launch_append_varlen(a, t_pos, dt == WALL_DTYPE_BF16, st), st);
+}
+
 size_t wall_attn_decode_workspace_size(int B, int T_kv, int HQ, int H, int V, int chunk) {
   if (B <= 0 || T_kv <= 0 || HQ <= 0 || H <= 0 || V <= 0 || chunk <= 0) return 0;
   const int ns = wall::decode_max_splits(B, T_kv, HQ, H, chunk);
   return wall::decode_workspace_bytes(B, HQ, V, ns);
 }
 
-wall_status_t wall_attn_decode(const void* q, const float* p_curr, const void* v,
-                               const void* k_tilde, const float* r_cache, const float* sink_bias,
-                               int B, int T_kv, int cap, int HQ, int H, int K, int V, int chunk,
-                               wall_dtype_t dt, float scale, void* o, float* lse, void* workspace,
-                               size_t workspace_bytes, wall_stream_t stream) {
+static wall_status_t decode_entry(const void* q, const float* p_curr, const void* v,
+                                  const void* k_tilde, const float* r_cache,
+                                  const float* sink_bias, const int32_t* seqlens, int B, int T_kv,
+                                  int cap, int HQ, int H, int K, int V, int chunk,
+                                  wall_dtype_t dt, float scale, void* o, float* lse,
+                                  void* workspace, size_t workspace_bytes, wall_stream_t stream) {
   if (B < 0 || T_kv < 1 || cap < T_kv || HQ <= 0 || H <= 0 || HQ % H != 0)
     return WALL_ERR_INVALID_ARG;
   if (dt != WALL_DTYPE_F32 && dt != WALL_DTYPE_BF16) return WALL_ERR_INVALID_ARG;
@@ -305,6 +331,7 @@ wall_status_t wall_attn_decode(const void* q, const float* p_curr, const void* v
   if (chunk != 32 && chunk != 64 && chunk != 128) return WALL_ERR_UNSUPPORTED;
   if (B == 0) return WALL_OK;
   if (!q || !p_curr || !v || !k_tilde || !r_cache || !o || !workspace) return WALL_ERR_INVALID_ARG;
+  if (seqlens && !aligned(seqlens, 4)) return WALL_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(p_curr, 16) || !aligned(v, 16) || !aligned(k_tilde, 16) ||
       !aligned(r_cache, 16) || !aligned(o, 16) || !aligned(workspace, 16) ||
       (sink_bias && !aligned(sink_bias, 4)) || (lse && !aligned(lse, 4)))
@@ -322,11 +349,33 @@ wall_status_t wall_attn_decode(const void* q, const float* p_curr, const void* v
   if (a.err == nullptr) return WALL_ERR_CUDA;
   a.wait_ns = wall::wait_limit_ns();
   a.fault = wall::fault_mode();
+  a.seqlens = seqlens;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   stage_event(0, st);
   const cudaError_t e = wall::launch_decode(a, dt == WALL_DTYPE_BF16, st);
   stage_event(2, st);
   return finish(e, st);
+}
+
+wall_status_t wall_attn_decode(const void* q, const float* p_curr, const void* v,
+                               const void* k_tilde, const float* r_cache, const float* sink_bias,
+                               int B, int T_kv, int cap, int HQ, int H, int K, int V, int chunk,
+                               wall_dtype_t dt, float scale, void* o, float* lse, void* workspace,
+                               size_t workspace_bytes, wall_stream_t stream) {
+  return decode_entry(q, p_curr, v, k_tilde, r_cache, sink_bias, nullptr, B, T_kv, cap, HQ, H, K,
+                      V, chunk, dt, scale, o, lse, workspace, workspace_bytes, stream);
+}
+
+wall_status_t wall_attn_decode_varlen(const void* q, const float* p_curr, const void* v,
+                                      const void* k_tilde, const float* r_cache,
+                                      const float* sink_bias, const int32_t* seqlens_kv, int B,
+                                      int max_T_kv, int cap, int HQ, int H, int K, int V,
+                                      int chunk, wall_dtype_t dt, float scale, void* o,
+                                      float* lse, void* workspace, size_t workspace_bytes,
+                                      wall_stream_t stream) {
+  if (B > 0 && seqlens_kv == nullptr) return WALL_ERR_INVALID_ARG;
+  return decode_entry(q, p_curr, v, k_tilde, r_cache, sink_bias, seqlens_kv, B, max_T_kv, cap, HQ,
+                      H, K, V, chunk, dt, scale, o, lse, workspace, workspace_bytes, stream);
 }
 
 wall_status_t wall_device_error(wall_stream_t stream) {

@@ -312,6 +312,56 @@ __global__ void __launch_bounds__(128) cache_segscan_kernel(
   p_last[static_cast<size_t>(bh) * KD + n] = carry;
 }
 
+// One-token append at a per-row position (batches whose sequences have
+// different lengths).  Thread: (batch row, query head, four channels).
+template <typename T, int KD>
+__global__ void __launch_bounds__(128) cache_append_varlen_kernel(
+    const T* __restrict__ k_new, const T* __restrict__ g_new, const float* __restrict__ p_prev,
+    const int* __restrict__ t_pos, int B, int cap, int HQ, int H, int C, T* __restrict__ k_tilde,
+    float* __restrict__ r_cache, float* __restrict__ p_last) {
+  constexpr int TPS = KD / 4;
+  const long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<long>(B) * HQ * TPS) return;
+  const int ch = static_cast<int>(idx % TPS) * 4;
+  const long bh = idx / TPS;
+  const int b = static_cast<int>(bh / HQ), hq = static_cast<int>(bh % HQ), kvh = hq / (HQ / H);
+  const int t = min(max(t_pos[b], 0), cap - 1);  // clamped to the cache
+  const int ncap = (cap + C - 1) / C;
+  Vec4<T> gv, kv;
+  gv.load(g_new + (static_cast<size_t>(b) * HQ + hq) * KD + ch);
+  kv.load(k_new + (static_cast<size_t>(b) * H + kvh) * KD + ch);
+  float g[4], k[4], P[4];
+  gv.get(g);
+  kv.get(k);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const float prev = t > 0 ? p_prev[static_cast<size_t>(bh) * KD + ch + c] : 0.f;
+    P[c] = fmaf(g[c], kLog2e, prev);
+  }
+  float* rr = r_cache + ((static_cast<size_t>(b) * ncap + t / C) * HQ + hq) * KD + ch;
+  if (t % C == 0) {
+    *reinterpret_cast<float4*>(rr) = make_float4(P[0], P[1], P[2], P[3]);  // new chunk anchor
+  } else {
+    const float4 R = *reinterpret_cast<const float4*>(rr);
+    k[0] *= ex2_approx(R.x - P[0]);
+    k[1] *= ex2_approx(R.y - P[1]);
+    k[2] *= ex2_approx(R.z - P[2]);
+    k[3] *= ex2_approx(R.w - P[3]);
+  }
+  Vec4<T>::store(k_tilde + ((static_cast<size_t>(b) * cap + t) * HQ + hq) * KD + ch, k);
+  *reinterpret_cast<float4*>(p_last + static_cast<size_t>(bh) * KD + ch) =
+      make_float4(P[0], P[1], P[2], P[3]);
+}
+
+template <typename T, int KD>
+cudaError_t append_varlen_impl(const CacheArgs& a, const int* t_pos, cudaStream_t st) {
+  const long n = static_cast<long>(a.B) * a.HQ * (KD / 4);
+  cache_append_varlen_kernel<T, KD><<<static_cast<unsigned>((n + 127) / 128), 128, 0, st>>>(
+      static_cast<const T*>(a.k_new), static_cast<const T*>(a.g_new), a.p_prev, t_pos, a.B, a.cap,
+      a.HQ, a.H, a.chunk, static_cast<T*>(a.k_tilde), a.r_cache, a.p_last);
+  return cudaGetLastError();
+}
+
 template <typename T, int KD>
 cudaError_t cache_impl(const CacheArgs& a, cudaStream_t st) {
   using CC = CacheCfg<T, KD>;
@@ -395,6 +445,15 @@ cudaError_t cache_impl(const CacheArgs& a, cudaStream_t st) {
 }
 
 }  // namespace
+
+cudaError_t launch_append_varlen(const CacheArgs& a, const int* t_pos, bool bf16, cudaStream_t st) {
+  if (bf16) {
+    return a.K == 64 ? append_varlen_impl<__nv_bfloat16, 64>(a, t_pos, st)
+                     : append_varlen_impl<__nv_bfloat16, 128>(a, t_pos, st);
+  }
+  return a.K == 64 ? append_varlen_impl<float, 64>(a, t_pos, st)
+                   : append_varlen_impl<float, 128>(a, t_pos, st);
+}
 
 cudaError_t launch_cache_build(const CacheArgs& a, bool bf16, cudaStream_t st) {
   if (bf16) return a.K == 64 ? cache_impl<__nv_bfloat16, 64>(a, st) : cache_impl<__nv_bfloat16, 128>(a, st);

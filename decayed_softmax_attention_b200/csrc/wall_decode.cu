@@ -91,7 +91,7 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
     const T* __restrict__ q, const float* __restrict__ p_curr, const float* __restrict__ r_cache,
     int T_kv, int cap, int HQ, int C, int cps, int nsplit, float sc, float* __restrict__ part,
-    int* err, uint64_t wait_ns, int fault) {
+    int* err, uint64_t wait_ns, int fault, const int* __restrict__ seqlens) {
   using D = DecCfg<T, KD, VD, G>;
   constexpr int LPH = 32 / G;    // lanes per query head
   constexpr int CPL = KD / LPH;  // k_tilde channels per lane
@@ -105,12 +105,15 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
 
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nchunks = (T_kv + C - 1) / C;
+  // rows of this batch row's cache: all T_kv, or its own length (clamped to
+  // [1, T_kv]); splits past the end of a shorter row hold no rows
+  const int T_b = seqlens ? max(1, min(seqlens[b], T_kv)) : T_kv;
+  const int nchunks = (T_b + C - 1) / C;
   const int ncap = (cap + C - 1) / C;
   const int ck0 = s * cps;
   const int ck1 = min(ck0 + cps, nchunks);
   const int row_begin = ck0 * C;
-  const int row_end = min(ck1 * C, T_kv);
+  const int row_end = min(ck1 * C, T_b);
   const int nst = row_end > row_begin ? (row_end - row_begin + D::SR - 1) / D::SR : 0;
 
   if (threadIdx.x == 0) {
@@ -340,7 +343,7 @@ cudaError_t decode_impl(const DecodeArgs& a, cudaStream_t st) {
   dim3 grid(a.nsplit, a.H, a.B);
   kern<<<grid, (D::NW + 1) * 32, D::SMEM, st>>>(
       tmK, tmV, static_cast<const T*>(a.q), a.p_curr, a.r_cache, a.T_kv, a.cap, a.HQ, a.chunk,
-      cps, a.nsplit, a.scale * kLog2e, a.part, a.err, a.wait_ns, a.fault);
+      cps, a.nsplit, a.scale * kLog2e, a.part, a.err, a.wait_ns, a.fault, a.seqlens);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (a.mid_event != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(a.mid_event), st);

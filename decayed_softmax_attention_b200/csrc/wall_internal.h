@@ -93,6 +93,8 @@ struct CacheArgs {
   int fault;         // testing hook: 3 = producer skips its first stage
 };
 cudaError_t launch_cache_build(const CacheArgs& a, bool bf16, cudaStream_t st);
+// One token per batch row at row b's own position t_pos[b] (device int32 [B]).
+cudaError_t launch_append_varlen(const CacheArgs& a, const int* t_pos, bool bf16, cudaStream_t st);
 
 struct DecodeArgs {
   const void* q;
@@ -111,6 +113,7 @@ struct DecodeArgs {
   int* err;         // device error word
   uint64_t wait_ns; // bounded-wait limit
   int fault;        // testing hook: 2 = producer skips its first stage
+  const int* seqlens = nullptr;  // optional device int32 [B]: rows of each batch row's cache
 };
 int decode_max_splits(int B, int T_kv, int HQ, int H, int chunk);
 int decode_num_splits(int B, int T_kv, int HQ, int H, int chunk);

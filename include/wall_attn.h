@@ -142,6 +142,24 @@ wall_status_t wall_build_kv_cache(const void* k_new, const void* g_new, const fl
                                   float* p_last, wall_stream_t stream);
 
 /*
+ * One-token append per batch row at that row's own position (SURVEY next row:
+ * per-sequence cache lengths; Wall Attention README, "Decode" append): for each
+ * b, row t = t_pos[b] of the cache gets k_tilde from k_new[b] and g_new[b];
+ * a chunk starting at t gets its anchor; p_last[b] = P at row t.
+ *   k_new [B, 1, H, K], g_new [B, 1, HQ, K]  dtype dt
+ *   p_prev [B, HQ, K] fp32  P at row t_pos[b] - 1 (ignored where t_pos[b] == 0)
+ *   t_pos  device int32 [B], values in [0, cap) (clamped on the device); a row
+ *          appended inside a chunk needs that chunk's anchor already written
+ *   k_tilde, r_cache, chunk as for wall_build_kv_cache; p_last may alias p_prev
+ * Use with wall_attn_decode_varlen (seqlens_kv[b] = t_pos[b] + 1).
+ */
+wall_status_t wall_append_kv_cache_varlen(const void* k_new, const void* g_new,
+                                          const float* p_prev, const int32_t* t_pos, int B,
+                                          int cap, int HQ, int H, int K, int chunk,
+                                          wall_dtype_t dt, void* k_tilde, float* r_cache,
+                                          float* p_last, wall_stream_t stream);
+
+/*
  * Single-step decode over the pre-rescaled cache (Wall Attention README,
  * "Decode"): the current query attends cache rows 0 .. T_kv - 1 (the current
  * token included: append first, then attend):
@@ -169,6 +187,25 @@ wall_status_t wall_attn_decode(const void* q, const float* p_curr, const void* v
                                int B, int T_kv, int cap, int HQ, int H, int K, int V, int chunk,
                                wall_dtype_t dt, float scale, void* o, float* lse, void* workspace,
                                size_t workspace_bytes, wall_stream_t stream);
+
+/*
+ * Decode over a batch whose cached sequences have different lengths (SURVEY
+ * next row: per-sequence cache lengths; the README's decode takes one length
+ * for the batch).  Same as wall_attn_decode except:
+ *   seqlens_kv  device int32 [B]: batch row b attends its cache rows
+ *               0 .. seqlens_kv[b] - 1; values must lie in [1, max_T_kv]
+ *               (they are clamped to it on the device)
+ *   max_T_kv    the largest length (<= cap); size the workspace with
+ *               wall_attn_decode_workspace_size(B, max_T_kv, HQ, H, V, chunk)
+ * p_curr[b] must be P at row seqlens_kv[b] - 1 of that row.
+ */
+wall_status_t wall_attn_decode_varlen(const void* q, const float* p_curr, const void* v,
+                                      const void* k_tilde, const float* r_cache,
+                                      const float* sink_bias, const int32_t* seqlens_kv, int B,
+                                      int max_T_kv, int cap, int HQ, int H, int K, int V,
+                                      int chunk, wall_dtype_t dt, float scale, void* o,
+                                      float* lse, void* workspace, size_t workspace_bytes,
+                                      wall_stream_t stream);
 
 /*
  * Decode without scratch allocation (no counterpart in the paper: this entry

@@ -197,3 +197,38 @@ def test_product_path_never_imports_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in text.lower().replace("oracle/", ""), f
+
+
+def test_decode_varlen_host_validation(lib):
+    def dv(**kw):
+        a = dict(q=_fake(), pc=_fake(), v=_fake(), kt=_fake(), r=_fake(), sink=None,
+                 lens=_fake(0x5000), B=2, Tkv=100, cap=128, HQ=8, H=2, K=128, V=128, C=64,
+                 dt=BF16, scale=0.0, o=_fake(), lse=None, ws=_fake(), wsb=1 << 40, stream=None)
+        a.update(kw)
+        return lib.wall_attn_decode_varlen(
+            a["q"], a["pc"], a["v"], a["kt"], a["r"], a["sink"], a["lens"], a["B"], a["Tkv"],
+            a["cap"], a["HQ"], a["H"], a["K"], a["V"], a["C"], a["dt"], a["scale"], a["o"],
+            a["lse"], a["ws"], a["wsb"], a["stream"])
+    assert dv(lens=None) == INVALID                       # the lengths are required
+    assert dv(lens=_fake(0x5002)) == INVALID              # int32 alignment
+    assert dv(Tkv=200) == INVALID                         # largest length beyond the cache
+    assert dv(HQ=96, H=3) == UNSUPPORTED
+    assert dv(wsb=16) == WORKSPACE
+    assert dv(B=0, lens=None) == 0                        # empty batch: no-op
+
+
+def test_append_varlen_host_validation(lib):
+    def av(**kw):
+        a = dict(k=_fake(), g=_fake(), pp=_fake(), tp=_fake(0x6000), B=2, cap=64, HQ=4, H=2,
+                 K=64, C=64, dt=BF16, kt=_fake(), r=_fake(), pl=_fake(), stream=None)
+        a.update(kw)
+        return lib.wall_append_kv_cache_varlen(a["k"], a["g"], a["pp"], a["tp"], a["B"], a["cap"],
+                                               a["HQ"], a["H"], a["K"], a["C"], a["dt"], a["kt"],
+                                               a["r"], a["pl"], a["stream"])
+    assert av(tp=None) == INVALID
+    assert av(pp=None) == INVALID
+    assert av(C=48) == UNSUPPORTED
+    assert av(K=80) == UNSUPPORTED
+    assert av(HQ=3) == INVALID
+    assert av(r=_fake(0x1004)) == INVALID
+    assert av(B=0) == 0

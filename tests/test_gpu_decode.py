@@ -123,6 +123,71 @@ def test_prefill_emits_decode_cache(wall, dtype, B, T, HQ, H, K, V, chunk, gs):
         assert_close(od[:, 0], ro, spec.torch_dtype, "decode after emitted cache")
 
 
+@pytest.mark.parametrize("dtype,lens,HQ,H,K,V", [
+    ("bf16", (100, 37, 200, 1, 129), 8, 2, 128, 128),
+    ("f32", (64, 65, 3), 4, 4, 64, 64),
+    ("bf16", (300, 5), 16, 1, 64, 128),
+])
+def test_decode_varlen_matches_prefill_rows(wall, dtype, lens, HQ, H, K, V):
+    """Per-sequence cache lengths: batch row b attends rows [0, lens[b]) of one shared cache
+    and must equal the prefill row lens[b] - 1 of its sequence."""
+    B, T = len(lens), max(lens)
+    spec, d = _inputs(B, T, HQ, H, K, V, dtype, seed=51, sink=True)
+    cache = wall.KVCache(B, T + 4, HQ, H, K, V, dtype=spec.torch_dtype, chunk=64)
+    cache.append(d["k"], d["g"], d["v"])
+    _, _, P = oracle.kv_cache(d["k"], d["g"], chunk=64, threads=ORACLE_THREADS)
+    p_curr = torch.tensor(np.stack([P[b, L - 1] for b, L in enumerate(lens)]),
+                          dtype=torch.float32, device="cuda")[:, None].contiguous()
+    q = torch.stack([d["q"][b, L - 1] for b, L in enumerate(lens)])[:, None].contiguous()
+    seqlens = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    lse = torch.empty((B, 1, HQ), dtype=torch.float32, device="cuda")
+    o = wall.wall_attn_decode(q, p_curr, cache.v, cache.k_tilde, cache.r_cache, T,
+                              sink_bias=d["sink_bias"], scale=d["scale"], lse=lse, seqlens=seqlens)
+    rows = [b * T + L - 1 for b, L in enumerate(lens)]
+    ro, rl = oracle.wall_fwd(d["q"], d["k"], d["v"], d["g"], sink_bias=d["sink_bias"],
+                             scale=d["scale"], rows=rows, threads=ORACLE_THREADS)
+    assert_close(o[:, 0], ro, spec.torch_dtype, "varlen decode")
+    np.testing.assert_allclose(lse[:, 0].double().cpu().numpy(), rl, rtol=1e-3, atol=1e-3)
+
+
+@pytest.mark.parametrize("dtype,start,HQ,H,K,V,steps", [
+    ("bf16", (60, 130, 1, 64), 8, 2, 128, 128, 12),
+    ("f32", (31, 2), 4, 4, 64, 64, 6),
+])
+def test_varlen_streaming_append_and_decode(wall, dtype, start, HQ, H, K, V, steps):
+    """A batch whose sequences have different lengths: per-row appends at each row's own
+    position, then a per-row-length decode; every step must equal the prefill row of the
+    token just appended, for every sequence."""
+    B, T = len(start), max(start) + steps
+    spec, d = _inputs(B, T, HQ, H, K, V, dtype, seed=61, sink=True)
+    C = 64
+    cap = T + 2
+    dt = spec.torch_dtype
+    kt = torch.zeros((B, cap, HQ, K), dtype=dt, device="cuda")
+    rc = torch.zeros((B, (cap + C - 1) // C, HQ, K), dtype=torch.float32, device="cuda")
+    p = torch.zeros((B, HQ, K), dtype=torch.float32, device="cuda")
+    vc = torch.zeros((B, cap, H, V), dtype=dt, device="cuda")
+    for b, L in enumerate(start):  # each row's own prefix, built through a one-row view
+        wall.wall_build_kv_cache(d["k"][b:b + 1, :L].contiguous(), d["g"][b:b + 1, :L].contiguous(),
+                                 kt[b:b + 1], rc[b:b + 1], p[b:b + 1], chunk=C)
+        vc[b, :T].copy_(d["v"][b])
+    lens = list(start)
+    for s_ in range(steps):
+        t_pos = torch.tensor(lens, dtype=torch.int32, device="cuda")
+        k_new = torch.stack([d["k"][b, L] for b, L in enumerate(lens)])[:, None].contiguous()
+        g_new = torch.stack([d["g"][b, L] for b, L in enumerate(lens)])[:, None].contiguous()
+        wall.wall_append_kv_cache_varlen(k_new, g_new, kt, rc, p, t_pos, chunk=C)
+        q = torch.stack([d["q"][b, L] for b, L in enumerate(lens)])[:, None].contiguous()
+        o = wall.wall_attn_decode(q, p[:, None].contiguous(), vc, kt, rc, max(lens) + 1,
+                                  sink_bias=d["sink_bias"], scale=d["scale"], chunk=C,
+                                  seqlens=t_pos + 1)
+        rows = [b * T + L for b, L in enumerate(lens)]
+        ro, _ = oracle.wall_fwd(d["q"], d["k"], d["v"], d["g"], sink_bias=d["sink_bias"],
+                                scale=d["scale"], rows=rows, threads=ORACLE_THREADS)
+        assert_close(o[:, 0], ro, dt, f"varlen step {s_}")
+        lens = [L + 1 for L in lens]
+
+
 STREAM = [
     dict(B=2, T0=200, steps=24, HQ=8, H=2, K=128, V=128, dtype="bf16", sink=True),
     dict(B=3, T0=130, steps=10, HQ=4, H=4, K=64, V=64, dtype="bf16", sink=False),
