@@ -52,11 +52,11 @@ TRAFFIC = {
     # profiles/wall_fwd_tc_long_prefill.md: 316.535808 MB read + 43.428608 MB written
     "prefill_main": {"bytes": 359964416, "source_sha": "820590f83f572f63"},
     # profiles/decode_split_b4_tkv32k.md, batch 4 scaled by 8 to batch 32 (traffic is
-    # proportional to the batch): (1.376462 GB + 5.344000 MB) * 8
-    "decode_split": {"bytes": 11054448000, "source_sha": "c266b24bc4b2797d"},
-    # profiles/cache_build_b4_t32k.md, batch 4 scaled by 8 to batch 32:
-    # (1.342212 GB + 1.070139 GB) * 8
-    "cache_build": {"bytes": 19298808000, "source_sha": "c4f6efa03b7cc36b"},
+    # proportional to the batch): (1.376487 GB + 5.113088 MB) * 8
+    "decode_split": {"bytes": 11052800704, "source_sha": "9d68ac5ccdae419f"},
+    # profiles/cache_build_b4_t32k.md, full-size capture (batch 32, 1-pass DRAM metrics):
+    # 10737913088 B read + 8820278528 B written
+    "cache_build": {"bytes": 19558191616, "source_sha": "b5fa331d20089736"},
 }
 KERNEL_SOURCES = {
     "prefill_main": "decayed_softmax_attention_b200/csrc/wall_fwd_tc.cu",
