@@ -11,6 +11,7 @@ the exact formulas and the readings taken where the page is silent):
   wall_fwd           -- prefill forward by the pairwise definition
   kv_cache           -- P, r_cache and k_tilde of the "Decode" section
   decode_from_cache  -- one decode step over (k_tilde, r_cache)
+  wall_bwd           -- gradients of the prefill forward (analytic, by the definition)
 """
 from __future__ import annotations
 
@@ -52,7 +53,10 @@ def _load():
     lib.wall_oracle_fwd.argtypes = [P, P, P, P, P, P, i, P, i, i, i, i, i, i, i, d, P, i64, P, P, i]
     lib.wall_oracle_kv_cache.argtypes = [P, P, i, i, i, i, i, i, P, P, P, P, i]
     lib.wall_oracle_decode_cache.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, i, i, d, P, P, i]
-    for f in (lib.wall_oracle_fwd, lib.wall_oracle_kv_cache, lib.wall_oracle_decode_cache):
+    lib.wall_oracle_bwd.argtypes = [P, P, P, P, P, P, i, P, i, i, i, i, i, i, i, d, P, P,
+                                    P, P, P, P, P, P, i]
+    for f in (lib.wall_oracle_fwd, lib.wall_oracle_kv_cache, lib.wall_oracle_decode_cache,
+              lib.wall_oracle_bwd):
         f.restype = ctypes.c_int
     lib.wall_oracle_max_threads.restype = ctypes.c_int
     _lib = lib
@@ -169,3 +173,43 @@ def decode_from_cache(q, p_curr, v, k_tilde, r_cache, T_kv, sink_bias=None, chun
     _check(rc, "decode_from_cache")
     return o, lse
 
+
+
+def wall_bwd(q, k, v, g, do, g_scalar=None, sink_bias=None, window=0, cu_seqlens=None,
+             scale=None, dlse=None, threads=0):
+    """Gradients of the prefill forward (double), by differentiating the definition.
+
+    Same inputs as ``wall_fwd`` plus do [B,T,HQ,V] (dL/do) and optional dlse [B,T,HQ].
+    Returns a dict: dq [B,T,HQ,K], dk [B,T,H,K], dv [B,T,H,V], dg [B,T,HQ,K],
+    dg_scalar [B,T,HQ] (None without g_scalar), dsink [HQ] (None without sink_bias).
+    dk and dv sum the query heads of each KV group; dsink sums the batch.
+    """
+    q, k, v, g, do = _f32(q), _f32(k), _f32(v), _f32(g), _f32(do)
+    gs, sink, dl = _f32(g_scalar), _f32(sink_bias), _f32(dlse)
+    B, T, HQ, K = q.shape
+    H, V = k.shape[2], v.shape[3]
+    cu = None
+    nseq = 0
+    if cu_seqlens is not None:
+        if hasattr(cu_seqlens, "detach"):
+            cu_seqlens = cu_seqlens.detach().cpu().numpy()
+        cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+        nseq = cu.shape[0] - 1
+    if scale is None or scale <= 0:
+        scale = K ** -0.5
+    dq = np.empty((B, T, HQ, K))
+    dkh = np.empty((B, T, HQ, K))
+    dvh = np.empty((B, T, HQ, V))
+    dg = np.empty((B, T, HQ, K))
+    dgs = np.empty((B, T, HQ)) if gs is not None else None
+    dsb = np.empty((B, HQ)) if sink is not None else None
+    rc = _load().wall_oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gs), _ptr(sink),
+                                 int(window or 0), _ptr(cu), nseq, B, T, HQ, H, K, V,
+                                 float(scale), _ptr(do), _ptr(dl), _ptr(dq), _ptr(dkh),
+                                 _ptr(dvh), _ptr(dg), _ptr(dgs), _ptr(dsb), int(threads))
+    _check(rc, "wall_bwd")
+    grp = HQ // H
+    dk = dkh.reshape(B, T, H, grp, K).sum(axis=3)
+    dv = dvh.reshape(B, T, H, grp, V).sum(axis=3)
+    return dict(dq=dq, dk=dk, dv=dv, dg=dg, dg_scalar=dgs,
+                dsink=None if dsb is None else dsb.sum(axis=0))

@@ -29,7 +29,10 @@
  *   - cumulative sums restart at every cu_seqlens document start;
  *   - query head hq reads KV head hq / (HQ / H);
  *   - lse is the natural-log normaliser, sink included;
- *   - the cache anchor is R_c = P[c*C], the chunk's first token.
+ *   - the cache anchor is R_c = P[c*C], the chunk's first token;
+ *   - the backward differentiates o (and, when given, lse) with respect to
+ *     every input; the sink gradient sums over the batch, k and v gradients
+ *     over the query heads of a KV group.
  *
  * Inputs are float32 arrays holding already-rounded values (bf16 or fp32);
  * every value is widened to double on use.  No blocking, fusion or reordering
@@ -261,6 +264,162 @@ int wall_oracle_decode_cache(const float* q, const double* p_curr, const float* 
       }
     }
     free(x);
+  }
+  return status;
+}
+
+/*
+ * Prefill backward, by differentiating the forward definition above (the
+ * README's intro and "Usage / Training-Prefill" sections define what is
+ * differentiated; its "code structure" section names the backward pass).
+ * With dO = dL/do and dl = dL/dlse (0 when dlse is NULL), per row t and head hq:
+ *   p_j = exp(x_j - lse), p_s = exp(sink - lse),  D = sum_c dO[t,c] o[t,c]
+ *   dx_j = p_j * (dO[t].v[j] - D + dl)                 (softmax Jacobian)
+ *   dq[t,n]   += scale dx_j k[j,n] exp(G[t,n] - G[j,n])
+ *   dk_h[j,n] += scale dx_j q[t,n] exp(G[t,n] - G[j,n])  (per query head)
+ *   dv_h[j,c] += p_j dO[t,c]
+ *   dG[t,n] += scale dx_j q[t,n] k[j,n] exp(...),  dG[j,n] -= the same term
+ *   dGs[t]  += dx_j,  dGs[j] -= dx_j
+ *   dsink_bh += p_s * (dl - D)                         (the sink's value is 0)
+ * and, G and Gs being inclusive prefix sums restarting at each document start,
+ *   dg[u] = sum_{w=u..e-1} dG[w],  dg_scalar[u] = sum_{w=u..e-1} dGs[w].
+ * Outputs (double): dq, dk_h, dg [B,T,HQ,K]; dv_h [B,T,HQ,V]; dg_scalar [B,T,HQ]
+ * (nullable); dsink_bh [B,HQ] (nullable).  dk_h and dv_h are per query head:
+ * the caller sums the heads of a KV group (and dsink_bh over b).
+ */
+int wall_oracle_bwd(const float* q, const float* k, const float* v, const float* g,
+                    const float* g_scalar, const float* sink, int window,
+                    const int32_t* cu_seqlens, int num_seqs, int B, int T, int HQ, int H,
+                    int K, int V, double scale, const float* dout, const float* dlse,
+                    double* dq, double* dk_h, double* dv_h, double* dg, double* dg_scalar,
+                    double* dsink_bh, int nthreads) {
+  if (B <= 0 || T <= 0 || HQ <= 0 || H <= 0 || K <= 0 || V <= 0 || HQ % H) return ORACLE_BAD_ARG;
+  if (cu_seqlens && (B != 1 || num_seqs <= 0 || cu_seqlens[0] != 0 || cu_seqlens[num_seqs] != T))
+    return ORACLE_BAD_ARG;
+  const int group = HQ / H;
+  set_threads(nthreads);
+  int status = ORACLE_OK;
+
+#pragma omp parallel
+  {
+    double* G = (double*)malloc(sizeof(double) * (size_t)T * K);
+    double* Gs = (double*)malloc(sizeof(double) * (size_t)T);
+    double* dG = (double*)malloc(sizeof(double) * (size_t)T * K);
+    double* dGs = (double*)malloc(sizeof(double) * (size_t)T);
+    double* x = (double*)malloc(sizeof(double) * (size_t)T);
+    double* orow = (double*)malloc(sizeof(double) * (size_t)V);
+    if (!G || !Gs || !dG || !dGs || !x || !orow) {
+#pragma omp atomic write
+      status = ORACLE_NO_MEM;
+    } else {
+#pragma omp for schedule(dynamic, 1)
+      for (int64_t bh = 0; bh < (int64_t)B * HQ; ++bh) {
+        const int b = (int)(bh / HQ), hq = (int)(bh % HQ), kv = hq / group;
+#define IDX_K(t) ((((size_t)b * T + (t)) * HQ + hq) * K)
+#define IDX_V(t) ((((size_t)b * T + (t)) * HQ + hq) * V)
+        for (int u = 0; u < T; ++u) {
+          int s, e;
+          doc_of(cu_seqlens, num_seqs, T, u, &s, &e);
+          const float* gu = g + IDX_K(u);
+          for (int n = 0; n < K; ++n) {
+            G[(size_t)u * K + n] = (u == s ? 0.0 : G[(size_t)(u - 1) * K + n]) + (double)gu[n];
+            dG[(size_t)u * K + n] = 0.0;
+            dq[IDX_K(u) + n] = 0.0;
+            dk_h[IDX_K(u) + n] = 0.0;
+          }
+          for (int c = 0; c < V; ++c) dv_h[IDX_V(u) + c] = 0.0;
+          const double gsu = g_scalar ? (double)g_scalar[((size_t)b * T + u) * HQ + hq] : 0.0;
+          Gs[u] = (u == s ? 0.0 : Gs[u - 1]) + gsu;
+          dGs[u] = 0.0;
+        }
+        double dsink = 0.0;
+        for (int t = 0; t < T; ++t) {
+          int s, e;
+          doc_of(cu_seqlens, num_seqs, T, t, &s, &e);
+          int j0 = s;
+          if (window > 0 && t - window + 1 > j0) j0 = t - window + 1;
+          const float* qt = q + IDX_K(t);
+          const float* dot_ = dout + IDX_V(t);
+          const double* Gt = G + (size_t)t * K;
+          /* forward again: logits, max, normaliser, output row */
+          double M = -INFINITY;
+          for (int j = j0; j <= t; ++j) {
+            const float* kj = k + (((size_t)b * T + j) * H + kv) * K;
+            const double* Gj = G + (size_t)j * K;
+            double dot = 0.0;
+            for (int n = 0; n < K; ++n) dot += (double)qt[n] * (double)kj[n] * exp(Gt[n] - Gj[n]);
+            x[j] = scale * dot + (Gs[t] - Gs[j]);
+            if (x[j] > M) M = x[j];
+          }
+          const double sb = sink ? (double)sink[hq] : -INFINITY;
+          if (sb > M) M = sb;
+          double Z = sink ? exp(sb - M) : 0.0;
+          for (int j = j0; j <= t; ++j) Z += exp(x[j] - M);
+          const double lse = M + log(Z);
+          for (int c = 0; c < V; ++c) orow[c] = 0.0;
+          for (int j = j0; j <= t; ++j) {
+            const double p = exp(x[j] - lse);
+            const float* vj = v + (((size_t)b * T + j) * H + kv) * V;
+            for (int c = 0; c < V; ++c) orow[c] += p * (double)vj[c];
+          }
+          double D = 0.0;
+          for (int c = 0; c < V; ++c) D += (double)dot_[c] * orow[c];
+          const double dl = dlse ? (double)dlse[((size_t)b * T + t) * HQ + hq] : 0.0;
+          /* backward through the softmax and the decayed scores */
+          for (int j = j0; j <= t; ++j) {
+            const double p = exp(x[j] - lse);
+            const float* kj = k + (((size_t)b * T + j) * H + kv) * K;
+            const float* vj = v + (((size_t)b * T + j) * H + kv) * V;
+            const double* Gj = G + (size_t)j * K;
+            double dP = 0.0;
+            for (int c = 0; c < V; ++c) dP += (double)dot_[c] * (double)vj[c];
+            const double dx = p * (dP - D + dl);
+            for (int c = 0; c < V; ++c) dv_h[IDX_V(j) + c] += p * (double)dot_[c];
+            for (int n = 0; n < K; ++n) {
+              const double w = scale * dx * exp(Gt[n] - Gj[n]);
+              dq[IDX_K(t) + n] += w * (double)kj[n];
+              dk_h[IDX_K(j) + n] += w * (double)qt[n];
+              const double term = w * (double)qt[n] * (double)kj[n];
+              dG[(size_t)t * K + n] += term;
+              dG[(size_t)j * K + n] -= term;
+            }
+            dGs[t] += dx;
+            dGs[j] -= dx;
+          }
+          if (sink) dsink += exp(sb - lse) * (dl - D);
+        }
+        /* reverse prefix sums inside each document */
+        for (int n = 0; n < K; ++n) {
+          double acc = 0.0;
+          for (int u = T - 1; u >= 0; --u) {
+            int s, e;
+            doc_of(cu_seqlens, num_seqs, T, u, &s, &e);
+            if (u == e - 1) acc = 0.0;
+            acc += dG[(size_t)u * K + n];
+            dg[IDX_K(u) + n] = acc;
+          }
+        }
+        if (dg_scalar) {
+          double acc = 0.0;
+          for (int u = T - 1; u >= 0; --u) {
+            int s, e;
+            doc_of(cu_seqlens, num_seqs, T, u, &s, &e);
+            if (u == e - 1) acc = 0.0;
+            acc += dGs[u];
+            dg_scalar[((size_t)b * T + u) * HQ + hq] = acc;
+          }
+        }
+        if (dsink_bh) dsink_bh[bh] = dsink;
+#undef IDX_K
+#undef IDX_V
+      }
+    }
+    free(G);
+    free(Gs);
+    free(dG);
+    free(dGs);
+    free(x);
+    free(orow);
   }
   return status;
 }

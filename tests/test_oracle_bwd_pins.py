@@ -1,0 +1,175 @@
+"""Pins for the oracle's backward pass, independent of its own formulation.
+
+The backward differentiates what the Wall Attention README defines (intro and
+"Usage / Training-Prefill" sections); its "code structure" and "Tests"
+sections name the backward kernel and check it with finite differences.  Here:
+  - central finite differences of the pure-Python brute-force forward (decay
+    as a product of per-step factors exp(g_u), no prefix sums anywhere), with
+    a loss L = sum(o * dO) + sum(lse * dlse), for every input including g,
+    g_scalar and the sink;
+  - g = 0 reduces to vanilla causal softmax attention: dq, dk, dv equal torch
+    autograd through a textbook dense attention in float64;
+  - invariants: shifting g (or g_scalar) at a document's first token changes
+    nothing, so its gradient there is zero; sum_j dv_j = sum_t (1 - p_sink) dO_t;
+  - a planted mistake in the analytic formula (on the CPU) is caught by the
+    finite-difference pin.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.test_oracle_pins import _brute, _inputs
+
+FD_H = 1e-5
+
+
+def _loss(d, do, dlse, window, cu, scale, **over):
+    a = {key: d[key] for key in ("q", "k", "v", "g", "g_scalar", "sink_bias")}
+    a.update(over)
+    o, lse = _brute(a["q"], a["k"], a["v"], a["g"], a["g_scalar"], a["sink_bias"], window, cu,
+                    scale)
+    val = float(np.sum(o * do))
+    if dlse is not None:
+        val += float(np.sum(lse * dlse))
+    return val
+
+
+def _fd_grad(d, name, do, dlse, window, cu, scale):
+    base = np.asarray(d[name], dtype=np.float64)
+    grad = np.zeros_like(base)
+    it = np.nditer(base, flags=["multi_index"])
+    for _ in it:
+        idx = it.multi_index
+        hi = base.copy()
+        lo = base.copy()
+        hi[idx] += FD_H
+        lo[idx] -= FD_H
+        grad[idx] = (_loss(d, do, dlse, window, cu, scale, **{name: hi}) -
+                     _loss(d, do, dlse, window, cu, scale, **{name: lo})) / (2 * FD_H)
+    return grad
+
+
+FD_CASES = [
+    dict(seed=11, B=1, T=7, HQ=2, H=1, K=3, V=2, gs=True, sink=True, dlse=True, window=0, cu=None),
+    dict(seed=12, B=2, T=6, HQ=2, H=2, K=2, V=3, gs=False, sink=False, dlse=False, window=3,
+         cu=None),
+    dict(seed=13, B=1, T=8, HQ=4, H=2, K=2, V=2, gs=True, sink=True, dlse=False, window=0,
+         cu=[0, 3, 8]),
+    dict(seed=14, B=1, T=8, HQ=2, H=1, K=3, V=2, gs=True, sink=False, dlse=True, window=4,
+         cu=[0, 5, 6, 8]),
+]
+
+
+def _fd_setup(case):
+    d = _inputs(case["seed"], B=case["B"], T=case["T"], HQ=case["HQ"], H=case["H"], K=case["K"],
+                V=case["V"], gscale=0.5, gs=case["gs"], sink=case["sink"])
+    # fp32-rounded values widened to double: the same point the oracle sees
+    d = {key: (None if val is None else val.astype(np.float64)) for key, val in d.items()}
+    rng = np.random.default_rng(case["seed"] + 100)
+    do = rng.standard_normal((case["B"], case["T"], case["HQ"], case["V"])).astype(np.float32)
+    dlse = (rng.standard_normal((case["B"], case["T"], case["HQ"])).astype(np.float32)
+            if case["dlse"] else None)
+    return d, do, dlse
+
+
+def _analytic(d, do, dlse, case, scale, fn=None):
+    fn = fn or oracle.wall_bwd
+    return fn(d["q"], d["k"], d["v"], d["g"], do, d["g_scalar"], d["sink_bias"],
+              window=case["window"], cu_seqlens=case["cu"], scale=scale, dlse=dlse)
+
+
+@pytest.mark.parametrize("case", FD_CASES)
+def test_gradients_match_finite_differences_of_brute_force(case):
+    d, do, dlse = _fd_setup(case)
+    scale = 0.7
+    got = _analytic(d, do, dlse, case, scale)
+    names = [("q", "dq"), ("k", "dk"), ("v", "dv"), ("g", "dg")]
+    if case["gs"]:
+        names.append(("g_scalar", "dg_scalar"))
+    if case["sink"]:
+        names.append(("sink_bias", "dsink"))
+    for inp, out in names:
+        fd = _fd_grad(d, inp, do.astype(np.float64),
+                      None if dlse is None else dlse.astype(np.float64), case["window"],
+                      case["cu"], scale)
+        np.testing.assert_allclose(got[out], fd, rtol=1e-6, atol=1e-7, err_msg=out)
+
+
+def _textbook_grads(q, k, v, do, scale, window, cu):
+    """torch autograd through dense masked softmax attention (float64), g = 0."""
+    B, T, HQ, K = q.shape
+    H = k.shape[2]
+    grp = HQ // H
+    doc = torch.zeros(T, dtype=torch.long)
+    if cu is not None:
+        for i in range(len(cu) - 1):
+            doc[cu[i]:cu[i + 1]] = i
+    i = torch.arange(T)[:, None]
+    j = torch.arange(T)[None, :]
+    allowed = (j <= i) & (doc[:, None] == doc[None, :])
+    if window > 0:
+        allowed &= (i - j) < window
+    tq = torch.tensor(q, dtype=torch.float64, requires_grad=True)
+    tk = torch.tensor(k, dtype=torch.float64, requires_grad=True)
+    tv = torch.tensor(v, dtype=torch.float64, requires_grad=True)
+    qh = tq.permute(0, 2, 1, 3)
+    kh = tk.permute(0, 2, 1, 3).repeat_interleave(grp, dim=1)
+    vh = tv.permute(0, 2, 1, 3).repeat_interleave(grp, dim=1)
+    o = torch.nn.functional.scaled_dot_product_attention(qh, kh, vh, attn_mask=allowed,
+                                                         scale=scale)
+    o.backward(torch.tensor(do, dtype=torch.float64).permute(0, 2, 1, 3))
+    return tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy()
+
+
+@pytest.mark.parametrize("case", [
+    dict(B=2, T=33, HQ=4, H=2, window=0, cu=None),
+    dict(B=1, T=40, HQ=3, H=1, window=6, cu=None),
+    dict(B=1, T=41, HQ=2, H=2, window=0, cu=[0, 1, 17, 30, 41]),
+])
+def test_g_zero_gradients_equal_textbook_attention(case):
+    d = _inputs(21, B=case["B"], T=case["T"], HQ=case["HQ"], H=case["H"], K=5, V=4)
+    rng = np.random.default_rng(22)
+    do = rng.standard_normal((case["B"], case["T"], case["HQ"], 4)).astype(np.float32)
+    g0 = np.zeros_like(d["g"])
+    got = oracle.wall_bwd(d["q"], d["k"], d["v"], g0, do, window=case["window"],
+                          cu_seqlens=case["cu"], scale=0.45)
+    dq, dk, dv = _textbook_grads(d["q"], d["k"], d["v"], do, 0.45, case["window"], case["cu"])
+    np.testing.assert_allclose(got["dq"], dq, rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(got["dk"], dk, rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(got["dv"], dv, rtol=1e-10, atol=1e-11)
+
+
+def test_document_start_gradients_vanish_and_value_gradients_sum():
+    cu = [0, 9, 10, 31, 48]
+    d = _inputs(31, B=1, T=48, HQ=4, H=2, K=6, V=5, gscale=0.4, gs=True, sink=True)
+    rng = np.random.default_rng(32)
+    do = rng.standard_normal((1, 48, 4, 5)).astype(np.float32)
+    got = oracle.wall_bwd(d["q"], d["k"], d["v"], d["g"], do, d["g_scalar"], d["sink_bias"],
+                          cu_seqlens=cu, scale=0.5)
+    big = np.abs(got["dg"]).max()
+    for s in cu[:-1]:
+        # g and g_scalar at a document's first token only shift every prefix of that document
+        assert np.abs(got["dg"][0, s]).max() < 1e-12 * max(1.0, big)
+        assert np.abs(got["dg_scalar"][0, s]).max() < 1e-12 * max(1.0, np.abs(got["dg_scalar"]).max())
+    # each row's weights sum to 1 - p_sink, so sum_j dv_j = sum_t (1 - p_sink_t) dO_t per KV head
+    _, lse = oracle.wall_fwd(d["q"], d["k"], d["v"], d["g"], d["g_scalar"], d["sink_bias"],
+                             cu_seqlens=cu, scale=0.5)
+    keep = 1.0 - np.exp(d["sink_bias"][None, None, :] - lse)          # [B,T,HQ]
+    want = (keep[..., None] * do).reshape(1, 48, 2, 2, 5).sum(axis=(1, 3))
+    np.testing.assert_allclose(got["dv"].sum(axis=1), want, rtol=1e-11, atol=1e-11)
+
+
+def test_planted_mistake_is_caught_by_finite_differences():
+    """Drop the key-side decay term from the analytic dg (a plausible slip)."""
+    case = FD_CASES[0]
+    d, do, dlse = _fd_setup(case)
+    scale = 0.7
+    good = _analytic(d, do, dlse, case, scale)
+    fd = _fd_grad(d, "g", do.astype(np.float64), dlse.astype(np.float64), case["window"],
+                  case["cu"], scale)
+    np.testing.assert_allclose(good["dg"], fd, rtol=1e-6, atol=1e-7)
+    # the mistaken gradient keeps only the query-side term q * dq, prefix-summed backwards
+    wrong_dG = np.asarray(d["q"]) * good["dq"]
+    wrong = np.flip(np.cumsum(np.flip(wrong_dG, axis=1), axis=1), axis=1)
+    assert np.abs(wrong - fd).max() > 1e-3
