@@ -26,8 +26,8 @@ import torch
 __all__ = [
     "WallError", "lib_path", "load_library", "wall_attn_fwd", "wall_attn_fwd_workspace_size",
     "wall_build_kv_cache", "wall_attn_decode", "wall_attn_decode_workspace_size",
-    "wall_attn_decode_noalloc", "wall_append_kv_cache_varlen",
-    "wall_device_error", "wall_debug_set_fault", "wall_debug_set_stage_events", "KVCache",
+    "wall_attn_decode_noalloc", "wall_append_kv_cache_varlen", "wall_attn_bwd",
+    "wall_attn_bwd_workspace_size", "wall_device_error", "wall_debug_set_fault", "wall_debug_set_stage_events", "KVCache",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -47,7 +47,7 @@ EXPORTED_SYMBOLS = (
     "wall_build_kv_cache", "wall_attn_decode_workspace_size", "wall_attn_decode",
     "wall_device_error", "wall_debug_set_fault", "wall_debug_set_stage_events",
     "wall_attn_decode_noalloc", "wall_attn_fwd_with_cache", "wall_attn_decode_varlen",
-    "wall_append_kv_cache_varlen",
+    "wall_append_kv_cache_varlen", "wall_attn_bwd_workspace_size", "wall_attn_bwd",
 )
 
 
@@ -86,6 +86,11 @@ def load_library():
     lib.wall_attn_fwd_with_cache.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P, P,
                                              P, S, I, I, P, P, P, P]
     lib.wall_attn_fwd_with_cache.restype = I
+    lib.wall_attn_bwd_workspace_size.argtypes = [I, I, I, I, I, I, I]
+    lib.wall_attn_bwd_workspace_size.restype = S
+    lib.wall_attn_bwd.argtypes = [P, P, P, P, P, P, I, P, I, I, I, I, I, I, I, I, F, P, P, P, P,
+                                  P, P, P, P, P, P, P, S, P]
+    lib.wall_attn_bwd.restype = I
     lib.wall_build_kv_cache.argtypes = [P, P, P, I, I, I, I, I, I, I, I, I, P, P, P, P]
     lib.wall_build_kv_cache.restype = I
     lib.wall_append_kv_cache_varlen.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P, P, P, P]
@@ -204,6 +209,58 @@ def wall_attn_fwd(q, k, v, g, g_scalar=None, sink_bias=None, window=0, cu_seqlen
         workspace.numel() * workspace.element_size(), _stream(q.device))
     _check(st, "wall_attn_fwd")
     return (out, lse) if return_lse else out
+
+
+def wall_attn_bwd_workspace_size(B, T, HQ, H, K, V, dtype) -> int:
+    code = WALL_DTYPE_BF16 if dtype == torch.bfloat16 else WALL_DTYPE_F32
+    return int(load_library().wall_attn_bwd_workspace_size(B, T, HQ, H, K, V, code))
+
+
+def wall_attn_bwd(q, k, v, g, o, lse, do, g_scalar=None, sink_bias=None, window=0,
+                  cu_seqlens=None, scale=None, dlse=None, workspace=None, grads=None):
+    """Prefill backward: gradients of a loss through o (and optionally lse).
+
+    o, lse: the forward's outputs for the same inputs; do [B,T,HQ,V] = dL/do;
+    dlse [B,T,HQ] fp32 or None.  Returns a dict with dq, dk, dv, dg (input dtype),
+    dg_scalar (with g_scalar) and dsink (fp32 [HQ], with sink_bias).  ``grads``: an
+    optional dict of preallocated outputs with those keys.
+    """
+    lib = load_library()
+    B, T, HQ, K = q.shape
+    H, V = k.shape[2], v.shape[3]
+    dt = q.dtype
+    code = _dtype_code(q)
+    dev = q.device
+    out = dict(grads or {})
+    shapes = dict(dq=(B, T, HQ, K), dk=(B, T, H, K), dv=(B, T, H, V), dg=(B, T, HQ, K))
+    if g_scalar is not None:
+        shapes["dg_scalar"] = (B, T, HQ)
+    for name, shp in shapes.items():
+        if out.get(name) is None:
+            out[name] = torch.empty(shp, dtype=dt, device=dev)
+    if sink_bias is not None and out.get("dsink") is None:
+        out["dsink"] = torch.empty((HQ,), dtype=torch.float32, device=dev)
+    need = wall_attn_bwd_workspace_size(B, T, HQ, H, K, V, dt)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    nseq = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    st = lib.wall_attn_bwd(
+        _dev(q, "q", dt), _dev(k, "k", dt, (B, T, H, K)), _dev(v, "v", dt, (B, T, H, V)),
+        _dev(g, "g", dt, (B, T, HQ, K)), _dev(g_scalar, "g_scalar", dt, (B, T, HQ)),
+        _dev(sink_bias, "sink_bias", torch.float32, (HQ,)), int(window or 0),
+        _dev(cu_seqlens, "cu_seqlens", torch.int32), nseq, B, T, HQ, H, K, V, code,
+        float(scale) if scale else 0.0, _dev(o, "o", dt, (B, T, HQ, V)),
+        _dev(lse, "lse", torch.float32, (B, T, HQ)), _dev(do, "do", dt, (B, T, HQ, V)),
+        _dev(dlse, "dlse", torch.float32, (B, T, HQ)),
+        *(_dev(out[n], n, dt, shapes[n]) for n in ("dq", "dk", "dv", "dg")),
+        _dev(out.get("dg_scalar"), "dg_scalar", dt, (B, T, HQ)),
+        _dev(out.get("dsink"), "dsink", torch.float32, (HQ,)),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(dev))
+    _check(st, "wall_attn_bwd")
+    out.setdefault("dg_scalar", None)
+    out.setdefault("dsink", None)
+    return out
 
 
 # ----------------------------------------------------------------- decode

@@ -258,6 +258,70 @@ wall_status_t wall_attn_fwd_with_cache(const void* q, const void* k, const void*
                   scale, o, lse, workspace, workspace_bytes, stream, &co);
 }
 
+size_t wall_attn_bwd_workspace_size(int B, int T, int HQ, int H, int K, int V, wall_dtype_t dt) {
+  (void)H;
+  if (B <= 0 || T <= 0 || HQ <= 0 || K <= 0 || V <= 0) return 0;
+  return wall::bwd_workspace_layout(B, T, HQ, K, V, dt == WALL_DTYPE_BF16, nullptr, nullptr,
+                                    nullptr);
+}
+
+wall_status_t wall_attn_bwd(const void* q, const void* k, const void* v, const void* g,
+                            const void* g_scalar, const float* sink_bias, int window,
+                            const int32_t* cu_seqlens, int num_seqs, int B, int T, int HQ, int H,
+                            int K, int V, wall_dtype_t dt, float scale, const void* o,
+                            const float* lse, const void* dout, const float* dlse, void* dq,
+                            void* dk, void* dv, void* dg, void* dg_scalar, float* dsink,
+                            void* workspace, size_t workspace_bytes, wall_stream_t stream) {
+  if (B < 0 || T < 0 || HQ <= 0 || H <= 0 || HQ % H != 0) return WALL_ERR_INVALID_ARG;
+  if (dt != WALL_DTYPE_F32 && dt != WALL_DTYPE_BF16) return WALL_ERR_INVALID_ARG;
+  if (!supported_dim(K) || !supported_dim(V)) return WALL_ERR_UNSUPPORTED;
+  if (cu_seqlens != nullptr && (B != 1 || num_seqs < 1)) return WALL_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) return WALL_OK;
+  const size_t esz = dt == WALL_DTYPE_BF16 ? 2 : 4;
+  if (!q || !k || !v || !g || !o || !lse || !dout || !dq || !dk || !dv || !dg || !workspace)
+    return WALL_ERR_INVALID_ARG;
+  if ((g_scalar == nullptr) != (dg_scalar == nullptr)) return WALL_ERR_INVALID_ARG;
+  if ((sink_bias == nullptr) != (dsink == nullptr)) return WALL_ERR_INVALID_ARG;
+  const void* a16[] = {q, k, v, g, o, dout, dq, dk, dv, dg};
+  for (const void* p : a16)
+    if (!aligned(p, 16)) return WALL_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256) || !aligned(lse, 4) || (dlse && !aligned(dlse, 4)) ||
+      (g_scalar && !aligned(g_scalar, esz)) || (dg_scalar && !aligned(dg_scalar, esz)) ||
+      (sink_bias && !aligned(sink_bias, 4)) || (dsink && !aligned(dsink, 4)) ||
+      (cu_seqlens && !aligned(cu_seqlens, 4)))
+    return WALL_ERR_INVALID_ARG;
+  const long long NB = (static_cast<long long>(T) + wall::kBlockRows - 1) / wall::kBlockRows;
+  if (NB * B * HQ > 0x7fffffffLL || static_cast<long long>(B) * T * HQ > 0x3fffffffLL)
+    return WALL_ERR_UNSUPPORTED;
+  const bool bf16 = dt == WALL_DTYPE_BF16;
+  const size_t need = wall::bwd_workspace_layout(B, T, HQ, K, V, bf16, nullptr, nullptr, nullptr);
+  if (workspace_bytes < need) return WALL_ERR_WORKSPACE;
+  if (!(scale > 0.f) || !std::isfinite(scale)) scale = 1.f / std::sqrt(static_cast<float>(K));
+
+  int* err = wall::device_error_word();
+  if (err == nullptr) return WALL_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+  wall::BwdArgs a;
+  wall::FwdArgs& f = a.f;
+  f.q = q; f.k = k; f.v = v; f.g = g; f.g_scalar = g_scalar; f.sink = sink_bias;
+  f.cu_seqlens = cu_seqlens; f.num_seqs = num_seqs; f.window = window > 0 ? window : 0;
+  f.B = B; f.T = T; f.HQ = HQ; f.H = H; f.K = K; f.V = V; f.NB = static_cast<int>(NB);
+  f.scale = scale; f.o = const_cast<void*>(o); f.lse = const_cast<float*>(lse); f.err = err;
+  f.wait_ns = wall::wait_limit_ns();
+  f.fault = g_fault_mode.load();
+  a.dout = dout; a.dlse = dlse;
+  a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dg_scalar = dg_scalar; a.dsink = dsink;
+  for (int i = 0; i < 3; ++i) a.ev[i] = g_stage_ev[i].load();
+  wall::FwdWork fw;
+  wall::BwdWork bw;
+  wall::bwd_workspace_layout(B, T, HQ, K, V, bf16, &fw, &bw, static_cast<char*>(workspace));
+
+  cudaError_t e = wall::launch_prep(f, fw, bf16, st);
+  if (e != cudaSuccess) return WALL_ERR_CUDA;
+  return finish(wall::launch_bwd(a, fw, bw, bf16, st), st);
+}
+
 wall_status_t wall_build_kv_cache(const void* k_new, const void* g_new, const float* p_prev,
                                   int B, int t_start, int T_new, int cap, int HQ, int H, int K,
                                   int chunk, wall_dtype_t dt, void* k_tilde, float* r_cache,

@@ -34,7 +34,7 @@ bool encode_tiled(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void
 //   ssa     [B*HQ][NB][4]  prefix of g_scalar * log2(e) before the block ([0] used)
 //   kx      [B*HQ][T][16]  bf16 key-side gate channels for the QK contraction:
 //           (hi, lo, 0, ..., 0) with hi + lo = ssl[t] / (scale * log2(e)), bf16 head/tail
-//   rowlo   [T]            first admitted key per row (packed documents only)
+//   rowlo   [NB*128]       first admitted key per row (packed documents only; rows < T set)
 struct FwdWork {
   void* qh;
   void* kh;
@@ -79,6 +79,52 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, const FwdWork& w, const CUtensorMap&
                           const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmKX,
                           cudaStream_t st);
 cudaError_t launch_fwd_simt(const FwdArgs& a, const FwdWork& w, cudaStream_t st);
+
+// Backward of the prefill.  Inputs as FwdArgs plus the forward's o and lse,
+// dO (and optional dlse); outputs dq, dk, dv, dg, dg_scalar (input dtype) and
+// dsink (fp32).
+struct BwdArgs {
+  FwdArgs f;            // forward inputs (f.o / f.lse: the forward's outputs)
+  const void* dout;     // [B, T, HQ, V]
+  const float* dlse;    // [B, T, HQ] or null
+  void* dq;             // [B, T, HQ, K]
+  void* dk;             // [B, T, H, K]
+  void* dv;             // [B, T, H, V]
+  void* dg;             // [B, T, HQ, K]
+  void* dg_scalar;      // [B, T, HQ] (with g_scalar)
+  float* dsink;         // [HQ] (with sink)
+  // optional cudaEvent_t recorded before the key-block contraction, between it
+  // and the query-block contraction, and after the latter (profiling hook)
+  void* ev[3] = {nullptr, nullptr, nullptr};
+};
+
+// Backward workspace (after the forward prepass's own FwdWork):
+//   rowt, colt, delta [B*HQ][NB*128] fp32 (padded rows: 16-byte aligned tiles);
+//   psd, rsA, rsB [B*HQ][T] fp32; accQ, accK [B*HQ][T][K] fp32;
+//   dvh [B*HQ][T][V] fp32; head, carry [B*HQ][NB][K+1]; sinkblk [B*HQ][NB].
+struct BwdWork {
+  float* rowt;   // Gs log2(e) - lse log2(e) per query row
+  float* colt;   // Gs log2(e) per key row (g_scalar only)
+  float* delta;  // dO.o - dlse
+  float* psd;
+  float* rsA;
+  float* rsB;
+  float* accQ;
+  float* accK;
+  float* dvh;
+  float* head;
+  float* carry;
+  float* sinkblk;
+};
+size_t bwd_workspace_layout(int B, int T, int HQ, int K, int V, bool bf16, FwdWork* fw,
+                            BwdWork* bw, char* base);
+// Everything after the prepass: bwd_pre, the two contraction kernels, the post
+// passes and the reductions.
+cudaError_t launch_bwd(const BwdArgs& a, const FwdWork& fw, const BwdWork& bw, bool bf16,
+                       cudaStream_t st);
+// The two bf16 tensor-core contraction kernels (key-block, query-block).
+cudaError_t launch_bwd_tc(const BwdArgs& a, const FwdWork& fw, const BwdWork& bw,
+                          cudaStream_t st);
 
 struct CacheArgs {
   const void* k_new;

@@ -301,7 +301,7 @@ size_t fwd_workspace_layout(int B, int T, int HQ, int K, bool bf16, FwdWork* w, 
   p->ssb = static_cast<float*>(take(BHQ * NB * 4));
   p->ssa = static_cast<float*>(take(BHQ * NB * 16));
   p->kx = take(BHQ * static_cast<size_t>(T) * 16 * 2);
-  p->rowlo = static_cast<int*>(take(static_cast<size_t>(T) * 4 + 16));
+  p->rowlo = static_cast<int*>(take(NB * kBlockRows * 4));  // padded: 128-row bulk copies
   return off;
 }
 

@@ -118,6 +118,40 @@ wall_status_t wall_attn_fwd_with_cache(const void* q, const void* k, const void*
                                        float* r_cache, float* p_last, wall_stream_t stream);
 
 /*
+ * Prefill backward (Wall Attention README, intro formula and "Usage /
+ * Training-Prefill"; its "code structure" section names the backward pass):
+ * the gradients of a loss L through o (and, optionally, lse) of
+ * wall_attn_fwd with respect to every input.  Same inputs and shapes as
+ * wall_attn_fwd, plus
+ *   o         [B, T, HQ, V]  dtype dt  the forward's output for these inputs
+ *   lse       [B, T, HQ]     fp32      the forward's lse (required)
+ *   dout      [B, T, HQ, V]  dtype dt  dL/do
+ *   dlse      [B, T, HQ]     fp32      nullable; dL/dlse (0 when NULL)
+ * and the outputs (all written in full, caller-owned):
+ *   dq        [B, T, HQ, K]  dtype dt
+ *   dk        [B, T, H,  K]  dtype dt  summed over the query heads of each KV group
+ *   dv        [B, T, H,  V]  dtype dt  likewise
+ *   dg        [B, T, HQ, K]  dtype dt
+ *   dg_scalar [B, T, HQ]     dtype dt  required iff g_scalar != NULL
+ *   dsink     [HQ]           fp32      required iff sink_bias != NULL; summed over B
+ *   workspace at least wall_attn_bwd_workspace_size(...) bytes, 256-byte
+ *             aligned, clobbered.
+ * The softmax statistics come from lse: o and lse must be those of the same
+ * inputs (the forward's own outputs).  Deterministic: no atomics, fixed
+ * reduction orders.  T == 0 (or B == 0) is a no-op returning WALL_OK.
+ */
+size_t wall_attn_bwd_workspace_size(int B, int T, int HQ, int H, int K, int V,
+                                    wall_dtype_t dt);
+
+wall_status_t wall_attn_bwd(const void* q, const void* k, const void* v, const void* g,
+                            const void* g_scalar, const float* sink_bias, int window,
+                            const int32_t* cu_seqlens, int num_seqs, int B, int T, int HQ,
+                            int H, int K, int V, wall_dtype_t dt, float scale, const void* o,
+                            const float* lse, const void* dout, const float* dlse, void* dq,
+                            void* dk, void* dv, void* dg, void* dg_scalar, float* dsink,
+                            void* workspace, size_t workspace_bytes, wall_stream_t stream);
+
+/*
  * Decode cache build / append (Wall Attention README, "Decode"):
  *   P = cumsum(g) * (1/ln 2);  k_tilde[j] = k[j] * exp2(R_c - P[j])
  * with one anchor vector R_c = P[c * chunk] per chunk of `chunk` tokens (the

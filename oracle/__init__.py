@@ -54,7 +54,7 @@ def _load():
     lib.wall_oracle_kv_cache.argtypes = [P, P, i, i, i, i, i, i, P, P, P, P, i]
     lib.wall_oracle_decode_cache.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, i, i, d, P, P, i]
     lib.wall_oracle_bwd.argtypes = [P, P, P, P, P, P, i, P, i, i, i, i, i, i, i, d, P, P,
-                                    P, P, P, P, P, P, i]
+                                    P, P, P, P, P, P, P, P, P, i]
     for f in (lib.wall_oracle_fwd, lib.wall_oracle_kv_cache, lib.wall_oracle_decode_cache,
               lib.wall_oracle_bwd):
         f.restype = ctypes.c_int
@@ -176,16 +176,23 @@ def decode_from_cache(q, p_curr, v, k_tilde, r_cache, T_kv, sink_bias=None, chun
 
 
 def wall_bwd(q, k, v, g, do, g_scalar=None, sink_bias=None, window=0, cu_seqlens=None,
-             scale=None, dlse=None, threads=0):
+             scale=None, dlse=None, o=None, lse=None, scales=False, threads=0):
     """Gradients of the prefill forward (double), by differentiating the definition.
 
     Same inputs as ``wall_fwd`` plus do [B,T,HQ,V] (dL/do) and optional dlse [B,T,HQ].
+    o [B,T,HQ,V] / lse [B,T,HQ] (optional): given forward results used in place of the
+    exact ones (in D = dO.o and p = exp(x - lse)); None: recomputed exactly.
     Returns a dict: dq [B,T,HQ,K], dk [B,T,H,K], dv [B,T,H,V], dg [B,T,HQ,K],
     dg_scalar [B,T,HQ] (None without g_scalar), dsink [HQ] (None without sink_bias).
     dk and dv sum the query heads of each KV group; dsink sums the batch.
+    scales=True adds "sigma": per output, the root of the sum of squares of the terms
+    each element sums (a scale for rounding-error tolerances, not a result), and
+    "sigma_abs": the same with each softmax-Jacobian factor dO.v - D + dlse taken as
+    |dO.v| + |D - dlse| (its size before that difference cancels; dv has no such factor).
     """
     q, k, v, g, do = _f32(q), _f32(k), _f32(v), _f32(g), _f32(do)
     gs, sink, dl = _f32(g_scalar), _f32(sink_bias), _f32(dlse)
+    o_in, lse_in = _f32(o), _f32(lse)
     B, T, HQ, K = q.shape
     H, V = k.shape[2], v.shape[3]
     cu = None
@@ -203,13 +210,35 @@ def wall_bwd(q, k, v, g, do, g_scalar=None, sink_bias=None, window=0, cu_seqlens
     dg = np.empty((B, T, HQ, K))
     dgs = np.empty((B, T, HQ)) if gs is not None else None
     dsb = np.empty((B, HQ)) if sink is not None else None
+    s2 = s2ptr = None
+    if scales:
+        s2 = [np.zeros((B, T, HQ, K)), np.zeros((B, T, HQ, K)), np.zeros((B, T, HQ, V)),
+              np.zeros((B, T, HQ, K)), np.zeros((B, T, HQ)), np.zeros((B, HQ)),
+              np.zeros((B, T, HQ, K)), np.zeros((B, T, HQ, K)), np.zeros((B, T, HQ, K)),
+              np.zeros((B, T, HQ)), np.zeros((B, HQ))]
+        s2ptr = (ctypes.c_void_p * 11)(*[a.ctypes.data for a in s2])
     rc = _load().wall_oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(gs), _ptr(sink),
                                  int(window or 0), _ptr(cu), nseq, B, T, HQ, H, K, V,
-                                 float(scale), _ptr(do), _ptr(dl), _ptr(dq), _ptr(dkh),
-                                 _ptr(dvh), _ptr(dg), _ptr(dgs), _ptr(dsb), int(threads))
+                                 float(scale), _ptr(do), _ptr(dl), _ptr(o_in), _ptr(lse_in),
+                                 _ptr(dq), _ptr(dkh),
+                                 _ptr(dvh), _ptr(dg), _ptr(dgs), _ptr(dsb),
+                                 None if s2ptr is None else ctypes.cast(s2ptr, ctypes.c_void_p),
+                                 int(threads))
     _check(rc, "wall_bwd")
     grp = HQ // H
     dk = dkh.reshape(B, T, H, grp, K).sum(axis=3)
     dv = dvh.reshape(B, T, H, grp, V).sum(axis=3)
-    return dict(dq=dq, dk=dk, dv=dv, dg=dg, dg_scalar=dgs,
-                dsink=None if dsb is None else dsb.sum(axis=0))
+    out = dict(dq=dq, dk=dk, dv=dv, dg=dg, dg_scalar=dgs,
+               dsink=None if dsb is None else dsb.sum(axis=0))
+    if scales:
+        out["sigma"] = dict(
+            dq=np.sqrt(s2[0]), dk=np.sqrt(s2[1].reshape(B, T, H, grp, K).sum(axis=3)),
+            dv=np.sqrt(s2[2].reshape(B, T, H, grp, V).sum(axis=3)), dg=np.sqrt(s2[3]),
+            dg_scalar=np.sqrt(s2[4]) if gs is not None else None,
+            dsink=np.sqrt(s2[5].sum(axis=0)) if sink is not None else None)
+        out["sigma_abs"] = dict(
+            dq=np.sqrt(s2[6]), dk=np.sqrt(s2[7].reshape(B, T, H, grp, K).sum(axis=3)),
+            dv=out["sigma"]["dv"], dg=np.sqrt(s2[8]),
+            dg_scalar=np.sqrt(s2[9]) if gs is not None else None,
+            dsink=np.sqrt(s2[10].sum(axis=0)) if sink is not None else None)
+    return out

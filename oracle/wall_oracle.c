@@ -286,13 +286,24 @@ int wall_oracle_decode_cache(const float* q, const double* p_curr, const float* 
  * Outputs (double): dq, dk_h, dg [B,T,HQ,K]; dv_h [B,T,HQ,V]; dg_scalar [B,T,HQ]
  * (nullable); dsink_bh [B,HQ] (nullable).  dk_h and dv_h are per query head:
  * the caller sums the heads of a KV group (and dsink_bh over b).
+ * o_in [B,T,HQ,V] and lse_in [B,T,HQ] (nullable) replace the recomputed forward
+ * output and normaliser in D and p: the backward evaluated from given forward
+ * results, as a backward kernel that receives them does.  NULL: exact values.
+ * s2 (nullable, 11 arrays): for every output element, the sum of the SQUARES of
+ * the terms it sums (a scale for rounding-error tolerances, not a result):
+ * s2[0] dq, s2[1] dk_h, s2[3] dg (reverse prefix sums of the squared dG terms),
+ * [B,T,HQ,K]; s2[2] dv_h [B,T,HQ,V]; s2[4] dg_scalar [B,T,HQ]; s2[5] dsink [B,HQ];
+ * s2[6..10]: the same for dq, dk_h, dg, dg_scalar, dsink with each term's
+ * dO.v[j] - D + dl replaced by |dO.v[j]| + |D - dl| (its size before that
+ * difference cancels).
  */
 int wall_oracle_bwd(const float* q, const float* k, const float* v, const float* g,
                     const float* g_scalar, const float* sink, int window,
                     const int32_t* cu_seqlens, int num_seqs, int B, int T, int HQ, int H,
                     int K, int V, double scale, const float* dout, const float* dlse,
-                    double* dq, double* dk_h, double* dv_h, double* dg, double* dg_scalar,
-                    double* dsink_bh, int nthreads) {
+                    const float* o_in, const float* lse_in, double* dq, double* dk_h,
+                    double* dv_h, double* dg, double* dg_scalar, double* dsink_bh,
+                    double* const* s2, int nthreads) {
   if (B <= 0 || T <= 0 || HQ <= 0 || H <= 0 || K <= 0 || V <= 0 || HQ % H) return ORACLE_BAD_ARG;
   if (cu_seqlens && (B != 1 || num_seqs <= 0 || cu_seqlens[0] != 0 || cu_seqlens[num_seqs] != T))
     return ORACLE_BAD_ARG;
@@ -306,9 +317,13 @@ int wall_oracle_bwd(const float* q, const float* k, const float* v, const float*
     double* Gs = (double*)malloc(sizeof(double) * (size_t)T);
     double* dG = (double*)malloc(sizeof(double) * (size_t)T * K);
     double* dGs = (double*)malloc(sizeof(double) * (size_t)T);
+    double* qG = (double*)malloc(sizeof(double) * (size_t)T * K);  /* squared dG terms */
+    double* qGs = (double*)malloc(sizeof(double) * (size_t)T);
+    double* aG = (double*)malloc(sizeof(double) * (size_t)T * K);  /* same, absolute */
+    double* aGs = (double*)malloc(sizeof(double) * (size_t)T);
     double* x = (double*)malloc(sizeof(double) * (size_t)T);
     double* orow = (double*)malloc(sizeof(double) * (size_t)V);
-    if (!G || !Gs || !dG || !dGs || !x || !orow) {
+    if (!G || !Gs || !dG || !dGs || !x || !orow || !qG || !qGs || !aG || !aGs) {
 #pragma omp atomic write
       status = ORACLE_NO_MEM;
     } else {
@@ -324,15 +339,22 @@ int wall_oracle_bwd(const float* q, const float* k, const float* v, const float*
           for (int n = 0; n < K; ++n) {
             G[(size_t)u * K + n] = (u == s ? 0.0 : G[(size_t)(u - 1) * K + n]) + (double)gu[n];
             dG[(size_t)u * K + n] = 0.0;
+            qG[(size_t)u * K + n] = aG[(size_t)u * K + n] = 0.0;
             dq[IDX_K(u) + n] = 0.0;
             dk_h[IDX_K(u) + n] = 0.0;
+            if (s2) s2[0][IDX_K(u) + n] = s2[1][IDX_K(u) + n] = 0.0;
+            if (s2) s2[6][IDX_K(u) + n] = s2[7][IDX_K(u) + n] = 0.0;
           }
-          for (int c = 0; c < V; ++c) dv_h[IDX_V(u) + c] = 0.0;
+          for (int c = 0; c < V; ++c) {
+            dv_h[IDX_V(u) + c] = 0.0;
+            if (s2) s2[2][IDX_V(u) + c] = 0.0;
+          }
+          qGs[u] = aGs[u] = 0.0;
           const double gsu = g_scalar ? (double)g_scalar[((size_t)b * T + u) * HQ + hq] : 0.0;
           Gs[u] = (u == s ? 0.0 : Gs[u - 1]) + gsu;
           dGs[u] = 0.0;
         }
-        double dsink = 0.0;
+        double dsink = 0.0, qsink = 0.0, asink = 0.0;
         for (int t = 0; t < T; ++t) {
           int s, e;
           doc_of(cu_seqlens, num_seqs, T, t, &s, &e);
@@ -355,12 +377,16 @@ int wall_oracle_bwd(const float* q, const float* k, const float* v, const float*
           if (sb > M) M = sb;
           double Z = sink ? exp(sb - M) : 0.0;
           for (int j = j0; j <= t; ++j) Z += exp(x[j] - M);
-          const double lse = M + log(Z);
+          const double lse = lse_in ? (double)lse_in[((size_t)b * T + t) * HQ + hq] : M + log(Z);
           for (int c = 0; c < V; ++c) orow[c] = 0.0;
-          for (int j = j0; j <= t; ++j) {
-            const double p = exp(x[j] - lse);
-            const float* vj = v + (((size_t)b * T + j) * H + kv) * V;
-            for (int c = 0; c < V; ++c) orow[c] += p * (double)vj[c];
+          if (o_in) {
+            for (int c = 0; c < V; ++c) orow[c] = (double)o_in[IDX_V(t) + c];
+          } else {
+            for (int j = j0; j <= t; ++j) {
+              const double p = exp(x[j] - lse);
+              const float* vj = v + (((size_t)b * T + j) * H + kv) * V;
+              for (int c = 0; c < V; ++c) orow[c] += p * (double)vj[c];
+            }
           }
           double D = 0.0;
           for (int c = 0; c < V; ++c) D += (double)dot_[c] * orow[c];
@@ -374,7 +400,11 @@ int wall_oracle_bwd(const float* q, const float* k, const float* v, const float*
             double dP = 0.0;
             for (int c = 0; c < V; ++c) dP += (double)dot_[c] * (double)vj[c];
             const double dx = p * (dP - D + dl);
-            for (int c = 0; c < V; ++c) dv_h[IDX_V(j) + c] += p * (double)dot_[c];
+            const double dxa = p * (fabs(dP) + fabs(D - dl));
+            for (int c = 0; c < V; ++c) {
+              dv_h[IDX_V(j) + c] += p * (double)dot_[c];
+              if (s2) s2[2][IDX_V(j) + c] += (p * (double)dot_[c]) * (p * (double)dot_[c]);
+            }
             for (int n = 0; n < K; ++n) {
               const double w = scale * dx * exp(Gt[n] - Gj[n]);
               dq[IDX_K(t) + n] += w * (double)kj[n];
@@ -382,34 +412,71 @@ int wall_oracle_bwd(const float* q, const float* k, const float* v, const float*
               const double term = w * (double)qt[n] * (double)kj[n];
               dG[(size_t)t * K + n] += term;
               dG[(size_t)j * K + n] -= term;
+              if (s2) {
+                const double wa = scale * dxa * exp(Gt[n] - Gj[n]);
+                const double ta = wa * (double)qt[n] * (double)kj[n];
+                s2[0][IDX_K(t) + n] += (w * (double)kj[n]) * (w * (double)kj[n]);
+                s2[1][IDX_K(j) + n] += (w * (double)qt[n]) * (w * (double)qt[n]);
+                s2[6][IDX_K(t) + n] += (wa * (double)kj[n]) * (wa * (double)kj[n]);
+                s2[7][IDX_K(j) + n] += (wa * (double)qt[n]) * (wa * (double)qt[n]);
+                qG[(size_t)t * K + n] += term * term;
+                qG[(size_t)j * K + n] += term * term;
+                aG[(size_t)t * K + n] += ta * ta;
+                aG[(size_t)j * K + n] += ta * ta;
+              }
             }
             dGs[t] += dx;
             dGs[j] -= dx;
+            qGs[t] += dx * dx;
+            qGs[j] += dx * dx;
+            aGs[t] += dxa * dxa;
+            aGs[j] += dxa * dxa;
           }
-          if (sink) dsink += exp(sb - lse) * (dl - D);
+          if (sink) {
+            const double ps = exp(sb - lse);
+            dsink += ps * (dl - D);
+            qsink += (ps * (dl - D)) * (ps * (dl - D));
+            asink += (ps * (fabs(dl) + fabs(D))) * (ps * (fabs(dl) + fabs(D)));
+          }
         }
         /* reverse prefix sums inside each document */
         for (int n = 0; n < K; ++n) {
-          double acc = 0.0;
+          double acc = 0.0, acc2 = 0.0, acc3 = 0.0;
           for (int u = T - 1; u >= 0; --u) {
             int s, e;
             doc_of(cu_seqlens, num_seqs, T, u, &s, &e);
-            if (u == e - 1) acc = 0.0;
+            if (u == e - 1) acc = acc2 = acc3 = 0.0;
             acc += dG[(size_t)u * K + n];
+            acc2 += qG[(size_t)u * K + n];
+            acc3 += aG[(size_t)u * K + n];
             dg[IDX_K(u) + n] = acc;
+            if (s2) {
+              s2[3][IDX_K(u) + n] = acc2;
+              s2[8][IDX_K(u) + n] = acc3;
+            }
           }
         }
         if (dg_scalar) {
-          double acc = 0.0;
+          double acc = 0.0, acc2 = 0.0, acc3 = 0.0;
           for (int u = T - 1; u >= 0; --u) {
             int s, e;
             doc_of(cu_seqlens, num_seqs, T, u, &s, &e);
-            if (u == e - 1) acc = 0.0;
+            if (u == e - 1) acc = acc2 = acc3 = 0.0;
             acc += dGs[u];
+            acc2 += qGs[u];
+            acc3 += aGs[u];
             dg_scalar[((size_t)b * T + u) * HQ + hq] = acc;
+            if (s2) {
+              s2[4][((size_t)b * T + u) * HQ + hq] = acc2;
+              s2[9][((size_t)b * T + u) * HQ + hq] = acc3;
+            }
           }
         }
         if (dsink_bh) dsink_bh[bh] = dsink;
+        if (s2) {
+          s2[5][bh] = qsink;
+          s2[10][bh] = asink;
+        }
 #undef IDX_K
 #undef IDX_V
       }
@@ -420,6 +487,10 @@ int wall_oracle_bwd(const float* q, const float* k, const float* v, const float*
     free(dGs);
     free(x);
     free(orow);
+    free(qG);
+    free(qGs);
+    free(aG);
+    free(aGs);
   }
   return status;
 }

@@ -232,3 +232,40 @@ def test_append_varlen_host_validation(lib):
     assert av(HQ=3) == INVALID
     assert av(r=_fake(0x1004)) == INVALID
     assert av(B=0) == 0
+
+
+def _bwd(lib, **kw):
+    a = dict(q=_fake(), k=_fake(), v=_fake(), g=_fake(), gs=None, sink=None, window=0, cu=None,
+             nseq=0, B=1, T=256, HQ=4, H=2, K=64, V=64, dt=BF16, scale=0.0, o=_fake(),
+             lse=_fake(), do=_fake(), dlse=None, dq=_fake(), dk=_fake(), dv=_fake(), dg=_fake(),
+             dgs=None, dsink=None, ws=_fake(0x100000), wsb=1 << 40, stream=None)
+    a.update(kw)
+    return lib.wall_attn_bwd(a["q"], a["k"], a["v"], a["g"], a["gs"], a["sink"], a["window"],
+                             a["cu"], a["nseq"], a["B"], a["T"], a["HQ"], a["H"], a["K"], a["V"],
+                             a["dt"], a["scale"], a["o"], a["lse"], a["do"], a["dlse"], a["dq"],
+                             a["dk"], a["dv"], a["dg"], a["dgs"], a["dsink"], a["ws"], a["wsb"],
+                             a["stream"])
+
+
+def test_bwd_host_validation(lib):
+    assert _bwd(lib, lse=None) == INVALID                 # the forward's lse is required
+    assert _bwd(lib, do=None) == INVALID
+    assert _bwd(lib, dg=None) == INVALID
+    assert _bwd(lib, gs=_fake()) == INVALID               # g_scalar without dg_scalar
+    assert _bwd(lib, dgs=_fake()) == INVALID              # dg_scalar without g_scalar
+    assert _bwd(lib, sink=_fake()) == INVALID             # sink without dsink
+    assert _bwd(lib, dq=_fake(0x1008)) == INVALID         # misaligned output
+    assert _bwd(lib, HQ=6, H=4) == INVALID
+    assert _bwd(lib, cu=_fake(), nseq=2, B=2) == INVALID  # packing needs B == 1
+    assert _bwd(lib, K=96) == UNSUPPORTED
+    assert _bwd(lib, dt=7) == INVALID
+    assert _bwd(lib, wsb=16) == WORKSPACE
+    assert _bwd(lib, T=0) == 0                            # empty input: no-op
+
+
+def test_bwd_workspace_size(lib):
+    fwd = lib.wall_attn_fwd_workspace_size(1, 1024, 8, 4, 64, 64, BF16)
+    bwd = lib.wall_attn_bwd_workspace_size(1, 1024, 8, 4, 64, 64, BF16)
+    # the prepass's workspace plus fp32 accumulators of dq, dk_h and dv_h
+    assert bwd >= fwd + 3 * 8 * 1024 * 64 * 4
+    assert lib.wall_attn_bwd_workspace_size(0, 1024, 8, 4, 64, 64, BF16) == 0

@@ -173,3 +173,21 @@ def test_planted_mistake_is_caught_by_finite_differences():
     wrong_dG = np.asarray(d["q"]) * good["dq"]
     wrong = np.flip(np.cumsum(np.flip(wrong_dG, axis=1), axis=1), axis=1)
     assert np.abs(wrong - fd).max() > 1e-3
+
+
+def test_given_forward_results_equal_recomputed_ones():
+    """Passing the oracle's own o and lse changes nothing; a shifted lse scales p."""
+    case = FD_CASES[2]
+    d, do, dlse = _fd_setup(case)
+    a = dict(window=case["window"], cu_seqlens=case["cu"], scale=0.7)
+    o, lse = oracle.wall_fwd(d["q"], d["k"], d["v"], d["g"], d["g_scalar"], d["sink_bias"], **a)
+    base = oracle.wall_bwd(d["q"], d["k"], d["v"], d["g"], do, d["g_scalar"], d["sink_bias"], **a)
+    given = oracle.wall_bwd(d["q"], d["k"], d["v"], d["g"], do, d["g_scalar"], d["sink_bias"],
+                            o=o.astype(np.float32), lse=lse.astype(np.float32), **a)
+    for name in ("dq", "dk", "dv", "dg", "dg_scalar", "dsink"):
+        np.testing.assert_allclose(given[name], base[name], rtol=1e-5, atol=1e-6, err_msg=name)
+    # every weight p = exp(x - lse) doubles when lse drops by ln 2: dv doubles exactly
+    half = oracle.wall_bwd(d["q"], d["k"], d["v"], d["g"], do, d["g_scalar"], d["sink_bias"],
+                           o=o.astype(np.float32), lse=(lse - np.log(2.0)).astype(np.float32), **a)
+    # (up to the fp32 rounding of the two lse arrays)
+    np.testing.assert_allclose(half["dv"], 2.0 * given["dv"], rtol=2e-5, atol=1e-9)
