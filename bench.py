@@ -515,6 +515,42 @@ def run_ours(args, world, rank, local):
                      "prefill_plain_ms": time_fn(prefill, n_rep),
                      "cache_build_of_prefill_ms": time_fn(build_only, n_rep)})
         del pc
+        # prefill backward on the same workload: gradients of sum(o * dO)
+        gdo = torch.Generator(device=dev).manual_seed(pspec.seed + 7)
+        dO = torch.randn((B, T, HQ, V), generator=gdo, device=dev).to(torch.bfloat16)
+        bws = torch.empty(wall.wall_attn_bwd_workspace_size(B, T, HQ, H, K, V, torch.bfloat16),
+                          dtype=torch.uint8, device=dev)
+        grads = {}
+
+        def backward():
+            grads.update(wall.wall_attn_bwd(pd["q"], pd["k"], pd["v"], pd["g"], o, lse, dO,
+                                            pd["g_scalar"], pd["sink_bias"], pd["window"], None,
+                                            pd["scale"], workspace=bws, grads=grads))
+
+        backward()
+        bev = [[ev() for _ in range(3)] for _ in range(n_rep)]
+        for trio in bev:
+            for e in trio:
+                e.record()
+        for i in range(n_rep):
+            wall.wall_debug_set_stage_events(*bev[i])
+            backward()
+            wall.wall_debug_set_stage_events()
+        torch.cuda.synchronize()
+        bwd_ms = time_fn(backward, n_rep)
+        kv_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in bev)
+        q_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in bev)
+        pairs = float(B * HQ * prefill_pairs(pspec))
+        algo = 2.5 * flops   # five pair-products: QK^T, dO V^T, P^T dO, dS^T Q, dS K
+        side.update({
+            "bwd_ms": bwd_ms, "bwd_TFLOPs_algorithmic": algo / (bwd_ms * 1e-3) / 1e12,
+            "bwd_frac_of_burst_peak": algo / (bwd_ms * 1e-3) / 1e12 / bf16_peak,
+            "bwd_dkdv_kernel_ms": kv_ms, "bwd_dq_kernel_ms": q_ms,
+            # executed tensor work: key-block 4 products per pair, query-block 3
+            "bwd_dkdv_kernel_TFLOPs": pairs * 2 * (2 * K + 2 * V) / (kv_ms * 1e-3) / 1e12,
+            "bwd_dq_kernel_TFLOPs": pairs * 2 * (2 * K + V) / (q_ms * 1e-3) / 1e12,
+            "bwd_outside_contractions_ms": bwd_ms - kv_ms - q_ms})
+        del bws, grads, dO
         side.update({"prefill_ms": statistics.mean(pre_ms),
                      "prefill_prepass_ms": statistics.mean(pre_prep_ms),
                      "prefill_main_ms": main_avg,

@@ -12,7 +12,8 @@
 //   S^T = Kh (Qh c)^T,  dP^T = V dO^T            (tcgen05, both operands in SMEM)
 //   dV += P^T dO,       dK += dS^T (Qh c)        (P^T, dS^T read from TMEM)
 // TMEM: S^T | dP^T | dV | dK = 4 x 128 columns; P^T (dS^T) are stored as packed
-// bf16 over the S^T (dP^T) columns.  MMA issue order per query tile i:
+// bf16 over the S^T (dP^T) columns (each elementwise half inside the columns it
+// read itself).  MMA issue order per query tile i:
 //   dV(i), S(i+1), dK(i), dP(i+1)
 // so the elementwise warpgroup's two passes (P from S; dS from dP) overlap
 // the tensor core, and every TMEM overwrite follows, in issue order, the MMA
@@ -24,10 +25,15 @@
 // TMEM: S0 | S1 | dP | dQ; S is double-buffered so S(j+1) is computed while
 // the elementwise warpgroup works on tile j.
 //
-// Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2
-// TMEM allocator; warpgroup 1 = elementwise + epilogue (one TMEM lane = one
-// row per thread); warpgroup 2 multiplies each streamed Qh (key-block kernel)
-// or Kh (query-block kernel) tile by c in shared memory.  Every wait is
+// Warp roles (512 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2
+// TMEM allocator; warpgroups 1 and 2 = elementwise + epilogue, one TMEM lane =
+// one row per thread, warpgroup 1 on the tile's columns 0-63 and warpgroup 2 on
+// 64-127 (two warps per SM sub-partition hide each other's MUFU and TMEM
+// latencies); warpgroup 3 multiplies each streamed Qh (key-block kernel) or Kh
+// (query-block kernel) tile by c in shared memory.  Registers are re-split at
+// start (setmaxnreg): 88 / 168 / 168 / 88 (sum 512 = 4 x the 128 of the
+// launch; no spills).  Per-column vectors of the elementwise passes are read 32
+// at a time as broadcast 16-byte loads, issued with the chunk's TMEM load.  Every wait is
 // bounded (device error word + CTA abort flag), copies in flight are drained
 // and TMEM is freed before exit.
 #include "wall_common.cuh"
@@ -76,8 +82,9 @@ struct BtcCfg {
   // kvfull, qfull[2], qready[2], qempty[2], sfull, dpfull, pready, dsready, final, mdrain
   static constexpr int A_NBAR = 1 + 2 + 2 + 2 + 6;
   static constexpr int A_MISC = A_BAR + A_NBAR * 8;
+  static constexpr int A_RS = A_MISC + 64;       // 128 fp32
   // at least 116 KB so that a second CTA never shares the SM (each takes all of TMEM)
-  static constexpr int A_SMEM = (A_MISC + 64 + 1024) > 118784 ? (A_MISC + 64 + 1024) : 118784;
+  static constexpr int A_SMEM = (A_RS + VEC + 1024) > 118784 ? (A_RS + VEC + 1024) : 118784;
   // query-block kernel
   static constexpr int KS = 3;                   // streamed key tiles
   static constexpr int B_Q = 0;
@@ -95,7 +102,8 @@ struct BtcCfg {
   // qfull, kfull[KS], kready[KS], kempty[KS], vfull, vempty, sfull[2], dpfull, dsready, final, mdrain
   static constexpr int B_NBAR = 1 + 3 * KS + 2 + 2 + 4;
   static constexpr int B_MISC = B_BAR + B_NBAR * 8;
-  static constexpr int B_SMEM = (B_MISC + 64 + 1024) > 118784 ? (B_MISC + 64 + 1024) : 118784;
+  static constexpr int B_RS = B_MISC + 64;       // 128 fp32
+  static constexpr int B_SMEM = (B_RS + VEC + 1024) > 118784 ? (B_RS + VEC + 1024) : 118784;
   static constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 128, 0, 0);
   static constexpr uint32_t IDESC_NK = idesc_bf16_f32(128, KD, 0, 1);  // N = KD, B MN-major
   static constexpr uint32_t IDESC_NV = idesc_bf16_f32(128, VD, 0, 1);  // N = VD, B MN-major
@@ -106,6 +114,13 @@ struct BtcCfg {
 __device__ __forceinline__ uint64_t kmaj_step(int kk) {
   return static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
 }
+// TMEM column of K-step kk (16 rows) of a packed-bf16 operand written by the
+// two elementwise halves: half h stores its 64 values of a row as 32 packed
+// columns at 64 h .. 64 h + 31 (inside the columns it read itself).
+__device__ __forceinline__ uint32_t packed_col(int kk) { return kk * 8 + (kk >= 4 ? 32 : 0); }
+// TMEM column where half cb/64 stores the packed chunk starting at column c.
+__device__ __forceinline__ uint32_t packed_dst(int c, int cb) { return cb + ((c - cb) >> 1); }
+
 // K-step offset (16 rows) inside an MN-major tile: 16 rows of 128 bytes.
 __device__ __forceinline__ uint64_t mnmaj_step(int kk) {
   return static_cast<uint64_t>((kk * 2048) >> 4);
@@ -179,6 +194,27 @@ __device__ __forceinline__ void rescale_tile(uint8_t* tile, const float* c, int 
   }
 }
 
+template <typename T>
+__device__ __forceinline__ T __uint_as_float_or_int(uint32_t u);
+template <>
+__device__ __forceinline__ float __uint_as_float_or_int<float>(uint32_t u) { return __uint_as_float(u); }
+template <>
+__device__ __forceinline__ int __uint_as_float_or_int<int>(uint32_t u) { return static_cast<int>(u); }
+
+// 32 consecutive fp32 (or int) values of a shared-memory vector, read as 8
+// 16-byte loads issued back to back (every thread reads the same addresses).
+template <typename T>
+__device__ __forceinline__ void load32(const T* src, T* dst) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 4) {
+    const uint4 u = *reinterpret_cast<const uint4*>(src + i);
+    dst[i] = __uint_as_float_or_int<T>(u.x);
+    dst[i + 1] = __uint_as_float_or_int<T>(u.y);
+    dst[i + 2] = __uint_as_float_or_int<T>(u.z);
+    dst[i + 3] = __uint_as_float_or_int<T>(u.w);
+  }
+}
+
 __device__ __forceinline__ int first_key(const int* lo_tab, int window, int t) {
   if (lo_tab != nullptr) return lo_tab[t];
   if (window > 0) return t - window + 1 > 0 ? t - window + 1 : 0;
@@ -187,7 +223,7 @@ __device__ __forceinline__ int first_key(const int* lo_tab, int window, int t) {
 
 // ============================================================== key-block kernel
 template <int KD, int VD, bool HAS_GS>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV,
@@ -221,6 +257,7 @@ __global__ void __launch_bounds__(384, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::A_MISC);
   int* abort_flag = reinterpret_cast<int*>(smem + C::A_MISC + 4);
   int* s_qhi = reinterpret_cast<int*>(smem + C::A_MISC + 8);
+  float* sRs = reinterpret_cast<float*>(smem + C::A_RS);  // [128] second half's row sums
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = warp >> 2;
   const int BHQ = p.B * p.HQ;
@@ -240,8 +277,8 @@ __global__ void __launch_bounds__(384, 1)
     }
     mbar_init(sfull, 1);
     mbar_init(dpfull, 1);
-    mbar_init(pready, 128);
-    mbar_init(dsready, 128);
+    mbar_init(pready, 256);
+    mbar_init(dsready, 256);
     mbar_init(final_bar, 1);
     mbar_init(mdrain, 1);
     *abort_flag = 0;
@@ -273,6 +310,7 @@ __global__ void __launch_bounds__(384, 1)
   constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 384;
 
   if (wg == 0) {
+    reg_dealloc<88>();
     if (warp == 0 && lane == 0) {
       // ----------------------------------------------------------- TMA producer
       tma_prefetch_desc(&tmQ);
@@ -347,7 +385,7 @@ __global__ void __launch_bounds__(384, 1)
           const uint64_t oo = static_cast<uint64_t>(s * (C::VB >> 4));
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            umma_ts(tDV, tS + kk * 8, dOm + oo + mnmaj_step(kk), C::IDESC_NV,
+            umma_ts(tDV, tS + packed_col(kk), dOm + oo + mnmaj_step(kk), C::IDESC_NV,
                     (it > 0 || kk > 0) ? 1u : 0u);
         }
         if (it + 1 < nt) {
@@ -361,7 +399,7 @@ __global__ void __launch_bounds__(384, 1)
           const uint64_t qo = static_cast<uint64_t>(s * (C::KB >> 4));
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            umma_ts(tDK, tDP + kk * 8, dQm + qo + mnmaj_step(kk), C::IDESC_NK,
+            umma_ts(tDK, tDP + packed_col(kk), dQm + qo + mnmaj_step(kk), C::IDESC_NK,
                     (it > 0 || kk > 0) ? 1u : 0u);
           umma_commit(&qempty[s]);
         }
@@ -371,9 +409,12 @@ __global__ void __launch_bounds__(384, 1)
       umma_commit(mdrain);
       mbar_drain(mdrain, 0, p.wait_ns);
     }
-  } else if (wg == 1) {
+  } else if (wg == 1 || wg == 2) {
     // ------------------------------------------------------------- elementwise + epilogue
-    const int r = tid - 128;                 // key row within the tile = TMEM lane
+    // warpgroup wg handles the query columns [64 (wg - 1), 64 wg) of every tile
+    reg_alloc<168>();
+    const int hc = wg - 1, cb = 64 * hc;
+    const int r = tid - 128 * wg;            // key row within the tile = TMEM lane
     const int j = j0 + r;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     bool ok = mbar_wait(kvfull, 0, wc);
@@ -397,31 +438,38 @@ __global__ void __launch_bounds__(384, 1)
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
       // pass 1: P^T = exp2(S^T sc + rowt - colt) over the admitted (query, key) pairs
-      uint32_t pk[64];
+      uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < 128; c += 32) {
-        float x[32];
+      for (int c = cb; c < cb + 64; c += 32) {
+        float x[32], rv[32];
         tmem_ld32(lane_base + COL_S + c, x);
+        load32(rowt + c, rv);
         tmem_wait_ld();
         fence_regs32(x);
+        if (full) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float pv[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int qc = c + e + h;
-            float y = fmaf(x[e + h], p.sc, rowt[qc]);
-            if (HAS_GS) y -= colj;
-            bool adm = true;
-            if (!full) {
-              const int q = q0 + qc;
-              adm = q < p.T && q >= j && (lo_tab ? lo[qc] : first_key(nullptr, p.window, q)) <= j;
-            }
-            pv[h] = adm ? ex2_approx(y) : 0.f;
+          for (int e = 0; e < 32; e += 2) {
+            const float p0 = ex2_approx(fmaf(x[e], p.sc, rv[e] - colj));
+            const float p1 = ex2_approx(fmaf(x[e + 1], p.sc, rv[e + 1] - colj));
+            pk[(c - cb + e) >> 1] = pack_bf16(p0, p1);
           }
-          pk[(c + e) >> 1] = pack_bf16(pv[0], pv[1]);
+        } else {
+          int lv[32];
+          if (lo_tab) load32(lo + c, lv);
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float pv[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int q = q0 + c + e + h;
+              const bool adm = q < p.T && q >= j &&
+                               (lo_tab ? lv[e + h] : first_key(nullptr, p.window, q)) <= j;
+              pv[h] = adm ? ex2_approx(fmaf(x[e + h], p.sc, rv[e + h] - colj)) : 0.f;
+            }
+            pk[(c - cb + e) >> 1] = pack_bf16(pv[0], pv[1]);
+          }
         }
-        tmem_st16(lane_base + COL_S + (c >> 1), pk + (c >> 1));
+        tmem_st16(lane_base + COL_S + packed_dst(c, cb), pk + ((c - cb) >> 1));
       }
       tmem_wait_st();
       tc_fence_before();
@@ -431,28 +479,33 @@ __global__ void __launch_bounds__(384, 1)
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 128; c += 32) {
-        float x[32];
+      for (int c = cb; c < cb + 64; c += 32) {
+        float x[32], dv[32];
         tmem_ld32(lane_base + COL_DP + c, x);
+        load32(del + c, dv);
         tmem_wait_ld();
         fence_regs32(x);
         uint32_t dk[16];
+        // rows past T: delta there is not defined (padding), p is 0
+        const int nvalid = full ? 32 : min(32, p.T - (q0 + c));
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const uint32_t u = pk[(c + e) >> 1];
-          const float pe = bf16_lo(u), po = bf16_hi(u);
-          const bool v0 = full || q0 + c + e < p.T, v1 = full || q0 + c + e + 1 < p.T;
-          const float d0 = v0 ? pe * (x[e] - del[c + e]) : 0.f;
-          const float d1 = v1 ? po * (x[e + 1] - del[c + e + 1]) : 0.f;
+          const uint32_t u = pk[(c - cb + e) >> 1];
+          const float d0 = e < nvalid ? bf16_lo(u) * (x[e] - dv[e]) : 0.f;
+          const float d1 = e + 1 < nvalid ? bf16_hi(u) * (x[e + 1] - dv[e + 1]) : 0.f;
           rsum += d0 + d1;
           dk[e >> 1] = pack_bf16(d0, d1);
         }
-        tmem_st16(lane_base + COL_DP + (c >> 1), dk);
+        tmem_st16(lane_base + COL_DP + packed_dst(c, cb), dk);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(dsready);
     }
+    // the two halves' row sums: the second half's go through shared memory
+    if (hc == 1) sRs[r] = rsum;
+    named_bar_sync(2, 256);
+    if (hc == 0) rsum += sRs[r];
     if (ok) {
       const bool got = mbar_wait(final_bar, 0, wc);
       ok = __all_sync(0xffffffffu, got);
@@ -463,7 +516,7 @@ __global__ void __launch_bounds__(384, 1)
       float* krow = p.acc + (static_cast<size_t>(bh) * p.T + (row_ok ? j : 0)) * KD;
       float* vrow = p.dvh + (static_cast<size_t>(bh) * p.T + (row_ok ? j : 0)) * VD;
 #pragma unroll 1
-      for (int c = 0; c < KD; c += 32) {
+      for (int c = hc * (KD / 2); c < (hc + 1) * (KD / 2); c += 32) {
         float x[32];
         tmem_ld32(lane_base + COL_DK + c, x);
         tmem_wait_ld();
@@ -475,7 +528,7 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
 #pragma unroll 1
-      for (int c = 0; c < VD; c += 32) {
+      for (int c = hc * (VD / 2); c < (hc + 1) * (VD / 2); c += 32) {
         float x[32];
         tmem_ld32(lane_base + COL_DV + c, x);
         tmem_wait_ld();
@@ -486,11 +539,12 @@ __global__ void __launch_bounds__(384, 1)
             *reinterpret_cast<float4*>(vrow + c + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
         }
       }
-      if (row_ok) p.rs[static_cast<size_t>(bh) * p.T + j] = rsum;
+      if (row_ok && hc == 0) p.rs[static_cast<size_t>(bh) * p.T + j] = rsum;
     }
   } else {
     // ------------------------------------------------------------- query-tile rescale (by c)
-    const int r = tid - 256;
+    reg_dealloc<88>();
+    const int r = tid - 384;
     bool ok = mbar_wait(kvfull, 0, wc);
     ok = !bar_any(1, 128, !ok);
     for (int it = 0; ok && it < nt; ++it) {
@@ -514,7 +568,7 @@ __global__ void __launch_bounds__(384, 1)
 
 // ============================================================== query-block kernel
 template <int KD, int VD, bool HAS_GS>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV,
@@ -549,6 +603,7 @@ __global__ void __launch_bounds__(384, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::B_MISC);
   int* abort_flag = reinterpret_cast<int*>(smem + C::B_MISC + 4);
   int* s_lo = reinterpret_cast<int*>(smem + C::B_MISC + 8);
+  float* sRs = reinterpret_cast<float*>(smem + C::B_RS);  // [128] second half's row sums
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wg = warp >> 2;
   const int BHQ = p.B * p.HQ;
@@ -572,7 +627,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&sfull[0], 1);
     mbar_init(&sfull[1], 1);
     mbar_init(dpfull, 1);
-    mbar_init(dsready, 128);
+    mbar_init(dsready, 256);
     mbar_init(final_bar, 1);
     mbar_init(mdrain, 1);
     *abort_flag = 0;
@@ -593,6 +648,7 @@ __global__ void __launch_bounds__(384, 1)
   constexpr uint32_t COL_S = 0, COL_DP = 256, COL_DQ = 384;
 
   if (wg == 0) {
+    reg_dealloc<88>();
     if (warp == 0 && lane == 0) {
       // ----------------------------------------------------------- TMA producer
       tma_prefetch_desc(&tmQ);
@@ -669,7 +725,7 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t ko = static_cast<uint64_t>(ks * (C::KB >> 4));
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // dQ += dS (Kh c): dS 128 queries x 128 keys in TMEM
-          umma_ts(tDQ, tDP + kk * 8, dKm + ko + mnmaj_step(kk), C::IDESC_NK,
+          umma_ts(tDQ, tDP + packed_col(kk), dKm + ko + mnmaj_step(kk), C::IDESC_NK,
                   (jt > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&kempty[ks]);
         if (jt + 1 < nt && !issue_dp(jt + 1)) { ok = false; break; }
@@ -679,9 +735,12 @@ __global__ void __launch_bounds__(384, 1)
       umma_commit(mdrain);
       mbar_drain(mdrain, 0, p.wait_ns);
     }
-  } else if (wg == 1) {
+  } else if (wg == 1 || wg == 2) {
     // ------------------------------------------------------------- elementwise + epilogue
-    const int r = tid - 128;  // query row within the tile = TMEM lane
+    // warpgroup wg handles the key columns [64 (wg - 1), 64 wg) of every tile
+    reg_alloc<168>();
+    const int hc = wg - 1, cb = 64 * hc;
+    const int r = tid - 128 * wg;  // query row within the tile = TMEM lane
     const int t = q0 + r;
     const bool row_ok = t < p.T;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16);
@@ -699,11 +758,14 @@ __global__ void __launch_bounds__(384, 1)
       got = got && mbar_wait(&sfull[jt & 1], (jt >> 1) & 1, wc);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
-      uint32_t pk[64];
+      const uint32_t colS = COL_S + 128 * (jt & 1);
+      // pass 1: p = exp2(S sc + rowt - colt), kept in registers as packed bf16
+      uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < 128; c += 32) {
-        float x[32];
-        tmem_ld32(lane_base + COL_S + 128 * (jt & 1) + c, x);
+      for (int c = cb; c < cb + 64; c += 32) {
+        float x[32], cv[32];
+        tmem_ld32(lane_base + colS + c, x);
+        if (HAS_GS) load32(colt + c, cv);
         tmem_wait_ld();
         fence_regs32(x);
 #pragma unroll
@@ -711,20 +773,20 @@ __global__ void __launch_bounds__(384, 1)
           float pv[2];
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int kc = c + e + h, key = k0 + kc;
-            float y = fmaf(x[e + h], p.sc, rowt);
-            if (HAS_GS) y -= colt[kc];
+            const int key = k0 + c + e + h;
+            const float y = fmaf(x[e + h], p.sc, HAS_GS ? rowt - cv[e + h] : rowt);
             const bool adm = full || (key <= t && key >= lo_t);
             pv[h] = adm ? ex2_approx(y) : 0.f;
           }
-          pk[(c + e) >> 1] = pack_bf16(pv[0], pv[1]);
+          pk[(c - cb + e) >> 1] = pack_bf16(pv[0], pv[1]);
         }
       }
+      // pass 2: dS = p (dP - delta) over dP's columns; row sums for dGs
       got = mbar_wait(dpfull, jt & 1, wc);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 128; c += 32) {
+      for (int c = cb; c < cb + 64; c += 32) {
         float x[32];
         tmem_ld32(lane_base + COL_DP + c, x);
         tmem_wait_ld();
@@ -732,18 +794,22 @@ __global__ void __launch_bounds__(384, 1)
         uint32_t dk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const uint32_t u = pk[(c + e) >> 1];
+          const uint32_t u = pk[(c - cb + e) >> 1];
           const float d0 = row_ok ? bf16_lo(u) * (x[e] - del) : 0.f;
           const float d1 = row_ok ? bf16_hi(u) * (x[e + 1] - del) : 0.f;
           rsum += d0 + d1;
           dk[e >> 1] = pack_bf16(d0, d1);
         }
-        tmem_st16(lane_base + COL_DP + (c >> 1), dk);
+        tmem_st16(lane_base + COL_DP + packed_dst(c, cb), dk);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(dsready);
     }
+    // the two halves' row sums: the second half's go through shared memory
+    if (hc == 1) sRs[r] = rsum;
+    named_bar_sync(2, 256);
+    if (hc == 0) rsum += sRs[r];
     if (ok) {
       const bool got = mbar_wait(final_bar, 0, wc);
       ok = __all_sync(0xffffffffu, got);
@@ -752,7 +818,7 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       float* qrow = p.acc + (static_cast<size_t>(bh) * p.T + (row_ok ? t : 0)) * KD;
 #pragma unroll 1
-      for (int c = 0; c < KD; c += 32) {
+      for (int c = hc * (KD / 2); c < (hc + 1) * (KD / 2); c += 32) {
         float x[32];
         tmem_ld32(lane_base + COL_DQ + c, x);
         tmem_wait_ld();
@@ -763,11 +829,12 @@ __global__ void __launch_bounds__(384, 1)
             *reinterpret_cast<float4*>(qrow + c + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
         }
       }
-      if (row_ok) p.rs[static_cast<size_t>(bh) * p.T + t] = rsum;
+      if (row_ok && hc == 0) p.rs[static_cast<size_t>(bh) * p.T + t] = rsum;
     }
   } else {
     // ------------------------------------------------------------- key-tile rescale (by c)
-    const int r = tid - 256;
+    reg_dealloc<88>();
+    const int r = tid - 384;
     bool ok = mbar_wait(qfull, 0, wc);
     ok = !bar_any(1, 128, !ok);
     for (int jt = 0; ok && jt < nt; ++jt) {
@@ -859,13 +926,13 @@ cudaError_t btc_impl(const BwdArgs& a, const FwdWork& fw, const BwdWork& bw, cud
   p.acc = bw.accK;
   p.dvh = bw.dvh;
   p.rs = bw.rsA;
-  kA<<<grid, 384, C::A_SMEM, st>>>(tmQ, tmK, tmV, tmDO, p);
+  kA<<<grid, 512, C::A_SMEM, st>>>(tmQ, tmK, tmV, tmDO, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   record_event(a.ev[1], st);
   p.acc = bw.accQ;
   p.dvh = nullptr;
   p.rs = bw.rsB;
-  kB<<<grid, 384, C::B_SMEM, st>>>(tmQ, tmK, tmV, tmDO, p);
+  kB<<<grid, 512, C::B_SMEM, st>>>(tmQ, tmK, tmV, tmDO, p);
   e = cudaGetLastError();
   record_event(a.ev[2], st);
   return e;
