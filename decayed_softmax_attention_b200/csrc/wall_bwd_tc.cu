@@ -165,8 +165,10 @@ __device__ __forceinline__ void fence_regs32(float* r) {
 }
 
 // Multiplies one 128-row tile of KD bf16 channels (128-byte swizzle, boxes of
-// 64 channels) by c[KD] in place; 128 threads, r = thread index.
-template <int KD>
+// 64 channels) by c[KD] in place; 128 threads, r = thread index.  BATCH chunks
+// are loaded before any is scaled and stored (4 where the rescale sits on the
+// critical path, 1 where it runs in the shadow of the loads).
+template <int KD, int BATCH>
 __device__ __forceinline__ void rescale_tile(uint8_t* tile, const float* c, int r) {
   constexpr int CPR = KD / 8;       // 16-byte chunks per row
   constexpr int RSTEP = 128 / CPR;  // rows between a thread's chunks
@@ -185,12 +187,19 @@ __device__ __forceinline__ void rescale_tile(uint8_t* tile, const float* c, int 
     }
   }
   uint8_t* base = tile + box * 16384;
-#pragma unroll 4
-  for (int m = 0; m < CPR; ++m) {
-    const int row = row0 + m * RSTEP;
-    // 128-byte swizzle: the 16-byte chunk index is XORed with the row's index mod 8
-    uint4* p = reinterpret_cast<uint4*>(base + row * 128 + ((c16 ^ (row & 7)) << 4));
-    *p = scale8(*p, chi, clo);
+#pragma unroll(BATCH == 1 ? 4 : CPR / BATCH)
+  for (int m0 = 0; m0 < CPR; m0 += BATCH) {
+    uint4* ptr[BATCH];
+    uint4 v[BATCH];
+#pragma unroll
+    for (int m = 0; m < BATCH; ++m) {
+      const int row = row0 + (m0 + m) * RSTEP;
+      // 128-byte swizzle: the 16-byte chunk index is XORed with the row's index mod 8
+      ptr[m] = reinterpret_cast<uint4*>(base + row * 128 + ((c16 ^ (row & 7)) << 4));
+      v[m] = *ptr[m];
+    }
+#pragma unroll
+    for (int m = 0; m < BATCH; ++m) *ptr[m] = scale8(v[m], chi, clo);
   }
 }
 
@@ -553,7 +562,7 @@ __global__ void __launch_bounds__(512, 1)
       float* cb = sC + s * KD;
       if (got && r < KD) cb[r] = ex2_approx((sAQ[s * KD + r] - sAK[r]) * kLog2e);
       if (bar_any(1, 128, !got || *abort_flag != 0)) break;
-      rescale_tile<KD>(sQ + s * C::KB, cb, r);
+      rescale_tile<KD, 4>(sQ + s * C::KB, cb, r);
       fence_proxy_async_smem();
       mbar_arrive(&qready[s]);
     }
@@ -843,7 +852,7 @@ __global__ void __launch_bounds__(512, 1)
       float* cb = sC + (jt & 1) * KD;
       if (got && r < KD) cb[r] = ex2_approx((sAQ[r] - sAK[ks * KD + r]) * kLog2e);
       if (bar_any(1, 128, !got || *abort_flag != 0)) break;
-      rescale_tile<KD>(sK + ks * C::KB, cb, r);
+      rescale_tile<KD, 1>(sK + ks * C::KB, cb, r);
       fence_proxy_async_smem();
       mbar_arrive(&kready[ks]);
     }
