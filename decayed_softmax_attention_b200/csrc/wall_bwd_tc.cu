@@ -57,6 +57,8 @@ struct BtcParams {
   float* rs;           // row sums of dS: rsA (per key) / rsB (per query) [bh][T]
   int* err;
   uint64_t wait_ns;
+  int fault;           // testing hook: 4 = key-block producer skips its first query tile,
+                       // 5 = query-block producer skips its first key tile
 };
 
 template <int KD, int VD>
@@ -338,22 +340,24 @@ __global__ void __launch_bounds__(512, 1)
         const int s = it & 1;
         if (it >= 2 && !mbar_wait(&qempty[s], ((it >> 1) - 1) & 1, wc)) break;
         const int q0 = (it_lo + it) * 128;
-        const uint32_t bytes = C::KB + C::VB + KD * 4 + 2 * C::VEC + (lo_tab ? C::VEC : 0);
-        mbar_arrive_expect_tx(&qfull[s], bytes);
-        for (int bx = 0; bx < C::KBOX; ++bx)
-          tma_load_3d(sQ + s * C::KB + bx * 16384, &tmQ, &qfull[s], bx * 64, q0, bh);
-        for (int bx = 0; bx < C::VBOX; ++bx)
-          tma_load_4d(sDO + s * C::VB + bx * 16384, &tmDO, &qfull[s], bx * 64, hq, q0, b);
-        bulk_load(sAQ + s * KD, p.AQ + (static_cast<size_t>(bh) * p.NB + 2 * (q0 / 256)) * KD,
-                  KD * 4, &qfull[s]);
-        bulk_load(sRowt + s * 128, p.rowt + bh * TP + q0, C::VEC, &qfull[s]);
-        bulk_load(sDel + s * 128, p.delta + bh * TP + q0, C::VEC, &qfull[s]);
-        if (lo_tab) bulk_load(sLo + s * 128, lo_tab + q0, C::VEC, &qfull[s]);
+        if (!(p.fault == 4 && it == 0)) {
+          const uint32_t bytes = C::KB + C::VB + KD * 4 + 2 * C::VEC + (lo_tab ? C::VEC : 0);
+          mbar_arrive_expect_tx(&qfull[s], bytes);
+          for (int bx = 0; bx < C::KBOX; ++bx)
+            tma_load_3d(sQ + s * C::KB + bx * 16384, &tmQ, &qfull[s], bx * 64, q0, bh);
+          for (int bx = 0; bx < C::VBOX; ++bx)
+            tma_load_4d(sDO + s * C::VB + bx * 16384, &tmDO, &qfull[s], bx * 64, hq, q0, b);
+          bulk_load(sAQ + s * KD, p.AQ + (static_cast<size_t>(bh) * p.NB + 2 * (q0 / 256)) * KD,
+                    KD * 4, &qfull[s]);
+          bulk_load(sRowt + s * 128, p.rowt + bh * TP + q0, C::VEC, &qfull[s]);
+          bulk_load(sDel + s * 128, p.delta + bh * TP + q0, C::VEC, &qfull[s]);
+          if (lo_tab) bulk_load(sLo + s * 128, lo_tab + q0, C::VEC, &qfull[s]);
+        }
         nq = it + 1;
       }
       mbar_drain(kvfull, 0, p.wait_ns);
       for (int it = nq > 2 ? nq - 2 : 0; it < nq; ++it)
-        mbar_drain(&qfull[it & 1], (it >> 1) & 1, p.wait_ns);
+        if (!(p.fault == 4 && it == 0)) mbar_drain(&qfull[it & 1], (it >> 1) & 1, p.wait_ns);
     } else if (warp == 1 && lane == 0) {
       // ----------------------------------------------------------- MMA issuer
       bool ok = mbar_wait(kvfull, 0, wc);
@@ -675,12 +679,14 @@ __global__ void __launch_bounds__(512, 1)
       for (int jt = 0; jt < nt; ++jt) {
         const int kt = kt_hi - jt, ks = jt % KS;
         if (jt >= KS && !mbar_wait(&kempty[ks], ((jt / KS) - 1) & 1, wc)) break;
-        mbar_arrive_expect_tx(&kfull[ks], C::KB + KD * 4 + (HAS_GS ? C::VEC : 0));
-        for (int bx = 0; bx < C::KBOX; ++bx)
-          tma_load_3d(sK + ks * C::KB + bx * 16384, &tmK, &kfull[ks], bx * 64, kt * 128, bh);
-        bulk_load(sAK + ks * KD, p.AK + (static_cast<size_t>(bh) * p.NB + kt) * KD, KD * 4,
-                  &kfull[ks]);
-        if (HAS_GS) bulk_load(sColt + ks * 128, p.colt + bh * TP + kt * 128, C::VEC, &kfull[ks]);
+        if (!(p.fault == 5 && jt == 0)) {
+          mbar_arrive_expect_tx(&kfull[ks], C::KB + KD * 4 + (HAS_GS ? C::VEC : 0));
+          for (int bx = 0; bx < C::KBOX; ++bx)
+            tma_load_3d(sK + ks * C::KB + bx * 16384, &tmK, &kfull[ks], bx * 64, kt * 128, bh);
+          bulk_load(sAK + ks * KD, p.AK + (static_cast<size_t>(bh) * p.NB + kt) * KD, KD * 4,
+                    &kfull[ks]);
+          if (HAS_GS) bulk_load(sColt + ks * 128, p.colt + bh * TP + kt * 128, C::VEC, &kfull[ks]);
+        }
         nk = jt + 1;
         if (jt >= 1 && !mbar_wait(vempty, (jt - 1) & 1, wc)) break;
         mbar_arrive_expect_tx(vfull, C::VB);
@@ -690,7 +696,7 @@ __global__ void __launch_bounds__(512, 1)
       }
       mbar_drain(qfull, 0, p.wait_ns);
       for (int jt = nk > KS ? nk - KS : 0; jt < nk; ++jt)
-        mbar_drain(&kfull[jt % KS], (jt / KS) & 1, p.wait_ns);
+        if (!(p.fault == 5 && jt == 0)) mbar_drain(&kfull[jt % KS], (jt / KS) & 1, p.wait_ns);
       if (nv > 0) mbar_drain(vfull, (nv - 1) & 1, p.wait_ns);
     } else if (warp == 1 && lane == 0) {
       // ----------------------------------------------------------- MMA issuer
@@ -922,6 +928,7 @@ cudaError_t btc_impl(const BwdArgs& a, const FwdWork& fw, const BwdWork& bw, cud
   p.sc = f.scale * kLog2e;
   p.err = f.err;
   p.wait_ns = f.wait_ns;
+  p.fault = f.fault;
   const unsigned grid = static_cast<unsigned>(f.NB) * BHQ;
 
   auto kA = bwd_dkdv_tc_kernel<KD, VD, HAS_GS>;

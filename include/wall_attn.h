@@ -289,7 +289,9 @@ wall_status_t wall_device_error(wall_stream_t stream);
  * run out and report WALL_ERR_DEVICE_TIMEOUT through the error word (no GPU
  * fault, no hang: every wait gives up after about wait_ms milliseconds):
  *   mode 1: prefill attention (first K/V tile), mode 2: decode split (first
- *   k_tilde/v stage), mode 3: cache build (first g/k stage).
+ *   k_tilde/v stage), mode 3: cache build (first g/k stage), mode 4: backward
+ *   key-block kernel (first query tile), mode 5: backward query-block kernel
+ *   (first key tile; bf16 only).
  * Outputs of the starved call are unspecified.  mode 0 restores normal
  * operation.  wait_ms <= 0 keeps the default limit (2000 ms).
  */

@@ -1,7 +1,8 @@
 """Failure detection without a GPU fault: the kernels' bounded waits.
 
 `wall_debug_set_fault(mode, ms)` makes one kernel's producer skip its first
-load (1: prefill attention, 2: decode split, 3: cache build), so the
+load (1: prefill attention, 2: decode split, 3: cache build, 4 / 5: the
+backward's key-block / query-block kernels), so the
 consumers' waits run out after `ms` milliseconds.  The kernel must then
 wind down on its own (drain its copies, free tensor memory), report
 WALL_ERR_DEVICE_TIMEOUT through the device error word, and leave the context
@@ -88,3 +89,42 @@ def test_cache_build_starved_consumers_time_out_and_recover():
     assert wall.wall_device_error() == 0
     kt, _, _ = oracle.kv_cache(d["k"], d["g"], chunk=64)
     assert_close(good.k_tilde, kt, torch.bfloat16, "cache after recovery")
+
+
+def _bwd_case(wall):
+    spec = W.PrefillSpec("fault_bwd", B=1, T=300, HQ=4, H=2, K=128, V=128, dtype="bf16",
+                         g_kind="negsoftplus", g_scalar=True, seed=9)
+    d = W.gen_prefill(spec, device="cuda")
+    o, lse = wall.wall_attn_fwd(d["q"], d["k"], d["v"], d["g"], d["g_scalar"], scale=d["scale"],
+                                return_lse=True)
+    do = torch.randn(o.shape, device="cuda",
+                     generator=torch.Generator(device="cuda").manual_seed(4)).to(torch.bfloat16)
+    return d, o, lse, do
+
+
+@pytest.mark.parametrize("mode", [4, 5], ids=["key_block", "query_block"])
+def test_backward_starved_consumers_time_out_and_recover(mode):
+    """Modes 4 / 5: a backward contraction kernel's producer skips its first tile."""
+    import decayed_softmax_attention_b200 as wall
+    from tests.test_gpu_bwd import assert_grad_close
+    d, o, lse, do = _bwd_case(wall)
+    assert wall.wall_device_error() == 0
+
+    def bwd():
+        return wall.wall_attn_bwd(d["q"], d["k"], d["v"], d["g"], o, lse, do, d["g_scalar"],
+                                  scale=d["scale"])
+
+    wall.wall_debug_set_fault(mode, 100)
+    try:
+        bwd()
+        status = wall.wall_device_error()
+    finally:
+        wall.wall_debug_set_fault(0, 0)
+    assert status == WALL_ERR_DEVICE_TIMEOUT
+    got = bwd()
+    assert wall.wall_device_error() == 0
+    ref = oracle.wall_bwd(d["q"], d["k"], d["v"], d["g"], do, d["g_scalar"], scale=d["scale"],
+                          o=o, lse=lse, scales=True)
+    for name in ("dq", "dk", "dv", "dg", "dg_scalar"):
+        assert_grad_close(got[name], ref[name], ref["sigma"][name], ref["sigma_abs"][name],
+                          torch.bfloat16, f"{name} after recovery")
