@@ -603,6 +603,49 @@ def run_ours(args, world, rank, local):
         side.update({"decode_varlen_ms": var_ms,
                      "decode_varlen_GBps": var_bytes / (var_ms * 1e-3) / 1e9,
                      "decode_varlen_frac_of_hbm": var_bytes / (var_ms * 1e-3) / 1e9 / hbm_peak})
+        # the same decode over a paged cache: 256-row blocks of the same rows, scattered
+        # through the pool by a seeded permutation (block tables)
+        pbs = 256
+        pmax = (cache.cap + pbs - 1) // pbs
+        nblk = dspec.B * pmax
+        perm = torch.randperm(nblk, generator=torch.Generator().manual_seed(4343))
+        ptable = perm.view(dspec.B, pmax).to(torch.int32).to(dev)
+        kt_pool = torch.empty((nblk, pbs, dspec.HQ, dspec.K), dtype=torch.bfloat16, device=dev)
+        v_pool = torch.empty((nblk, pbs, dspec.H, dspec.V), dtype=torch.bfloat16, device=dev)
+        r_pool = torch.empty((nblk, pbs // dspec.C, dspec.HQ, dspec.K), dtype=torch.float32,
+                             device=dev)
+        n = (cache.cap // pbs) * pbs   # whole blocks; the lengths above never exceed T0 <= n
+        nb_full = n // pbs
+        for b in range(dspec.B):   # setup only: copy each row's blocks into their pool slots
+            idx = ptable[b, :nb_full].long()
+            kt_pool[idx] = cache.k_tilde[b, :n].reshape(-1, pbs, dspec.HQ, dspec.K)
+            v_pool[idx] = cache.v[b, :n].reshape(-1, pbs, dspec.H, dspec.V)
+            r_pool[idx] = cache.r_cache[b, :n // dspec.C].reshape(-1, pbs // dspec.C, dspec.HQ,
+                                                                 dspec.K)
+        if n >= T0:
+            pws = torch.empty(wall.wall_attn_decode_workspace_size(
+                dspec.B, pmax * pbs, dspec.HQ, dspec.H, dspec.V, dspec.C), dtype=torch.uint8,
+                device=dev)
+
+            def dec_paged():
+                wall.wall_attn_decode_paged(qv, cache.p[:, None], v_pool, kt_pool, r_pool, seqlens,
+                                            ptable, scale=dspec.K ** -0.5, chunk=dspec.C,
+                                            out=dout, workspace=pws)
+
+            dec_paged()
+            pa, pz = ev(), ev()
+            torch.cuda.synchronize()
+            pa.record()
+            for _ in range(10):
+                dec_paged()
+            pz.record()
+            torch.cuda.synchronize()
+            pg_ms = pa.elapsed_time(pz) / 10
+            side.update({"decode_paged_ms": pg_ms, "decode_paged_block_rows": pbs,
+                         "decode_paged_GBps": var_bytes / (pg_ms * 1e-3) / 1e9,
+                         "decode_paged_frac_of_hbm": var_bytes / (pg_ms * 1e-3) / 1e9 / hbm_peak})
+            del pws
+        del kt_pool, v_pool, r_pool
         side.update({"cache_build_prefix_ms": build_ms,
                      "cache_build_prefix_GBps": build_gbps,
                      "cache_build_roofline": {

@@ -27,7 +27,8 @@ __all__ = [
     "WallError", "lib_path", "load_library", "wall_attn_fwd", "wall_attn_fwd_workspace_size",
     "wall_build_kv_cache", "wall_attn_decode", "wall_attn_decode_workspace_size",
     "wall_attn_decode_noalloc", "wall_append_kv_cache_varlen", "wall_attn_bwd",
-    "wall_attn_bwd_workspace_size", "wall_device_error", "wall_debug_set_fault", "wall_debug_set_stage_events", "KVCache",
+    "wall_attn_bwd_workspace_size", "wall_build_kv_cache_paged", "wall_append_kv_cache_paged",
+    "wall_attn_decode_paged", "PagedKVCache", "wall_device_error", "wall_debug_set_fault", "wall_debug_set_stage_events", "KVCache",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -48,6 +49,7 @@ EXPORTED_SYMBOLS = (
     "wall_device_error", "wall_debug_set_fault", "wall_debug_set_stage_events",
     "wall_attn_decode_noalloc", "wall_attn_fwd_with_cache", "wall_attn_decode_varlen",
     "wall_append_kv_cache_varlen", "wall_attn_bwd_workspace_size", "wall_attn_bwd",
+    "wall_build_kv_cache_paged", "wall_append_kv_cache_paged", "wall_attn_decode_paged",
 )
 
 
@@ -91,6 +93,15 @@ def load_library():
     lib.wall_attn_bwd.argtypes = [P, P, P, P, P, P, I, P, I, I, I, I, I, I, I, I, F, P, P, P, P,
                                   P, P, P, P, P, P, P, S, P]
     lib.wall_attn_bwd.restype = I
+    lib.wall_build_kv_cache_paged.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, P, P,
+                                              P, P]
+    lib.wall_build_kv_cache_paged.restype = I
+    lib.wall_append_kv_cache_paged.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, I, I, P, P, P,
+                                               P]
+    lib.wall_append_kv_cache_paged.restype = I
+    lib.wall_attn_decode_paged.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I,
+                                           F, P, P, P, S, P]
+    lib.wall_attn_decode_paged.restype = I
     lib.wall_build_kv_cache.argtypes = [P, P, P, I, I, I, I, I, I, I, I, I, P, P, P, P]
     lib.wall_build_kv_cache.restype = I
     lib.wall_append_kv_cache_varlen.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P, P, P, P]
@@ -350,6 +361,84 @@ def wall_attn_decode(q, p_curr, v, k_tilde, r_cache, T_kv, sink_bias=None, scale
     return out
 
 
+# ----------------------------------------------------------------- paged caches
+def _pool_dims(k_tilde_pool, block_table, chunk):
+    nblk, bs = k_tilde_pool.shape[0], k_tilde_pool.shape[1]
+    return nblk, bs, block_table.shape[1], bs // chunk
+
+
+def wall_build_kv_cache_paged(k_new, g_new, block_table, k_tilde_pool, r_pool, p_last, t_start=0,
+                              p_prev=None, chunk=64):
+    """wall_build_kv_cache into a paged pool: rows t_start .. t_start+T_new-1 of each batch row,
+    addressed through block_table [B, max_blocks] (int32, device)."""
+    lib = load_library()
+    B, T_new, H, K = k_new.shape
+    HQ = g_new.shape[2]
+    dt = k_new.dtype
+    nblk, bs, maxblk, cpb = _pool_dims(k_tilde_pool, block_table, chunk)
+    st = lib.wall_build_kv_cache_paged(
+        _dev(k_new, "k_new", dt), _dev(g_new, "g_new", dt, (B, T_new, HQ, K)),
+        _dev(p_prev, "p_prev", torch.float32, (B, HQ, K)),
+        _dev(block_table, "block_table", torch.int32, (B, maxblk)), maxblk, B, int(t_start), T_new,
+        nblk, bs, HQ, H, K, int(chunk), _dtype_code(k_new),
+        _dev(k_tilde_pool, "k_tilde_pool", dt, (nblk, bs, HQ, K)),
+        _dev(r_pool, "r_pool", torch.float32, (nblk, cpb, HQ, K)),
+        _dev(p_last, "p_last", torch.float32, (B, HQ, K)), _stream(k_new.device))
+    _check(st, "wall_build_kv_cache_paged")
+    return p_last
+
+
+def wall_append_kv_cache_paged(k_new, g_new, block_table, k_tilde_pool, r_pool, p_last, t_pos,
+                               p_prev=None, chunk=64):
+    """One token per batch row at row b's own position t_pos[b], into a paged pool."""
+    lib = load_library()
+    B, _, H, K = k_new.shape
+    HQ = g_new.shape[2]
+    dt = k_new.dtype
+    nblk, bs, maxblk, cpb = _pool_dims(k_tilde_pool, block_table, chunk)
+    if p_prev is None:
+        p_prev = p_last
+    st = lib.wall_append_kv_cache_paged(
+        _dev(k_new, "k_new", dt, (B, 1, H, K)), _dev(g_new, "g_new", dt, (B, 1, HQ, K)),
+        _dev(p_prev, "p_prev", torch.float32, (B, HQ, K)), _dev(t_pos, "t_pos", torch.int32, (B,)),
+        _dev(block_table, "block_table", torch.int32, (B, maxblk)), maxblk, B, nblk, bs, HQ, H, K,
+        int(chunk), _dtype_code(k_new), _dev(k_tilde_pool, "k_tilde_pool", dt, (nblk, bs, HQ, K)),
+        _dev(r_pool, "r_pool", torch.float32, (nblk, cpb, HQ, K)),
+        _dev(p_last, "p_last", torch.float32, (B, HQ, K)), _stream(k_new.device))
+    _check(st, "wall_append_kv_cache_paged")
+    return p_last
+
+
+def wall_attn_decode_paged(q, p_curr, v_pool, k_tilde_pool, r_pool, seqlens, block_table,
+                           sink_bias=None, scale=None, chunk=64, out=None, lse=None,
+                           workspace=None):
+    """One decode step over paged caches: batch row b attends its rows [0, seqlens[b])."""
+    lib = load_library()
+    B = q.shape[0]
+    nblk, bs, HQ, K = k_tilde_pool.shape
+    H, V = v_pool.shape[2], v_pool.shape[3]
+    maxblk = block_table.shape[1]
+    dt = k_tilde_pool.dtype
+    if out is None:
+        out = torch.empty((B, 1, HQ, V), dtype=dt, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(
+            max(wall_attn_decode_workspace_size(B, maxblk * bs, HQ, H, V, chunk), 1),
+            dtype=torch.uint8, device=q.device)
+    st = lib.wall_attn_decode_paged(
+        _dev(q, "q", dt), _dev(p_curr, "p_curr", torch.float32),
+        _dev(v_pool, "v_pool", dt, (nblk, bs, H, V)), _dev(k_tilde_pool, "k_tilde_pool", dt),
+        _dev(r_pool, "r_pool", torch.float32, (nblk, bs // chunk, HQ, K)),
+        _dev(sink_bias, "sink_bias", torch.float32, (HQ,)),
+        _dev(seqlens, "seqlens", torch.int32, (B,)),
+        _dev(block_table, "block_table", torch.int32, (B, maxblk)), maxblk, B, nblk, bs, HQ, H, K,
+        V, int(chunk), _dtype_code(k_tilde_pool), float(scale) if scale else 0.0,
+        _dev(out, "out", dt), _dev(lse, "lse", torch.float32), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(q.device))
+    _check(st, "wall_attn_decode_paged")
+    return out
+
+
 def wall_attn_decode_noalloc(q, p_curr, v, k_tilde, r_cache, T_kv, out, lse=None,
                              sink_bias=None, scale=None, chunk=64):
     """wall_attn_decode without a workspace: the split partials live in a fixed
@@ -419,3 +508,97 @@ class KVCache:
         return wall_attn_decode(q, self.p, self.v, self.k_tilde, self.r_cache, self.length,
                                 sink_bias=sink_bias, scale=scale, chunk=self.chunk, out=out,
                                 lse=lse, workspace=self.workspace)
+
+
+class PagedKVCache:
+    """A paged decode cache: pools of fixed-size blocks plus one block table per sequence.
+
+    Blocks are handed out from a free list on the host as sequences grow
+    (``reserve``) and returned when a sequence is dropped (``release``); the
+    device block table is refreshed from the host copy after each change.  Value
+    rows are written by ``append`` (a scatter through the table) or by the caller.
+    """
+
+    def __init__(self, B, num_blocks, block_size, max_blocks, HQ, H, K, V, dtype=torch.bfloat16,
+                 chunk=64, device="cuda"):
+        if block_size % chunk:
+            raise ValueError("block_size must be a multiple of chunk")
+        self.B, self.HQ, self.H, self.K, self.V, self.chunk = B, HQ, H, K, V, chunk
+        self.num_blocks, self.block_size, self.max_blocks = num_blocks, block_size, max_blocks
+        self.k_tilde = torch.empty((num_blocks, block_size, HQ, K), dtype=dtype, device=device)
+        self.r_cache = torch.empty((num_blocks, block_size // chunk, HQ, K), dtype=torch.float32,
+                                   device=device)
+        self.v = torch.zeros((num_blocks, block_size, H, V), dtype=dtype, device=device)
+        self.p = torch.zeros((B, HQ, K), dtype=torch.float32, device=device)
+        self.free = list(range(num_blocks))
+        self.host_table = [[] for _ in range(B)]
+        self.block_table = torch.zeros((B, max_blocks), dtype=torch.int32, device=device)
+        self.lengths = [0] * B
+        self.workspace = torch.empty(
+            max(wall_attn_decode_workspace_size(B, max_blocks * block_size, HQ, H, V, chunk), 1),
+            dtype=torch.uint8, device=device)
+
+    def _sync_table(self):
+        t = torch.zeros((self.B, self.max_blocks), dtype=torch.int32)
+        for b, blocks in enumerate(self.host_table):
+            if blocks:
+                t[b, :len(blocks)] = torch.tensor(blocks, dtype=torch.int32)
+        self.block_table.copy_(t)
+
+    def reserve(self, b, rows):
+        """Make batch row b hold at least `rows` rows (allocates blocks)."""
+        need = (rows + self.block_size - 1) // self.block_size
+        if need > self.max_blocks:
+            raise ValueError("sequence longer than max_blocks * block_size")
+        changed = False
+        while len(self.host_table[b]) < need:
+            if not self.free:
+                raise MemoryError("paged cache pool exhausted")
+            self.host_table[b].append(self.free.pop(0))
+            changed = True
+        if changed:
+            self._sync_table()
+
+    def release(self, b):
+        self.free.extend(self.host_table[b])
+        self.host_table[b] = []
+        self.lengths[b] = 0
+        self._sync_table()
+
+    def rows_of(self, b, t0, t1):
+        """Physical pool rows of logical rows [t0, t1) of batch row b (host list)."""
+        bs = self.block_size
+        return [self.host_table[b][t // bs] * bs + t % bs for t in range(t0, t1)]
+
+    def prefill(self, k, g, v):
+        """Build rows 0 .. T-1 of every batch row (all rows start empty)."""
+        B, T = k.shape[0], k.shape[1]
+        for b in range(B):
+            self.reserve(b, T)
+        wall_build_kv_cache_paged(k, g, self.block_table, self.k_tilde, self.r_cache, self.p,
+                                  t_start=0, chunk=self.chunk)
+        for b in range(B):
+            rows = torch.tensor(self.rows_of(b, 0, T), device=self.v.device)
+            self.v.view(-1, self.H, self.V)[rows] = v[b]
+            self.lengths[b] = T
+        return self.p
+
+    def append(self, k_new, g_new, v_new, t_pos):
+        """One token per batch row at t_pos (host list of ints) = each row's current length."""
+        for b, t in enumerate(t_pos):
+            self.reserve(b, t + 1)
+        tp = torch.tensor(t_pos, dtype=torch.int32, device=k_new.device)
+        wall_append_kv_cache_paged(k_new, g_new, self.block_table, self.k_tilde, self.r_cache,
+                                   self.p, tp, chunk=self.chunk)
+        rows = torch.tensor([self.rows_of(b, t, t + 1)[0] for b, t in enumerate(t_pos)],
+                            device=self.v.device)
+        self.v.view(-1, self.H, self.V)[rows] = v_new[:, 0]
+        for b, t in enumerate(t_pos):
+            self.lengths[b] = t + 1
+        return self.p
+
+    def decode(self, q, sink_bias=None, scale=None, out=None, lse=None):
+        seqlens = torch.tensor(self.lengths, dtype=torch.int32, device=q.device)
+        return wall_attn_decode_paged(q, self.p[:, None], self.v, self.k_tilde, self.r_cache,
+                                      seqlens, self.block_table, sink_bias=sink_bias, scale=scale,
+                                      chunk=self.chunk, out=out, lse=lse, workspace=self.workspace)

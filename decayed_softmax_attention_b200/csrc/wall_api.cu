@@ -322,10 +322,10 @@ wall_status_t wall_attn_bwd(const void* q, const void* k, const void* v, const v
   return finish(wall::launch_bwd(a, fw, bw, bf16, st), st);
 }
 
-wall_status_t wall_build_kv_cache(const void* k_new, const void* g_new, const float* p_prev,
-                                  int B, int t_start, int T_new, int cap, int HQ, int H, int K,
-                                  int chunk, wall_dtype_t dt, void* k_tilde, float* r_cache,
-                                  float* p_last, wall_stream_t stream) {
+static wall_status_t build_entry(const void* k_new, const void* g_new, const float* p_prev,
+                                 int B, int t_start, int T_new, int cap, int HQ, int H, int K,
+                                 int chunk, wall_dtype_t dt, void* k_tilde, float* r_cache,
+                                 float* p_last, wall_stream_t stream, const wall::PageMap* pm) {
   if (B < 0 || t_start < 0 || T_new < 0 || cap < 0 || HQ <= 0 || H <= 0 || HQ % H != 0)
     return WALL_ERR_INVALID_ARG;
   if (dt != WALL_DTYPE_F32 && dt != WALL_DTYPE_BF16) return WALL_ERR_INVALID_ARG;
@@ -347,15 +347,55 @@ wall_status_t wall_build_kv_cache(const void* k_new, const void* g_new, const fl
   if (a.err == nullptr) return WALL_ERR_CUDA;
   a.wait_ns = wall::wait_limit_ns();
   a.fault = wall::fault_mode();
+  if (pm != nullptr) a.pm = *pm;
+  a.pm.cap = cap;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   return finish(wall::launch_cache_build(a, dt == WALL_DTYPE_BF16, st), st);
 }
 
-wall_status_t wall_append_kv_cache_varlen(const void* k_new, const void* g_new,
-                                          const float* p_prev, const int32_t* t_pos, int B,
-                                          int cap, int HQ, int H, int K, int chunk,
-                                          wall_dtype_t dt, void* k_tilde, float* r_cache,
-                                          float* p_last, wall_stream_t stream) {
+wall_status_t wall_build_kv_cache(const void* k_new, const void* g_new, const float* p_prev,
+                                  int B, int t_start, int T_new, int cap, int HQ, int H, int K,
+                                  int chunk, wall_dtype_t dt, void* k_tilde, float* r_cache,
+                                  float* p_last, wall_stream_t stream) {
+  return build_entry(k_new, g_new, p_prev, B, t_start, T_new, cap, HQ, H, K, chunk, dt, k_tilde,
+                     r_cache, p_last, stream, nullptr);
+}
+
+// Checks shared by the paged calls; fills *pm.  Returns WALL_OK or an error.
+static wall_status_t page_map(const int32_t* block_table, int max_blocks, int num_blocks,
+                              int block_size, int chunk, int B, wall::PageMap* pm) {
+  if (max_blocks < 1 || num_blocks < 1 || block_size < 1) return WALL_ERR_INVALID_ARG;
+  if (chunk != 32 && chunk != 64 && chunk != 128) return WALL_ERR_UNSUPPORTED;
+  if (block_size % chunk != 0 || block_size > (1 << 20)) return WALL_ERR_UNSUPPORTED;
+  if (static_cast<long long>(max_blocks) * block_size > 0x7fffffffLL ||
+      static_cast<long long>(num_blocks) * block_size > 0x7fffffffLL ||
+      static_cast<long long>(B) * max_blocks > 0x7fffffffLL)
+    return WALL_ERR_UNSUPPORTED;
+  if (B > 0 && (block_table == nullptr || !aligned(block_table, 4))) return WALL_ERR_INVALID_ARG;
+  pm->bt = block_table;
+  pm->maxblk = max_blocks;
+  pm->bs = block_size;
+  pm->nblk = num_blocks;
+  return WALL_OK;
+}
+
+wall_status_t wall_build_kv_cache_paged(const void* k_new, const void* g_new,
+                                        const float* p_prev, const int32_t* block_table,
+                                        int max_blocks, int B, int t_start, int T_new,
+                                        int num_blocks, int block_size, int HQ, int H, int K,
+                                        int chunk, wall_dtype_t dt, void* k_tilde_pool,
+                                        float* r_pool, float* p_last, wall_stream_t stream) {
+  wall::PageMap pm;
+  const wall_status_t ps = page_map(block_table, max_blocks, num_blocks, block_size, chunk, B, &pm);
+  if (ps != WALL_OK) return ps;
+  return build_entry(k_new, g_new, p_prev, B, t_start, T_new, max_blocks * block_size, HQ, H, K,
+                     chunk, dt, k_tilde_pool, r_pool, p_last, stream, &pm);
+}
+
+static wall_status_t append_entry(const void* k_new, const void* g_new, const float* p_prev,
+                                  const int32_t* t_pos, int B, int cap, int HQ, int H, int K,
+                                  int chunk, wall_dtype_t dt, void* k_tilde, float* r_cache,
+                                  float* p_last, wall_stream_t stream, const wall::PageMap* pm) {
   if (B < 0 || cap < 1 || HQ <= 0 || H <= 0 || HQ % H != 0) return WALL_ERR_INVALID_ARG;
   if (dt != WALL_DTYPE_F32 && dt != WALL_DTYPE_BF16) return WALL_ERR_INVALID_ARG;
   if (!supported_dim(K)) return WALL_ERR_UNSUPPORTED;
@@ -372,8 +412,32 @@ wall_status_t wall_append_kv_cache_varlen(const void* k_new, const void* g_new,
   a.B = B; a.t_start = 0; a.T_new = 1; a.cap = cap; a.HQ = HQ; a.H = H; a.K = K;
   a.chunk = chunk; a.k_tilde = k_tilde; a.r_cache = r_cache; a.p_last = p_last;
   a.err = nullptr; a.wait_ns = 0; a.fault = 0;
+  if (pm != nullptr) a.pm = *pm;
+  a.pm.cap = cap;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   return finish(wall::launch_append_varlen(a, t_pos, dt == WALL_DTYPE_BF16, st), st);
+}
+
+wall_status_t wall_append_kv_cache_varlen(const void* k_new, const void* g_new,
+                                          const float* p_prev, const int32_t* t_pos, int B,
+                                          int cap, int HQ, int H, int K, int chunk,
+                                          wall_dtype_t dt, void* k_tilde, float* r_cache,
+                                          float* p_last, wall_stream_t stream) {
+  return append_entry(k_new, g_new, p_prev, t_pos, B, cap, HQ, H, K, chunk, dt, k_tilde, r_cache,
+                      p_last, stream, nullptr);
+}
+
+wall_status_t wall_append_kv_cache_paged(const void* k_new, const void* g_new,
+                                         const float* p_prev, const int32_t* t_pos,
+                                         const int32_t* block_table, int max_blocks, int B,
+                                         int num_blocks, int block_size, int HQ, int H, int K,
+                                         int chunk, wall_dtype_t dt, void* k_tilde_pool,
+                                         float* r_pool, float* p_last, wall_stream_t stream) {
+  wall::PageMap pm;
+  const wall_status_t ps = page_map(block_table, max_blocks, num_blocks, block_size, chunk, B, &pm);
+  if (ps != WALL_OK) return ps;
+  return append_entry(k_new, g_new, p_prev, t_pos, B, max_blocks * block_size, HQ, H, K, chunk,
+                      dt, k_tilde_pool, r_pool, p_last, stream, &pm);
 }
 
 size_t wall_attn_decode_workspace_size(int B, int T_kv, int HQ, int H, int V, int chunk) {
@@ -387,7 +451,8 @@ static wall_status_t decode_entry(const void* q, const float* p_curr, const void
                                   const float* sink_bias, const int32_t* seqlens, int B, int T_kv,
                                   int cap, int HQ, int H, int K, int V, int chunk,
                                   wall_dtype_t dt, float scale, void* o, float* lse,
-                                  void* workspace, size_t workspace_bytes, wall_stream_t stream) {
+                                  void* workspace, size_t workspace_bytes, wall_stream_t stream,
+                                  const wall::PageMap* pm = nullptr) {
   if (B < 0 || T_kv < 1 || cap < T_kv || HQ <= 0 || H <= 0 || HQ % H != 0)
     return WALL_ERR_INVALID_ARG;
   if (dt != WALL_DTYPE_F32 && dt != WALL_DTYPE_BF16) return WALL_ERR_INVALID_ARG;
@@ -414,6 +479,8 @@ static wall_status_t decode_entry(const void* q, const float* p_curr, const void
   a.wait_ns = wall::wait_limit_ns();
   a.fault = wall::fault_mode();
   a.seqlens = seqlens;
+  if (pm != nullptr) a.pm = *pm;
+  a.pm.cap = cap;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   stage_event(0, st);
   const cudaError_t e = wall::launch_decode(a, dt == WALL_DTYPE_BF16, st);
@@ -440,6 +507,24 @@ wall_status_t wall_attn_decode_varlen(const void* q, const float* p_curr, const 
   if (B > 0 && seqlens_kv == nullptr) return WALL_ERR_INVALID_ARG;
   return decode_entry(q, p_curr, v, k_tilde, r_cache, sink_bias, seqlens_kv, B, max_T_kv, cap, HQ,
                       H, K, V, chunk, dt, scale, o, lse, workspace, workspace_bytes, stream);
+}
+
+wall_status_t wall_attn_decode_paged(const void* q, const float* p_curr, const void* v_pool,
+                                     const void* k_tilde_pool, const float* r_pool,
+                                     const float* sink_bias, const int32_t* seqlens_kv,
+                                     const int32_t* block_table, int max_blocks, int B,
+                                     int num_blocks, int block_size, int HQ, int H, int K, int V,
+                                     int chunk, wall_dtype_t dt, float scale, void* o, float* lse,
+                                     void* workspace, size_t workspace_bytes,
+                                     wall_stream_t stream) {
+  if (B > 0 && seqlens_kv == nullptr) return WALL_ERR_INVALID_ARG;
+  wall::PageMap pm;
+  const wall_status_t ps = page_map(block_table, max_blocks, num_blocks, block_size, chunk, B, &pm);
+  if (ps != WALL_OK) return ps;
+  const int rows = max_blocks * block_size;
+  return decode_entry(q, p_curr, v_pool, k_tilde_pool, r_pool, sink_bias, seqlens_kv, B, rows,
+                      rows, HQ, H, K, V, chunk, dt, scale, o, lse, workspace, workspace_bytes,
+                      stream, &pm);
 }
 
 wall_status_t wall_device_error(wall_stream_t stream) {

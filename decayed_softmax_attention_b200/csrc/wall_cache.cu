@@ -55,10 +55,10 @@ struct CacheCfg {
   static constexpr int ROWB = KD * ESZ;      // bytes of one head row
 };
 
-template <typename T, int KD>
+template <typename T, int KD, bool PAGED>
 __global__ void __launch_bounds__(160) cache_build_kernel(
     const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmK,
-    const float* __restrict__ p_prev, int t_start, int T_new, int cap, int HQ, int G, int HPC,
+    const float* __restrict__ p_prev, int t_start, int T_new, PageMap pm, int HQ, int G, int HPC,
     int NKV, int C, int seg_first, int seg_rows, T* __restrict__ k_tilde,
     float* __restrict__ r_cache, float* __restrict__ p_last, int* err, uint64_t wait_ns,
     int fault) {
@@ -123,10 +123,20 @@ __global__ void __launch_bounds__(160) cache_build_kernel(
   const int ch = (ct % CC::TPS) * 4;
   const int hq = hq0 + hl;
   const size_t bh = static_cast<size_t>(b) * HQ + hq;
-  const int ncap = (cap + C - 1) / C;
+  // this thread's four channels of cache row ta / of the anchor of ta's chunk:
+  // dense caches step through rows with one add, paged ones go through the table
   const size_t hstep = static_cast<size_t>(HQ) * KD;
-  T* op = k_tilde + ((static_cast<size_t>(b) * cap + t_start) * HQ + hq) * KD + ch;
-  float* rp = r_cache + (static_cast<size_t>(b) * ncap * HQ + hq) * KD + ch;  // + chunk * hstep
+  T* const op = k_tilde + (static_cast<size_t>(b) * pm.cap * HQ + hq) * KD + ch;
+  float* const rp = r_cache + (static_cast<size_t>(b) * ((pm.cap + C - 1) / C) * HQ + hq) * KD + ch;
+  const int cshift = __ffs(C) - 1;  // C is a power of two
+  auto krow = [=](int ta) -> T* {
+    if constexpr (PAGED) return k_tilde + (pm.row(b, ta) * HQ + hq) * KD + ch;
+    else return op + static_cast<size_t>(ta) * hstep;
+  };
+  auto rslot = [=](int ta) -> float* {
+    if constexpr (PAGED) return r_cache + (pm.chunk(b, ta, C) * HQ + hq) * KD + ch;
+    else return rp + static_cast<size_t>(ta >> cshift) * hstep;
+  };
 
   float carry[4], loc[4], r0[4];
 #pragma unroll
@@ -138,21 +148,19 @@ __global__ void __launch_bounds__(160) cache_build_kernel(
   if (active && segmented) {
     // P just before the segment (read before this thread overwrites the slot
     // with the chunk's anchor at the segment's first row)
-    const float4 c4 = *reinterpret_cast<const float4*>(
-        rp + static_cast<size_t>((t_start + rb) / C) * hstep);
+    const float4 c4 = *reinterpret_cast<const float4*>(rslot(t_start + rb));
     carry[0] = c4.x;
     carry[1] = c4.y;
     carry[2] = c4.z;
     carry[3] = c4.w;
   } else if (active && t_start % C != 0) {
     // the chunk holding t_start was anchored by an earlier call
-    const float* rr = rp + static_cast<size_t>(t_start / C) * hstep;
+    const float* rr = rslot(t_start);
 #pragma unroll
     for (int c = 0; c < 4; ++c) r0[c] = rr[c] - carry[c];
   }
 
   const int cmask = C - 1;  // C is a power of two
-  const int cshift = __ffs(C) - 1;
   const int gstr = HPC * KD, kstr = NKV * KD;  // shared-memory row strides (elements)
   // One row: fold g into the prefix, anchor at a chunk head, rescale k.
   auto row = [&](const T* g_s, const T* k_s, T* o_g, bool head, int ta) {
@@ -174,7 +182,7 @@ __global__ void __launch_bounds__(160) cache_build_kernel(
     if (head) {
 #pragma unroll
       for (int c = 0; c < 4; ++c) r0[c] = loc[c];
-      *reinterpret_cast<float4*>(rp + static_cast<size_t>(ta >> cshift) * hstep) =
+      *reinterpret_cast<float4*>(rslot(ta)) =
           make_float4(carry[0] + loc[0], carry[1] + loc[1], carry[2] + loc[2], carry[3] + loc[3]);
     }
 #pragma unroll
@@ -197,21 +205,21 @@ __global__ void __launch_bounds__(160) cache_build_kernel(
       const int t0 = rb + i * D;
       const int ta0 = t_start + t0;
       const int hr = (C - (ta0 & cmask)) & cmask;  // stage row that opens a chunk (>= D: none)
-      T* ob = op + static_cast<size_t>(t0) * hstep;
+      T* ob = PAGED ? nullptr : krow(ta0);
       if (t0 + D <= re) {
 #pragma unroll
         for (int r = 0; r < D; ++r) {
-          row(sg, sk, ob, r == hr, ta0 + r);
+          row(sg, sk, PAGED ? krow(ta0 + r) : ob, r == hr, ta0 + r);
           sg += gstr;
           sk += kstr;
-          ob += hstep;
+          if (!PAGED) ob += hstep;
         }
       } else {
         for (int r = 0; r < re - t0; ++r) {
-          row(sg, sk, ob, r == hr, ta0 + r);
+          row(sg, sk, PAGED ? krow(ta0 + r) : ob, r == hr, ta0 + r);
           sg += gstr;
           sk += kstr;
-          ob += hstep;
+          if (!PAGED) ob += hstep;
         }
       }
     }
@@ -232,7 +240,7 @@ __device__ __forceinline__ void store_one(float* p, float x) { *p = x; }
 // in the anchor slot of the segment's first chunk until pass 3 overwrites it.
 template <typename T, int KD>
 __global__ void __launch_bounds__(128) cache_segsum_kernel(
-    const T* __restrict__ g_new, int t_start, int T_new, int cap, int HQ, int HPC, int C,
+    const T* __restrict__ g_new, int t_start, int T_new, PageMap pm, int HQ, int HPC, int C,
     int seg_first, int seg_rows, float* __restrict__ r_cache) {
   using CC = CacheCfg<T, KD>;
   constexpr int U = 8;  // rows whose loads are issued together
@@ -267,8 +275,7 @@ __global__ void __launch_bounds__(128) cache_segsum_kernel(
       }
     }
   }
-  const int ncap = (cap + C - 1) / C;
-  float* rr = r_cache + ((static_cast<size_t>(b) * ncap + (t_start + rb) / C) * HQ + hq) * KD + ch;
+  float* rr = r_cache + (pm.chunk(b, t_start + rb, C) * HQ + hq) * KD + ch;
   *reinterpret_cast<float4*>(rr) =
       make_float4(tot[0] + loc[0], tot[1] + loc[1], tot[2] + loc[2], tot[3] + loc[3]);
 }
@@ -280,31 +287,28 @@ __global__ void __launch_bounds__(128) cache_segsum_kernel(
 template <typename T, int KD>
 __global__ void __launch_bounds__(128) cache_segscan_kernel(
     const T* __restrict__ k_new, const T* __restrict__ g_new, const float* __restrict__ p_prev,
-    int B, int t_start, int T_new, int cap, int HQ, int H, int C, int seg_first, int seg_rows,
+    int B, int t_start, int T_new, PageMap pm, int HQ, int H, int C, int seg_first, int seg_rows,
     int nseg, T* __restrict__ k_tilde, float* __restrict__ r_cache, float* __restrict__ p_last) {
   const long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= static_cast<long>(B) * HQ * KD) return;
   const int n = static_cast<int>(idx % KD);
   const long bh = idx / KD;
   const int b = static_cast<int>(bh / HQ), hq = static_cast<int>(bh % HQ), kvh = hq / (HQ / H);
-  const int ncap = (cap + C - 1) / C;
-  const size_t hstep = static_cast<size_t>(HQ) * KD;
-  float* rp = r_cache + (static_cast<size_t>(b) * ncap * HQ + hq) * KD + n;  // + chunk * hstep
+  auto rslot = [&](int ta) { return r_cache + (pm.chunk(b, ta, C) * HQ + hq) * KD + n; };
   float carry = p_prev ? p_prev[static_cast<size_t>(bh) * KD + n] : 0.f;
   if (seg_first > 0) {
-    const float r0 = rp[static_cast<size_t>(t_start / C) * hstep] - carry;
+    const float r0 = *rslot(t_start) - carry;
     float loc = 0.f;
     for (int t = 0; t < seg_first; ++t) {
       const size_t row = static_cast<size_t>(b) * T_new + t;
       loc = fmaf(load1(g_new + (row * HQ + hq) * KD + n), kLog2e, loc);
       const float kv = load1(k_new + (row * H + kvh) * KD + n);
-      store_one(k_tilde + ((static_cast<size_t>(b) * cap + t_start + t) * HQ + hq) * KD + n,
-                kv * ex2_approx(r0 - loc));
+      store_one(k_tilde + (pm.row(b, t_start + t) * HQ + hq) * KD + n, kv * ex2_approx(r0 - loc));
     }
     carry += loc;
   }
   for (int s = 0; s < nseg; ++s) {
-    float* rr = rp + static_cast<size_t>((t_start + seg_first + s * seg_rows) / C) * hstep;
+    float* rr = rslot(t_start + seg_first + s * seg_rows);
     const float tot = *rr;
     *rr = carry;
     carry += tot;
@@ -317,16 +321,15 @@ __global__ void __launch_bounds__(128) cache_segscan_kernel(
 template <typename T, int KD>
 __global__ void __launch_bounds__(128) cache_append_varlen_kernel(
     const T* __restrict__ k_new, const T* __restrict__ g_new, const float* __restrict__ p_prev,
-    const int* __restrict__ t_pos, int B, int cap, int HQ, int H, int C, T* __restrict__ k_tilde,
-    float* __restrict__ r_cache, float* __restrict__ p_last) {
+    const int* __restrict__ t_pos, int B, PageMap pm, int HQ, int H, int C,
+    T* __restrict__ k_tilde, float* __restrict__ r_cache, float* __restrict__ p_last) {
   constexpr int TPS = KD / 4;
   const long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= static_cast<long>(B) * HQ * TPS) return;
   const int ch = static_cast<int>(idx % TPS) * 4;
   const long bh = idx / TPS;
   const int b = static_cast<int>(bh / HQ), hq = static_cast<int>(bh % HQ), kvh = hq / (HQ / H);
-  const int t = min(max(t_pos[b], 0), cap - 1);  // clamped to the cache
-  const int ncap = (cap + C - 1) / C;
+  const int t = min(max(t_pos[b], 0), pm.rows() - 1);  // clamped to the cache
   Vec4<T> gv, kv;
   gv.load(g_new + (static_cast<size_t>(b) * HQ + hq) * KD + ch);
   kv.load(k_new + (static_cast<size_t>(b) * H + kvh) * KD + ch);
@@ -338,7 +341,7 @@ __global__ void __launch_bounds__(128) cache_append_varlen_kernel(
     const float prev = t > 0 ? p_prev[static_cast<size_t>(bh) * KD + ch + c] : 0.f;
     P[c] = fmaf(g[c], kLog2e, prev);
   }
-  float* rr = r_cache + ((static_cast<size_t>(b) * ncap + t / C) * HQ + hq) * KD + ch;
+  float* rr = r_cache + (pm.chunk(b, t, C) * HQ + hq) * KD + ch;
   if (t % C == 0) {
     *reinterpret_cast<float4*>(rr) = make_float4(P[0], P[1], P[2], P[3]);  // new chunk anchor
   } else {
@@ -348,7 +351,7 @@ __global__ void __launch_bounds__(128) cache_append_varlen_kernel(
     k[2] *= ex2_approx(R.z - P[2]);
     k[3] *= ex2_approx(R.w - P[3]);
   }
-  Vec4<T>::store(k_tilde + ((static_cast<size_t>(b) * cap + t) * HQ + hq) * KD + ch, k);
+  Vec4<T>::store(k_tilde + (pm.row(b, t) * HQ + hq) * KD + ch, k);
   *reinterpret_cast<float4*>(p_last + static_cast<size_t>(bh) * KD + ch) =
       make_float4(P[0], P[1], P[2], P[3]);
 }
@@ -357,7 +360,7 @@ template <typename T, int KD>
 cudaError_t append_varlen_impl(const CacheArgs& a, const int* t_pos, cudaStream_t st) {
   const long n = static_cast<long>(a.B) * a.HQ * (KD / 4);
   cache_append_varlen_kernel<T, KD><<<static_cast<unsigned>((n + 127) / 128), 128, 0, st>>>(
-      static_cast<const T*>(a.k_new), static_cast<const T*>(a.g_new), a.p_prev, t_pos, a.B, a.cap,
+      static_cast<const T*>(a.k_new), static_cast<const T*>(a.g_new), a.p_prev, t_pos, a.B, a.pm,
       a.HQ, a.H, a.chunk, static_cast<T*>(a.k_tilde), a.r_cache, a.p_last);
   return cudaGetLastError();
 }
@@ -418,26 +421,26 @@ cudaError_t cache_impl(const CacheArgs& a, cudaStream_t st) {
   }
   const int stage = CC::D * (hpc + nkv) * CC::ROWB;
   const int smem = CC::NS * stage + 2 * CC::NS * 8 + 16;
-  auto kern = cache_build_kernel<T, KD>;
+  auto kern = a.pm.paged() ? cache_build_kernel<T, KD, true> : cache_build_kernel<T, KD, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   if (nseg > 0) {
     cache_segsum_kernel<T, KD><<<dim3(a.HQ / hpc, a.B, nseg), 128, 0, st>>>(
-        static_cast<const T*>(a.g_new), a.t_start, a.T_new, a.cap, a.HQ, hpc, a.chunk, seg_first,
+        static_cast<const T*>(a.g_new), a.t_start, a.T_new, a.pm, a.HQ, hpc, a.chunk, seg_first,
         seg_rows, a.r_cache);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const long nthr = static_cast<long>(a.B) * a.HQ * KD;
     cache_segscan_kernel<T, KD><<<static_cast<unsigned>((nthr + 127) / 128), 128, 0, st>>>(
         static_cast<const T*>(a.k_new), static_cast<const T*>(a.g_new), a.p_prev, a.B, a.t_start,
-        a.T_new, a.cap, a.HQ, a.H, a.chunk, seg_first, seg_rows, nseg,
+        a.T_new, a.pm, a.HQ, a.H, a.chunk, seg_first, seg_rows, nseg,
         static_cast<T*>(a.k_tilde), a.r_cache, a.p_last);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   const int nwc = (hpc * CC::TPS + 31) / 32;
   dim3 grid(a.HQ / hpc, a.B, nseg > 0 ? nseg : 1);
-  kern<<<grid, (nwc + 1) * 32, smem, st>>>(tmG, tmK, a.p_prev, a.t_start, a.T_new, a.cap, a.HQ, G,
+  kern<<<grid, (nwc + 1) * 32, smem, st>>>(tmG, tmK, a.p_prev, a.t_start, a.T_new, a.pm, a.HQ, G,
                                            hpc, nkv, a.chunk, seg_first, seg_rows,
                                            static_cast<T*>(a.k_tilde), a.r_cache, a.p_last,
                                            a.err, a.wait_ns, a.fault);

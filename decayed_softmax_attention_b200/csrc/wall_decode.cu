@@ -86,12 +86,12 @@ struct DecCfg {
   static_assert(SR % NW == 0, "rows per stage must split over the consumer warps");
 };
 
-template <typename T, int KD, int VD, int G>
+template <typename T, int KD, int VD, int G, bool PAGED>
 __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_split_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
     const T* __restrict__ q, const float* __restrict__ p_curr, const float* __restrict__ r_cache,
-    int T_kv, int cap, int HQ, int C, int cps, int nsplit, float sc, float* __restrict__ part,
-    int* err, uint64_t wait_ns, int fault, const int* __restrict__ seqlens) {
+    int T_kv, int HQ, int C, int cps, int nsplit, float sc, float* __restrict__ part,
+    int* err, uint64_t wait_ns, int fault, const int* __restrict__ seqlens, PageMap pm) {
   using D = DecCfg<T, KD, VD, G>;
   constexpr int LPH = 32 / G;    // lanes per query head
   constexpr int CPL = KD / LPH;  // k_tilde channels per lane
@@ -109,7 +109,7 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
   // [1, T_kv]); splits past the end of a shorter row hold no rows
   const int T_b = seqlens ? max(1, min(seqlens[b], T_kv)) : T_kv;
   const int nchunks = (T_b + C - 1) / C;
-  const int ncap = (cap + C - 1) / C;
+  const int ncap = (pm.cap + C - 1) / C;  // anchor chunks per batch row (dense caches)
   const int ck0 = s * cps;
   const int ck1 = min(ck0 + cps, nchunks);
   const int row_begin = ck0 * C;
@@ -139,11 +139,16 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
         const int row0 = row_begin + i * D::SR;
         uint8_t* st = dsm + slot * D::STAGE;
         if (!(fault == 2 && i == 0)) {  // testing hook: starve the consumers
+          // a stage never straddles a cache block: it starts on a chunk
+          // boundary plus a multiple of SR, and SR divides C divides the block
+          const int trow = PAGED ? static_cast<int>(pm.row(b, row0)) : row0;
+          const int tb = PAGED ? 0 : b;
+          const size_t rslot = PAGED ? pm.chunk(b, row0, C)
+                                     : static_cast<size_t>(b) * ncap + row0 / C;
           mbar_arrive_expect_tx(&full[slot], D::STAGE);
-          tma_load_4d(st, &tmK, &full[slot], 0, h * G, row0, b);
-          tma_load_4d(st + D::K_BYTES, &tmV, &full[slot], 0, h, row0, b);
-          bulk_load(st + D::K_BYTES + D::V_BYTES,
-                    r_cache + ((static_cast<size_t>(b) * ncap + row0 / C) * HQ + h * G) * KD,
+          tma_load_4d(st, &tmK, &full[slot], 0, h * G, trow, tb);
+          tma_load_4d(st + D::K_BYTES, &tmV, &full[slot], 0, h, trow, tb);
+          bulk_load(st + D::K_BYTES + D::V_BYTES, r_cache + (rslot * HQ + h * G) * KD,
                     D::R_BYTES, &full[slot]);
         }
         issued = i + 1;
@@ -190,6 +195,11 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
         load_n<T, CPL>(reinterpret_cast<const T*>(st) + (r0 + rr) * D::GK + lane * CPL, kf);
         load_n<T, VPL>(reinterpret_cast<const T*>(st + D::K_BYTES) + (r0 + rr) * VD + lane * VPL,
                        vv[rr]);
+        if (PAGED && row0 + r0 + rr >= row_end) {
+          // past this row's length: a paged block may hold anything there
+#pragma unroll
+          for (int c = 0; c < VPL; ++c) vv[rr][c] = 0.f;
+        }
         float d = 0.f;
 #pragma unroll
         for (int e = 0; e < CPL; ++e) d = fmaf(qt[e], kf[e], d);
@@ -314,36 +324,43 @@ cudaError_t decode_impl(const DecodeArgs& a, cudaStream_t st) {
   const CUtensorMapDataType tdt =
       sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   CUtensorMap tmK, tmV;
-  {  // k_tilde [B, cap, HQ, K], rows limited to T_kv
-    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(KD), static_cast<cuuint64_t>(a.HQ),
-                                static_cast<cuuint64_t>(a.T_kv), static_cast<cuuint64_t>(a.B)};
+  // dense: [B, cap, ...] with rows limited to T_kv; paged: the pool as one
+  // batch row of nblk * bs rows
+  const bool paged = a.pm.paged();
+  const cuuint64_t rows = paged ? static_cast<cuuint64_t>(a.pm.nblk) * a.pm.bs
+                                : static_cast<cuuint64_t>(a.T_kv);
+  const cuuint64_t rstride = paged ? rows : static_cast<cuuint64_t>(a.cap);
+  const cuuint64_t nb = paged ? 1 : static_cast<cuuint64_t>(a.B);
+  {  // k_tilde
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(KD), static_cast<cuuint64_t>(a.HQ), rows,
+                                nb};
     const cuuint64_t strides[3] = {static_cast<cuuint64_t>(KD) * sizeof(T),
                                    static_cast<cuuint64_t>(a.HQ) * KD * sizeof(T),
-                                   static_cast<cuuint64_t>(a.cap) * a.HQ * KD * sizeof(T)};
+                                   rstride * a.HQ * KD * sizeof(T)};
     const cuuint32_t box[4] = {static_cast<cuuint32_t>(KD), static_cast<cuuint32_t>(G),
                                static_cast<cuuint32_t>(D::SR), 1};
     if (!encode_tiled(&tmK, tdt, 4, a.k_tilde, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   }
-  {  // v [B, cap, H, V]
-    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(VD), static_cast<cuuint64_t>(a.H),
-                                static_cast<cuuint64_t>(a.T_kv), static_cast<cuuint64_t>(a.B)};
+  {  // v
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(VD), static_cast<cuuint64_t>(a.H), rows,
+                                nb};
     const cuuint64_t strides[3] = {static_cast<cuuint64_t>(VD) * sizeof(T),
                                    static_cast<cuuint64_t>(a.H) * VD * sizeof(T),
-                                   static_cast<cuuint64_t>(a.cap) * a.H * VD * sizeof(T)};
+                                   rstride * a.H * VD * sizeof(T)};
     const cuuint32_t box[4] = {static_cast<cuuint32_t>(VD), 1, static_cast<cuuint32_t>(D::SR), 1};
     if (!encode_tiled(&tmV, tdt, 4, a.v, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   }
-  auto kern = decode_split_kernel<T, KD, VD, G>;
+  auto kern = paged ? decode_split_kernel<T, KD, VD, G, true> : decode_split_kernel<T, KD, VD, G, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, D::SMEM);
   if (e != cudaSuccess) return e;
   const int nchunks = (a.T_kv + a.chunk - 1) / a.chunk;
   const int cps = (nchunks + a.nsplit - 1) / a.nsplit;
   dim3 grid(a.nsplit, a.H, a.B);
   kern<<<grid, (D::NW + 1) * 32, D::SMEM, st>>>(
-      tmK, tmV, static_cast<const T*>(a.q), a.p_curr, a.r_cache, a.T_kv, a.cap, a.HQ, a.chunk,
-      cps, a.nsplit, a.scale * kLog2e, a.part, a.err, a.wait_ns, a.fault, a.seqlens);
+      tmK, tmV, static_cast<const T*>(a.q), a.p_curr, a.r_cache, a.T_kv, a.HQ, a.chunk,
+      cps, a.nsplit, a.scale * kLog2e, a.part, a.err, a.wait_ns, a.fault, a.seqlens, a.pm);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (a.mid_event != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(a.mid_event), st);

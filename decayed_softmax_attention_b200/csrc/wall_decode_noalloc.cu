@@ -82,6 +82,7 @@ extern "C" wall_status_t wall_attn_decode_noalloc(
   wall::DecodeArgs a;
   a.q = q; a.p_curr = p_curr; a.v = v; a.k_tilde = k_tilde; a.r_cache = r_cache;
   a.sink = sink_bias; a.B = B; a.T_kv = T_kv; a.cap = cap; a.HQ = HQ; a.H = H; a.K = K;
+  a.pm.cap = cap;
   a.V = V; a.chunk = chunk; a.scale = scale; a.o = o; a.lse = lse;
   a.part = scratch; a.nsplit = ns; a.mid_event = nullptr;
   a.err = wall::device_error_word();

@@ -126,6 +126,36 @@ cudaError_t launch_bwd(const BwdArgs& a, const FwdWork& fw, const BwdWork& bw, b
 cudaError_t launch_bwd_tc(const BwdArgs& a, const FwdWork& fw, const BwdWork& bw,
                           cudaStream_t st);
 
+// Where cache row t of batch row b lives.  Dense caches: row b * cap + t of a
+// [B, cap, ...] array.  Paged caches (block tables, as in PagedAttention): a
+// pool of nblk blocks of bs rows; row t of batch row b is row t % bs of block
+// bt[b * maxblk + t / bs] (clamped into the pool, so a bad table entry never
+// addresses memory outside it).  Anchor chunks of C rows never straddle a
+// block (bs is a multiple of C).
+struct PageMap {
+  const int* bt = nullptr;
+  int maxblk = 0, bs = 0, nblk = 0;
+  int cap = 0;
+  __host__ __device__ bool paged() const { return bt != nullptr; }
+  // rows a batch row can hold
+  __host__ __device__ int rows() const { return bt ? maxblk * bs : cap; }
+#ifdef __CUDACC__
+  __device__ __forceinline__ int block_of(int b, int t) const {
+    const int pb = __ldg(bt + static_cast<size_t>(b) * maxblk + t / bs);
+    return pb < 0 ? 0 : (pb >= nblk ? nblk - 1 : pb);
+  }
+  __device__ __forceinline__ size_t row(int b, int t) const {
+    if (!bt) return static_cast<size_t>(b) * cap + t;
+    return static_cast<size_t>(block_of(b, t)) * bs + t % bs;
+  }
+  // anchor slot of the chunk holding row t
+  __device__ __forceinline__ size_t chunk(int b, int t, int C) const {
+    if (!bt) return static_cast<size_t>(b) * ((cap + C - 1) / C) + t / C;
+    return static_cast<size_t>(block_of(b, t)) * (bs / C) + (t % bs) / C;
+  }
+#endif
+};
+
 struct CacheArgs {
   const void* k_new;
   const void* g_new;
@@ -137,6 +167,7 @@ struct CacheArgs {
   int* err;          // device error word (bounded waits)
   uint64_t wait_ns;  // limit of each bounded wait
   int fault;         // testing hook: 3 = producer skips its first stage
+  PageMap pm;        // paged cache (pm.bt set) or dense (pm.cap = cap)
 };
 cudaError_t launch_cache_build(const CacheArgs& a, bool bf16, cudaStream_t st);
 // One token per batch row at row b's own position t_pos[b] (device int32 [B]).
@@ -160,6 +191,7 @@ struct DecodeArgs {
   uint64_t wait_ns; // bounded-wait limit
   int fault;        // testing hook: 2 = producer skips its first stage
   const int* seqlens = nullptr;  // optional device int32 [B]: rows of each batch row's cache
+  PageMap pm;                    // paged cache (pm.bt set; seqlens required) or dense
 };
 int decode_max_splits(int B, int T_kv, int HQ, int H, int chunk);
 int decode_num_splits(int B, int T_kv, int HQ, int H, int chunk);

@@ -176,8 +176,8 @@ wall_status_t wall_build_kv_cache(const void* k_new, const void* g_new, const fl
                                   float* p_last, wall_stream_t stream);
 
 /*
- * One-token append per batch row at that row's own position (SURVEY next row:
- * per-sequence cache lengths; Wall Attention README, "Decode" append): for each
+ * One-token append per batch row at that row's own position (batches whose
+ * sequences have different lengths; Wall Attention README, "Decode" append): for each
  * b, row t = t_pos[b] of the cache gets k_tilde from k_new[b] and g_new[b];
  * a chunk starting at t gets its anchor; p_last[b] = P at row t.
  *   k_new [B, 1, H, K], g_new [B, 1, HQ, K]  dtype dt
@@ -223,9 +223,9 @@ wall_status_t wall_attn_decode(const void* q, const float* p_curr, const void* v
                                size_t workspace_bytes, wall_stream_t stream);
 
 /*
- * Decode over a batch whose cached sequences have different lengths (SURVEY
- * next row: per-sequence cache lengths; the README's decode takes one length
- * for the batch).  Same as wall_attn_decode except:
+ * Decode over a batch whose cached sequences have different lengths (the
+ * README's decode takes one length for the whole batch).  Same as
+ * wall_attn_decode except:
  *   seqlens_kv  device int32 [B]: batch row b attends its cache rows
  *               0 .. seqlens_kv[b] - 1; values must lie in [1, max_T_kv]
  *               (they are clamped to it on the device)
@@ -240,6 +240,49 @@ wall_status_t wall_attn_decode_varlen(const void* q, const float* p_curr, const 
                                       int chunk, wall_dtype_t dt, float scale, void* o,
                                       float* lse, void* workspace, size_t workspace_bytes,
                                       wall_stream_t stream);
+
+/*
+ * Paged decode caches (block tables, after the PagedAttention scheme the pages
+ * describe: a pool of fixed-size physical blocks; each sequence lists the
+ * blocks that hold its logical rows).  Row t of batch row b lives in row
+ * t % block_size of pool block block_table[b * max_blocks + t / block_size].
+ *   block_table  device int32 [B, max_blocks]; entries must lie in
+ *                [0, num_blocks) (they are clamped into the pool on the device,
+ *                so a bad entry never addresses memory outside it)
+ *   k_tilde_pool [num_blocks, block_size, HQ, K]  dtype dt
+ *   r_pool       [num_blocks, block_size / chunk, HQ, K] fp32 (anchors of the
+ *                block's chunks)
+ *   v_pool       [num_blocks, block_size, H, V]   dtype dt (caller-written, as
+ *                the dense v cache)
+ * block_size must be a multiple of chunk (so a chunk never straddles a block).
+ * Each call is the dense call of the same name with the cache rows addressed
+ * through the table; a batch row's capacity is max_blocks * block_size rows.
+ * wall_attn_decode_paged requires seqlens_kv (as wall_attn_decode_varlen);
+ * size its workspace with wall_attn_decode_workspace_size(B, max_blocks *
+ * block_size, HQ, H, V, chunk).
+ */
+wall_status_t wall_build_kv_cache_paged(const void* k_new, const void* g_new,
+                                        const float* p_prev, const int32_t* block_table,
+                                        int max_blocks, int B, int t_start, int T_new,
+                                        int num_blocks, int block_size, int HQ, int H, int K,
+                                        int chunk, wall_dtype_t dt, void* k_tilde_pool,
+                                        float* r_pool, float* p_last, wall_stream_t stream);
+
+wall_status_t wall_append_kv_cache_paged(const void* k_new, const void* g_new,
+                                         const float* p_prev, const int32_t* t_pos,
+                                         const int32_t* block_table, int max_blocks, int B,
+                                         int num_blocks, int block_size, int HQ, int H, int K,
+                                         int chunk, wall_dtype_t dt, void* k_tilde_pool,
+                                         float* r_pool, float* p_last, wall_stream_t stream);
+
+wall_status_t wall_attn_decode_paged(const void* q, const float* p_curr, const void* v_pool,
+                                     const void* k_tilde_pool, const float* r_pool,
+                                     const float* sink_bias, const int32_t* seqlens_kv,
+                                     const int32_t* block_table, int max_blocks, int B,
+                                     int num_blocks, int block_size, int HQ, int H, int K, int V,
+                                     int chunk, wall_dtype_t dt, float scale, void* o, float* lse,
+                                     void* workspace, size_t workspace_bytes,
+                                     wall_stream_t stream);
 
 /*
  * Decode without scratch allocation (no counterpart in the paper: this entry

@@ -19,7 +19,7 @@
  *   - "Decode (cache build)": P = cumsum(g) * (1/ln 2) (exp2 domain),
  *     k_tilde[j] = k[j] * exp2(R_c - P[j]) with one anchor vector R_c per
  *     chunk of C tokens; the decode reads k_tilde and r_cache.
- * Readings of points the page leaves open (each is also listed in the design doc):
+ * Readings of points the page leaves open:
  *   - scale multiplies only the decayed q.k sum (not g_scalar, not the sink);
  *   - g_scalar adds Gs[i] - Gs[j] to the logit, Gs its inclusive cumsum;
  *   - sink_bias is one extra logit per head with a zero value vector;

@@ -269,3 +269,54 @@ def test_bwd_workspace_size(lib):
     # the prepass's workspace plus fp32 accumulators of dq, dk_h and dv_h
     assert bwd >= fwd + 3 * 8 * 1024 * 64 * 4
     assert lib.wall_attn_bwd_workspace_size(0, 1024, 8, 4, 64, 64, BF16) == 0
+
+
+def test_paged_host_validation(lib):
+    def dec(**kw):
+        a = dict(q=_fake(), p=_fake(), vp=_fake(), kp=_fake(), rp=_fake(), sink=None,
+                 sl=_fake(0x7000), bt=_fake(0x8000), maxblk=4, B=2, nblk=8, bs=64, HQ=4, H=2,
+                 K=128, V=128, C=64, dt=BF16, scale=0.0, o=_fake(), lse=None, ws=_fake(),
+                 wsb=1 << 30, stream=None)
+        a.update(kw)
+        return lib.wall_attn_decode_paged(a["q"], a["p"], a["vp"], a["kp"], a["rp"], a["sink"],
+                                          a["sl"], a["bt"], a["maxblk"], a["B"], a["nblk"], a["bs"],
+                                          a["HQ"], a["H"], a["K"], a["V"], a["C"], a["dt"],
+                                          a["scale"], a["o"], a["lse"], a["ws"], a["wsb"],
+                                          a["stream"])
+    assert dec(bt=None) == INVALID            # the block table is required
+    assert dec(sl=None) == INVALID            # so are the per-sequence lengths
+    assert dec(bs=96) == UNSUPPORTED          # block size not a multiple of the chunk
+    assert dec(bs=32) == UNSUPPORTED          # smaller than the chunk
+    assert dec(maxblk=0) == INVALID
+    assert dec(nblk=0) == INVALID
+    assert dec(bt=_fake(0x8002)) == INVALID   # misaligned table
+    assert dec(wsb=16) == WORKSPACE
+    assert dec(B=0) == 0
+
+    def app(**kw):
+        a = dict(k=_fake(), g=_fake(), pp=_fake(), tp=_fake(0x6000), bt=_fake(0x8000), maxblk=4,
+                 B=2, nblk=8, bs=64, HQ=4, H=2, K=64, C=64, dt=BF16, kp=_fake(), rp=_fake(),
+                 pl=_fake(), stream=None)
+        a.update(kw)
+        return lib.wall_append_kv_cache_paged(a["k"], a["g"], a["pp"], a["tp"], a["bt"], a["maxblk"],
+                                              a["B"], a["nblk"], a["bs"], a["HQ"], a["H"], a["K"],
+                                              a["C"], a["dt"], a["kp"], a["rp"], a["pl"], a["stream"])
+    assert app(bt=None) == INVALID
+    assert app(tp=None) == INVALID
+    assert app(bs=100) == UNSUPPORTED
+    assert app(B=0) == 0
+
+    def build(**kw):
+        a = dict(k=_fake(), g=_fake(), pp=None, bt=_fake(0x8000), maxblk=4, B=2, t0=0, Tn=100,
+                 nblk=8, bs=64, HQ=4, H=2, K=128, C=64, dt=BF16, kp=_fake(), rp=_fake(),
+                 pl=_fake(), stream=None)
+        a.update(kw)
+        return lib.wall_build_kv_cache_paged(a["k"], a["g"], a["pp"], a["bt"], a["maxblk"], a["B"],
+                                             a["t0"], a["Tn"], a["nblk"], a["bs"], a["HQ"], a["H"],
+                                             a["K"], a["C"], a["dt"], a["kp"], a["rp"], a["pl"],
+                                             a["stream"])
+    assert build(Tn=300) == INVALID           # more rows than max_blocks * block_size
+    assert build(t0=64) == INVALID            # appending needs p_prev
+    assert build(bt=None) == INVALID
+    assert build(bs=48) == UNSUPPORTED
+    assert build(Tn=0) == 0
