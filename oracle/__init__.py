@@ -10,7 +10,8 @@ Functions (each follows the Wall Attention README; see the C file's header for
 the exact formulas and the readings taken where the page is silent):
   wall_fwd           -- prefill forward by the pairwise definition
   kv_cache           -- P, r_cache and k_tilde of the "Decode" section
-  decode_from_cache  -- one decode step over (k_tilde, r_cache)
+  decode_from_cache  -- one decode step over (k_tilde, r_cache), optionally with the gate
+  gate_cache         -- the scalar gate's prefix PS in exp2 units (decode with g_scalar)
   wall_bwd           -- gradients of the prefill forward (analytic, by the definition)
 """
 from __future__ import annotations
@@ -52,7 +53,8 @@ def _load():
     i, d, i64 = ctypes.c_int, ctypes.c_double, ctypes.c_int64
     lib.wall_oracle_fwd.argtypes = [P, P, P, P, P, P, i, P, i, i, i, i, i, i, i, d, P, i64, P, P, i]
     lib.wall_oracle_kv_cache.argtypes = [P, P, i, i, i, i, i, i, P, P, P, P, i]
-    lib.wall_oracle_decode_cache.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, i, i, d, P, P, i]
+    lib.wall_oracle_decode_cache.argtypes = [P, P, P, P, P, P, P, P, i, i, i, i, i, i, i, i, d, P,
+                                             P, i]
     lib.wall_oracle_bwd.argtypes = [P, P, P, P, P, P, i, P, i, i, i, i, i, i, i, d, P, P,
                                     P, P, P, P, P, P, P, P, P, i]
     for f in (lib.wall_oracle_fwd, lib.wall_oracle_kv_cache, lib.wall_oracle_decode_cache,
@@ -148,12 +150,21 @@ def kv_cache(k, g, HQ=None, chunk=64, anchors=None, threads=0):
     return kt, rc_, P
 
 
+def gate_cache(g_scalar):
+    """PS = cumsum(g_scalar over time) * (1/ln 2) [B,T,HQ] (double): the scalar gate's prefix in
+    the exp2 units of the decode cache."""
+    gs = np.asarray(_f32(g_scalar), dtype=np.float64)
+    return np.cumsum(gs, axis=1) / np.log(2.0)
+
+
 def decode_from_cache(q, p_curr, v, k_tilde, r_cache, T_kv, sink_bias=None, chunk=64,
-                      scale=None, threads=0):
+                      scale=None, gs_curr=None, gs_cache=None, threads=0):
     """One decode step over the pre-rescaled cache (double).
 
     q [B,HQ,K] (or [B,1,HQ,K]); p_curr [B,HQ,K]; v [B,cap,H,V]; k_tilde [B,cap,HQ,K];
     r_cache [B,ceil(cap/C),HQ,K]; the first T_kv cache rows are attended.
+    gs_curr [B,HQ] / gs_cache [B,cap,HQ] (optional, together): the scalar gate's prefix PS
+    (see gate_cache) at the current row and at every cache row.
     Returns (o [B,HQ,V], lse [B,HQ]).
     """
     q = _f32(q)
@@ -167,7 +178,12 @@ def decode_from_cache(q, p_curr, v, k_tilde, r_cache, T_kv, sink_bias=None, chun
         scale = K ** -0.5
     o = np.empty((B, HQ, V), dtype=np.float64)
     lse = np.empty((B, HQ), dtype=np.float64)
+    gcur = None if gs_curr is None else _f64(np.asarray(gs_curr).reshape(B, HQ))
+    gcache = None if gs_cache is None else _f64(gs_cache)
+    if (gcur is None) != (gcache is None):
+        raise ValueError("gs_curr and gs_cache go together")
     rc = _load().wall_oracle_decode_cache(_ptr(q), _ptr(p), _ptr(v), _ptr(kt), _ptr(r), _ptr(sink),
+                                          _ptr(gcur), _ptr(gcache),
                                           B, int(T_kv), cap, HQ, H, K, V, int(chunk), float(scale),
                                           _ptr(o), _ptr(lse), int(threads))
     _check(rc, "decode_from_cache")

@@ -215,9 +215,13 @@ int wall_oracle_kv_cache(const float* k, const float* g, int B, int T, int HQ, i
  *   softmax over j (plus the optional sink logit), o = sum_j w_j v[j].
  * q [B,HQ,K] float; p_curr [B,HQ,K], k_tilde [B,cap,HQ,K], r_cache
  * [B,ceil(cap/C),HQ,K] double; v [B,cap,H,V] float.  o [B,HQ,V], lse [B,HQ].
+ * With the scalar gate (gs_curr [B,HQ] and gs_cache [B,cap,HQ], both double,
+ * nullable together): PS = cumsum(g_scalar) * (1/ln 2) in the same exp2 units
+ * as P, and the logit gains (gs_curr - gs_cache[j]) * ln 2 = Gs[t] - Gs[j].
  */
 int wall_oracle_decode_cache(const float* q, const double* p_curr, const float* v,
                              const double* k_tilde, const double* r_cache, const float* sink,
+                             const double* gs_curr, const double* gs_cache,
                              int B, int T_kv, int cap, int HQ, int H, int K, int V, int C,
                              double scale, double* o, double* lse, int nthreads) {
   if (B <= 0 || T_kv <= 0 || cap < T_kv || HQ <= 0 || H <= 0 || K <= 0 || V <= 0 || C <= 0 ||
@@ -246,6 +250,9 @@ int wall_oracle_decode_cache(const float* q, const double* p_curr, const float* 
           double dot = 0.0;
           for (int n = 0; n < K; ++n) dot += (double)qv[n] * kt[n] * exp2(pc[n] - R[n]);
           x[j] = scale * dot;
+          if (gs_cache)
+            x[j] += (gs_curr[(size_t)b * HQ + hq] - gs_cache[((size_t)b * cap + j) * HQ + hq]) *
+                    log(2.0);
           if (x[j] > M) M = x[j];
         }
         const double sb = sink ? (double)sink[hq] : -INFINITY;

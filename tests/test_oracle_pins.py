@@ -338,3 +338,30 @@ def test_plausible_mistakes_are_caught():
     o_rep, _ = oracle.wall_fwd(d2["q"], k_rep, v_rep, d2["g"])
     np.testing.assert_allclose(o_rep, o2, rtol=1e-13, atol=1e-13)
     assert np.max(np.abs(o_alt - o2)) > 1e-3
+
+
+def test_decode_with_gate_equals_prefill_rows_with_g_scalar():
+    """The scalar gate in decode: PS = cumsum(g_scalar)/ln2 per row, the logit gains
+    (PS_t - PS_j) ln 2; decode at step t equals the prefill row t with g_scalar (README
+    "Tests": decode == prefill), with and without a sink."""
+    rng = np.random.default_rng(23)
+    B, T, HQ, H, K, V, C = 2, 70, 4, 2, 8, 5, 16
+    q, k, v = _rand(rng, B, T, HQ, K), _rand(rng, B, T, H, K), _rand(rng, B, T, H, V)
+    g = (-np.abs(0.4 * _rand(rng, B, T, HQ, K))).astype(np.float32)
+    gs = (-np.abs(0.7 * _rand(rng, B, T, HQ))).astype(np.float32)
+    kt, r, P = oracle.kv_cache(k, g, chunk=C)
+    PS = oracle.gate_cache(gs)
+    np.testing.assert_allclose(PS[:, -1] * np.log(2.0), gs.astype(np.float64).sum(axis=1),
+                               rtol=1e-12)
+    for sink in (None, _rand(rng, HQ)):
+        o_pre, lse_pre = oracle.wall_fwd(q, k, v, g, gs, sink_bias=sink)
+        for t in (0, 17, 33, T - 1):
+            o, lse = oracle.decode_from_cache(q[:, t], P[:, t], v, kt, r, T_kv=t + 1,
+                                              sink_bias=sink, chunk=C, gs_curr=PS[:, t],
+                                              gs_cache=PS)
+            np.testing.assert_allclose(o, o_pre[:, t], rtol=1e-10, atol=1e-12)
+            np.testing.assert_allclose(lse, lse_pre[:, t], rtol=1e-10, atol=1e-12)
+        # without the gate terms the decode no longer matches (the gate matters here)
+        o, _ = oracle.decode_from_cache(q[:, T - 1], P[:, T - 1], v, kt, r, T_kv=T,
+                                        sink_bias=sink, chunk=C)
+        assert np.abs(o - o_pre[:, T - 1]).max() > 1e-3
