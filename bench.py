@@ -646,6 +646,36 @@ def run_ours(args, world, rank, local):
                          "decode_paged_frac_of_hbm": var_bytes / (pg_ms * 1e-3) / 1e9 / hbm_peak})
             del pws
         del kt_pool, v_pool, r_pool
+        # the same per-sequence-length decode with the scalar gate (a gate cache of PS rows)
+        gsd = (-torch.nn.functional.softplus(
+            torch.randn((dspec.B, T0, dspec.HQ), generator=torch.Generator(device=dev).manual_seed(77),
+                        device=dev) - 4.0)).to(torch.bfloat16)
+        gs_cache = torch.empty((dspec.B, cache.cap, dspec.HQ), dtype=torch.float32, device=dev)
+        gs_last = torch.empty((dspec.B, dspec.HQ), dtype=torch.float32, device=dev)
+        wall.wall_build_gate_cache(gsd, gs_cache, gs_last)
+        gws = torch.empty(wall.wall_attn_decode_workspace_size(
+            dspec.B, T0, dspec.HQ, dspec.H, dspec.V, dspec.C), dtype=torch.uint8, device=dev)
+
+        def dec_gated():
+            wall.wall_attn_decode_gated(qv, cache.p[:, None], gs_last, cache.v, cache.k_tilde,
+                                        cache.r_cache, gs_cache, T_kv=T0, seqlens=seqlens,
+                                        scale=dspec.K ** -0.5, chunk=dspec.C, out=dout,
+                                        workspace=gws)
+
+        dec_gated()
+        ga, gz = ev(), ev()
+        torch.cuda.synchronize()
+        ga.record()
+        for _ in range(10):
+            dec_gated()
+        gz.record()
+        torch.cuda.synchronize()
+        gt_ms = ga.elapsed_time(gz) / 10
+        gate_bytes = var_bytes + sum(int(L) for L in lens) * dspec.HQ * 4
+        side.update({"decode_gated_ms": gt_ms,
+                     "decode_gated_GBps": gate_bytes / (gt_ms * 1e-3) / 1e9,
+                     "decode_gated_frac_of_hbm": gate_bytes / (gt_ms * 1e-3) / 1e9 / hbm_peak})
+        del gs_cache, gs_last, gws, gsd
         side.update({"cache_build_prefix_ms": build_ms,
                      "cache_build_prefix_GBps": build_gbps,
                      "cache_build_roofline": {

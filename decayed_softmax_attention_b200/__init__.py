@@ -28,7 +28,8 @@ __all__ = [
     "wall_build_kv_cache", "wall_attn_decode", "wall_attn_decode_workspace_size",
     "wall_attn_decode_noalloc", "wall_append_kv_cache_varlen", "wall_attn_bwd",
     "wall_attn_bwd_workspace_size", "wall_build_kv_cache_paged", "wall_append_kv_cache_paged",
-    "wall_attn_decode_paged", "PagedKVCache", "wall_device_error", "wall_debug_set_fault", "wall_debug_set_stage_events", "KVCache",
+    "wall_attn_decode_paged", "PagedKVCache", "wall_build_gate_cache", "wall_append_gate_cache",
+    "wall_attn_decode_gated", "wall_device_error", "wall_debug_set_fault", "wall_debug_set_stage_events", "KVCache",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -50,6 +51,7 @@ EXPORTED_SYMBOLS = (
     "wall_attn_decode_noalloc", "wall_attn_fwd_with_cache", "wall_attn_decode_varlen",
     "wall_append_kv_cache_varlen", "wall_attn_bwd_workspace_size", "wall_attn_bwd",
     "wall_build_kv_cache_paged", "wall_append_kv_cache_paged", "wall_attn_decode_paged",
+    "wall_build_gate_cache", "wall_append_gate_cache", "wall_attn_decode_gated",
 )
 
 
@@ -102,6 +104,13 @@ def load_library():
     lib.wall_attn_decode_paged.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I,
                                            F, P, P, P, S, P]
     lib.wall_attn_decode_paged.restype = I
+    lib.wall_build_gate_cache.argtypes = [P, P, P, I, I, I, I, I, I, I, I, I, P, P, P]
+    lib.wall_build_gate_cache.restype = I
+    lib.wall_append_gate_cache.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P, P, P]
+    lib.wall_append_gate_cache.restype = I
+    lib.wall_attn_decode_gated.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I,
+                                           I, I, I, F, P, P, P, S, P]
+    lib.wall_attn_decode_gated.restype = I
     lib.wall_build_kv_cache.argtypes = [P, P, P, I, I, I, I, I, I, I, I, I, P, P, P, P]
     lib.wall_build_kv_cache.restype = I
     lib.wall_append_kv_cache_varlen.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P, P, P, P]
@@ -439,6 +448,82 @@ def wall_attn_decode_paged(q, p_curr, v_pool, k_tilde_pool, r_pool, seqlens, blo
     return out
 
 
+# ----------------------------------------------------------------- scalar gate in decode
+def _gate_table(gs_cache, block_table):
+    """(block_table, max_blocks, num_blocks, block_size, cap) for a dense or paged gate cache."""
+    if block_table is None:
+        return None, 0, 0, 0, gs_cache.shape[1]
+    return block_table, block_table.shape[1], gs_cache.shape[0], gs_cache.shape[1], 0
+
+
+def wall_build_gate_cache(gs_new, gs_cache, gs_last, t_start=0, gs_prev=None, block_table=None):
+    """PS rows t_start .. t_start+T_new-1 of the scalar-gate cache from gs_new [B,T_new,HQ]."""
+    lib = load_library()
+    B, T_new, HQ = gs_new.shape
+    bt, mb, nb, bs, cap = _gate_table(gs_cache, block_table)
+    st = lib.wall_build_gate_cache(
+        _dev(gs_new, "gs_new", gs_new.dtype), _dev(gs_prev, "gs_prev", torch.float32, (B, HQ)),
+        _dev(bt, "block_table", torch.int32), mb, nb, bs, B, int(t_start), T_new, cap, HQ,
+        _dtype_code(gs_new), _dev(gs_cache, "gs_cache", torch.float32),
+        _dev(gs_last, "gs_last", torch.float32, (B, HQ)), _stream(gs_new.device))
+    _check(st, "wall_build_gate_cache")
+    return gs_last
+
+
+def wall_append_gate_cache(gs_new, gs_cache, gs_last, t_pos, gs_prev=None, block_table=None):
+    """One gate row per batch row at t_pos[b] from gs_new [B,1,HQ] (gs_prev defaults to gs_last)."""
+    lib = load_library()
+    B, _, HQ = gs_new.shape
+    bt, mb, nb, bs, cap = _gate_table(gs_cache, block_table)
+    if gs_prev is None:
+        gs_prev = gs_last
+    st = lib.wall_append_gate_cache(
+        _dev(gs_new, "gs_new", gs_new.dtype, (B, 1, HQ)),
+        _dev(gs_prev, "gs_prev", torch.float32, (B, HQ)), _dev(t_pos, "t_pos", torch.int32, (B,)),
+        _dev(bt, "block_table", torch.int32), mb, nb, bs, B, cap, HQ, _dtype_code(gs_new),
+        _dev(gs_cache, "gs_cache", torch.float32), _dev(gs_last, "gs_last", torch.float32, (B, HQ)),
+        _stream(gs_new.device))
+    _check(st, "wall_append_gate_cache")
+    return gs_last
+
+
+def wall_attn_decode_gated(q, p_curr, gs_curr, v, k_tilde, r_cache, gs_cache, T_kv=None,
+                           seqlens=None, block_table=None, sink_bias=None, scale=None, chunk=64,
+                           out=None, lse=None, workspace=None):
+    """wall_attn_decode (dense; T_kv rows or per-row seqlens) or wall_attn_decode_paged
+    (block_table + seqlens) with the scalar gate: gs_curr [B,HQ] = PS at the current row."""
+    lib = load_library()
+    B = q.shape[0]
+    dt = k_tilde.dtype
+    if block_table is None:
+        _, cap, HQ, K = k_tilde.shape
+        H, V = v.shape[2], v.shape[3]
+        mb = nb = bs = 0
+        rows = int(T_kv)
+    else:
+        nb, bs, HQ, K = k_tilde.shape
+        H, V = v.shape[2], v.shape[3]
+        mb = block_table.shape[1]
+        cap = rows = mb * bs
+    if out is None:
+        out = torch.empty((B, 1, HQ, V), dtype=dt, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(wall_attn_decode_workspace_size(B, rows, HQ, H, V, chunk), 1),
+                                dtype=torch.uint8, device=q.device)
+    st = lib.wall_attn_decode_gated(
+        _dev(q, "q", dt), _dev(p_curr, "p_curr", torch.float32),
+        _dev(gs_curr, "gs_curr", torch.float32), _dev(v, "v", dt), _dev(k_tilde, "k_tilde", dt),
+        _dev(r_cache, "r_cache", torch.float32), _dev(gs_cache, "gs_cache", torch.float32),
+        _dev(sink_bias, "sink_bias", torch.float32, (HQ,)),
+        _dev(seqlens, "seqlens", torch.int32, (B,)), _dev(block_table, "block_table", torch.int32),
+        mb, nb, bs, B, rows, cap, HQ, H, K, V, int(chunk), _dtype_code(k_tilde),
+        float(scale) if scale else 0.0, _dev(out, "out", dt), _dev(lse, "lse", torch.float32),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(q.device))
+    _check(st, "wall_attn_decode_gated")
+    return out
+
+
 def wall_attn_decode_noalloc(q, p_curr, v, k_tilde, r_cache, T_kv, out, lse=None,
                              sink_bias=None, scale=None, chunk=64):
     """wall_attn_decode without a workspace: the split partials live in a fixed
@@ -483,8 +568,12 @@ class KVCache:
     the next decode step.
     """
 
-    def __init__(self, B, cap, HQ, H, K, V, dtype=torch.bfloat16, chunk=64, device="cuda"):
+    def __init__(self, B, cap, HQ, H, K, V, dtype=torch.bfloat16, chunk=64, device="cuda",
+                 gate=False):
         self.B, self.cap, self.HQ, self.H, self.K, self.V, self.chunk = B, cap, HQ, H, K, V, chunk
+        # scalar gate (models with g_scalar): PS per row and head, and PS at the last row
+        self.gs_cache = torch.empty((B, cap, HQ), dtype=torch.float32, device=device) if gate else None
+        self.gs = torch.zeros((B, HQ), dtype=torch.float32, device=device) if gate else None
         nc = (cap + chunk - 1) // chunk
         self.k_tilde = torch.empty((B, cap, HQ, K), dtype=dtype, device=device)
         self.r_cache = torch.empty((B, nc, HQ, K), dtype=torch.float32, device=device)
@@ -494,17 +583,27 @@ class KVCache:
         self.workspace = torch.empty(max(wall_attn_decode_workspace_size(B, cap, HQ, H, V, chunk), 1),
                                      dtype=torch.uint8, device=device)
 
-    def append(self, k_new, g_new, v_new=None):
+    def append(self, k_new, g_new, v_new=None, gs_new=None):
         T_new = k_new.shape[1]
         if v_new is not None:
             self.v[:, self.length:self.length + T_new].copy_(v_new)
         wall_build_kv_cache(k_new, g_new, self.k_tilde, self.r_cache, self.p,
                             t_start=self.length, p_prev=self.p if self.length > 0 else None,
                             chunk=self.chunk)
+        if self.gs_cache is not None:
+            if gs_new is None:
+                raise ValueError("this cache carries the scalar gate: pass gs_new")
+            wall_build_gate_cache(gs_new, self.gs_cache, self.gs, t_start=self.length,
+                                  gs_prev=self.gs if self.length > 0 else None)
         self.length += T_new
         return self.p
 
     def decode(self, q, sink_bias=None, scale=None, out=None, lse=None):
+        if self.gs_cache is not None:
+            return wall_attn_decode_gated(q, self.p, self.gs, self.v, self.k_tilde, self.r_cache,
+                                          self.gs_cache, T_kv=self.length, sink_bias=sink_bias,
+                                          scale=scale, chunk=self.chunk, out=out, lse=lse,
+                                          workspace=self.workspace)
         return wall_attn_decode(q, self.p, self.v, self.k_tilde, self.r_cache, self.length,
                                 sink_bias=sink_bias, scale=scale, chunk=self.chunk, out=out,
                                 lse=lse, workspace=self.workspace)
@@ -520,7 +619,7 @@ class PagedKVCache:
     """
 
     def __init__(self, B, num_blocks, block_size, max_blocks, HQ, H, K, V, dtype=torch.bfloat16,
-                 chunk=64, device="cuda"):
+                 chunk=64, device="cuda", gate=False):
         if block_size % chunk:
             raise ValueError("block_size must be a multiple of chunk")
         self.B, self.HQ, self.H, self.K, self.V, self.chunk = B, HQ, H, K, V, chunk
@@ -530,6 +629,9 @@ class PagedKVCache:
                                    device=device)
         self.v = torch.zeros((num_blocks, block_size, H, V), dtype=dtype, device=device)
         self.p = torch.zeros((B, HQ, K), dtype=torch.float32, device=device)
+        self.gs_cache = (torch.empty((num_blocks, block_size, HQ), dtype=torch.float32,
+                                     device=device) if gate else None)
+        self.gs = torch.zeros((B, HQ), dtype=torch.float32, device=device) if gate else None
         self.free = list(range(num_blocks))
         self.host_table = [[] for _ in range(B)]
         self.block_table = torch.zeros((B, max_blocks), dtype=torch.int32, device=device)
@@ -570,26 +672,34 @@ class PagedKVCache:
         bs = self.block_size
         return [self.host_table[b][t // bs] * bs + t % bs for t in range(t0, t1)]
 
-    def prefill(self, k, g, v):
+    def prefill(self, k, g, v, gs=None):
         """Build rows 0 .. T-1 of every batch row (all rows start empty)."""
         B, T = k.shape[0], k.shape[1]
         for b in range(B):
             self.reserve(b, T)
         wall_build_kv_cache_paged(k, g, self.block_table, self.k_tilde, self.r_cache, self.p,
                                   t_start=0, chunk=self.chunk)
+        if self.gs_cache is not None:
+            if gs is None:
+                raise ValueError("this cache carries the scalar gate: pass gs")
+            wall_build_gate_cache(gs, self.gs_cache, self.gs, block_table=self.block_table)
         for b in range(B):
             rows = torch.tensor(self.rows_of(b, 0, T), device=self.v.device)
             self.v.view(-1, self.H, self.V)[rows] = v[b]
             self.lengths[b] = T
         return self.p
 
-    def append(self, k_new, g_new, v_new, t_pos):
+    def append(self, k_new, g_new, v_new, t_pos, gs_new=None):
         """One token per batch row at t_pos (host list of ints) = each row's current length."""
         for b, t in enumerate(t_pos):
             self.reserve(b, t + 1)
         tp = torch.tensor(t_pos, dtype=torch.int32, device=k_new.device)
         wall_append_kv_cache_paged(k_new, g_new, self.block_table, self.k_tilde, self.r_cache,
                                    self.p, tp, chunk=self.chunk)
+        if self.gs_cache is not None:
+            if gs_new is None:
+                raise ValueError("this cache carries the scalar gate: pass gs_new")
+            wall_append_gate_cache(gs_new, self.gs_cache, self.gs, tp, block_table=self.block_table)
         rows = torch.tensor([self.rows_of(b, t, t + 1)[0] for b, t in enumerate(t_pos)],
                             device=self.v.device)
         self.v.view(-1, self.H, self.V)[rows] = v_new[:, 0]
@@ -599,6 +709,12 @@ class PagedKVCache:
 
     def decode(self, q, sink_bias=None, scale=None, out=None, lse=None):
         seqlens = torch.tensor(self.lengths, dtype=torch.int32, device=q.device)
+        if self.gs_cache is not None:
+            return wall_attn_decode_gated(q, self.p[:, None], self.gs, self.v, self.k_tilde,
+                                          self.r_cache, self.gs_cache, seqlens=seqlens,
+                                          block_table=self.block_table, sink_bias=sink_bias,
+                                          scale=scale, chunk=self.chunk, out=out, lse=lse,
+                                          workspace=self.workspace)
         return wall_attn_decode_paged(q, self.p[:, None], self.v, self.k_tilde, self.r_cache,
                                       seqlens, self.block_table, sink_bias=sink_bias, scale=scale,
                                       chunk=self.chunk, out=out, lse=lse, workspace=self.workspace)

@@ -452,7 +452,9 @@ static wall_status_t decode_entry(const void* q, const float* p_curr, const void
                                   int cap, int HQ, int H, int K, int V, int chunk,
                                   wall_dtype_t dt, float scale, void* o, float* lse,
                                   void* workspace, size_t workspace_bytes, wall_stream_t stream,
-                                  const wall::PageMap* pm = nullptr) {
+                                  const wall::PageMap* pm = nullptr,
+                                  const float* gs_cache = nullptr,
+                                  const float* gs_curr = nullptr) {
   if (B < 0 || T_kv < 1 || cap < T_kv || HQ <= 0 || H <= 0 || HQ % H != 0)
     return WALL_ERR_INVALID_ARG;
   if (dt != WALL_DTYPE_F32 && dt != WALL_DTYPE_BF16) return WALL_ERR_INVALID_ARG;
@@ -481,6 +483,8 @@ static wall_status_t decode_entry(const void* q, const float* p_curr, const void
   a.seqlens = seqlens;
   if (pm != nullptr) a.pm = *pm;
   a.pm.cap = cap;
+  a.gs_cache = gs_cache;
+  a.gs_curr = gs_curr;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   stage_event(0, st);
   const cudaError_t e = wall::launch_decode(a, dt == WALL_DTYPE_BF16, st);
@@ -525,6 +529,105 @@ wall_status_t wall_attn_decode_paged(const void* q, const float* p_curr, const v
   return decode_entry(q, p_curr, v_pool, k_tilde_pool, r_pool, sink_bias, seqlens_kv, B, rows,
                       rows, HQ, H, K, V, chunk, dt, scale, o, lse, workspace, workspace_bytes,
                       stream, &pm);
+}
+
+// Gate cache entries: dense when block_table is NULL (gs_cache [B, cap, HQ]),
+// paged otherwise (gs_cache [num_blocks, block_size, HQ]).
+static wall_status_t gate_map(const int32_t* block_table, int max_blocks, int num_blocks,
+                              int block_size, int B, int cap, wall::PageMap* pm) {
+  if (block_table == nullptr) {
+    if (cap < 1) return WALL_ERR_INVALID_ARG;
+    pm->cap = cap;
+    return WALL_OK;
+  }
+  // any block size works for the gate cache (one value per row and head)
+  if (max_blocks < 1 || num_blocks < 1 || block_size < 1) return WALL_ERR_INVALID_ARG;
+  if (static_cast<long long>(max_blocks) * block_size > 0x7fffffffLL ||
+      static_cast<long long>(num_blocks) * block_size > 0x7fffffffLL)
+    return WALL_ERR_UNSUPPORTED;
+  if (!aligned(block_table, 4)) return WALL_ERR_INVALID_ARG;
+  pm->bt = block_table;
+  pm->maxblk = max_blocks;
+  pm->bs = block_size;
+  pm->nblk = num_blocks;
+  pm->cap = max_blocks * block_size;
+  (void)B;
+  return WALL_OK;
+}
+
+wall_status_t wall_build_gate_cache(const void* gs_new, const float* gs_prev,
+                                    const int32_t* block_table, int max_blocks, int num_blocks,
+                                    int block_size, int B, int t_start, int T_new, int cap, int HQ,
+                                    wall_dtype_t dt, float* gs_cache, float* gs_last,
+                                    wall_stream_t stream) {
+  if (B < 0 || t_start < 0 || T_new < 0 || HQ <= 0) return WALL_ERR_INVALID_ARG;
+  if (dt != WALL_DTYPE_F32 && dt != WALL_DTYPE_BF16) return WALL_ERR_INVALID_ARG;
+  wall::PageMap pm;
+  const wall_status_t ps = gate_map(block_table, max_blocks, num_blocks, block_size, B, cap, &pm);
+  if (ps != WALL_OK) return ps;
+  if (static_cast<long long>(t_start) + T_new > pm.rows()) return WALL_ERR_INVALID_ARG;
+  if (B == 0 || T_new == 0) return WALL_OK;
+  if ((t_start > 0) != (gs_prev != nullptr)) return WALL_ERR_INVALID_ARG;
+  if (!gs_new || !gs_cache || !gs_last) return WALL_ERR_INVALID_ARG;
+  if (!aligned(gs_cache, 4) || !aligned(gs_last, 4) || (gs_prev && !aligned(gs_prev, 4)) ||
+      !aligned(gs_new, dt == WALL_DTYPE_BF16 ? 2 : 4))
+    return WALL_ERR_INVALID_ARG;
+  if (B > 65535) return WALL_ERR_UNSUPPORTED;
+  wall::GateArgs a;
+  a.gs_new = gs_new; a.gs_prev = gs_prev; a.t_pos = nullptr;
+  a.B = B; a.t_start = t_start; a.T_new = T_new; a.HQ = HQ;
+  a.gcache = gs_cache; a.gs_last = gs_last; a.pm = pm;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(wall::launch_gate_cache(a, dt == WALL_DTYPE_BF16, st), st);
+}
+
+wall_status_t wall_append_gate_cache(const void* gs_new, const float* gs_prev,
+                                     const int32_t* t_pos, const int32_t* block_table,
+                                     int max_blocks, int num_blocks, int block_size, int B,
+                                     int cap, int HQ, wall_dtype_t dt, float* gs_cache,
+                                     float* gs_last, wall_stream_t stream) {
+  if (B < 0 || HQ <= 0) return WALL_ERR_INVALID_ARG;
+  if (dt != WALL_DTYPE_F32 && dt != WALL_DTYPE_BF16) return WALL_ERR_INVALID_ARG;
+  wall::PageMap pm;
+  const wall_status_t ps = gate_map(block_table, max_blocks, num_blocks, block_size, B, cap, &pm);
+  if (ps != WALL_OK) return ps;
+  if (B == 0) return WALL_OK;
+  if (!gs_new || !gs_prev || !t_pos || !gs_cache || !gs_last) return WALL_ERR_INVALID_ARG;
+  if (!aligned(gs_cache, 4) || !aligned(gs_last, 4) || !aligned(gs_prev, 4) ||
+      !aligned(t_pos, 4) || !aligned(gs_new, dt == WALL_DTYPE_BF16 ? 2 : 4))
+    return WALL_ERR_INVALID_ARG;
+  wall::GateArgs a;
+  a.gs_new = gs_new; a.gs_prev = gs_prev; a.t_pos = t_pos;
+  a.B = B; a.t_start = 0; a.T_new = 1; a.HQ = HQ;
+  a.gcache = gs_cache; a.gs_last = gs_last; a.pm = pm;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return finish(wall::launch_gate_cache(a, dt == WALL_DTYPE_BF16, st), st);
+}
+
+wall_status_t wall_attn_decode_gated(const void* q, const float* p_curr, const float* gs_curr,
+                                     const void* v, const void* k_tilde, const float* r_cache,
+                                     const float* gs_cache, const float* sink_bias,
+                                     const int32_t* seqlens_kv, const int32_t* block_table,
+                                     int max_blocks, int num_blocks, int block_size, int B,
+                                     int T_kv, int cap, int HQ, int H, int K, int V, int chunk,
+                                     wall_dtype_t dt, float scale, void* o, float* lse,
+                                     void* workspace, size_t workspace_bytes,
+                                     wall_stream_t stream) {
+  if (B > 0 && (gs_curr == nullptr || gs_cache == nullptr)) return WALL_ERR_INVALID_ARG;
+  if (B > 0 && (!aligned(gs_curr, 4) || !aligned(gs_cache, 4))) return WALL_ERR_INVALID_ARG;
+  if (block_table == nullptr) {
+    return decode_entry(q, p_curr, v, k_tilde, r_cache, sink_bias, seqlens_kv, B, T_kv, cap, HQ,
+                        H, K, V, chunk, dt, scale, o, lse, workspace, workspace_bytes, stream,
+                        nullptr, gs_cache, gs_curr);
+  }
+  if (B > 0 && seqlens_kv == nullptr) return WALL_ERR_INVALID_ARG;
+  wall::PageMap pm;
+  const wall_status_t ps = page_map(block_table, max_blocks, num_blocks, block_size, chunk, B, &pm);
+  if (ps != WALL_OK) return ps;
+  const int rows = max_blocks * block_size;
+  return decode_entry(q, p_curr, v, k_tilde, r_cache, sink_bias, seqlens_kv, B, rows, rows, HQ, H,
+                      K, V, chunk, dt, scale, o, lse, workspace, workspace_bytes, stream, &pm,
+                      gs_cache, gs_curr);
 }
 
 wall_status_t wall_device_error(wall_stream_t stream) {

@@ -356,6 +356,107 @@ __global__ void __launch_bounds__(128) cache_append_varlen_kernel(
       make_float4(P[0], P[1], P[2], P[3]);
 }
 
+// ----------------------------------------------------------------- scalar-gate cache
+// PS[t] = (PS before t_start) + sum_{u <= t} g_scalar[u] * log2(e): the scalar
+// gate's prefix in the exp2 units of the decode cache, one fp32 per (row,
+// query head).  Thread (segment of kGateSeg rows, head): head fastest, so a
+// warp reads whole rows.  Three passes: segment sums (kept in the cache row
+// that opens the segment), their prefix per head, then the rows.
+constexpr int kGateSeg = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(256) gate_segsum_kernel(const T* __restrict__ gs_new,
+                                                          int t_start, int T_new, int HQ,
+                                                          PageMap pm, float* __restrict__ gcache) {
+  const int nseg = (T_new + kGateSeg - 1) / kGateSeg;
+  const long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<long>(nseg) * HQ) return;
+  const int hq = static_cast<int>(idx % HQ), seg = static_cast<int>(idx / HQ), b = blockIdx.y;
+  const int r0 = seg * kGateSeg, r1 = min(r0 + kGateSeg, T_new);
+  const T* src = gs_new + (static_cast<size_t>(b) * T_new) * HQ + hq;
+  float acc = 0.f;
+  for (int r = r0; r < r1; ++r) acc = fmaf(load1(src + static_cast<size_t>(r) * HQ), kLog2e, acc);
+  gcache[pm.row(b, t_start + r0) * HQ + hq] = acc;
+}
+
+// One thread per (batch, head): the segment sums become the prefix before each
+// segment, in place; the total goes to gs_last.
+__global__ void __launch_bounds__(128) gate_scan_kernel(const float* __restrict__ gs_prev,
+                                                        int B, int t_start, int T_new, int HQ,
+                                                        PageMap pm, float* __restrict__ gcache,
+                                                        float* __restrict__ gs_last) {
+  const long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<long>(B) * HQ) return;
+  const int b = static_cast<int>(idx / HQ), hq = static_cast<int>(idx % HQ);
+  float carry = (t_start > 0 && gs_prev != nullptr) ? gs_prev[idx] : 0.f;
+  const int nseg = (T_new + kGateSeg - 1) / kGateSeg;
+  for (int sg = 0; sg < nseg; ++sg) {
+    float* slot = gcache + pm.row(b, t_start + sg * kGateSeg) * HQ + hq;
+    const float tot = *slot;
+    *slot = carry;
+    carry += tot;
+  }
+  gs_last[idx] = carry;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) gate_write_kernel(const T* __restrict__ gs_new, int t_start,
+                                                         int T_new, int HQ, PageMap pm,
+                                                         float* __restrict__ gcache) {
+  const int nseg = (T_new + kGateSeg - 1) / kGateSeg;
+  const long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<long>(nseg) * HQ) return;
+  const int hq = static_cast<int>(idx % HQ), seg = static_cast<int>(idx / HQ), b = blockIdx.y;
+  const int r0 = seg * kGateSeg, r1 = min(r0 + kGateSeg, T_new);
+  const T* src = gs_new + (static_cast<size_t>(b) * T_new) * HQ + hq;
+  float acc = gcache[pm.row(b, t_start + r0) * HQ + hq];  // prefix before the segment
+  for (int r = r0; r < r1; ++r) {
+    acc = fmaf(load1(src + static_cast<size_t>(r) * HQ), kLog2e, acc);
+    gcache[pm.row(b, t_start + r) * HQ + hq] = acc;
+  }
+}
+
+// One token per batch row at its own position t_pos[b]: thread per (batch, head).
+template <typename T>
+__global__ void __launch_bounds__(128) gate_append_kernel(const T* __restrict__ gs_new,
+                                                          const float* __restrict__ gs_prev,
+                                                          const int* __restrict__ t_pos, int B,
+                                                          int HQ, PageMap pm,
+                                                          float* __restrict__ gcache,
+                                                          float* __restrict__ gs_last) {
+  const long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<long>(B) * HQ) return;
+  const int b = static_cast<int>(idx / HQ), hq = static_cast<int>(idx % HQ);
+  const int t = min(max(t_pos[b], 0), pm.rows() - 1);
+  const float prev = t > 0 ? gs_prev[idx] : 0.f;
+  const float ps = fmaf(load1(gs_new + idx), kLog2e, prev);
+  gcache[pm.row(b, t) * HQ + hq] = ps;
+  gs_last[idx] = ps;
+}
+
+template <typename T>
+cudaError_t gate_impl(const GateArgs& a, cudaStream_t st) {
+  const T* gs = static_cast<const T*>(a.gs_new);
+  if (a.t_pos != nullptr) {
+    const long n = static_cast<long>(a.B) * a.HQ;
+    gate_append_kernel<T><<<static_cast<unsigned>((n + 127) / 128), 128, 0, st>>>(
+        gs, a.gs_prev, a.t_pos, a.B, a.HQ, a.pm, a.gcache, a.gs_last);
+    return cudaGetLastError();
+  }
+  const int nseg = (a.T_new + kGateSeg - 1) / kGateSeg;
+  const long nthr = static_cast<long>(nseg) * a.HQ;
+  const dim3 grid(static_cast<unsigned>((nthr + 255) / 256), a.B);
+  gate_segsum_kernel<T><<<grid, 256, 0, st>>>(gs, a.t_start, a.T_new, a.HQ, a.pm, a.gcache);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long nbh = static_cast<long>(a.B) * a.HQ;
+  gate_scan_kernel<<<static_cast<unsigned>((nbh + 127) / 128), 128, 0, st>>>(
+      a.gs_prev, a.B, a.t_start, a.T_new, a.HQ, a.pm, a.gcache, a.gs_last);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  gate_write_kernel<T><<<grid, 256, 0, st>>>(gs, a.t_start, a.T_new, a.HQ, a.pm, a.gcache);
+  return cudaGetLastError();
+}
+
 template <typename T, int KD>
 cudaError_t append_varlen_impl(const CacheArgs& a, const int* t_pos, cudaStream_t st) {
   const long n = static_cast<long>(a.B) * a.HQ * (KD / 4);
@@ -456,6 +557,10 @@ cudaError_t launch_append_varlen(const CacheArgs& a, const int* t_pos, bool bf16
   }
   return a.K == 64 ? append_varlen_impl<float, 64>(a, t_pos, st)
                    : append_varlen_impl<float, 128>(a, t_pos, st);
+}
+
+cudaError_t launch_gate_cache(const GateArgs& a, bool bf16, cudaStream_t st) {
+  return bf16 ? gate_impl<__nv_bfloat16>(a, st) : gate_impl<float>(a, st);
 }
 
 cudaError_t launch_cache_build(const CacheArgs& a, bool bf16, cudaStream_t st) {

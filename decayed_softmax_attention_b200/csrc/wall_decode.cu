@@ -1,6 +1,7 @@
 // Wall attention single-step decode (Wall Attention README, "Decode") over the
 // pre-rescaled cache that wall_cache.cu builds:
 //   x_j = scale * sum_n q[n] k_tilde[j,n] exp2(p_curr[n] - R_{j/C}[n])
+// (+ (PS_t - PS_j) ln 2 with the scalar gate's cache, the forward's Gs_t - Gs_j)
 //
 // The decode is a GEMV-like pass that streams k_tilde and v from HBM once.
 // Grid = (split, KV head, batch); one CTA serves the HQ/H query heads that
@@ -86,12 +87,13 @@ struct DecCfg {
   static_assert(SR % NW == 0, "rows per stage must split over the consumer warps");
 };
 
-template <typename T, int KD, int VD, int G, bool PAGED>
+template <typename T, int KD, int VD, int G, bool PAGED, bool GATE>
 __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_split_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
     const T* __restrict__ q, const float* __restrict__ p_curr, const float* __restrict__ r_cache,
     int T_kv, int HQ, int C, int cps, int nsplit, float sc, float* __restrict__ part,
-    int* err, uint64_t wait_ns, int fault, const int* __restrict__ seqlens, PageMap pm) {
+    int* err, uint64_t wait_ns, int fault, const int* __restrict__ seqlens, PageMap pm,
+    const float* __restrict__ gs_cache, const float* __restrict__ gs_curr) {
   using D = DecCfg<T, KD, VD, G>;
   constexpr int LPH = 32 / G;    // lanes per query head
   constexpr int CPL = KD / LPH;  // k_tilde channels per lane
@@ -166,6 +168,8 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
     load_n<float, CPL>(p_curr + (static_cast<size_t>(b) * HQ + hq) * KD + cofs, pc);
 #pragma unroll
     for (int e = 0; e < CPL; ++e) qv[e] *= sc;
+    // scalar gate: the logit gains PS(current row) - PS(row j), exp2 units
+    const float gcur = GATE ? gs_curr[static_cast<size_t>(b) * HQ + hq] : 0.f;
     float m = -INFINITY, l = 0.f;
     float o[G][VPL];
 #pragma unroll
@@ -188,7 +192,14 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
         for (int e = 0; e < CPL; ++e) qt[e] = qv[e] * exp2f(pc[e] - R[e]);
       }
       const int r0 = warp * D::RPW;
-      float sres[D::RPW], vv[D::RPW][VPL];
+      float sres[D::RPW], vv[D::RPW][VPL], gsv[D::RPW];
+      if (GATE) {
+        // the stage lies in one block of a paged cache (see the producer)
+        const size_t prow0 = PAGED ? pm.row(b, row0) : static_cast<size_t>(b) * pm.cap + row0;
+#pragma unroll
+        for (int rr = 0; rr < D::RPW; ++rr)
+          gsv[rr] = row0 + r0 + rr < row_end ? gs_cache[(prow0 + r0 + rr) * HQ + hq] : 0.f;
+      }
 #pragma unroll
       for (int rr = 0; rr < D::RPW; ++rr) {
         float kf[CPL];
@@ -212,6 +223,7 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
 #pragma unroll
         for (int off = LPH / 2; off > 0; off >>= 1)
           sres[rr] += __shfl_xor_sync(0xffffffffu, sres[rr], off);
+        if (GATE) sres[rr] += gcur - gsv[rr];
         if (row0 + r0 + rr >= row_end) sres[rr] = -INFINITY;
       }
       float mloc = sres[0];
@@ -352,7 +364,11 @@ cudaError_t decode_impl(const DecodeArgs& a, cudaStream_t st) {
     if (!encode_tiled(&tmV, tdt, 4, a.v, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   }
-  auto kern = paged ? decode_split_kernel<T, KD, VD, G, true> : decode_split_kernel<T, KD, VD, G, false>;
+  const bool gate = a.gs_cache != nullptr;
+  auto kern = paged ? (gate ? decode_split_kernel<T, KD, VD, G, true, true>
+                            : decode_split_kernel<T, KD, VD, G, true, false>)
+                    : (gate ? decode_split_kernel<T, KD, VD, G, false, true>
+                            : decode_split_kernel<T, KD, VD, G, false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, D::SMEM);
   if (e != cudaSuccess) return e;
   const int nchunks = (a.T_kv + a.chunk - 1) / a.chunk;
@@ -360,7 +376,8 @@ cudaError_t decode_impl(const DecodeArgs& a, cudaStream_t st) {
   dim3 grid(a.nsplit, a.H, a.B);
   kern<<<grid, (D::NW + 1) * 32, D::SMEM, st>>>(
       tmK, tmV, static_cast<const T*>(a.q), a.p_curr, a.r_cache, a.T_kv, a.HQ, a.chunk,
-      cps, a.nsplit, a.scale * kLog2e, a.part, a.err, a.wait_ns, a.fault, a.seqlens, a.pm);
+      cps, a.nsplit, a.scale * kLog2e, a.part, a.err, a.wait_ns, a.fault, a.seqlens, a.pm,
+      a.gs_cache, a.gs_curr);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (a.mid_event != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(a.mid_event), st);

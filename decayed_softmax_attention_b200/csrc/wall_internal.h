@@ -170,6 +170,20 @@ struct CacheArgs {
   PageMap pm;        // paged cache (pm.bt set) or dense (pm.cap = cap)
 };
 cudaError_t launch_cache_build(const CacheArgs& a, bool bf16, cudaStream_t st);
+// Scalar-gate cache: PS = prefix of g_scalar * log2(e) per (row, query head),
+// rows t_start .. t_start + T_new - 1 (t_pos null) or one row per batch row at
+// t_pos[b].  gcache [B, cap, HQ] (dense) or [nblk, bs, HQ] (paged) fp32.
+struct GateArgs {
+  const void* gs_new;     // [B, T_new, HQ] input dtype
+  const float* gs_prev;   // [B, HQ] PS before the first new row (null at row 0)
+  const int* t_pos;       // [B] or null
+  int B, t_start, T_new, HQ;
+  float* gcache;
+  float* gs_last;         // [B, HQ] PS at the last new row
+  PageMap pm;
+};
+cudaError_t launch_gate_cache(const GateArgs& a, bool bf16, cudaStream_t st);
+
 // One token per batch row at row b's own position t_pos[b] (device int32 [B]).
 cudaError_t launch_append_varlen(const CacheArgs& a, const int* t_pos, bool bf16, cudaStream_t st);
 
@@ -192,6 +206,8 @@ struct DecodeArgs {
   int fault;        // testing hook: 2 = producer skips its first stage
   const int* seqlens = nullptr;  // optional device int32 [B]: rows of each batch row's cache
   PageMap pm;                    // paged cache (pm.bt set; seqlens required) or dense
+  const float* gs_cache = nullptr;  // scalar-gate cache (null: no gate) [B, cap, HQ] / pool
+  const float* gs_curr = nullptr;   // [B, HQ] PS of the current row
 };
 int decode_max_splits(int B, int T_kv, int HQ, int H, int chunk);
 int decode_num_splits(int B, int T_kv, int HQ, int H, int chunk);

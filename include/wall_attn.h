@@ -211,8 +211,8 @@ wall_status_t wall_append_kv_cache_varlen(const void* k_new, const void* g_new,
  * split count grows with T_kv, so a workspace sized for T_kv = cap serves
  * every step of a streaming loop.
  * Requires 1 <= T_kv <= cap, chunk in {32, 64, 128}, HQ / H in
- * {1, 2, 4, 8, 16}.  Decode has no g_scalar term (the README's decode call
- * takes none).
+ * {1, 2, 4, 8, 16}.  No g_scalar term here (the README's decode call takes
+ * none); wall_attn_decode_gated adds it.
  */
 size_t wall_attn_decode_workspace_size(int B, int T_kv, int HQ, int H, int V, int chunk);
 
@@ -281,6 +281,45 @@ wall_status_t wall_attn_decode_paged(const void* q, const float* p_curr, const v
                                      const int32_t* block_table, int max_blocks, int B,
                                      int num_blocks, int block_size, int HQ, int H, int K, int V,
                                      int chunk, wall_dtype_t dt, float scale, void* o, float* lse,
+                                     void* workspace, size_t workspace_bytes,
+                                     wall_stream_t stream);
+
+/*
+ * Scalar gate in decode (the forward's g_scalar term Gs[t] - Gs[j] through the
+ * cache; the README's decode call has no gate, so these calls are separate).
+ * The gate cache holds PS[t] = sum_{u <= t} g_scalar[u] * log2(e) per (row,
+ * query head), fp32, in the exp2 units of P:
+ *   dense  gs_cache [B, cap, HQ]                       (block_table NULL)
+ *   paged  gs_cache [num_blocks, block_size, HQ]       (same table as k_tilde)
+ * wall_build_gate_cache writes rows t_start .. t_start + T_new - 1 from
+ * gs_new [B, T_new, HQ] (dtype dt); gs_prev [B, HQ] = PS at row t_start - 1
+ * (NULL iff t_start == 0); gs_last [B, HQ] = PS at the last new row.
+ * wall_append_gate_cache writes one row per batch row at t_pos[b] (device
+ * int32 [B]) from gs_new [B, 1, HQ], with gs_prev = PS at row t_pos[b] - 1.
+ * wall_attn_decode_gated is wall_attn_decode (block_table NULL, seqlens_kv
+ * optional) or wall_attn_decode_paged (block_table set, seqlens_kv required)
+ * plus gs_curr [B, HQ] = PS at the current row and the gate cache; the logit
+ * of row j gains (gs_curr - gs_cache[j]) ln 2.  Workspace as for those calls.
+ */
+wall_status_t wall_build_gate_cache(const void* gs_new, const float* gs_prev,
+                                    const int32_t* block_table, int max_blocks, int num_blocks,
+                                    int block_size, int B, int t_start, int T_new, int cap, int HQ,
+                                    wall_dtype_t dt, float* gs_cache, float* gs_last,
+                                    wall_stream_t stream);
+
+wall_status_t wall_append_gate_cache(const void* gs_new, const float* gs_prev,
+                                     const int32_t* t_pos, const int32_t* block_table,
+                                     int max_blocks, int num_blocks, int block_size, int B,
+                                     int cap, int HQ, wall_dtype_t dt, float* gs_cache,
+                                     float* gs_last, wall_stream_t stream);
+
+wall_status_t wall_attn_decode_gated(const void* q, const float* p_curr, const float* gs_curr,
+                                     const void* v, const void* k_tilde, const float* r_cache,
+                                     const float* gs_cache, const float* sink_bias,
+                                     const int32_t* seqlens_kv, const int32_t* block_table,
+                                     int max_blocks, int num_blocks, int block_size, int B,
+                                     int T_kv, int cap, int HQ, int H, int K, int V, int chunk,
+                                     wall_dtype_t dt, float scale, void* o, float* lse,
                                      void* workspace, size_t workspace_bytes,
                                      wall_stream_t stream);
 

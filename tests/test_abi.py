@@ -320,3 +320,35 @@ def test_paged_host_validation(lib):
     assert build(bt=None) == INVALID
     assert build(bs=48) == UNSUPPORTED
     assert build(Tn=0) == 0
+
+
+def test_gate_host_validation(lib):
+    def build(**kw):
+        a = dict(gs=_fake(), gp=None, bt=None, mb=0, nb=0, bs=0, B=2, t0=0, Tn=10, cap=64, HQ=4,
+                 dt=BF16, gc=_fake(), gl=_fake(), stream=None)
+        a.update(kw)
+        return lib.wall_build_gate_cache(a["gs"], a["gp"], a["bt"], a["mb"], a["nb"], a["bs"], a["B"],
+                                         a["t0"], a["Tn"], a["cap"], a["HQ"], a["dt"], a["gc"],
+                                         a["gl"], a["stream"])
+    assert build(Tn=100) == INVALID          # beyond cap
+    assert build(t0=5) == INVALID            # appending needs gs_prev
+    assert build(gc=None) == INVALID
+    assert build(bt=_fake(0x8000), mb=0, nb=4, bs=16) == INVALID
+    assert build(Tn=0) == 0
+
+    def dec(**kw):
+        a = dict(q=_fake(), p=_fake(), gcur=_fake(), v=_fake(), kt=_fake(), r=_fake(), gc=_fake(),
+                 sink=None, sl=None, bt=None, mb=0, nb=0, bs=0, B=2, T=64, cap=64, HQ=4, H=2,
+                 K=128, V=128, C=64, dt=BF16, scale=0.0, o=_fake(), lse=None, ws=_fake(),
+                 wsb=1 << 30, stream=None)
+        a.update(kw)
+        return lib.wall_attn_decode_gated(a["q"], a["p"], a["gcur"], a["v"], a["kt"], a["r"],
+                                          a["gc"], a["sink"], a["sl"], a["bt"], a["mb"], a["nb"],
+                                          a["bs"], a["B"], a["T"], a["cap"], a["HQ"], a["H"], a["K"],
+                                          a["V"], a["C"], a["dt"], a["scale"], a["o"], a["lse"],
+                                          a["ws"], a["wsb"], a["stream"])
+    assert dec(gcur=None) == INVALID
+    assert dec(gc=None) == INVALID
+    assert dec(bt=_fake(0x8000), mb=2, nb=4, bs=64) == INVALID   # paged needs seqlens
+    assert dec(K=96) == UNSUPPORTED
+    assert dec(B=0) == 0
