@@ -29,7 +29,8 @@ __all__ = [
     "wall_attn_decode_noalloc", "wall_append_kv_cache_varlen", "wall_attn_bwd",
     "wall_attn_bwd_workspace_size", "wall_build_kv_cache_paged", "wall_append_kv_cache_paged",
     "wall_attn_decode_paged", "PagedKVCache", "wall_build_gate_cache", "wall_append_gate_cache",
-    "wall_attn_decode_gated", "wall_device_error", "wall_debug_set_fault", "wall_debug_set_stage_events", "KVCache",
+    "wall_attn_decode_gated", "wall_attn_chunk", "wall_attn_chunk_workspace_size",
+    "wall_device_error", "wall_debug_set_fault", "wall_debug_set_stage_events", "KVCache",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -52,6 +53,7 @@ EXPORTED_SYMBOLS = (
     "wall_append_kv_cache_varlen", "wall_attn_bwd_workspace_size", "wall_attn_bwd",
     "wall_build_kv_cache_paged", "wall_append_kv_cache_paged", "wall_attn_decode_paged",
     "wall_build_gate_cache", "wall_append_gate_cache", "wall_attn_decode_gated",
+    "wall_attn_chunk_workspace_size", "wall_attn_chunk",
 )
 
 
@@ -111,6 +113,11 @@ def load_library():
     lib.wall_attn_decode_gated.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I,
                                            I, I, I, F, P, P, P, S, P]
     lib.wall_attn_decode_gated.restype = I
+    lib.wall_attn_chunk_workspace_size.argtypes = [I, I, I, I]
+    lib.wall_attn_chunk_workspace_size.restype = S
+    lib.wall_attn_chunk.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, F, P, P, P, P,
+                                    P, P, P, S, P]
+    lib.wall_attn_chunk.restype = I
     lib.wall_build_kv_cache.argtypes = [P, P, P, I, I, I, I, I, I, I, I, I, P, P, P, P]
     lib.wall_build_kv_cache.restype = I
     lib.wall_append_kv_cache_varlen.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P, P, P, P]
@@ -521,6 +528,44 @@ def wall_attn_decode_gated(q, p_curr, gs_curr, v, k_tilde, r_cache, gs_cache, T_
         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         _stream(q.device))
     _check(st, "wall_attn_decode_gated")
+    return out
+
+
+# ----------------------------------------------------------------- chunked prefill
+def wall_attn_chunk_workspace_size(B, M, HQ, K) -> int:
+    return int(load_library().wall_attn_chunk_workspace_size(B, M, HQ, K))
+
+
+def wall_attn_chunk(q, k_new, g_new, k_tilde, r_cache, p_last, v_cache, t_start, p_prev=None,
+                    sink_bias=None, window=0, scale=None, chunk=64, out=None, lse=None,
+                    workspace=None):
+    """M new tokens at rows t_start.. of the cache: append their keys, then attend rows
+    0 .. t_start + i.  q [B,M,HQ,K]; v_cache rows of the chunk must already hold its values.
+    Returns o [B,M,HQ,V].  p_prev defaults to p_last (updated in place)."""
+    lib = load_library()
+    B, M, HQ, K = q.shape
+    H = k_new.shape[2]
+    cap, V = v_cache.shape[1], v_cache.shape[3]
+    dt = q.dtype
+    if p_prev is None and t_start > 0:
+        p_prev = p_last
+    if out is None:
+        out = torch.empty((B, M, HQ, V), dtype=dt, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(wall_attn_chunk_workspace_size(B, M, HQ, K), 1),
+                                dtype=torch.uint8, device=q.device)
+    st = lib.wall_attn_chunk(
+        _dev(q, "q", dt), _dev(k_new, "k_new", dt, (B, M, H, K)),
+        _dev(g_new, "g_new", dt, (B, M, HQ, K)), _dev(p_prev, "p_prev", torch.float32, (B, HQ, K)),
+        _dev(sink_bias, "sink_bias", torch.float32, (HQ,)), int(window or 0), B, int(t_start), M,
+        cap, HQ, H, K, V, int(chunk), _dtype_code(q), float(scale) if scale else 0.0,
+        _dev(k_tilde, "k_tilde", dt, (B, cap, HQ, K)),
+        _dev(r_cache, "r_cache", torch.float32, (B, (cap + chunk - 1) // chunk, HQ, K)),
+        _dev(p_last, "p_last", torch.float32, (B, HQ, K)), _dev(v_cache, "v_cache", dt),
+        _dev(out, "out", dt, (B, M, HQ, V)), _dev(lse, "lse", torch.float32, (B, M, HQ)),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(q.device))
+    _check(st, "wall_attn_chunk")
     return out
 
 

@@ -630,6 +630,53 @@ wall_status_t wall_attn_decode_gated(const void* q, const float* p_curr, const f
                       gs_cache, gs_curr);
 }
 
+size_t wall_attn_chunk_workspace_size(int B, int M, int HQ, int K) {
+  if (B <= 0 || M <= 0 || HQ <= 0 || K <= 0) return 0;
+  return wall::chunk_workspace_bytes(B, M, HQ, K);
+}
+
+wall_status_t wall_attn_chunk(const void* q, const void* k_new, const void* g_new,
+                              const float* p_prev, const float* sink_bias, int window, int B,
+                              int t_start, int M, int cap, int HQ, int H, int K, int V, int chunk,
+                              wall_dtype_t dt, float scale, void* k_tilde, float* r_cache,
+                              float* p_last, const void* v_cache, void* o, float* lse,
+                              void* workspace, size_t workspace_bytes, wall_stream_t stream) {
+  if (B < 0 || t_start < 0 || M < 0 || cap < 0 || HQ <= 0 || H <= 0 || HQ % H != 0)
+    return WALL_ERR_INVALID_ARG;
+  if (dt != WALL_DTYPE_F32 && dt != WALL_DTYPE_BF16) return WALL_ERR_INVALID_ARG;
+  if (dt != WALL_DTYPE_BF16) return WALL_ERR_UNSUPPORTED;  // tensor-core path only
+  if (!supported_dim(K) || !supported_dim(V)) return WALL_ERR_UNSUPPORTED;
+  if (chunk != 32 && chunk != 64 && chunk != 128) return WALL_ERR_UNSUPPORTED;
+  if (static_cast<long long>(t_start) + M > cap) return WALL_ERR_INVALID_ARG;
+  if (B == 0 || M == 0) return WALL_OK;
+  if ((t_start > 0) != (p_prev != nullptr)) return WALL_ERR_INVALID_ARG;
+  const void* a16[] = {q, k_new, g_new, k_tilde, r_cache, p_last, v_cache, o, workspace};
+  for (const void* ptr : a16)
+    if (ptr == nullptr || !aligned(ptr, 16)) return WALL_ERR_INVALID_ARG;
+  if ((p_prev && !aligned(p_prev, 16)) || (sink_bias && !aligned(sink_bias, 4)) ||
+      (lse && !aligned(lse, 4)) || !aligned(workspace, 256))
+    return WALL_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * HQ * ((M + 255) / 256) > 0x7fffffffLL || B > 65535)
+    return WALL_ERR_UNSUPPORTED;
+  if (workspace_bytes < wall::chunk_workspace_bytes(B, M, HQ, K)) return WALL_ERR_WORKSPACE;
+  if (!(scale > 0.f) || !std::isfinite(scale)) scale = 1.f / std::sqrt(static_cast<float>(K));
+  wall::ChunkArgs a;
+  a.q = q; a.k_new = k_new; a.g_new = g_new; a.p_prev = p_prev; a.sink = sink_bias;
+  a.window = window > 0 ? window : 0;
+  a.B = B; a.t0 = t_start; a.M = M; a.cap = cap; a.HQ = HQ; a.H = H; a.K = K; a.V = V;
+  a.chunk = chunk; a.scale = scale; a.k_tilde = k_tilde; a.r_cache = r_cache; a.p_last = p_last;
+  a.v_cache = v_cache; a.o = o; a.lse = lse; a.workspace = workspace;
+  a.err = wall::device_error_word();
+  if (a.err == nullptr) return WALL_ERR_CUDA;
+  a.wait_ns = wall::wait_limit_ns();
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  stage_event(0, st);
+  a.ev_mid = g_stage_ev[1].load();
+  const cudaError_t e = wall::launch_chunk(a, st);
+  stage_event(2, st);
+  return finish(e, st);
+}
+
 wall_status_t wall_device_error(wall_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return WALL_ERR_CUDA;

@@ -187,6 +187,32 @@ cudaError_t launch_gate_cache(const GateArgs& a, bool bf16, cudaStream_t st);
 // One token per batch row at row b's own position t_pos[b] (device int32 [B]).
 cudaError_t launch_append_varlen(const CacheArgs& a, const int* t_pos, bool bf16, cudaStream_t st);
 
+// A chunk of M new tokens at positions t0 .. t0 + M - 1 (chunked prefill,
+// multi-token decode): append its keys to the dense cache, then its queries
+// attend cache rows 0 .. t0 + i.  bf16 only.
+struct ChunkArgs {
+  const void* q;       // [B, M, HQ, K]
+  const void* k_new;   // [B, M, H, K]
+  const void* g_new;   // [B, M, HQ, K]
+  const float* p_prev; // [B, HQ, K] P at row t0 - 1 (null iff t0 == 0)
+  const float* sink;
+  int window;
+  int B, t0, M, cap, HQ, H, K, V, chunk;
+  float scale;
+  void* k_tilde;       // [B, cap, HQ, K]
+  float* r_cache;      // [B, ceil(cap/chunk), HQ, K]
+  float* p_last;       // [B, HQ, K]
+  const void* v_cache; // [B, cap, H, V] (rows t0 .. t0 + M - 1 written by the caller)
+  void* o;             // [B, M, HQ, V]
+  float* lse;          // [B, M, HQ] or null
+  void* workspace;
+  int* err;
+  uint64_t wait_ns;
+  void* ev_mid = nullptr;  // optional event recorded before the attention kernel
+};
+size_t chunk_workspace_bytes(int B, int M, int HQ, int K);
+cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t st);
+
 struct DecodeArgs {
   const void* q;
   const float* p_curr;

@@ -324,6 +324,32 @@ wall_status_t wall_attn_decode_gated(const void* q, const float* p_curr, const f
                                      wall_stream_t stream);
 
 /*
+ * A chunk of new tokens against the cache (chunked prefill; multi-token
+ * decode): M tokens at positions t_start .. t_start + M - 1 of each batch row.
+ * The call first appends their keys to the dense decode cache exactly as
+ * wall_build_kv_cache(k_new, g_new, p_prev, B, t_start, M, cap, ...) does
+ * (k_tilde rows, chunk anchors, p_last), then every new query i attends cache
+ * rows 0 .. t_start + i (causal; window > 0 keeps t_start + i - j < window;
+ * optional sink), with the cache's per-chunk anchors folded into tile rescales
+ * (Wall Attention README "Decode" cache, the forward's score).  The result
+ * equals rows t_start .. t_start + M - 1 of the prefill of the whole sequence.
+ *   q        [B, M, HQ, K]   k_new [B, M, H, K]   g_new [B, M, HQ, K]   (bf16)
+ *   v_cache  [B, cap, H, V]  rows t_start .. t_start + M - 1 already hold the
+ *            chunk's values (caller-written, as for the decode)
+ *   o        [B, M, HQ, V] bf16;  lse [B, M, HQ] fp32 (nullable)
+ *   workspace >= wall_attn_chunk_workspace_size(B, M, HQ, K) bytes, 256-aligned
+ * bf16 only (fp32: WALL_ERR_UNSUPPORTED); no g_scalar term.
+ */
+size_t wall_attn_chunk_workspace_size(int B, int M, int HQ, int K);
+
+wall_status_t wall_attn_chunk(const void* q, const void* k_new, const void* g_new,
+                              const float* p_prev, const float* sink_bias, int window, int B,
+                              int t_start, int M, int cap, int HQ, int H, int K, int V, int chunk,
+                              wall_dtype_t dt, float scale, void* k_tilde, float* r_cache,
+                              float* p_last, const void* v_cache, void* o, float* lse,
+                              void* workspace, size_t workspace_bytes, wall_stream_t stream);
+
+/*
  * Decode without scratch allocation (no counterpart in the paper: this entry
  * point exists for callers of this library, not for the method).
  *

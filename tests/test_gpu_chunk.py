@@ -1,0 +1,95 @@
+"""Chunked prefill / multi-token decode against the cache (wall_attn_chunk).
+
+A sequence fed in chunks (each chunk's keys appended to the decode cache, its
+queries attending cache rows 0 .. t0 + i) must reproduce the prefill of the
+whole sequence row for row (the oracle's rows), whatever the chunk sizes: a
+single token (multi-token decode with M = 1), sizes that are not multiples
+of the 128-row tiles, and chunks that start inside an anchor chunk.  The cache
+buffers start as NaN, so a read of a row past the rows in use would show.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from tests.gpu_util import ORACLE_THREADS, assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def wall():
+    import decayed_softmax_attention_b200 as w
+    w.load_library()
+    return w
+
+
+CASES = [
+    dict(B=2, sizes=(300, 129, 1, 270), HQ=8, H=2, K=128, V=128, C=64, window=0, sink=True),
+    dict(B=1, sizes=(1, 511, 2, 64), HQ=4, H=1, K=64, V=128, C=32, window=0, sink=False),
+    dict(B=2, sizes=(200, 333, 17), HQ=4, H=2, K=128, V=64, C=128, window=150, sink=True),
+    dict(B=1, sizes=(640,), HQ=16, H=2, K=128, V=128, C=64, window=0, sink=True),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "-".join(map(str, c["sizes"])) + f"C{c['C']}")
+def test_chunks_reproduce_the_prefill(wall, case):
+    B, HQ, H, K, V, C = case["B"], case["HQ"], case["H"], case["K"], case["V"], case["C"]
+    T = sum(case["sizes"])
+    spec = W.PrefillSpec("chunk", B=B, T=T, HQ=HQ, H=H, K=K, V=V, dtype="bf16",
+                         g_kind="negsoftplus", sink=case["sink"], window=case["window"], seed=101)
+    d = W.gen_prefill(spec, device="cuda")
+    cap = T + 37
+    nan = float("nan")
+    kt = torch.full((B, cap, HQ, K), nan, dtype=torch.bfloat16, device="cuda")
+    rc = torch.full((B, (cap + C - 1) // C, HQ, K), nan, dtype=torch.float32, device="cuda")
+    p = torch.full((B, HQ, K), nan, dtype=torch.float32, device="cuda")
+    vc = torch.full((B, cap, H, V), nan, dtype=torch.bfloat16, device="cuda")
+    ro, rl = oracle.wall_fwd(d["q"], d["k"], d["v"], d["g"], sink_bias=d["sink_bias"],
+                             window=d["window"], scale=d["scale"], threads=ORACLE_THREADS)
+    t0 = 0
+    for M in case["sizes"]:
+        sl = slice(t0, t0 + M)
+        vc[:, sl].copy_(d["v"][:, sl])
+        lse = torch.empty((B, M, HQ), dtype=torch.float32, device="cuda")
+        o = wall.wall_attn_chunk(d["q"][:, sl].contiguous(), d["k"][:, sl].contiguous(),
+                                 d["g"][:, sl].contiguous(), kt, rc, p, vc, t0,
+                                 sink_bias=d["sink_bias"], window=d["window"], scale=d["scale"],
+                                 chunk=C, lse=lse)
+        torch.cuda.synchronize()
+        assert wall.wall_device_error() == 0
+        assert_close(o, ro[:, sl], torch.bfloat16, f"chunk at {t0} (M={M})")
+        assert_close(lse, rl[:, sl], torch.bfloat16, f"chunk lse at {t0} (M={M})")
+        t0 += M
+    # the cache the chunks built equals the oracle's
+    ktr, _, P = oracle.kv_cache(d["k"], d["g"], chunk=C, threads=ORACLE_THREADS)
+    assert_close(kt[:, :T], ktr, torch.bfloat16, "cache built by the chunks")
+    np.testing.assert_allclose(p.double().cpu().numpy(), P[:, -1], rtol=1e-4, atol=1e-3)
+
+
+def test_chunk_then_decode(wall):
+    """A chunked prefill followed by single-token decode steps on the same cache."""
+    B, HQ, H, K, V, C = 2, 8, 2, 128, 128, 64
+    T0, S = 450, 6
+    T = T0 + S
+    spec = W.PrefillSpec("chunk_dec", B=B, T=T, HQ=HQ, H=H, K=K, V=V, dtype="bf16",
+                         g_kind="negsoftplus", sink=True, seed=102)
+    d = W.gen_prefill(spec, device="cuda")
+    cache = wall.KVCache(B, T, HQ, H, K, V, dtype=torch.bfloat16, chunk=C)
+    cache.v[:, :T0].copy_(d["v"][:, :T0])
+    wall.wall_attn_chunk(d["q"][:, :T0].contiguous(), d["k"][:, :T0].contiguous(),
+                         d["g"][:, :T0].contiguous(), cache.k_tilde, cache.r_cache, cache.p,
+                         cache.v, 0, sink_bias=d["sink_bias"], scale=d["scale"], chunk=C)
+    cache.length = T0
+    rows = np.array([b * T + t for b in range(B) for t in range(T0, T)], dtype=np.int64)
+    ro, _ = oracle.wall_fwd(d["q"], d["k"], d["v"], d["g"], sink_bias=d["sink_bias"],
+                            scale=d["scale"], rows=rows, threads=ORACLE_THREADS)
+    ro = ro.reshape(B, S, HQ, V)
+    for s_ in range(S):
+        t = T0 + s_
+        cache.append(d["k"][:, t:t + 1].contiguous(), d["g"][:, t:t + 1].contiguous(),
+                     d["v"][:, t:t + 1].contiguous())
+        o = cache.decode(d["q"][:, t:t + 1].contiguous(), sink_bias=d["sink_bias"],
+                         scale=d["scale"])
+        assert_close(o[:, 0], ro[:, s_], torch.bfloat16, f"decode after chunk, step {s_}")
