@@ -515,6 +515,29 @@ def run_ours(args, world, rank, local):
                      "prefill_plain_ms": time_fn(prefill, n_rep),
                      "cache_build_of_prefill_ms": time_fn(build_only, n_rep)})
         del pc
+        # the same prefill fed as 8 chunks of 1024 tokens against the decode cache
+        # (chunked prefill: each chunk's keys appended, its queries over the cache
+        # rows before them); no gate term on this path, so g_scalar is left out
+        nchk = 8
+        Mc = T // nchk
+        cc = wall.KVCache(B, T, HQ, H, K, V, dtype=torch.bfloat16, chunk=64, device=dev)
+        cc.v.copy_(pd["v"])
+        co = torch.empty((B, Mc, HQ, V), dtype=torch.bfloat16, device=dev)
+        cws = torch.empty(wall.wall_attn_chunk_workspace_size(B, Mc, HQ, K), dtype=torch.uint8,
+                          device=dev)
+        chunks = [(pd["q"][:, i * Mc:(i + 1) * Mc].contiguous(),
+                   pd["k"][:, i * Mc:(i + 1) * Mc].contiguous(),
+                   pd["g"][:, i * Mc:(i + 1) * Mc].contiguous()) for i in range(nchk)]
+
+        def chunked():
+            for i, (qc, kc, gc) in enumerate(chunks):
+                wall.wall_attn_chunk(qc, kc, gc, cc.k_tilde, cc.r_cache, cc.p, cc.v, i * Mc,
+                                     scale=pd["scale"], chunk=64, out=co, workspace=cws)
+
+        chk_ms = time_fn(chunked, n_rep)
+        side.update({"chunked_prefill_8x1024_ms": chk_ms,
+                     "chunked_prefill_TFLOPs": flops / (chk_ms * 1e-3) / 1e12})
+        del cc, co, cws, chunks
         # prefill backward on the same workload: gradients of sum(o * dO)
         gdo = torch.Generator(device=dev).manual_seed(pspec.seed + 7)
         dO = torch.randn((B, T, HQ, V), generator=gdo, device=dev).to(torch.bfloat16)
@@ -676,6 +699,38 @@ def run_ours(args, world, rank, local):
                      "decode_gated_GBps": gate_bytes / (gt_ms * 1e-3) / 1e9,
                      "decode_gated_frac_of_hbm": gate_bytes / (gt_ms * 1e-3) / 1e9 / hbm_peak})
         del gs_cache, gs_last, gws, gsd
+        # multi-token decode: 4 new tokens per sequence against the T0-row cache in one
+        # chunk call (append + attend); timing only (the rows after T0 are overwritten)
+        Mt = 4
+        g4 = torch.Generator(device=dev).manual_seed(78)
+        q4 = torch.randn((dspec.B, Mt, dspec.HQ, dspec.K), generator=g4, device=dev).to(torch.bfloat16)
+        k4 = torch.randn((dspec.B, Mt, dspec.H, dspec.K), generator=g4, device=dev).to(torch.bfloat16)
+        gg4 = (-torch.nn.functional.softplus(torch.randn((dspec.B, Mt, dspec.HQ, dspec.K),
+                                                         generator=g4, device=dev) - 4.0)).to(torch.bfloat16)
+        p4 = cache.p.clone()
+        o4 = torch.empty((dspec.B, Mt, dspec.HQ, dspec.V), dtype=torch.bfloat16, device=dev)
+        w4 = torch.empty(wall.wall_attn_chunk_workspace_size(dspec.B, Mt, dspec.HQ, dspec.K),
+                         dtype=torch.uint8, device=dev)
+
+        def dec_multi():
+            wall.wall_attn_chunk(q4, k4, gg4, cache.k_tilde, cache.r_cache, cache.p, cache.v, T0,
+                                 p_prev=p4, scale=dspec.K ** -0.5, chunk=dspec.C, out=o4,
+                                 workspace=w4)
+
+        dec_multi()
+        ma, mz = ev(), ev()
+        torch.cuda.synchronize()
+        ma.record()
+        for _ in range(10):
+            dec_multi()
+        mz.record()
+        torch.cuda.synchronize()
+        mt_ms = ma.elapsed_time(mz) / 10
+        mt_bytes = decode_bytes(dspec, T0 + Mt)
+        side.update({"decode_4tokens_chunk_ms": mt_ms,
+                     "decode_4tokens_chunk_GBps": mt_bytes / (mt_ms * 1e-3) / 1e9,
+                     "decode_4tokens_chunk_frac_of_hbm": mt_bytes / (mt_ms * 1e-3) / 1e9 / hbm_peak})
+        del q4, k4, gg4, p4, o4, w4
         side.update({"cache_build_prefix_ms": build_ms,
                      "cache_build_prefix_GBps": build_gbps,
                      "cache_build_roofline": {

@@ -491,48 +491,104 @@ __global__ void __launch_bounds__(512, 1)
 // The chunk's query side: P_i = P_prev + prefix of g * log2(e) over the chunk;
 // per 256-row query block AQ = P just before the block and
 // qh_i = q_i exp2(P_i - AQ) (a block-local prefix, so the exponent stays
-// bounded).  Thread: (batch * head, four channels), walking the chunk's rows.
+// bounded).  One CTA per (256-row block, batch * head); thread (channel group
+// of 4, row group of RPG rows).  Pass 1 sums g per block; pass 2 adds the
+// earlier blocks' sums to P_prev (AQ), scans the row groups in shared memory
+// and writes qh.
 template <int KD>
-__global__ void __launch_bounds__(128) chunk_prep_kernel(
-    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ g,
-    const float* __restrict__ p_prev, int B, int M, int t0, int HQ, int NQB,
-    __nv_bfloat16* __restrict__ qh, float* __restrict__ AQ) {
-  constexpr int TPS = KD / 4;
-  const long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= static_cast<long>(B) * HQ * TPS) return;
-  const int ch = static_cast<int>(idx % TPS) * 4;
-  const long bh = idx / TPS;
-  const int b = static_cast<int>(bh / HQ), hq = static_cast<int>(bh % HQ);
-  float P[4];
-#pragma unroll
-  for (int c = 0; c < 4; ++c) P[c] = (t0 > 0 && p_prev) ? p_prev[bh * KD + ch + c] : 0.f;
+struct ChunkPrepCfg {
+  static constexpr int CG = KD / 4;        // channel groups of 4
+  static constexpr int RG = 256 / CG;      // row groups
+  static constexpr int RPG = 256 / RG;     // rows per row group
+};
+
+template <int KD>
+__device__ __forceinline__ void chunk_rowgroup_sum(const __nv_bfloat16* gb, size_t rstep, int r0,
+                                                   int r1, float* acc) {
+#pragma unroll 4
+  for (int r = r0; r < r1; ++r) {
+    const uint2 gu = *reinterpret_cast<const uint2*>(gb + r * rstep);
+    acc[0] = fmaf(bf16_lo(gu.x), kLog2e, acc[0]);
+    acc[1] = fmaf(bf16_hi(gu.x), kLog2e, acc[1]);
+    acc[2] = fmaf(bf16_lo(gu.y), kLog2e, acc[2]);
+    acc[3] = fmaf(bf16_hi(gu.y), kLog2e, acc[3]);
+  }
+}
+
+template <int KD>
+__global__ void __launch_bounds__(256) chunk_sum_kernel(const __nv_bfloat16* __restrict__ g,
+                                                        int M, int HQ, int NQB,
+                                                        float* __restrict__ bsum) {
+  using PC = ChunkPrepCfg<KD>;
+  __shared__ float tot[PC::RG][KD];
+  const int blk = blockIdx.x, bh = blockIdx.y, b = bh / HQ, hq = bh % HQ;
+  const int cg = threadIdx.x % PC::CG, rg = threadIdx.x / PC::CG;
+  const int r0 = blk * 256 + rg * PC::RPG, r1 = min(M, r0 + PC::RPG);
   const size_t rstep = static_cast<size_t>(HQ) * KD;
-  const __nv_bfloat16* qb = q + (static_cast<size_t>(b) * M * HQ + hq) * KD + ch;
-  const __nv_bfloat16* gb = g + (static_cast<size_t>(b) * M * HQ + hq) * KD + ch;
-  __nv_bfloat16* ob = qh + static_cast<size_t>(bh) * M * KD + ch;
-  for (int blk = 0; blk < NQB; ++blk) {
-    *reinterpret_cast<float4*>(AQ + (static_cast<size_t>(bh) * NQB + blk) * KD + ch) =
-        make_float4(P[0], P[1], P[2], P[3]);
-    float loc[4] = {0.f, 0.f, 0.f, 0.f};
-    const int r1 = min(M, (blk + 1) * 256);
-    for (int r = blk * 256; r < r1; ++r) {
-      const uint2 gu = *reinterpret_cast<const uint2*>(gb + r * rstep);
-      const uint2 qu = *reinterpret_cast<const uint2*>(qb + r * rstep);
-      const float gv[4] = {bf16_lo(gu.x), bf16_hi(gu.x), bf16_lo(gu.y), bf16_hi(gu.y)};
-      const float qv[4] = {bf16_lo(qu.x), bf16_hi(qu.x), bf16_lo(qu.y), bf16_hi(qu.y)};
-      float o4[4];
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  chunk_rowgroup_sum<KD>(g + (static_cast<size_t>(b) * M * HQ + hq) * KD + cg * 4, rstep, r0, r1,
+                         acc);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        loc[c] = fmaf(gv[c], kLog2e, loc[c]);
-        o4[c] = qv[c] * ex2_approx(loc[c]);
-      }
-      uint2 ou;
-      ou.x = pack_bf16(o4[0], o4[1]);
-      ou.y = pack_bf16(o4[2], o4[3]);
-      *reinterpret_cast<uint2*>(ob + static_cast<size_t>(r) * KD) = ou;
+  for (int c = 0; c < 4; ++c) tot[rg][cg * 4 + c] = acc[c];
+  __syncthreads();
+  if (threadIdx.x < KD) {
+    float sum = 0.f;
+    for (int r = 0; r < PC::RG; ++r) sum += tot[r][threadIdx.x];
+    bsum[(static_cast<size_t>(bh) * NQB + blk) * KD + threadIdx.x] = sum;
+  }
+}
+
+template <int KD>
+__global__ void __launch_bounds__(256) chunk_apply_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ g,
+    const float* __restrict__ p_prev, const float* __restrict__ bsum, int M, int t0, int HQ,
+    int NQB, __nv_bfloat16* __restrict__ qh, float* __restrict__ AQ) {
+  using PC = ChunkPrepCfg<KD>;
+  __shared__ float tot[PC::RG][KD];
+  const int blk = blockIdx.x, bh = blockIdx.y, b = bh / HQ, hq = bh % HQ;
+  const int cg = threadIdx.x % PC::CG, rg = threadIdx.x / PC::CG;
+  const int r0 = blk * 256 + rg * PC::RPG, r1 = min(M, r0 + PC::RPG);
+  const size_t rstep = static_cast<size_t>(HQ) * KD;
+  const __nv_bfloat16* gb = g + (static_cast<size_t>(b) * M * HQ + hq) * KD + cg * 4;
+  const __nv_bfloat16* qb = q + (static_cast<size_t>(b) * M * HQ + hq) * KD + cg * 4;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  chunk_rowgroup_sum<KD>(gb, rstep, r0, r1, acc);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tot[rg][cg * 4 + c] = acc[c];
+  __syncthreads();
+  if (rg == 0) {  // AQ = P_prev + the earlier blocks' sums
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int n = cg * 4 + c;
+      float aq = (t0 > 0 && p_prev) ? p_prev[static_cast<size_t>(bh) * KD + n] : 0.f;
+      for (int k = 0; k < blk; ++k) aq += bsum[(static_cast<size_t>(bh) * NQB + k) * KD + n];
+      AQ[(static_cast<size_t>(bh) * NQB + blk) * KD + n] = aq;
     }
+  }
+  float loc[4];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) P[c] += loc[c];
+  for (int c = 0; c < 4; ++c) {
+    float pre = 0.f;
+    for (int r = 0; r < rg; ++r) pre += tot[r][cg * 4 + c];
+    loc[c] = pre;
+  }
+  __nv_bfloat16* ob = qh + static_cast<size_t>(bh) * M * KD + cg * 4;
+#pragma unroll 4
+  for (int r = r0; r < r1; ++r) {
+    const uint2 gu = *reinterpret_cast<const uint2*>(gb + r * rstep);
+    const uint2 qu = *reinterpret_cast<const uint2*>(qb + r * rstep);
+    const float gv[4] = {bf16_lo(gu.x), bf16_hi(gu.x), bf16_lo(gu.y), bf16_hi(gu.y)};
+    const float qv[4] = {bf16_lo(qu.x), bf16_hi(qu.x), bf16_lo(qu.y), bf16_hi(qu.y)};
+    float o4[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      loc[c] = fmaf(gv[c], kLog2e, loc[c]);
+      o4[c] = qv[c] * ex2_approx(loc[c]);
+    }
+    uint2 ou;
+    ou.x = pack_bf16(o4[0], o4[1]);
+    ou.y = pack_bf16(o4[2], o4[3]);
+    *reinterpret_cast<uint2*>(ob + static_cast<size_t>(r) * KD) = ou;
   }
 }
 
@@ -615,26 +671,36 @@ size_t align256c(size_t x) { return (x + 255) / 256 * 256; }
 size_t chunk_workspace_bytes(int B, int M, int HQ, int K) {
   const size_t BHQ = static_cast<size_t>(B) * HQ;
   const size_t NQB = (static_cast<size_t>(M) + 255) / 256;
-  return align256c(BHQ * M * K * 2) + align256c(BHQ * NQB * K * 4);
+  return align256c(BHQ * M * K * 2) + 2 * align256c(BHQ * NQB * K * 4);
 }
 
 template <int KD>
-cudaError_t chunk_prep(const ChunkArgs& a, void* qh, float* AQ, cudaStream_t st) {
-  const long nthr = static_cast<long>(a.B) * a.HQ * (KD / 4);
-  chunk_prep_kernel<KD><<<static_cast<unsigned>((nthr + 127) / 128), 128, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.g_new),
-      a.p_prev, a.B, a.M, a.t0, a.HQ, (a.M + 255) / 256, static_cast<__nv_bfloat16*>(qh), AQ);
+cudaError_t chunk_prep(const ChunkArgs& a, void* qh, float* AQ, float* bsum, cudaStream_t st) {
+  const int NQB = (a.M + 255) / 256;
+  const dim3 grid(NQB, a.B * a.HQ);
+  const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(a.g_new);
+  if (NQB > 1) {
+    chunk_sum_kernel<KD><<<grid, 256, 0, st>>>(g, a.M, a.HQ, NQB, bsum);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  chunk_apply_kernel<KD><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.q), g,
+                                               a.p_prev, bsum, a.M, a.t0, a.HQ, NQB,
+                                               static_cast<__nv_bfloat16*>(qh), AQ);
   return cudaGetLastError();
 }
 
 cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t st) {
   char* ws = static_cast<char*>(a.workspace);
   const size_t BHQ = static_cast<size_t>(a.B) * a.HQ;
+  const size_t NQB = (static_cast<size_t>(a.M) + 255) / 256;
   void* qh = ws;
   float* AQ = reinterpret_cast<float*>(ws + align256c(BHQ * a.M * a.K * 2));
+  float* bsum = reinterpret_cast<float*>(reinterpret_cast<char*>(AQ) + align256c(BHQ * NQB * a.K * 4));
   // 1. the chunk's queries, anchored (reads p_prev before the append below
   //    overwrites p_last, which may be the same buffer)
-  cudaError_t e = a.K == 64 ? chunk_prep<64>(a, qh, AQ, st) : chunk_prep<128>(a, qh, AQ, st);
+  cudaError_t e = a.K == 64 ? chunk_prep<64>(a, qh, AQ, bsum, st)
+                            : chunk_prep<128>(a, qh, AQ, bsum, st);
   if (e != cudaSuccess) return e;
   // 2. the chunk's keys join the cache (rows t0 .. t0 + M - 1)
   CacheArgs c;

@@ -177,6 +177,16 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
 #pragma unroll
       for (int c = 0; c < VPL; ++c) o[hh][c] = 0.f;
     int cur_chunk = -1;
+    // scalar gate: this lane's head, the warp's rows of a stage, loaded one stage ahead
+    float gnext[D::RPW];
+    auto gate_load = [&](int i, float* dst) {
+      const int rb = row_begin + i * D::SR, r0 = warp * D::RPW;
+      const size_t prow0 = PAGED ? pm.row(b, rb) : static_cast<size_t>(b) * pm.cap + rb;
+#pragma unroll
+      for (int rr = 0; rr < D::RPW; ++rr)
+        dst[rr] = rb + r0 + rr < row_end ? gs_cache[(prow0 + r0 + rr) * HQ + hq] : 0.f;
+    };
+    if (GATE && nst > 0) gate_load(0, gnext);
     for (int i = 0; i < nst; ++i) {
       const int slot = i % D::NS;
       const bool got = mbar_wait(&full[slot], (i / D::NS) & 1, wc);
@@ -194,11 +204,10 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
       const int r0 = warp * D::RPW;
       float sres[D::RPW], vv[D::RPW][VPL], gsv[D::RPW];
       if (GATE) {
-        // the stage lies in one block of a paged cache (see the producer)
-        const size_t prow0 = PAGED ? pm.row(b, row0) : static_cast<size_t>(b) * pm.cap + row0;
+        // (a stage lies in one block of a paged cache, see the producer)
 #pragma unroll
-        for (int rr = 0; rr < D::RPW; ++rr)
-          gsv[rr] = row0 + r0 + rr < row_end ? gs_cache[(prow0 + r0 + rr) * HQ + hq] : 0.f;
+        for (int rr = 0; rr < D::RPW; ++rr) gsv[rr] = gnext[rr];
+        if (i + 1 < nst) gate_load(i + 1, gnext);
       }
 #pragma unroll
       for (int rr = 0; rr < D::RPW; ++rr) {
