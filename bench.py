@@ -55,8 +55,8 @@ TRAFFIC = {
     # proportional to the batch): (1.376487 GB + 5.113088 MB) * 8
     "decode_split": {"bytes": 11052800704, "source_sha": "9d68ac5ccdae419f"},
     # profiles/cache_build_b4_t32k.md, full-size capture (batch 32, 1-pass DRAM metrics):
-    # 10737913088 B read + 8820278528 B written
-    "cache_build": {"bytes": 19558191616, "source_sha": "b5fa331d20089736"},
+    # 10737661184 B read + 8819417344 B written
+    "cache_build": {"bytes": 19557078528, "source_sha": "5ff2742a5cd5b984"},
 }
 KERNEL_SOURCES = {
     "prefill_main": "decayed_softmax_attention_b200/csrc/wall_fwd_tc.cu",
@@ -523,7 +523,7 @@ def run_ours(args, world, rank, local):
         cc = wall.KVCache(B, T, HQ, H, K, V, dtype=torch.bfloat16, chunk=64, device=dev)
         cc.v.copy_(pd["v"])
         co = torch.empty((B, Mc, HQ, V), dtype=torch.bfloat16, device=dev)
-        cws = torch.empty(wall.wall_attn_chunk_workspace_size(B, Mc, HQ, K), dtype=torch.uint8,
+        cws = torch.empty(wall.wall_attn_chunk_workspace_size(B, Mc, T, HQ, H, K, V, 64), dtype=torch.uint8,
                           device=dev)
         chunks = [(pd["q"][:, i * Mc:(i + 1) * Mc].contiguous(),
                    pd["k"][:, i * Mc:(i + 1) * Mc].contiguous(),
@@ -700,37 +700,40 @@ def run_ours(args, world, rank, local):
                      "decode_gated_frac_of_hbm": gate_bytes / (gt_ms * 1e-3) / 1e9 / hbm_peak})
         del gs_cache, gs_last, gws, gsd
         # multi-token decode: 4 new tokens per sequence against the T0-row cache in one
-        # chunk call (append + attend); timing only (the rows after T0 are overwritten)
+        # chunk call (append + attend); timing only (the rows after T0 are overwritten);
+        # needs room for the 4 rows after T0
         Mt = 4
-        g4 = torch.Generator(device=dev).manual_seed(78)
-        q4 = torch.randn((dspec.B, Mt, dspec.HQ, dspec.K), generator=g4, device=dev).to(torch.bfloat16)
-        k4 = torch.randn((dspec.B, Mt, dspec.H, dspec.K), generator=g4, device=dev).to(torch.bfloat16)
-        gg4 = (-torch.nn.functional.softplus(torch.randn((dspec.B, Mt, dspec.HQ, dspec.K),
-                                                         generator=g4, device=dev) - 4.0)).to(torch.bfloat16)
-        p4 = cache.p.clone()
-        o4 = torch.empty((dspec.B, Mt, dspec.HQ, dspec.V), dtype=torch.bfloat16, device=dev)
-        w4 = torch.empty(wall.wall_attn_chunk_workspace_size(dspec.B, Mt, dspec.HQ, dspec.K),
-                         dtype=torch.uint8, device=dev)
+        if dspec.cap >= T0 + Mt:
+            g4 = torch.Generator(device=dev).manual_seed(78)
+            q4 = torch.randn((dspec.B, Mt, dspec.HQ, dspec.K), generator=g4, device=dev).to(torch.bfloat16)
+            k4 = torch.randn((dspec.B, Mt, dspec.H, dspec.K), generator=g4, device=dev).to(torch.bfloat16)
+            gg4 = (-torch.nn.functional.softplus(torch.randn((dspec.B, Mt, dspec.HQ, dspec.K),
+                                                             generator=g4, device=dev) - 4.0)).to(torch.bfloat16)
+            p4 = cache.p.clone()
+            o4 = torch.empty((dspec.B, Mt, dspec.HQ, dspec.V), dtype=torch.bfloat16, device=dev)
+            w4 = torch.empty(wall.wall_attn_chunk_workspace_size(dspec.B, Mt, dspec.cap, dspec.HQ,
+                                                             dspec.H, dspec.K, dspec.V, dspec.C),
+                             dtype=torch.uint8, device=dev)
 
-        def dec_multi():
-            wall.wall_attn_chunk(q4, k4, gg4, cache.k_tilde, cache.r_cache, cache.p, cache.v, T0,
-                                 p_prev=p4, scale=dspec.K ** -0.5, chunk=dspec.C, out=o4,
-                                 workspace=w4)
+            def dec_multi():
+                wall.wall_attn_chunk(q4, k4, gg4, cache.k_tilde, cache.r_cache, cache.p, cache.v, T0,
+                                     p_prev=p4, scale=dspec.K ** -0.5, chunk=dspec.C, out=o4,
+                                     workspace=w4)
 
-        dec_multi()
-        ma, mz = ev(), ev()
-        torch.cuda.synchronize()
-        ma.record()
-        for _ in range(10):
             dec_multi()
-        mz.record()
-        torch.cuda.synchronize()
-        mt_ms = ma.elapsed_time(mz) / 10
-        mt_bytes = decode_bytes(dspec, T0 + Mt)
-        side.update({"decode_4tokens_chunk_ms": mt_ms,
-                     "decode_4tokens_chunk_GBps": mt_bytes / (mt_ms * 1e-3) / 1e9,
-                     "decode_4tokens_chunk_frac_of_hbm": mt_bytes / (mt_ms * 1e-3) / 1e9 / hbm_peak})
-        del q4, k4, gg4, p4, o4, w4
+            ma, mz = ev(), ev()
+            torch.cuda.synchronize()
+            ma.record()
+            for _ in range(10):
+                dec_multi()
+            mz.record()
+            torch.cuda.synchronize()
+            mt_ms = ma.elapsed_time(mz) / 10
+            mt_bytes = decode_bytes(dspec, T0 + Mt)
+            side.update({"decode_4tokens_chunk_ms": mt_ms,
+                         "decode_4tokens_chunk_GBps": mt_bytes / (mt_ms * 1e-3) / 1e9,
+                         "decode_4tokens_chunk_frac_of_hbm": mt_bytes / (mt_ms * 1e-3) / 1e9 / hbm_peak})
+            del q4, k4, gg4, p4, o4, w4
         side.update({"cache_build_prefix_ms": build_ms,
                      "cache_build_prefix_GBps": build_gbps,
                      "cache_build_roofline": {

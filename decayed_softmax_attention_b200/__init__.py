@@ -113,7 +113,7 @@ def load_library():
     lib.wall_attn_decode_gated.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I,
                                            I, I, I, F, P, P, P, S, P]
     lib.wall_attn_decode_gated.restype = I
-    lib.wall_attn_chunk_workspace_size.argtypes = [I, I, I, I]
+    lib.wall_attn_chunk_workspace_size.argtypes = [I, I, I, I, I, I, I, I]
     lib.wall_attn_chunk_workspace_size.restype = S
     lib.wall_attn_chunk.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, F, P, P, P, P,
                                     P, P, P, S, P]
@@ -532,8 +532,8 @@ def wall_attn_decode_gated(q, p_curr, gs_curr, v, k_tilde, r_cache, gs_cache, T_
 
 
 # ----------------------------------------------------------------- chunked prefill
-def wall_attn_chunk_workspace_size(B, M, HQ, K) -> int:
-    return int(load_library().wall_attn_chunk_workspace_size(B, M, HQ, K))
+def wall_attn_chunk_workspace_size(B, M, cap, HQ, H, K, V, chunk=64) -> int:
+    return int(load_library().wall_attn_chunk_workspace_size(B, M, cap, HQ, H, K, V, chunk))
 
 
 def wall_attn_chunk(q, k_new, g_new, k_tilde, r_cache, p_last, v_cache, t_start, p_prev=None,
@@ -552,7 +552,8 @@ def wall_attn_chunk(q, k_new, g_new, k_tilde, r_cache, p_last, v_cache, t_start,
     if out is None:
         out = torch.empty((B, M, HQ, V), dtype=dt, device=q.device)
     if workspace is None:
-        workspace = torch.empty(max(wall_attn_chunk_workspace_size(B, M, HQ, K), 1),
+        workspace = torch.empty(max(wall_attn_chunk_workspace_size(B, M, cap, HQ, H, K, V,
+                                                                   chunk), 1),
                                 dtype=torch.uint8, device=q.device)
     st = lib.wall_attn_chunk(
         _dev(q, "q", dt), _dev(k_new, "k_new", dt, (B, M, H, K)),

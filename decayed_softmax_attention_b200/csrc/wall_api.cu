@@ -630,9 +630,12 @@ wall_status_t wall_attn_decode_gated(const void* q, const float* p_curr, const f
                       gs_cache, gs_curr);
 }
 
-size_t wall_attn_chunk_workspace_size(int B, int M, int HQ, int K) {
-  if (B <= 0 || M <= 0 || HQ <= 0 || K <= 0) return 0;
-  return wall::chunk_workspace_bytes(B, M, HQ, K);
+size_t wall_attn_chunk_workspace_size(int B, int M, int cap, int HQ, int H, int K, int V,
+                                      int chunk) {
+  if (B <= 0 || M <= 0 || cap <= 0 || HQ <= 0 || H <= 0 || HQ % H != 0 || K <= 0 || V <= 0 ||
+      chunk <= 0)
+    return 0;
+  return wall::chunk_workspace_bytes(B, M, cap, HQ, H, K, V, chunk);
 }
 
 wall_status_t wall_attn_chunk(const void* q, const void* k_new, const void* g_new,
@@ -658,7 +661,8 @@ wall_status_t wall_attn_chunk(const void* q, const void* k_new, const void* g_ne
     return WALL_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * HQ * ((M + 255) / 256) > 0x7fffffffLL || B > 65535)
     return WALL_ERR_UNSUPPORTED;
-  if (workspace_bytes < wall::chunk_workspace_bytes(B, M, HQ, K)) return WALL_ERR_WORKSPACE;
+  if (workspace_bytes < wall::chunk_workspace_bytes(B, M, cap, HQ, H, K, V, chunk))
+    return WALL_ERR_WORKSPACE;
   if (!(scale > 0.f) || !std::isfinite(scale)) scale = 1.f / std::sqrt(static_cast<float>(K));
   wall::ChunkArgs a;
   a.q = q; a.k_new = k_new; a.g_new = g_new; a.p_prev = p_prev; a.sink = sink_bias;

@@ -668,10 +668,13 @@ size_t align256c(size_t x) { return (x + 255) / 256 * 256; }
 
 }  // namespace
 
-size_t chunk_workspace_bytes(int B, int M, int HQ, int K) {
+size_t chunk_workspace_bytes(int B, int M, int cap, int HQ, int H, int K, int V, int chunk) {
   const size_t BHQ = static_cast<size_t>(B) * HQ;
   const size_t NQB = (static_cast<size_t>(M) + 255) / 256;
-  return align256c(BHQ * M * K * 2) + 2 * align256c(BHQ * NQB * K * 4);
+  const size_t prep = align256c(BHQ * M * K * 2) + 2 * align256c(BHQ * NQB * K * 4);
+  return prep + (chunk_split_applies(M, HQ, H)
+                     ? align256c(chunk_split_part_bytes(B, M, cap, HQ, H, V, chunk))
+                     : 0);
 }
 
 template <int KD>
@@ -711,7 +714,13 @@ cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t st) {
   c.pm.cap = a.cap;
   e = launch_cache_build(c, true, st);
   if (e != cudaSuccess) return e;
-  // 3. the chunk's queries attend the cache
+  // 3. the chunk's queries attend the cache: a few tokens per sequence the
+  //    decode's way, longer chunks in 128-row tensor-core query tiles
+  if (chunk_split_applies(a.M, a.HQ, a.H)) {
+    float* part = reinterpret_cast<float*>(reinterpret_cast<char*>(bsum) +
+                                           align256c(BHQ * NQB * a.K * 4));
+    return launch_chunk_split(a, qh, AQ, part, st);
+  }
   if (a.K == 64 && a.V == 64) return chunk_by_c<64, 64>(a, qh, AQ, st);
   if (a.K == 64 && a.V == 128) return chunk_by_c<64, 128>(a, qh, AQ, st);
   if (a.K == 128 && a.V == 64) return chunk_by_c<128, 64>(a, qh, AQ, st);

@@ -160,12 +160,21 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
     }
   } else {
     // ------------------------------------------------------------- consumers
+    // A lane's channels of its head come in 16-byte pieces that interleave with
+    // the other lanes of the head: piece j of lane l starts at channel
+    // (l + LPH j) PC, so a quarter-warp's loads cover contiguous bytes.
+    constexpr int PC0 = 16 / static_cast<int>(sizeof(T));
+    constexpr int PC = PC0 < CPL ? PC0 : CPL;
     const int hl = lane / LPH;
     const int hq = h * G + hl;
-    const int cofs = (lane % LPH) * CPL;
+    const int chan0 = hl * KD + (lane % LPH) * PC;  // piece j: chan0 + j * LPH * PC
     float qv[CPL], pc[CPL], qt[CPL];
-    load_n<T, CPL>(q + (static_cast<size_t>(b) * HQ + hq) * KD + cofs, qv);
-    load_n<float, CPL>(p_curr + (static_cast<size_t>(b) * HQ + hq) * KD + cofs, pc);
+#pragma unroll
+    for (int j = 0; j < CPL / PC; ++j) {
+      const size_t off = (static_cast<size_t>(b) * HQ + h * G) * KD + chan0 + j * LPH * PC;
+      load_n<T, PC>(q + off, qv + j * PC);
+      load_n<float, PC>(p_curr + off, pc + j * PC);
+    }
 #pragma unroll
     for (int e = 0; e < CPL; ++e) qv[e] *= sc;
     // scalar gate: the logit gains PS(current row) - PS(row j), exp2 units
@@ -196,8 +205,9 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
       if (row0 / C != cur_chunk) {
         cur_chunk = row0 / C;
         float R[CPL];
-        load_n<float, CPL>(reinterpret_cast<const float*>(st + D::K_BYTES + D::V_BYTES) +
-                               lane * CPL, R);
+        const float* sr = reinterpret_cast<const float*>(st + D::K_BYTES + D::V_BYTES);
+#pragma unroll
+        for (int j = 0; j < CPL / PC; ++j) load_n<float, PC>(sr + chan0 + j * LPH * PC, R + j * PC);
 #pragma unroll
         for (int e = 0; e < CPL; ++e) qt[e] = qv[e] * exp2f(pc[e] - R[e]);
       }
@@ -212,7 +222,10 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
 #pragma unroll
       for (int rr = 0; rr < D::RPW; ++rr) {
         float kf[CPL];
-        load_n<T, CPL>(reinterpret_cast<const T*>(st) + (r0 + rr) * D::GK + lane * CPL, kf);
+#pragma unroll
+        for (int j = 0; j < CPL / PC; ++j)
+          load_n<T, PC>(reinterpret_cast<const T*>(st) + (r0 + rr) * D::GK + chan0 + j * LPH * PC,
+                        kf + j * PC);
         load_n<T, VPL>(reinterpret_cast<const T*>(st + D::K_BYTES) + (r0 + rr) * VD + lane * VPL,
                        vv[rr]);
         if (PAGED && row0 + r0 + rr >= row_end) {
@@ -465,6 +478,20 @@ int decode_num_splits(int B, int T_kv, int HQ, int H, int chunk) {
 
 size_t decode_workspace_bytes(int B, int HQ, int V, int nsplit) {
   return static_cast<size_t>(B) * HQ * nsplit * (V + 2) * sizeof(float);
+}
+
+cudaError_t launch_decode_combine_bf16(const float* part, int nsplit, int nbh, int HQ,
+                                      const float* sink, void* o, float* lse, int V,
+                                      cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>((nbh + 3) / 4);
+  __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(o);
+  if (V == 64)
+    decode_combine_kernel<__nv_bfloat16, 64><<<grid, 128, 0, st>>>(part, nsplit, nbh, HQ, sink, ob, lse);
+  else if (V == 128)
+    decode_combine_kernel<__nv_bfloat16, 128><<<grid, 128, 0, st>>>(part, nsplit, nbh, HQ, sink, ob, lse);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, bool bf16, cudaStream_t st) {

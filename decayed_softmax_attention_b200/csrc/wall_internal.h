@@ -210,8 +210,18 @@ struct ChunkArgs {
   uint64_t wait_ns;
   void* ev_mid = nullptr;  // optional event recorded before the attention kernel
 };
-size_t chunk_workspace_bytes(int B, int M, int HQ, int K);
+size_t chunk_workspace_bytes(int B, int M, int cap, int HQ, int H, int K, int V, int chunk);
 cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t st);
+// Few-token chunks (M <= 2 * 16 / group) attend through a split-KV pass in the
+// decode's style instead of 128-row tensor-core query tiles.
+bool chunk_split_applies(int M, int HQ, int H);
+size_t chunk_split_part_bytes(int B, int M, int cap, int HQ, int H, int V, int chunk);
+cudaError_t launch_chunk_split(const ChunkArgs& a, const void* qh, const float* AQ, float* part,
+                               cudaStream_t st);
+// The decode's split combine (merge per-split partials, add the sink), bf16 output.
+cudaError_t launch_decode_combine_bf16(const float* part, int nsplit, int nbh, int HQ,
+                                      const float* sink, void* o, float* lse, int V,
+                                      cudaStream_t st);
 
 struct DecodeArgs {
   const void* q;

@@ -337,10 +337,16 @@ wall_status_t wall_attn_decode_gated(const void* q, const float* p_curr, const f
  *   v_cache  [B, cap, H, V]  rows t_start .. t_start + M - 1 already hold the
  *            chunk's values (caller-written, as for the decode)
  *   o        [B, M, HQ, V] bf16;  lse [B, M, HQ] fp32 (nullable)
- *   workspace >= wall_attn_chunk_workspace_size(B, M, HQ, K) bytes, 256-aligned
+ *   workspace >= wall_attn_chunk_workspace_size(B, M, cap, HQ, H, K, V, chunk)
+ *            bytes, 256-aligned
  * bf16 only (fp32: WALL_ERR_UNSUPPORTED); no g_scalar term.
+ * A chunk of at most 2 * 16 / (HQ / H) tokens (multi-token decode) attends
+ * through a split-KV pass that streams the cache once per KV head; longer
+ * chunks through 128-row tensor-core query tiles.  Both give the same result
+ * within the usual tolerance.
  */
-size_t wall_attn_chunk_workspace_size(int B, int M, int HQ, int K);
+size_t wall_attn_chunk_workspace_size(int B, int M, int cap, int HQ, int H, int K, int V,
+                                      int chunk);
 
 wall_status_t wall_attn_chunk(const void* q, const void* k_new, const void* g_new,
                               const float* p_prev, const float* sink_bias, int window, int B,

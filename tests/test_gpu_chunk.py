@@ -6,6 +6,12 @@ whole sequence row for row (the oracle's rows), whatever the chunk sizes: a
 single token (multi-token decode with M = 1), sizes that are not multiples
 of the 128-row tiles, and chunks that start inside an anchor chunk.  The cache
 buffers start as NaN, so a read of a row past the rows in use would show.
+
+A few tokens per sequence (at most 2 * 16 / group: multi-token decode, e.g.
+speculative verification) take the split-KV pass instead of the tensor-core
+query tiles; FEW_CASES run every group size on both sides of that bound, with
+one and two token groups per CTA, a partly filled second group, windows that
+skip whole anchor chunks and enough prefix chunks for several splits.
 """
 import numpy as np
 import pytest
@@ -33,7 +39,21 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("case", CASES, ids=lambda c: "-".join(map(str, c["sizes"])) + f"C{c['C']}")
+# (group HQ / H: tokens per split-KV CTA 16 / group; chunks up to twice that take the split pass)
+FEW_CASES = [
+    dict(B=2, sizes=(700, 4, 8, 1, 7, 9, 3), HQ=8, H=2, K=128, V=128, C=64, window=0, sink=True),
+    dict(B=1, sizes=(517, 16, 32, 5, 33), HQ=2, H=2, K=64, V=64, C=32, window=0, sink=False),
+    dict(B=2, sizes=(300, 8, 16, 3), HQ=4, H=2, K=128, V=64, C=128, window=200, sink=True),
+    dict(B=1, sizes=(450, 3, 4, 2, 5), HQ=8, H=1, K=64, V=128, C=64, window=0, sink=True),
+    dict(B=3, sizes=(333, 1, 2, 1, 3), HQ=16, H=1, K=128, V=128, C=64, window=100, sink=False),
+]
+
+
+def _ids(c):
+    return "-".join(map(str, c["sizes"])) + f"C{c['C']}G{c['HQ'] // c['H']}"
+
+
+@pytest.mark.parametrize("case", CASES + FEW_CASES, ids=_ids)
 def test_chunks_reproduce_the_prefill(wall, case):
     B, HQ, H, K, V, C = case["B"], case["HQ"], case["H"], case["K"], case["V"], case["C"]
     T = sum(case["sizes"])
