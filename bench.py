@@ -7,7 +7,8 @@ One step is one pass of the whole hot path over synthetic inputs:
     tcgen05 attention kernel;
   * a 64-token streaming decode on the decode workload (B=32, prefix
     T_kv=32768 built once in set-up, HQ=32, H=8, K=V=128, C=64): per token,
-    append to the pre-rescaled cache, then split-KV decode + combine.
+    one decode step that appends the token to the pre-rescaled cache inside
+    the split-KV decode, then the combine.
 
 Printed (rank 0, one JSON line): prefill TFLOP/s (the headline `value`),
 decode KV GB/s (`decode`), each with its roofline fraction against the
@@ -298,7 +299,7 @@ def config_block(pspec, dspec, n):
     if dspec is not None:
         c["workload"] += (f"; decode: B={dspec.B} T_kv={dspec.T0}->{dspec.cap} HQ={dspec.HQ} "
                           f"H={dspec.H} K={dspec.K} V={dspec.V} C={dspec.C} {dspec.dtype}, "
-                          f"{dspec.steps} streaming steps (append + decode)")
+                          f"{dspec.steps} streaming steps (wall_attn_decode_step: append fused into the decode)")
     return c
 
 
@@ -346,6 +347,7 @@ def run_ours(args, world, rank, local):
         k_steps = [dd["k"][:, T0 + s:T0 + s + 1].contiguous() for s in range(S)]
         g_steps = [dd["g"][:, T0 + s:T0 + s + 1].contiguous() for s in range(S)]
         q_steps = [dd["q"][:, s:s + 1].contiguous() for s in range(S)]
+        v_steps = [dd["v"][:, T0 + s:T0 + s + 1].contiguous() for s in range(S)]
         del dd
         dout = torch.empty((dspec.B, 1, dspec.HQ, dspec.V), dtype=torch.bfloat16, device=dev)
         dlse = torch.empty((dspec.B, 1, dspec.HQ), dtype=torch.float32, device=dev)
@@ -400,11 +402,11 @@ def run_ours(args, world, rank, local):
         if do_decode:
             cache.length = T0
             cache.p.copy_(p_prefix)
-            for s in range(S):
-                cache.append(k_steps[s], g_steps[s])
+            for s in range(S):  # one decode step per token, the append fused in
                 if i is not None:
                     wall.wall_debug_set_stage_events(*dec_ev[i][s])
-                cache.decode(q_steps[s], scale=dspec.K ** -0.5, out=dout, lse=dlse)
+                cache.step(q_steps[s], k_steps[s], g_steps[s], v_steps[s], scale=dspec.K ** -0.5,
+                           out=dout, lse=dlse)
                 if i is not None:
                     wall.wall_debug_set_stage_events()
 
@@ -734,6 +736,26 @@ def run_ours(args, world, rank, local):
                          "decode_4tokens_chunk_GBps": mt_bytes / (mt_ms * 1e-3) / 1e9,
                          "decode_4tokens_chunk_frac_of_hbm": mt_bytes / (mt_ms * 1e-3) / 1e9 / hbm_peak})
             del q4, k4, gg4, p4, o4, w4
+        # the same token as append + decode (two calls), against the main loop's fused step;
+        # timing only (row T0 is rewritten with the same values)
+        if dspec.cap >= T0 + 1:
+            def split_step():
+                cache.length = T0
+                cache.append(k_steps[0], g_steps[0])
+                cache.decode(q_steps[0], scale=dspec.K ** -0.5, out=dout, lse=dlse)
+
+            split_step()
+            fa, fz = ev(), ev()
+            torch.cuda.synchronize()
+            fa.record()
+            for _ in range(10):
+                split_step()
+            fz.record()
+            torch.cuda.synchronize()
+            sp_ms = fa.elapsed_time(fz) / 10
+            side.update({"decode_append_then_decode_ms": sp_ms,
+                         "decode_append_then_decode_frac_of_hbm":
+                             decode_bytes(dspec, T0 + 1) / (sp_ms * 1e-3) / 1e9 / hbm_peak})
         side.update({"cache_build_prefix_ms": build_ms,
                      "cache_build_prefix_GBps": build_gbps,
                      "cache_build_roofline": {

@@ -30,6 +30,7 @@ __all__ = [
     "wall_attn_bwd_workspace_size", "wall_build_kv_cache_paged", "wall_append_kv_cache_paged",
     "wall_attn_decode_paged", "PagedKVCache", "wall_build_gate_cache", "wall_append_gate_cache",
     "wall_attn_decode_gated", "wall_attn_chunk", "wall_attn_chunk_workspace_size",
+    "wall_attn_decode_step",
     "wall_device_error", "wall_debug_set_fault", "wall_debug_set_stage_events", "KVCache",
     "EXPORTED_SYMBOLS",
 ]
@@ -53,7 +54,7 @@ EXPORTED_SYMBOLS = (
     "wall_append_kv_cache_varlen", "wall_attn_bwd_workspace_size", "wall_attn_bwd",
     "wall_build_kv_cache_paged", "wall_append_kv_cache_paged", "wall_attn_decode_paged",
     "wall_build_gate_cache", "wall_append_gate_cache", "wall_attn_decode_gated",
-    "wall_attn_chunk_workspace_size", "wall_attn_chunk",
+    "wall_attn_chunk_workspace_size", "wall_attn_chunk", "wall_attn_decode_step",
 )
 
 
@@ -106,6 +107,9 @@ def load_library():
     lib.wall_attn_decode_paged.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I,
                                            F, P, P, P, S, P]
     lib.wall_attn_decode_paged.restype = I
+    lib.wall_attn_decode_step.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I,
+                                          I, I, F, P, P, P, P, P, P, S, P]
+    lib.wall_attn_decode_step.restype = I
     lib.wall_build_gate_cache.argtypes = [P, P, P, I, I, I, I, I, I, I, I, I, P, P, P]
     lib.wall_build_gate_cache.restype = I
     lib.wall_append_gate_cache.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P, P, P]
@@ -455,6 +459,58 @@ def wall_attn_decode_paged(q, p_curr, v_pool, k_tilde_pool, r_pool, seqlens, blo
     return out
 
 
+def wall_attn_decode_step(q, k_new, g_new, v_new, k_tilde, r_cache, v_cache, p_prev, p_last,
+                          T_kv=None, seqlens=None, block_table=None, sink_bias=None, scale=None,
+                          chunk=64, out=None, lse=None, workspace=None):
+    """One decode step with the append fused in: the new token of batch row b (k_new, g_new,
+    v_new [B,1,...]) joins the cache at row T_b - 1 (T_b = seqlens[b], else T_kv) and its
+    query attends rows 0 .. T_b - 1.  Dense caches [B,cap,...] (block_table None) or pools
+    [num_blocks,block_size,...] with a block table (seqlens required).  p_prev is P at the
+    previous row; P at the new row is written to p_last (a different buffer)."""
+    lib = load_library()
+    B, _, HQ, K = q.shape
+    H, V = k_new.shape[2], v_new.shape[3]
+    dt = k_tilde.dtype
+    if block_table is None:
+        cap = k_tilde.shape[1]
+        maxblk = nblk = bs = 0
+        rows = cap
+        if T_kv is None:
+            raise ValueError("dense caches need T_kv")
+        r_shape = (B, (cap + chunk - 1) // chunk, HQ, K)
+        kv_shape, v_shape = (B, cap, HQ, K), (B, cap, H, V)
+    else:
+        nblk, bs = k_tilde.shape[0], k_tilde.shape[1]
+        maxblk = block_table.shape[1]
+        cap = rows = maxblk * bs
+        if seqlens is None:
+            raise ValueError("paged caches need seqlens")
+        T_kv = rows if T_kv is None else T_kv
+        r_shape = (nblk, bs // chunk, HQ, K)
+        kv_shape, v_shape = (nblk, bs, HQ, K), (nblk, bs, H, V)
+    if out is None:
+        out = torch.empty((B, 1, HQ, V), dtype=dt, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(wall_attn_decode_workspace_size(B, rows if block_table is not None
+                                                                    else T_kv, HQ, H, V, chunk), 1),
+                                dtype=torch.uint8, device=q.device)
+    st = lib.wall_attn_decode_step(
+        _dev(q, "q", dt, (B, 1, HQ, K)), _dev(k_new, "k_new", dt, (B, 1, H, K)),
+        _dev(g_new, "g_new", dt, (B, 1, HQ, K)), _dev(v_new, "v_new", dt, (B, 1, H, V)),
+        _dev(p_prev, "p_prev", torch.float32, (B, HQ, K)),
+        _dev(p_last, "p_last", torch.float32, (B, HQ, K)),
+        _dev(sink_bias, "sink_bias", torch.float32, (HQ,)),
+        _dev(seqlens, "seqlens", torch.int32, (B,)),
+        _dev(block_table, "block_table", torch.int32), maxblk, nblk, bs, B, int(T_kv), cap, HQ, H,
+        K, V, int(chunk), _dtype_code(k_tilde), float(scale) if scale else 0.0,
+        _dev(k_tilde, "k_tilde", dt, kv_shape), _dev(r_cache, "r_cache", torch.float32, r_shape),
+        _dev(v_cache, "v_cache", dt, v_shape), _dev(out, "out", dt, (B, 1, HQ, V)),
+        _dev(lse, "lse", torch.float32), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(q.device))
+    _check(st, "wall_attn_decode_step")
+    return out
+
+
 # ----------------------------------------------------------------- scalar gate in decode
 def _gate_table(gs_cache, block_table):
     """(block_table, max_blocks, num_blocks, block_size, cap) for a dense or paged gate cache."""
@@ -625,6 +681,7 @@ class KVCache:
         self.r_cache = torch.empty((B, nc, HQ, K), dtype=torch.float32, device=device)
         self.v = torch.empty((B, cap, H, V), dtype=dtype, device=device)
         self.p = torch.zeros((B, HQ, K), dtype=torch.float32, device=device)
+        self._p_next = torch.zeros_like(self.p)  # P_last of a fused step (must not be p_prev)
         self.length = 0
         self.workspace = torch.empty(max(wall_attn_decode_workspace_size(B, cap, HQ, H, V, chunk), 1),
                                      dtype=torch.uint8, device=device)
@@ -654,6 +711,18 @@ class KVCache:
                                 sink_bias=sink_bias, scale=scale, chunk=self.chunk, out=out,
                                 lse=lse, workspace=self.workspace)
 
+    def step(self, q, k_new, g_new, v_new, sink_bias=None, scale=None, out=None, lse=None):
+        """append(k_new, g_new, v_new) then decode(q), fused into the decode's launches."""
+        if self.gs_cache is not None:
+            raise ValueError("the fused step carries no scalar gate: use append + decode")
+        o = wall_attn_decode_step(q, k_new, g_new, v_new, self.k_tilde, self.r_cache, self.v,
+                                  self.p, self._p_next, T_kv=self.length + 1, sink_bias=sink_bias,
+                                  scale=scale, chunk=self.chunk, out=out, lse=lse,
+                                  workspace=self.workspace)
+        self.p, self._p_next = self._p_next, self.p
+        self.length += 1
+        return o
+
 
 class PagedKVCache:
     """A paged decode cache: pools of fixed-size blocks plus one block table per sequence.
@@ -675,6 +744,7 @@ class PagedKVCache:
                                    device=device)
         self.v = torch.zeros((num_blocks, block_size, H, V), dtype=dtype, device=device)
         self.p = torch.zeros((B, HQ, K), dtype=torch.float32, device=device)
+        self._p_next = torch.zeros_like(self.p)  # P_last of a fused step (must not be p_prev)
         self.gs_cache = (torch.empty((num_blocks, block_size, HQ), dtype=torch.float32,
                                      device=device) if gate else None)
         self.gs = torch.zeros((B, HQ), dtype=torch.float32, device=device) if gate else None
@@ -764,3 +834,20 @@ class PagedKVCache:
         return wall_attn_decode_paged(q, self.p[:, None], self.v, self.k_tilde, self.r_cache,
                                       seqlens, self.block_table, sink_bias=sink_bias, scale=scale,
                                       chunk=self.chunk, out=out, lse=lse, workspace=self.workspace)
+
+    def step(self, q, k_new, g_new, v_new, t_pos, sink_bias=None, scale=None, out=None, lse=None):
+        """append(k_new, g_new, v_new, t_pos) then decode(q), fused into the decode's launches;
+        t_pos (host list) = each row's current length, where its new token goes."""
+        if self.gs_cache is not None:
+            raise ValueError("the fused step carries no scalar gate: use append + decode")
+        for b, t in enumerate(t_pos):
+            self.reserve(b, t + 1)
+        seqlens = torch.tensor([t + 1 for t in t_pos], dtype=torch.int32, device=q.device)
+        o = wall_attn_decode_step(q, k_new, g_new, v_new, self.k_tilde, self.r_cache, self.v,
+                                  self.p, self._p_next, seqlens=seqlens,
+                                  block_table=self.block_table, sink_bias=sink_bias, scale=scale,
+                                  chunk=self.chunk, out=out, lse=lse, workspace=self.workspace)
+        self.p, self._p_next = self._p_next, self.p
+        for b, t in enumerate(t_pos):
+            self.lengths[b] = t + 1
+        return o

@@ -454,7 +454,8 @@ static wall_status_t decode_entry(const void* q, const float* p_curr, const void
                                   void* workspace, size_t workspace_bytes, wall_stream_t stream,
                                   const wall::PageMap* pm = nullptr,
                                   const float* gs_cache = nullptr,
-                                  const float* gs_curr = nullptr) {
+                                  const float* gs_curr = nullptr,
+                                  const wall::DecodeFuse* fu = nullptr) {
   if (B < 0 || T_kv < 1 || cap < T_kv || HQ <= 0 || H <= 0 || HQ % H != 0)
     return WALL_ERR_INVALID_ARG;
   if (dt != WALL_DTYPE_F32 && dt != WALL_DTYPE_BF16) return WALL_ERR_INVALID_ARG;
@@ -467,6 +468,17 @@ static wall_status_t decode_entry(const void* q, const float* p_curr, const void
       !aligned(r_cache, 16) || !aligned(o, 16) || !aligned(workspace, 16) ||
       (sink_bias && !aligned(sink_bias, 4)) || (lse && !aligned(lse, 4)))
     return WALL_ERR_INVALID_ARG;
+  if (fu != nullptr) {
+    if (!fu->k_new || !fu->g_new || !fu->v_new || !fu->p_last || !aligned(fu->k_new, 16) ||
+        !aligned(fu->g_new, 16) || !aligned(fu->v_new, 16) || !aligned(fu->p_last, 16))
+      return WALL_ERR_INVALID_ARG;
+    // other CTAs read p_prev while the one holding a row's new token writes P_last
+    const size_t pb = static_cast<size_t>(B) * HQ * K * sizeof(float);
+    const char* a0 = reinterpret_cast<const char*>(p_curr);
+    const char* a1 = reinterpret_cast<const char*>(fu->p_last);
+    if (a0 < a1 + pb && a1 < a0 + pb) return WALL_ERR_INVALID_ARG;
+    if (gs_cache != nullptr) return WALL_ERR_UNSUPPORTED;
+  }
   const int ns = wall::decode_num_splits(B, T_kv, HQ, H, chunk);
   if (workspace_bytes < wall::decode_workspace_bytes(B, HQ, V, ns)) return WALL_ERR_WORKSPACE;
   if (!(scale > 0.f) || !std::isfinite(scale)) scale = 1.f / std::sqrt(static_cast<float>(K));
@@ -485,6 +497,7 @@ static wall_status_t decode_entry(const void* q, const float* p_curr, const void
   a.pm.cap = cap;
   a.gs_cache = gs_cache;
   a.gs_curr = gs_curr;
+  if (fu != nullptr) a.fuse = *fu;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   stage_event(0, st);
   const cudaError_t e = wall::launch_decode(a, dt == WALL_DTYPE_BF16, st);
@@ -529,6 +542,33 @@ wall_status_t wall_attn_decode_paged(const void* q, const float* p_curr, const v
   return decode_entry(q, p_curr, v_pool, k_tilde_pool, r_pool, sink_bias, seqlens_kv, B, rows,
                       rows, HQ, H, K, V, chunk, dt, scale, o, lse, workspace, workspace_bytes,
                       stream, &pm);
+}
+
+wall_status_t wall_attn_decode_step(const void* q, const void* k_new, const void* g_new,
+                                    const void* v_new, const float* p_prev, float* p_last,
+                                    const float* sink_bias, const int32_t* seqlens_kv,
+                                    const int32_t* block_table, int max_blocks, int num_blocks,
+                                    int block_size, int B, int T_kv, int cap, int HQ, int H,
+                                    int K, int V, int chunk, wall_dtype_t dt, float scale,
+                                    void* k_tilde, float* r_cache, void* v_cache, void* o,
+                                    float* lse, void* workspace, size_t workspace_bytes,
+                                    wall_stream_t stream) {
+  wall::DecodeFuse fu;
+  fu.k_new = k_new; fu.g_new = g_new; fu.v_new = v_new; fu.p_last = p_last;
+  fu.k_tilde = k_tilde; fu.r_cache = r_cache; fu.v = v_cache;
+  if (block_table == nullptr)
+    return decode_entry(q, p_prev, v_cache, k_tilde, r_cache, sink_bias, seqlens_kv, B, T_kv, cap,
+                        HQ, H, K, V, chunk, dt, scale, o, lse, workspace, workspace_bytes, stream,
+                        nullptr, nullptr, nullptr, &fu);
+  if (B > 0 && seqlens_kv == nullptr) return WALL_ERR_INVALID_ARG;
+  wall::PageMap pm;
+  const wall_status_t ps = page_map(block_table, max_blocks, num_blocks, block_size, chunk, B, &pm);
+  if (ps != WALL_OK) return ps;
+  const int rows = max_blocks * block_size;
+  (void)cap;
+  return decode_entry(q, p_prev, v_cache, k_tilde, r_cache, sink_bias, seqlens_kv, B,
+                      T_kv < rows ? T_kv : rows, rows, HQ, H, K, V, chunk, dt, scale, o, lse,
+                      workspace, workspace_bytes, stream, &pm, nullptr, nullptr, &fu);
 }
 
 // Gate cache entries: dense when block_table is NULL (gs_cache [B, cap, HQ]),

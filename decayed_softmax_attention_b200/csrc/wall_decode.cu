@@ -56,6 +56,11 @@ __device__ __forceinline__ void load_n(const T* p, float* f) {
 
 __device__ __forceinline__ void store1(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
 __device__ __forceinline__ void store1(float* p, float x) { *p = x; }
+// x rounded as store1 would store it to p's type
+__device__ __forceinline__ float as_stored(const __nv_bfloat16*, float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
+__device__ __forceinline__ float as_stored(const float*, float x) { return x; }
 
 // ----------------------------------------------------------------- split-KV decode
 // Rows of one (batch, KV head) are streamed through a ring of shared-memory
@@ -87,13 +92,21 @@ struct DecCfg {
   static_assert(SR % NW == 0, "rows per stage must split over the consumer warps");
 };
 
-template <typename T, int KD, int VD, int G, bool PAGED, bool GATE>
+// FUSED: the step's new token (row T_b - 1 of each batch row) is not in the
+// cache yet.  The stream stops before it; the CTA whose split holds that row
+// forms it from k_new, g_new and p_prev exactly as the append does (P = p_prev
+// + g log2 e, a new chunk anchor or the stored one, k_tilde rounded to the cache
+// dtype), scores it after its streamed rows, and writes the row, its value, a
+// new anchor and P_last back to the cache.  No other CTA reads that row, that
+// anchor or P_last, so one launch both appends and attends.
+template <typename T, int KD, int VD, int G, bool PAGED, bool GATE, bool FUSED>
 __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_split_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
     const T* __restrict__ q, const float* __restrict__ p_curr, const float* __restrict__ r_cache,
     int T_kv, int HQ, int C, int cps, int nsplit, float sc, float* __restrict__ part,
     int* err, uint64_t wait_ns, int fault, const int* __restrict__ seqlens, PageMap pm,
-    const float* __restrict__ gs_cache, const float* __restrict__ gs_curr) {
+    const float* __restrict__ gs_cache, const float* __restrict__ gs_curr, DecodeFuse fu) {
+  static_assert(!(GATE && FUSED), "the fused append carries no scalar gate");
   using D = DecCfg<T, KD, VD, G>;
   constexpr int LPH = 32 / G;    // lanes per query head
   constexpr int CPL = KD / LPH;  // k_tilde channels per lane
@@ -116,7 +129,9 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
   const int ck1 = min(ck0 + cps, nchunks);
   const int row_begin = ck0 * C;
   const int row_end = min(ck1 * C, T_b);
-  const int nst = row_end > row_begin ? (row_end - row_begin + D::SR - 1) / D::SR : 0;
+  const int t_new = T_b - 1;                                // FUSED: the appended row
+  const int s_end = FUSED ? min(row_end, t_new) : row_end;  // rows streamed from the cache
+  const int nst = s_end > row_begin ? (s_end - row_begin + D::SR - 1) / D::SR : 0;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < D::NS; ++i) {
@@ -173,7 +188,15 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
     for (int j = 0; j < CPL / PC; ++j) {
       const size_t off = (static_cast<size_t>(b) * HQ + h * G) * KD + chan0 + j * LPH * PC;
       load_n<T, PC>(q + off, qv + j * PC);
-      load_n<float, PC>(p_curr + off, pc + j * PC);
+      if (FUSED) {  // P of the new row, as the append forms it
+        float gn[PC], pp[PC];
+        load_n<T, PC>(static_cast<const T*>(fu.g_new) + off, gn);
+        if (t_new > 0) load_n<float, PC>(p_curr + off, pp);
+#pragma unroll
+        for (int e = 0; e < PC; ++e) pc[j * PC + e] = fmaf(gn[e], kLog2e, t_new > 0 ? pp[e] : 0.f);
+      } else {
+        load_n<float, PC>(p_curr + off, pc + j * PC);
+      }
     }
 #pragma unroll
     for (int e = 0; e < CPL; ++e) qv[e] *= sc;
@@ -228,8 +251,11 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
                         kf + j * PC);
         load_n<T, VPL>(reinterpret_cast<const T*>(st + D::K_BYTES) + (r0 + rr) * VD + lane * VPL,
                        vv[rr]);
-        if (PAGED && row0 + r0 + rr >= row_end) {
-          // past this row's length: a paged block may hold anything there
+        if ((PAGED || FUSED || seqlens != nullptr) && row0 + r0 + rr >= s_end) {
+          // past the streamed rows: a row past a shorter batch row's length, a
+          // paged block, or the row the fused append is about to write may hold
+          // anything there (its weight is 0, but 0 x NaN is not); past T_kv of
+          // a dense cache the tensor map already reads zeros
 #pragma unroll
           for (int c = 0; c < VPL; ++c) vv[rr][c] = 0.f;
         }
@@ -246,7 +272,7 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
         for (int off = LPH / 2; off > 0; off >>= 1)
           sres[rr] += __shfl_xor_sync(0xffffffffu, sres[rr], off);
         if (GATE) sres[rr] += gcur - gsv[rr];
-        if (row0 + r0 + rr >= row_end) sres[rr] = -INFINITY;
+        if (row0 + r0 + rr >= s_end) sres[rr] = -INFINITY;
       }
       float mloc = sres[0];
 #pragma unroll
@@ -273,6 +299,61 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
 #pragma unroll
           for (int c = 0; c < VPL; ++c) o[hh][c] = fmaf(ph, vv[rr][c], o[hh][c]);
         }
+      }
+    }
+    if (FUSED && warp == 0 && t_new >= row_begin && t_new < row_end) {
+      // ---- the appended row: formed here, scored last, written to the cache
+      const bool fresh = t_new % C == 0;  // the row opens a chunk: its anchor is its own P
+      const size_t rslot = PAGED ? pm.chunk(b, t_new, C) : static_cast<size_t>(b) * ncap + t_new / C;
+      float* ra = fu.r_cache + (rslot * HQ + h * G) * KD;
+      const size_t prow = PAGED ? pm.row(b, t_new) : static_cast<size_t>(b) * pm.cap + t_new;
+      T* kw = static_cast<T*>(fu.k_tilde) + (prow * HQ + h * G) * KD;
+      const int kofs = chan0 - hl * KD;  // this lane's first channel within its head
+      float d = 0.f;
+#pragma unroll
+      for (int j = 0; j < CPL / PC; ++j) {
+        float R[PC], kn[PC];
+        if (fresh) {
+#pragma unroll
+          for (int e = 0; e < PC; ++e) R[e] = pc[j * PC + e];
+        } else {
+          load_n<float, PC>(ra + chan0 + j * LPH * PC, R);
+        }
+        load_n<T, PC>(static_cast<const T*>(fu.k_new) + (static_cast<size_t>(b) * gridDim.y + h) * KD +
+                          kofs + j * LPH * PC, kn);
+#pragma unroll
+        for (int e = 0; e < PC; ++e) {
+          const int n = j * PC + e;
+          const float kt = fresh ? kn[e] : kn[e] * ex2_approx(R[e] - pc[n]);
+          store1(kw + chan0 + j * LPH * PC + e, kt);
+          const float ktr = as_stored(kw, kt);  // as the cache holds it
+          d = fmaf(qv[n] * exp2f(pc[n] - R[e]), ktr, d);
+          if (fresh) ra[chan0 + j * LPH * PC + e] = pc[n];
+          fu.p_last[(static_cast<size_t>(b) * HQ + h * G) * KD + chan0 + j * LPH * PC + e] = pc[n];
+        }
+      }
+#pragma unroll
+      for (int off = LPH / 2; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+      float vn[VPL];
+      T* vw = static_cast<T*>(fu.v) + (prow * gridDim.y + h) * VD + lane * VPL;
+      load_n<T, VPL>(static_cast<const T*>(fu.v_new) + (static_cast<size_t>(b) * gridDim.y + h) * VD +
+                         lane * VPL, vn);
+#pragma unroll
+      for (int c = 0; c < VPL; ++c) {
+        store1(vw + c, vn[c]);
+        vn[c] = as_stored(vw, vn[c]);
+      }
+      const float mn = fmaxf(m, d);
+      const float alpha = exp2f(m - mn);
+      const float pr = exp2f(d - mn);
+      l = l * alpha + pr;
+      m = mn;
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+        const float ah = __shfl_sync(0xffffffffu, alpha, hh * LPH);
+        const float ph = __shfl_sync(0xffffffffu, pr, hh * LPH);
+#pragma unroll
+        for (int c = 0; c < VPL; ++c) o[hh][c] = fmaf(ph, vn[c], o[hh][c] * ah);
       }
     }
     if (lane % LPH == 0) {
@@ -387,10 +468,14 @@ cudaError_t decode_impl(const DecodeArgs& a, cudaStream_t st) {
       return cudaErrorInvalidValue;
   }
   const bool gate = a.gs_cache != nullptr;
-  auto kern = paged ? (gate ? decode_split_kernel<T, KD, VD, G, true, true>
-                            : decode_split_kernel<T, KD, VD, G, true, false>)
-                    : (gate ? decode_split_kernel<T, KD, VD, G, false, true>
-                            : decode_split_kernel<T, KD, VD, G, false, false>);
+  const bool fused = a.fuse.k_new != nullptr;
+  if (gate && fused) return cudaErrorInvalidValue;
+  auto kern = fused ? (paged ? decode_split_kernel<T, KD, VD, G, true, false, true>
+                             : decode_split_kernel<T, KD, VD, G, false, false, true>)
+              : paged ? (gate ? decode_split_kernel<T, KD, VD, G, true, true, false>
+                              : decode_split_kernel<T, KD, VD, G, true, false, false>)
+                      : (gate ? decode_split_kernel<T, KD, VD, G, false, true, false>
+                              : decode_split_kernel<T, KD, VD, G, false, false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, D::SMEM);
   if (e != cudaSuccess) return e;
   const int nchunks = (a.T_kv + a.chunk - 1) / a.chunk;
@@ -399,7 +484,7 @@ cudaError_t decode_impl(const DecodeArgs& a, cudaStream_t st) {
   kern<<<grid, (D::NW + 1) * 32, D::SMEM, st>>>(
       tmK, tmV, static_cast<const T*>(a.q), a.p_curr, a.r_cache, a.T_kv, a.HQ, a.chunk,
       cps, a.nsplit, a.scale * kLog2e, a.part, a.err, a.wait_ns, a.fault, a.seqlens, a.pm,
-      a.gs_cache, a.gs_curr);
+      a.gs_cache, a.gs_curr, a.fuse);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (a.mid_event != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(a.mid_event), st);

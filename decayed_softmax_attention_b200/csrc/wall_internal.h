@@ -223,6 +223,19 @@ cudaError_t launch_decode_combine_bf16(const float* part, int nsplit, int nbh, i
                                       const float* sink, void* o, float* lse, int V,
                                       cudaStream_t st);
 
+// Append fused into the decode step: the new token's k, g, v (one per batch
+// row) join the cache inside the decode kernel.  In this mode DecodeArgs'
+// p_curr holds P of the previous row (p_prev) and the kernel writes P_last.
+struct DecodeFuse {
+  const void* k_new = nullptr;  // [B, H, K]
+  const void* g_new = nullptr;  // [B, HQ, K]
+  const void* v_new = nullptr;  // [B, H, V]
+  float* p_last = nullptr;      // [B, HQ, K], must not overlap p_prev
+  void* k_tilde = nullptr;      // the cache, written at each batch row's new row
+  float* r_cache = nullptr;
+  void* v = nullptr;
+};
+
 struct DecodeArgs {
   const void* q;
   const float* p_curr;
@@ -242,6 +255,7 @@ struct DecodeArgs {
   int fault;        // testing hook: 2 = producer skips its first stage
   const int* seqlens = nullptr;  // optional device int32 [B]: rows of each batch row's cache
   PageMap pm;                    // paged cache (pm.bt set; seqlens required) or dense
+  DecodeFuse fuse;               // fuse.k_new set: append the new row inside the decode
   const float* gs_cache = nullptr;  // scalar-gate cache (null: no gate) [B, cap, HQ] / pool
   const float* gs_curr = nullptr;   // [B, HQ] PS of the current row
 };

@@ -285,6 +285,41 @@ wall_status_t wall_attn_decode_paged(const void* q, const float* p_curr, const v
                                      wall_stream_t stream);
 
 /*
+ * One decode step with the append fused in (Wall Attention README, "Decode":
+ * the streaming loop appends each new token to the cache, then attends it).
+ * One new token per batch row, at row t_b = T_b - 1 where T_b is the row's
+ * length after this step: T_kv (seqlens_kv NULL) or seqlens_kv[b].  The call
+ * writes that row exactly as wall_append_kv_cache_varlen(t_pos = t_b) does
+ * (k_tilde row, the chunk's anchor when t_b % chunk == 0, P_last = p_prev +
+ * g_new * log2(e)), stores v_new in the value cache's row t_b, and returns
+ * o / lse of the token's query over rows 0 .. t_b, all in the decode's kernel
+ * launches (no separate append).
+ *   q      [B, 1, HQ, K]   k_new [B, 1, H, K]   g_new [B, 1, HQ, K]
+ *   v_new  [B, 1, H, V]    (dtype dt)
+ *   p_prev [B, HQ, K] fp32 = P at row t_b - 1 (read only where t_b > 0)
+ *   p_last [B, HQ, K] fp32, written; must not overlap p_prev (several CTAs
+ *          read p_prev while one writes P_last): WALL_ERR_INVALID_ARG
+ *   dense  (block_table NULL): k_tilde [B, cap, HQ, K], r_cache
+ *          [B, ceil(cap / chunk), HQ, K] fp32, v_cache [B, cap, H, V];
+ *          T_kv <= cap; max_blocks, num_blocks, block_size ignored
+ *   paged  (block_table set): the pools of wall_attn_decode_paged;
+ *          seqlens_kv required; cap ignored
+ *   T_kv   the largest T_b (values of seqlens_kv above it are clamped to it)
+ * Workspace: wall_attn_decode_workspace_size(B, T_kv, HQ, H, V, chunk) (paged:
+ * with T_kv = max_blocks * block_size).  No scalar gate (use the separate
+ * gate-cache calls and wall_attn_decode_gated).
+ */
+wall_status_t wall_attn_decode_step(const void* q, const void* k_new, const void* g_new,
+                                    const void* v_new, const float* p_prev, float* p_last,
+                                    const float* sink_bias, const int32_t* seqlens_kv,
+                                    const int32_t* block_table, int max_blocks, int num_blocks,
+                                    int block_size, int B, int T_kv, int cap, int HQ, int H,
+                                    int K, int V, int chunk, wall_dtype_t dt, float scale,
+                                    void* k_tilde, float* r_cache, void* v_cache, void* o,
+                                    float* lse, void* workspace, size_t workspace_bytes,
+                                    wall_stream_t stream);
+
+/*
  * Scalar gate in decode (the forward's g_scalar term Gs[t] - Gs[j] through the
  * cache; the README's decode call has no gate, so these calls are separate).
  * The gate cache holds PS[t] = sum_{u <= t} g_scalar[u] * log2(e) per (row,

@@ -352,3 +352,32 @@ def test_gate_host_validation(lib):
     assert dec(bt=_fake(0x8000), mb=2, nb=4, bs=64) == INVALID   # paged needs seqlens
     assert dec(K=96) == UNSUPPORTED
     assert dec(B=0) == 0
+
+
+def _step(lib, **kw):
+    a = dict(q=_fake(), kn=_fake(0x2000), gn=_fake(0x3000), vn=_fake(0x4000), pp=_fake(0x10000),
+             pl=_fake(0x20000), sink=None, seqlens=None, bt=None, maxblk=0, nblk=0, bs=0, B=2,
+             T=100, cap=128, HQ=8, H=2, K=128, V=128, chunk=64, dt=BF16, scale=0.0,
+             kt=_fake(0x40000), rc=_fake(0x50000), vc=_fake(0x60000), o=_fake(0x70000), lse=None,
+             ws=_fake(0x100000), wsb=1 << 40, stream=None)
+    a.update(kw)
+    return lib.wall_attn_decode_step(
+        a["q"], a["kn"], a["gn"], a["vn"], a["pp"], a["pl"], a["sink"], a["seqlens"], a["bt"],
+        a["maxblk"], a["nblk"], a["bs"], a["B"], a["T"], a["cap"], a["HQ"], a["H"], a["K"], a["V"],
+        a["chunk"], a["dt"], a["scale"], a["kt"], a["rc"], a["vc"], a["o"], a["lse"], a["ws"],
+        a["wsb"], a["stream"])
+
+
+def test_decode_step_host_validation(lib):
+    # P_last must not overlap p_prev (other CTAs read p_prev while one writes P_last)
+    assert _step(lib, pl=_fake(0x10000)) == INVALID
+    assert _step(lib, pl=_fake(0x10000 + 2 * 8 * 128 * 4 - 16)) == INVALID
+    assert _step(lib, kn=None) == INVALID
+    assert _step(lib, vn=_fake(0x4008)) == INVALID           # misaligned
+    assert _step(lib, T=129) == INVALID                      # more rows than the cache holds
+    assert _step(lib, chunk=48) == UNSUPPORTED
+    assert _step(lib, HQ=6, H=2) == UNSUPPORTED              # group of 3
+    assert _step(lib, wsb=16) == WORKSPACE
+    # paged: the per-row lengths are required
+    assert _step(lib, bt=_fake(0x80000), maxblk=4, nblk=16, bs=64) == INVALID
+    assert _step(lib, B=0) == 0
