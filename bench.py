@@ -53,8 +53,8 @@ TRAFFIC = {
     # profiles/wall_fwd_tc_long_prefill.md: 316.535808 MB read + 43.428608 MB written
     "prefill_main": {"bytes": 359964416, "source_sha": "820590f83f572f63"},
     # profiles/decode_split_b4_tkv32k.md, batch 4 scaled by 8 to batch 32 (traffic is
-    # proportional to the batch): (1.376514 GB + 4.980480 MB) * 8
-    "decode_split": {"bytes": 11051955840, "source_sha": "df3156d666239da5"},
+    # proportional to the batch): (1.375950 GB + 5.537536 MB) * 8
+    "decode_split": {"bytes": 11051900288, "source_sha": "453f90616c845a14"},
     # profiles/cache_build_b4_t32k.md, full-size capture (batch 32, 1-pass DRAM metrics):
     # 10737661184 B read + 8819417344 B written
     "cache_build": {"bytes": 19557078528, "source_sha": "5ff2742a5cd5b984"},
