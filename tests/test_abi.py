@@ -381,3 +381,43 @@ def test_decode_step_host_validation(lib):
     # paged: the per-row lengths are required
     assert _step(lib, bt=_fake(0x80000), maxblk=4, nblk=16, bs=64) == INVALID
     assert _step(lib, B=0) == 0
+
+
+def test_chunk_workspace_size(lib):
+    # invalid shapes: 0
+    assert lib.wall_attn_chunk_workspace_size(0, 4, 1024, 32, 8, 128, 128, 64) == 0
+    assert lib.wall_attn_chunk_workspace_size(2, 4, 1024, 6, 4, 128, 128, 64) == 0  # HQ % H
+    # a few tokens per sequence (group 4: up to 8) also hold the split-KV partials, which
+    # grow with the cache capacity; longer chunks need only the anchored queries
+    small = [lib.wall_attn_chunk_workspace_size(32, 4, cap, 32, 8, 128, 128, 64)
+             for cap in (64, 1024, 32832)]
+    assert small[0] <= small[1] <= small[2]
+    prep4 = 32 * 32 * 4 * 128 * 2
+    assert small[2] > prep4 + 32 * 4 * 32 * 130 * 4   # at least one split's partials
+    big = [lib.wall_attn_chunk_workspace_size(1, 1024, cap, 32, 8, 128, 128, 64)
+           for cap in (1024, 32832)]
+    assert big[0] == big[1]
+    # the bound: 2 * 16 / group tokens (group 16: 2 tokens; 3 take the tensor-core tiles)
+    g16 = [lib.wall_attn_chunk_workspace_size(1, m, 32832, 16, 1, 128, 128, 64) for m in (2, 3)]
+    assert g16[0] > g16[1]
+
+
+def test_new_calls_fail_loudly_without_cuda_tensors():
+    import torch
+    bf = torch.bfloat16
+    with pytest.raises((ValueError, ImportError)):
+        wall.wall_attn_chunk(torch.zeros(1, 4, 4, 64, dtype=bf), torch.zeros(1, 4, 2, 64, dtype=bf),
+                             torch.zeros(1, 4, 4, 64, dtype=bf),
+                             torch.zeros(1, 64, 4, 64, dtype=bf),
+                             torch.zeros(1, 1, 4, 64), torch.zeros(1, 4, 64),
+                             torch.zeros(1, 64, 2, 64, dtype=bf), 0, workspace=torch.zeros(1 << 20,
+                                                                                          dtype=torch.uint8))
+    with pytest.raises((ValueError, ImportError)):
+        wall.wall_attn_decode_step(torch.zeros(1, 1, 4, 64, dtype=bf),
+                                   torch.zeros(1, 1, 2, 64, dtype=bf),
+                                   torch.zeros(1, 1, 4, 64, dtype=bf),
+                                   torch.zeros(1, 1, 2, 64, dtype=bf),
+                                   torch.zeros(1, 64, 4, 64, dtype=bf), torch.zeros(1, 1, 4, 64),
+                                   torch.zeros(1, 64, 2, 64, dtype=bf), torch.zeros(1, 4, 64),
+                                   torch.zeros(1, 4, 64), T_kv=1,
+                                   workspace=torch.zeros(1 << 20, dtype=torch.uint8))
