@@ -254,7 +254,8 @@ def run_reference(args, world, rank):
     if rank != 0:
         return 0
     import oracle
-    spec, _ = shard_specs(0)
+    spec, dspec = shard_specs(0)
+    dspec = replace(dspec, steps=args.decode_steps)
     host = host_inputs(W.gen_prefill(spec, device="cpu"))
     threads = oracle.max_threads()
     # size the per-step sample to about 2 s of oracle work
@@ -276,7 +277,7 @@ def run_reference(args, world, rank):
         "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_block(spec, None, args.gpus),
+        "config": config_block(spec, dspec, args.gpus),  # the same config line as our arm
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
