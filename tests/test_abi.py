@@ -421,3 +421,31 @@ def test_new_calls_fail_loudly_without_cuda_tensors():
                                    torch.zeros(1, 64, 2, 64, dtype=bf), torch.zeros(1, 4, 64),
                                    torch.zeros(1, 4, 64), T_kv=1,
                                    workspace=torch.zeros(1 << 20, dtype=torch.uint8))
+
+
+def test_paged_cache_block_allocation_on_the_host():
+    """PagedKVCache's free list and block tables (host logic; no kernel runs)."""
+    import torch
+    c = wall.PagedKVCache(2, num_blocks=5, block_size=64, max_blocks=3, HQ=4, H=2, K=64, V=64,
+                          chunk=32, device="cpu")
+    c.reserve(0, 65)                  # two blocks
+    c.reserve(1, 1)                   # one block
+    assert [len(t) for t in c.host_table] == [2, 1]
+    assert sorted(c.host_table[0] + c.host_table[1] + c.free) == list(range(5))
+    assert c.block_table[0, :2].tolist() == c.host_table[0]
+    # logical row t of a sequence lives in row t % 64 of its (t // 64)-th block
+    rows = c.rows_of(0, 62, 66)
+    b0, b1 = c.host_table[0]
+    assert rows == [b0 * 64 + 62, b0 * 64 + 63, b1 * 64, b1 * 64 + 1]
+    c.reserve(0, 65)                  # already held: nothing changes
+    assert len(c.free) == 2
+    with pytest.raises(ValueError):
+        c.reserve(1, 3 * 64 + 1)      # longer than max_blocks * block_size
+    c.reserve(1, 3 * 64)              # takes the last two free blocks
+    with pytest.raises(MemoryError):
+        c.reserve(0, 3 * 64)          # the pool is exhausted
+    c.release(1)
+    assert len(c.free) == 3 and c.lengths[1] == 0 and c.host_table[1] == []
+    assert c.block_table[1].tolist() == [0, 0, 0]
+    with pytest.raises(ValueError):
+        wall.PagedKVCache(1, 4, 48, 2, 4, 2, 64, 64, chunk=32, device="cpu")  # 48 % 32 != 0
