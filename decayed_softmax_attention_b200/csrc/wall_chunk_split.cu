@@ -68,8 +68,8 @@ struct MultiCfg {
   static constexpr int RING = NS * STAGE;
   static constexpr int MERGE = NW * MQ * G * (VD + 2) * 4;  // overlays the ring after the loop
   static constexpr int BODY = RING > MERGE ? RING : MERGE;
-  static constexpr int OFF_Q = BODY;                       // [MQ][GK] fp32, scaled queries
-  static constexpr int OFF_AQ = OFF_Q + MQ * GK * 4;       // [GK] fp32
+  static constexpr int OFF_Q = BODY;                       // [MQ][CPL][32] fp32, scaled queries
+  static constexpr int OFF_AQ = OFF_Q + MQ * GK * 4;       // [CPL][32] fp32 (GK = 32 CPL)
   static constexpr int OFF_P = OFF_AQ + GK * 4;            // [NW][RB + 1][MQ * G] fp32
   static constexpr int OFF_BAR = OFF_P + NW * (RB + 1) * MQ * G * 4;
   static constexpr int SMEM = OFF_BAR + 2 * NS * 8 + 16 + 128;
@@ -145,14 +145,20 @@ __global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_s
     *abort_flag = 0;
     fence_mbar_init();
   }
-  // the group's queries (scaled, fp32; zero past the chunk's last token) and AQ
-  for (int e = threadIdx.x; e < MQ * D::GK; e += (D::NW + 1) * 32) {
-    const int m = e / D::GK, hl = (e % D::GK) / KD, n = e % KD;
-    const size_t bh = static_cast<size_t>(b) * HQ + h * G + hl;
-    sQ[e] = m0 + m < M ? sc * __bfloat162float(qh[(bh * M + m0 + m) * KD + n]) : 0.f;
+  // the group's queries (scaled, fp32; zero past the chunk's last token) and AQ,
+  // lane-major: element e of lane L's channels at [e][L] (queries [m][e][L]), so the
+  // warp's loads of one element are 32 consecutive words (no bank conflicts)
+  for (int idx = threadIdx.x; idx < MQ * CPL * 32; idx += (D::NW + 1) * 32) {
+    const int L = idx & 31, m = (idx >> 5) / CPL, e = (idx >> 5) % CPL;
+    const int n = (L % LPH) * PC + (e / PC) * LPH * PC + e % PC;  // channel within the head
+    const size_t bh = static_cast<size_t>(b) * HQ + h * G + L / LPH;
+    sQ[idx] = m0 + m < M ? sc * __bfloat162float(qh[(bh * M + m0 + m) * KD + n]) : 0.f;
   }
-  for (int e = threadIdx.x; e < D::GK; e += (D::NW + 1) * 32)
-    sAQ[e] = AQ[(static_cast<size_t>(b) * HQ + h * G) * KD + e];
+  for (int idx = threadIdx.x; idx < CPL * 32; idx += (D::NW + 1) * 32) {
+    const int L = idx & 31, e = idx >> 5;
+    const int n = (L % LPH) * PC + (e / PC) * LPH * PC + e % PC;
+    sAQ[idx] = AQ[(static_cast<size_t>(b) * HQ + h * G + L / LPH) * KD + n];
+  }
   __syncthreads();
   const WaitCtl wc{abort_flag, err, wait_ns};
 
@@ -210,11 +216,12 @@ __global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_s
         for (int e = 0; e < CPL; e += 2) {
           const int n = chan0 + (e / PC) * LPH * PC + e % PC;
           const float2 r2 = *reinterpret_cast<const float2*>(R + n);
-          const float2 a2 = *reinterpret_cast<const float2*>(sAQ + n);
-          const float2 f = make_float2(exp2f(a2.x - r2.x), exp2f(a2.y - r2.y));
+          const float2 f = make_float2(exp2f(sAQ[e * 32 + lane] - r2.x),
+                                       exp2f(sAQ[(e + 1) * 32 + lane] - r2.y));
 #pragma unroll
           for (int m = 0; m < MQ; ++m)
-            qt2[m][e / 2] = __fmul2_rn(*reinterpret_cast<const float2*>(sQ + m * D::GK + n), f);
+            qt2[m][e / 2] = __fmul2_rn(
+                make_float2(sQ[(m * CPL + e) * 32 + lane], sQ[(m * CPL + e + 1) * 32 + lane]), f);
         }
       }
       const __nv_bfloat16* sk = reinterpret_cast<const __nv_bfloat16*>(st);
