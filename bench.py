@@ -801,7 +801,9 @@ def run_ours(args, world, rank, local):
         e2e_ms = reduce_max(a.elapsed_time(b_), world, dev)
         line["e2e"] = {"value": weak_scaling_rate(prefill_flops(pspec), args.steps, world, e2e_ms) / 1e12,
                        "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-    line["gpu_launches"] = args.steps * ((3 if do_prefill else 0) + 3 * S)
+    # per timed step: prefill = prepass (2) + attention (1); each decode token = the fused
+    # decode split (append inside) + the combine (2)
+    line["gpu_launches"] = args.steps * ((3 if do_prefill else 0) + (2 * S if do_decode else 0))
     line["clocks"] = clk
     if rank != 0:
         return 0

@@ -712,7 +712,11 @@ class KVCache:
                                 lse=lse, workspace=self.workspace)
 
     def step(self, q, k_new, g_new, v_new, sink_bias=None, scale=None, out=None, lse=None):
-        """append(k_new, g_new, v_new) then decode(q), fused into the decode's launches."""
+        """append(k_new, g_new, v_new) then decode(q), fused into the decode's launches.
+
+        The kernel reads P from one buffer and writes the new P to another, so after the
+        call ``self.p`` is the other tensor: read ``cache.p`` afresh, do not keep a reference.
+        """
         if self.gs_cache is not None:
             raise ValueError("the fused step carries no scalar gate: use append + decode")
         o = wall_attn_decode_step(q, k_new, g_new, v_new, self.k_tilde, self.r_cache, self.v,
@@ -837,7 +841,8 @@ class PagedKVCache:
 
     def step(self, q, k_new, g_new, v_new, t_pos, sink_bias=None, scale=None, out=None, lse=None):
         """append(k_new, g_new, v_new, t_pos) then decode(q), fused into the decode's launches;
-        t_pos (host list) = each row's current length, where its new token goes."""
+        t_pos (host list) = each row's current length, where its new token goes.  As for
+        KVCache.step, ``self.p`` is a different tensor after the call."""
         if self.gs_cache is not None:
             raise ValueError("the fused step carries no scalar gate: use append + decode")
         for b, t in enumerate(t_pos):
