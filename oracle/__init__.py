@@ -13,6 +13,7 @@ the exact formulas and the readings taken where the page is silent):
   decode_from_cache  -- one decode step over (k_tilde, r_cache), optionally with the gate
   gate_cache         -- the scalar gate's prefix PS in exp2 units (decode with g_scalar)
   wall_bwd           -- gradients of the prefill forward (analytic, by the definition)
+  wall_bwd_rows      -- the same gradients at selected query / key rows (numpy, for long T)
 """
 from __future__ import annotations
 
@@ -257,4 +258,83 @@ def wall_bwd(q, k, v, g, do, g_scalar=None, sink_bias=None, window=0, cu_seqlens
             dv=out["sigma"]["dv"], dg=np.sqrt(s2[8]),
             dg_scalar=np.sqrt(s2[9]) if gs is not None else None,
             dsink=np.sqrt(s2[10].sum(axis=0)) if sink is not None else None)
+    return out
+
+
+def wall_bwd_rows(q, k, v, g, do, o, lse, q_rows=(), k_rows=(), g_scalar=None, window=0,
+                  cu_seqlens=None, scale=None, dlse=None, batch=0):
+    """Selected rows of the prefill backward of one batch row, in double precision, straight
+    from the definition (numpy; for long sequences where the full oracle is too slow).
+
+    The same gradients as ``wall_bwd`` with given o / lse (the sink enters through lse
+    only): dq at query rows ``q_rows`` [n, HQ, K]; dk [n, H, K] and dv [n, H, V] at key rows
+    ``k_rows``, summed over the query heads of each KV group.  With p = exp(x - lse) and
+    dS = p (dO.v - dO.o + dlse):
+        dq_i = scale sum_j dS_ij k_j exp(G_i - G_j)
+        dk_j = scale sum_i dS_ij q_i exp(G_i - G_j),   dv_j = sum_i p_ij dO_i
+    over the admitted pairs (causal, same document, window).  Also returns "sigma" and
+    "sigma_abs" for each, defined as in ``wall_bwd``.
+    """
+    cv = lambda x: None if x is None else _f64(_f32(x))[batch]
+    q, k, v, g, do, o, lse = (cv(x) for x in (q, k, v, g, do, o, lse))
+    gs, dl = cv(g_scalar), cv(dlse)
+    T, HQ, K = q.shape
+    H, V = k.shape[1], v.shape[2]
+    grp = HQ // H
+    if scale is None or scale <= 0:
+        scale = K ** -0.5
+    G = np.cumsum(g, axis=0)                                   # [T, HQ, K], natural log
+    Gs = np.cumsum(gs, axis=0) if gs is not None else np.zeros((T, HQ))
+    doc = np.zeros(T, dtype=np.int64)
+    if cu_seqlens is not None:
+        cu = np.asarray(cu_seqlens.detach().cpu().numpy() if hasattr(cu_seqlens, "detach")
+                        else cu_seqlens, dtype=np.int64)
+        for d_ in range(len(cu) - 1):
+            doc[cu[d_]:cu[d_ + 1]] = d_
+    delta = np.einsum("thv,thv->th", do, o) - (dl if dl is not None else 0.0)
+    pos = np.arange(T)
+
+    def pairs(i, j):  # admitted (query i, key j) for arrays i, j of equal shape
+        ok = (j <= i) & (doc[i] == doc[j])
+        if window and window > 0:
+            ok &= (i - j) < window
+        return ok
+
+    q_rows, k_rows = list(q_rows), list(k_rows)
+    out = {n: np.zeros(s) for n, s in (("dq", (len(q_rows), HQ, K)), ("dk", (len(k_rows), H, K)),
+                                         ("dv", (len(k_rows), H, V)))}
+    s2 = {n: np.zeros_like(a) for n, a in out.items()}
+    sa = {n: np.zeros_like(a) for n, a in out.items()}
+    for r, i in enumerate(q_rows):
+        js = pos[pairs(np.full(T, i), pos)]
+        for hq in range(HQ):
+            kv = hq // grp
+            dec = np.exp(G[i, hq][None, :] - G[js, hq])               # [nj, K]
+            x = scale * (q[i, hq][None, :] * k[js, kv] * dec).sum(axis=1) + Gs[i, hq] - Gs[js, hq]
+            p = np.exp(x - lse[i, hq])
+            dP = v[js, kv] @ do[i, hq]
+            t = scale * (p * (dP - delta[i, hq]))[:, None] * k[js, kv] * dec
+            ta = scale * (p * (np.abs(dP) + np.abs(delta[i, hq])))[:, None] * k[js, kv] * dec
+            out["dq"][r, hq] = t.sum(axis=0)
+            s2["dq"][r, hq] = (t * t).sum(axis=0)
+            sa["dq"][r, hq] = (ta * ta).sum(axis=0)
+    for r, j in enumerate(k_rows):
+        is_ = pos[pairs(pos, np.full(T, j))]
+        for hq in range(HQ):
+            kv = hq // grp
+            dec = np.exp(G[is_, hq] - G[j, hq][None, :])              # [ni, K]
+            x = scale * (q[is_, hq] * k[j, kv][None, :] * dec).sum(axis=1) + Gs[is_, hq] - Gs[j, hq]
+            p = np.exp(x - lse[is_, hq])
+            dP = do[is_, hq] @ v[j, kv]
+            t = scale * (p * (dP - delta[is_, hq]))[:, None] * q[is_, hq] * dec
+            ta = scale * (p * (np.abs(dP) + np.abs(delta[is_, hq])))[:, None] * q[is_, hq] * dec
+            tv = p[:, None] * do[is_, hq]
+            out["dk"][r, kv] += t.sum(axis=0)
+            s2["dk"][r, kv] += (t * t).sum(axis=0)
+            sa["dk"][r, kv] += (ta * ta).sum(axis=0)
+            out["dv"][r, kv] += tv.sum(axis=0)
+            s2["dv"][r, kv] += (tv * tv).sum(axis=0)
+            sa["dv"][r, kv] += (tv * tv).sum(axis=0)
+    out["sigma"] = {n: np.sqrt(a) for n, a in s2.items()}
+    out["sigma_abs"] = {n: np.sqrt(a) for n, a in sa.items()}
     return out

@@ -191,3 +191,36 @@ def test_given_forward_results_equal_recomputed_ones():
                            o=o.astype(np.float32), lse=(lse - np.log(2.0)).astype(np.float32), **a)
     # (up to the fp32 rounding of the two lse arrays)
     np.testing.assert_allclose(half["dv"], 2.0 * given["dv"], rtol=2e-5, atol=1e-9)
+
+
+@pytest.mark.parametrize("case", [
+    dict(seed=41, B=2, T=37, HQ=4, H=2, K=6, V=5, gs=True, sink=True, window=0, cu=None,
+         dlse=True, batch=1),
+    dict(seed=42, B=1, T=45, HQ=4, H=1, K=4, V=3, gs=False, sink=False, window=9,
+         cu=[0, 13, 14, 45], dlse=False, batch=0),
+])
+def test_row_backward_equals_full_oracle(case):
+    """The numpy row backward (used at full size on the GPU machine) equals the C oracle's
+    gradients and sigma scales at the sampled rows, given the same o and lse."""
+    d = _inputs(case["seed"], B=case["B"], T=case["T"], HQ=case["HQ"], H=case["H"], K=case["K"],
+                V=case["V"], gscale=0.3, gs=case["gs"], sink=case["sink"])
+    rng = np.random.default_rng(case["seed"] + 1)
+    do = rng.standard_normal((case["B"], case["T"], case["HQ"], case["V"])).astype(np.float32)
+    dlse = (rng.standard_normal((case["B"], case["T"], case["HQ"])).astype(np.float32)
+            if case["dlse"] else None)
+    a = dict(window=case["window"], cu_seqlens=case["cu"], scale=0.6)
+    o, lse = oracle.wall_fwd(d["q"], d["k"], d["v"], d["g"], d["g_scalar"], d["sink_bias"], **a)
+    o, lse = o.astype(np.float32), lse.astype(np.float32)
+    full = oracle.wall_bwd(d["q"], d["k"], d["v"], d["g"], do, d["g_scalar"], d["sink_bias"],
+                           dlse=dlse, o=o, lse=lse, scales=True, **a)
+    qr, kr = [0, 1, 13, case["T"] - 2, case["T"] - 1], [0, 5, 13, 14, case["T"] - 1]
+    rows = oracle.wall_bwd_rows(d["q"], d["k"], d["v"], d["g"], do, o, lse, q_rows=qr, k_rows=kr,
+                                g_scalar=d["g_scalar"], dlse=dlse, batch=case["batch"], **a)
+    b = case["batch"]
+    for name, idx in (("dq", qr), ("dk", kr), ("dv", kr)):
+        np.testing.assert_allclose(rows[name], full[name][b, idx], rtol=1e-9, atol=1e-12,
+                                   err_msg=name)
+        np.testing.assert_allclose(rows["sigma"][name], full["sigma"][name][b, idx], rtol=1e-9,
+                                   atol=1e-12, err_msg="sigma " + name)
+        np.testing.assert_allclose(rows["sigma_abs"][name], full["sigma_abs"][name][b, idx],
+                                   rtol=1e-9, atol=1e-12, err_msg="sigma_abs " + name)
