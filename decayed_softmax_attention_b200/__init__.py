@@ -39,11 +39,13 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "_lib", "libwall_attn.so")
 
 WALL_OK = 0
+WALL_ERR_DEVICE_TIMEOUT = 4
+WALL_ERR_RANGE = 6
 WALL_DTYPE_F32 = 0
 WALL_DTYPE_BF16 = 1
 _STATUS = {
     0: "WALL_OK", 1: "WALL_ERR_INVALID_ARG", 2: "WALL_ERR_UNSUPPORTED", 3: "WALL_ERR_CUDA",
-    4: "WALL_ERR_DEVICE_TIMEOUT", 5: "WALL_ERR_WORKSPACE",
+    4: "WALL_ERR_DEVICE_TIMEOUT", 5: "WALL_ERR_WORKSPACE", 6: "WALL_ERR_RANGE",
 }
 
 EXPORTED_SYMBOLS = (

@@ -109,6 +109,8 @@ const char* wall_status_string(wall_status_t s) {
     case WALL_ERR_CUDA: return "WALL_ERR_CUDA: a CUDA call failed";
     case WALL_ERR_DEVICE_TIMEOUT: return "WALL_ERR_DEVICE_TIMEOUT: a bounded device wait gave up";
     case WALL_ERR_WORKSPACE: return "WALL_ERR_WORKSPACE: workspace too small";
+    case WALL_ERR_RANGE:
+      return "WALL_ERR_RANGE: decay within one anchor span exceeds the representable range";
   }
   return "WALL_ERR_UNKNOWN";
 }
@@ -186,6 +188,7 @@ wall_status_t fwd_impl(const void* q, const void* k, const void* v, const void* 
   if (!bf16) {
     e = wall::launch_fwd_simt(a, w, st);
     stage_event(2, st);
+    if (e == cudaSuccess) e = wall::launch_fwd_diag(a, w, bf16, st);
     return finish(e, st);
   }
 
@@ -224,6 +227,7 @@ wall_status_t fwd_impl(const void* q, const void* k, const void* v, const void* 
   }
   e = wall::launch_fwd_tc(a, w, tmQ, tmK, tmV, tmKX, st);
   stage_event(2, st);
+  if (e == cudaSuccess) e = wall::launch_fwd_diag(a, w, bf16, st);
   return finish(e, st);
 }
 
@@ -310,6 +314,7 @@ wall_status_t wall_attn_bwd(const void* q, const void* k, const void* v, const v
   f.scale = scale; f.o = const_cast<void*>(o); f.lse = const_cast<float*>(lse); f.err = err;
   f.wait_ns = wall::wait_limit_ns();
   f.fault = g_fault_mode.load();
+  f.wide_is_error = true;  // the backward's tiles have no exact path for wide blocks yet
   a.dout = dout; a.dlse = dlse;
   a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dg_scalar = dg_scalar; a.dsink = dsink;
   for (int i = 0; i < 3; ++i) a.ev[i] = g_stage_ev[i].load();
@@ -411,7 +416,8 @@ static wall_status_t append_entry(const void* k_new, const void* g_new, const fl
   a.k_new = k_new; a.g_new = g_new; a.p_prev = p_prev;
   a.B = B; a.t_start = 0; a.T_new = 1; a.cap = cap; a.HQ = HQ; a.H = H; a.K = K;
   a.chunk = chunk; a.k_tilde = k_tilde; a.r_cache = r_cache; a.p_last = p_last;
-  a.err = nullptr; a.wait_ns = 0; a.fault = 0;
+  a.err = wall::device_error_word(); a.wait_ns = 0; a.fault = 0;
+  if (a.err == nullptr) return WALL_ERR_CUDA;
   if (pm != nullptr) a.pm = *pm;
   a.pm.cap = cap;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -729,7 +735,7 @@ wall_status_t wall_device_error(wall_stream_t stream) {
   if (h != 0) {
     const int zero = 0;
     if (cudaMemcpyToSymbol(g_wall_err, &zero, sizeof(int)) != cudaSuccess) return WALL_ERR_CUDA;
-    return WALL_ERR_DEVICE_TIMEOUT;
+    return (h & wall::kDevErrTimeout) ? WALL_ERR_DEVICE_TIMEOUT : WALL_ERR_RANGE;
   }
   return WALL_OK;
 }

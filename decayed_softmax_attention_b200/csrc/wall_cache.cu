@@ -162,6 +162,7 @@ __global__ void __launch_bounds__(160) cache_build_kernel(
 
   const int cmask = C - 1;  // C is a power of two
   const int gstr = HPC * KD, kstr = NKV * KD;  // shared-memory row strides (elements)
+  float kx = 0.f;  // largest exponent R_c - P_j of this thread's rows (cache range check)
   // One row: fold g into the prefix, anchor at a chunk head, rescale k.
   auto row = [&](const T* g_s, const T* k_s, T* o_g, bool head, int ta) {
     Vec4<T> gv, kv;
@@ -186,7 +187,10 @@ __global__ void __launch_bounds__(160) cache_build_kernel(
           make_float4(carry[0] + loc[0], carry[1] + loc[1], carry[2] + loc[2], carry[3] + loc[3]);
     }
 #pragma unroll
-    for (int c = 0; c < 4; ++c) k[c] *= ex2_approx(r0[c] - loc[c]);
+    for (int c = 0; c < 4; ++c) {
+      kx = fmaxf(kx, r0[c] - loc[c]);
+      k[c] *= ex2_approx(r0[c] - loc[c]);
+    }
     Vec4<T>::store(o_g, k);
   };
 
@@ -229,6 +233,7 @@ __global__ void __launch_bounds__(160) cache_build_kernel(
   if (ok && active && !segmented)
     *reinterpret_cast<float4*>(p_last + bh * KD + ch) =
         make_float4(carry[0] + loc[0], carry[1] + loc[1], carry[2] + loc[2], carry[3] + loc[3]);
+  if (kx > kCacheRangeLog2) atomicOr(err, kDevErrRange);
 }
 
 __device__ __forceinline__ void store_one(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
@@ -288,7 +293,8 @@ template <typename T, int KD>
 __global__ void __launch_bounds__(128) cache_segscan_kernel(
     const T* __restrict__ k_new, const T* __restrict__ g_new, const float* __restrict__ p_prev,
     int B, int t_start, int T_new, PageMap pm, int HQ, int H, int C, int seg_first, int seg_rows,
-    int nseg, T* __restrict__ k_tilde, float* __restrict__ r_cache, float* __restrict__ p_last) {
+    int nseg, T* __restrict__ k_tilde, float* __restrict__ r_cache, float* __restrict__ p_last,
+    int* err) {
   const long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= static_cast<long>(B) * HQ * KD) return;
   const int n = static_cast<int>(idx % KD);
@@ -305,6 +311,7 @@ __global__ void __launch_bounds__(128) cache_segscan_kernel(
       const float kv = load1(k_new + (row * H + kvh) * KD + n);
       store_one(k_tilde + (pm.row(b, t_start + t) * HQ + hq) * KD + n, kv * ex2_approx(r0 - loc));
     }
+    if (r0 - loc > kCacheRangeLog2) atomicOr(err, kDevErrRange);
     carry += loc;
   }
   for (int s = 0; s < nseg; ++s) {
@@ -322,7 +329,7 @@ template <typename T, int KD>
 __global__ void __launch_bounds__(128) cache_append_varlen_kernel(
     const T* __restrict__ k_new, const T* __restrict__ g_new, const float* __restrict__ p_prev,
     const int* __restrict__ t_pos, int B, PageMap pm, int HQ, int H, int C,
-    T* __restrict__ k_tilde, float* __restrict__ r_cache, float* __restrict__ p_last) {
+    T* __restrict__ k_tilde, float* __restrict__ r_cache, float* __restrict__ p_last, int* err) {
   constexpr int TPS = KD / 4;
   const long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= static_cast<long>(B) * HQ * TPS) return;
@@ -346,6 +353,8 @@ __global__ void __launch_bounds__(128) cache_append_varlen_kernel(
     *reinterpret_cast<float4*>(rr) = make_float4(P[0], P[1], P[2], P[3]);  // new chunk anchor
   } else {
     const float4 R = *reinterpret_cast<const float4*>(rr);
+    if (fmaxf(fmaxf(R.x - P[0], R.y - P[1]), fmaxf(R.z - P[2], R.w - P[3])) > kCacheRangeLog2)
+      atomicOr(err, kDevErrRange);
     k[0] *= ex2_approx(R.x - P[0]);
     k[1] *= ex2_approx(R.y - P[1]);
     k[2] *= ex2_approx(R.z - P[2]);
@@ -462,7 +471,7 @@ cudaError_t append_varlen_impl(const CacheArgs& a, const int* t_pos, cudaStream_
   const long n = static_cast<long>(a.B) * a.HQ * (KD / 4);
   cache_append_varlen_kernel<T, KD><<<static_cast<unsigned>((n + 127) / 128), 128, 0, st>>>(
       static_cast<const T*>(a.k_new), static_cast<const T*>(a.g_new), a.p_prev, t_pos, a.B, a.pm,
-      a.HQ, a.H, a.chunk, static_cast<T*>(a.k_tilde), a.r_cache, a.p_last);
+      a.HQ, a.H, a.chunk, static_cast<T*>(a.k_tilde), a.r_cache, a.p_last, a.err);
   return cudaGetLastError();
 }
 
@@ -535,7 +544,7 @@ cudaError_t cache_impl(const CacheArgs& a, cudaStream_t st) {
     cache_segscan_kernel<T, KD><<<static_cast<unsigned>((nthr + 127) / 128), 128, 0, st>>>(
         static_cast<const T*>(a.k_new), static_cast<const T*>(a.g_new), a.p_prev, a.B, a.t_start,
         a.T_new, a.pm, a.HQ, a.H, a.chunk, seg_first, seg_rows, nseg,
-        static_cast<T*>(a.k_tilde), a.r_cache, a.p_last);
+        static_cast<T*>(a.k_tilde), a.r_cache, a.p_last, a.err);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -110,7 +110,7 @@ __global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_s
     const __nv_bfloat16* __restrict__ qh, const float* __restrict__ AQ,
     const float* __restrict__ r_cache, int t0, int M, int HQ, int C, int cap, int window,
     int ck_lo, int cps, int nsplit, int ntg, float sc, float* __restrict__ part, int* err,
-    uint64_t wait_ns) {
+    uint64_t wait_ns, const int* __restrict__ wide) {
   using D = MultiCfg<KD, VD, G>;
   constexpr int MQ = D::MQ, LPH = D::LPH, CPL = D::CPL, VPL = D::VPL, RB = D::RB, NV = D::NV;
   constexpr int NO = D::NO, REP = D::REP, MG = MQ * G;
@@ -194,6 +194,10 @@ __global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_s
     for (int c = 0; c < VPL; ++c) o2[kp][c] = make_float2(0.f, 0.f);
   const int hl = lane / LPH, l = lane % LPH;
   const int chan0 = hl * KD + l * PC;  // channel of piece j: chan0 + j * LPH * PC
+  // Strong decay inside the chunk (one 256-row query block): this head's rows
+  // from t0 on are left to the diagonal kernel (masked here, factors kept finite).
+  const bool wide_h = wide[static_cast<size_t>(b) * HQ + h * G + hl] != 0;
+  const int row_cap = wide_h ? t0 - 1 : 0x7fffffff;
   const int base = NV >= LPH ? l * NO : l / REP;  // first owned score index (token-major)
   const int m_own = base / RB;                    // this lane's token
   if (warp < D::NW) {
@@ -216,8 +220,10 @@ __global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_s
         for (int e = 0; e < CPL; e += 2) {
           const int n = chan0 + (e / PC) * LPH * PC + e % PC;
           const float2 r2 = *reinterpret_cast<const float2*>(R + n);
-          const float2 f = make_float2(exp2f(sAQ[e * 32 + lane] - r2.x),
-                                       exp2f(sAQ[(e + 1) * 32 + lane] - r2.y));
+          const bool own = wide_h && cur_chunk * C >= t0;
+          const float2 f = own ? make_float2(0.f, 0.f)
+                               : make_float2(exp2f(sAQ[e * 32 + lane] - r2.x),
+                                             exp2f(sAQ[(e + 1) * 32 + lane] - r2.y));
 #pragma unroll
           for (int m = 0; m < MQ; ++m)
             qt2[m][e / 2] = __fmul2_rn(
@@ -254,7 +260,7 @@ __global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_s
 #pragma unroll
         for (int j = 0; j < NO; ++j) {
           const int row = row0 + rg0 + (base % RB) + j;
-          const bool ok = mg_own < M && row < row_end && row <= t0 + mg_own &&
+          const bool ok = mg_own < M && row < row_end && row <= t0 + mg_own && row <= row_cap &&
                           (window == 0 || t0 + mg_own - row < window);
           v[j] = ok ? v[j] : -INFINITY;
           mx = fmaxf(mx, v[j]);
@@ -358,8 +364,8 @@ __global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_s
 }
 
 template <int KD, int VD, int G>
-cudaError_t chunk_split_impl(const ChunkArgs& a, const void* qh, const float* AQ, float* part,
-                             cudaStream_t st) {
+cudaError_t chunk_split_impl(const ChunkArgs& a, const void* qh, const float* AQ, const int* wide,
+                             float* lse, float* part, cudaStream_t st) {
   using D = MultiCfg<KD, VD, G>;
   CUtensorMap tmK, tmV;
   // the maps end at the chunk's last row: rows past it arrive as zeros
@@ -405,22 +411,22 @@ cudaError_t chunk_split_impl(const ChunkArgs& a, const void* qh, const float* AQ
   if (a.ev_mid != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(a.ev_mid), st);
   kern<<<grid, (D::NW + 1) * 32, D::SMEM, st>>>(
       tmK, tmV, static_cast<const __nv_bfloat16*>(qh), AQ, a.r_cache, a.t0, a.M, a.HQ, a.chunk,
-      a.cap, a.window, ck_lo, cps, nsplit, ntg, a.scale * kLog2e, part, a.err, a.wait_ns);
+      a.cap, a.window, ck_lo, cps, nsplit, ntg, a.scale * kLog2e, part, a.err, a.wait_ns, wide);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_decode_combine_bf16(part, nsplit, a.B * a.M * a.HQ, a.HQ, a.sink, a.o, a.lse, VD,
+  return launch_decode_combine_bf16(part, nsplit, a.B * a.M * a.HQ, a.HQ, a.sink, a.o, lse, VD,
                                     st);
 }
 
 template <int KD, int VD>
-cudaError_t chunk_split_by_group(const ChunkArgs& a, const void* qh, const float* AQ, float* part,
-                                 cudaStream_t st) {
+cudaError_t chunk_split_by_group(const ChunkArgs& a, const void* qh, const float* AQ,
+                                 const int* wide, float* lse, float* part, cudaStream_t st) {
   switch (a.HQ / a.H) {
-    case 1: return chunk_split_impl<KD, VD, 1>(a, qh, AQ, part, st);
-    case 2: return chunk_split_impl<KD, VD, 2>(a, qh, AQ, part, st);
-    case 4: return chunk_split_impl<KD, VD, 4>(a, qh, AQ, part, st);
-    case 8: return chunk_split_impl<KD, VD, 8>(a, qh, AQ, part, st);
-    case 16: return chunk_split_impl<KD, VD, 16>(a, qh, AQ, part, st);
+    case 1: return chunk_split_impl<KD, VD, 1>(a, qh, AQ, wide, lse, part, st);
+    case 2: return chunk_split_impl<KD, VD, 2>(a, qh, AQ, wide, lse, part, st);
+    case 4: return chunk_split_impl<KD, VD, 4>(a, qh, AQ, wide, lse, part, st);
+    case 8: return chunk_split_impl<KD, VD, 8>(a, qh, AQ, wide, lse, part, st);
+    case 16: return chunk_split_impl<KD, VD, 16>(a, qh, AQ, wide, lse, part, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -438,12 +444,12 @@ size_t chunk_split_part_bytes(int B, int M, int cap, int HQ, int H, int V, int c
          sizeof(float);
 }
 
-cudaError_t launch_chunk_split(const ChunkArgs& a, const void* qh, const float* AQ, float* part,
-                               cudaStream_t st) {
-  if (a.K == 64 && a.V == 64) return chunk_split_by_group<64, 64>(a, qh, AQ, part, st);
-  if (a.K == 64 && a.V == 128) return chunk_split_by_group<64, 128>(a, qh, AQ, part, st);
-  if (a.K == 128 && a.V == 64) return chunk_split_by_group<128, 64>(a, qh, AQ, part, st);
-  if (a.K == 128 && a.V == 128) return chunk_split_by_group<128, 128>(a, qh, AQ, part, st);
+cudaError_t launch_chunk_split(const ChunkArgs& a, const void* qh, const float* AQ,
+                               const int* wide, float* lse, float* part, cudaStream_t st) {
+  if (a.K == 64 && a.V == 64) return chunk_split_by_group<64, 64>(a, qh, AQ, wide, lse, part, st);
+  if (a.K == 64 && a.V == 128) return chunk_split_by_group<64, 128>(a, qh, AQ, wide, lse, part, st);
+  if (a.K == 128 && a.V == 64) return chunk_split_by_group<128, 64>(a, qh, AQ, wide, lse, part, st);
+  if (a.K == 128 && a.V == 128) return chunk_split_by_group<128, 128>(a, qh, AQ, wide, lse, part, st);
   return cudaErrorInvalidValue;
 }
 

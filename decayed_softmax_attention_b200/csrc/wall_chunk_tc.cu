@@ -23,6 +23,7 @@ struct ChunkParams {
   const float* AQ;       // [B*HQ][NQB][KD] log2 units: P just before each 256-row query block
   const float* r_cache;  // [B, ncap, HQ, KD] anchors (log2 units)
   const float* sink;
+  const int* wide;  // [B*HQ][NQB]: the block's own rows are left to the diagonal kernel
   int window;
   int B, M, t0, HQ, H, cap, NQB;
   float sc;  // scale * log2(e)
@@ -183,9 +184,13 @@ __global__ void __launch_bounds__(512, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // key-tile ranges (tile index kt = cache row / 128) of query tiles A and B
-  const int ktA_hi = (p.t0 + min(q0 + C::BM, p.M) - 1) / C::BN;
-  const int ktB_hi = has_b ? (p.t0 + min(q0 + 2 * C::BM, p.M) - 1) / C::BN : ktA_hi;
+  // key-tile ranges (tile index kt = cache row / 128) of query tiles A and B; a
+  // wide block (strong decay inside it) stops before its own first row abs0
+  const bool wide = p.wide[static_cast<size_t>(bh) * p.NQB + qblk] != 0;
+  const int abs0 = p.t0 + q0;
+  const int wide_hi = abs0 > 0 ? (abs0 - 1) / C::BN : -1;
+  const int ktA_hi = wide ? wide_hi : (p.t0 + min(q0 + C::BM, p.M) - 1) / C::BN;
+  const int ktB_hi = wide ? wide_hi : has_b ? (p.t0 + min(q0 + 2 * C::BM, p.M) - 1) / C::BN : ktA_hi;
   const int ktA_lo = sched_lo[0] / C::BN;
   const int ktB_lo = has_b ? sched_lo[1] / C::BN : ktB_hi + 1;
   const int kt_hi = has_b ? ktB_hi : ktA_hi;
@@ -315,7 +320,7 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const uint32_t colS = C::COL_S + 128 * X, colO = C::COL_O + 128 * X;
     const int lo = row_ok ? my_lo : 0;
-    const int hi = row_ok ? gi : -1;
+    const int hi = row_ok ? (wide ? min(gi, abs0 - 1) : gi) : -1;
     const float2 sc2 = make_float2(p.sc, p.sc);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
@@ -448,9 +453,12 @@ __global__ void __launch_bounds__(512, 1)
       const bool got = mbar_wait(&kfull[ks], (j / C::KS) & 1, wc);
       float* cb = sC + (j & 1) * C::NRC * KD;
       if (got && r < KD) {
+        const int kt = kt_hi - j;
 #pragma unroll
-        for (int c = 0; c < C::NRC; ++c)
-          cb[c * KD + r] = ex2_approx(sAQ[r] - sR[(ks * C::NRC + c) * KD + r]);
+        for (int c = 0; c < C::NRC; ++c)  // a wide block's own chunks: masked, kept finite
+          cb[c * KD + r] = (wide && kt * C::BN + c * CH >= abs0)
+                               ? 0.f
+                               : ex2_approx(sAQ[r] - sR[(ks * C::NRC + c) * KD + r]);
       }
       if (bar_or(1, 128, !got || *abort_flag != 0)) break;
       uint8_t* tile = sK + ks * C::K_BYTES + box * 16384;
@@ -542,9 +550,11 @@ template <int KD>
 __global__ void __launch_bounds__(256) chunk_apply_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ g,
     const float* __restrict__ p_prev, const float* __restrict__ bsum, int M, int t0, int HQ,
-    int NQB, __nv_bfloat16* __restrict__ qh, float* __restrict__ AQ) {
+    int NQB, __nv_bfloat16* __restrict__ qh, float* __restrict__ AQ, int* __restrict__ wide) {
   using PC = ChunkPrepCfg<KD>;
   __shared__ float tot[PC::RG][KD];
+  __shared__ int s_span;  // largest |P_i - AQ| of the block (float bits), log2 units
+  if (threadIdx.x == 0) s_span = 0;
   const int blk = blockIdx.x, bh = blockIdx.y, b = bh / HQ, hq = bh % HQ;
   const int cg = threadIdx.x % PC::CG, rg = threadIdx.x / PC::CG;
   const int r0 = blk * 256 + rg * PC::RPG, r1 = min(M, r0 + PC::RPG);
@@ -573,6 +583,7 @@ __global__ void __launch_bounds__(256) chunk_apply_kernel(
     loc[c] = pre;
   }
   __nv_bfloat16* ob = qh + static_cast<size_t>(bh) * M * KD + cg * 4;
+  float span = 0.f;
 #pragma unroll 4
   for (int r = r0; r < r1; ++r) {
     const uint2 gu = *reinterpret_cast<const uint2*>(gb + r * rstep);
@@ -583,6 +594,7 @@ __global__ void __launch_bounds__(256) chunk_apply_kernel(
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       loc[c] = fmaf(gv[c], kLog2e, loc[c]);
+      span = fmaxf(span, fabsf(loc[c]));
       o4[c] = qv[c] * ex2_approx(loc[c]);
     }
     uint2 ou;
@@ -590,10 +602,18 @@ __global__ void __launch_bounds__(256) chunk_apply_kernel(
     ou.y = pack_bf16(o4[2], o4[3]);
     *reinterpret_cast<uint2*>(ob + static_cast<size_t>(r) * KD) = ou;
   }
+  // The block's own cache chunks carry anchors P at rows inside it, so the
+  // factor exp2(AQ - R_c) spans the same range as the query factor.
+  if (span > 0.f) atomicMax(&s_span, __float_as_int(span));
+  __syncthreads();
+  if (threadIdx.x == 0)
+    wide[static_cast<size_t>(bh) * NQB + blk] =
+        __int_as_float(s_span) > kPrefillSpanNats * kLog2e ? 1 : 0;
 }
 
 template <int KD, int VD, int CH>
-cudaError_t chunk_impl(const ChunkArgs& a, void* qh, float* AQ, cudaStream_t st) {
+cudaError_t chunk_impl(const ChunkArgs& a, void* qh, float* AQ, const int* wide, float* lse,
+                       cudaStream_t st) {
   using C = ChCfg<KD, VD, CH>;
   const int BHQ = a.B * a.HQ;
   const int NQB = (a.M + 255) / 256;
@@ -635,6 +655,7 @@ cudaError_t chunk_impl(const ChunkArgs& a, void* qh, float* AQ, cudaStream_t st)
   p.AQ = AQ;
   p.r_cache = a.r_cache;
   p.sink = a.sink;
+  p.wide = wide;
   p.window = a.window;
   p.B = a.B;
   p.M = a.M;
@@ -645,7 +666,7 @@ cudaError_t chunk_impl(const ChunkArgs& a, void* qh, float* AQ, cudaStream_t st)
   p.NQB = NQB;
   p.sc = a.scale * kLog2e;
   p.o = static_cast<__nv_bfloat16*>(a.o);
-  p.lse = a.lse;
+  p.lse = lse;
   p.err = a.err;
   p.wait_ns = a.wait_ns;
   const unsigned grid = static_cast<unsigned>(NQB) * BHQ;
@@ -655,11 +676,12 @@ cudaError_t chunk_impl(const ChunkArgs& a, void* qh, float* AQ, cudaStream_t st)
 }
 
 template <int KD, int VD>
-cudaError_t chunk_by_c(const ChunkArgs& a, void* qh, float* AQ, cudaStream_t st) {
+cudaError_t chunk_by_c(const ChunkArgs& a, void* qh, float* AQ, const int* wide, float* lse,
+                       cudaStream_t st) {
   switch (a.chunk) {
-    case 32: return chunk_impl<KD, VD, 32>(a, qh, AQ, st);
-    case 64: return chunk_impl<KD, VD, 64>(a, qh, AQ, st);
-    case 128: return chunk_impl<KD, VD, 128>(a, qh, AQ, st);
+    case 32: return chunk_impl<KD, VD, 32>(a, qh, AQ, wide, lse, st);
+    case 64: return chunk_impl<KD, VD, 64>(a, qh, AQ, wide, lse, st);
+    case 128: return chunk_impl<KD, VD, 128>(a, qh, AQ, wide, lse, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -671,14 +693,16 @@ size_t align256c(size_t x) { return (x + 255) / 256 * 256; }
 size_t chunk_workspace_bytes(int B, int M, int cap, int HQ, int H, int K, int V, int chunk) {
   const size_t BHQ = static_cast<size_t>(B) * HQ;
   const size_t NQB = (static_cast<size_t>(M) + 255) / 256;
-  const size_t prep = align256c(BHQ * M * K * 2) + 2 * align256c(BHQ * NQB * K * 4);
+  const size_t prep = align256c(BHQ * M * K * 2) + 2 * align256c(BHQ * NQB * K * 4) +
+                      align256c(BHQ * NQB * 4) + align256c(BHQ * M * 4);
   return prep + (chunk_split_applies(M, HQ, H)
                      ? align256c(chunk_split_part_bytes(B, M, cap, HQ, H, V, chunk))
                      : 0);
 }
 
 template <int KD>
-cudaError_t chunk_prep(const ChunkArgs& a, void* qh, float* AQ, float* bsum, cudaStream_t st) {
+cudaError_t chunk_prep(const ChunkArgs& a, void* qh, float* AQ, float* bsum, int* wide,
+                       cudaStream_t st) {
   const int NQB = (a.M + 255) / 256;
   const dim3 grid(NQB, a.B * a.HQ);
   const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(a.g_new);
@@ -689,7 +713,7 @@ cudaError_t chunk_prep(const ChunkArgs& a, void* qh, float* AQ, float* bsum, cud
   }
   chunk_apply_kernel<KD><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.q), g,
                                                a.p_prev, bsum, a.M, a.t0, a.HQ, NQB,
-                                               static_cast<__nv_bfloat16*>(qh), AQ);
+                                               static_cast<__nv_bfloat16*>(qh), AQ, wide);
   return cudaGetLastError();
 }
 
@@ -698,12 +722,19 @@ cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t st) {
   const size_t BHQ = static_cast<size_t>(a.B) * a.HQ;
   const size_t NQB = (static_cast<size_t>(a.M) + 255) / 256;
   void* qh = ws;
-  float* AQ = reinterpret_cast<float*>(ws + align256c(BHQ * a.M * a.K * 2));
-  float* bsum = reinterpret_cast<float*>(reinterpret_cast<char*>(AQ) + align256c(BHQ * NQB * a.K * 4));
+  char* cur = ws + align256c(BHQ * a.M * a.K * 2);
+  float* AQ = reinterpret_cast<float*>(cur);
+  cur += align256c(BHQ * NQB * a.K * 4);
+  float* bsum = reinterpret_cast<float*>(cur);
+  cur += align256c(BHQ * NQB * a.K * 4);
+  int* wide = reinterpret_cast<int*>(cur);
+  cur += align256c(BHQ * NQB * 4);
+  float* lse = a.lse != nullptr ? a.lse : reinterpret_cast<float*>(cur);
+  cur += align256c(BHQ * a.M * 4);
   // 1. the chunk's queries, anchored (reads p_prev before the append below
   //    overwrites p_last, which may be the same buffer)
-  cudaError_t e = a.K == 64 ? chunk_prep<64>(a, qh, AQ, bsum, st)
-                            : chunk_prep<128>(a, qh, AQ, bsum, st);
+  cudaError_t e = a.K == 64 ? chunk_prep<64>(a, qh, AQ, bsum, wide, st)
+                            : chunk_prep<128>(a, qh, AQ, bsum, wide, st);
   if (e != cudaSuccess) return e;
   // 2. the chunk's keys join the cache (rows t0 .. t0 + M - 1)
   CacheArgs c;
@@ -717,15 +748,28 @@ cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t st) {
   // 3. the chunk's queries attend the cache: a few tokens per sequence the
   //    decode's way, longer chunks in 128-row tensor-core query tiles
   if (chunk_split_applies(a.M, a.HQ, a.H)) {
-    float* part = reinterpret_cast<float*>(reinterpret_cast<char*>(bsum) +
-                                           align256c(BHQ * NQB * a.K * 4));
-    return launch_chunk_split(a, qh, AQ, part, st);
+    e = launch_chunk_split(a, qh, AQ, wide, lse, reinterpret_cast<float*>(cur), st);
+  } else if (a.K == 64 && a.V == 64) {
+    e = chunk_by_c<64, 64>(a, qh, AQ, wide, lse, st);
+  } else if (a.K == 64 && a.V == 128) {
+    e = chunk_by_c<64, 128>(a, qh, AQ, wide, lse, st);
+  } else if (a.K == 128 && a.V == 64) {
+    e = chunk_by_c<128, 64>(a, qh, AQ, wide, lse, st);
+  } else if (a.K == 128 && a.V == 128) {
+    e = chunk_by_c<128, 128>(a, qh, AQ, wide, lse, st);
+  } else {
+    return cudaErrorInvalidValue;
   }
-  if (a.K == 64 && a.V == 64) return chunk_by_c<64, 64>(a, qh, AQ, st);
-  if (a.K == 64 && a.V == 128) return chunk_by_c<64, 128>(a, qh, AQ, st);
-  if (a.K == 128 && a.V == 64) return chunk_by_c<128, 64>(a, qh, AQ, st);
-  if (a.K == 128 && a.V == 128) return chunk_by_c<128, 128>(a, qh, AQ, st);
-  return cudaErrorInvalidValue;
+  if (e != cudaSuccess) return e;
+  // 4. wide blocks (strong decay inside a 256-row query block): the chunk's own
+  //    pairs there, exactly, merged with the result for the rows before
+  DiagParams d;
+  d.q = a.q; d.k = a.k_new; d.g = a.g_new; d.gs = nullptr; d.v = a.v_cache;
+  d.sink = a.sink; d.rowlo = nullptr; d.wide = wide; d.window = a.window;
+  d.B = a.B; d.Tb = a.M; d.HQ = a.HQ; d.H = a.H; d.NQB = static_cast<int>(NQB);
+  d.vT = a.cap; d.voff = a.t0; d.pos0 = a.t0;
+  d.scale = a.scale; d.o = a.o; d.lse = lse;
+  return launch_diag(d, true, a.K, a.V, st);
 }
 
 }  // namespace wall

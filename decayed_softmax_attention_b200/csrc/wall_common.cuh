@@ -17,6 +17,17 @@
 namespace wall {
 
 constexpr int kDevErrTimeout = 1;
+// A decode-cache row whose factor 2^(R_c - P_j) exceeds 2^kCacheRangeLog2:
+// the decay accumulated since its chunk's anchor row is too strong for the
+// cache format (a bf16/fp32 key times that factor would leave the exponent
+// range), so the row cannot be represented.  Reported, never silent.
+constexpr int kDevErrRange = 2;
+constexpr float kCacheRangeLog2 = 100.f;
+// Prefill: a 256-row query block whose anchored factors exp(G_i - AQ) or
+// exp(AQ - AK) inside the block would span more than this many nats (in any
+// channel) has its in-block pairs evaluated exactly by the diagonal kernel
+// instead of the anchored tensor-core tiles.
+constexpr float kPrefillSpanNats = 64.f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 

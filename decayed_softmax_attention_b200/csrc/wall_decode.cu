@@ -324,6 +324,7 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
 #pragma unroll
         for (int e = 0; e < PC; ++e) {
           const int n = j * PC + e;
+          if (!fresh && R[e] - pc[n] > kCacheRangeLog2) atomicOr(err, kDevErrRange);
           const float kt = fresh ? kn[e] : kn[e] * ex2_approx(R[e] - pc[n]);
           store1(kw + chan0 + j * LPH * PC + e, kt);
           const float ktr = as_stored(kw, kt);  // as the cache holds it

@@ -22,7 +22,7 @@ __global__ void __launch_bounds__(256) wall_fwd_simt_kernel(
     const float* __restrict__ qh, const float* __restrict__ kh, const float* __restrict__ v,
     const float* __restrict__ AQ, const float* __restrict__ AK, const float* __restrict__ ssl,
     const float* __restrict__ ssa, const float* __restrict__ sink, const int* __restrict__ rowlo,
-    int window, int B, int T, int HQ, int H, int NB, float sc, float* __restrict__ o,
+    const int* __restrict__ wide, int window, int B, int T, int HQ, int H, int NB, float sc, float* __restrict__ o,
     float* __restrict__ lse) {
   constexpr int VC = VD / 16;  // O columns per thread
   extern __shared__ float sm[];
@@ -70,7 +70,11 @@ __global__ void __launch_bounds__(256) wall_fwd_simt_kernel(
                           ssl[static_cast<size_t>(bh) * NB * kBlockRows + min(i, NB * kBlockRows - 1)];
   }
   __syncthreads();
-  const int kt_hi = min(q0 + SB - 1, T - 1) / SB;
+  // A wide 256-row block (strong decay inside it) leaves its own keys to the
+  // diagonal kernel.
+  const int a0 = q0 / (2 * kBlockRows);
+  const bool is_wide = wide[static_cast<size_t>(bh) * ((NB + 1) / 2) + a0] != 0;
+  const int kt_hi = is_wide ? a0 * (2 * kBlockRows / SB) - 1 : min(q0 + SB - 1, T - 1) / SB;
   const int kt_lo = s_lo == 0x7fffffff ? kt_hi : s_lo / SB;
 
   float m[4], l[4], acc[4][VC];
@@ -202,8 +206,9 @@ cudaError_t simt_impl(const FwdArgs& a, const FwdWork& w, cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>(nqb) * a.B * a.HQ;
   kern<<<grid, 256, smem, st>>>(static_cast<const float*>(w.qh), static_cast<const float*>(w.kh),
                                 static_cast<const float*>(a.v), w.AQ, w.AK, w.ssl, w.ssa, a.sink,
-                                a.cu_seqlens ? w.rowlo : nullptr, a.window, a.B, a.T, a.HQ, a.H,
-                                a.NB, a.scale * kLog2e, static_cast<float*>(a.o), a.lse);
+                                a.cu_seqlens ? w.rowlo : nullptr, w.wide, a.window, a.B, a.T,
+                                a.HQ, a.H, a.NB, a.scale * kLog2e, static_cast<float*>(a.o),
+                                a.lse != nullptr ? a.lse : w.lse_ws);
   return cudaGetLastError();
 }
 

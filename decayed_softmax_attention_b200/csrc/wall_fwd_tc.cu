@@ -44,6 +44,7 @@ struct TcParams {
   const float* ssa;
   const float* sink;
   const int* rowlo;
+  const int* wide;  // per (batch*head, 256-row query block): own key tiles left to the diagonal kernel
   int window;
   int B, T, HQ, H, NB;
   float sc;  // scale * log2(e)
@@ -223,8 +224,10 @@ __global__ void __launch_bounds__(512, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // key-tile ranges (tile index kt = key row / 128) of query tiles A and B
-  const int ktA_hi = 2 * qblk, ktB_hi = 2 * qblk + 1;
+  // key-tile ranges (tile index kt = key row / 128) of query tiles A and B; a
+  // wide block (strong decay inside it) stops before its own two key tiles
+  const bool wide = p.wide[static_cast<size_t>(bh) * NQB + qblk] != 0;
+  const int ktA_hi = wide ? 2 * qblk - 1 : 2 * qblk, ktB_hi = wide ? 2 * qblk - 1 : 2 * qblk + 1;
   const int ktA_lo = sched_lo[0] / C::BN;
   const int ktB_lo = has_b ? sched_lo[1] / C::BN : ktB_hi + 1;
   const int kt_hi = has_b ? ktB_hi : ktA_hi;
@@ -555,6 +558,7 @@ cudaError_t tc_impl(const FwdArgs& a, const FwdWork& w, const CUtensorMap& tmQ,
   p.ssa = w.ssa;
   p.sink = a.sink;
   p.rowlo = a.cu_seqlens ? w.rowlo : nullptr;
+  p.wide = w.wide;
   p.window = a.window;
   p.B = a.B;
   p.T = a.T;
@@ -563,7 +567,7 @@ cudaError_t tc_impl(const FwdArgs& a, const FwdWork& w, const CUtensorMap& tmQ,
   p.NB = a.NB;
   p.sc = a.scale * kLog2e;
   p.o = static_cast<__nv_bfloat16*>(a.o);
-  p.lse = a.lse;
+  p.lse = a.lse != nullptr ? a.lse : w.lse_ws;
   p.err = a.err;
   p.wait_ns = a.wait_ns;
   p.fault = a.fault;

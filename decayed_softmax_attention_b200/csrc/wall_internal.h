@@ -35,6 +35,12 @@ bool encode_tiled(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void
 //   kx      [B*HQ][T][16]  bf16 key-side gate channels for the QK contraction:
 //           (hi, lo, 0, ..., 0) with hi + lo = ssl[t] / (scale * log2(e)), bf16 head/tail
 //   rowlo   [NB*128]       first admitted key per row (packed documents only; rows < T set)
+//   wide    [B*HQ][NQB]    int32, NQB = ceil(T / 256): 1 when the anchored factors of the
+//           256-row query block would span more than kPrefillSpanNats in some channel
+//           (strong decay); the attention kernels then skip the block's own key tiles
+//           and the diagonal kernel evaluates those pairs exactly
+//   lse_ws  [B*T*HQ]       fp32 lse when the caller passes none (the diagonal kernel
+//           merges through lse)
 struct FwdWork {
   void* qh;
   void* kh;
@@ -46,6 +52,8 @@ struct FwdWork {
   float* ssa;
   void* kx;
   int* rowlo;
+  int* wide;
+  float* lse_ws;
 };
 
 struct FwdArgs {
@@ -70,6 +78,9 @@ struct FwdArgs {
   float* r_out = nullptr;     // [B, ceil(cap/chunk), HQ, K] fp32
   float* plast_out = nullptr; // [B, HQ, K] fp32
   int cache_cap = 0, cache_chunk = 64;
+  // Set by callers that cannot evaluate wide blocks exactly (the backward): the
+  // prepass then records kDevErrRange in the error word for every wide block.
+  bool wide_is_error = false;
 };
 
 size_t fwd_workspace_layout(int B, int T, int HQ, int K, bool bf16, FwdWork* w, char* base);
@@ -79,6 +90,28 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, const FwdWork& w, const CUtensorMap&
                           const CUtensorMap& tmK, const CUtensorMap& tmV, const CUtensorMap& tmKX,
                           cudaStream_t st);
 cudaError_t launch_fwd_simt(const FwdArgs& a, const FwdWork& w, cudaStream_t st);
+// Exact in-block pairs of the wide query blocks (both dtypes), merged with the
+// attention kernel's (o, lse) of the same rows.  Runs after the attention kernel,
+// which must have covered exactly the keys before each wide block.
+struct DiagParams {
+  const void* q;      // [B, Tb, HQ, K]
+  const void* k;      // [B, Tb, H, K]
+  const void* g;      // [B, Tb, HQ, K]
+  const void* gs;     // [B, Tb, HQ] or null
+  const void* v;      // local row t of batch row b: row (b * vT + voff + t) of [*, H, V]
+  const float* sink;  // [HQ] or null
+  const int* rowlo;   // first admitted key (absolute position) per row, or null
+  const int* wide;    // [B*HQ][NQB] flags, NQB = ceil(Tb / 256)
+  int window;
+  int B, Tb, HQ, H, NQB;
+  int vT, voff;
+  int pos0;           // absolute position of local row 0 (window, rowlo)
+  float scale;
+  void* o;            // [B, Tb, HQ, V]: the attention kernel's rows on entry
+  float* lse;         // [B, Tb, HQ]: likewise (natural log, sink included)
+};
+cudaError_t launch_diag(const DiagParams& p, bool bf16, int K, int V, cudaStream_t st);
+cudaError_t launch_fwd_diag(const FwdArgs& a, const FwdWork& w, bool bf16, cudaStream_t st);
 
 // Backward of the prefill.  Inputs as FwdArgs plus the forward's o and lse,
 // dO (and optional dlse); outputs dq, dk, dv, dg, dg_scalar (input dtype) and
@@ -216,8 +249,8 @@ cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t st);
 // decode's style instead of 128-row tensor-core query tiles.
 bool chunk_split_applies(int M, int HQ, int H);
 size_t chunk_split_part_bytes(int B, int M, int cap, int HQ, int H, int V, int chunk);
-cudaError_t launch_chunk_split(const ChunkArgs& a, const void* qh, const float* AQ, float* part,
-                               cudaStream_t st);
+cudaError_t launch_chunk_split(const ChunkArgs& a, const void* qh, const float* AQ,
+                               const int* wide, float* lse, float* part, cudaStream_t st);
 // The decode's split combine (merge per-split partials, add the sink), bf16 output.
 cudaError_t launch_decode_combine_bf16(const float* part, int nsplit, int nbh, int HQ,
                                       const float* sink, void* o, float* lse, int V,

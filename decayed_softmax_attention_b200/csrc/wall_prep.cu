@@ -7,10 +7,17 @@
 // and AK = G at the last row of the key's 128-row block, the first and last
 // factors are folded once into qh and kh here, and the middle one (one vector
 // per (query block, key block) pair) is applied to each key tile inside the
-// main kernel.  Every factor then spans at most 256 rows, so the exponents
-// stay bounded at any sequence length.  Prefix sums run over the whole row;
-// with packed documents only differences inside a document are ever used, so
-// they equal the per-document sums of the definition.
+// main kernel.  For a key block that ends before the query block starts, and
+// a decay g <= 0, all three factors are at most 1: they can only underflow,
+// and only where the true product is smaller still, so those tiles are exact
+// for any decay strength.  Inside the query block (its own two key tiles) the
+// query factor shrinks while exp(AQ - AK) grows, each spanning up to 256 rows
+// of accumulated decay; a block where that span exceeds kPrefillSpanNats in
+// any channel is flagged "wide", the attention kernels skip its own key tiles
+// and the diagonal kernel (wall_fwd_diag.cu) evaluates those pairs exactly.
+// Prefix sums run over the whole row; with packed documents only differences
+// inside a document are ever used, so they equal the per-document sums of the
+// definition.
 #include "wall_common.cuh"
 #include "wall_internal.h"
 
@@ -30,13 +37,15 @@ __global__ void __launch_bounds__(256, 3) prep_local_kernel(
     int HQ, int H, int NB, Tin* __restrict__ qh, Tin* __restrict__ kh, float* __restrict__ bsum,
     float* __restrict__ ssl, float* __restrict__ ssb, __nv_bfloat16* __restrict__ kx,
     float inv_scale, int* __restrict__ rowlo, Tin* __restrict__ kt, float* __restrict__ rc,
-    int cap, int C) {
+    int cap, int C, int* __restrict__ wide, int* __restrict__ err, int wide_err) {
   constexpr int CG = KD / 8;
   constexpr int RG = 128 / CG;
   constexpr int RPG = 128 / RG;
   __shared__ float tot[2][RG][KD];
   __shared__ float gfirst[2][RG][KD];  // g at the first row of each row group (cache output)
   __shared__ float wsum[2][4];
+  __shared__ int s_span;  // largest |exp argument| of the block's anchored factors (float bits)
+  if (threadIdx.x == 0) s_span = 0;
 
   const int half = threadIdx.x >> 7, tid = threadIdx.x & 127;
   const int blk = blockIdx.x * 2 + half;  // 128-row block of this half
@@ -115,6 +124,10 @@ __global__ void __launch_bounds__(256, 3) prep_local_kernel(
   const Tin* kb = k + (static_cast<size_t>(b) * T) * krow + static_cast<size_t>(kvh) * KD + cg * 8;
   Tin* qo = qh + static_cast<size_t>(bh) * T * KD + cg * 8;
   Tin* ko = kh + static_cast<size_t>(bh) * T * KD + cg * 8;
+  // |G_t - AQ| over this thread's rows and channels: the exponent of the query
+  // factor, and (at each half's last row) of the in-block key-tile factor.
+  float span = 0.f;
+  float kspan = 0.f;  // largest exponent of an emitted cache row (natural log)
   for (int m0 = 0; m0 < RPG; m0 += U2) {
     Raw8<Tin> gv[U2], rq[U2], rk[U2];
 #pragma unroll
@@ -139,6 +152,8 @@ __global__ void __launch_bounds__(256, 3) prep_local_kernel(
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           run[c] += f[c];
+          span = fmaxf(span, fabsf(qoff[c] + run[c]));
+          kspan = fmaxf(kspan, cst[c] - run[c]);
           z[c] = y[c] * ex2_approx((cst[c] - run[c]) * kLog2e);  // decode cache row (if kt)
           x[c] *= ex2_approx((qoff[c] + run[c]) * kLog2e);
           y[c] *= ex2_approx((total[c] - run[c]) * kLog2e);
@@ -149,6 +164,16 @@ __global__ void __launch_bounds__(256, 3) prep_local_kernel(
           store8(kt + ((static_cast<size_t>(b) * cap + t) * HQ + hq) * KD + cg * 8, z);
       }
     }
+  }
+
+  if (kt != nullptr && kspan * kLog2e > kCacheRangeLog2) atomicOr(err, kDevErrRange);
+  // Non-negative floats order like their bit patterns.
+  if (span > 0.f) atomicMax(&s_span, __float_as_int(span));
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int w = __int_as_float(s_span) > kPrefillSpanNats ? 1 : 0;
+    wide[static_cast<size_t>(bh) * gridDim.x + blockIdx.x] = w;
+    if (w && wide_err) atomicOr(err, kDevErrRange);
   }
 
   // Scalar gate: negated 128-block-local inclusive prefix (log2 units), one row per thread.
@@ -256,7 +281,8 @@ cudaError_t prep_impl(const FwdArgs& a, const FwdWork& w, cudaStream_t st) {
       static_cast<const Tin*>(a.g_scalar), a.cu_seqlens, a.num_seqs, a.window, a.T, a.HQ, a.H,
       a.NB, static_cast<Tin*>(w.qh), static_cast<Tin*>(w.kh), w.bsum, w.ssl, w.ssb,
       sizeof(Tin) == 2 ? static_cast<__nv_bfloat16*>(w.kx) : nullptr, 1.f / (a.scale * kLog2e),
-      w.rowlo, static_cast<Tin*>(a.kt_out), a.r_out, a.cache_cap, a.cache_chunk);
+      w.rowlo, static_cast<Tin*>(a.kt_out), a.r_out, a.cache_cap, a.cache_chunk, w.wide, a.err,
+      a.wide_is_error ? 1 : 0);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   prep_scan_kernel<KD><<<BHQ, KD + 32, 0, st>>>(w.bsum, a.g_scalar ? w.ssb : nullptr, a.NB, w.AQ,
@@ -302,6 +328,8 @@ size_t fwd_workspace_layout(int B, int T, int HQ, int K, bool bf16, FwdWork* w, 
   p->ssa = static_cast<float*>(take(BHQ * NB * 16));
   p->kx = take(BHQ * static_cast<size_t>(T) * 16 * 2);
   p->rowlo = static_cast<int*>(take(NB * kBlockRows * 4));  // padded: 128-row bulk copies
+  p->wide = static_cast<int*>(take(BHQ * ((NB + 1) / 2) * 4));
+  p->lse_ws = static_cast<float*>(take(BHQ * static_cast<size_t>(T) * 4));
   return off;
 }
 

@@ -50,7 +50,8 @@ typedef enum {
   WALL_ERR_UNSUPPORTED = 2,    /* valid but not implemented (e.g. K = 96) */
   WALL_ERR_CUDA = 3,           /* a CUDA runtime/driver call failed */
   WALL_ERR_DEVICE_TIMEOUT = 4, /* a bounded device-side wait gave up */
-  WALL_ERR_WORKSPACE = 5       /* workspace too small */
+  WALL_ERR_WORKSPACE = 5,      /* workspace too small */
+  WALL_ERR_RANGE = 6           /* decay too strong for a decode cache chunk (see below) */
 } wall_status_t;
 
 typedef enum { WALL_DTYPE_F32 = 0, WALL_DTYPE_BF16 = 1 } wall_dtype_t;

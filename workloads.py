@@ -38,7 +38,8 @@ class PrefillSpec:
     K: int
     V: int
     dtype: str                  # "f32" | "bf16"
-    g_kind: str = "normal002"   # "normal002": 0.02*N(0,1); "negsoftplus": -softplus(N(0,1)-4); "zero"
+    g_kind: str = "normal002"   # "normal002": 0.02*N(0,1); "negsoftplus": -softplus(N(0,1)-4); "zero";
+                                # strong decay: "strong", "strong_cache", "strong_all", "spike" (_decay)
     g_scalar: bool = False      # draw g_scalar = -softplus(N(0,1)-4) [B,T,HQ]
     sink: bool = False          # draw sink_bias ~ N(0,1) [HQ]
     window: int = 0             # <=0: no window
@@ -130,6 +131,29 @@ def _decay(kind, shape, gen, device):
         return 0.02 * z
     if kind == "negsoftplus":
         return -torch.nn.functional.softplus(z - 4.0)
+    # Strong per-channel decay (the method's g = -softplus(.) is unbounded below): a few
+    # channels forget within a handful of tokens while the rest keep a long memory.
+    sp = torch.nn.functional.softplus
+    K = shape[-1]
+    quarter = max(3, K // 4)
+    if kind == "strong":        # channels 0..2 constant -0.5, -2, -8; next quarter
+        g = -sp(z - 4.0)        # -softplus(N+2) (~2.1 per token); the rest -softplus(N-4)
+        g[..., 3:quarter] = -sp(z[..., 3:quarter] + 2.0)
+        g[..., 0], g[..., 1], g[..., 2] = -0.5, -2.0, -8.0
+        return g
+    if kind == "strong_cache":  # strong, yet inside one 32-row cache chunk's range:
+        g = -sp(z - 4.0)        # channels 0, 1 constant -0.5, -2; next quarter -softplus(N+1)
+        g[..., 2:quarter] = -sp(z[..., 2:quarter] + 1.0)
+        g[..., 0], g[..., 1] = -0.5, -2.0
+        return g
+    if kind == "strong_all":    # every channel -softplus(N(0,1)+2)
+        return -sp(z + 2.0)
+    if kind == "spike":         # mild everywhere except a decay of 100 in channel 5 at two
+        g = -sp(z - 4.0)        # rows (T/3 and 2T/3): only the blocks holding them are wide
+        T = shape[1]
+        for t in (T // 3, (2 * T) // 3):
+            g[:, t, ..., 5] = -100.0
+        return g
     raise ValueError(f"unknown decay distribution {kind!r}")
 
 
