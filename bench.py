@@ -48,14 +48,14 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic of the prefill attention kernel per launch on the long workload
 # (dram__bytes_read.sum + dram__bytes_write.sum from one ncu capture) and the
 # hash of the kernel source it was taken on; reported as null once the kernel
-# source changes.  Filled from profiles/ after each capture.
+# source changes.  Filled in after each capture.
 TRAFFIC = {
-    # profiles/wall_fwd_tc_long_prefill.md: 316.535808 MB read + 43.428608 MB written
+    # full capture on the long prefill: 316.535808 MB read + 43.428608 MB written
     "prefill_main": {"bytes": 359964416, "source_sha": "820590f83f572f63"},
-    # profiles/decode_split_b4_tkv32k.md, batch 4 scaled by 8 to batch 32 (traffic is
+    # capture of the decode workload at batch 4, scaled by 8 to batch 32 (traffic is
     # proportional to the batch): (1.375950 GB + 5.537536 MB) * 8
     "decode_split": {"bytes": 11051900288, "source_sha": "453f90616c845a14"},
-    # profiles/cache_build_b4_t32k.md, full-size capture (batch 32, 1-pass DRAM metrics):
+    # full-size capture of the cache build (batch 32, 1-pass DRAM metrics):
     # 10737661184 B read + 8819417344 B written
     "cache_build": {"bytes": 19557078528, "source_sha": "5ff2742a5cd5b984"},
 }

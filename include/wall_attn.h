@@ -51,7 +51,8 @@ typedef enum {
   WALL_ERR_CUDA = 3,           /* a CUDA runtime/driver call failed */
   WALL_ERR_DEVICE_TIMEOUT = 4, /* a bounded device-side wait gave up */
   WALL_ERR_WORKSPACE = 5,      /* workspace too small */
-  WALL_ERR_RANGE = 6           /* decay too strong for a decode cache chunk (see below) */
+  WALL_ERR_RANGE = 6           /* decay too strong for a decode cache chunk, or (backward)
+                                  for the anchored tiles: see wall_device_error */
 } wall_status_t;
 
 typedef enum { WALL_DTYPE_F32 = 0, WALL_DTYPE_BF16 = 1 } wall_dtype_t;
@@ -428,8 +429,17 @@ wall_status_t wall_attn_decode_noalloc(const void* q, const float* p_curr, const
 /*
  * Synchronises `stream`, then reads and clears this device's error word.
  * Returns WALL_ERR_DEVICE_TIMEOUT if any kernel since the last read gave up a
- * bounded wait (its outputs are then unspecified), WALL_ERR_CUDA if the
- * synchronisation failed, WALL_OK otherwise.
+ * bounded wait (its outputs are then unspecified); else WALL_ERR_RANGE if a
+ * kernel met decay it cannot represent (outputs unspecified where it did):
+ *   - a decode-cache row whose factor exp2(R_c - P_j) exceeds 2^100, i.e. a
+ *     channel decayed by more than ~69 nats since its chunk's first row
+ *     (the Wall Attention README's cache keeps one anchor per chunk; a
+ *     smaller chunk raises the bound), written by any cache build, append,
+ *     fused decode step or prefill that emits the cache;
+ *   - wall_attn_bwd on inputs with a 256-row block whose decay exceeds 64 nats
+ *     in some channel.
+ * The prefill and chunk outputs themselves are exact for any g <= 0.
+ * WALL_ERR_CUDA if the synchronisation failed, WALL_OK otherwise.
  */
 wall_status_t wall_device_error(wall_stream_t stream);
 
