@@ -61,6 +61,29 @@ __device__ __forceinline__ float as_stored(const __nv_bfloat16*, float x) {
   return __bfloat162float(__float2bfloat16_rn(x));
 }
 __device__ __forceinline__ float as_stored(const float*, float x) { return x; }
+// N consecutive values in as few stores as their alignment allows (the address
+// is aligned to the whole piece: 8 bytes, or N * sizeof(T) when smaller)
+template <typename T, int N>
+__device__ __forceinline__ void store_n(T* p, const float* f) {
+  if constexpr (sizeof(T) == 2 && N % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < N; i += 4) {
+      uint2 u;
+      u.x = pack_bf16(f[i], f[i + 1]);
+      u.y = pack_bf16(f[i + 2], f[i + 3]);
+      *reinterpret_cast<uint2*>(p + i) = u;
+    }
+  } else if constexpr (sizeof(T) == 2 && N % 2 == 0) {
+#pragma unroll
+    for (int i = 0; i < N; i += 2) *reinterpret_cast<uint32_t*>(p + i) = pack_bf16(f[i], f[i + 1]);
+  } else if constexpr (sizeof(T) == 4 && N % 2 == 0) {
+#pragma unroll
+    for (int i = 0; i < N; i += 2) *reinterpret_cast<float2*>(p + i) = make_float2(f[i], f[i + 1]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; ++i) store1(p + i, f[i]);
+  }
+}
 
 // ----------------------------------------------------------------- split-KV decode
 // Rows of one (batch, KV head) are streamed through a ring of shared-memory
@@ -82,8 +105,8 @@ struct DecCfg {
   static constexpr int V_BYTES = SR * VD * ESZ;
   static constexpr int R_BYTES = GK * 4;
   static constexpr int STAGE = K_BYTES + V_BYTES + R_BYTES;
-  static constexpr int MERGE = NW * G * (VD + 2) * 4;
-  static constexpr int NS0 = (196608 - MERGE) / STAGE;
+  static constexpr int MERGE = (NW + 1) * G * (VD + 2) * 4;  // + the fused step's new row
+  static constexpr int NS0 = (225280 - MERGE) / STAGE;
   static constexpr int NS = NS0 > 4 ? 4 : NS0;                     // stages in the ring
   static constexpr int OFF_BAR = NS * STAGE;
   static constexpr int OFF_MERGE = OFF_BAR + 2 * NS * 8 + 16;
@@ -93,14 +116,16 @@ struct DecCfg {
 };
 
 // FUSED: the step's new token (row T_b - 1 of each batch row) is not in the
-// cache yet.  The stream stops before it; the CTA whose split holds that row
-// forms it from k_new, g_new and p_prev exactly as the append does (P = p_prev
-// + g log2 e, a new chunk anchor or the stored one, k_tilde rounded to the cache
-// dtype), scores it after its streamed rows, and writes the row, its value, a
-// new anchor and P_last back to the cache.  No other CTA reads that row, that
-// anchor or P_last, so one launch both appends and attends.
+// cache yet.  The stream stops before it; in the CTA whose split holds that
+// row, one extra warp forms it from k_new, g_new and p_prev exactly as the
+// append does (P = p_prev + g log2 e, a new chunk anchor or the stored one,
+// k_tilde rounded to the cache dtype), scores it, and writes the row, its
+// value, a new anchor and P_last back to the cache, all while the other warps
+// stream; its (score, 1, value row) joins the CTA's merge as one more partial.
+// No other CTA reads that row, that anchor or P_last, so one launch both
+// appends and attends.
 template <typename T, int KD, int VD, int G, bool PAGED, bool GATE, bool FUSED>
-__global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_split_kernel(
+__global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 2) * 32) decode_split_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
     const T* __restrict__ q, const float* __restrict__ p_curr, const float* __restrict__ r_cache,
     int T_kv, int HQ, int C, int cps, int nsplit, float sc, float* __restrict__ part,
@@ -115,8 +140,8 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
   uint64_t* full = reinterpret_cast<uint64_t*>(dsm + D::OFF_BAR);
   uint64_t* empty = full + D::NS;
   int* abort_flag = reinterpret_cast<int*>(dsm + D::OFF_BAR + 2 * D::NS * 8);
-  float* sm_ml = reinterpret_cast<float*>(dsm + D::OFF_MERGE);       // [NW][G][2]
-  float* sm_o = sm_ml + D::NW * G * 2;                               // [NW][G][VD]
+  float* sm_ml = reinterpret_cast<float*>(dsm + D::OFF_MERGE);       // [NW + 1][G][2]
+  float* sm_o = sm_ml + (D::NW + 1) * G * 2;                         // [NW + 1][G][VD]
 
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -200,6 +225,67 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
     }
 #pragma unroll
     for (int e = 0; e < CPL; ++e) qv[e] *= sc;
+    if (FUSED && warp == D::NW + 1) {
+      // ---- the fused step's new row, formed by a warp of its own while the
+      // other warps stream the cache: its score and value enter the CTA's merge
+      // as one more partial (max = its score, sum = 1, o = its value row)
+      const bool mine = t_new >= row_begin && t_new < row_end;
+      float d = -INFINITY;
+      float vn[VPL];
+#pragma unroll
+      for (int c = 0; c < VPL; ++c) vn[c] = 0.f;
+      if (mine) {
+        const bool fresh = t_new % C == 0;  // the row opens a chunk: its anchor is its own P
+        const size_t rslot = PAGED ? pm.chunk(b, t_new, C) : static_cast<size_t>(b) * ncap + t_new / C;
+        float* ra = fu.r_cache + (rslot * HQ + h * G) * KD;
+        const size_t prow = PAGED ? pm.row(b, t_new) : static_cast<size_t>(b) * pm.cap + t_new;
+        T* kw = static_cast<T*>(fu.k_tilde) + (prow * HQ + h * G) * KD;
+        const int kofs = chan0 - hl * KD;  // this lane's first channel within its head
+        T* vw = static_cast<T*>(fu.v) + (prow * gridDim.y + h) * VD + lane * VPL;
+        load_n<T, VPL>(static_cast<const T*>(fu.v_new) + (static_cast<size_t>(b) * gridDim.y + h) * VD +
+                           lane * VPL, vn);
+        float acc = 0.f;
+#pragma unroll
+        for (int j = 0; j < CPL / PC; ++j) {
+          float R[PC], kn[PC];
+          if (fresh) {
+#pragma unroll
+            for (int e = 0; e < PC; ++e) R[e] = pc[j * PC + e];
+          } else {
+            load_n<float, PC>(ra + chan0 + j * LPH * PC, R);
+          }
+          load_n<T, PC>(static_cast<const T*>(fu.k_new) + (static_cast<size_t>(b) * gridDim.y + h) * KD +
+                            kofs + j * LPH * PC, kn);
+          float kt[PC];
+#pragma unroll
+          for (int e = 0; e < PC; ++e) {
+            const int n = j * PC + e;
+            if (!fresh && R[e] - pc[n] > kCacheRangeLog2) atomicOr(err, kDevErrRange);
+            kt[e] = as_stored(kw, fresh ? kn[e] : kn[e] * ex2_approx(R[e] - pc[n]));  // as the cache holds it
+            acc = fmaf(qv[n] * exp2f(pc[n] - R[e]), kt[e], acc);
+          }
+          // whole 16-byte pieces (a lane's piece is PC contiguous channels)
+          store_n<T, PC>(kw + chan0 + j * LPH * PC, kt);
+          if (fresh) store_n<float, PC>(ra + chan0 + j * LPH * PC, pc + j * PC);
+          store_n<float, PC>(fu.p_last + (static_cast<size_t>(b) * HQ + h * G) * KD + chan0 + j * LPH * PC,
+                             pc + j * PC);
+        }
+#pragma unroll
+        for (int off = LPH / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        d = acc;
+#pragma unroll
+        for (int c = 0; c < VPL; ++c) vn[c] = as_stored(vw, vn[c]);
+        store_n<T, VPL>(vw, vn);
+      }
+      if (lane % LPH == 0) {
+        sm_ml[(D::NW * G + hl) * 2] = d;
+        sm_ml[(D::NW * G + hl) * 2 + 1] = 1.f;
+      }
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+        for (int c = 0; c < VPL; ++c) sm_o[(D::NW * G + hh) * VD + lane * VPL + c] = vn[c];
+    } else {
     // scalar gate: the logit gains PS(current row) - PS(row j), exp2 units
     const float gcur = GATE ? gs_curr[static_cast<size_t>(b) * HQ + hq] : 0.f;
     float m = -INFINITY, l = 0.f;
@@ -301,62 +387,6 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
         }
       }
     }
-    if (FUSED && warp == 0 && t_new >= row_begin && t_new < row_end) {
-      // ---- the appended row: formed here, scored last, written to the cache
-      const bool fresh = t_new % C == 0;  // the row opens a chunk: its anchor is its own P
-      const size_t rslot = PAGED ? pm.chunk(b, t_new, C) : static_cast<size_t>(b) * ncap + t_new / C;
-      float* ra = fu.r_cache + (rslot * HQ + h * G) * KD;
-      const size_t prow = PAGED ? pm.row(b, t_new) : static_cast<size_t>(b) * pm.cap + t_new;
-      T* kw = static_cast<T*>(fu.k_tilde) + (prow * HQ + h * G) * KD;
-      const int kofs = chan0 - hl * KD;  // this lane's first channel within its head
-      float d = 0.f;
-#pragma unroll
-      for (int j = 0; j < CPL / PC; ++j) {
-        float R[PC], kn[PC];
-        if (fresh) {
-#pragma unroll
-          for (int e = 0; e < PC; ++e) R[e] = pc[j * PC + e];
-        } else {
-          load_n<float, PC>(ra + chan0 + j * LPH * PC, R);
-        }
-        load_n<T, PC>(static_cast<const T*>(fu.k_new) + (static_cast<size_t>(b) * gridDim.y + h) * KD +
-                          kofs + j * LPH * PC, kn);
-#pragma unroll
-        for (int e = 0; e < PC; ++e) {
-          const int n = j * PC + e;
-          if (!fresh && R[e] - pc[n] > kCacheRangeLog2) atomicOr(err, kDevErrRange);
-          const float kt = fresh ? kn[e] : kn[e] * ex2_approx(R[e] - pc[n]);
-          store1(kw + chan0 + j * LPH * PC + e, kt);
-          const float ktr = as_stored(kw, kt);  // as the cache holds it
-          d = fmaf(qv[n] * exp2f(pc[n] - R[e]), ktr, d);
-          if (fresh) ra[chan0 + j * LPH * PC + e] = pc[n];
-          fu.p_last[(static_cast<size_t>(b) * HQ + h * G) * KD + chan0 + j * LPH * PC + e] = pc[n];
-        }
-      }
-#pragma unroll
-      for (int off = LPH / 2; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-      float vn[VPL];
-      T* vw = static_cast<T*>(fu.v) + (prow * gridDim.y + h) * VD + lane * VPL;
-      load_n<T, VPL>(static_cast<const T*>(fu.v_new) + (static_cast<size_t>(b) * gridDim.y + h) * VD +
-                         lane * VPL, vn);
-#pragma unroll
-      for (int c = 0; c < VPL; ++c) {
-        store1(vw + c, vn[c]);
-        vn[c] = as_stored(vw, vn[c]);
-      }
-      const float mn = fmaxf(m, d);
-      const float alpha = exp2f(m - mn);
-      const float pr = exp2f(d - mn);
-      l = l * alpha + pr;
-      m = mn;
-#pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
-        const float ah = __shfl_sync(0xffffffffu, alpha, hh * LPH);
-        const float ph = __shfl_sync(0xffffffffu, pr, hh * LPH);
-#pragma unroll
-        for (int c = 0; c < VPL; ++c) o[hh][c] = fmaf(ph, vn[c], o[hh][c] * ah);
-      }
-    }
     if (lane % LPH == 0) {
       sm_ml[(warp * G + hl) * 2] = m;
       sm_ml[(warp * G + hl) * 2 + 1] = l;
@@ -365,14 +395,16 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
     for (int hh = 0; hh < G; ++hh)
 #pragma unroll
       for (int c = 0; c < VPL; ++c) sm_o[(warp * G + hh) * VD + lane * VPL + c] = o[hh][c];
+    }
   }
   __syncthreads();
+  constexpr int NPART = D::NW + (FUSED ? 1 : 0);  // partials to merge
   // merge the consumer warps of this CTA into one partial per query head
-  for (int e = threadIdx.x; e < G * (VD + 2); e += (D::NW + 1) * 32) {
+  for (int e = threadIdx.x; e < G * (VD + 2); e += blockDim.x) {
     const int hh = e / (VD + 2), c = e % (VD + 2);
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < D::NW; ++w) M = fmaxf(M, sm_ml[(w * G + hh) * 2]);
+    for (int w = 0; w < NPART; ++w) M = fmaxf(M, sm_ml[(w * G + hh) * 2]);
     float val;
     if (M == -INFINITY) {
       val = (c == VD) ? -INFINITY : 0.f;
@@ -381,7 +413,7 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 1) * 32) decode_sp
     } else {
       val = 0.f;
 #pragma unroll
-      for (int w = 0; w < D::NW; ++w) {
+      for (int w = 0; w < NPART; ++w) {
         const float mw = sm_ml[(w * G + hh) * 2];
         if (mw == -INFINITY) continue;
         const float wt = exp2f(mw - M);
@@ -482,7 +514,7 @@ cudaError_t decode_impl(const DecodeArgs& a, cudaStream_t st) {
   const int nchunks = (a.T_kv + a.chunk - 1) / a.chunk;
   const int cps = (nchunks + a.nsplit - 1) / a.nsplit;
   dim3 grid(a.nsplit, a.H, a.B);
-  kern<<<grid, (D::NW + 1) * 32, D::SMEM, st>>>(
+  kern<<<grid, (D::NW + (fused ? 2 : 1)) * 32, D::SMEM, st>>>(
       tmK, tmV, static_cast<const T*>(a.q), a.p_curr, a.r_cache, a.T_kv, a.HQ, a.chunk,
       cps, a.nsplit, a.scale * kLog2e, a.part, a.err, a.wait_ns, a.fault, a.seqlens, a.pm,
       a.gs_cache, a.gs_curr, a.fuse);
