@@ -262,7 +262,7 @@ def wall_bwd(q, k, v, g, do, g_scalar=None, sink_bias=None, window=0, cu_seqlens
 
 
 def wall_bwd_rows(q, k, v, g, do, o, lse, q_rows=(), k_rows=(), g_scalar=None, window=0,
-                  cu_seqlens=None, scale=None, dlse=None, batch=0):
+                  cu_seqlens=None, scale=None, dlse=None, batch=0, tail=0, tail_heads=None):
     """Selected rows of the prefill backward of one batch row, in double precision, straight
     from the definition (numpy; for long sequences where the full oracle is too slow).
 
@@ -274,6 +274,15 @@ def wall_bwd_rows(q, k, v, g, do, o, lse, q_rows=(), k_rows=(), g_scalar=None, w
         dk_j = scale sum_i dS_ij q_i exp(G_i - G_j),   dv_j = sum_i p_ij dO_i
     over the admitted pairs (causal, same document, window).  Also returns "sigma" and
     "sigma_abs" for each, defined as in ``wall_bwd``.
+
+    tail > 0 adds dg [tail, HQ, K] (and dg_scalar [tail, HQ] with g_scalar) at the last
+    ``tail`` rows, which must lie in the last document.  G is an inclusive prefix sum, so
+    dg_u is the sum over rows t >= u of the document of
+        dG_t = q_t * dq_t - k_t * dk_t^(hq)    (dk of query head hq alone)
+    and dg_scalar_u that of dGs_t = sum_j dS_tj - sum_i dS_it; the last rows need only
+    the last rows' terms.  sigma: the root of the sum of squares of every pair term the
+    element sums, as ``wall_bwd`` defines it.  tail_heads: the query heads to compute
+    (default all); the tail arrays then hold those heads in that order.
     """
     cv = lambda x: None if x is None else _f64(_f32(x))[batch]
     q, k, v, g, do, o, lse = (cv(x) for x in (q, k, v, g, do, o, lse))
@@ -335,6 +344,48 @@ def wall_bwd_rows(q, k, v, g, do, o, lse, q_rows=(), k_rows=(), g_scalar=None, w
             out["dv"][r, kv] += tv.sum(axis=0)
             s2["dv"][r, kv] += (tv * tv).sum(axis=0)
             sa["dv"][r, kv] += (tv * tv).sum(axis=0)
+    if tail > 0:
+        t0 = T - tail
+        assert doc[t0] == doc[T - 1], "the tail rows must lie in one (the last) document"
+        heads = list(range(HQ)) if tail_heads is None else list(tail_heads)
+        nh = len(heads)
+        dG = np.zeros((tail, nh, K))
+        dGs = np.zeros((tail, nh))
+        gq2, gqa = np.zeros((tail, nh, K)), np.zeros((tail, nh, K))
+        gs2, gsa = np.zeros((tail, nh)), np.zeros((tail, nh))
+        for r, t in enumerate(range(t0, T)):
+            js = pos[pairs(np.full(T, t), pos)]       # row t as the query
+            is_ = pos[pairs(pos, np.full(T, t))]      # row t as the key
+            for hi, hq in enumerate(heads):
+                kv = hq // grp
+                dec = np.exp(G[t, hq][None, :] - G[js, hq])
+                x = scale * (q[t, hq][None, :] * k[js, kv] * dec).sum(axis=1) + Gs[t, hq] - Gs[js, hq]
+                p = np.exp(x - lse[t, hq])
+                dP = v[js, kv] @ do[t, hq]
+                ds = p * (dP - delta[t, hq])
+                tq = q[t, hq][None, :] * scale * ds[:, None] * k[js, kv] * dec
+                tqa = np.abs(q[t, hq])[None, :] * scale * (p * (np.abs(dP) + np.abs(delta[t, hq])))[:, None] * k[js, kv] * dec
+                dec = np.exp(G[is_, hq] - G[t, hq][None, :])
+                x = scale * (q[is_, hq] * k[t, kv][None, :] * dec).sum(axis=1) + Gs[is_, hq] - Gs[t, hq]
+                p2 = np.exp(x - lse[is_, hq])
+                dP2 = do[is_, hq] @ v[t, kv]
+                ds2 = p2 * (dP2 - delta[is_, hq])
+                tk = k[t, kv][None, :] * scale * ds2[:, None] * q[is_, hq] * dec
+                tka = np.abs(k[t, kv])[None, :] * scale * (p2 * (np.abs(dP2) + np.abs(delta[is_, hq])))[:, None] * q[is_, hq] * dec
+                dG[r, hi] = tq.sum(axis=0) - tk.sum(axis=0)
+                dGs[r, hi] = ds.sum() - ds2.sum()
+                gq2[r, hi] = (tq * tq).sum(axis=0) + (tk * tk).sum(axis=0)
+                gqa[r, hi] = (tqa * tqa).sum(axis=0) + (tka * tka).sum(axis=0)
+                gs2[r, hi] = (ds * ds).sum() + (ds2 * ds2).sum()
+                da = p * (np.abs(dP) + np.abs(delta[t, hq]))
+                da2 = p2 * (np.abs(dP2) + np.abs(delta[is_, hq]))
+                gsa[r, hi] = (da * da).sum() + (da2 * da2).sum()
+        rev = lambda a: np.cumsum(a[::-1], axis=0)[::-1]
+        out["dg"] = rev(dG)
+        s2["dg"], sa["dg"] = rev(gq2), rev(gqa)
+        if gs is not None:
+            out["dg_scalar"] = rev(dGs)
+            s2["dg_scalar"], sa["dg_scalar"] = rev(gs2), rev(gsa)
     out["sigma"] = {n: np.sqrt(a) for n, a in s2.items()}
     out["sigma_abs"] = {n: np.sqrt(a) for n, a in sa.items()}
     return out

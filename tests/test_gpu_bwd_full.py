@@ -9,7 +9,11 @@ The full oracle is far too slow at this size, so the check is twofold:
     rows), from the same o and lse, within the per-element sigma bound of test_gpu_bwd;
   - a property that holds at any size: every row's weights sum to 1 (no sink in this
     workload), so sum_j dv_j equals the sum of dO over all rows and the group's query
-    heads, per KV head and channel.
+    heads, per KV head and channel;
+  - dg and dg_scalar, the reverse prefix sums that cross all 64 row blocks: at the last
+    160 rows (across the last block boundary) against the row oracle for four query
+    heads, and at row 0, where they are exactly zero (the scores depend on G and Gs only
+    through differences), so what remains there is the rounding of the whole chain.
 """
 import numpy as np
 import pytest
@@ -54,3 +58,24 @@ def test_long_prefill_backward_sampled_rows():
     assert bool((err <= bound).all()), (
         f"sum_j dv_j vs sum dO: max err {float(err.max()):.3e}, "
         f"max bound {float(bound.max()):.3e}")
+
+    # dg, dg_scalar at the last rows (they sum dG over the rows after them only)
+    tail, heads = 160, [0, 9, 18, 31]
+    rt = oracle.wall_bwd_rows(d["q"], d["k"], d["v"], d["g"], do, o, lse, tail=tail,
+                              tail_heads=heads, g_scalar=d["g_scalar"], window=d["window"],
+                              scale=d["scale"])
+    for name, sl in (("dg", (0, slice(T - tail, T), heads)),
+                     ("dg_scalar", (0, slice(T - tail, T), heads))):
+        assert_grad_close(got[name][sl], rt[name], rt["sigma"][name], rt["sigma_abs"][name],
+                          torch.bfloat16, f"full size {name} (last {tail} rows)")
+    # row 0: zero in exact arithmetic; the sum of every row's dG, through all block carries
+    dg0 = got["dg"][0, 0].double()                                     # [HQ, K]
+    qdq = (d["q"][0].double() * got["dq"][0].double())                 # [T, HQ, K]
+    s_dg = qdq.pow(2).sum(dim=0).sqrt()                                # rounding scale
+    assert bool((dg0.abs() <= 0.05 * s_dg + 1e-6).all()), (
+        f"dg at row 0: max |dg| {float(dg0.abs().max()):.3e} vs scale {float(s_dg.max()):.3e}")
+    dgs = got["dg_scalar"][0].double()                                 # [T, HQ]
+    steps = torch.cat([dgs[:-1] - dgs[1:], dgs[-1:]], dim=0)           # per-row dGs (rounded)
+    s_gs = steps.pow(2).sum(dim=0).sqrt()
+    assert bool((dgs[0].abs() <= 0.05 * s_gs + 1e-6).all()), (
+        f"dg_scalar at row 0: max {float(dgs[0].abs().max()):.3e} vs scale {float(s_gs.max()):.3e}")

@@ -193,3 +193,35 @@ def test_fused_step_paged(wall, bs):
         assert torch.equal(fused.k_tilde.view(-1, HQ, K)[rows], sep.k_tilde.view(-1, HQ, K)[rows])
         assert torch.equal(fused.v.view(-1, H, V)[rows], sep.v.view(-1, H, V)[rows])
     assert torch.equal(fused.p, sep.p)
+
+
+def test_fused_step_full_decode_workload(wall):
+    """The benchmark's decode loop at its full size (B=32, T_kv=32768 prefix, HQ=32, H=8,
+    K=V=128, C=64): build the prefix, run 3 fused steps, and check batch rows 0 and 31
+    against the oracle's prefill rows of the appended tokens."""
+    spec = W.DECODE["decode"]
+    steps = 3
+    d = W.gen_decode(spec, device="cuda")
+    B, T0, HQ, H, K, V = spec.B, spec.T0, spec.HQ, spec.H, spec.K, spec.V
+    cache = wall.KVCache(B, spec.cap, HQ, H, K, V, dtype=torch.bfloat16, chunk=spec.C)
+    cache.append(d["k"][:, :T0].contiguous(), d["g"][:, :T0].contiguous(),
+                 d["v"][:, :T0].contiguous())
+    outs = []
+    for s_ in range(steps):
+        t = T0 + s_
+        k1, g1, v1 = (d[n][:, t:t + 1].contiguous() for n in ("k", "g", "v"))
+        outs.append(cache.step(d["q"][:, s_:s_ + 1].contiguous(), k1, g1, v1,
+                               scale=d["scale"]).clone())
+    torch.cuda.synchronize()
+    assert wall.wall_device_error() == 0
+    T = T0 + steps
+    for b in (0, 31):
+        qf = torch.zeros((1, T, HQ, K), dtype=torch.bfloat16)
+        for s_ in range(steps):
+            qf[0, T0 + s_] = d["q"][b, s_].cpu()
+        rows = np.array([T0 + s_ for s_ in range(steps)], dtype=np.int64)
+        ro, _ = oracle.wall_fwd(qf, d["k"][b:b + 1, :T].cpu(), d["v"][b:b + 1, :T].cpu(),
+                                d["g"][b:b + 1, :T].cpu(), scale=d["scale"], rows=rows,
+                                threads=ORACLE_THREADS)
+        for s_ in range(steps):
+            assert_close(outs[s_][b, 0], ro[s_], torch.bfloat16, f"fused full decode b={b} step {s_}")

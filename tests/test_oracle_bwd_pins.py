@@ -217,6 +217,19 @@ def test_row_backward_equals_full_oracle(case):
     rows = oracle.wall_bwd_rows(d["q"], d["k"], d["v"], d["g"], do, o, lse, q_rows=qr, k_rows=kr,
                                 g_scalar=d["g_scalar"], dlse=dlse, batch=case["batch"], **a)
     b = case["batch"]
+    # dg / dg_scalar at the last rows (the tail lies in the last document)
+    tail = 9
+    tr = list(range(case["T"] - tail, case["T"]))
+    rt = oracle.wall_bwd_rows(d["q"], d["k"], d["v"], d["g"], do, o, lse, tail=tail,
+                              g_scalar=d["g_scalar"], dlse=dlse, batch=case["batch"], **a)
+    names = ["dg"] + (["dg_scalar"] if d["g_scalar"] is not None else [])
+    for name in names:
+        np.testing.assert_allclose(rt[name], full[name][b, tr], rtol=1e-9, atol=1e-12,
+                                   err_msg=name)
+        np.testing.assert_allclose(rt["sigma"][name], full["sigma"][name][b, tr], rtol=1e-9,
+                                   atol=1e-12, err_msg="sigma " + name)
+        np.testing.assert_allclose(rt["sigma_abs"][name], full["sigma_abs"][name][b, tr],
+                                   rtol=1e-9, atol=1e-12, err_msg="sigma_abs " + name)
     for name, idx in (("dq", qr), ("dk", kr), ("dv", kr)):
         np.testing.assert_allclose(rows[name], full[name][b, idx], rtol=1e-9, atol=1e-12,
                                    err_msg=name)
