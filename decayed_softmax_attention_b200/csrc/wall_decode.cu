@@ -104,7 +104,12 @@ struct DecCfg {
   static constexpr int K_BYTES = SR * GK * ESZ;
   static constexpr int V_BYTES = SR * VD * ESZ;
   static constexpr int R_BYTES = GK * 4;
-  static constexpr int STAGE = K_BYTES + V_BYTES + R_BYTES;
+  // scalar-gate rows of the stage ([SR][GB] fp32: the group's heads, padded to a
+  // 16-byte TMA box row), reserved in every stage, loaded only by the gated decode
+  static constexpr int GB = G >= 4 ? G : 4;
+  static constexpr int GT_BYTES = SR * GB * 4;
+  static constexpr int LOAD_BYTES = K_BYTES + V_BYTES + R_BYTES;
+  static constexpr int STAGE = LOAD_BYTES + GT_BYTES;
   static constexpr int MERGE = (NW + 1) * G * (VD + 2) * 4;  // + the fused step's new row
   static constexpr int NS0 = (225280 - MERGE) / STAGE;
   static constexpr int NS = NS0 > 4 ? 4 : NS0;                     // stages in the ring
@@ -127,7 +132,7 @@ struct DecCfg {
 template <typename T, int KD, int VD, int G, bool PAGED, bool GATE, bool FUSED>
 __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 2) * 32) decode_split_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-    const T* __restrict__ q, const float* __restrict__ p_curr, const float* __restrict__ r_cache,
+    const __grid_constant__ CUtensorMap tmG, int gtma, const T* __restrict__ q, const float* __restrict__ p_curr, const float* __restrict__ r_cache,
     int T_kv, int HQ, int C, int cps, int nsplit, float sc, float* __restrict__ part,
     int* err, uint64_t wait_ns, int fault, const int* __restrict__ seqlens, PageMap pm,
     const float* __restrict__ gs_cache, const float* __restrict__ gs_curr, DecodeFuse fu) {
@@ -187,11 +192,14 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 2) * 32) decode_sp
           const int tb = PAGED ? 0 : b;
           const size_t rslot = PAGED ? pm.chunk(b, row0, C)
                                      : static_cast<size_t>(b) * ncap + row0 / C;
-          mbar_arrive_expect_tx(&full[slot], D::STAGE);
+          const bool gload = GATE && gtma;
+          mbar_arrive_expect_tx(&full[slot], D::LOAD_BYTES + (gload ? D::GT_BYTES : 0));
           tma_load_4d(st, &tmK, &full[slot], 0, h * G, trow, tb);
           tma_load_4d(st + D::K_BYTES, &tmV, &full[slot], 0, h, trow, tb);
           bulk_load(st + D::K_BYTES + D::V_BYTES, r_cache + (rslot * HQ + h * G) * KD,
                     D::R_BYTES, &full[slot]);
+          if (gload)
+            tma_load_3d(st + D::LOAD_BYTES, &tmG, &full[slot], (h * G / D::GB) * D::GB, trow, tb);
         }
         issued = i + 1;
       }
@@ -304,7 +312,8 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 2) * 32) decode_sp
       for (int rr = 0; rr < D::RPW; ++rr)
         dst[rr] = rb + r0 + rr < row_end ? gs_cache[(prow0 + r0 + rr) * HQ + hq] : 0.f;
     };
-    if (GATE && nst > 0) gate_load(0, gnext);
+    if (GATE && !gtma && nst > 0) gate_load(0, gnext);
+    const int gcol = hq - (h * G / D::GB) * D::GB;  // this head's column of a staged gate row
     for (int i = 0; i < nst; ++i) {
       const int slot = i % D::NS;
       const bool got = mbar_wait(&full[slot], (i / D::NS) & 1, wc);
@@ -322,7 +331,11 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 2) * 32) decode_sp
       }
       const int r0 = warp * D::RPW;
       float sres[D::RPW], vv[D::RPW][VPL], gsv[D::RPW];
-      if (GATE) {
+      if (GATE && gtma) {  // staged with the stage's rows by the producer
+        const float* sg = reinterpret_cast<const float*>(st + D::LOAD_BYTES);
+#pragma unroll
+        for (int rr = 0; rr < D::RPW; ++rr) gsv[rr] = sg[(r0 + rr) * D::GB + gcol];
+      } else if (GATE) {
         // (a stage lies in one block of a paged cache, see the producer)
 #pragma unroll
         for (int rr = 0; rr < D::RPW; ++rr) gsv[rr] = gnext[rr];
@@ -503,6 +516,20 @@ cudaError_t decode_impl(const DecodeArgs& a, cudaStream_t st) {
   const bool gate = a.gs_cache != nullptr;
   const bool fused = a.fuse.k_new != nullptr;
   if (gate && fused) return cudaErrorInvalidValue;
+  // scalar-gate rows through the stage ring when a gate-cache row is a whole number
+  // of 16-byte pieces (HQ % 4 == 0); otherwise each lane loads its rows itself
+  CUtensorMap tmG = tmK;
+  int gtma = 0;
+  if (gate && a.HQ % 4 == 0) {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(a.HQ), rows, nb};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(a.HQ) * 4,
+                                   rstride * a.HQ * 4};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(D::GB), static_cast<cuuint32_t>(D::SR), 1};
+    if (!encode_tiled(&tmG, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, a.gs_cache, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+    gtma = 1;
+  }
   auto kern = fused ? (paged ? decode_split_kernel<T, KD, VD, G, true, false, true>
                              : decode_split_kernel<T, KD, VD, G, false, false, true>)
               : paged ? (gate ? decode_split_kernel<T, KD, VD, G, true, true, false>
@@ -515,7 +542,7 @@ cudaError_t decode_impl(const DecodeArgs& a, cudaStream_t st) {
   const int cps = (nchunks + a.nsplit - 1) / a.nsplit;
   dim3 grid(a.nsplit, a.H, a.B);
   kern<<<grid, (D::NW + (fused ? 2 : 1)) * 32, D::SMEM, st>>>(
-      tmK, tmV, static_cast<const T*>(a.q), a.p_curr, a.r_cache, a.T_kv, a.HQ, a.chunk,
+      tmK, tmV, tmG, gtma, static_cast<const T*>(a.q), a.p_curr, a.r_cache, a.T_kv, a.HQ, a.chunk,
       cps, a.nsplit, a.scale * kLog2e, a.part, a.err, a.wait_ns, a.fault, a.seqlens, a.pm,
       a.gs_cache, a.gs_curr, a.fuse);
   e = cudaGetLastError();
