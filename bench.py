@@ -245,6 +245,63 @@ def cpu_baseline(spec, host, budget_s=15.0):
                       f"{dt:.1f} s"}
 
 
+def rows_flops(spec, rows):
+    """Algorithmic FLOPs of the given query rows (batch row 0): admitted keys x 2(K+V) x HQ."""
+    cu = [0]
+    for L in (spec.docs if spec.docs is not None else (spec.T,)):
+        cu.append(cu[-1] + L)
+    total = 0
+    for t in rows:
+        t = int(t)
+        start = max(c for c in cu[:-1] if c <= t)
+        lo = max(start, t - spec.window + 1) if spec.window > 0 else start
+        total += t - lo + 1
+    return float(total * spec.HQ * 2 * (spec.K + spec.V))
+
+
+def cpu_per_config(decode_rows):
+    """The oracle on the host cores for the other workloads (reported baselines only):
+    the tiny and GQA prefills in full, the packed varlen + window prefill on 512 evenly
+    spaced rows, and the decode workload's direct decode oracle (each step = the prefill
+    row of the appended token) for batch rows 0 and 31 over the timed steps."""
+    import numpy as np
+    import oracle
+    threads = oracle.max_threads()
+    out = {}
+    for name, n_rows in (("tiny", None), ("gqa", None), ("varlen_window", 512)):
+        spec = W.PREFILL[name]
+        host = host_inputs(W.gen_prefill(spec, device="cpu"))
+        rows = None if n_rows is None else oracle_sample_rows(spec, n_rows)
+        t0 = time.perf_counter()
+        oracle.wall_fwd(host["q"], host["k"], host["v"], host["g"], host["g_scalar"],
+                        host["sink_bias"], window=spec.window, cu_seqlens=host["cu_seqlens"],
+                        scale=spec.softmax_scale, rows=rows, threads=threads)
+        dt = time.perf_counter() - t0
+        flops = prefill_flops(spec) if rows is None else rows_flops(spec, rows)
+        out[name] = {"value": flops / dt / 1e12, "unit": "TFLOP/s", "seconds": dt,
+                     "sample": ("all rows" if rows is None else
+                                f"{len(rows)} query rows evenly spaced over T={spec.T}, all heads")}
+    if decode_rows is not None:
+        dspec, rows_by_b = decode_rows
+        t0 = time.perf_counter()
+        nbytes = 0
+        for b, (qf, kb, vb, gb, rows) in rows_by_b.items():
+            oracle.wall_fwd(qf, kb, vb, gb, scale=dspec.K ** -0.5, rows=rows, threads=threads)
+            for t in rows:
+                one = replace(dspec, B=1)
+                nbytes += decode_bytes(one, int(t) + 1)
+        dt = time.perf_counter() - t0
+        nb = len(rows_by_b)
+        steps = len(next(iter(rows_by_b.values()))[4])
+        out["decode"] = {
+            "value": nbytes / dt / 1e9, "unit": "GB/s", "seconds": dt,
+            "sample": f"batch rows {sorted(rows_by_b)} of B={dspec.B}, {steps} streaming steps each "
+                      f"(T_kv {dspec.T0 + 1}..{dspec.T0 + steps}), all {dspec.HQ} heads",
+            "extrapolated_ms_per_token_all_batch_rows": 1e3 * dt / steps * dspec.B / nb,
+            "extrapolation": f"per-step time of the {nb} sampled rows x B/{nb} (label: extrapolated)"}
+    return out
+
+
 def host_inputs(d):
     return {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
 
@@ -349,6 +406,17 @@ def run_ours(args, world, rank, local):
         g_steps = [dd["g"][:, T0 + s:T0 + s + 1].contiguous() for s in range(S)]
         q_steps = [dd["q"][:, s:s + 1].contiguous() for s in range(S)]
         v_steps = [dd["v"][:, T0 + s:T0 + s + 1].contiguous() for s in range(S)]
+        decode_rows = None
+        if world == 1 and not args.no_cpu_baseline:
+            import numpy as np
+            rows_by_b = {}
+            for b_ in sorted({0, dspec.B - 1}):
+                qf = torch.zeros((1, T0 + S, dspec.HQ, dspec.K), dtype=torch.bfloat16)
+                qf[0, T0:T0 + S] = dd["q"][b_].cpu()
+                rows_by_b[b_] = (qf, dd["k"][b_:b_ + 1].cpu(), dd["v"][b_:b_ + 1].cpu(),
+                                 dd["g"][b_:b_ + 1].cpu(),
+                                 np.arange(T0, T0 + S, dtype=np.int64))
+            decode_rows = (dspec, rows_by_b)
         del dd
         dout = torch.empty((dspec.B, 1, dspec.HQ, dspec.V), dtype=torch.bfloat16, device=dev)
         dlse = torch.empty((dspec.B, 1, dspec.HQ), dtype=torch.float32, device=dev)
@@ -478,6 +546,47 @@ def run_ours(args, world, rank, local):
                      "prefill_alone_main_TFLOPs": flops / (alone_main * 1e-3) / 1e12,
                      "prefill_alone_main_frac_of_burst_peak":
                          flops / (alone_main * 1e-3) / 1e12 / bf16_peak})
+        # secondary bound of the attention kernel: one exponential per admitted score on
+        # the MUFU, 16 per clock per SM (at the maximum SM clock)
+        n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+        mufu_peak = 16.0 * n_sm * peaks.get("sm_max_mhz", 1965.0) * 1e6
+        exps = float(pspec.B * pspec.HQ * prefill_pairs(pspec))
+        side["mufu"] = {"exps_per_launch": exps, "achieved_per_s": exps / (alone_main * 1e-3),
+                        "peak_per_s": mufu_peak,
+                        "frac": exps / (alone_main * 1e-3) / mufu_peak,
+                        "note": "kernel timed alone; 16 MUFU ops per clock per SM x SMs x max clock"}
+        # the other prefill workloads (GQA; packed varlen + window + sink), timed alone
+        for name in ("gqa", "varlen_window"):
+            ospec = W.PREFILL[name]
+            od = W.gen_prefill(ospec, device=dev)
+            oo = torch.empty((ospec.B, ospec.T, ospec.HQ, ospec.V), dtype=torch.bfloat16, device=dev)
+            ol = torch.empty((ospec.B, ospec.T, ospec.HQ), dtype=torch.float32, device=dev)
+            ows = torch.empty(wall.wall_attn_fwd_workspace_size(ospec.B, ospec.T, ospec.HQ, ospec.H,
+                                                                ospec.K, ospec.V, torch.bfloat16),
+                              dtype=torch.uint8, device=dev)
+
+            def run_other():
+                wall.wall_attn_fwd(od["q"], od["k"], od["v"], od["g"], od["g_scalar"], od["sink_bias"],
+                                   window=od["window"], cu_seqlens=od["cu_seqlens"],
+                                   scale=od["scale"], out=oo, lse=ol, workspace=ows,
+                                   return_lse=True)
+            run_other()
+            oev = [[ev() for _ in range(3)] for _ in range(args.steps)]
+            for trio in oev:
+                for e in trio:
+                    e.record()
+            for i in range(args.steps):
+                wall.wall_debug_set_stage_events(*oev[i])
+                run_other()
+                wall.wall_debug_set_stage_events()
+            torch.cuda.synchronize()
+            om = statistics.mean(e[1].elapsed_time(e[2]) for e in oev)
+            oa = statistics.mean(e[0].elapsed_time(e[2]) for e in oev)
+            of = prefill_flops(ospec)
+            side.update({f"prefill_{name}_ms": oa, f"prefill_{name}_main_ms": om,
+                         f"prefill_{name}_main_TFLOPs": of / (om * 1e-3) / 1e12,
+                         f"prefill_{name}_main_frac_of_burst_peak": of / (om * 1e-3) / 1e12 / bf16_peak})
+            del od, oo, ol, ows
         # prefill that also emits its decode cache, against prefill + a separate build
         pc = wall.KVCache(B, T, HQ, H, K, V, dtype=torch.bfloat16, chunk=64, device=dev)
 
@@ -801,14 +910,16 @@ def run_ours(args, world, rank, local):
         e2e_ms = reduce_max(a.elapsed_time(b_), world, dev)
         line["e2e"] = {"value": weak_scaling_rate(prefill_flops(pspec), args.steps, world, e2e_ms) / 1e12,
                        "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-    # per timed step: prefill = prepass (2) + attention (1); each decode token = the fused
-    # decode split (append inside) + the combine (2)
-    line["gpu_launches"] = args.steps * ((3 if do_prefill else 0) + (2 * S if do_decode else 0))
+    # per timed step: prefill = prepass (2) + attention (1) + the wide-block pass (1, which
+    # exits at once on these inputs); each decode token = the fused decode split (append
+    # inside) + the combine (2)
+    line["gpu_launches"] = args.steps * ((4 if do_prefill else 0) + (2 * S if do_decode else 0))
     line["clocks"] = clk
     if rank != 0:
         return 0
     if world == 1 and do_prefill and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(pspec, host_inputs(pd))
+        line["cpu_baseline"]["per_config"] = cpu_per_config(decode_rows if do_decode else None)
     print(json.dumps(line), flush=True)
     return 0
 

@@ -716,6 +716,7 @@ wall_status_t wall_attn_chunk(const void* q, const void* k_new, const void* g_ne
   a.B = B; a.t0 = t_start; a.M = M; a.cap = cap; a.HQ = HQ; a.H = H; a.K = K; a.V = V;
   a.chunk = chunk; a.scale = scale; a.k_tilde = k_tilde; a.r_cache = r_cache; a.p_last = p_last;
   a.v_cache = v_cache; a.o = o; a.lse = lse; a.workspace = workspace;
+  a.fault = wall::fault_mode();
   a.err = wall::device_error_word();
   if (a.err == nullptr) return WALL_ERR_CUDA;
   a.wait_ns = wall::wait_limit_ns();

@@ -110,7 +110,7 @@ __global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_s
     const __nv_bfloat16* __restrict__ qh, const float* __restrict__ AQ,
     const float* __restrict__ r_cache, int t0, int M, int HQ, int C, int cap, int window,
     int ck_lo, int cps, int nsplit, int ntg, float sc, float* __restrict__ part, int* err,
-    uint64_t wait_ns, const int* __restrict__ wide) {
+    uint64_t wait_ns, const int* __restrict__ wide, int fault) {
   using D = MultiCfg<KD, VD, G>;
   constexpr int MQ = D::MQ, LPH = D::LPH, CPL = D::CPL, VPL = D::VPL, RB = D::RB, NV = D::NV;
   constexpr int NO = D::NO, REP = D::REP, MG = MQ * G;
@@ -173,16 +173,18 @@ __global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_s
         if (i >= D::NS && !mbar_wait(&empty[slot], ((i / D::NS) - 1) & 1, wc)) break;
         const int row0 = row_begin + i * D::SR;
         uint8_t* st = dsm + slot * D::STAGE;
-        mbar_arrive_expect_tx(&full[slot], D::STAGE);
-        tma_load_4d(st, &tmK, &full[slot], 0, h * G, row0, b);
-        tma_load_4d(st + D::K_BYTES, &tmV, &full[slot], 0, h, row0, b);
-        bulk_load(st + D::K_BYTES + D::V_BYTES,
-                  r_cache + ((static_cast<size_t>(b) * ncap + row0 / C) * HQ + h * G) * KD,
-                  D::R_BYTES, &full[slot]);
+        if (!(fault == 7 && i == 0)) {  // testing hook: starve the consumers
+          mbar_arrive_expect_tx(&full[slot], D::STAGE);
+          tma_load_4d(st, &tmK, &full[slot], 0, h * G, row0, b);
+          tma_load_4d(st + D::K_BYTES, &tmV, &full[slot], 0, h, row0, b);
+          bulk_load(st + D::K_BYTES + D::V_BYTES,
+                    r_cache + ((static_cast<size_t>(b) * ncap + row0 / C) * HQ + h * G) * KD,
+                    D::R_BYTES, &full[slot]);
+        }
         issued = i + 1;
       }
       for (int i = issued > D::NS ? issued - D::NS : 0; i < issued; ++i)
-        mbar_drain(&full[i % D::NS], (i / D::NS) & 1, wait_ns);
+        if (!(fault == 7 && i == 0)) mbar_drain(&full[i % D::NS], (i / D::NS) & 1, wait_ns);
     }
   }
   float mrun = -INFINITY, lpart = 0.f;  // the owned token's running max, partial sum
@@ -411,7 +413,8 @@ cudaError_t chunk_split_impl(const ChunkArgs& a, const void* qh, const float* AQ
   if (a.ev_mid != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(a.ev_mid), st);
   kern<<<grid, (D::NW + 1) * 32, D::SMEM, st>>>(
       tmK, tmV, static_cast<const __nv_bfloat16*>(qh), AQ, a.r_cache, a.t0, a.M, a.HQ, a.chunk,
-      a.cap, a.window, ck_lo, cps, nsplit, ntg, a.scale * kLog2e, part, a.err, a.wait_ns, wide);
+      a.cap, a.window, ck_lo, cps, nsplit, ntg, a.scale * kLog2e, part, a.err, a.wait_ns, wide,
+      a.fault);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_decode_combine_bf16(part, nsplit, a.B * a.M * a.HQ, a.HQ, a.sink, a.o, lse, VD,

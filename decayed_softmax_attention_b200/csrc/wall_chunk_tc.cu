@@ -31,6 +31,7 @@ struct ChunkParams {
   float* lse;        // [B, M, HQ]
   int* err;
   uint64_t wait_ns;
+  int fault;  // testing hook: 6 = the producer skips its first key tile
 };
 
 template <int KD, int VD, int CH>
@@ -218,17 +219,19 @@ __global__ void __launch_bounds__(512, 1)
         const int kt = kt_hi - j;
         const int ks = j % C::KS;
         if (j >= C::KS && !mbar_wait(&kempty[ks], ((j / C::KS) - 1) & 1, wc)) break;
-        mbar_arrive_expect_tx(&kfull[ks], C::K_BYTES + C::NRC * KD * 4);
-        for (int bx = 0; bx < C::QBOX; ++bx)
-          tma_load_4d(sK + ks * C::K_BYTES + bx * 16384, &tmK, &kfull[ks], bx * 64, hq,
-                      kt * C::BN, b);
-        for (int c = 0; c < C::NRC; ++c) {
-          // anchors of the tile's chunks; a chunk past the last row in use (its rows
-          // arrive as zeros and are masked) reads that row's anchor instead
-          const int ck = min(kt * C::NRC + c, last_chunk);
-          bulk_load(sR + (ks * C::NRC + c) * KD,
-                    p.r_cache + ((static_cast<size_t>(b) * ncap + ck) * p.HQ + hq) * KD, KD * 4,
-                    &kfull[ks]);
+        if (!(p.fault == 6 && j == 0)) {  // testing hook: starve the consumers
+          mbar_arrive_expect_tx(&kfull[ks], C::K_BYTES + C::NRC * KD * 4);
+          for (int bx = 0; bx < C::QBOX; ++bx)
+            tma_load_4d(sK + ks * C::K_BYTES + bx * 16384, &tmK, &kfull[ks], bx * 64, hq,
+                        kt * C::BN, b);
+          for (int c = 0; c < C::NRC; ++c) {
+            // anchors of the tile's chunks; a chunk past the last row in use (its rows
+            // arrive as zeros and are masked) reads that row's anchor instead
+            const int ck = min(kt * C::NRC + c, last_chunk);
+            bulk_load(sR + (ks * C::NRC + c) * KD,
+                      p.r_cache + ((static_cast<size_t>(b) * ncap + ck) * p.HQ + hq) * KD,
+                      KD * 4, &kfull[ks]);
+          }
         }
         nk = j + 1;
         const int vs = j % C::VS;
@@ -241,7 +244,7 @@ __global__ void __launch_bounds__(512, 1)
       }
       mbar_drain(qfull, 0, p.wait_ns);
       for (int j = nk > C::KS ? nk - C::KS : 0; j < nk; ++j)
-        mbar_drain(&kfull[j % C::KS], (j / C::KS) & 1, p.wait_ns);
+        if (!(p.fault == 6 && j == 0)) mbar_drain(&kfull[j % C::KS], (j / C::KS) & 1, p.wait_ns);
       for (int j = nv > C::VS ? nv - C::VS : 0; j < nv; ++j)
         mbar_drain(&vfull[j % C::VS], (j / C::VS) & 1, p.wait_ns);
     } else if (warp == 1 && lane == 0) {
@@ -669,6 +672,7 @@ cudaError_t chunk_impl(const ChunkArgs& a, void* qh, float* AQ, const int* wide,
   p.lse = lse;
   p.err = a.err;
   p.wait_ns = a.wait_ns;
+  p.fault = a.fault;
   const unsigned grid = static_cast<unsigned>(NQB) * BHQ;
   if (a.ev_mid != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(a.ev_mid), st);
   kern<<<grid, 512, C::SMEM_ALLOC, st>>>(tmQ, tmK, tmV, p);

@@ -242,6 +242,7 @@ struct ChunkArgs {
   int* err;
   uint64_t wait_ns;
   void* ev_mid = nullptr;  // optional event recorded before the attention kernel
+  int fault = 0;           // testing hook: 6 = chunk tile kernel, 7 = few-token split kernel
 };
 size_t chunk_workspace_bytes(int B, int M, int cap, int HQ, int H, int K, int V, int chunk);
 cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t st);

@@ -451,7 +451,9 @@ wall_status_t wall_device_error(wall_stream_t stream);
  *   mode 1: prefill attention (first K/V tile), mode 2: decode split (first
  *   k_tilde/v stage), mode 3: cache build (first g/k stage), mode 4: backward
  *   key-block kernel (first query tile), mode 5: backward query-block kernel
- *   (first key tile; bf16 only).
+ *   (first key tile; bf16 only), mode 6: wall_attn_chunk's tensor-core tile
+ *   kernel (first cache key tile), mode 7: wall_attn_chunk's few-token split
+ *   kernel (first k_tilde/v stage).
  * Outputs of the starved call are unspecified.  mode 0 restores normal
  * operation.  wait_ms <= 0 keeps the default limit (2000 ms).
  */

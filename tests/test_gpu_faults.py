@@ -2,7 +2,8 @@
 
 `wall_debug_set_fault(mode, ms)` makes one kernel's producer skip its first
 load (1: prefill attention, 2: decode split, 3: cache build, 4 / 5: the
-backward's key-block / query-block kernels), so the
+backward's key-block / query-block kernels, 6 / 7: the chunk path's tile and
+few-token split kernels), so the
 consumers' waits run out after `ms` milliseconds.  The kernel must then
 wind down on its own (drain its copies, free tensor memory), report
 WALL_ERR_DEVICE_TIMEOUT through the device error word, and leave the context
@@ -128,3 +129,36 @@ def test_backward_starved_consumers_time_out_and_recover(mode):
     for name in ("dq", "dk", "dv", "dg", "dg_scalar"):
         assert_grad_close(got[name], ref[name], ref["sigma"][name], ref["sigma_abs"][name],
                           torch.bfloat16, f"{name} after recovery")
+
+
+@pytest.mark.parametrize("mode,M", [(6, 300), (7, 4)], ids=["chunk_tile", "chunk_split"])
+def test_chunk_starved_consumers_time_out_and_recover(mode, M):
+    """Modes 6 / 7: the chunk path's tensor-core tile kernel (a 300-token chunk) or its
+    few-token split kernel (4 tokens) loses its first load; the call reports
+    WALL_ERR_DEVICE_TIMEOUT and the same chunk, called again, matches the oracle."""
+    import decayed_softmax_attention_b200 as wall
+    B, T0, HQ, H, K, V, C = 2, 200, 8, 2, 128, 128, 64
+    T = T0 + M
+    spec = W.PrefillSpec("fault_chunk", B=B, T=T, HQ=HQ, H=H, K=K, V=V, dtype="bf16",
+                         g_kind="negsoftplus", seed=9)
+    d = W.gen_prefill(spec, device="cuda")
+    cache = wall.KVCache(B, T, HQ, H, K, V, dtype=torch.bfloat16, chunk=C)
+    cache.append(d["k"][:, :T0].contiguous(), d["g"][:, :T0].contiguous(),
+                 d["v"][:, :T0].contiguous())
+    cache.v[:, T0:T].copy_(d["v"][:, T0:T])
+    p_prev = cache.p.clone()
+    sl = slice(T0, T)
+    args = [d["q"][:, sl].contiguous(), d["k"][:, sl].contiguous(), d["g"][:, sl].contiguous(),
+            cache.k_tilde, cache.r_cache, cache.p, cache.v, T0]
+    assert wall.wall_device_error() == 0
+    wall.wall_debug_set_fault(mode, 100)
+    try:
+        wall.wall_attn_chunk(*args, p_prev=p_prev, scale=d["scale"], chunk=C)
+        status = wall.wall_device_error()
+    finally:
+        wall.wall_debug_set_fault(0, 0)
+    assert status == WALL_ERR_DEVICE_TIMEOUT
+    o = wall.wall_attn_chunk(*args, p_prev=p_prev, scale=d["scale"], chunk=C)
+    assert wall.wall_device_error() == 0
+    ro, _ = oracle.wall_fwd(d["q"], d["k"], d["v"], d["g"], scale=d["scale"])
+    assert_close(o, ro[:, sl], torch.bfloat16, f"chunk after recovery (mode {mode})")
