@@ -168,6 +168,8 @@ __global__ void __launch_bounds__(512, 1)
   const int b = bh / p.HQ, hq = bh % p.HQ, kvh = hq / (p.HQ / p.H);
   const int q0 = qblk * 2 * C::BM;
   const bool has_b = q0 + C::BM < p.T;
+  // issued first: the load's latency hides behind the set-up below
+  const int wide_flag = __ldg(p.wide + static_cast<size_t>(bh) * NQB + qblk);
 
   if (tid == 0) {
     mbar_init(qfull, 1);
@@ -226,7 +228,7 @@ __global__ void __launch_bounds__(512, 1)
   const uint32_t tmem_base = *tmem_slot;
   // key-tile ranges (tile index kt = key row / 128) of query tiles A and B; a
   // wide block (strong decay inside it) stops before its own two key tiles
-  const bool wide = p.wide[static_cast<size_t>(bh) * NQB + qblk] != 0;
+  const bool wide = wide_flag != 0;
   const int ktA_hi = wide ? 2 * qblk - 1 : 2 * qblk, ktB_hi = wide ? 2 * qblk - 1 : 2 * qblk + 1;
   const int ktA_lo = sched_lo[0] / C::BN;
   const int ktB_lo = has_b ? sched_lo[1] / C::BN : ktB_hi + 1;

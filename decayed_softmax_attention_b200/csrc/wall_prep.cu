@@ -167,8 +167,10 @@ __global__ void __launch_bounds__(256, 3) prep_local_kernel(
   }
 
   if (kt != nullptr && kspan * kLog2e > kCacheRangeLog2) atomicOr(err, kDevErrRange);
-  // Non-negative floats order like their bit patterns.
-  if (span > 0.f) atomicMax(&s_span, __float_as_int(span));
+  // Non-negative floats order like their bit patterns; one shared atomic per warp.
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) span = fmaxf(span, __shfl_xor_sync(0xffffffffu, span, off));
+  if ((threadIdx.x & 31) == 0 && span > 0.f) atomicMax(&s_span, __float_as_int(span));
   __syncthreads();
   if (threadIdx.x == 0) {
     const int w = __int_as_float(s_span) > kPrefillSpanNats ? 1 : 0;
