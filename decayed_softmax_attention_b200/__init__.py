@@ -57,6 +57,7 @@ EXPORTED_SYMBOLS = (
     "wall_build_kv_cache_paged", "wall_append_kv_cache_paged", "wall_attn_decode_paged",
     "wall_build_gate_cache", "wall_append_gate_cache", "wall_attn_decode_gated",
     "wall_attn_chunk_workspace_size", "wall_attn_chunk", "wall_attn_decode_step",
+    "wall_attn_decode_step_gated",
 )
 
 
@@ -112,6 +113,9 @@ def load_library():
     lib.wall_attn_decode_step.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I,
                                           I, I, F, P, P, P, P, P, P, S, P]
     lib.wall_attn_decode_step.restype = I
+    lib.wall_attn_decode_step_gated.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, I, I, I, I,
+                                                I, I, I, I, I, I, I, I, F, P, P, P, P, P, P, S, P]
+    lib.wall_attn_decode_step_gated.restype = I
     lib.wall_build_gate_cache.argtypes = [P, P, P, I, I, I, I, I, I, I, I, I, P, P, P]
     lib.wall_build_gate_cache.restype = I
     lib.wall_append_gate_cache.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P, P, P]
@@ -513,6 +517,61 @@ def wall_attn_decode_step(q, k_new, g_new, v_new, k_tilde, r_cache, v_cache, p_p
     return out
 
 
+def wall_attn_decode_step_gated(q, k_new, g_new, v_new, gs_new, k_tilde, r_cache, v_cache, p_prev,
+                                p_last, gs_cache, gs_prev, gs_last, T_kv=None, seqlens=None,
+                                block_table=None, sink_bias=None, scale=None, chunk=64, out=None,
+                                lse=None, workspace=None):
+    """wall_attn_decode_step with the scalar gate: gs_new [B,1,HQ] is the new token's g_scalar;
+    gs_prev / gs_last [B,HQ] fp32 are PS at the previous / new row (different buffers); the
+    gate cache row of the new token is written.  Other arguments as wall_attn_decode_step."""
+    lib = load_library()
+    B, _, HQ, K = q.shape
+    H, V = k_new.shape[2], v_new.shape[3]
+    dt = k_tilde.dtype
+    if block_table is None:
+        cap = k_tilde.shape[1]
+        maxblk = nblk = bs = 0
+        rows = cap
+        if T_kv is None:
+            raise ValueError("dense caches need T_kv")
+        r_shape = (B, (cap + chunk - 1) // chunk, HQ, K)
+        kv_shape, v_shape, g_shape = (B, cap, HQ, K), (B, cap, H, V), (B, cap, HQ)
+    else:
+        nblk, bs = k_tilde.shape[0], k_tilde.shape[1]
+        maxblk = block_table.shape[1]
+        cap = rows = maxblk * bs
+        if seqlens is None:
+            raise ValueError("paged caches need seqlens")
+        T_kv = rows if T_kv is None else T_kv
+        r_shape = (nblk, bs // chunk, HQ, K)
+        kv_shape, v_shape, g_shape = (nblk, bs, HQ, K), (nblk, bs, H, V), (nblk, bs, HQ)
+    if out is None:
+        out = torch.empty((B, 1, HQ, V), dtype=dt, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(wall_attn_decode_workspace_size(B, rows if block_table is not None
+                                                                    else T_kv, HQ, H, V, chunk), 1),
+                                dtype=torch.uint8, device=q.device)
+    st = lib.wall_attn_decode_step_gated(
+        _dev(q, "q", dt, (B, 1, HQ, K)), _dev(k_new, "k_new", dt, (B, 1, H, K)),
+        _dev(g_new, "g_new", dt, (B, 1, HQ, K)), _dev(v_new, "v_new", dt, (B, 1, H, V)),
+        _dev(gs_new, "gs_new", dt, (B, 1, HQ)),
+        _dev(p_prev, "p_prev", torch.float32, (B, HQ, K)),
+        _dev(p_last, "p_last", torch.float32, (B, HQ, K)),
+        _dev(gs_prev, "gs_prev", torch.float32, (B, HQ)),
+        _dev(gs_last, "gs_last", torch.float32, (B, HQ)),
+        _dev(gs_cache, "gs_cache", torch.float32, g_shape),
+        _dev(sink_bias, "sink_bias", torch.float32, (HQ,)),
+        _dev(seqlens, "seqlens", torch.int32, (B,)),
+        _dev(block_table, "block_table", torch.int32), maxblk, nblk, bs, B, int(T_kv), cap, HQ, H,
+        K, V, int(chunk), _dtype_code(k_tilde), float(scale) if scale else 0.0,
+        _dev(k_tilde, "k_tilde", dt, kv_shape), _dev(r_cache, "r_cache", torch.float32, r_shape),
+        _dev(v_cache, "v_cache", dt, v_shape), _dev(out, "out", dt, (B, 1, HQ, V)),
+        _dev(lse, "lse", torch.float32), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(q.device))
+    _check(st, "wall_attn_decode_step_gated")
+    return out
+
+
 # ----------------------------------------------------------------- scalar gate in decode
 def _gate_table(gs_cache, block_table):
     """(block_table, max_blocks, num_blocks, block_size, cap) for a dense or paged gate cache."""
@@ -678,6 +737,7 @@ class KVCache:
         # scalar gate (models with g_scalar): PS per row and head, and PS at the last row
         self.gs_cache = torch.empty((B, cap, HQ), dtype=torch.float32, device=device) if gate else None
         self.gs = torch.zeros((B, HQ), dtype=torch.float32, device=device) if gate else None
+        self._gs_next = torch.zeros_like(self.gs) if gate else None  # PS out of a fused step
         nc = (cap + chunk - 1) // chunk
         self.k_tilde = torch.empty((B, cap, HQ, K), dtype=dtype, device=device)
         self.r_cache = torch.empty((B, nc, HQ, K), dtype=torch.float32, device=device)
@@ -713,18 +773,29 @@ class KVCache:
                                 sink_bias=sink_bias, scale=scale, chunk=self.chunk, out=out,
                                 lse=lse, workspace=self.workspace)
 
-    def step(self, q, k_new, g_new, v_new, sink_bias=None, scale=None, out=None, lse=None):
-        """append(k_new, g_new, v_new) then decode(q), fused into the decode's launches.
+    def step(self, q, k_new, g_new, v_new, sink_bias=None, scale=None, out=None, lse=None,
+             gs_new=None):
+        """append(k_new, g_new, v_new) then decode(q), fused into the decode's launches
+        (with the scalar gate, gs_new [B,1,HQ] joins the gate cache the same way).
 
-        The kernel reads P from one buffer and writes the new P to another, so after the
-        call ``self.p`` is the other tensor: read ``cache.p`` afresh, do not keep a reference.
+        The kernel reads P (and PS) from one buffer and writes the new value to another, so
+        after the call ``self.p`` / ``self.gs`` are the other tensors: read them afresh.
         """
         if self.gs_cache is not None:
-            raise ValueError("the fused step carries no scalar gate: use append + decode")
-        o = wall_attn_decode_step(q, k_new, g_new, v_new, self.k_tilde, self.r_cache, self.v,
-                                  self.p, self._p_next, T_kv=self.length + 1, sink_bias=sink_bias,
-                                  scale=scale, chunk=self.chunk, out=out, lse=lse,
-                                  workspace=self.workspace)
+            if gs_new is None:
+                raise ValueError("this cache carries the scalar gate: pass gs_new")
+            o = wall_attn_decode_step_gated(q, k_new, g_new, v_new, gs_new, self.k_tilde,
+                                            self.r_cache, self.v, self.p, self._p_next,
+                                            self.gs_cache, self.gs, self._gs_next,
+                                            T_kv=self.length + 1, sink_bias=sink_bias,
+                                            scale=scale, chunk=self.chunk, out=out, lse=lse,
+                                            workspace=self.workspace)
+            self.gs, self._gs_next = self._gs_next, self.gs
+        else:
+            o = wall_attn_decode_step(q, k_new, g_new, v_new, self.k_tilde, self.r_cache, self.v,
+                                      self.p, self._p_next, T_kv=self.length + 1,
+                                      sink_bias=sink_bias, scale=scale, chunk=self.chunk, out=out,
+                                      lse=lse, workspace=self.workspace)
         self.p, self._p_next = self._p_next, self.p
         self.length += 1
         return o
@@ -754,6 +825,7 @@ class PagedKVCache:
         self.gs_cache = (torch.empty((num_blocks, block_size, HQ), dtype=torch.float32,
                                      device=device) if gate else None)
         self.gs = torch.zeros((B, HQ), dtype=torch.float32, device=device) if gate else None
+        self._gs_next = torch.zeros_like(self.gs) if gate else None  # PS out of a fused step
         self.free = list(range(num_blocks))
         self.host_table = [[] for _ in range(B)]
         self.block_table = torch.zeros((B, max_blocks), dtype=torch.int32, device=device)
@@ -841,19 +913,30 @@ class PagedKVCache:
                                       seqlens, self.block_table, sink_bias=sink_bias, scale=scale,
                                       chunk=self.chunk, out=out, lse=lse, workspace=self.workspace)
 
-    def step(self, q, k_new, g_new, v_new, t_pos, sink_bias=None, scale=None, out=None, lse=None):
+    def step(self, q, k_new, g_new, v_new, t_pos, sink_bias=None, scale=None, out=None, lse=None,
+             gs_new=None):
         """append(k_new, g_new, v_new, t_pos) then decode(q), fused into the decode's launches;
         t_pos (host list) = each row's current length, where its new token goes.  As for
-        KVCache.step, ``self.p`` is a different tensor after the call."""
-        if self.gs_cache is not None:
-            raise ValueError("the fused step carries no scalar gate: use append + decode")
+        KVCache.step, ``self.p`` (and ``self.gs``) are different tensors after the call."""
         for b, t in enumerate(t_pos):
             self.reserve(b, t + 1)
         seqlens = torch.tensor([t + 1 for t in t_pos], dtype=torch.int32, device=q.device)
-        o = wall_attn_decode_step(q, k_new, g_new, v_new, self.k_tilde, self.r_cache, self.v,
-                                  self.p, self._p_next, seqlens=seqlens,
-                                  block_table=self.block_table, sink_bias=sink_bias, scale=scale,
-                                  chunk=self.chunk, out=out, lse=lse, workspace=self.workspace)
+        if self.gs_cache is not None:
+            if gs_new is None:
+                raise ValueError("this cache carries the scalar gate: pass gs_new")
+            o = wall_attn_decode_step_gated(q, k_new, g_new, v_new, gs_new, self.k_tilde,
+                                            self.r_cache, self.v, self.p, self._p_next,
+                                            self.gs_cache, self.gs, self._gs_next,
+                                            seqlens=seqlens, block_table=self.block_table,
+                                            sink_bias=sink_bias, scale=scale, chunk=self.chunk,
+                                            out=out, lse=lse, workspace=self.workspace)
+            self.gs, self._gs_next = self._gs_next, self.gs
+        else:
+            o = wall_attn_decode_step(q, k_new, g_new, v_new, self.k_tilde, self.r_cache, self.v,
+                                      self.p, self._p_next, seqlens=seqlens,
+                                      block_table=self.block_table, sink_bias=sink_bias,
+                                      scale=scale, chunk=self.chunk, out=out, lse=lse,
+                                      workspace=self.workspace)
         self.p, self._p_next = self._p_next, self.p
         for b, t in enumerate(t_pos):
             self.lengths[b] = t + 1

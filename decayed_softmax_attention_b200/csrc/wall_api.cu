@@ -483,7 +483,15 @@ static wall_status_t decode_entry(const void* q, const float* p_curr, const void
     const char* a0 = reinterpret_cast<const char*>(p_curr);
     const char* a1 = reinterpret_cast<const char*>(fu->p_last);
     if (a0 < a1 + pb && a1 < a0 + pb) return WALL_ERR_INVALID_ARG;
-    if (gs_cache != nullptr) return WALL_ERR_UNSUPPORTED;
+    if (gs_cache != nullptr) {  // gated step: the new token's g_scalar, PS in and out
+      if (!fu->gs_new || !fu->gs_last || (T_kv > 1 && !fu->gs_prev) || !aligned(fu->gs_last, 4) ||
+          (fu->gs_prev && !aligned(fu->gs_prev, 4)))
+        return WALL_ERR_INVALID_ARG;
+      const size_t gb = static_cast<size_t>(B) * HQ * sizeof(float);
+      const char* g0 = reinterpret_cast<const char*>(fu->gs_prev);
+      const char* g1 = reinterpret_cast<const char*>(fu->gs_last);
+      if (g0 != nullptr && g0 < g1 + gb && g1 < g0 + gb) return WALL_ERR_INVALID_ARG;
+    }
   }
   const int ns = wall::decode_num_splits(B, T_kv, HQ, H, chunk);
   if (workspace_bytes < wall::decode_workspace_bytes(B, HQ, V, ns)) return WALL_ERR_WORKSPACE;
@@ -575,6 +583,34 @@ wall_status_t wall_attn_decode_step(const void* q, const void* k_new, const void
   return decode_entry(q, p_prev, v_cache, k_tilde, r_cache, sink_bias, seqlens_kv, B,
                       T_kv < rows ? T_kv : rows, rows, HQ, H, K, V, chunk, dt, scale, o, lse,
                       workspace, workspace_bytes, stream, &pm, nullptr, nullptr, &fu);
+}
+
+wall_status_t wall_attn_decode_step_gated(
+    const void* q, const void* k_new, const void* g_new, const void* v_new, const void* gs_new,
+    const float* p_prev, float* p_last, const float* gs_prev, float* gs_last, float* gs_cache,
+    const float* sink_bias, const int32_t* seqlens_kv, const int32_t* block_table, int max_blocks,
+    int num_blocks, int block_size, int B, int T_kv, int cap, int HQ, int H, int K, int V,
+    int chunk, wall_dtype_t dt, float scale, void* k_tilde, float* r_cache, void* v_cache,
+    void* o, float* lse, void* workspace, size_t workspace_bytes, wall_stream_t stream) {
+  if (B > 0 && (gs_cache == nullptr || gs_new == nullptr || !aligned(gs_cache, 4)))
+    return WALL_ERR_INVALID_ARG;
+  wall::DecodeFuse fu;
+  fu.k_new = k_new; fu.g_new = g_new; fu.v_new = v_new; fu.p_last = p_last;
+  fu.k_tilde = k_tilde; fu.r_cache = r_cache; fu.v = v_cache;
+  fu.gs_new = gs_new; fu.gs_prev = gs_prev; fu.gs_last = gs_last;
+  if (block_table == nullptr)
+    return decode_entry(q, p_prev, v_cache, k_tilde, r_cache, sink_bias, seqlens_kv, B, T_kv, cap,
+                        HQ, H, K, V, chunk, dt, scale, o, lse, workspace, workspace_bytes, stream,
+                        nullptr, gs_cache, nullptr, &fu);
+  if (B > 0 && seqlens_kv == nullptr) return WALL_ERR_INVALID_ARG;
+  wall::PageMap pm;
+  const wall_status_t ps = page_map(block_table, max_blocks, num_blocks, block_size, chunk, B, &pm);
+  if (ps != WALL_OK) return ps;
+  const int rows = max_blocks * block_size;
+  (void)cap;
+  return decode_entry(q, p_prev, v_cache, k_tilde, r_cache, sink_bias, seqlens_kv, B,
+                      T_kv < rows ? T_kv : rows, rows, HQ, H, K, V, chunk, dt, scale, o, lse,
+                      workspace, workspace_bytes, stream, &pm, gs_cache, nullptr, &fu);
 }
 
 // Gate cache entries: dense when block_table is NULL (gs_cache [B, cap, HQ]),

@@ -136,7 +136,6 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 2) * 32) decode_sp
     int T_kv, int HQ, int C, int cps, int nsplit, float sc, float* __restrict__ part,
     int* err, uint64_t wait_ns, int fault, const int* __restrict__ seqlens, PageMap pm,
     const float* __restrict__ gs_cache, const float* __restrict__ gs_curr, DecodeFuse fu) {
-  static_assert(!(GATE && FUSED), "the fused append carries no scalar gate");
   using D = DecCfg<T, KD, VD, G>;
   constexpr int LPH = 32 / G;    // lanes per query head
   constexpr int CPL = KD / LPH;  // k_tilde channels per lane
@@ -284,6 +283,13 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 2) * 32) decode_sp
 #pragma unroll
         for (int c = 0; c < VPL; ++c) vn[c] = as_stored(vw, vn[c]);
         store_n<T, VPL>(vw, vn);
+        if (GATE && lane % LPH == 0) {  // the new row's gate prefix PS (its own term is 0)
+          const size_t gi = static_cast<size_t>(b) * HQ + hq;
+          const float ps = fmaf(load1(static_cast<const T*>(fu.gs_new) + gi), kLog2e,
+                                t_new > 0 ? fu.gs_prev[gi] : 0.f);
+          const_cast<float*>(gs_cache)[prow * HQ + hq] = ps;
+          fu.gs_last[gi] = ps;
+        }
       }
       if (lane % LPH == 0) {
         sm_ml[(D::NW * G + hl) * 2] = d;
@@ -295,7 +301,15 @@ __global__ void __launch_bounds__((DecCfg<T, KD, VD, G>::NW + 2) * 32) decode_sp
         for (int c = 0; c < VPL; ++c) sm_o[(D::NW * G + hh) * VD + lane * VPL + c] = vn[c];
     } else {
     // scalar gate: the logit gains PS(current row) - PS(row j), exp2 units
-    const float gcur = GATE ? gs_curr[static_cast<size_t>(b) * HQ + hq] : 0.f;
+    // (fused: PS of the new row, from the previous row's PS and the token's g_scalar)
+    float gcur = 0.f;
+    if (GATE && FUSED) {
+      const size_t i = static_cast<size_t>(b) * HQ + hq;
+      gcur = fmaf(load1(static_cast<const T*>(fu.gs_new) + i), kLog2e,
+                  t_new > 0 ? fu.gs_prev[i] : 0.f);
+    } else if (GATE) {
+      gcur = gs_curr[static_cast<size_t>(b) * HQ + hq];
+    }
     float m = -INFINITY, l = 0.f;
     float o[G][VPL];
 #pragma unroll
@@ -515,7 +529,7 @@ cudaError_t decode_impl(const DecodeArgs& a, cudaStream_t st) {
   }
   const bool gate = a.gs_cache != nullptr;
   const bool fused = a.fuse.k_new != nullptr;
-  if (gate && fused) return cudaErrorInvalidValue;
+  if (gate && fused && a.fuse.gs_new == nullptr) return cudaErrorInvalidValue;
   // scalar-gate rows through the stage ring when a gate-cache row is a whole number
   // of 16-byte pieces (HQ % 4 == 0); otherwise each lane loads its rows itself
   CUtensorMap tmG = tmK;
@@ -530,8 +544,10 @@ cudaError_t decode_impl(const DecodeArgs& a, cudaStream_t st) {
       return cudaErrorInvalidValue;
     gtma = 1;
   }
-  auto kern = fused ? (paged ? decode_split_kernel<T, KD, VD, G, true, false, true>
-                             : decode_split_kernel<T, KD, VD, G, false, false, true>)
+  auto kern = fused ? (paged ? (gate ? decode_split_kernel<T, KD, VD, G, true, true, true>
+                                     : decode_split_kernel<T, KD, VD, G, true, false, true>)
+                             : (gate ? decode_split_kernel<T, KD, VD, G, false, true, true>
+                                     : decode_split_kernel<T, KD, VD, G, false, false, true>))
               : paged ? (gate ? decode_split_kernel<T, KD, VD, G, true, true, false>
                               : decode_split_kernel<T, KD, VD, G, true, false, false>)
                       : (gate ? decode_split_kernel<T, KD, VD, G, false, true, false>

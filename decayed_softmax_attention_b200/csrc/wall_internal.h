@@ -268,6 +268,11 @@ struct DecodeFuse {
   void* k_tilde = nullptr;      // the cache, written at each batch row's new row
   float* r_cache = nullptr;
   void* v = nullptr;
+  // scalar gate (with DecodeArgs::gs_cache): the new token's g_scalar [B, HQ] (input
+  // dtype), PS at the previous row [B, HQ] and PS at the new row (out, another buffer)
+  const void* gs_new = nullptr;
+  const float* gs_prev = nullptr;
+  float* gs_last = nullptr;
 };
 
 struct DecodeArgs {

@@ -308,8 +308,8 @@ wall_status_t wall_attn_decode_paged(const void* q, const float* p_curr, const v
  *          seqlens_kv required; cap ignored
  *   T_kv   the largest T_b (values of seqlens_kv above it are clamped to it)
  * Workspace: wall_attn_decode_workspace_size(B, T_kv, HQ, H, V, chunk) (paged:
- * with T_kv = max_blocks * block_size).  No scalar gate (use the separate
- * gate-cache calls and wall_attn_decode_gated).
+ * with T_kv = max_blocks * block_size).  With the scalar gate use
+ * wall_attn_decode_step_gated below.
  */
 wall_status_t wall_attn_decode_step(const void* q, const void* k_new, const void* g_new,
                                     const void* v_new, const float* p_prev, float* p_last,
@@ -320,6 +320,25 @@ wall_status_t wall_attn_decode_step(const void* q, const void* k_new, const void
                                     void* k_tilde, float* r_cache, void* v_cache, void* o,
                                     float* lse, void* workspace, size_t workspace_bytes,
                                     wall_stream_t stream);
+
+/*
+ * wall_attn_decode_step with the scalar gate (the forward's additive term
+ * Gs[t] - Gs[j], Wall Attention README "Usage" optional arguments, through the
+ * gate cache described below): the same arguments plus
+ *   gs_new   [B, 1, HQ] dtype dt   the new token's g_scalar
+ *   gs_prev  [B, HQ] fp32          PS at row t_b - 1 (read only where t_b > 0)
+ *   gs_last  [B, HQ] fp32          out: PS at row t_b; must not overlap gs_prev
+ *   gs_cache the gate cache (dense [B, cap, HQ] or the pool [num_blocks,
+ *            block_size, HQ] of the same block table), row t_b written
+ * Row j's logit gains (PS[t_b] - PS[j]) ln 2; the new row's own term is 0.
+ */
+wall_status_t wall_attn_decode_step_gated(
+    const void* q, const void* k_new, const void* g_new, const void* v_new, const void* gs_new,
+    const float* p_prev, float* p_last, const float* gs_prev, float* gs_last, float* gs_cache,
+    const float* sink_bias, const int32_t* seqlens_kv, const int32_t* block_table, int max_blocks,
+    int num_blocks, int block_size, int B, int T_kv, int cap, int HQ, int H, int K, int V,
+    int chunk, wall_dtype_t dt, float scale, void* k_tilde, float* r_cache, void* v_cache,
+    void* o, float* lse, void* workspace, size_t workspace_bytes, wall_stream_t stream);
 
 /*
  * Scalar gate in decode (the forward's g_scalar term Gs[t] - Gs[j] through the

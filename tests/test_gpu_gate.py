@@ -126,3 +126,77 @@ def test_gated_paged_streaming(wall):
             assert_close(o[:, 0], ro, torch.bfloat16, f"gated paged step {s_}")
         lens = [L + 1 for L in lens]
     assert wall.wall_device_error() == 0
+
+
+@pytest.mark.parametrize("dtype,HQ,H,K,V,T0", [
+    ("bf16", 8, 2, 128, 128, 190),   # staged gate rows (HQ % 4 == 0)
+    ("f32", 4, 1, 64, 128, 0),       # from an empty cache: the first step has no PS before it
+    ("bf16", 2, 2, 64, 64, 70),      # HQ = 2: gate rows loaded per lane
+    ("bf16", 16, 1, 128, 64, 33),    # a group of 16 query heads
+], ids=lambda x: str(x))
+def test_gated_fused_step_matches_prefill(wall, dtype, HQ, H, K, V, T0):
+    """The fused append + decode step with the scalar gate: every step equals the oracle's
+    prefill row with g_scalar, and afterwards the gate cache equals the oracle's PS."""
+    B, S = 2, 40
+    T = T0 + S
+    spec, d = _inputs(B, T, HQ, H, K, V, dtype, seed=94)
+    dt = spec.torch_dtype
+    cache = wall.KVCache(B, T, HQ, H, K, V, dtype=dt, chunk=64, gate=True)
+    for t_ in (cache.k_tilde, cache.v, cache.r_cache, cache.gs_cache):
+        t_.fill_(float("nan"))
+    if T0 > 0:
+        cache.append(d["k"][:, :T0].contiguous(), d["g"][:, :T0].contiguous(),
+                     d["v"][:, :T0].contiguous(), d["g_scalar"][:, :T0].contiguous())
+    rows = np.array([b * T + t for b in range(B) for t in range(T0, T)], dtype=np.int64)
+    ro, _ = oracle.wall_fwd(d["q"], d["k"], d["v"], d["g"], d["g_scalar"], d["sink_bias"],
+                            scale=d["scale"], rows=rows, threads=ORACLE_THREADS)
+    ro = ro.reshape(B, S, HQ, V)
+    for s_ in range(S):
+        t = T0 + s_
+        sl = slice(t, t + 1)
+        o = cache.step(d["q"][:, sl].contiguous(), d["k"][:, sl].contiguous(),
+                       d["g"][:, sl].contiguous(), d["v"][:, sl].contiguous(),
+                       sink_bias=d["sink_bias"], scale=d["scale"],
+                       gs_new=d["g_scalar"][:, sl].contiguous())
+        assert_close(o[:, 0], ro[:, s_], dt, f"gated fused step {s_}")
+    torch.cuda.synchronize()
+    assert wall.wall_device_error() == 0
+    PS = oracle.gate_cache(d["g_scalar"])
+    np.testing.assert_allclose(cache.gs_cache[:, :T].double().cpu().numpy(), PS[:, :T],
+                               rtol=2e-6, atol=2e-5)
+    np.testing.assert_allclose(cache.gs.double().cpu().numpy(), PS[:, T - 1], rtol=2e-6, atol=2e-5)
+
+
+def test_gated_fused_step_paged(wall):
+    """Paged caches with per-row lengths: gated fused steps through growing block tables."""
+    start, steps, bs = (130, 64), 30, 64
+    B, HQ, H, K, V = len(start), 4, 1, 128, 64
+    T = max(start) + steps
+    spec, d = _inputs(B, T, HQ, H, K, V, "bf16", seed=95)
+    maxblk = (T + bs - 1) // bs
+    cache = wall.PagedKVCache(B, num_blocks=B * maxblk + 1, block_size=bs, max_blocks=maxblk,
+                              HQ=HQ, H=H, K=K, V=V, chunk=64, gate=True)
+    for b, L in enumerate(start):
+        cache.reserve(b, L)
+    for b, L in enumerate(start):
+        tb = cache.block_table[b:b + 1].contiguous()
+        wall.wall_build_kv_cache_paged(d["k"][b:b + 1, :L].contiguous(),
+                                       d["g"][b:b + 1, :L].contiguous(), tb, cache.k_tilde,
+                                       cache.r_cache, cache.p[b:b + 1], chunk=64)
+        wall.wall_build_gate_cache(d["g_scalar"][b:b + 1, :L].contiguous(), cache.gs_cache,
+                                   cache.gs[b:b + 1], block_table=tb)
+        rows = torch.tensor(cache.rows_of(b, 0, L), device="cuda")
+        cache.v.view(-1, H, V)[rows] = d["v"][b, :L]
+        cache.lengths[b] = L
+    lens = list(start)
+    for s_ in range(steps):
+        pick = lambda x: torch.stack([x[b, L] for b, L in enumerate(lens)])[:, None].contiguous()
+        o = cache.step(pick(d["q"]), pick(d["k"]), pick(d["g"]), pick(d["v"]), lens,
+                       sink_bias=d["sink_bias"], scale=d["scale"], gs_new=pick(d["g_scalar"]))
+        if s_ % 5 == 0 or s_ == steps - 1:
+            rows = [b * T + L for b, L in enumerate(lens)]
+            ro, _ = oracle.wall_fwd(d["q"], d["k"], d["v"], d["g"], d["g_scalar"], d["sink_bias"],
+                                    scale=d["scale"], rows=rows, threads=ORACLE_THREADS)
+            assert_close(o[:, 0], ro, torch.bfloat16, f"gated paged fused step {s_}")
+        lens = [L + 1 for L in lens]
+    assert wall.wall_device_error() == 0
