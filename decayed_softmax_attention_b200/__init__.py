@@ -57,7 +57,7 @@ EXPORTED_SYMBOLS = (
     "wall_build_kv_cache_paged", "wall_append_kv_cache_paged", "wall_attn_decode_paged",
     "wall_build_gate_cache", "wall_append_gate_cache", "wall_attn_decode_gated",
     "wall_attn_chunk_workspace_size", "wall_attn_chunk", "wall_attn_decode_step",
-    "wall_attn_decode_step_gated",
+    "wall_attn_decode_step_gated", "wall_attn_chunk_gated",
 )
 
 
@@ -128,6 +128,9 @@ def load_library():
     lib.wall_attn_chunk.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, F, P, P, P, P,
                                     P, P, P, S, P]
     lib.wall_attn_chunk.restype = I
+    lib.wall_attn_chunk_gated.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I,
+                                          F, P, P, P, P, P, P, P, P, P, S, P]
+    lib.wall_attn_chunk_gated.restype = I
     lib.wall_build_kv_cache.argtypes = [P, P, P, I, I, I, I, I, I, I, I, I, P, P, P, P]
     lib.wall_build_kv_cache.restype = I
     lib.wall_append_kv_cache_varlen.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P, P, P, P]
@@ -655,10 +658,12 @@ def wall_attn_chunk_workspace_size(B, M, cap, HQ, H, K, V, chunk=64) -> int:
 
 def wall_attn_chunk(q, k_new, g_new, k_tilde, r_cache, p_last, v_cache, t_start, p_prev=None,
                     sink_bias=None, window=0, scale=None, chunk=64, out=None, lse=None,
-                    workspace=None):
+                    workspace=None, gs_new=None, gs_cache=None, gs_last=None, gs_prev=None):
     """M new tokens at rows t_start.. of the cache: append their keys, then attend rows
     0 .. t_start + i.  q [B,M,HQ,K]; v_cache rows of the chunk must already hold its values.
-    Returns o [B,M,HQ,V].  p_prev defaults to p_last (updated in place)."""
+    Returns o [B,M,HQ,V].  p_prev defaults to p_last (updated in place).  With the scalar
+    gate: gs_new [B,M,HQ] (the chunk's g_scalar), gs_cache [B,cap,HQ] fp32, gs_last [B,HQ]
+    (PS at the last row; gs_prev defaults to it, updated in place)."""
     lib = load_library()
     B, M, HQ, K = q.shape
     H = k_new.shape[2]
@@ -672,6 +677,26 @@ def wall_attn_chunk(q, k_new, g_new, k_tilde, r_cache, p_last, v_cache, t_start,
         workspace = torch.empty(max(wall_attn_chunk_workspace_size(B, M, cap, HQ, H, K, V,
                                                                    chunk), 1),
                                 dtype=torch.uint8, device=q.device)
+    if gs_new is not None:
+        if gs_prev is None and t_start > 0:
+            gs_prev = gs_last
+        st = lib.wall_attn_chunk_gated(
+            _dev(q, "q", dt), _dev(k_new, "k_new", dt, (B, M, H, K)),
+            _dev(g_new, "g_new", dt, (B, M, HQ, K)), _dev(gs_new, "gs_new", dt, (B, M, HQ)),
+            _dev(p_prev, "p_prev", torch.float32, (B, HQ, K)),
+            _dev(gs_prev, "gs_prev", torch.float32, (B, HQ)),
+            _dev(sink_bias, "sink_bias", torch.float32, (HQ,)), int(window or 0), B, int(t_start),
+            M, cap, HQ, H, K, V, int(chunk), _dtype_code(q), float(scale) if scale else 0.0,
+            _dev(k_tilde, "k_tilde", dt, (B, cap, HQ, K)),
+            _dev(r_cache, "r_cache", torch.float32, (B, (cap + chunk - 1) // chunk, HQ, K)),
+            _dev(p_last, "p_last", torch.float32, (B, HQ, K)),
+            _dev(gs_cache, "gs_cache", torch.float32, (B, cap, HQ)),
+            _dev(gs_last, "gs_last", torch.float32, (B, HQ)), _dev(v_cache, "v_cache", dt),
+            _dev(out, "out", dt, (B, M, HQ, V)), _dev(lse, "lse", torch.float32, (B, M, HQ)),
+            _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+            _stream(q.device))
+        _check(st, "wall_attn_chunk_gated")
+        return out
     st = lib.wall_attn_chunk(
         _dev(q, "q", dt), _dev(k_new, "k_new", dt, (B, M, H, K)),
         _dev(g_new, "g_new", dt, (B, M, HQ, K)), _dev(p_prev, "p_prev", torch.float32, (B, HQ, K)),

@@ -720,12 +720,14 @@ size_t wall_attn_chunk_workspace_size(int B, int M, int cap, int HQ, int H, int 
   return wall::chunk_workspace_bytes(B, M, cap, HQ, H, K, V, chunk);
 }
 
-wall_status_t wall_attn_chunk(const void* q, const void* k_new, const void* g_new,
+static wall_status_t chunk_impl(const void* q, const void* k_new, const void* g_new,
                               const float* p_prev, const float* sink_bias, int window, int B,
                               int t_start, int M, int cap, int HQ, int H, int K, int V, int chunk,
                               wall_dtype_t dt, float scale, void* k_tilde, float* r_cache,
                               float* p_last, const void* v_cache, void* o, float* lse,
-                              void* workspace, size_t workspace_bytes, wall_stream_t stream) {
+                              void* workspace, size_t workspace_bytes, wall_stream_t stream,
+                              const void* gs_new, const float* gs_prev, float* gs_cache,
+                              float* gs_last) {
   if (B < 0 || t_start < 0 || M < 0 || cap < 0 || HQ <= 0 || H <= 0 || HQ % H != 0)
     return WALL_ERR_INVALID_ARG;
   if (dt != WALL_DTYPE_F32 && dt != WALL_DTYPE_BF16) return WALL_ERR_INVALID_ARG;
@@ -735,6 +737,12 @@ wall_status_t wall_attn_chunk(const void* q, const void* k_new, const void* g_ne
   if (static_cast<long long>(t_start) + M > cap) return WALL_ERR_INVALID_ARG;
   if (B == 0 || M == 0) return WALL_OK;
   if ((t_start > 0) != (p_prev != nullptr)) return WALL_ERR_INVALID_ARG;
+  if (gs_new != nullptr) {  // scalar gate: g_scalar of the chunk, PS in and out, gate cache
+    if (!gs_cache || !gs_last || (t_start > 0) != (gs_prev != nullptr) ||
+        !aligned(gs_new, 2) || !aligned(gs_cache, 4) || !aligned(gs_last, 4) ||
+        (gs_prev && !aligned(gs_prev, 4)))
+      return WALL_ERR_INVALID_ARG;
+  }
   const void* a16[] = {q, k_new, g_new, k_tilde, r_cache, p_last, v_cache, o, workspace};
   for (const void* ptr : a16)
     if (ptr == nullptr || !aligned(ptr, 16)) return WALL_ERR_INVALID_ARG;
@@ -753,6 +761,7 @@ wall_status_t wall_attn_chunk(const void* q, const void* k_new, const void* g_ne
   a.chunk = chunk; a.scale = scale; a.k_tilde = k_tilde; a.r_cache = r_cache; a.p_last = p_last;
   a.v_cache = v_cache; a.o = o; a.lse = lse; a.workspace = workspace;
   a.fault = wall::fault_mode();
+  a.gs_new = gs_new; a.gs_prev = gs_prev; a.gs_cache = gs_cache; a.gs_last = gs_last;
   a.err = wall::device_error_word();
   if (a.err == nullptr) return WALL_ERR_CUDA;
   a.wait_ns = wall::wait_limit_ns();
@@ -762,6 +771,31 @@ wall_status_t wall_attn_chunk(const void* q, const void* k_new, const void* g_ne
   const cudaError_t e = wall::launch_chunk(a, st);
   stage_event(2, st);
   return finish(e, st);
+}
+
+wall_status_t wall_attn_chunk(const void* q, const void* k_new, const void* g_new,
+                              const float* p_prev, const float* sink_bias, int window, int B,
+                              int t_start, int M, int cap, int HQ, int H, int K, int V, int chunk,
+                              wall_dtype_t dt, float scale, void* k_tilde, float* r_cache,
+                              float* p_last, const void* v_cache, void* o, float* lse,
+                              void* workspace, size_t workspace_bytes, wall_stream_t stream) {
+  return chunk_impl(q, k_new, g_new, p_prev, sink_bias, window, B, t_start, M, cap, HQ, H, K, V,
+                    chunk, dt, scale, k_tilde, r_cache, p_last, v_cache, o, lse, workspace,
+                    workspace_bytes, stream, nullptr, nullptr, nullptr, nullptr);
+}
+
+wall_status_t wall_attn_chunk_gated(const void* q, const void* k_new, const void* g_new,
+                                    const void* gs_new, const float* p_prev, const float* gs_prev,
+                                    const float* sink_bias, int window, int B, int t_start, int M,
+                                    int cap, int HQ, int H, int K, int V, int chunk,
+                                    wall_dtype_t dt, float scale, void* k_tilde, float* r_cache,
+                                    float* p_last, float* gs_cache, float* gs_last,
+                                    const void* v_cache, void* o, float* lse, void* workspace,
+                                    size_t workspace_bytes, wall_stream_t stream) {
+  if (B > 0 && M > 0 && gs_new == nullptr) return WALL_ERR_INVALID_ARG;
+  return chunk_impl(q, k_new, g_new, p_prev, sink_bias, window, B, t_start, M, cap, HQ, H, K, V,
+                    chunk, dt, scale, k_tilde, r_cache, p_last, v_cache, o, lse, workspace,
+                    workspace_bytes, stream, gs_new, gs_prev, gs_cache, gs_last);
 }
 
 wall_status_t wall_device_error(wall_stream_t stream) {

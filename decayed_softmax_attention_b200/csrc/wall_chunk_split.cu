@@ -110,7 +110,7 @@ __global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_s
     const __nv_bfloat16* __restrict__ qh, const float* __restrict__ AQ,
     const float* __restrict__ r_cache, int t0, int M, int HQ, int C, int cap, int window,
     int ck_lo, int cps, int nsplit, int ntg, float sc, float* __restrict__ part, int* err,
-    uint64_t wait_ns, const int* __restrict__ wide, int fault) {
+    uint64_t wait_ns, const int* __restrict__ wide, int fault, const float* __restrict__ gs_cache) {
   using D = MultiCfg<KD, VD, G>;
   constexpr int MQ = D::MQ, LPH = D::LPH, CPL = D::CPL, VPL = D::VPL, RB = D::RB, NV = D::NV;
   constexpr int NO = D::NO, REP = D::REP, MG = MQ * G;
@@ -204,6 +204,11 @@ __global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_s
   const int m_own = base / RB;                    // this lane's token
   if (warp < D::NW) {
     // ------------------------------------------------------------- consumers
+    // scalar gate: the logit gains PS(token's row) - PS(key row), log2 units
+    const size_t gsb = static_cast<size_t>(b) * cap;
+    const int ghq = h * G + hl;
+    const float gs_tok = (gs_cache != nullptr && m0 + m_own < M)
+                             ? gs_cache[(gsb + t0 + m0 + m_own) * HQ + ghq] : 0.f;
     float* pb = reinterpret_cast<float*>(dsm + D::OFF_P) + warp * (RB + 1) * MG;  // [RB][MG]
     float* ab = pb + RB * MG;                                                     // [MG]
     float2 qt2[MQ][CPL / 2];
@@ -264,7 +269,9 @@ __global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_s
           const int row = row0 + rg0 + (base % RB) + j;
           const bool ok = mg_own < M && row < row_end && row <= t0 + mg_own && row <= row_cap &&
                           (window == 0 || t0 + mg_own - row < window);
-          v[j] = ok ? v[j] : -INFINITY;
+          const float gterm = (gs_cache != nullptr && ok) ? gs_tok - gs_cache[(gsb + row) * HQ + ghq]
+                                                          : 0.f;
+          v[j] = ok ? v[j] + gterm : -INFINITY;
           mx = fmaxf(mx, v[j]);
         }
 #pragma unroll
@@ -414,7 +421,7 @@ cudaError_t chunk_split_impl(const ChunkArgs& a, const void* qh, const float* AQ
   kern<<<grid, (D::NW + 1) * 32, D::SMEM, st>>>(
       tmK, tmV, static_cast<const __nv_bfloat16*>(qh), AQ, a.r_cache, a.t0, a.M, a.HQ, a.chunk,
       a.cap, a.window, ck_lo, cps, nsplit, ntg, a.scale * kLog2e, part, a.err, a.wait_ns, wide,
-      a.fault);
+      a.fault, a.gs_cache);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_decode_combine_bf16(part, nsplit, a.B * a.M * a.HQ, a.HQ, a.sink, a.o, lse, VD,

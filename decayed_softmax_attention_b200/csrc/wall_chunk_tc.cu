@@ -32,6 +32,7 @@ struct ChunkParams {
   int* err;
   uint64_t wait_ns;
   int fault;  // testing hook: 6 = the producer skips its first key tile
+  const float* gs_cache;  // scalar gate: PS per (cache row, query head), log2 units, or null
 };
 
 template <int KD, int VD, int CH>
@@ -49,7 +50,8 @@ struct ChCfg {
   static constexpr int OFF_AQ = OFF_V + VS * V_BYTES;
   static constexpr int OFF_R = OFF_AQ + KD * 4;                // [KS][NRC][KD]
   static constexpr int OFF_C = OFF_R + KS * NRC * KD * 4;      // [2][NRC][KD]
-  static constexpr int OFF_BAR = OFF_C + 2 * NRC * KD * 4;
+  static constexpr int OFF_GS = OFF_C + 2 * NRC * KD * 4;         // [2 tiles][2][BN] fp32
+  static constexpr int OFF_BAR = OFF_GS + 2 * 2 * BN * 4;
   // qfull, kfull[KS], kready[KS], kempty[KS], vfull[VS], vempty[VS], sfull[2], pfull[2],
   // ofinal, mdrain
   static constexpr int NBAR = 1 + 3 * KS + 2 * VS + 2 + 2 + 2;
@@ -100,7 +102,7 @@ __device__ __forceinline__ void reg_fence32(float* r) {
                  "+f"(r[24]), "+f"(r[25]), "+f"(r[26]), "+f"(r[27]), "+f"(r[28]), "+f"(r[29]),
                  "+f"(r[30]), "+f"(r[31]));
 }
-template <int KD, int VD, int CH>
+template <int KD, int VD, int CH, bool GS>
 __global__ void __launch_bounds__(512, 1)
     wall_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
@@ -115,6 +117,7 @@ __global__ void __launch_bounds__(512, 1)
   float* sAQ = reinterpret_cast<float*>(smem + C::OFF_AQ);
   float* sR = reinterpret_cast<float*>(smem + C::OFF_R);
   float* sC = reinterpret_cast<float*>(smem + C::OFF_C);
+  float* sGS = reinterpret_cast<float*>(smem + C::OFF_GS);  // [query tile][2][BN] gate prefixes
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* qfull = bars;
   uint64_t* kfull = bars + 1;
@@ -328,11 +331,27 @@ __global__ void __launch_bounds__(512, 1)
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     const int jf = X == 0 ? jfA : jfB, jl = X == 0 ? jlA : jlB;
+    // Scalar gate: the logit gains PS(query row) - PS(key row) (log2 units).  Thread r
+    // of the warpgroup loads key row kt * BN + r of each tile, one tile ahead; the
+    // warpgroup shares the tile's 128 values through shared memory.
+    const size_t gsb = static_cast<size_t>(b) * p.cap;  // first gate row of this batch row
+    const int nrows = p.t0 + p.M;                       // gate rows written so far
+    auto gate_row = [&](int r) -> float {
+      return (r >= 0 && r < nrows) ? p.gs_cache[(gsb + r) * p.HQ + hq] : 0.f;
+    };
+    const float gs_row = (GS && row_ok) ? gate_row(gi) : 0.f;
+    float gs_next = (GS && jl >= jf) ? gate_row((kt_hi - jf) * C::BN + row) : 0.f;
     for (int j = jf; j <= jl; ++j) {
       const int cnt = j - jf;
       const int kt = kt_hi - j;
+      float* gsl = sGS + (X * 2 + (cnt & 1)) * C::BN;
+      if (GS) {
+        gsl[row] = gs_next;
+        if (j < jl) gs_next = gate_row((kt - 1) * C::BN + row);
+      }
       const bool got = mbar_wait(&sfull[X], cnt & 1, wc);
-      if (!__all_sync(0xffffffffu, got)) {
+      // gated: one decision for the whole warpgroup (the barrier also publishes gsl)
+      if (GS ? bar_or(2 + X, 128, !got) : !__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
       }
@@ -352,13 +371,22 @@ __global__ void __launch_bounds__(512, 1)
           if (jg < lo || jg > hi) s[jj] = -INFINITY;
         }
       }
+      if (GS) {  // s <- s * sc - PS(key row); the row's PS joins through off below
+#pragma unroll
+        for (int jj = 0; jj < C::BN; jj += 4) {
+          const float4 g4 = *reinterpret_cast<const float4*>(gsl + jj);
+          const float2 a = ffma2(make_float2(s[jj], s[jj + 1]), sc2, make_float2(-g4.x, -g4.y));
+          const float2 c = ffma2(make_float2(s[jj + 2], s[jj + 3]), sc2, make_float2(-g4.z, -g4.w));
+          s[jj] = a.x; s[jj + 1] = a.y; s[jj + 2] = c.x; s[jj + 3] = c.y;
+        }
+      }
       float mx0 = s[0], mx1 = s[1];
 #pragma unroll
       for (int jj = 2; jj < C::BN; jj += 4) {
         mx0 = fmax3(mx0, s[jj], s[jj + 1]);
         mx1 = fmax3(mx1, s[jj + 2], s[jj + 3]);
       }
-      const float mt = fmaxf(mx0, mx1) * p.sc;
+      const float mt = GS ? fmaxf(mx0, mx1) + gs_row : fmaxf(mx0, mx1) * p.sc;
       const bool need = mt > m_used + 8.f;
       float alpha = 1.f;
       if (need) {
@@ -367,14 +395,15 @@ __global__ void __launch_bounds__(512, 1)
         m_used = mt;
       }
       const float base = (m_used == -INFINITY) ? 0.f : m_used;
-      const float2 off = make_float2(-base, -base);
+      const float2 off = make_float2(gs_row - base, gs_row - base);
+      const float2 mul = GS ? make_float2(1.f, 1.f) : sc2;  // (gated scores are already scaled)
       float2 rs = make_float2(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < C::BN; c += 32) {
         uint32_t pk[16];
 #pragma unroll
         for (int jj = 0; jj < 32; jj += 2) {
-          const float2 t = ffma2(make_float2(s[c + jj], s[c + jj + 1]), sc2, off);
+          const float2 t = ffma2(make_float2(s[c + jj], s[c + jj + 1]), mul, off);
           const float2 pv = make_float2(ex2_approx(t.x), ex2_approx(t.y));
           rs = fadd2(rs, pv);
           pk[jj >> 1] = pack_bf16(pv.x, pv.y);
@@ -651,7 +680,8 @@ cudaError_t chunk_impl(const ChunkArgs& a, void* qh, float* AQ, const int* wide,
                       CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
-  auto kern = wall_chunk_tc_kernel<KD, VD, CH>;
+  auto kern = a.gs_cache != nullptr ? wall_chunk_tc_kernel<KD, VD, CH, true>
+                                    : wall_chunk_tc_kernel<KD, VD, CH, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
   if (e != cudaSuccess) return e;
   ChunkParams p;
@@ -673,6 +703,7 @@ cudaError_t chunk_impl(const ChunkArgs& a, void* qh, float* AQ, const int* wide,
   p.err = a.err;
   p.wait_ns = a.wait_ns;
   p.fault = a.fault;
+  p.gs_cache = a.gs_cache;
   const unsigned grid = static_cast<unsigned>(NQB) * BHQ;
   if (a.ev_mid != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(a.ev_mid), st);
   kern<<<grid, 512, C::SMEM_ALLOC, st>>>(tmQ, tmK, tmV, p);
@@ -749,6 +780,15 @@ cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t st) {
   c.pm.cap = a.cap;
   e = launch_cache_build(c, true, st);
   if (e != cudaSuccess) return e;
+  if (a.gs_new != nullptr) {  // the chunk's gate prefixes join the gate cache
+    GateArgs ga;
+    ga.gs_new = a.gs_new; ga.gs_prev = a.t0 > 0 ? a.gs_prev : nullptr; ga.t_pos = nullptr;
+    ga.B = a.B; ga.t_start = a.t0; ga.T_new = a.M; ga.HQ = a.HQ;
+    ga.gcache = a.gs_cache; ga.gs_last = a.gs_last;
+    ga.pm.cap = a.cap;
+    e = launch_gate_cache(ga, true, st);
+    if (e != cudaSuccess) return e;
+  }
   // 3. the chunk's queries attend the cache: a few tokens per sequence the
   //    decode's way, longer chunks in 128-row tensor-core query tiles
   if (chunk_split_applies(a.M, a.HQ, a.H)) {
@@ -768,7 +808,7 @@ cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t st) {
   // 4. wide blocks (strong decay inside a 256-row query block): the chunk's own
   //    pairs there, exactly, merged with the result for the rows before
   DiagParams d;
-  d.q = a.q; d.k = a.k_new; d.g = a.g_new; d.gs = nullptr; d.v = a.v_cache;
+  d.q = a.q; d.k = a.k_new; d.g = a.g_new; d.gs = a.gs_new; d.v = a.v_cache;
   d.sink = a.sink; d.rowlo = nullptr; d.wide = wide; d.window = a.window;
   d.B = a.B; d.Tb = a.M; d.HQ = a.HQ; d.H = a.H; d.NQB = static_cast<int>(NQB);
   d.vT = a.cap; d.voff = a.t0; d.pos0 = a.t0;

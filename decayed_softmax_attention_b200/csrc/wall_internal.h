@@ -243,6 +243,13 @@ struct ChunkArgs {
   uint64_t wait_ns;
   void* ev_mid = nullptr;  // optional event recorded before the attention kernel
   int fault = 0;           // testing hook: 6 = chunk tile kernel, 7 = few-token split kernel
+  // scalar gate (null gs_new: none): the chunk's g_scalar [B, M, HQ] (input dtype), PS
+  // at row t0 - 1 [B, HQ] (null iff t0 == 0), the gate cache [B, cap, HQ] (rows t0 ..
+  // written here) and PS at the chunk's last row [B, HQ] (may alias gs_prev)
+  const void* gs_new = nullptr;
+  const float* gs_prev = nullptr;
+  float* gs_cache = nullptr;
+  float* gs_last = nullptr;
 };
 size_t chunk_workspace_bytes(int B, int M, int cap, int HQ, int H, int K, int V, int chunk);
 cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t st);

@@ -395,7 +395,8 @@ wall_status_t wall_attn_decode_gated(const void* q, const float* p_curr, const f
  *   o        [B, M, HQ, V] bf16;  lse [B, M, HQ] fp32 (nullable)
  *   workspace >= wall_attn_chunk_workspace_size(B, M, cap, HQ, H, K, V, chunk)
  *            bytes, 256-aligned
- * bf16 only (fp32: WALL_ERR_UNSUPPORTED); no g_scalar term.
+ * bf16 only (fp32: WALL_ERR_UNSUPPORTED); the scalar gate through
+ * wall_attn_chunk_gated below.
  * A chunk of at most 2 * 16 / (HQ / H) tokens (multi-token decode) attends
  * through a split-KV pass that streams the cache once per KV head; longer
  * chunks through 128-row tensor-core query tiles.  Both give the same result
@@ -410,6 +411,27 @@ wall_status_t wall_attn_chunk(const void* q, const void* k_new, const void* g_ne
                               wall_dtype_t dt, float scale, void* k_tilde, float* r_cache,
                               float* p_last, const void* v_cache, void* o, float* lse,
                               void* workspace, size_t workspace_bytes, wall_stream_t stream);
+
+/*
+ * wall_attn_chunk with the scalar gate (the forward's additive term Gs[i] - Gs[j],
+ * Wall Attention README "Usage" optional arguments): the chunk's gate prefixes
+ * join the gate cache first, exactly as wall_build_gate_cache(gs_new, gs_prev,
+ * t_start, ...) writes them, then query i's logit of cache row j gains
+ * (PS[t_start + i] - PS[j]) ln 2.
+ *   gs_new    [B, M, HQ] bf16          the chunk's g_scalar
+ *   gs_prev   [B, HQ] fp32             PS at row t_start - 1 (NULL iff t_start == 0)
+ *   gs_cache  [B, cap, HQ] fp32        the dense gate cache (rows t_start .. written)
+ *   gs_last   [B, HQ] fp32             out: PS at the chunk's last row (may alias gs_prev)
+ * Other arguments and the workspace as wall_attn_chunk.
+ */
+wall_status_t wall_attn_chunk_gated(const void* q, const void* k_new, const void* g_new,
+                                    const void* gs_new, const float* p_prev, const float* gs_prev,
+                                    const float* sink_bias, int window, int B, int t_start, int M,
+                                    int cap, int HQ, int H, int K, int V, int chunk,
+                                    wall_dtype_t dt, float scale, void* k_tilde, float* r_cache,
+                                    float* p_last, float* gs_cache, float* gs_last,
+                                    const void* v_cache, void* o, float* lse, void* workspace,
+                                    size_t workspace_bytes, wall_stream_t stream);
 
 /*
  * Decode without scratch allocation (no counterpart in the paper: this entry

@@ -113,3 +113,54 @@ def test_chunk_then_decode(wall):
         o = cache.decode(d["q"][:, t:t + 1].contiguous(), sink_bias=d["sink_bias"],
                          scale=d["scale"])
         assert_close(o[:, 0], ro[:, s_], torch.bfloat16, f"decode after chunk, step {s_}")
+
+
+GATED_CASES = [
+    dict(B=2, sizes=(300, 129, 1, 270), HQ=8, H=2, K=128, V=128, C=64, window=0, sink=True,
+         g_kind="negsoftplus"),
+    dict(B=2, sizes=(517, 4, 8, 1, 3), HQ=8, H=2, K=128, V=64, C=32, window=150, sink=False,
+         g_kind="negsoftplus"),
+    dict(B=1, sizes=(600, 260), HQ=4, H=1, K=64, V=128, C=32, window=0, sink=True,
+         g_kind="strong_cache"),  # wide blocks: the exact in-block pass carries the gate too
+]
+
+
+@pytest.mark.parametrize("case", GATED_CASES, ids=_ids)
+def test_gated_chunks_reproduce_the_prefill(wall, case):
+    """wall_attn_chunk_gated: chunks of a sequence with the scalar gate equal the oracle's
+    prefill rows with g_scalar, through the tile kernel, the few-token split pass and the
+    wide-block pass; the gate cache the chunks build equals the oracle's PS."""
+    B, HQ, H, K, V, C = case["B"], case["HQ"], case["H"], case["K"], case["V"], case["C"]
+    T = sum(case["sizes"])
+    spec = W.PrefillSpec("chunk_gate", B=B, T=T, HQ=HQ, H=H, K=K, V=V, dtype="bf16",
+                         g_kind=case["g_kind"], g_scalar=True, sink=case["sink"],
+                         window=case["window"], seed=103)
+    d = W.gen_prefill(spec, device="cuda")
+    cap = T + 9
+    nan = float("nan")
+    kt = torch.full((B, cap, HQ, K), nan, dtype=torch.bfloat16, device="cuda")
+    rc = torch.full((B, (cap + C - 1) // C, HQ, K), nan, dtype=torch.float32, device="cuda")
+    p = torch.full((B, HQ, K), nan, dtype=torch.float32, device="cuda")
+    vc = torch.full((B, cap, H, V), nan, dtype=torch.bfloat16, device="cuda")
+    gsc = torch.full((B, cap, HQ), nan, dtype=torch.float32, device="cuda")
+    gsl = torch.full((B, HQ), nan, dtype=torch.float32, device="cuda")
+    ro, rl = oracle.wall_fwd(d["q"], d["k"], d["v"], d["g"], d["g_scalar"], d["sink_bias"],
+                             window=d["window"], scale=d["scale"], threads=ORACLE_THREADS)
+    t0 = 0
+    for M in case["sizes"]:
+        sl = slice(t0, t0 + M)
+        vc[:, sl].copy_(d["v"][:, sl])
+        lse = torch.empty((B, M, HQ), dtype=torch.float32, device="cuda")
+        o = wall.wall_attn_chunk(d["q"][:, sl].contiguous(), d["k"][:, sl].contiguous(),
+                                 d["g"][:, sl].contiguous(), kt, rc, p, vc, t0,
+                                 sink_bias=d["sink_bias"], window=d["window"], scale=d["scale"],
+                                 chunk=C, lse=lse, gs_new=d["g_scalar"][:, sl].contiguous(),
+                                 gs_cache=gsc, gs_last=gsl)
+        torch.cuda.synchronize()
+        assert wall.wall_device_error() == 0
+        assert_close(o, ro[:, sl], torch.bfloat16, f"gated chunk at {t0} (M={M})")
+        assert_close(lse, rl[:, sl], torch.bfloat16, f"gated chunk lse at {t0} (M={M})")
+        t0 += M
+    PS = oracle.gate_cache(d["g_scalar"])
+    np.testing.assert_allclose(gsc[:, :T].double().cpu().numpy(), PS, rtol=2e-6, atol=2e-5)
+    np.testing.assert_allclose(gsl.double().cpu().numpy(), PS[:, -1], rtol=2e-6, atol=2e-5)
