@@ -123,7 +123,7 @@ def load_library():
     lib.wall_attn_decode_gated.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I,
                                            I, I, I, F, P, P, P, S, P]
     lib.wall_attn_decode_gated.restype = I
-    lib.wall_attn_chunk_workspace_size.argtypes = [I, I, I, I, I, I, I, I]
+    lib.wall_attn_chunk_workspace_size.argtypes = [I, I, I, I, I, I, I, I, I]
     lib.wall_attn_chunk_workspace_size.restype = S
     lib.wall_attn_chunk.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, F, P, P, P, P,
                                     P, P, P, S, P]
@@ -652,8 +652,10 @@ def wall_attn_decode_gated(q, p_curr, gs_curr, v, k_tilde, r_cache, gs_cache, T_
 
 
 # ----------------------------------------------------------------- chunked prefill
-def wall_attn_chunk_workspace_size(B, M, cap, HQ, H, K, V, chunk=64) -> int:
-    return int(load_library().wall_attn_chunk_workspace_size(B, M, cap, HQ, H, K, V, chunk))
+def wall_attn_chunk_workspace_size(B, M, cap, HQ, H, K, V, chunk=64,
+                                   dtype=torch.bfloat16) -> int:
+    code = WALL_DTYPE_F32 if dtype == torch.float32 else WALL_DTYPE_BF16
+    return int(load_library().wall_attn_chunk_workspace_size(B, M, cap, HQ, H, K, V, chunk, code))
 
 
 def wall_attn_chunk(q, k_new, g_new, k_tilde, r_cache, p_last, v_cache, t_start, p_prev=None,
@@ -675,7 +677,7 @@ def wall_attn_chunk(q, k_new, g_new, k_tilde, r_cache, p_last, v_cache, t_start,
         out = torch.empty((B, M, HQ, V), dtype=dt, device=q.device)
     if workspace is None:
         workspace = torch.empty(max(wall_attn_chunk_workspace_size(B, M, cap, HQ, H, K, V,
-                                                                   chunk), 1),
+                                                                   chunk, dt), 1),
                                 dtype=torch.uint8, device=q.device)
     if gs_new is not None:
         if gs_prev is None and t_start > 0:

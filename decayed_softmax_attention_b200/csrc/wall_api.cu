@@ -713,11 +713,11 @@ wall_status_t wall_attn_decode_gated(const void* q, const float* p_curr, const f
 }
 
 size_t wall_attn_chunk_workspace_size(int B, int M, int cap, int HQ, int H, int K, int V,
-                                      int chunk) {
+                                      int chunk, wall_dtype_t dt) {
   if (B <= 0 || M <= 0 || cap <= 0 || HQ <= 0 || H <= 0 || HQ % H != 0 || K <= 0 || V <= 0 ||
       chunk <= 0)
     return 0;
-  return wall::chunk_workspace_bytes(B, M, cap, HQ, H, K, V, chunk);
+  return wall::chunk_workspace_bytes(B, M, cap, HQ, H, K, V, chunk, dt != WALL_DTYPE_F32);
 }
 
 static wall_status_t chunk_impl(const void* q, const void* k_new, const void* g_new,
@@ -731,15 +731,19 @@ static wall_status_t chunk_impl(const void* q, const void* k_new, const void* g_
   if (B < 0 || t_start < 0 || M < 0 || cap < 0 || HQ <= 0 || H <= 0 || HQ % H != 0)
     return WALL_ERR_INVALID_ARG;
   if (dt != WALL_DTYPE_F32 && dt != WALL_DTYPE_BF16) return WALL_ERR_INVALID_ARG;
-  if (dt != WALL_DTYPE_BF16) return WALL_ERR_UNSUPPORTED;  // tensor-core path only
+  const bool bf16 = dt == WALL_DTYPE_BF16;
   if (!supported_dim(K) || !supported_dim(V)) return WALL_ERR_UNSUPPORTED;
   if (chunk != 32 && chunk != 64 && chunk != 128) return WALL_ERR_UNSUPPORTED;
   if (static_cast<long long>(t_start) + M > cap) return WALL_ERR_INVALID_ARG;
   if (B == 0 || M == 0) return WALL_OK;
+  // fp32 chunks take the split-KV pass: power-of-two groups, B * M * HQ rows in an int
+  if (!bf16 && (!wall::chunk_split_applies(M, HQ, H, false) ||
+                static_cast<long long>(B) * M * HQ > 0x7fffffffLL))
+    return WALL_ERR_UNSUPPORTED;
   if ((t_start > 0) != (p_prev != nullptr)) return WALL_ERR_INVALID_ARG;
   if (gs_new != nullptr) {  // scalar gate: g_scalar of the chunk, PS in and out, gate cache
     if (!gs_cache || !gs_last || (t_start > 0) != (gs_prev != nullptr) ||
-        !aligned(gs_new, 2) || !aligned(gs_cache, 4) || !aligned(gs_last, 4) ||
+        !aligned(gs_new, bf16 ? 2 : 4) || !aligned(gs_cache, 4) || !aligned(gs_last, 4) ||
         (gs_prev && !aligned(gs_prev, 4)))
       return WALL_ERR_INVALID_ARG;
   }
@@ -751,14 +755,14 @@ static wall_status_t chunk_impl(const void* q, const void* k_new, const void* g_
     return WALL_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * HQ * ((M + 255) / 256) > 0x7fffffffLL || B > 65535)
     return WALL_ERR_UNSUPPORTED;
-  if (workspace_bytes < wall::chunk_workspace_bytes(B, M, cap, HQ, H, K, V, chunk))
+  if (workspace_bytes < wall::chunk_workspace_bytes(B, M, cap, HQ, H, K, V, chunk, bf16))
     return WALL_ERR_WORKSPACE;
   if (!(scale > 0.f) || !std::isfinite(scale)) scale = 1.f / std::sqrt(static_cast<float>(K));
   wall::ChunkArgs a;
   a.q = q; a.k_new = k_new; a.g_new = g_new; a.p_prev = p_prev; a.sink = sink_bias;
   a.window = window > 0 ? window : 0;
   a.B = B; a.t0 = t_start; a.M = M; a.cap = cap; a.HQ = HQ; a.H = H; a.K = K; a.V = V;
-  a.chunk = chunk; a.scale = scale; a.k_tilde = k_tilde; a.r_cache = r_cache; a.p_last = p_last;
+  a.chunk = chunk; a.bf16 = bf16; a.scale = scale; a.k_tilde = k_tilde; a.r_cache = r_cache; a.p_last = p_last;
   a.v_cache = v_cache; a.o = o; a.lse = lse; a.workspace = workspace;
   a.fault = wall::fault_mode();
   a.gs_new = gs_new; a.gs_prev = gs_prev; a.gs_cache = gs_cache; a.gs_last = gs_last;

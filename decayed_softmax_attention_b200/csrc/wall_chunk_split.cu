@@ -8,20 +8,33 @@
 namespace wall {
 namespace {
 
+// N consecutive elements as floats (N = 2, 4 or a multiple of 8).
 template <int N>
-__device__ __forceinline__ void load_bf16_n(const __nv_bfloat16* p, float* f) {
+__device__ __forceinline__ void load_n(const __nv_bfloat16* p, float* f) {
   if constexpr (N % 8 == 0) {
 #pragma unroll
     for (int i = 0; i < N; i += 8) load8(p + i, f + i);
   } else if constexpr (N == 4) {
-    const uint2 u = *reinterpret_cast<const uint2*>(p);
-    f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x); f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
+    load4(p, f);
   } else {
     static_assert(N == 2, "unsupported vector width");
     const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
     f[0] = bf16_lo(u); f[1] = bf16_hi(u);
   }
 }
+template <int N>
+__device__ __forceinline__ void load_n(const float* p, float* f) {
+  if constexpr (N % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < N; i += 4) load4(p + i, f + i);
+  } else {
+    static_assert(N == 2, "unsupported vector width");
+    const float2 u = *reinterpret_cast<const float2*>(p);
+    f[0] = u.x; f[1] = u.y;
+  }
+}
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_f32(float x) { return x; }
 
 // ----------------------------------------------------------------- few-token chunks
 // A chunk of M new tokens per sequence (multi-token decode, e.g. speculative
@@ -43,14 +56,19 @@ __device__ __forceinline__ void load_bf16_n(const __nv_bfloat16* p, float* f) {
 // the value accumulators through shared memory (each lane holds V / 32
 // channels of o for every head and token).  Per-lane state: queries
 // MQ * CPL = KD / 2 floats, accumulators MQ * G * VD / 32 = VD / 2 floats.
-template <int KD, int VD, int G>
+//
+// fp32 caches take the same pass for chunks of any length (there is no fp32
+// tensor-core tile): each CTA then stops at its token group's last causal row
+// and starts at its first token's window, and reads the anchor AQ of the
+// group's 256-row query block.
+template <int KD, int VD, int G, int ES>
 struct MultiCfg {
   static constexpr int MQ = 16 / G;  // tokens per CTA
   static constexpr int LPH = 32 / G;
   static constexpr int CPL = KD / LPH;
   static constexpr int VPL = VD / 32;
   static constexpr int GK = G * KD;
-  static constexpr int SR0 = 32768 / (GK * 2);
+  static constexpr int SR0 = 32768 / (GK * ES);
   static constexpr int SR = SR0 > 32 ? 32 : (SR0 < 8 ? 8 : SR0);  // rows per stage
   static constexpr int NW = 8;                                     // consumer warps
   static constexpr int RPW = SR / NW;                              // rows per warp per stage
@@ -59,8 +77,8 @@ struct MultiCfg {
   static constexpr int NO = NV >= LPH ? NV / LPH : 1;              // sums a lane owns
   static constexpr int REP = NV >= LPH ? 1 : LPH / NV;             // lanes holding each sum
   static constexpr int TSPAN = RB / NO;                            // owners per token
-  static constexpr int K_BYTES = SR * GK * 2;
-  static constexpr int V_BYTES = SR * VD * 2;
+  static constexpr int K_BYTES = SR * GK * ES;
+  static constexpr int V_BYTES = SR * VD * ES;
   static constexpr int R_BYTES = GK * 4;
   static constexpr int STAGE = K_BYTES + V_BYTES + R_BYTES;
   static constexpr int NS0 = 172032 / STAGE;
@@ -104,20 +122,23 @@ __device__ __forceinline__ void reduce_scatter(float* v, int lane) {
   }
 }
 
-template <int KD, int VD, int G>
-__global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_split_kernel(
-    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-    const __nv_bfloat16* __restrict__ qh, const float* __restrict__ AQ,
-    const float* __restrict__ r_cache, int t0, int M, int HQ, int C, int cap, int window,
-    int ck_lo, int cps, int nsplit, int ntg, float sc, float* __restrict__ part, int* err,
-    uint64_t wait_ns, const int* __restrict__ wide, int fault, const float* __restrict__ gs_cache) {
-  using D = MultiCfg<KD, VD, G>;
+template <int KD, int VD, int G, typename T>
+__global__ void __launch_bounds__((MultiCfg<KD, VD, G, sizeof(T)>::NW + 1) * 32, 1)
+    chunk_split_kernel(const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const T* __restrict__ qh,
+                       const float* __restrict__ AQ, const float* __restrict__ r_cache, int t0,
+                       int M, int HQ, int C, int cap, int window, int ck_lo, int cps, int nsplit,
+                       int ntg, float sc, float* __restrict__ part, int* err, uint64_t wait_ns,
+                       const int* __restrict__ wide, int fault,
+                       const float* __restrict__ gs_cache) {
+  using D = MultiCfg<KD, VD, G, sizeof(T)>;
   constexpr int MQ = D::MQ, LPH = D::LPH, CPL = D::CPL, VPL = D::VPL, RB = D::RB, NV = D::NV;
   constexpr int NO = D::NO, REP = D::REP, MG = MQ * G;
   // channels per k_tilde load; a lane's pieces interleave with the other lanes
   // of its head (piece j of lane l starts at channel (l + LPH j) PC), so each
   // quarter-warp's 16-byte loads cover 128 contiguous bytes (no bank conflicts)
-  constexpr int PC = CPL < 8 ? CPL : 8;
+  constexpr int PW = 16 / static_cast<int>(sizeof(T));
+  constexpr int PC = CPL < PW ? CPL : PW;
   extern __shared__ __align__(128) uint8_t dsm[];
   uint64_t* full = reinterpret_cast<uint64_t*>(dsm + D::OFF_BAR);
   uint64_t* empty = full + D::NS;
@@ -132,10 +153,14 @@ __global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_s
   const int ncap = (cap + C - 1) / C;
   const int ck0 = ck_lo + s * cps;
   const int ck1 = min(ck0 + cps, nchunks);
-  const int row_begin = ck0 * C;
-  const int row_end = min(ck1 * C, T_b);
-  const int nst = row_end > row_begin ? (row_end - row_begin + D::SR - 1) / D::SR : 0;
   const int m0 = tg * MQ;  // first token of this CTA's group
+  const int qb = m0 >> 8;  // its 256-row query block (MQ divides 256)
+  // rows the group can see: up to its last token's row, from its first token's
+  // window on (chunk-aligned, so every stage stays inside one anchor chunk)
+  const int lo_g = window > 0 ? max(0, t0 + m0 + 1 - window) / C * C : 0;
+  const int row_begin = max(ck0 * C, lo_g);
+  const int row_end = min(min(ck1 * C, T_b), t0 + min(m0 + MQ, M));
+  const int nst = row_end > row_begin ? (row_end - row_begin + D::SR - 1) / D::SR : 0;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < D::NS; ++i) {
@@ -152,12 +177,13 @@ __global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_s
     const int L = idx & 31, m = (idx >> 5) / CPL, e = (idx >> 5) % CPL;
     const int n = (L % LPH) * PC + (e / PC) * LPH * PC + e % PC;  // channel within the head
     const size_t bh = static_cast<size_t>(b) * HQ + h * G + L / LPH;
-    sQ[idx] = m0 + m < M ? sc * __bfloat162float(qh[(bh * M + m0 + m) * KD + n]) : 0.f;
+    sQ[idx] = m0 + m < M ? sc * to_f32(qh[(bh * M + m0 + m) * KD + n]) : 0.f;
   }
+  const int NQB = (M + 255) >> 8;
   for (int idx = threadIdx.x; idx < CPL * 32; idx += (D::NW + 1) * 32) {
     const int L = idx & 31, e = idx >> 5;
     const int n = (L % LPH) * PC + (e / PC) * LPH * PC + e % PC;
-    sAQ[idx] = AQ[(static_cast<size_t>(b) * HQ + h * G + L / LPH) * KD + n];
+    sAQ[idx] = AQ[((static_cast<size_t>(b) * HQ + h * G + L / LPH) * NQB + qb) * KD + n];
   }
   __syncthreads();
   const WaitCtl wc{abort_flag, err, wait_ns};
@@ -196,10 +222,11 @@ __global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_s
     for (int c = 0; c < VPL; ++c) o2[kp][c] = make_float2(0.f, 0.f);
   const int hl = lane / LPH, l = lane % LPH;
   const int chan0 = hl * KD + l * PC;  // channel of piece j: chan0 + j * LPH * PC
-  // Strong decay inside the chunk (one 256-row query block): this head's rows
-  // from t0 on are left to the diagonal kernel (masked here, factors kept finite).
-  const bool wide_h = wide[static_cast<size_t>(b) * HQ + h * G + hl] != 0;
-  const int row_cap = wide_h ? t0 - 1 : 0x7fffffff;
+  // Strong decay inside the group's 256-row query block: this head's rows of
+  // that block are left to the diagonal kernel (masked here, factors kept finite).
+  const int qrow0 = t0 + (qb << 8);  // cache row of the block's first token
+  const bool wide_h = wide[(static_cast<size_t>(b) * HQ + h * G + hl) * NQB + qb] != 0;
+  const int row_cap = wide_h ? qrow0 - 1 : 0x7fffffff;
   const int base = NV >= LPH ? l * NO : l / REP;  // first owned score index (token-major)
   const int m_own = base / RB;                    // this lane's token
   if (warp < D::NW) {
@@ -227,7 +254,7 @@ __global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_s
         for (int e = 0; e < CPL; e += 2) {
           const int n = chan0 + (e / PC) * LPH * PC + e % PC;
           const float2 r2 = *reinterpret_cast<const float2*>(R + n);
-          const bool own = wide_h && cur_chunk * C >= t0;
+          const bool own = wide_h && cur_chunk * C >= qrow0;
           const float2 f = own ? make_float2(0.f, 0.f)
                                : make_float2(exp2f(sAQ[e * 32 + lane] - r2.x),
                                              exp2f(sAQ[(e + 1) * 32 + lane] - r2.y));
@@ -237,8 +264,8 @@ __global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_s
                 make_float2(sQ[(m * CPL + e) * 32 + lane], sQ[(m * CPL + e + 1) * 32 + lane]), f);
         }
       }
-      const __nv_bfloat16* sk = reinterpret_cast<const __nv_bfloat16*>(st);
-      const __nv_bfloat16* sv = reinterpret_cast<const __nv_bfloat16*>(st + D::K_BYTES);
+      const T* sk = reinterpret_cast<const T*>(st);
+      const T* sv = reinterpret_cast<const T*>(st + D::K_BYTES);
 #pragma unroll 1
       for (int gq = 0; gq < D::RPW / RB; ++gq) {
         const int rg0 = warp * D::RPW + gq * RB;  // first row of the group within the stage
@@ -251,7 +278,7 @@ __global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_s
 #pragma unroll
           for (int e0 = 0; e0 < CPL; e0 += PC) {
             float kf[PC];
-            load_bf16_n<PC>(sk + (rg0 + rb) * D::GK + chan0 + (e0 / PC) * LPH * PC, kf);
+            load_n<PC>(sk + (rg0 + rb) * D::GK + chan0 + (e0 / PC) * LPH * PC, kf);
 #pragma unroll
             for (int e = 0; e < PC; e += 2)
 #pragma unroll
@@ -306,7 +333,7 @@ __global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_s
 #pragma unroll
         for (int rb = 0; rb < RB; ++rb) {
           float vf[VPL];
-          load_bf16_n<VPL>(sv + (rg0 + rb) * VD + lane * VPL, vf);
+          load_n<VPL>(sv + (rg0 + rb) * VD + lane * VPL, vf);
 #pragma unroll
           for (int k = 0; k < MG; k += 4) {
             const float4 p4 = *reinterpret_cast<const float4*>(pb + rb * MG + k);
@@ -372,37 +399,47 @@ __global__ void __launch_bounds__((MultiCfg<KD, VD, G>::NW + 1) * 32, 1) chunk_s
   }
 }
 
-template <int KD, int VD, int G>
+// Splits per (token group, KV head, batch row): the decode's bound with every
+// token group counted as a batch row of its own.
+int chunk_max_splits(int B, int M, int cap, int HQ, int H, int chunk) {
+  const int ntg = (M + 16 / (HQ / H) - 1) / (16 / (HQ / H));
+  const long groups = static_cast<long>(B) * ntg;
+  return decode_max_splits(groups > 0x7fffffffL ? 0x7fffffff : static_cast<int>(groups), cap, HQ,
+                           H, chunk);
+}
+
+template <int KD, int VD, int G, typename T>
 cudaError_t chunk_split_impl(const ChunkArgs& a, const void* qh, const float* AQ, const int* wide,
                              float* lse, float* part, cudaStream_t st) {
-  using D = MultiCfg<KD, VD, G>;
+  using D = MultiCfg<KD, VD, G, sizeof(T)>;
+  constexpr CUtensorMapDataType TD =
+      sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  constexpr cuuint64_t ES = sizeof(T);
   CUtensorMap tmK, tmV;
   // the maps end at the chunk's last row: rows past it arrive as zeros
   const cuuint64_t rows = static_cast<cuuint64_t>(a.t0) + a.M;
   {
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(KD), static_cast<cuuint64_t>(a.HQ), rows,
                                 static_cast<cuuint64_t>(a.B)};
-    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(KD) * 2,
-                                   static_cast<cuuint64_t>(a.HQ) * KD * 2,
-                                   static_cast<cuuint64_t>(a.cap) * a.HQ * KD * 2};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(KD) * ES,
+                                   static_cast<cuuint64_t>(a.HQ) * KD * ES,
+                                   static_cast<cuuint64_t>(a.cap) * a.HQ * KD * ES};
     const cuuint32_t box[4] = {static_cast<cuuint32_t>(KD), static_cast<cuuint32_t>(G),
                                static_cast<cuuint32_t>(D::SR), 1};
-    if (!encode_tiled(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.k_tilde, dims, strides, box,
-                      CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!encode_tiled(&tmK, TD, 4, a.k_tilde, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   }
   {
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(VD), static_cast<cuuint64_t>(a.H), rows,
                                 static_cast<cuuint64_t>(a.B)};
-    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(VD) * 2,
-                                   static_cast<cuuint64_t>(a.H) * VD * 2,
-                                   static_cast<cuuint64_t>(a.cap) * a.H * VD * 2};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(VD) * ES,
+                                   static_cast<cuuint64_t>(a.H) * VD * ES,
+                                   static_cast<cuuint64_t>(a.cap) * a.H * VD * ES};
     const cuuint32_t box[4] = {static_cast<cuuint32_t>(VD), 1, static_cast<cuuint32_t>(D::SR), 1};
-    if (!encode_tiled(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.v_cache, dims, strides, box,
-                      CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!encode_tiled(&tmV, TD, 4, a.v_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   }
-  auto kern = chunk_split_kernel<KD, VD, G>;
+  auto kern = chunk_split_kernel<KD, VD, G, T>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, D::SMEM);
   if (e != cudaSuccess) return e;
   const int T_b = a.t0 + a.M;
@@ -412,55 +449,62 @@ cudaError_t chunk_split_impl(const ChunkArgs& a, const void* qh, const float* AQ
   const int nch = (T_b + a.chunk - 1) / a.chunk - ck_lo;
   const int ntg = (a.M + D::MQ - 1) / D::MQ;
   int ns = decode_num_splits(a.B * ntg, nch * a.chunk, a.HQ, a.H, a.chunk);
-  const int ns_cap = decode_max_splits(a.B, a.cap, a.HQ, a.H, a.chunk);
+  const int ns_cap = chunk_max_splits(a.B, a.M, a.cap, a.HQ, a.H, a.chunk);
   if (ns > ns_cap) ns = ns_cap;
   const int cps = (nch + ns - 1) / ns;
   const int nsplit = (nch + cps - 1) / cps;
   dim3 grid(nsplit * ntg, a.H, a.B);
   if (a.ev_mid != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(a.ev_mid), st);
   kern<<<grid, (D::NW + 1) * 32, D::SMEM, st>>>(
-      tmK, tmV, static_cast<const __nv_bfloat16*>(qh), AQ, a.r_cache, a.t0, a.M, a.HQ, a.chunk,
-      a.cap, a.window, ck_lo, cps, nsplit, ntg, a.scale * kLog2e, part, a.err, a.wait_ns, wide,
-      a.fault, a.gs_cache);
+      tmK, tmV, static_cast<const T*>(qh), AQ, a.r_cache, a.t0, a.M, a.HQ, a.chunk, a.cap,
+      a.window, ck_lo, cps, nsplit, ntg, a.scale * kLog2e, part, a.err, a.wait_ns, wide, a.fault,
+      a.gs_cache);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_decode_combine_bf16(part, nsplit, a.B * a.M * a.HQ, a.HQ, a.sink, a.o, lse, VD,
-                                    st);
+  return launch_decode_combine(part, nsplit, a.B * a.M * a.HQ, a.HQ, a.sink, a.o, lse, VD,
+                               sizeof(T) == 2, st);
 }
 
-template <int KD, int VD>
+template <int KD, int VD, typename T>
 cudaError_t chunk_split_by_group(const ChunkArgs& a, const void* qh, const float* AQ,
                                  const int* wide, float* lse, float* part, cudaStream_t st) {
   switch (a.HQ / a.H) {
-    case 1: return chunk_split_impl<KD, VD, 1>(a, qh, AQ, wide, lse, part, st);
-    case 2: return chunk_split_impl<KD, VD, 2>(a, qh, AQ, wide, lse, part, st);
-    case 4: return chunk_split_impl<KD, VD, 4>(a, qh, AQ, wide, lse, part, st);
-    case 8: return chunk_split_impl<KD, VD, 8>(a, qh, AQ, wide, lse, part, st);
-    case 16: return chunk_split_impl<KD, VD, 16>(a, qh, AQ, wide, lse, part, st);
+    case 1: return chunk_split_impl<KD, VD, 1, T>(a, qh, AQ, wide, lse, part, st);
+    case 2: return chunk_split_impl<KD, VD, 2, T>(a, qh, AQ, wide, lse, part, st);
+    case 4: return chunk_split_impl<KD, VD, 4, T>(a, qh, AQ, wide, lse, part, st);
+    case 8: return chunk_split_impl<KD, VD, 8, T>(a, qh, AQ, wide, lse, part, st);
+    case 16: return chunk_split_impl<KD, VD, 16, T>(a, qh, AQ, wide, lse, part, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
+template <typename T>
+cudaError_t chunk_split_by_dims(const ChunkArgs& a, const void* qh, const float* AQ,
+                                const int* wide, float* lse, float* part, cudaStream_t st) {
+  if (a.K == 64 && a.V == 64) return chunk_split_by_group<64, 64, T>(a, qh, AQ, wide, lse, part, st);
+  if (a.K == 64 && a.V == 128) return chunk_split_by_group<64, 128, T>(a, qh, AQ, wide, lse, part, st);
+  if (a.K == 128 && a.V == 64) return chunk_split_by_group<128, 64, T>(a, qh, AQ, wide, lse, part, st);
+  if (a.K == 128 && a.V == 128) return chunk_split_by_group<128, 128, T>(a, qh, AQ, wide, lse, part, st);
+  return cudaErrorInvalidValue;
+}
+
 }  // namespace
 
-bool chunk_split_applies(int M, int HQ, int H) {
+bool chunk_split_applies(int M, int HQ, int H, bool bf16) {
   const int g = HQ / H;
   const bool pow2 = g == 1 || g == 2 || g == 4 || g == 8 || g == 16;
-  return pow2 && M >= 1 && M <= 2 * (16 / g);
+  return pow2 && M >= 1 && (!bf16 || M <= 2 * (16 / g));
 }
 
 size_t chunk_split_part_bytes(int B, int M, int cap, int HQ, int H, int V, int chunk) {
-  return static_cast<size_t>(B) * M * HQ * decode_max_splits(B, cap, HQ, H, chunk) * (V + 2) *
+  return static_cast<size_t>(B) * M * HQ * chunk_max_splits(B, M, cap, HQ, H, chunk) * (V + 2) *
          sizeof(float);
 }
 
 cudaError_t launch_chunk_split(const ChunkArgs& a, const void* qh, const float* AQ,
                                const int* wide, float* lse, float* part, cudaStream_t st) {
-  if (a.K == 64 && a.V == 64) return chunk_split_by_group<64, 64>(a, qh, AQ, wide, lse, part, st);
-  if (a.K == 64 && a.V == 128) return chunk_split_by_group<64, 128>(a, qh, AQ, wide, lse, part, st);
-  if (a.K == 128 && a.V == 64) return chunk_split_by_group<128, 64>(a, qh, AQ, wide, lse, part, st);
-  if (a.K == 128 && a.V == 128) return chunk_split_by_group<128, 128>(a, qh, AQ, wide, lse, part, st);
-  return cudaErrorInvalidValue;
+  return a.bf16 ? chunk_split_by_dims<__nv_bfloat16>(a, qh, AQ, wide, lse, part, st)
+                : chunk_split_by_dims<float>(a, qh, AQ, wide, lse, part, st);
 }
 
 }  // namespace wall

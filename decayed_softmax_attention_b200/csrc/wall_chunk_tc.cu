@@ -542,23 +542,21 @@ struct ChunkPrepCfg {
   static constexpr int RPG = 256 / RG;     // rows per row group
 };
 
-template <int KD>
-__device__ __forceinline__ void chunk_rowgroup_sum(const __nv_bfloat16* gb, size_t rstep, int r0,
-                                                   int r1, float* acc) {
+template <int KD, typename T>
+__device__ __forceinline__ void chunk_rowgroup_sum(const T* gb, size_t rstep, int r0, int r1,
+                                                   float* acc) {
 #pragma unroll 4
   for (int r = r0; r < r1; ++r) {
-    const uint2 gu = *reinterpret_cast<const uint2*>(gb + r * rstep);
-    acc[0] = fmaf(bf16_lo(gu.x), kLog2e, acc[0]);
-    acc[1] = fmaf(bf16_hi(gu.x), kLog2e, acc[1]);
-    acc[2] = fmaf(bf16_lo(gu.y), kLog2e, acc[2]);
-    acc[3] = fmaf(bf16_hi(gu.y), kLog2e, acc[3]);
+    float gv[4];
+    load4(gb + r * rstep, gv);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[c] = fmaf(gv[c], kLog2e, acc[c]);
   }
 }
 
-template <int KD>
-__global__ void __launch_bounds__(256) chunk_sum_kernel(const __nv_bfloat16* __restrict__ g,
-                                                        int M, int HQ, int NQB,
-                                                        float* __restrict__ bsum) {
+template <int KD, typename T>
+__global__ void __launch_bounds__(256) chunk_sum_kernel(const T* __restrict__ g, int M, int HQ,
+                                                        int NQB, float* __restrict__ bsum) {
   using PC = ChunkPrepCfg<KD>;
   __shared__ float tot[PC::RG][KD];
   const int blk = blockIdx.x, bh = blockIdx.y, b = bh / HQ, hq = bh % HQ;
@@ -578,11 +576,13 @@ __global__ void __launch_bounds__(256) chunk_sum_kernel(const __nv_bfloat16* __r
   }
 }
 
-template <int KD>
+// qh is written in the input's type (bf16 feeds the tensor-core tiles, fp32
+// the exact split pass).
+template <int KD, typename T>
 __global__ void __launch_bounds__(256) chunk_apply_kernel(
-    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ g,
-    const float* __restrict__ p_prev, const float* __restrict__ bsum, int M, int t0, int HQ,
-    int NQB, __nv_bfloat16* __restrict__ qh, float* __restrict__ AQ, int* __restrict__ wide) {
+    const T* __restrict__ q, const T* __restrict__ g, const float* __restrict__ p_prev,
+    const float* __restrict__ bsum, int M, int t0, int HQ, int NQB, T* __restrict__ qh,
+    float* __restrict__ AQ, int* __restrict__ wide) {
   using PC = ChunkPrepCfg<KD>;
   __shared__ float tot[PC::RG][KD];
   __shared__ int s_span;  // largest |P_i - AQ| of the block (float bits), log2 units
@@ -591,8 +591,8 @@ __global__ void __launch_bounds__(256) chunk_apply_kernel(
   const int cg = threadIdx.x % PC::CG, rg = threadIdx.x / PC::CG;
   const int r0 = blk * 256 + rg * PC::RPG, r1 = min(M, r0 + PC::RPG);
   const size_t rstep = static_cast<size_t>(HQ) * KD;
-  const __nv_bfloat16* gb = g + (static_cast<size_t>(b) * M * HQ + hq) * KD + cg * 4;
-  const __nv_bfloat16* qb = q + (static_cast<size_t>(b) * M * HQ + hq) * KD + cg * 4;
+  const T* gb = g + (static_cast<size_t>(b) * M * HQ + hq) * KD + cg * 4;
+  const T* qb = q + (static_cast<size_t>(b) * M * HQ + hq) * KD + cg * 4;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   chunk_rowgroup_sum<KD>(gb, rstep, r0, r1, acc);
 #pragma unroll
@@ -614,25 +614,20 @@ __global__ void __launch_bounds__(256) chunk_apply_kernel(
     for (int r = 0; r < rg; ++r) pre += tot[r][cg * 4 + c];
     loc[c] = pre;
   }
-  __nv_bfloat16* ob = qh + static_cast<size_t>(bh) * M * KD + cg * 4;
+  T* ob = qh + static_cast<size_t>(bh) * M * KD + cg * 4;
   float span = 0.f;
 #pragma unroll 4
   for (int r = r0; r < r1; ++r) {
-    const uint2 gu = *reinterpret_cast<const uint2*>(gb + r * rstep);
-    const uint2 qu = *reinterpret_cast<const uint2*>(qb + r * rstep);
-    const float gv[4] = {bf16_lo(gu.x), bf16_hi(gu.x), bf16_lo(gu.y), bf16_hi(gu.y)};
-    const float qv[4] = {bf16_lo(qu.x), bf16_hi(qu.x), bf16_lo(qu.y), bf16_hi(qu.y)};
-    float o4[4];
+    float gv[4], qv[4], o4[4];
+    load4(gb + r * rstep, gv);
+    load4(qb + r * rstep, qv);
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       loc[c] = fmaf(gv[c], kLog2e, loc[c]);
       span = fmaxf(span, fabsf(loc[c]));
       o4[c] = qv[c] * ex2_approx(loc[c]);
     }
-    uint2 ou;
-    ou.x = pack_bf16(o4[0], o4[1]);
-    ou.y = pack_bf16(o4[2], o4[3]);
-    *reinterpret_cast<uint2*>(ob + static_cast<size_t>(r) * KD) = ou;
+    store4(ob + static_cast<size_t>(r) * KD, o4);
   }
   // The block's own cache chunks carry anchors P at rows inside it, so the
   // factor exp2(AQ - R_c) spans the same range as the query factor.
@@ -725,30 +720,32 @@ size_t align256c(size_t x) { return (x + 255) / 256 * 256; }
 
 }  // namespace
 
-size_t chunk_workspace_bytes(int B, int M, int cap, int HQ, int H, int K, int V, int chunk) {
+size_t chunk_workspace_bytes(int B, int M, int cap, int HQ, int H, int K, int V, int chunk,
+                             bool bf16) {
   const size_t BHQ = static_cast<size_t>(B) * HQ;
   const size_t NQB = (static_cast<size_t>(M) + 255) / 256;
-  const size_t prep = align256c(BHQ * M * K * 2) + 2 * align256c(BHQ * NQB * K * 4) +
+  const size_t es = bf16 ? 2 : 4;
+  const size_t prep = align256c(BHQ * M * K * es) + 2 * align256c(BHQ * NQB * K * 4) +
                       align256c(BHQ * NQB * 4) + align256c(BHQ * M * 4);
-  return prep + (chunk_split_applies(M, HQ, H)
+  return prep + (chunk_split_applies(M, HQ, H, bf16)
                      ? align256c(chunk_split_part_bytes(B, M, cap, HQ, H, V, chunk))
                      : 0);
 }
 
-template <int KD>
+template <int KD, typename T>
 cudaError_t chunk_prep(const ChunkArgs& a, void* qh, float* AQ, float* bsum, int* wide,
                        cudaStream_t st) {
   const int NQB = (a.M + 255) / 256;
   const dim3 grid(NQB, a.B * a.HQ);
-  const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(a.g_new);
+  const T* g = static_cast<const T*>(a.g_new);
   if (NQB > 1) {
-    chunk_sum_kernel<KD><<<grid, 256, 0, st>>>(g, a.M, a.HQ, NQB, bsum);
+    chunk_sum_kernel<KD, T><<<grid, 256, 0, st>>>(g, a.M, a.HQ, NQB, bsum);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  chunk_apply_kernel<KD><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.q), g,
-                                               a.p_prev, bsum, a.M, a.t0, a.HQ, NQB,
-                                               static_cast<__nv_bfloat16*>(qh), AQ, wide);
+  chunk_apply_kernel<KD, T><<<grid, 256, 0, st>>>(static_cast<const T*>(a.q), g, a.p_prev, bsum,
+                                                  a.M, a.t0, a.HQ, NQB, static_cast<T*>(qh), AQ,
+                                                  wide);
   return cudaGetLastError();
 }
 
@@ -757,7 +754,7 @@ cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t st) {
   const size_t BHQ = static_cast<size_t>(a.B) * a.HQ;
   const size_t NQB = (static_cast<size_t>(a.M) + 255) / 256;
   void* qh = ws;
-  char* cur = ws + align256c(BHQ * a.M * a.K * 2);
+  char* cur = ws + align256c(BHQ * a.M * a.K * (a.bf16 ? 2 : 4));
   float* AQ = reinterpret_cast<float*>(cur);
   cur += align256c(BHQ * NQB * a.K * 4);
   float* bsum = reinterpret_cast<float*>(cur);
@@ -768,8 +765,13 @@ cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t st) {
   cur += align256c(BHQ * a.M * 4);
   // 1. the chunk's queries, anchored (reads p_prev before the append below
   //    overwrites p_last, which may be the same buffer)
-  cudaError_t e = a.K == 64 ? chunk_prep<64>(a, qh, AQ, bsum, wide, st)
-                            : chunk_prep<128>(a, qh, AQ, bsum, wide, st);
+  cudaError_t e;
+  if (a.bf16)
+    e = a.K == 64 ? chunk_prep<64, __nv_bfloat16>(a, qh, AQ, bsum, wide, st)
+                  : chunk_prep<128, __nv_bfloat16>(a, qh, AQ, bsum, wide, st);
+  else
+    e = a.K == 64 ? chunk_prep<64, float>(a, qh, AQ, bsum, wide, st)
+                  : chunk_prep<128, float>(a, qh, AQ, bsum, wide, st);
   if (e != cudaSuccess) return e;
   // 2. the chunk's keys join the cache (rows t0 .. t0 + M - 1)
   CacheArgs c;
@@ -778,7 +780,7 @@ cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t st) {
   c.chunk = a.chunk; c.k_tilde = a.k_tilde; c.r_cache = a.r_cache; c.p_last = a.p_last;
   c.err = a.err; c.wait_ns = a.wait_ns; c.fault = 0;
   c.pm.cap = a.cap;
-  e = launch_cache_build(c, true, st);
+  e = launch_cache_build(c, a.bf16, st);
   if (e != cudaSuccess) return e;
   if (a.gs_new != nullptr) {  // the chunk's gate prefixes join the gate cache
     GateArgs ga;
@@ -786,13 +788,16 @@ cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t st) {
     ga.B = a.B; ga.t_start = a.t0; ga.T_new = a.M; ga.HQ = a.HQ;
     ga.gcache = a.gs_cache; ga.gs_last = a.gs_last;
     ga.pm.cap = a.cap;
-    e = launch_gate_cache(ga, true, st);
+    e = launch_gate_cache(ga, a.bf16, st);
     if (e != cudaSuccess) return e;
   }
-  // 3. the chunk's queries attend the cache: a few tokens per sequence the
-  //    decode's way, longer chunks in 128-row tensor-core query tiles
-  if (chunk_split_applies(a.M, a.HQ, a.H)) {
+  // 3. the chunk's queries attend the cache: a few tokens per sequence (and
+  //    fp32 chunks of any length) the decode's way, longer bf16 chunks in
+  //    128-row tensor-core query tiles
+  if (chunk_split_applies(a.M, a.HQ, a.H, a.bf16)) {
     e = launch_chunk_split(a, qh, AQ, wide, lse, reinterpret_cast<float*>(cur), st);
+  } else if (!a.bf16) {
+    return cudaErrorInvalidValue;
   } else if (a.K == 64 && a.V == 64) {
     e = chunk_by_c<64, 64>(a, qh, AQ, wide, lse, st);
   } else if (a.K == 64 && a.V == 128) {
@@ -813,7 +818,7 @@ cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t st) {
   d.B = a.B; d.Tb = a.M; d.HQ = a.HQ; d.H = a.H; d.NQB = static_cast<int>(NQB);
   d.vT = a.cap; d.voff = a.t0; d.pos0 = a.t0;
   d.scale = a.scale; d.o = a.o; d.lse = lse;
-  return launch_diag(d, true, a.K, a.V, st);
+  return launch_diag(d, a.bf16, a.K, a.V, st);
 }
 
 }  // namespace wall

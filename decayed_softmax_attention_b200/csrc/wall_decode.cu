@@ -641,17 +641,24 @@ size_t decode_workspace_bytes(int B, int HQ, int V, int nsplit) {
   return static_cast<size_t>(B) * HQ * nsplit * (V + 2) * sizeof(float);
 }
 
-cudaError_t launch_decode_combine_bf16(const float* part, int nsplit, int nbh, int HQ,
-                                      const float* sink, void* o, float* lse, int V,
-                                      cudaStream_t st) {
+cudaError_t launch_decode_combine(const float* part, int nsplit, int nbh, int HQ,
+                                  const float* sink, void* o, float* lse, int V, bool bf16,
+                                  cudaStream_t st) {
   const unsigned grid = static_cast<unsigned>((nbh + 3) / 4);
-  __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(o);
-  if (V == 64)
-    decode_combine_kernel<__nv_bfloat16, 64><<<grid, 128, 0, st>>>(part, nsplit, nbh, HQ, sink, ob, lse);
-  else if (V == 128)
-    decode_combine_kernel<__nv_bfloat16, 128><<<grid, 128, 0, st>>>(part, nsplit, nbh, HQ, sink, ob, lse);
-  else
-    return cudaErrorInvalidValue;
+  if (V != 64 && V != 128) return cudaErrorInvalidValue;
+  if (bf16) {
+    __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(o);
+    if (V == 64)
+      decode_combine_kernel<__nv_bfloat16, 64><<<grid, 128, 0, st>>>(part, nsplit, nbh, HQ, sink, ob, lse);
+    else
+      decode_combine_kernel<__nv_bfloat16, 128><<<grid, 128, 0, st>>>(part, nsplit, nbh, HQ, sink, ob, lse);
+  } else {
+    float* of = static_cast<float*>(o);
+    if (V == 64)
+      decode_combine_kernel<float, 64><<<grid, 128, 0, st>>>(part, nsplit, nbh, HQ, sink, of, lse);
+    else
+      decode_combine_kernel<float, 128><<<grid, 128, 0, st>>>(part, nsplit, nbh, HQ, sink, of, lse);
+  }
   return cudaGetLastError();
 }
 

@@ -231,6 +231,7 @@ struct ChunkArgs {
   const float* sink;
   int window;
   int B, t0, M, cap, HQ, H, K, V, chunk;
+  bool bf16;           // element type of q, k_new, g_new, gs_new, k_tilde, v_cache, o
   float scale;
   void* k_tilde;       // [B, cap, HQ, K]
   float* r_cache;      // [B, ceil(cap/chunk), HQ, K]
@@ -251,18 +252,20 @@ struct ChunkArgs {
   float* gs_cache = nullptr;
   float* gs_last = nullptr;
 };
-size_t chunk_workspace_bytes(int B, int M, int cap, int HQ, int H, int K, int V, int chunk);
+size_t chunk_workspace_bytes(int B, int M, int cap, int HQ, int H, int K, int V, int chunk,
+                             bool bf16);
 cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t st);
-// Few-token chunks (M <= 2 * 16 / group) attend through a split-KV pass in the
-// decode's style instead of 128-row tensor-core query tiles.
-bool chunk_split_applies(int M, int HQ, int H);
+// Few-token bf16 chunks (M <= 2 * 16 / group) and fp32 chunks of any length
+// attend through a split-KV pass in the decode's style instead of 128-row
+// tensor-core query tiles (power-of-two groups).
+bool chunk_split_applies(int M, int HQ, int H, bool bf16);
 size_t chunk_split_part_bytes(int B, int M, int cap, int HQ, int H, int V, int chunk);
 cudaError_t launch_chunk_split(const ChunkArgs& a, const void* qh, const float* AQ,
                                const int* wide, float* lse, float* part, cudaStream_t st);
-// The decode's split combine (merge per-split partials, add the sink), bf16 output.
-cudaError_t launch_decode_combine_bf16(const float* part, int nsplit, int nbh, int HQ,
-                                      const float* sink, void* o, float* lse, int V,
-                                      cudaStream_t st);
+// The decode's split combine (merge per-split partials, add the sink).
+cudaError_t launch_decode_combine(const float* part, int nsplit, int nbh, int HQ,
+                                  const float* sink, void* o, float* lse, int V, bool bf16,
+                                  cudaStream_t st);
 
 // Append fused into the decode step: the new token's k, g, v (one per batch
 // row) join the cache inside the decode kernel.  In this mode DecodeArgs'

@@ -389,21 +389,24 @@ wall_status_t wall_attn_decode_gated(const void* q, const float* p_curr, const f
  * optional sink), with the cache's per-chunk anchors folded into tile rescales
  * (Wall Attention README "Decode" cache, the forward's score).  The result
  * equals rows t_start .. t_start + M - 1 of the prefill of the whole sequence.
- *   q        [B, M, HQ, K]   k_new [B, M, H, K]   g_new [B, M, HQ, K]   (bf16)
+ *   q        [B, M, HQ, K]   k_new [B, M, H, K]   g_new [B, M, HQ, K]   (dt)
  *   v_cache  [B, cap, H, V]  rows t_start .. t_start + M - 1 already hold the
  *            chunk's values (caller-written, as for the decode)
- *   o        [B, M, HQ, V] bf16;  lse [B, M, HQ] fp32 (nullable)
- *   workspace >= wall_attn_chunk_workspace_size(B, M, cap, HQ, H, K, V, chunk)
+ *   o        [B, M, HQ, V] dt;  lse [B, M, HQ] fp32 (nullable)
+ *   workspace >= wall_attn_chunk_workspace_size(B, M, cap, HQ, H, K, V, chunk, dt)
  *            bytes, 256-aligned
- * bf16 only (fp32: WALL_ERR_UNSUPPORTED); the scalar gate through
- * wall_attn_chunk_gated below.
- * A chunk of at most 2 * 16 / (HQ / H) tokens (multi-token decode) attends
- * through a split-KV pass that streams the cache once per KV head; longer
- * chunks through 128-row tensor-core query tiles.  Both give the same result
- * within the usual tolerance.
+ * The scalar gate goes through wall_attn_chunk_gated below.
+ * bf16: a chunk of at most 2 * 16 / (HQ / H) tokens (multi-token decode)
+ * attends through a split-KV pass that streams the cache once per KV head;
+ * longer chunks through 128-row tensor-core query tiles.  Both give the same
+ * result within the usual tolerance.
+ * fp32 (the exact path, no tensor cores): every chunk takes the split-KV pass,
+ * each group of 16 / (HQ / H) tokens streaming the cache rows it can see;
+ * HQ / H must be 1, 2, 4, 8 or 16 and B * M * HQ < 2^31, else
+ * WALL_ERR_UNSUPPORTED.
  */
 size_t wall_attn_chunk_workspace_size(int B, int M, int cap, int HQ, int H, int K, int V,
-                                      int chunk);
+                                      int chunk, wall_dtype_t dt);
 
 wall_status_t wall_attn_chunk(const void* q, const void* k_new, const void* g_new,
                               const float* p_prev, const float* sink_bias, int window, int B,
@@ -418,7 +421,7 @@ wall_status_t wall_attn_chunk(const void* q, const void* k_new, const void* g_ne
  * join the gate cache first, exactly as wall_build_gate_cache(gs_new, gs_prev,
  * t_start, ...) writes them, then query i's logit of cache row j gains
  * (PS[t_start + i] - PS[j]) ln 2.
- *   gs_new    [B, M, HQ] bf16          the chunk's g_scalar
+ *   gs_new    [B, M, HQ] dt            the chunk's g_scalar
  *   gs_prev   [B, HQ] fp32             PS at row t_start - 1 (NULL iff t_start == 0)
  *   gs_cache  [B, cap, HQ] fp32        the dense gate cache (rows t_start .. written)
  *   gs_last   [B, HQ] fp32             out: PS at the chunk's last row (may alias gs_prev)

@@ -384,22 +384,30 @@ def test_decode_step_host_validation(lib):
 
 
 def test_chunk_workspace_size(lib):
+    BF, F32 = wall.WALL_DTYPE_BF16, wall.WALL_DTYPE_F32
     # invalid shapes: 0
-    assert lib.wall_attn_chunk_workspace_size(0, 4, 1024, 32, 8, 128, 128, 64) == 0
-    assert lib.wall_attn_chunk_workspace_size(2, 4, 1024, 6, 4, 128, 128, 64) == 0  # HQ % H
+    assert lib.wall_attn_chunk_workspace_size(0, 4, 1024, 32, 8, 128, 128, 64, BF) == 0
+    assert lib.wall_attn_chunk_workspace_size(2, 4, 1024, 6, 4, 128, 128, 64, BF) == 0  # HQ % H
     # a few tokens per sequence (group 4: up to 8) also hold the split-KV partials, which
     # grow with the cache capacity; longer chunks need only the anchored queries
-    small = [lib.wall_attn_chunk_workspace_size(32, 4, cap, 32, 8, 128, 128, 64)
+    small = [lib.wall_attn_chunk_workspace_size(32, 4, cap, 32, 8, 128, 128, 64, BF)
              for cap in (64, 1024, 32832)]
     assert small[0] <= small[1] <= small[2]
     prep4 = 32 * 32 * 4 * 128 * 2
     assert small[2] > prep4 + 32 * 4 * 32 * 130 * 4   # at least one split's partials
-    big = [lib.wall_attn_chunk_workspace_size(1, 1024, cap, 32, 8, 128, 128, 64)
+    big = [lib.wall_attn_chunk_workspace_size(1, 1024, cap, 32, 8, 128, 128, 64, BF)
            for cap in (1024, 32832)]
     assert big[0] == big[1]
     # the bound: 2 * 16 / group tokens (group 16: 2 tokens; 3 take the tensor-core tiles)
-    g16 = [lib.wall_attn_chunk_workspace_size(1, m, 32832, 16, 1, 128, 128, 64) for m in (2, 3)]
+    g16 = [lib.wall_attn_chunk_workspace_size(1, m, 32832, 16, 1, 128, 128, 64, BF)
+           for m in (2, 3)]
     assert g16[0] > g16[1]
+    # fp32 chunks of any length take the split pass: fp32 anchored queries plus one
+    # partial (V + 2 floats) per token, query head and split, at least one split
+    for M in (3, 1024):
+        f = lib.wall_attn_chunk_workspace_size(1, M, 32832, 16, 1, 128, 128, 64, F32)
+        assert f >= 16 * M * 128 * 4 + 16 * M * 130 * 4
+        assert f > lib.wall_attn_chunk_workspace_size(1, M, 32832, 16, 1, 128, 128, 64, BF)
 
 
 def test_new_calls_fail_loudly_without_cuda_tensors():

@@ -12,6 +12,10 @@ speculative verification) take the split-KV pass instead of the tensor-core
 query tiles; FEW_CASES run every group size on both sides of that bound, with
 one and two token groups per CTA, a partly filled second group, windows that
 skip whole anchor chunks and enough prefix chunks for several splits.
+
+fp32 caches take the split-KV pass for chunks of every length (F32_CASES):
+chunks spanning several 256-row query blocks, every group size, windows, the
+scalar gate and wide blocks (strong decay) inside a long chunk.
 """
 import numpy as np
 import pytest
@@ -164,3 +168,68 @@ def test_gated_chunks_reproduce_the_prefill(wall, case):
     PS = oracle.gate_cache(d["g_scalar"])
     np.testing.assert_allclose(gsc[:, :T].double().cpu().numpy(), PS, rtol=2e-6, atol=2e-5)
     np.testing.assert_allclose(gsl.double().cpu().numpy(), PS[:, -1], rtol=2e-6, atol=2e-5)
+
+
+F32_CASES = [
+    dict(B=2, sizes=(600, 300, 1, 5), HQ=8, H=2, K=128, V=128, C=64, window=0, sink=True,
+         g_kind="negsoftplus", gate=False),
+    dict(B=1, sizes=(513, 2, 270), HQ=2, H=2, K=64, V=64, C=32, window=0, sink=False,
+         g_kind="negsoftplus", gate=True),
+    dict(B=2, sizes=(333, 444), HQ=4, H=2, K=128, V=64, C=128, window=200, sink=True,
+         g_kind="negsoftplus", gate=False),
+    dict(B=1, sizes=(260, 31, 600), HQ=16, H=1, K=64, V=128, C=64, window=0, sink=True,
+         g_kind="negsoftplus", gate=True),
+    dict(B=1, sizes=(700, 300), HQ=8, H=1, K=128, V=128, C=32, window=0, sink=False,
+         g_kind="strong_cache", gate=True),  # wide blocks inside long fp32 chunks
+]
+
+
+@pytest.mark.parametrize("case", F32_CASES, ids=_ids)
+def test_fp32_chunks_reproduce_the_prefill(wall, case):
+    """wall_attn_chunk(_gated) with fp32 inputs and cache: every chunk length through the
+    split-KV pass, equal to the oracle's prefill rows at the fp32 tolerance."""
+    B, HQ, H, K, V, C = case["B"], case["HQ"], case["H"], case["K"], case["V"], case["C"]
+    T = sum(case["sizes"])
+    spec = W.PrefillSpec("chunk_f32", B=B, T=T, HQ=HQ, H=H, K=K, V=V, dtype="f32",
+                         g_kind=case["g_kind"], g_scalar=case["gate"], sink=case["sink"],
+                         window=case["window"], seed=104)
+    d = W.gen_prefill(spec, device="cuda")
+    cap = T + 21
+    nan = float("nan")
+    f32 = torch.float32
+    kt = torch.full((B, cap, HQ, K), nan, dtype=f32, device="cuda")
+    rc = torch.full((B, (cap + C - 1) // C, HQ, K), nan, dtype=f32, device="cuda")
+    p = torch.full((B, HQ, K), nan, dtype=f32, device="cuda")
+    vc = torch.full((B, cap, H, V), nan, dtype=f32, device="cuda")
+    gsc = torch.full((B, cap, HQ), nan, dtype=f32, device="cuda")
+    gsl = torch.full((B, HQ), nan, dtype=f32, device="cuda")
+    ro, rl = oracle.wall_fwd(d["q"], d["k"], d["v"], d["g"], d.get("g_scalar"), d["sink_bias"],
+                             window=d["window"], scale=d["scale"], threads=ORACLE_THREADS)
+    t0 = 0
+    for M in case["sizes"]:
+        sl = slice(t0, t0 + M)
+        vc[:, sl].copy_(d["v"][:, sl])
+        lse = torch.empty((B, M, HQ), dtype=f32, device="cuda")
+        gate = {}
+        if case["gate"]:
+            gate = dict(gs_new=d["g_scalar"][:, sl].contiguous(), gs_cache=gsc, gs_last=gsl)
+        o = wall.wall_attn_chunk(d["q"][:, sl].contiguous(), d["k"][:, sl].contiguous(),
+                                 d["g"][:, sl].contiguous(), kt, rc, p, vc, t0,
+                                 sink_bias=d["sink_bias"], window=d["window"], scale=d["scale"],
+                                 chunk=C, lse=lse, **gate)
+        torch.cuda.synchronize()
+        assert wall.wall_device_error() == 0
+        assert o.dtype == f32
+        assert_close(o, ro[:, sl], f32, f"fp32 chunk at {t0} (M={M})")
+        assert_close(lse, rl[:, sl], f32, f"fp32 chunk lse at {t0} (M={M})")
+        t0 += M
+    ktr, _, P = oracle.kv_cache(d["k"], d["g"], chunk=C, threads=ORACLE_THREADS)
+    # k_tilde = k 2^(R_c - P_j) from fp32 prefixes: a rounding of P (log2 units, ulp about
+    # 2^-23 |P|) moves the factor by ln 2 times it, so under strong decay (|P| in the
+    # thousands) the relative bound grows with max |P|; 16 roundings of headroom
+    rtol_k = 1e-4 + 16 * 2.0 ** -23 * np.log(2.0) * float(np.abs(P).max())
+    got = kt[:, :T].double().cpu().numpy()
+    bad = ~(np.abs(got - ktr) <= 1e-4 + rtol_k * np.abs(ktr))
+    assert not bad.any(), (f"fp32 cache built by the chunks: {int(bad.sum())} outside "
+                           f"rtol {rtol_k:.2e}, first {np.argwhere(bad)[:3].tolist()}")
+    np.testing.assert_allclose(p.double().cpu().numpy(), P[:, -1], rtol=1e-5, atol=1e-4)
