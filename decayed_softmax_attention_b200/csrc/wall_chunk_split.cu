@@ -415,33 +415,6 @@ cudaError_t chunk_split_impl(const ChunkArgs& a, const void* qh, const float* AQ
   constexpr CUtensorMapDataType TD =
       sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   constexpr cuuint64_t ES = sizeof(T);
-  CUtensorMap tmK, tmV;
-  // the maps end at the chunk's last row: rows past it arrive as zeros
-  const cuuint64_t rows = static_cast<cuuint64_t>(a.t0) + a.M;
-  {
-    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(KD), static_cast<cuuint64_t>(a.HQ), rows,
-                                static_cast<cuuint64_t>(a.B)};
-    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(KD) * ES,
-                                   static_cast<cuuint64_t>(a.HQ) * KD * ES,
-                                   static_cast<cuuint64_t>(a.cap) * a.HQ * KD * ES};
-    const cuuint32_t box[4] = {static_cast<cuuint32_t>(KD), static_cast<cuuint32_t>(G),
-                               static_cast<cuuint32_t>(D::SR), 1};
-    if (!encode_tiled(&tmK, TD, 4, a.k_tilde, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
-      return cudaErrorInvalidValue;
-  }
-  {
-    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(VD), static_cast<cuuint64_t>(a.H), rows,
-                                static_cast<cuuint64_t>(a.B)};
-    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(VD) * ES,
-                                   static_cast<cuuint64_t>(a.H) * VD * ES,
-                                   static_cast<cuuint64_t>(a.cap) * a.H * VD * ES};
-    const cuuint32_t box[4] = {static_cast<cuuint32_t>(VD), 1, static_cast<cuuint32_t>(D::SR), 1};
-    if (!encode_tiled(&tmV, TD, 4, a.v_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
-      return cudaErrorInvalidValue;
-  }
-  auto kern = chunk_split_kernel<KD, VD, G, T>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, D::SMEM);
-  if (e != cudaSuccess) return e;
   const int T_b = a.t0 + a.M;
   // chunks wholly before the first token's window are skipped
   const int lo = a.window > 0 ? (a.t0 + 1 - a.window > 0 ? a.t0 + 1 - a.window : 0) : 0;
@@ -453,13 +426,45 @@ cudaError_t chunk_split_impl(const ChunkArgs& a, const void* qh, const float* AQ
   if (ns > ns_cap) ns = ns_cap;
   const int cps = (nch + ns - 1) / ns;
   const int nsplit = (nch + cps - 1) / cps;
-  dim3 grid(nsplit * ntg, a.H, a.B);
-  if (a.ev_mid != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(a.ev_mid), st);
-  kern<<<grid, (D::NW + 1) * 32, D::SMEM, st>>>(
-      tmK, tmV, static_cast<const T*>(qh), AQ, a.r_cache, a.t0, a.M, a.HQ, a.chunk, a.cap,
-      a.window, ck_lo, cps, nsplit, ntg, a.scale * kLog2e, part, a.err, a.wait_ns, wide, a.fault,
-      a.gs_cache);
-  e = cudaGetLastError();
+  cudaError_t e;
+  if constexpr (sizeof(T) == 2 && G <= 8) {
+    e = launch_chunk_mma<KD, VD, G>(a, qh, AQ, wide, part, ck_lo, cps, nsplit, ntg, st);
+  } else {
+    CUtensorMap tmK, tmV;
+    // the maps end at the chunk's last row: rows past it arrive as zeros
+    const cuuint64_t rows = static_cast<cuuint64_t>(a.t0) + a.M;
+    {
+      const cuuint64_t dims[4] = {static_cast<cuuint64_t>(KD), static_cast<cuuint64_t>(a.HQ), rows,
+                                  static_cast<cuuint64_t>(a.B)};
+      const cuuint64_t strides[3] = {static_cast<cuuint64_t>(KD) * ES,
+                                     static_cast<cuuint64_t>(a.HQ) * KD * ES,
+                                     static_cast<cuuint64_t>(a.cap) * a.HQ * KD * ES};
+      const cuuint32_t box[4] = {static_cast<cuuint32_t>(KD), static_cast<cuuint32_t>(G),
+                                 static_cast<cuuint32_t>(D::SR), 1};
+      if (!encode_tiled(&tmK, TD, 4, a.k_tilde, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    }
+    {
+      const cuuint64_t dims[4] = {static_cast<cuuint64_t>(VD), static_cast<cuuint64_t>(a.H), rows,
+                                  static_cast<cuuint64_t>(a.B)};
+      const cuuint64_t strides[3] = {static_cast<cuuint64_t>(VD) * ES,
+                                     static_cast<cuuint64_t>(a.H) * VD * ES,
+                                     static_cast<cuuint64_t>(a.cap) * a.H * VD * ES};
+      const cuuint32_t box[4] = {static_cast<cuuint32_t>(VD), 1, static_cast<cuuint32_t>(D::SR), 1};
+      if (!encode_tiled(&tmV, TD, 4, a.v_cache, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    }
+    auto kern = chunk_split_kernel<KD, VD, G, T>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, D::SMEM);
+    if (e != cudaSuccess) return e;
+    dim3 grid(nsplit * ntg, a.H, a.B);
+    if (a.ev_mid != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(a.ev_mid), st);
+    kern<<<grid, (D::NW + 1) * 32, D::SMEM, st>>>(
+        tmK, tmV, static_cast<const T*>(qh), AQ, a.r_cache, a.t0, a.M, a.HQ, a.chunk, a.cap,
+        a.window, ck_lo, cps, nsplit, ntg, a.scale * kLog2e, part, a.err, a.wait_ns, wide,
+        a.fault, a.gs_cache);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return e;
   return launch_decode_combine(part, nsplit, a.B * a.M * a.HQ, a.HQ, a.sink, a.o, lse, VD,
                                sizeof(T) == 2, st);

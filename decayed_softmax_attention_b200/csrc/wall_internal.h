@@ -260,6 +260,12 @@ cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t st);
 // tensor-core query tiles (power-of-two groups).
 bool chunk_split_applies(int M, int HQ, int H, bool bf16);
 size_t chunk_split_part_bytes(int B, int M, int cap, int HQ, int H, int V, int chunk);
+// The split pass on the tensor cores (bf16, groups of 1, 2, 4 or 8): writes the
+// same per-split partials as the SIMT pass.
+template <int KD, int VD, int G>
+cudaError_t launch_chunk_mma(const ChunkArgs& a, const void* qh, const float* AQ, const int* wide,
+                             float* part, int ck_lo, int cps, int nsplit, int ntg,
+                             cudaStream_t st);
 cudaError_t launch_chunk_split(const ChunkArgs& a, const void* qh, const float* AQ,
                                const int* wide, float* lse, float* part, cudaStream_t st);
 // The decode's split combine (merge per-split partials, add the sink).

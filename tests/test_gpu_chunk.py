@@ -233,3 +233,35 @@ def test_fp32_chunks_reproduce_the_prefill(wall, case):
     assert not bad.any(), (f"fp32 cache built by the chunks: {int(bad.sum())} outside "
                            f"rtol {rtol_k:.2e}, first {np.argwhere(bad)[:3].tolist()}")
     np.testing.assert_allclose(p.double().cpu().numpy(), P[:, -1], rtol=1e-5, atol=1e-4)
+
+
+def test_four_token_chunk_full_decode_workload(wall):
+    """The benchmark's multi-token decode at full size (B=32, T_kv=32768 prefix, HQ=32, H=8,
+    K=V=128, C=64, 4 new tokens per sequence through the tensor-core split pass): batch rows
+    0 and 31 against the oracle's prefill rows of the 4 tokens."""
+    spec = W.DECODE["decode"]
+    Mt = 4
+    d = W.gen_decode(spec, device="cuda")
+    B, T0, HQ, H, K, V = spec.B, spec.T0, spec.HQ, spec.H, spec.K, spec.V
+    cache = wall.KVCache(B, spec.cap, HQ, H, K, V, dtype=torch.bfloat16, chunk=spec.C)
+    cache.append(d["k"][:, :T0].contiguous(), d["g"][:, :T0].contiguous(),
+                 d["v"][:, :T0].contiguous())
+    sl = slice(T0, T0 + Mt)
+    cache.v[:, sl].copy_(d["v"][:, sl])
+    q4 = d["q"][:, :Mt].contiguous()
+    lse = torch.empty((B, Mt, HQ), dtype=torch.float32, device="cuda")
+    o = wall.wall_attn_chunk(q4, d["k"][:, sl].contiguous(), d["g"][:, sl].contiguous(),
+                             cache.k_tilde, cache.r_cache, cache.p, cache.v, T0,
+                             scale=d["scale"], chunk=spec.C, lse=lse)
+    torch.cuda.synchronize()
+    assert wall.wall_device_error() == 0
+    T = T0 + Mt
+    for b in (0, 31):
+        qf = torch.zeros((1, T, HQ, K), dtype=torch.bfloat16)
+        qf[0, sl] = q4[b].cpu()
+        rows = np.arange(T0, T, dtype=np.int64)
+        ro, rl = oracle.wall_fwd(qf, d["k"][b:b + 1, :T].cpu(), d["v"][b:b + 1, :T].cpu(),
+                                 d["g"][b:b + 1, :T].cpu(), scale=d["scale"], rows=rows,
+                                 threads=ORACLE_THREADS)
+        assert_close(o[b], ro.reshape(Mt, HQ, V), torch.bfloat16, f"4-token chunk b={b}")
+        assert_close(lse[b], rl.reshape(Mt, HQ), torch.bfloat16, f"4-token chunk lse b={b}")
