@@ -493,8 +493,10 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
   if (lse != nullptr && lane == 0) lse[bhq] = (M + log2f(Z)) * kLn2;
 }
 
+// The SIMT split pass (fp32 caches, 16-head groups; bf16 with smaller groups
+// runs on the tensor cores, wall_split_mma.cu).
 template <typename T, int KD, int VD, int G>
-cudaError_t decode_impl(const DecodeArgs& a, cudaStream_t st) {
+cudaError_t decode_split_simt(const DecodeArgs& a, cudaStream_t st) {
   using D = DecCfg<T, KD, VD, G>;
   const CUtensorMapDataType tdt =
       sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
@@ -561,7 +563,17 @@ cudaError_t decode_impl(const DecodeArgs& a, cudaStream_t st) {
       tmK, tmV, tmG, gtma, static_cast<const T*>(a.q), a.p_curr, a.r_cache, a.T_kv, a.HQ, a.chunk,
       cps, a.nsplit, a.scale * kLog2e, a.part, a.err, a.wait_ns, a.fault, a.seqlens, a.pm,
       a.gs_cache, a.gs_curr, a.fuse);
-  e = cudaGetLastError();
+  return cudaGetLastError();
+}
+
+template <typename T, int KD, int VD, int G>
+cudaError_t decode_impl(const DecodeArgs& a, cudaStream_t st) {
+  cudaError_t e;
+  if constexpr (sizeof(T) == 2 && G <= 8) {
+    e = launch_decode_mma<KD, VD, G>(a, st);
+  } else {
+    e = decode_split_simt<T, KD, VD, G>(a, st);
+  }
   if (e != cudaSuccess) return e;
   if (a.mid_event != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(a.mid_event), st);
   const int nbh = a.B * a.HQ;

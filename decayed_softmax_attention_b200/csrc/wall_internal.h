@@ -260,8 +260,8 @@ cudaError_t launch_chunk(const ChunkArgs& a, cudaStream_t st);
 // tensor-core query tiles (power-of-two groups).
 bool chunk_split_applies(int M, int HQ, int H, bool bf16);
 size_t chunk_split_part_bytes(int B, int M, int cap, int HQ, int H, int V, int chunk);
-// The split pass on the tensor cores (bf16, groups of 1, 2, 4 or 8): writes the
-// same per-split partials as the SIMT pass.
+// The few-token split pass on the tensor cores (bf16, groups of 1, 2, 4 or 8):
+// writes the same per-split partials as the SIMT pass.
 template <int KD, int VD, int G>
 cudaError_t launch_chunk_mma(const ChunkArgs& a, const void* qh, const float* AQ, const int* wide,
                              float* part, int ck_lo, int cps, int nsplit, int ntg,
@@ -319,5 +319,10 @@ int decode_num_splits(int B, int T_kv, int HQ, int H, int chunk);
 size_t decode_workspace_bytes(int B, int HQ, int V, int nsplit);
 bool decode_supported(int K, int V, int group);
 cudaError_t launch_decode(const DecodeArgs& a, bool bf16, cudaStream_t st);
+// The decode's split pass on the tensor cores (bf16, groups of 1, 2, 4 or 8):
+// writes the same per-split partials as the SIMT split kernel (the combine
+// is the caller's).
+template <int KD, int VD, int G>
+cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t st);
 
 }  // namespace wall
