@@ -61,7 +61,7 @@ TRAFFIC = {
 }
 KERNEL_SOURCES = {
     "prefill_main": "decayed_softmax_attention_b200/csrc/wall_fwd_tc.cu",
-    "decode_split": "decayed_softmax_attention_b200/csrc/wall_decode.cu",
+    "decode_split": "decayed_softmax_attention_b200/csrc/wall_split_mma.cu",
     "cache_build": "decayed_softmax_attention_b200/csrc/wall_cache.cu",
 }
 
@@ -702,7 +702,8 @@ def run_ours(args, world, rank, local):
             "metric": f"wall_attn_decode KV GB/s (B={dspec.B}, T_kv {T0 + 1}..{T0 + S})",
             "value": dec_value, "unit": "GB/s",
             "ms_per_token": statistics.mean(x for r in dec_ms for x in r),
-            "roofline": {"kernel": "decode_split_kernel", "bound": "hbm", "achieved": dec_achieved,
+            "roofline": {"kernel": "split_mma_kernel (decode split pass, fused append)",
+                         "bound": "hbm", "achieved": dec_achieved,
                          "peak": hbm_peak, "unit": "GB/s", "frac": dec_achieved / hbm_peak,
                          "traffic": traffic_for("decode_split"),
                          "peak_source": f"{peak_src} hbm_gbs",

@@ -493,7 +493,8 @@ static wall_status_t decode_entry(const void* q, const float* p_curr, const void
       if (g0 != nullptr && g0 < g1 + gb && g1 < g0 + gb) return WALL_ERR_INVALID_ARG;
     }
   }
-  const int ns = wall::decode_num_splits(B, T_kv, HQ, H, chunk);
+  const int ns = wall::decode_num_splits(
+      B, T_kv, HQ, H, chunk, wall::decode_ctas_per_sm(K, V, HQ / H, dt == WALL_DTYPE_BF16));
   if (workspace_bytes < wall::decode_workspace_bytes(B, HQ, V, ns)) return WALL_ERR_WORKSPACE;
   if (!(scale > 0.f) || !std::isfinite(scale)) scale = 1.f / std::sqrt(static_cast<float>(K));
   wall::DecodeArgs a;

@@ -421,7 +421,8 @@ cudaError_t chunk_split_impl(const ChunkArgs& a, const void* qh, const float* AQ
   const int ck_lo = lo / a.chunk;
   const int nch = (T_b + a.chunk - 1) / a.chunk - ck_lo;
   const int ntg = (a.M + D::MQ - 1) / D::MQ;
-  int ns = decode_num_splits(a.B * ntg, nch * a.chunk, a.HQ, a.H, a.chunk);
+  int ns = decode_num_splits(a.B * ntg, nch * a.chunk, a.HQ, a.H, a.chunk,
+                             decode_ctas_per_sm(KD, VD, G, sizeof(T) == 2));
   const int ns_cap = chunk_max_splits(a.B, a.M, a.cap, a.HQ, a.H, a.chunk);
   if (ns > ns_cap) ns = ns_cap;
   const int cps = (nch + ns - 1) / ns;

@@ -624,14 +624,14 @@ int decode_max_splits(int B, int T_kv, int HQ, int H, int chunk) {
   return static_cast<int>(ns);
 }
 
-// Splits actually launched (one CTA per SM is resident): the count up to the
-// bound whose CTAs fill the last wave best, preferring fewer splits; chunks are
-// dealt out evenly so no split is empty.
-int decode_num_splits(int B, int T_kv, int HQ, int H, int chunk) {
+// Splits actually launched (ctas_per_sm CTAs of the split pass are resident on
+// an SM): the count up to the bound whose CTAs fill the last wave best,
+// preferring fewer splits; chunks are dealt out evenly so no split is empty.
+int decode_num_splits(int B, int T_kv, int HQ, int H, int chunk, int ctas_per_sm) {
   const int ns_max = decode_max_splits(B, T_kv, HQ, H, chunk);
   const int nchunks = (T_kv + chunk - 1) / chunk;
   const long groups = static_cast<long>(B) * H;
-  const long sms = 148;
+  const long sms = 148L * (ctas_per_sm > 0 ? ctas_per_sm : 1);
   int best = 1;
   double best_eff = -1.0;
   for (int ns = 1; ns <= ns_max; ++ns) {

@@ -67,7 +67,8 @@ extern "C" wall_status_t wall_attn_decode_noalloc(
   const size_t fit = kScratchFloats / per_split;
   if (fit < 1) return WALL_ERR_WORKSPACE;
   const int nchunks = (T_kv + chunk - 1) / chunk;
-  int ns = wall::decode_num_splits(B, T_kv, HQ, H, chunk);
+  int ns = wall::decode_num_splits(B, T_kv, HQ, H, chunk,
+                                   wall::decode_ctas_per_sm(K, V, HQ / H, dt == WALL_DTYPE_BF16));
   if (static_cast<size_t>(ns) > fit) {
     const int capped = static_cast<int>(fit);
     const int cps = (nchunks + capped - 1) / capped;

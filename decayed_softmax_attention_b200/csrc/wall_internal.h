@@ -315,7 +315,10 @@ struct DecodeArgs {
   const float* gs_curr = nullptr;   // [B, HQ] PS of the current row
 };
 int decode_max_splits(int B, int T_kv, int HQ, int H, int chunk);
-int decode_num_splits(int B, int T_kv, int HQ, int H, int chunk);
+int decode_num_splits(int B, int T_kv, int HQ, int H, int chunk, int ctas_per_sm = 1);
+// CTAs of the decode's split pass resident on an SM: the tensor-core pass
+// (bf16, groups of 1-8) runs several small CTAs, the SIMT pass one.
+int decode_ctas_per_sm(int K, int V, int group, bool bf16);
 size_t decode_workspace_bytes(int B, int HQ, int V, int nsplit);
 bool decode_supported(int K, int V, int group);
 cudaError_t launch_decode(const DecodeArgs& a, bool bf16, cudaStream_t st);

@@ -36,6 +36,8 @@
 // (P = p_prev + g log2 e, a fresh chunk anchor or the stored one, k_tilde
 // rounded to the cache dtype), written to the cache, scored, and merged into
 // the consumer's partial of the CTA whose split holds it.
+#include <atomic>
+
 #include "wall_common.cuh"
 #include "wall_internal.h"
 
@@ -648,6 +650,44 @@ cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t st) {
                  : run_split_mma<KD, VD, G, true, false>(tmK, tmV, p, grid, st);
   return fused ? run_split_mma<KD, VD, G, false, true>(tmK, tmV, p, grid, st)
                : run_split_mma<KD, VD, G, false, false>(tmK, tmV, p, grid, st);
+}
+
+namespace {
+template <int KD, int VD, int G>
+int mma_ctas_per_sm() {
+  static std::atomic<int> cached{0};
+  const int v = cached.load();
+  if (v > 0) return v;
+  using D = MmaCfg<KD, VD, G>;
+  auto kern = split_mma_kernel<KD, VD, G, false, false>;
+  int n = 0;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, D::SMEM_ALLOC) !=
+          cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 64, D::SMEM_ALLOC) != cudaSuccess ||
+      n < 1)
+    n = 1;
+  cached.store(n);
+  return n;
+}
+template <int KD, int VD>
+int mma_ctas_by_group(int group) {
+  switch (group) {
+    case 1: return mma_ctas_per_sm<KD, VD, 1>();
+    case 2: return mma_ctas_per_sm<KD, VD, 2>();
+    case 4: return mma_ctas_per_sm<KD, VD, 4>();
+    case 8: return mma_ctas_per_sm<KD, VD, 8>();
+    default: return 1;
+  }
+}
+}  // namespace
+
+int decode_ctas_per_sm(int K, int V, int group, bool bf16) {
+  if (!bf16) return 1;
+  if (K == 64 && V == 64) return mma_ctas_by_group<64, 64>(group);
+  if (K == 64 && V == 128) return mma_ctas_by_group<64, 128>(group);
+  if (K == 128 && V == 64) return mma_ctas_by_group<128, 64>(group);
+  if (K == 128 && V == 128) return mma_ctas_by_group<128, 128>(group);
+  return 1;
 }
 
 #define WALL_SPLIT_MMA(KD, VD, G)                                                               \
