@@ -50,14 +50,14 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # hash of the kernel source it was taken on; reported as null once the kernel
 # source changes.  Filled in after each capture.
 TRAFFIC = {
-    # full capture on the long prefill: 316.535808 MB read + 43.428608 MB written
-    "prefill_main": {"bytes": 359964416, "source_sha": "820590f83f572f63"},
-    # capture of the decode workload at batch 4, scaled by 8 to batch 32 (traffic is
-    # proportional to the batch): (1.375950 GB + 5.537536 MB) * 8
-    "decode_split": {"bytes": 11051900288, "source_sha": "453f90616c845a14"},
+    # full capture on the long prefill: 318.078976 MB read + 44.150016 MB written
+    "prefill_main": {"bytes": 362228992, "source_sha": "bbdfce647d9e4ec6"},
+    # capture of the decode step at batch 4, scaled by 8 to batch 32 (traffic is
+    # proportional to the batch): (1.376312 GB + 4.968448 MB) * 8
+    "decode_split": {"bytes": 11050243584, "source_sha": "abf8446f86c17272"},
     # full-size capture of the cache build (batch 32, 1-pass DRAM metrics):
-    # 10737661184 B read + 8819417344 B written
-    "cache_build": {"bytes": 19557078528, "source_sha": "5ff2742a5cd5b984"},
+    # 10738862336 B read + 8820070400 B written
+    "cache_build": {"bytes": 19558932736, "source_sha": "ef8c7faf6102f370"},
 }
 KERNEL_SOURCES = {
     "prefill_main": "decayed_softmax_attention_b200/csrc/wall_fwd_tc.cu",
