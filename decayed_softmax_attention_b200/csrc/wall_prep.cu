@@ -24,6 +24,21 @@
 namespace wall {
 namespace {
 
+// bar.red.or over `nthreads` threads of named barrier `id`: a barrier whose
+// result (any thread's predicate) every participant sees.
+__device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
 // One CTA per (256-row query block, batch*query head); each half of the CTA
 // (128 threads) owns one 128-row key block.  Thread layout per half: CG
 // channel groups of 8 channels x RG row groups of RPG consecutive rows.
@@ -291,6 +306,252 @@ __global__ void __launch_bounds__(256, KT ? (KD == 64 ? 2 : 3) : (sizeof(Tin) ==
   }
 }
 
+// TMA-staged prepass for bf16 inputs whose T is a multiple of 256 (no decode-
+// cache output): the same arithmetic as prep_local_kernel, fed by bulk tensor
+// copies.  One CTA per (256-row block, batch*query head): the block's g tile
+// (256 rows x K) is copied into shared memory once and serves both passes; the
+// q and k rows stream through a two-stage ring.  Consumer thread (cg, rg) owns 8
+// channels of a run of RPG consecutive rows, so a ring stage that brings 2 rows
+// of every thread's run (one 5-D copy per 64-channel box: rows, row groups, head,
+// batch) gives every thread work.  A producer warp issues the copies; all loads
+// are in flight without holding registers.  Two (K = 128) or three (K = 64) CTAs
+// per SM.
+template <int KD>
+struct PrepTmaCfg {
+  static constexpr int CG = KD / 8;       // channel groups of 8
+  static constexpr int RG = 256 / CG;     // row groups of the 256-row block
+  static constexpr int RPG = 256 / RG;    // rows per row group
+  static constexpr int NBOX = KD / 64;    // 64-channel boxes
+  static constexpr int RPS = 2;           // rows of each row group per ring stage
+  static constexpr int NSTG = RPG / RPS;  // stages per block
+  static constexpr int NS = 2;            // ring depth
+  static constexpr int G_BOX = RG * RPG * 128;  // one box of the g tile
+  static constexpr int A_BOX = RG * RPS * 128;  // one box of one array in a stage
+  static constexpr int STAGE = 2 * NBOX * A_BOX;  // q then k
+  static constexpr int OFF_G = 0;
+  static constexpr int OFF_R = NBOX * G_BOX;
+  static constexpr int OFF_TOT = OFF_R + NS * STAGE;  // float [RG][KD]
+  static constexpr int OFF_BAR = OFF_TOT + RG * KD * 4;
+  static constexpr int SMEM = OFF_BAR + (1 + 2 * NS) * 8 + 16;
+};
+
+template <int KD>
+__global__ void __launch_bounds__(288, 1) prep_tma_kernel(
+    const __grid_constant__ CUtensorMap tmGt, const __grid_constant__ CUtensorMap tmQr,
+    const __grid_constant__ CUtensorMap tmKr, const __nv_bfloat16* __restrict__ gs,
+    const int32_t* __restrict__ cu, int nseq, int window, int T, int HQ, int H, int NB,
+    __nv_bfloat16* __restrict__ qh, __nv_bfloat16* __restrict__ kh, float* __restrict__ bsum,
+    float* __restrict__ ssl, float* __restrict__ ssb, __nv_bfloat16* __restrict__ kx,
+    float inv_scale, int* __restrict__ rowlo, int* __restrict__ wide, int* __restrict__ err,
+    int wide_err, uint64_t wait_ns) {
+  using PC = PrepTmaCfg<KD>;
+  extern __shared__ __align__(128) uint8_t psm[];
+  float* tot = reinterpret_cast<float*>(psm + PC::OFF_TOT);
+  uint64_t* gfull = reinterpret_cast<uint64_t*>(psm + PC::OFF_BAR);
+  uint64_t* full = gfull + 1;
+  uint64_t* empty = full + PC::NS;
+  int* abort_flag = reinterpret_cast<int*>(empty + PC::NS);
+  int* s_span = abort_flag + 1;
+  __shared__ float wsum[2][4];
+
+  const int bp = blockIdx.x, bh = blockIdx.y;  // 256-row block, batch*query head
+  const int b = bh / HQ, hq = bh % HQ, kvh = hq / (HQ / H);
+  if (threadIdx.x == 0) {
+    mbar_init(gfull, 1);
+    for (int i = 0; i < PC::NS; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 8);  // one arrival per consumer warp
+    }
+    *abort_flag = 0;
+    *s_span = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const WaitCtl wc{abort_flag, err, wait_ns};
+
+  if (threadIdx.x >= 256) {
+    // ------------------------------------------------------------- producer
+    if (threadIdx.x == 256) {
+      tma_prefetch_desc(&tmGt);
+      tma_prefetch_desc(&tmQr);
+      tma_prefetch_desc(&tmKr);
+      const int grp0 = bp * PC::RG;  // the block's first row group
+      mbar_arrive_expect_tx(gfull, PC::NBOX * PC::G_BOX);
+      for (int x = 0; x < PC::NBOX; ++x)
+        tma_load_5d(psm + PC::OFF_G + x * PC::G_BOX, &tmGt, gfull, x * 64, 0, grp0, hq, b);
+      int issued = 0;
+      for (int st = 0; st < PC::NSTG; ++st) {
+        const int slot = st % PC::NS;
+        if (st >= PC::NS && !mbar_wait(&empty[slot], ((st / PC::NS) - 1) & 1, wc)) break;
+        uint8_t* dst = psm + PC::OFF_R + slot * PC::STAGE;
+        mbar_arrive_expect_tx(&full[slot], PC::STAGE);
+        for (int x = 0; x < PC::NBOX; ++x) {
+          tma_load_5d(dst + x * PC::A_BOX, &tmQr, &full[slot], x * 64, st * PC::RPS, grp0, hq, b);
+          tma_load_5d(dst + (PC::NBOX + x) * PC::A_BOX, &tmKr, &full[slot], x * 64, st * PC::RPS,
+                      grp0, kvh, b);
+        }
+        issued = st + 1;
+      }
+      // every copy issued lands before the CTA may exit
+      mbar_drain(gfull, 0, wait_ns);
+      for (int st = issued > PC::NS ? issued - PC::NS : 0; st < issued; ++st)
+        mbar_drain(&full[st % PC::NS], (st / PC::NS) & 1, wait_ns);
+    }
+    return;
+  }
+
+  // --------------------------------------------------------------- consumers
+  const int tid = threadIdx.x;
+  const int cg = tid % PC::CG, rg = tid / PC::CG;
+  const int box = cg >> 3, cw = cg & 7;  // 64-channel box, 16-byte chunk within its row
+  const int half = (rg * PC::RPG) >> 7;  // the 128-row key block of this thread's rows
+  const int t0 = bp * 256 + rg * PC::RPG;
+  const uint8_t* gt = psm + PC::OFF_G + box * PC::G_BOX + (rg * PC::RPG) * 128 + cw * 16;
+
+  // ---- pass 1: g summed over this thread's rows (from the resident g tile)
+  bool ok = mbar_wait(gfull, 0, wc);
+  float2 acc[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) acc[c] = make_float2(0.f, 0.f);
+  if (ok) {
+#pragma unroll 4
+    for (int m = 0; m < PC::RPG; ++m) {
+      float f[8];
+      load8(reinterpret_cast<const __nv_bfloat16*>(gt + m * 128), f);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[c] = __fadd2_rn(acc[c], make_float2(f[2 * c], f[2 * c + 1]));
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    tot[rg * KD + cg * 8 + 2 * c] = acc[c].x;
+    tot[rg * KD + cg * 8 + 2 * c + 1] = acc[c].y;
+  }
+  ok = !bar_red_or(1, 256, !ok);  // (a consumer-only barrier: the producer does not join)
+  // qa: query exponent (G_t - AQ) log2 e, advanced per row; ka: (AK - AQ) log2 e
+  constexpr int RGH = PC::RG / 2;  // row groups per 128-row half
+  float qa[8], ka[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float pre = 0.f, all = 0.f, first = 0.f;
+#pragma unroll
+    for (int r = 0; r < RGH; ++r) {
+      const float x = tot[(half * RGH + r) * KD + cg * 8 + c];
+      all += x;
+      if (half * RGH + r < rg) pre += x;
+      if (half == 1) first += tot[r * KD + cg * 8 + c];
+    }
+    qa[c] = (first + pre) * kLog2e;
+    ka[c] = (first + all) * kLog2e;
+    if (rg == half * RGH && bp * 2 + half < NB)
+      bsum[(static_cast<size_t>(bh) * NB + bp * 2 + half) * KD + cg * 8 + c] = all;
+  }
+
+  // ---- pass 2: qh = q 2^qa, kh = k 2^(ka - qa), q and k rows from the ring
+  __nv_bfloat16* qo = qh + (static_cast<size_t>(bh) * T + t0) * KD + cg * 8;
+  __nv_bfloat16* ko = kh + (static_cast<size_t>(bh) * T + t0) * KD + cg * 8;
+  float span = 0.f;
+  for (int st = 0; ok && st < PC::NSTG; ++st) {
+    const int slot = st % PC::NS;
+    const bool got = mbar_wait(&full[slot], (st / PC::NS) & 1, wc);
+    if (!__all_sync(0xffffffffu, got)) {
+      ok = false;
+      break;
+    }
+    const uint8_t* sq = psm + PC::OFF_R + slot * PC::STAGE + box * PC::A_BOX +
+                        (rg * PC::RPS) * 128 + cw * 16;
+    const uint8_t* sk = sq + PC::NBOX * PC::A_BOX;
+#pragma unroll
+    for (int r = 0; r < PC::RPS; ++r) {
+      const int m = st * PC::RPS + r;
+      float f[8], x[8], y[8];
+      load8(reinterpret_cast<const __nv_bfloat16*>(gt + m * 128), f);
+      load8(reinterpret_cast<const __nv_bfloat16*>(sq + r * 128), x);
+      load8(reinterpret_cast<const __nv_bfloat16*>(sk + r * 128), y);
+      // exp(a) as 2^(a log2 e): one MUFU op each (relative error ~2^-22)
+#pragma unroll
+      for (int c = 0; c < 8; c += 2) {
+        const float2 a = __ffma2_rn(make_float2(f[c], f[c + 1]), make_float2(kLog2e, kLog2e),
+                                    make_float2(qa[c], qa[c + 1]));
+        qa[c] = a.x;
+        qa[c + 1] = a.y;
+        span = fmaxf(span, fmaxf(fabsf(a.x), fabsf(a.y)));
+        const float2 kk = __fadd2_rn(make_float2(ka[c], ka[c + 1]), make_float2(-a.x, -a.y));
+        const float2 xr = __fmul2_rn(make_float2(x[c], x[c + 1]),
+                                     make_float2(ex2_approx(a.x), ex2_approx(a.y)));
+        const float2 yr = __fmul2_rn(make_float2(y[c], y[c + 1]),
+                                     make_float2(ex2_approx(kk.x), ex2_approx(kk.y)));
+        x[c] = xr.x; x[c + 1] = xr.y;
+        y[c] = yr.x; y[c + 1] = yr.y;
+      }
+      store8(qo + static_cast<size_t>(m) * KD, x);
+      store8(ko + static_cast<size_t>(m) * KD, y);
+    }
+    __syncwarp();
+    if ((tid & 31) == 0) mbar_arrive(&empty[slot]);  // this warp no longer reads the stage
+  }
+
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) span = fmaxf(span, __shfl_xor_sync(0xffffffffu, span, off));
+  if ((tid & 31) == 0 && span > 0.f) atomicMax(s_span, __float_as_int(span));
+  named_bar_sync(1, 256);
+  if (tid == 0) {
+    const int w = __int_as_float(*s_span) > kPrefillSpanNats * kLog2e ? 1 : 0;
+    wide[static_cast<size_t>(bh) * gridDim.x + bp] = w;
+    if (w && wide_err) atomicOr(err, kDevErrRange);
+  }
+
+  // Scalar gate: negated 128-block-local inclusive prefix (log2 units), one row per thread.
+  const int blk = bp * 2 + (tid >> 7), tr = tid & 127, hf = tid >> 7;
+  if (gs != nullptr) {
+    const int t = blk * kBlockRows + tr;
+    float x = (t < T) ? load1(gs + (static_cast<size_t>(b) * T + t) * HQ + hq) * kLog2e : 0.f;
+    const int lane = tr & 31, wid = tr >> 5;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += y;
+    }
+    if (lane == 31) wsum[hf][wid] = x;
+    named_bar_sync(1, 256);
+    for (int w = 0; w < wid; ++w) x += wsum[hf][w];
+    if (blk < NB) {
+      ssl[static_cast<size_t>(bh) * NB * kBlockRows + blk * kBlockRows + tr] = -x;  // negated
+      if (tr == kBlockRows - 1) ssb[static_cast<size_t>(bh) * NB + blk] = x;
+    }
+    // key-side gate term as two extra bf16 channels of the key operand (hi + lo =
+    // -x / (scale * log2(e)) to ~16 significant bits; the query side carries ones)
+    if (kx != nullptr && t < T) {
+      const float val = -x * inv_scale;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(val);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(val - __bfloat162float(hi));
+      uint4 u;
+      u.x = static_cast<uint32_t>(__bfloat16_as_ushort(hi)) |
+            (static_cast<uint32_t>(__bfloat16_as_ushort(lo)) << 16);
+      u.y = u.z = u.w = 0u;
+      uint4* dst = reinterpret_cast<uint4*>(kx + (static_cast<size_t>(bh) * T + t) * 16);
+      dst[0] = u;
+      dst[1] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+
+  // First admitted key of each row for packed documents (shared by all heads).
+  if (cu != nullptr && bh == 0) {
+    const int t = blk * kBlockRows + tr;
+    if (t < T) {
+      int lo = 0, hi = nseq;  // largest d with cu[d] <= t
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (cu[mid] <= t) lo = mid; else hi = mid;
+      }
+      int s0 = cu[lo];
+      s0 = s0 < 0 ? 0 : (s0 > t ? t : s0);
+      if (window > 0 && t - window + 1 > s0) s0 = t - window + 1;
+      rowlo[t] = s0;
+    }
+  }
+}
+
 // Exclusive scan of the block sums over the blocks of one (batch, head): one
 // warp per channel, lane l owning blocks [l PB, (l + 1) PB); each lane sums its
 // blocks, a shuffle scan gives every lane the sum before its first block, and
@@ -357,21 +618,78 @@ __global__ void __launch_bounds__(KD) cache_anchor_kernel(const float* __restric
   *slot = (*slot + AQ[(static_cast<size_t>(bh) * NB + blk) * KD + n]) * kLog2e;
 }
 
+// The TMA-staged prepass: bf16, no cache output, T a multiple of 256.  Returns
+// false (nothing launched) when its tensor maps cannot be encoded.
+template <int KD>
+bool prep_tma(const FwdArgs& a, const FwdWork& w, cudaStream_t st, cudaError_t* e) {
+  using PC = PrepTmaCfg<KD>;
+  const int BHQ = a.B * a.HQ;
+  CUtensorMap tmGt, tmQr, tmKr;
+  const cuuint64_t grp = static_cast<cuuint64_t>(a.T) / PC::RPG;
+  {
+    const cuuint64_t dims[5] = {static_cast<cuuint64_t>(KD), static_cast<cuuint64_t>(PC::RPG), grp,
+                                static_cast<cuuint64_t>(a.HQ), static_cast<cuuint64_t>(a.B)};
+    const cuuint64_t row = static_cast<cuuint64_t>(a.HQ) * KD * 2;
+    const cuuint64_t strides[4] = {row, row * PC::RPG, static_cast<cuuint64_t>(KD) * 2,
+                                   row * static_cast<cuuint64_t>(a.T)};
+    const cuuint32_t boxg[5] = {64, static_cast<cuuint32_t>(PC::RPG),
+                                static_cast<cuuint32_t>(PC::RG), 1, 1};
+    const cuuint32_t boxq[5] = {64, static_cast<cuuint32_t>(PC::RPS),
+                                static_cast<cuuint32_t>(PC::RG), 1, 1};
+    if (!encode_tiled(&tmGt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, a.g, dims, strides, boxg,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_tiled(&tmQr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, a.q, dims, strides, boxq,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+      return false;
+  }
+  {
+    const cuuint64_t dims[5] = {static_cast<cuuint64_t>(KD), static_cast<cuuint64_t>(PC::RPG), grp,
+                                static_cast<cuuint64_t>(a.H), static_cast<cuuint64_t>(a.B)};
+    const cuuint64_t row = static_cast<cuuint64_t>(a.H) * KD * 2;
+    const cuuint64_t strides[4] = {row, row * PC::RPG, static_cast<cuuint64_t>(KD) * 2,
+                                   row * static_cast<cuuint64_t>(a.T)};
+    const cuuint32_t boxk[5] = {64, static_cast<cuuint32_t>(PC::RPS),
+                                static_cast<cuuint32_t>(PC::RG), 1, 1};
+    if (!encode_tiled(&tmKr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, a.k, dims, strides, boxk,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+      return false;
+  }
+  auto kern = prep_tma_kernel<KD>;
+  *e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PC::SMEM);
+  if (*e != cudaSuccess) return true;
+  kern<<<dim3(a.T / 256, BHQ), 288, PC::SMEM, st>>>(
+      tmGt, tmQr, tmKr, static_cast<const __nv_bfloat16*>(a.g_scalar), a.cu_seqlens, a.num_seqs,
+      a.window, a.T, a.HQ, a.H, a.NB, static_cast<__nv_bfloat16*>(w.qh),
+      static_cast<__nv_bfloat16*>(w.kh), w.bsum, w.ssl, w.ssb, static_cast<__nv_bfloat16*>(w.kx),
+      1.f / (a.scale * kLog2e), w.rowlo, w.wide, a.err, a.wide_is_error ? 1 : 0, a.wait_ns);
+  *e = cudaGetLastError();
+  return true;
+}
+
 template <typename Tin, int KD>
 cudaError_t prep_impl(const FwdArgs& a, const FwdWork& w, cudaStream_t st) {
   const int BHQ = a.B * a.HQ;
   dim3 grid((a.NB + 1) / 2, BHQ);
-  auto kern = a.kt_out != nullptr ? prep_local_kernel<Tin, KD, true>
-                                   : prep_local_kernel<Tin, KD, false>;
-  kern<<<grid, 256, 0, st>>>(
-      static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.g),
-      static_cast<const Tin*>(a.g_scalar), a.cu_seqlens, a.num_seqs, a.window, a.T, a.HQ, a.H,
-      a.NB, static_cast<Tin*>(w.qh), static_cast<Tin*>(w.kh), w.bsum, w.ssl, w.ssb,
-      sizeof(Tin) == 2 ? static_cast<__nv_bfloat16*>(w.kx) : nullptr, 1.f / (a.scale * kLog2e),
-      w.rowlo, static_cast<Tin*>(a.kt_out), a.r_out, a.cache_cap, a.cache_chunk, w.wide, a.err,
-      a.wide_is_error ? 1 : 0);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  bool staged = false;
+  cudaError_t e = cudaSuccess;
+  if constexpr (sizeof(Tin) == 2) {
+    if (a.kt_out == nullptr && a.T % 256 == 0) staged = prep_tma<KD>(a, w, st, &e);
+  }
+  if (staged) {
+    if (e != cudaSuccess) return e;
+  } else {
+    auto kern = a.kt_out != nullptr ? prep_local_kernel<Tin, KD, true>
+                                     : prep_local_kernel<Tin, KD, false>;
+    kern<<<grid, 256, 0, st>>>(
+        static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.g),
+        static_cast<const Tin*>(a.g_scalar), a.cu_seqlens, a.num_seqs, a.window, a.T, a.HQ, a.H,
+        a.NB, static_cast<Tin*>(w.qh), static_cast<Tin*>(w.kh), w.bsum, w.ssl, w.ssb,
+        sizeof(Tin) == 2 ? static_cast<__nv_bfloat16*>(w.kx) : nullptr, 1.f / (a.scale * kLog2e),
+        w.rowlo, static_cast<Tin*>(a.kt_out), a.r_out, a.cache_cap, a.cache_chunk, w.wide, a.err,
+        a.wide_is_error ? 1 : 0);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   prep_scan_kernel<KD><<<dim3(BHQ, KD / 8), 288, 0, st>>>(w.bsum, a.g_scalar ? w.ssb : nullptr, a.NB, w.AQ,
                                                  w.AK, w.ssa, a.kt_out ? a.plast_out : nullptr);
   e = cudaGetLastError();
