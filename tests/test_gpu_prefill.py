@@ -91,6 +91,10 @@ EDGE = [
     dict(T=257, K=64, V=128), dict(T=257, K=128, V=64), dict(T=200, HQ=4, H=1),
     dict(T=200, HQ=6, H=3, sink=True, window=50),
     dict(T=300, HQ=16, H=1), dict(T=200, HQ=8, H=1, window=100, g_scalar=True),
+    # T a multiple of 256 (bf16 takes the TMA-staged prepass): documents, window, gate;
+    # K = 64 with GQA
+    dict(T=512, docs=(1, 255, 200, 56), window=100, g_scalar=True),
+    dict(T=768, K=64, V=128, HQ=8, H=2, sink=True),
 ]
 
 

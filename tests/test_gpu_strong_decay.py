@@ -51,6 +51,7 @@ PREFILL_CASES = [
     dict(T=300, g_kind="strong"),
     dict(T=2000, g_kind="strong", g_scalar=True, sink=True),
     dict(T=2000, g_kind="strong_all"),
+    dict(T=1024, g_kind="strong", g_scalar=True),  # (bf16: the TMA-staged prepass)
     dict(T=1000, g_kind="spike", HQ=4, H=1),
     dict(T=777, g_kind="strong", window=300, sink=True),
     dict(T=700, g_kind="strong", docs=(1, 255, 300, 144), g_scalar=True),
