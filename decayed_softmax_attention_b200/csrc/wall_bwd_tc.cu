@@ -31,9 +31,11 @@
 // 64-127 (two warps per SM sub-partition hide each other's MUFU and TMEM
 // latencies); warpgroup 3 multiplies each streamed Qh (key-block kernel) or Kh
 // (query-block kernel) tile by c in shared memory.  Registers are re-split at
-// start (setmaxnreg): 88 / 168 / 168 / 88 (sum 512 = 4 x the 128 of the
-// launch; no spills).  Per-column vectors of the elementwise passes are read 32
-// at a time as broadcast 16-byte loads, issued with the chunk's TMEM load.  Every wait is
+// start (setmaxnreg): 88 / 168 / 168 / 88 in the key-block kernel, 88 / 176 /
+// 176 / 72 in the query-block kernel (each sums to 512 = 4 x the 128 of the
+// launch).  The elementwise passes run on fp32 pairs (.f32x2 fma / mul / add):
+// P stays in registers as fp32 between the two passes, and the per-column
+// vectors are read 4 at a time as broadcast 16-byte loads.  Every wait is
 // bounded (device error word + CTA abort flag), copies in flight are drained
 // and TMEM is freed before exit.
 #include "wall_common.cuh"
@@ -433,7 +435,9 @@ __global__ void __launch_bounds__(512, 1)
     bool ok = mbar_wait(kvfull, 0, wc);
     ok = __all_sync(0xffffffffu, ok);
     const float colj = (HAS_GS && ok) ? sColt[r] : 0.f;
-    float rsum = 0.f;
+    const float2 ncol2 = make_float2(-colj, -colj), sc2 = make_float2(p.sc, p.sc);
+    const float2 neg1 = make_float2(-1.f, -1.f);
+    float2 rs2 = make_float2(0.f, 0.f);
     for (int it = 0; ok && it < nt; ++it) {
       const int s = it & 1;
       const int q0 = (it_lo + it) * 128;
@@ -450,39 +454,41 @@ __global__ void __launch_bounds__(512, 1)
       got = mbar_wait(sfull, it & 1, wc);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
-      // pass 1: P^T = exp2(S^T sc + rowt - colt) over the admitted (query, key) pairs
-      uint32_t pk[32];
+      // pass 1: P^T = exp2(S^T sc + rowt - colt) over the admitted (query, key)
+      // pairs; fp32 pairs stay in registers for pass 2, bf16 pairs go to TMEM
+      float2 pf[32];
 #pragma unroll
-      for (int c = cb; c < cb + 64; c += 32) {
-        float x[32], rv[32];
-        tmem_ld32(lane_base + COL_S + c, x);
-        load32(rowt + c, rv);
+      for (int c = 0; c < 64; c += 32) {
+        float x[32];
+        tmem_ld32(lane_base + COL_S + cb + c, x);
         tmem_wait_ld();
         fence_regs32(x);
-        if (full) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const float4 r4 = *reinterpret_cast<const float4*>(rowt + cb + c + e);
+          const float2 y0 = ffma2(make_float2(x[e], x[e + 1]), sc2,
+                                  fadd2(make_float2(r4.x, r4.y), ncol2));  // rowt - colt
+          const float2 y1 = ffma2(make_float2(x[e + 2], x[e + 3]), sc2,
+                                  fadd2(make_float2(r4.z, r4.w), ncol2));
+          pf[(c + e) >> 1] = make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
+          pf[(c + e + 2) >> 1] = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
+        }
+        if (!full) {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float p0 = ex2_approx(fmaf(x[e], p.sc, rv[e] - colj));
-            const float p1 = ex2_approx(fmaf(x[e + 1], p.sc, rv[e + 1] - colj));
-            pk[(c - cb + e) >> 1] = pack_bf16(p0, p1);
-          }
-        } else {
-          int lv[32];
-          if (lo_tab) load32(lo + c, lv);
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float pv[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int q = q0 + c + e + h;
-              const bool adm = q < p.T && q >= j &&
-                               (lo_tab ? lv[e + h] : first_key(nullptr, p.window, q)) <= j;
-              pv[h] = adm ? ex2_approx(fmaf(x[e + h], p.sc, rv[e + h] - colj)) : 0.f;
-            }
-            pk[(c - cb + e) >> 1] = pack_bf16(pv[0], pv[1]);
+            const int q = q0 + cb + c + e;
+            int2 l2 = make_int2(0, 0);
+            if (lo_tab) l2 = *reinterpret_cast<const int2*>(lo + cb + c + e);
+            const int f0 = lo_tab ? l2.x : first_key(nullptr, p.window, q);
+            const int f1 = lo_tab ? l2.y : first_key(nullptr, p.window, q + 1);
+            if (!(q < p.T && q >= j && f0 <= j)) pf[(c + e) >> 1].x = 0.f;
+            if (!(q + 1 < p.T && q + 1 >= j && f1 <= j)) pf[(c + e) >> 1].y = 0.f;
           }
         }
-        tmem_st16(lane_base + COL_S + packed_dst(c, cb), pk + ((c - cb) >> 1));
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(pf[(c >> 1) + e].x, pf[(c >> 1) + e].y);
+        tmem_st16(lane_base + COL_S + packed_dst(cb + c, cb), pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -492,30 +498,40 @@ __global__ void __launch_bounds__(512, 1)
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
-      for (int c = cb; c < cb + 64; c += 32) {
-        float x[32], dv[32];
-        tmem_ld32(lane_base + COL_DP + c, x);
-        load32(del + c, dv);
+      for (int c = 0; c < 64; c += 32) {
+        float x[32];
+        tmem_ld32(lane_base + COL_DP + cb + c, x);
         tmem_wait_ld();
         fence_regs32(x);
+        // query columns past T: delta there is not defined (padding); taken as 0
+        // there, where p = 0 and dP = 0 (dO's rows past T are zero-filled)
+        const int nvalid = full ? 32 : p.T - (q0 + cb + c);
         uint32_t dk[16];
-        // rows past T: delta there is not defined (padding), p is 0
-        const int nvalid = full ? 32 : min(32, p.T - (q0 + c));
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const uint32_t u = pk[(c - cb + e) >> 1];
-          const float d0 = e < nvalid ? bf16_lo(u) * (x[e] - dv[e]) : 0.f;
-          const float d1 = e + 1 < nvalid ? bf16_hi(u) * (x[e + 1] - dv[e + 1]) : 0.f;
-          rsum += d0 + d1;
-          dk[e >> 1] = pack_bf16(d0, d1);
+        for (int e = 0; e < 32; e += 4) {
+          float4 d4 = *reinterpret_cast<const float4*>(del + cb + c + e);
+          if (e + 3 >= nvalid) {
+            if (e >= nvalid) d4.x = 0.f;
+            if (e + 1 >= nvalid) d4.y = 0.f;
+            if (e + 2 >= nvalid) d4.z = 0.f;
+            d4.w = 0.f;
+          }
+          const float2 d0 = fmul2(pf[(c + e) >> 1],
+                                  ffma2(make_float2(d4.x, d4.y), neg1, make_float2(x[e], x[e + 1])));
+          const float2 d1 = fmul2(pf[(c + e + 2) >> 1],
+                                  ffma2(make_float2(d4.z, d4.w), neg1, make_float2(x[e + 2], x[e + 3])));
+          rs2 = fadd2(rs2, fadd2(d0, d1));
+          dk[e >> 1] = pack_bf16(d0.x, d0.y);
+          dk[(e >> 1) + 1] = pack_bf16(d1.x, d1.y);
         }
-        tmem_st16(lane_base + COL_DP + packed_dst(c, cb), dk);
+        tmem_st16(lane_base + COL_DP + packed_dst(cb + c, cb), dk);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(dsready);
     }
     // the two halves' row sums: the second half's go through shared memory
+    float rsum = rs2.x + rs2.y;
     if (hc == 1) sRs[r] = rsum;
     named_bar_sync(2, 256);
     if (hc == 0) rsum += sRs[r];
@@ -753,7 +769,7 @@ __global__ void __launch_bounds__(512, 1)
   } else if (wg == 1 || wg == 2) {
     // ------------------------------------------------------------- elementwise + epilogue
     // warpgroup wg handles the key columns [64 (wg - 1), 64 wg) of every tile
-    reg_alloc<168>();
+    reg_alloc<176>();
     const int hc = wg - 1, cb = 64 * hc;
     const int r = tid - 128 * wg;  // query row within the tile = TMEM lane
     const int t = q0 + r;
@@ -764,7 +780,9 @@ __global__ void __launch_bounds__(512, 1)
     bool ok = mbar_wait(qfull, 0, wc);
     ok = __all_sync(0xffffffffu, ok);
     const float rowt = ok ? sRowt[r] : 0.f, del = ok ? sDel[r] : 0.f;
-    float rsum = 0.f;
+    const float2 rowt2 = make_float2(rowt, rowt), del2 = make_float2(del, del);
+    const float2 sc2 = make_float2(p.sc, p.sc), neg1 = make_float2(-1.f, -1.f);
+    float2 rs2 = make_float2(0.f, 0.f);
     for (int jt = 0; ok && jt < nt; ++jt) {
       const int ks = jt % KS, k0 = (kt_hi - jt) * 128;
       const float* colt = sColt + ks * 128;
@@ -774,54 +792,64 @@ __global__ void __launch_bounds__(512, 1)
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
       const uint32_t colS = COL_S + 128 * (jt & 1);
-      // pass 1: p = exp2(S sc + rowt - colt), kept in registers as packed bf16
-      uint32_t pk[32];
+      // pass 1: p = exp2(S sc + rowt - colt), kept in registers as fp32 pairs
+      // (fma(colt, -1, rowt) is the rounded difference rowt - colt)
+      float2 pf[32];
 #pragma unroll
-      for (int c = cb; c < cb + 64; c += 32) {
-        float x[32], cv[32];
-        tmem_ld32(lane_base + colS + c, x);
-        if (HAS_GS) load32(colt + c, cv);
+      for (int c = 0; c < 64; c += 32) {
+        float x[32];
+        tmem_ld32(lane_base + colS + cb + c, x);
         tmem_wait_ld();
         fence_regs32(x);
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float pv[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int key = k0 + c + e + h;
-            const float y = fmaf(x[e + h], p.sc, HAS_GS ? rowt - cv[e + h] : rowt);
-            const bool adm = full || (key <= t && key >= lo_t);
-            pv[h] = adm ? ex2_approx(y) : 0.f;
+        for (int e = 0; e < 32; e += 4) {
+          float2 off0 = rowt2, off1 = rowt2;
+          if (HAS_GS) {
+            const float4 c4 = *reinterpret_cast<const float4*>(colt + cb + c + e);
+            off0 = ffma2(make_float2(c4.x, c4.y), neg1, rowt2);
+            off1 = ffma2(make_float2(c4.z, c4.w), neg1, rowt2);
           }
-          pk[(c - cb + e) >> 1] = pack_bf16(pv[0], pv[1]);
+          const float2 y0 = ffma2(make_float2(x[e], x[e + 1]), sc2, off0);
+          const float2 y1 = ffma2(make_float2(x[e + 2], x[e + 3]), sc2, off1);
+          pf[(c + e) >> 1] = make_float2(ex2_approx(y0.x), ex2_approx(y0.y));
+          pf[(c + e + 2) >> 1] = make_float2(ex2_approx(y1.x), ex2_approx(y1.y));
+        }
+        if (!full) {  // keys after the row, before its first key, or past T: p = 0
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int key = k0 + cb + c + e;
+            if (key > t || key < lo_t) pf[(c + e) >> 1].x = 0.f;
+            if (key + 1 > t || key + 1 < lo_t) pf[(c + e) >> 1].y = 0.f;
+          }
         }
       }
-      // pass 2: dS = p (dP - delta) over dP's columns; row sums for dGs
+      // pass 2: dS = p (dP - delta) over dP's columns; row sums for dGs.  A row
+      // past T has p = 0 and feeds only its own dQ row and row sum, never stored.
       got = mbar_wait(dpfull, jt & 1, wc);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
-      for (int c = cb; c < cb + 64; c += 32) {
+      for (int c = 0; c < 64; c += 32) {
         float x[32];
-        tmem_ld32(lane_base + COL_DP + c, x);
+        tmem_ld32(lane_base + COL_DP + cb + c, x);
         tmem_wait_ld();
         fence_regs32(x);
         uint32_t dk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const uint32_t u = pk[(c - cb + e) >> 1];
-          const float d0 = row_ok ? bf16_lo(u) * (x[e] - del) : 0.f;
-          const float d1 = row_ok ? bf16_hi(u) * (x[e + 1] - del) : 0.f;
-          rsum += d0 + d1;
-          dk[e >> 1] = pack_bf16(d0, d1);
+          const float2 dd = ffma2(del2, neg1, make_float2(x[e], x[e + 1]));  // dP - delta
+          const float2 d = fmul2(pf[(c + e) >> 1], dd);
+          rs2 = fadd2(rs2, d);
+          dk[e >> 1] = pack_bf16(d.x, d.y);
         }
-        tmem_st16(lane_base + COL_DP + packed_dst(c, cb), dk);
+        tmem_st16(lane_base + COL_DP + packed_dst(cb + c, cb), dk);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(dsready);
     }
     // the two halves' row sums: the second half's go through shared memory
+    float rsum = rs2.x + rs2.y;
     if (hc == 1) sRs[r] = rsum;
     named_bar_sync(2, 256);
     if (hc == 0) rsum += sRs[r];
@@ -848,7 +876,7 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else {
     // ------------------------------------------------------------- key-tile rescale (by c)
-    reg_dealloc<88>();
+    reg_dealloc<72>();  // 88 + 2 x 176 + 72 = 512 registers per thread-quad
     const int r = tid - 384;
     bool ok = mbar_wait(qfull, 0, wc);
     ok = !bar_any(1, 128, !ok);
