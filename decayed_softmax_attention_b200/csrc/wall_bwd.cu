@@ -453,66 +453,292 @@ __device__ __forceinline__ bool bit_of(const uint32_t* mask, int u) {
   return (mask[u >> 5] >> (u & 31)) & 1u;
 }
 
-// One CTA per (128-row block, batch * query head); thread n walks channel n
-// down the block's rows, rebuilding the block-local prefix L of g:
+// Two consecutive elements (bf16: one 4-byte access; f32: one 8-byte access).
+__device__ __forceinline__ float2 load2(const __nv_bfloat16* p) {
+  const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+  return make_float2(bf16_lo(u), bf16_hi(u));
+}
+__device__ __forceinline__ float2 load2(const float* p) {
+  return *reinterpret_cast<const float2*>(p);
+}
+__device__ __forceinline__ void store2(__nv_bfloat16* p, float2 f) {
+  *reinterpret_cast<uint32_t*>(p) = pack_bf16(f.x, f.y);
+}
+__device__ __forceinline__ void store2(float* p, float2 f) { *reinterpret_cast<float2*>(p) = f; }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return make_float2(a.x + b.x, a.y + b.y); }
+
+// The post passes split a 128-row block over 8 warps of 16 rows; a lane owns
+// two adjacent channels of a 64-channel group.
+constexpr int kPostRows = 16;
+constexpr int kPostWarps = kBlockRows / kPostRows;
+constexpr int kPostThreads = kPostWarps * 32 + 32;  // + one warp for the scalar channels
+
+// The first document start inside the block (row > b0), or b1.
+__device__ __forceinline__ int first_doc_start(const uint32_t* mask, int b0, int b1) {
+#pragma unroll
+  for (int w = 0; w < 4; ++w)
+    if (mask[w] != 0u) return min(b1, b0 + 32 * w + __ffs(static_cast<int>(mask[w])) - 1);
+  return b1;
+}
+
+// One CTA per (128-row block, batch * KV head, 64-channel group).  For every
+// query head of the KV group, the block-local prefix L of g is rebuilt (each
+// warp's segment sum through shared memory, then a walk down its 16 rows):
 //   G[t] - AQ = L[t] (+ the first half's block sum in an odd block),
 //   AK - G[t] = (block sum) - L[t].
-// Writes dq (final), dk_h (over accK), dG = q dq - k dk_h (over accQ), and the
-// block's "head": the sum of dG from the block's first row up to the first
-// document start inside the block.  Thread KD does the gate channel
-// (dGs = rsB - rsA, over rsB) and sums the block's sink terms.
-template <typename Tin, int KD, bool HAS_GS>
-__global__ void __launch_bounds__(KD + 32) bwd_post_local_kernel(
+// Writes dq (final), dG = q dq - k dk_h (over accQ) and the block's "head": the
+// sum of dG from the block's first row up to the first document start inside
+// the block.  dk and dv are the sums of dk_h = scale e^{AK-G} accK and of dv_h
+// over the group's query heads, formed in registers and written once.  The
+// last warp (channel group 0) does the gate channel (dGs = rsB - rsA, over
+// rsB) and the block's sink sums.
+template <typename Tin, int KD, int VD, bool HAS_GS>
+__global__ void __launch_bounds__(kPostThreads, 2) bwd_post_local_kernel(
     const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ g,
     const float* __restrict__ bsum, const int32_t* __restrict__ cu, int nseq, int T, int HQ, int H,
-    int NB, float scale, float* __restrict__ accQ, float* __restrict__ accK,
-    const float* __restrict__ rsA, float* __restrict__ rsB, const float* __restrict__ psd,
-    Tin* __restrict__ dq, float* __restrict__ head, float* __restrict__ sinkblk) {
+    int NB, float scale, float* __restrict__ accQ, const float* __restrict__ accK,
+    const float* __restrict__ dvh, const float* __restrict__ rsA, float* __restrict__ rsB,
+    const float* __restrict__ psd, Tin* __restrict__ dq, Tin* __restrict__ dk,
+    Tin* __restrict__ dv, float* __restrict__ head, float* __restrict__ sinkblk) {
   __shared__ uint32_t mask[4];
-  const int blk = blockIdx.x, bh = blockIdx.y;
-  const int HQk = HQ;
-  const int b = bh / HQk, hq = bh % HQk, kvh = hq / (HQk / H);
+  __shared__ float2 ssum[2][kPostWarps][32];
+  __shared__ float2 hred[2][kPostWarps][32];
+  const int blk = blockIdx.x, z = blockIdx.z;
+  const int b = blockIdx.y / H, kvh = blockIdx.y % H, grp = HQ / H;
   const int b0 = blk * kBlockRows, b1 = min(T, b0 + kBlockRows);
   doc_start_mask(cu, nseq, b0, b1, mask);
-  const int tid = threadIdx.x;
-  const size_t hbase = (static_cast<size_t>(bh) * NB + blk) * (KD + 1);
-  if (tid < KD) {
-    const int n = tid;
-    const float qoff = (blk & 1) ? bsum[(static_cast<size_t>(bh) * NB + blk - 1) * KD + n] : 0.f;
-    const float tot = bsum[(static_cast<size_t>(bh) * NB + blk) * KD + n];
-    float L = 0.f, hsum = 0.f;
-    bool in_head = true;
-#pragma unroll 4
-    for (int u = b0; u < b1; ++u) {
-      if (u > b0 && bit_of(mask, u - b0)) in_head = false;
-      const size_t iq = ((static_cast<size_t>(b) * T + u) * HQ + hq) * KD + n;
-      const size_t ik = ((static_cast<size_t>(b) * T + u) * H + kvh) * KD + n;
-      const size_t ia = (static_cast<size_t>(bh) * T + u) * KD + n;
-      L += load1(g + iq);
-      const float dqv = scale * ex2_approx((qoff + L) * kLog2e) * accQ[ia];
-      const float dkv = scale * ex2_approx((tot - L) * kLog2e) * accK[ia];
-      store1(dq + iq, dqv);
-      accK[ia] = dkv;
-      const float dG = load1(q + iq) * dqv - load1(k + ik) * dkv;
-      accQ[ia] = dG;
-      if (in_head) hsum += dG;
-    }
-    head[hbase + n] = hsum;
-  } else if (tid == KD) {
-    float hsum = 0.f, ssum = 0.f;
-    bool in_head = true;
-    for (int u = b0; u < b1; ++u) {
-      if (u > b0 && bit_of(mask, u - b0)) in_head = false;
-      const size_t i = static_cast<size_t>(bh) * T + u;
-      if (HAS_GS) {
-        const float d = rsB[i] - rsA[i];
-        rsB[i] = d;
-        if (in_head) hsum += d;
+  const int fds = first_doc_start(mask, b0, b1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp < kPostWarps) {
+    const int u0 = b0 + warp * kPostRows;
+    const int nrow = max(0, min(kPostRows, b1 - u0));
+    const int n = z * 64 + 2 * lane;
+    if (z * 64 < KD) {
+      float2 dks[kPostRows];
+#pragma unroll
+      for (int r = 0; r < kPostRows; ++r) dks[r] = make_float2(0.f, 0.f);
+      for (int m = 0; m < grp; ++m) {
+        const int hq = kvh * grp + m, bh = b * HQ + hq;
+        const Tin* grow = g + (static_cast<size_t>(b) * T * HQ + hq) * KD + n;  // row stride HQ*KD
+        const size_t rs = static_cast<size_t>(HQ) * KD;
+        float2 sg = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int r = 0; r < kPostRows; ++r)
+          if (r < nrow) sg = add2(sg, load2(grow + (u0 + r) * rs));
+        ssum[m & 1][warp][lane] = sg;
+        named_bar_sync(1, kPostWarps * 32);
+        float2 L = make_float2(0.f, 0.f);
+        for (int w = 0; w < warp; ++w) L = add2(L, ssum[m & 1][w][lane]);
+        const size_t bb = static_cast<size_t>(bh) * NB + blk;
+        const float2 tot = load2(bsum + bb * KD + n);
+        const float2 qoff = (blk & 1) ? load2(bsum + (bb - 1) * KD + n) : make_float2(0.f, 0.f);
+        float2 hs = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int r = 0; r < kPostRows; ++r) {
+          if (r < nrow) {
+            const int u = u0 + r;
+            const size_t iq = ((static_cast<size_t>(b) * T + u) * HQ + hq) * KD + n;
+            const size_t ik = ((static_cast<size_t>(b) * T + u) * H + kvh) * KD + n;
+            const size_t ia = (static_cast<size_t>(bh) * T + u) * KD + n;
+            L = add2(L, load2(g + iq));
+            const float2 aq = load2(accQ + ia), ak = load2(accK + ia);
+            const float2 dqv = make_float2(scale * ex2_approx((qoff.x + L.x) * kLog2e) * aq.x,
+                                           scale * ex2_approx((qoff.y + L.y) * kLog2e) * aq.y);
+            const float2 dkv = make_float2(scale * ex2_approx((tot.x - L.x) * kLog2e) * ak.x,
+                                           scale * ex2_approx((tot.y - L.y) * kLog2e) * ak.y);
+            store2(dq + iq, dqv);
+            const float2 qv = load2(q + iq), kv = load2(k + ik);
+            const float2 dG = make_float2(qv.x * dqv.x - kv.x * dkv.x, qv.y * dqv.y - kv.y * dkv.y);
+            store2(accQ + ia, dG);
+            dks[r] = add2(dks[r], dkv);
+            if (u < fds) hs = add2(hs, dG);
+          }
+        }
+        hred[m & 1][warp][lane] = hs;
+        named_bar_sync(1, kPostWarps * 32);
+        if (warp == 0) {
+          float2 h = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int w = 0; w < kPostWarps; ++w) h = add2(h, hred[m & 1][w][lane]);
+          // rows of head are KD + 1 floats: an odd row starts off an 8-byte boundary
+          float* hp = head + (static_cast<size_t>(bh) * NB + blk) * (KD + 1) + n;
+          hp[0] = h.x;
+          hp[1] = h.y;
+        }
       }
-      if (psd != nullptr) ssum += psd[i];
+#pragma unroll
+      for (int r = 0; r < kPostRows; ++r)
+        if (r < nrow)
+          store2(dk + ((static_cast<size_t>(b) * T + u0 + r) * H + kvh) * KD + n, dks[r]);
     }
-    head[hbase + KD] = hsum;
-    if (psd != nullptr) sinkblk[static_cast<size_t>(bh) * NB + blk] = ssum;
+    if (z * 64 < VD) {
+#pragma unroll 4
+      for (int r = 0; r < kPostRows; ++r) {
+        if (r < nrow) {
+          const int u = u0 + r;
+          float2 s = make_float2(0.f, 0.f);
+          for (int m = 0; m < grp; ++m)
+            s = add2(s, load2(dvh + ((static_cast<size_t>(b) * HQ + kvh * grp + m) * T + u) * VD + n));
+          store2(dv + ((static_cast<size_t>(b) * T + u) * H + kvh) * VD + n, s);
+        }
+      }
+    }
+  } else if (z == 0) {
+    for (int m = 0; m < grp; ++m) {
+      const int bh = b * HQ + kvh * grp + m;
+      float hs = 0.f, ss = 0.f;
+      for (int u = b0 + lane; u < b1; u += 32) {
+        const size_t i = static_cast<size_t>(bh) * T + u;
+        if (HAS_GS) {
+          const float d = rsB[i] - rsA[i];
+          rsB[i] = d;
+          if (u < fds) hs += d;
+        }
+        if (psd != nullptr) ss += psd[i];
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        hs += __shfl_xor_sync(0xffffffffu, hs, off);
+        ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      }
+      if (lane == 0) {
+        head[(static_cast<size_t>(bh) * NB + blk) * (KD + 1) + KD] = hs;
+        if (psd != nullptr) sinkblk[static_cast<size_t>(bh) * NB + blk] = ss;
+      }
+    }
+  }
+}
+
+// The same pass for a group of GS query heads known at compile time: rows
+// outer, heads inner, so every row issues the group's loads together and the
+// per-head prefix state stays in registers; all heads' segment offsets are
+// found before the walk (one barrier), the head sums after it (one more).
+template <typename Tin, int KD, int VD, bool HAS_GS, int GS>
+__global__ void __launch_bounds__(kPostThreads, GS <= 4 ? 2 : 1) bwd_post_local_group_kernel(
+    const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ g,
+    const float* __restrict__ bsum, const int32_t* __restrict__ cu, int nseq, int T, int HQ, int H,
+    int NB, float scale, float* __restrict__ accQ, const float* __restrict__ accK,
+    const float* __restrict__ dvh, const float* __restrict__ rsA, float* __restrict__ rsB,
+    const float* __restrict__ psd, Tin* __restrict__ dq, Tin* __restrict__ dk,
+    Tin* __restrict__ dv, float* __restrict__ head, float* __restrict__ sinkblk) {
+  __shared__ uint32_t mask[4];
+  __shared__ float2 red[GS][kPostWarps][32];
+  const int blk = blockIdx.x, z = blockIdx.z;
+  const int b = blockIdx.y / H, kvh = blockIdx.y % H;
+  const int b0 = blk * kBlockRows, b1 = min(T, b0 + kBlockRows);
+  doc_start_mask(cu, nseq, b0, b1, mask);
+  const int fds = first_doc_start(mask, b0, b1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp < kPostWarps) {
+    const int u0 = b0 + warp * kPostRows;
+    const int nrow = max(0, min(kPostRows, b1 - u0));
+    const int n = z * 64 + 2 * lane;
+    const int hq0 = kvh * GS, bh0 = b * HQ + hq0;
+    if (z * 64 < KD) {
+      // row u0 of head hq0; head m is + m*KD (q, g, dq) or + m*T*KD (accQ, accK)
+      const size_t iq0 = ((static_cast<size_t>(b) * T + u0) * HQ + hq0) * KD + n;
+      const size_t ia0 = (static_cast<size_t>(bh0) * T + u0) * KD + n;
+      const size_t ik0 = ((static_cast<size_t>(b) * T + u0) * H + kvh) * KD + n;
+      const int sq = HQ * KD, sk = H * KD;      // row strides
+      const size_t sh = static_cast<size_t>(T) * KD;  // head stride of accQ / accK
+      float2 L[GS];
+#pragma unroll
+      for (int m = 0; m < GS; ++m) L[m] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int r = 0; r < kPostRows; ++r)
+        if (r < nrow) {
+#pragma unroll
+          for (int m = 0; m < GS; ++m) L[m] = add2(L[m], load2(g + iq0 + r * sq + m * KD));
+        }
+#pragma unroll
+      for (int m = 0; m < GS; ++m) red[m][warp][lane] = L[m];
+      named_bar_sync(1, kPostWarps * 32);
+      float2 tot[GS], qoff[GS], hs[GS];
+#pragma unroll
+      for (int m = 0; m < GS; ++m) {
+        L[m] = make_float2(0.f, 0.f);
+        for (int w = 0; w < warp; ++w) L[m] = add2(L[m], red[m][w][lane]);
+        const size_t bb = static_cast<size_t>(bh0 + m) * NB + blk;
+        tot[m] = load2(bsum + bb * KD + n);
+        qoff[m] = (blk & 1) ? load2(bsum + (bb - 1) * KD + n) : make_float2(0.f, 0.f);
+        hs[m] = make_float2(0.f, 0.f);
+      }
+      named_bar_sync(1, kPostWarps * 32);  // red is reused for the head sums
+#pragma unroll 2
+      for (int r = 0; r < kPostRows; ++r) {
+        if (r < nrow) {
+          const int u = u0 + r;
+          const float2 kv = load2(k + ik0 + r * sk);
+          float2 dks = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int m = 0; m < GS; ++m) {
+            const size_t iq = iq0 + r * sq + m * KD, ia = ia0 + r * KD + m * sh;
+            L[m] = add2(L[m], load2(g + iq));
+            const float2 aq = load2(accQ + ia), ak = load2(accK + ia), qv = load2(q + iq);
+            const float2 dqv = make_float2(scale * ex2_approx((qoff[m].x + L[m].x) * kLog2e) * aq.x,
+                                           scale * ex2_approx((qoff[m].y + L[m].y) * kLog2e) * aq.y);
+            const float2 dkv = make_float2(scale * ex2_approx((tot[m].x - L[m].x) * kLog2e) * ak.x,
+                                           scale * ex2_approx((tot[m].y - L[m].y) * kLog2e) * ak.y);
+            store2(dq + iq, dqv);
+            const float2 dG = make_float2(qv.x * dqv.x - kv.x * dkv.x, qv.y * dqv.y - kv.y * dkv.y);
+            store2(accQ + ia, dG);
+            dks = add2(dks, dkv);
+            if (u < fds) hs[m] = add2(hs[m], dG);
+          }
+          store2(dk + ik0 + r * sk, dks);
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < GS; ++m) red[m][warp][lane] = hs[m];
+      named_bar_sync(1, kPostWarps * 32);
+      if (warp < GS) {  // warp m sums head m's partial sums
+        float2 h = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < kPostWarps; ++w) h = add2(h, red[warp][w][lane]);
+        // rows of head are KD + 1 floats: an odd row starts off an 8-byte boundary
+        float* hp = head + (static_cast<size_t>(bh0 + warp) * NB + blk) * (KD + 1) + n;
+        hp[0] = h.x;
+        hp[1] = h.y;
+      }
+    }
+    if (z * 64 < VD) {
+      const size_t iv0 = (static_cast<size_t>(bh0) * T + u0) * VD + n;
+      const size_t io0 = ((static_cast<size_t>(b) * T + u0) * H + kvh) * VD + n;
+      const size_t shv = static_cast<size_t>(T) * VD;
+#pragma unroll 4
+      for (int r = 0; r < kPostRows; ++r) {
+        if (r < nrow) {
+          float2 s = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int m = 0; m < GS; ++m) s = add2(s, load2(dvh + iv0 + r * VD + m * shv));
+          store2(dv + io0 + r * (H * VD), s);
+        }
+      }
+    }
+  } else if (z == 0) {
+#pragma unroll 1
+    for (int m = 0; m < GS; ++m) {
+      const int bh = b * HQ + kvh * GS + m;
+      float hsg = 0.f, ss = 0.f;
+      for (int u = b0 + lane; u < b1; u += 32) {
+        const size_t i = static_cast<size_t>(bh) * T + u;
+        if (HAS_GS) {
+          const float d = rsB[i] - rsA[i];
+          rsB[i] = d;
+          if (u < fds) hsg += d;
+        }
+        if (psd != nullptr) ss += psd[i];
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        hsg += __shfl_xor_sync(0xffffffffu, hsg, off);
+        ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      }
+      if (lane == 0) {
+        head[(static_cast<size_t>(bh) * NB + blk) * (KD + 1) + KD] = hsg;
+        if (psd != nullptr) sinkblk[static_cast<size_t>(bh) * NB + blk] = ss;
+      }
+    }
   }
 }
 
@@ -545,29 +771,57 @@ __global__ void __launch_bounds__(KD + 32) bwd_post_scan_kernel(
   }
 }
 
-// One CTA per (128-row block, batch * query head): the reverse prefix sums
-// inside each document, dg[u] = sum of dG over rows u..(document end - 1).
+// One CTA per (128-row block, batch * query head, 64-channel group): the reverse
+// prefix sums inside each document, dg[u] = sum of dG over rows u..(document
+// end - 1).  Each warp publishes its rows' sum up to its first document start
+// and whether one starts there; the carry into a warp is the block's carry
+// passed back through the later warps (cut at the first of them that holds a
+// document start).  The last warp (channel group 0) does the gate channel.
 template <typename Tin, int KD, bool HAS_GS>
-__global__ void __launch_bounds__(KD + 32) bwd_post_final_kernel(
+__global__ void __launch_bounds__(kPostThreads) bwd_post_final_kernel(
     const float* __restrict__ dG, const float* __restrict__ dGs, const float* __restrict__ carry,
     const int32_t* __restrict__ cu, int nseq, int T, int HQ, int NB, Tin* __restrict__ dg,
     Tin* __restrict__ dgs) {
   __shared__ uint32_t mask[4];
-  const int blk = blockIdx.x, bh = blockIdx.y;
+  __shared__ float2 hsum[kPostWarps][32];
+  __shared__ int hstart[kPostWarps];
+  const int blk = blockIdx.x, bh = blockIdx.y, z = blockIdx.z;
   const int b = bh / HQ, hq = bh % HQ;
   const int b0 = blk * kBlockRows, b1 = min(T, b0 + kBlockRows);
   doc_start_mask(cu, nseq, b0, b1, mask);
-  const int tid = threadIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t cbase = (static_cast<size_t>(bh) * NB + blk) * (KD + 1);
-  if (tid < KD) {
-    float acc = carry[cbase + tid];
-#pragma unroll 4
-    for (int u = b1 - 1; u >= b0; --u) {
-      acc += dG[(static_cast<size_t>(bh) * T + u) * KD + tid];
-      store1(dg + ((static_cast<size_t>(b) * T + u) * HQ + hq) * KD + tid, acc);
-      if (u > b0 && bit_of(mask, u - b0)) acc = 0.f;
+  if (warp < kPostWarps) {
+    const int u0 = b0 + warp * kPostRows;
+    const int nrow = max(0, min(kPostRows, b1 - u0));
+    const int n = z * 64 + 2 * lane;
+    // bit r: a document starts at row u0 + r (never at b0 itself)
+    const uint32_t bits = (mask[warp >> 1] >> ((warp & 1) * kPostRows)) & 0xffffu;
+    float2 x[kPostRows];
+#pragma unroll
+    for (int r = 0; r < kPostRows; ++r)
+      x[r] = r < nrow ? load2(dG + (static_cast<size_t>(bh) * T + u0 + r) * KD + n)
+                      : make_float2(0.f, 0.f);
+    const int first = bits != 0u ? __ffs(static_cast<int>(bits)) - 1 : kPostRows;
+    float2 h = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int r = 0; r < kPostRows; ++r)
+      if (r < first) h = add2(h, x[r]);
+    hsum[warp][lane] = h;
+    if (lane == 0) hstart[warp] = bits != 0u;
+    named_bar_sync(1, kPostWarps * 32);
+    float2 acc = make_float2(carry[cbase + n], carry[cbase + n + 1]);  // rows of KD + 1 floats
+    for (int w = kPostWarps - 1; w > warp; --w)
+      acc = hstart[w] ? hsum[w][lane] : add2(hsum[w][lane], acc);
+#pragma unroll
+    for (int r = kPostRows - 1; r >= 0; --r) {
+      if (r < nrow) {
+        acc = add2(acc, x[r]);
+        store2(dg + ((static_cast<size_t>(b) * T + u0 + r) * HQ + hq) * KD + n, acc);
+      }
+      if ((bits >> r) & 1u) acc = make_float2(0.f, 0.f);
     }
-  } else if (HAS_GS && tid == KD) {
+  } else if (HAS_GS && z == 0 && lane == 0) {
     float acc = carry[cbase + KD];
     for (int u = b1 - 1; u >= b0; --u) {
       acc += dGs[static_cast<size_t>(bh) * T + u];
@@ -575,35 +829,6 @@ __global__ void __launch_bounds__(KD + 32) bwd_post_final_kernel(
       if (u > b0 && bit_of(mask, u - b0)) acc = 0.f;
     }
   }
-}
-
-// dk / dv of each KV head: the sum over the query heads of its group.
-// src [B*HQ][T][D] fp32, dst [B, T, H, D]; 4 channels per thread.
-template <typename Tin, int D>
-__global__ void __launch_bounds__(256) bwd_group_sum_kernel(const float* __restrict__ src, int B,
-                                                            int T, int HQ, int H,
-                                                            Tin* __restrict__ dst) {
-  const long long idx = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
-  const long long total = static_cast<long long>(B) * T * H * (D / 4);
-  if (idx >= total) return;
-  const int d4 = static_cast<int>(idx % (D / 4));
-  const long long rest = idx / (D / 4);
-  const int kvh = static_cast<int>(rest % H);
-  const int t = static_cast<int>((rest / H) % T);
-  const int b = static_cast<int>(rest / (static_cast<long long>(H) * T));
-  const int grp = HQ / H;
-  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int m = 0; m < grp; ++m) {
-    const int hq = kvh * grp + m;
-    const float4 x = *reinterpret_cast<const float4*>(
-        src + ((static_cast<size_t>(b) * HQ + hq) * T + t) * D + d4 * 4);
-    s.x += x.x; s.y += x.y; s.z += x.z; s.w += x.w;
-  }
-  Tin* o = dst + ((static_cast<size_t>(b) * T + t) * H + kvh) * D + d4 * 4;
-  store1(o, s.x);
-  store1(o + 1, s.y);
-  store1(o + 2, s.z);
-  store1(o + 3, s.w);
 }
 
 // dsink[hq] = sum over batch and blocks of the per-block sink sums (fixed order).
@@ -670,6 +895,28 @@ cudaError_t contract_simt(const BwdArgs& a, const FwdWork& fw, const BwdWork& bw
 }
 
 template <typename Tin, int KD, int VD, bool HAS_GS>
+cudaError_t launch_post_local(const BwdArgs& a, const FwdWork& fw, const BwdWork& bw,
+                              cudaStream_t st) {
+  const FwdArgs& f = a.f;
+  const dim3 grid(f.NB, f.B * f.H, (KD > VD ? KD : VD) / 64);  // 64-channel groups
+  auto go = [&](auto kern) {
+    kern<<<grid, kPostThreads, 0, st>>>(
+        static_cast<const Tin*>(f.q), static_cast<const Tin*>(f.k), static_cast<const Tin*>(f.g),
+        fw.bsum, f.cu_seqlens, f.num_seqs, f.T, f.HQ, f.H, f.NB, f.scale, bw.accQ, bw.accK,
+        bw.dvh, bw.rsA, bw.rsB, f.sink ? bw.psd : nullptr, static_cast<Tin*>(a.dq),
+        static_cast<Tin*>(a.dk), static_cast<Tin*>(a.dv), bw.head, bw.sinkblk);
+    return cudaGetLastError();
+  };
+  switch (f.HQ / f.H) {  // query heads per KV head
+    case 1: return go(bwd_post_local_group_kernel<Tin, KD, VD, HAS_GS, 1>);
+    case 2: return go(bwd_post_local_group_kernel<Tin, KD, VD, HAS_GS, 2>);
+    case 4: return go(bwd_post_local_group_kernel<Tin, KD, VD, HAS_GS, 4>);
+    case 8: return go(bwd_post_local_group_kernel<Tin, KD, VD, HAS_GS, 8>);
+    default: return go(bwd_post_local_kernel<Tin, KD, VD, HAS_GS>);
+  }
+}
+
+template <typename Tin, int KD, int VD, bool HAS_GS>
 cudaError_t bwd_impl(const BwdArgs& a, const FwdWork& fw, const BwdWork& bw, cudaStream_t st) {
   const FwdArgs& f = a.f;
   const int BHQ = f.B * f.HQ;
@@ -682,26 +929,13 @@ cudaError_t bwd_impl(const BwdArgs& a, const FwdWork& fw, const BwdWork& bw, cud
   // bf16: tensor-core contraction kernels; fp32: exact CUDA-core kernels
   e = sizeof(Tin) == 2 ? launch_bwd_tc(a, fw, bw, st) : contract_simt<Tin, KD, VD, HAS_GS>(a, fw, bw, st);
   if (e != cudaSuccess) return e;
-  const dim3 pgrid(f.NB, BHQ);
-  bwd_post_local_kernel<Tin, KD, HAS_GS><<<pgrid, KD + 32, 0, st>>>(
-      static_cast<const Tin*>(f.q), static_cast<const Tin*>(f.k), static_cast<const Tin*>(f.g),
-      fw.bsum, f.cu_seqlens, f.num_seqs, f.T, f.HQ, f.H, f.NB, f.scale, bw.accQ, bw.accK, bw.rsA,
-      bw.rsB, f.sink ? bw.psd : nullptr, static_cast<Tin*>(a.dq), bw.head, bw.sinkblk);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = launch_post_local<Tin, KD, VD, HAS_GS>(a, fw, bw, st)) != cudaSuccess) return e;
   bwd_post_scan_kernel<KD><<<BHQ, KD + 32, 0, st>>>(bw.head, f.cu_seqlens, f.num_seqs, f.T, f.NB,
                                                      bw.carry);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  bwd_post_final_kernel<Tin, KD, HAS_GS><<<pgrid, KD + 32, 0, st>>>(
+  bwd_post_final_kernel<Tin, KD, HAS_GS><<<dim3(f.NB, BHQ, KD / 64), kPostThreads, 0, st>>>(
       bw.accQ, bw.rsB, bw.carry, f.cu_seqlens, f.num_seqs, f.T, f.HQ, f.NB,
       static_cast<Tin*>(a.dg), static_cast<Tin*>(a.dg_scalar));
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const long long nk = static_cast<long long>(f.B) * f.T * f.H * (KD / 4);
-  bwd_group_sum_kernel<Tin, KD><<<static_cast<unsigned>((nk + 255) / 256), 256, 0, st>>>(
-      bw.accK, f.B, f.T, f.HQ, f.H, static_cast<Tin*>(a.dk));
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const long long nv = static_cast<long long>(f.B) * f.T * f.H * (VD / 4);
-  bwd_group_sum_kernel<Tin, VD><<<static_cast<unsigned>((nv + 255) / 256), 256, 0, st>>>(
-      bw.dvh, f.B, f.T, f.HQ, f.H, static_cast<Tin*>(a.dv));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (f.sink != nullptr) {
     bwd_sink_sum_kernel<<<f.HQ, 256, 0, st>>>(bw.sinkblk, f.B, f.HQ, f.NB, a.dsink);

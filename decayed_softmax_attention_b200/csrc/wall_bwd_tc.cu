@@ -207,27 +207,6 @@ __device__ __forceinline__ void rescale_tile(uint8_t* tile, const float* c, int 
   }
 }
 
-template <typename T>
-__device__ __forceinline__ T __uint_as_float_or_int(uint32_t u);
-template <>
-__device__ __forceinline__ float __uint_as_float_or_int<float>(uint32_t u) { return __uint_as_float(u); }
-template <>
-__device__ __forceinline__ int __uint_as_float_or_int<int>(uint32_t u) { return static_cast<int>(u); }
-
-// 32 consecutive fp32 (or int) values of a shared-memory vector, read as 8
-// 16-byte loads issued back to back (every thread reads the same addresses).
-template <typename T>
-__device__ __forceinline__ void load32(const T* src, T* dst) {
-#pragma unroll
-  for (int i = 0; i < 32; i += 4) {
-    const uint4 u = *reinterpret_cast<const uint4*>(src + i);
-    dst[i] = __uint_as_float_or_int<T>(u.x);
-    dst[i + 1] = __uint_as_float_or_int<T>(u.y);
-    dst[i + 2] = __uint_as_float_or_int<T>(u.z);
-    dst[i + 3] = __uint_as_float_or_int<T>(u.w);
-  }
-}
-
 __device__ __forceinline__ int first_key(const int* lo_tab, int window, int t) {
   if (lo_tab != nullptr) return lo_tab[t];
   if (window > 0) return t - window + 1 > 0 ? t - window + 1 : 0;

@@ -116,6 +116,12 @@ CASES = [
                   docs=(200, 133), seed=15),
     W.PrefillSpec("bwd_k64v128", B=2, T=190, HQ=4, H=2, K=64, V=128, dtype="bf16",
                   g_scalar=True, sink=True, seed=16),
+    # 3 query heads per KV head (the post pass's general group path), documents + gate
+    W.PrefillSpec("bwd_group3", B=1, T=300, HQ=6, H=2, K=64, V=64, dtype="bf16",
+                  g_scalar=True, docs=(90, 210), seed=17),
+    # 8 query heads per KV head, ragged tail
+    W.PrefillSpec("bwd_group8", B=1, T=270, HQ=8, H=1, K=128, V=128, dtype="bf16",
+                  g_kind="negsoftplus", seed=18),
 ]
 
 
