@@ -46,7 +46,8 @@ __device__ __forceinline__ float gate_row(const float* ssl, const float* ssa, in
 }
 
 // ------------------------------------------------------------------ bwd_pre
-// One warp per (b, t, hq) row.  Per (batch * head) rows of stride TP = NB*128
+// VD/8 lanes per (b, t, hq) row (a warp covers 32*8/VD rows), each lane one
+// 8-channel chunk of o and dO.  Per (batch * head) rows of stride TP = NB*128
 // (16-byte aligned slices for bulk copies):
 //   rowt  = Gs[t] log2(e) - lse[t] log2(e)   (query-side constant of log2 p)
 //   colt  = Gs[t] log2(e)                    (key side; with g_scalar only)
@@ -58,17 +59,22 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(
     const float* __restrict__ dlse, const float* __restrict__ sink, const float* __restrict__ ssl,
     const float* __restrict__ ssa, int B, int T, int HQ, int NB, float* __restrict__ rowt,
     float* __restrict__ colt, float* __restrict__ delta, float* __restrict__ psd) {
-  const long long r = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (r >= static_cast<long long>(B) * T * HQ) return;
-  const Tin* orow = o + r * VD;
-  const Tin* drow = dout + r * VD;
+  constexpr int LPR = VD / 8;  // lanes per row
+  const int lane = threadIdx.x & 31, l = lane % LPR;
+  const long long r = ((static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) >> 5) * (32 / LPR) +
+                      lane / LPR;
+  const bool row_ok = r < static_cast<long long>(B) * T * HQ;
   float acc = 0.f;
+  if (row_ok) {
+    float a[8], d[8];
+    load8(o + r * VD + l * 8, a);
+    load8(dout + r * VD + l * 8, d);
 #pragma unroll
-  for (int c = lane; c < VD; c += 32) acc = fmaf(load1(orow + c), load1(drow + c), acc);
+    for (int e = 0; e < 8; ++e) acc = fmaf(a[e], d[e], acc);
+  }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) {
+  for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (row_ok && l == 0) {
     const int hq = static_cast<int>(r % HQ);
     const long long bt = r / HQ;
     const int t = static_cast<int>(bt % T), b = static_cast<int>(bt / T);
@@ -609,6 +615,36 @@ __global__ void __launch_bounds__(kPostThreads, 2) bwd_post_local_kernel(
   }
 }
 
+// One row of the fixed-group post pass: the row's loads for all GS heads, then
+// dq, dG (over accQ) and the group's dk.
+template <typename Tin, int KD, int GS>
+__device__ __forceinline__ void post_row(int r, bool in_head, const Tin* __restrict__ q,
+                                         const Tin* __restrict__ k, const Tin* __restrict__ g,
+                                         float* __restrict__ accQ, const float* __restrict__ accK,
+                                         Tin* __restrict__ dq, Tin* __restrict__ dk, size_t iq0,
+                                         size_t ia0, size_t ik0, int sq, int sk, size_t sh,
+                                         float scale, float2 (&L)[GS], const float2 (&tot)[GS],
+                                         const float2 (&qoff)[GS], float2 (&hs)[GS]) {
+  const float2 kv = load2(k + ik0 + r * sk);
+  float2 dks = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int m = 0; m < GS; ++m) {
+    const size_t iq = iq0 + r * sq + m * KD, ia = ia0 + r * KD + m * sh;
+    L[m] = add2(L[m], load2(g + iq));
+    const float2 aq = load2(accQ + ia), ak = load2(accK + ia), qv = load2(q + iq);
+    const float2 dqv = make_float2(scale * ex2_approx((qoff[m].x + L[m].x) * kLog2e) * aq.x,
+                                   scale * ex2_approx((qoff[m].y + L[m].y) * kLog2e) * aq.y);
+    const float2 dkv = make_float2(scale * ex2_approx((tot[m].x - L[m].x) * kLog2e) * ak.x,
+                                   scale * ex2_approx((tot[m].y - L[m].y) * kLog2e) * ak.y);
+    store2(dq + iq, dqv);
+    const float2 dG = make_float2(qv.x * dqv.x - kv.x * dkv.x, qv.y * dqv.y - kv.y * dkv.y);
+    store2(accQ + ia, dG);
+    dks = add2(dks, dkv);
+    if (in_head) hs[m] = add2(hs[m], dG);
+  }
+  store2(dk + ik0 + r * sk, dks);
+}
+
 // The same pass for a group of GS query heads known at compile time: rows
 // outer, heads inner, so every row issues the group's loads together and the
 // per-head prefix state stays in registers; all heads' segment offsets are
@@ -644,12 +680,16 @@ __global__ void __launch_bounds__(kPostThreads, GS <= 4 ? 2 : 1) bwd_post_local_
       float2 L[GS];
 #pragma unroll
       for (int m = 0; m < GS; ++m) L[m] = make_float2(0.f, 0.f);
+      if (nrow == kPostRows) {
 #pragma unroll
-      for (int r = 0; r < kPostRows; ++r)
-        if (r < nrow) {
+        for (int r = 0; r < kPostRows; ++r)
 #pragma unroll
           for (int m = 0; m < GS; ++m) L[m] = add2(L[m], load2(g + iq0 + r * sq + m * KD));
-        }
+      } else {
+        for (int r = 0; r < nrow; ++r)
+#pragma unroll
+          for (int m = 0; m < GS; ++m) L[m] = add2(L[m], load2(g + iq0 + r * sq + m * KD));
+      }
 #pragma unroll
       for (int m = 0; m < GS; ++m) red[m][warp][lane] = L[m];
       named_bar_sync(1, kPostWarps * 32);
@@ -664,29 +704,16 @@ __global__ void __launch_bounds__(kPostThreads, GS <= 4 ? 2 : 1) bwd_post_local_
         hs[m] = make_float2(0.f, 0.f);
       }
       named_bar_sync(1, kPostWarps * 32);  // red is reused for the head sums
-#pragma unroll 2
-      for (int r = 0; r < kPostRows; ++r) {
-        if (r < nrow) {
-          const int u = u0 + r;
-          const float2 kv = load2(k + ik0 + r * sk);
-          float2 dks = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int m = 0; m < GS; ++m) {
-            const size_t iq = iq0 + r * sq + m * KD, ia = ia0 + r * KD + m * sh;
-            L[m] = add2(L[m], load2(g + iq));
-            const float2 aq = load2(accQ + ia), ak = load2(accK + ia), qv = load2(q + iq);
-            const float2 dqv = make_float2(scale * ex2_approx((qoff[m].x + L[m].x) * kLog2e) * aq.x,
-                                           scale * ex2_approx((qoff[m].y + L[m].y) * kLog2e) * aq.y);
-            const float2 dkv = make_float2(scale * ex2_approx((tot[m].x - L[m].x) * kLog2e) * ak.x,
-                                           scale * ex2_approx((tot[m].y - L[m].y) * kLog2e) * ak.y);
-            store2(dq + iq, dqv);
-            const float2 dG = make_float2(qv.x * dqv.x - kv.x * dkv.x, qv.y * dqv.y - kv.y * dkv.y);
-            store2(accQ + ia, dG);
-            dks = add2(dks, dkv);
-            if (u < fds) hs[m] = add2(hs[m], dG);
-          }
-          store2(dk + ik0 + r * sk, dks);
-        }
+      if (nrow == kPostRows) {  // no row past T: a guard-free walk the compiler can pipeline
+        constexpr int kUnroll = GS <= 2 ? 4 : 2;
+#pragma unroll kUnroll
+        for (int r = 0; r < kPostRows; ++r)
+          post_row<Tin, KD, GS>(r, u0 + r < fds, q, k, g, accQ, accK, dq, dk, iq0, ia0, ik0, sq, sk,
+                                sh, scale, L, tot, qoff, hs);
+      } else {
+        for (int r = 0; r < nrow; ++r)
+          post_row<Tin, KD, GS>(r, u0 + r < fds, q, k, g, accQ, accK, dq, dk, iq0, ia0, ik0, sq, sk,
+                                sh, scale, L, tot, qoff, hs);
       }
 #pragma unroll
       for (int m = 0; m < GS; ++m) red[m][warp][lane] = hs[m];
@@ -921,7 +948,8 @@ cudaError_t bwd_impl(const BwdArgs& a, const FwdWork& fw, const BwdWork& bw, cud
   const FwdArgs& f = a.f;
   const int BHQ = f.B * f.HQ;
   const long long rows = static_cast<long long>(f.B) * f.T * f.HQ;
-  bwd_pre_kernel<Tin, VD, HAS_GS><<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(
+  const long long pre_warps = (rows + 32 / (VD / 8) - 1) / (32 / (VD / 8));
+  bwd_pre_kernel<Tin, VD, HAS_GS><<<static_cast<unsigned>((pre_warps * 32 + 255) / 256), 256, 0, st>>>(
       static_cast<const Tin*>(f.o), static_cast<const Tin*>(a.dout), f.lse, a.dlse, f.sink, fw.ssl,
       fw.ssa, f.B, f.T, f.HQ, f.NB, bw.rowt, bw.colt, bw.delta, f.sink ? bw.psd : nullptr);
   cudaError_t e = cudaGetLastError();
