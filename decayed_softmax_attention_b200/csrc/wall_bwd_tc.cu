@@ -84,7 +84,7 @@ struct BtcCfg {
   static constexpr int A_C = A_COLT + VEC;       // 2 x KD fp32
   static constexpr int A_BAR = A_C + 2 * KD * 4;
   // kvfull, qfull[2], qready[2], qempty[2], sfull, dpfull, pready, dsready, final, mdrain
-  static constexpr int A_NBAR = 1 + 2 + 2 + 2 + 6;
+  static constexpr int A_NBAR = 1 + 2 + 2 + 2 + 6 + 2;  // + qready_hi[2]
   static constexpr int A_MISC = A_BAR + A_NBAR * 8;
   static constexpr int A_RS = A_MISC + 64;       // 128 fp32
   // at least 116 KB so that a second CTA never shares the SM (each takes all of TMEM)
@@ -170,8 +170,8 @@ __device__ __forceinline__ void fence_regs32(float* r) {
 
 // Multiplies one 128-row tile of KD bf16 channels (128-byte swizzle, boxes of
 // 64 channels) by c[KD] in place; 128 threads, r = thread index.  BATCH chunks
-// are loaded before any is scaled and stored (4 where the rescale sits on the
-// critical path, 1 where it runs in the shadow of the loads).
+// are loaded before any is scaled and stored (the query-block kernel's key
+// tiles; the key-block kernel rescales its query tiles box by box instead).
 template <int KD, int BATCH>
 __device__ __forceinline__ void rescale_tile(uint8_t* tile, const float* c, int r) {
   constexpr int CPR = KD / 8;       // 16-byte chunks per row
@@ -205,6 +205,36 @@ __device__ __forceinline__ void rescale_tile(uint8_t* tile, const float* c, int 
 #pragma unroll
     for (int m = 0; m < BATCH; ++m) *ptr[m] = scale8(v[m], chi, clo);
   }
+}
+
+// Multiplies one 64-channel box (128 rows x 8 chunks of 16 bytes, 128-byte
+// swizzle) of a tile by c[box*64 ..] in place; 128 threads, r = thread index:
+// chunk r & 7 of rows (r >> 3) + 16 m, all 8 loaded before any is stored.
+__device__ __forceinline__ void rescale_box(uint8_t* tile, const float* c, int r, int box) {
+  const int c16 = r & 7, row0 = r >> 3;
+  __nv_bfloat162 chi[4], clo[4];
+  {
+    const float4 c0 = *reinterpret_cast<const float4*>(c + box * 64 + c16 * 8);
+    const float4 c1 = *reinterpret_cast<const float4*>(c + box * 64 + c16 * 8 + 4);
+    const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      chi[i] = __floats2bfloat162_rn(cv[2 * i], cv[2 * i + 1]);
+      const float2 h = __bfloat1622float2(chi[i]);
+      clo[i] = __floats2bfloat162_rn(cv[2 * i] - h.x, cv[2 * i + 1] - h.y);
+    }
+  }
+  uint8_t* base = tile + box * 16384;
+  uint4* ptr[8];
+  uint4 v[8];
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    const int row = row0 + 16 * m;
+    ptr[m] = reinterpret_cast<uint4*>(base + row * 128 + ((c16 ^ (row & 7)) << 4));
+    v[m] = *ptr[m];
+  }
+#pragma unroll
+  for (int m = 0; m < 8; ++m) *ptr[m] = scale8(v[m], chi, clo);
 }
 
 __device__ __forceinline__ int first_key(const int* lo_tab, int window, int t) {
@@ -246,6 +276,7 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* dsready = bars + 10;
   uint64_t* final_bar = bars + 11;
   uint64_t* mdrain = bars + 12;
+  uint64_t* qready_hi = bars + 13;  // [2]: channels 64.. of the stage rescaled
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::A_MISC);
   int* abort_flag = reinterpret_cast<int*>(smem + C::A_MISC + 4);
   int* s_qhi = reinterpret_cast<int*>(smem + C::A_MISC + 8);
@@ -265,6 +296,7 @@ __global__ void __launch_bounds__(512, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&qfull[s], 1);
       mbar_init(&qready[s], 128);
+      mbar_init(&qready_hi[s], 128);
       mbar_init(&qempty[s], 1);
     }
     mbar_init(sfull, 1);
@@ -351,12 +383,20 @@ __global__ void __launch_bounds__(512, 1)
       const uint64_t dOm = sw128_desc(smem_u32(sDO), 16384, 1024);   // B of dV (MN-major)
       const uint32_t tS = tmem_base + COL_S, tDP = tmem_base + COL_DP;
       const uint32_t tDV = tmem_base + COL_DV, tDK = tmem_base + COL_DK;
-      auto issue_s = [&](int it) {
+      // S^T over the first 64 channels once they are rescaled (the caller waits
+      // on qready), the rest after qready_hi
+      auto issue_s = [&](int it) -> bool {
         const uint64_t qo = static_cast<uint64_t>((it & 1) * (C::KB >> 4));
 #pragma unroll
-        for (int kk = 0; kk < KD / 16; ++kk)
+        for (int kk = 0; kk < KD / 16; ++kk) {
+          if (kk == 4) {
+            if (!mbar_wait(&qready_hi[it & 1], (it >> 1) & 1, wc)) return false;
+            tc_fence_after();
+          }
           umma_ss(tS, dKa + kmaj_step(kk), dQk + qo + kmaj_step(kk), C::IDESC_SS, kk > 0 ? 1u : 0u);
+        }
         umma_commit(sfull);
+        return true;
       };
       auto issue_dp = [&](int it) {
         const uint64_t oo = static_cast<uint64_t>((it & 1) * (C::VB >> 4));
@@ -368,8 +408,8 @@ __global__ void __launch_bounds__(512, 1)
       if (ok) ok = mbar_wait(&qready[0], 0, wc);
       if (ok) {
         tc_fence_after();
-        issue_s(0);
-        issue_dp(0);
+        ok = issue_s(0);
+        if (ok) issue_dp(0);
       }
       for (int it = 0; ok && it < nt; ++it) {
         const int s = it & 1;
@@ -385,7 +425,7 @@ __global__ void __launch_bounds__(512, 1)
         if (it + 1 < nt) {
           if (!mbar_wait(&qready[(it + 1) & 1], ((it + 1) >> 1) & 1, wc)) { ok = false; break; }
           tc_fence_after();
-          issue_s(it + 1);
+          if (!issue_s(it + 1)) { ok = false; break; }
         }
         if (!mbar_wait(dsready, it & 1, wc)) { ok = false; break; }
         tc_fence_after();
@@ -561,9 +601,12 @@ __global__ void __launch_bounds__(512, 1)
       float* cb = sC + s * KD;
       if (got && r < KD) cb[r] = ex2_approx((sAQ[s * KD + r] - sAK[r]) * kLog2e);
       if (bar_any(1, 128, !got || *abort_flag != 0)) break;
-      rescale_tile<KD, 4>(sQ + s * C::KB, cb, r);
+      rescale_box(sQ + s * C::KB, cb, r, 0);
       fence_proxy_async_smem();
       mbar_arrive(&qready[s]);
+      if (KD > 64) rescale_box(sQ + s * C::KB, cb, r, 1);
+      fence_proxy_async_smem();
+      mbar_arrive(&qready_hi[s]);
     }
   }
 
@@ -865,7 +908,7 @@ __global__ void __launch_bounds__(512, 1)
       float* cb = sC + (jt & 1) * KD;
       if (got && r < KD) cb[r] = ex2_approx((sAQ[r] - sAK[ks * KD + r]) * kLog2e);
       if (bar_any(1, 128, !got || *abort_flag != 0)) break;
-      rescale_tile<KD, 1>(sK + ks * C::KB, cb, r);
+      rescale_tile<KD, 4>(sK + ks * C::KB, cb, r);
       fence_proxy_async_smem();
       mbar_arrive(&kready[ks]);
     }
