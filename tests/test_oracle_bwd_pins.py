@@ -58,6 +58,9 @@ FD_CASES = [
          cu=[0, 3, 8]),
     dict(seed=14, B=1, T=8, HQ=2, H=1, K=3, V=2, gs=True, sink=False, dlse=True, window=4,
          cu=[0, 5, 6, 8]),
+    # three query heads per KV head: dk, dv summed over a group of 3
+    dict(seed=15, B=1, T=6, HQ=3, H=1, K=2, V=2, gs=True, sink=True, dlse=False, window=0,
+         cu=[0, 2, 6]),
 ]
 
 
